@@ -1,0 +1,252 @@
+"""Plain CPU oracle for the TokenGate gated-prefill hot path (NumPy, float64).
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product path imports, calls or links this file:
+only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` use it.
+It shares no code with the CUDA path; both sides consume the same seeded input bytes.
+
+Sources (web pages about "TokenGate: Adapting LLMs for Fast and Memory-Efficient Prefill
+with Learned Token Pruning"):
+  * aitualizate.com article "TokenGate acelera prefill LLM con poda inteligente de tokens",
+    section "Cómo funciona TokenGate: tres fases para seleccionar los tokens" (phases 1-3)
+    and the paragraph on token-gated attention ("Cómo consigue entrenar una selección top-K").
+  * thelatestinai.com paper page "TokenGate: Adapting LLMs for Fast and Memory-Efficient
+    Prefill with Learned Token Pruning", Figure 1 caption, panels (a)-(c).
+
+Each function is the plain definition of the step it names, written out with library
+primitives (matmul, erf, lexsort); nothing is blocked, fused or reordered. Where the pages
+leave a step open, the reading taken is stated in the function's docstring:
+  * gate map g = sigmoid(score), log g as a stable log-sigmoid;
+  * GELU with the exact error function; biases b1 (per hidden unit) and b2 (scalar);
+  * K counts the context tokens kept by top-K; the question tail is always added on top;
+  * equal scores keep the lower index; -0 equals +0; NaN ranks below -inf;
+  * the gate enters attention as log g_j added to the logit (= weight times g_j, then
+    row renormalisation); an optional per-head gain multiplies that bias; an
+    "unnormalised" variant multiplies the weight by g_j without renormalising;
+  * causal mask on original positions (key allowed iff pos_j <= pos_i, same sequence);
+    grouped KV heads map query head h to KV head h // (Hq / Hkv).
+
+Every function is pinned by tests/test_oracle_pins.py against closed forms, textbook
+values, brute force and invariants. Parity is unpinned for nothing in this file.
+"""
+from __future__ import annotations
+
+import numpy as np
+from scipy.special import erf
+
+LOG2E = 1.4426950408889634
+
+# --------------------------------------------------------------------------- phase 2: score
+
+
+def gelu(z):
+    """GELU with the exact error function: z * Phi(z) = 0.5 z (1 + erf(z / sqrt 2))."""
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * z * (1.0 + erf(z / np.sqrt(2.0)))
+
+
+def gate_scores(H, W1, b1, w2, b2):
+    """One scalar importance score per token from its hidden state at layer L.
+
+    aitualizate.com article, phase 2 ("una pequeña red neuronal multicapa ... asigna una
+    puntuación individual a cada token"); thelatestinai.com page, Figure 1(b) ("scores each
+    hidden state with a small scoring network"). The network is d -> dg -> 1 with GELU:
+        s_i = w2 . GELU(W1 h_i + b1) + b2
+    H: [n, d]; W1: [dg, d] (output-major, like nn.Linear); b1: [dg] or None; w2: [dg];
+    b2: scalar. The hidden layer is kept at full precision (no rounding between layers).
+    """
+    H = np.asarray(H, dtype=np.float64)
+    W1 = np.asarray(W1, dtype=np.float64)
+    w2 = np.asarray(w2, dtype=np.float64).reshape(-1)
+    z = H @ W1.T
+    if b1 is not None:
+        z = z + np.asarray(b1, dtype=np.float64)[None, :]
+    return gelu(z) @ w2 + float(b2)
+
+
+def gate_value(s):
+    """Gate value g = sigmoid(s) and log g, the latter as a stable log-sigmoid.
+
+    The pages forward each kept token's importance score into attention (thelatestinai.com,
+    Figure 1(b)-(c), "gate value g_j") but do not print the score -> g map; sigmoid is the
+    reading taken. log g = -log1p(exp(-s)) for s >= 0, s - log1p(exp(s)) otherwise, so it is
+    finite for every finite s (no row can become all -inf).
+    """
+    s = np.asarray(s, dtype=np.float64)
+    g = np.empty_like(s)
+    pos = s >= 0
+    e = np.exp(-np.abs(s))
+    g[pos] = 1.0 / (1.0 + e[pos])
+    g[~pos] = e[~pos] / (1.0 + e[~pos])
+    logg = np.where(pos, -np.log1p(e), s - np.log1p(e))
+    return g, logg
+
+
+# --------------------------------------------------------------------------- phase 2: top-K
+
+
+def kept_count(n, q, k):
+    """Rows kept for one sequence: min(K, N - q) context tokens plus the q question tokens."""
+    return min(max(int(k), 0), int(n) - int(q)) + int(q)
+
+
+def topk_select(s, seqlens, q_len, k):
+    """Top-K over the context part of each packed sequence; the question tail is always kept.
+
+    aitualizate.com article, phase 2 ("un selector top-K conserva los K tokens con mayor
+    puntuación") and the restriction that only the document may be pruned ("la pregunta
+    nunca se elimina"); thelatestinai.com page, Figure 1(a) ("the gate module keeps K").
+
+    Per sequence b (packed at offset start_b): the context positions are [0, N_b - q_b),
+    the question tail is [N_b - q_b, N_b). The context is fully sorted by (score
+    descending, index ascending) - NaN after every number, -0 equal to +0 - and the first
+    min(K_b, N_b - q_b) are kept. The result, with the tail appended, is sorted ascending.
+
+    Returns (kept, cu_kept): kept is int64 [M_tot] of packed (global) row indices,
+    cu_kept int64 [B+1].
+    """
+    s = np.asarray(s, dtype=np.float64)
+    kept, cu = [], [0]
+    start = 0
+    for n, q, kb in zip(seqlens, q_len, k):
+        n, q = int(n), int(q)
+        n_ctx = n - q
+        kc = min(max(int(kb), 0), n_ctx)
+        ctx = s[start : start + n_ctx]
+        is_nan = np.isnan(ctx)
+        neg = np.where(is_nan, 0.0, -ctx) + 0.0  # + 0.0 turns -0 into +0
+        idx = np.arange(n_ctx)
+        order = np.lexsort((idx, neg, is_nan))  # primary: not-NaN first; then -s; then index
+        sel = np.sort(order[:kc])
+        rows = np.concatenate([sel, np.arange(n_ctx, n)]) + start
+        kept.append(rows)
+        cu.append(cu[-1] + rows.size)
+        start += n
+    kept = np.concatenate(kept) if kept else np.zeros(0, dtype=np.int64)
+    return kept.astype(np.int64), np.asarray(cu, dtype=np.int64)
+
+
+# --------------------------------------------------------------------------- forward kept
+
+
+def gather(H, s, kept, seqlens, q_len, cu_kept, question_gate_one=False):
+    """Kept hidden states with their gate values and original positions.
+
+    thelatestinai.com page, Figure 1(b) ("forwards the kept hidden states together with
+    their importance scores"); aitualizate.com article, phase 3 (layers above L receive only
+    the kept tokens). pos is each kept row's index within its own sequence (the original
+    position id the causal mask uses). With ``question_gate_one`` the question-tail rows get
+    g = 1, log g = 0 instead of their own gate value.
+
+    Returns (H_kept [M, d] (same dtype/bits as H), pos int64 [M], g [M], logg [M]).
+    """
+    H = np.asarray(H)
+    kept = np.asarray(kept, dtype=np.int64)
+    starts = np.concatenate([[0], np.cumsum(seqlens)])[:-1]
+    seq_of_row = np.repeat(np.arange(len(seqlens)), np.diff(np.asarray(cu_kept)))
+    pos = kept - starts[seq_of_row]
+    g, logg = gate_value(np.asarray(s, dtype=np.float64)[kept])
+    if question_gate_one:
+        for b, q in enumerate(q_len):
+            hi = int(cu_kept[b + 1])
+            g[hi - int(q) : hi] = 1.0
+            logg[hi - int(q) : hi] = 0.0
+    return H[kept], pos, g, logg
+
+
+# --------------------------------------------------------------------------- phase 3: attention
+
+
+def gated_attention(Q, K, V, logg, pos, cu_kept, Hq, Hkv, scale, head_gain=None,
+                    unnormalised=False, rows=None):
+    """Token-gated causal attention over the kept tokens, per sequence and query head.
+
+    thelatestinai.com page, Figure 1(c): each attention weight is multiplied by the gate
+    value g_j of its key. Read with the row renormalised, this equals adding log g_j to the
+    logit (aitualizate.com article: the score becomes a bias on the attention logits, with a
+    per-head gain). For query row i, head h, KV head h // (Hq/Hkv):
+        S_ij = scale * q_i . k_j + gain_h * log g_j,   allowed iff pos_j <= pos_i
+        O_i  = sum_j softmax_j(S_i) v_j,   LSE_i = logsumexp_j S_ij
+    Unnormalised variant: O_i = sum_j softmax_j(scale q_i . k_j) * g_j^gain_h * v_j, and
+    LSE is that of the unbiased logits.
+
+    Q: [M, Hq, D]; K, V: [M, Hkv, D]; logg: [M] or None (g == 1); pos: [M]; cu_kept [B+1].
+    rows: optional global query rows to evaluate (default: all). Returns (O [R, Hq, D],
+    LSE [Hq, R]) for the R evaluated rows, float64.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    M = Q.shape[0]
+    D = Q.shape[2]
+    G = Hq // Hkv
+    assert Hq % Hkv == 0 and K.shape[1] == Hkv
+    pos = np.asarray(pos, dtype=np.int64)
+    lg = np.zeros(M) if logg is None else np.asarray(logg, dtype=np.float64)
+    gain = np.ones(Hq) if head_gain is None else np.asarray(head_gain, dtype=np.float64)
+    rows = np.arange(M) if rows is None else np.asarray(rows, dtype=np.int64)
+    cu = np.asarray(cu_kept, dtype=np.int64)
+    O = np.zeros((rows.size, Hq, D))
+    LSE = np.zeros((Hq, rows.size))
+    seq = np.searchsorted(cu, rows, side="right") - 1
+    for b in range(cu.size - 1):
+        sel = np.nonzero(seq == b)[0]
+        if sel.size == 0:
+            continue
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        r = rows[sel]
+        allowed = pos[lo:hi][None, :] <= pos[r][:, None]
+        for h in range(Hq):
+            kv = h // G
+            logits = scale * (Q[r, h, :] @ K[lo:hi, kv, :].T)
+            bias = gain[h] * lg[lo:hi]
+            S = logits if unnormalised else logits + bias[None, :]
+            S = np.where(allowed, S, -np.inf)
+            m = S.max(axis=1, keepdims=True)
+            P = np.exp(S - m)
+            l = P.sum(axis=1, keepdims=True)
+            P = P / l
+            if unnormalised:
+                O[sel, h, :] = P @ (np.exp(bias)[:, None] * V[lo:hi, kv, :])
+            else:
+                O[sel, h, :] = P @ V[lo:hi, kv, :]
+            LSE[h, sel] = (m + np.log(l))[:, 0]
+    return O, LSE
+
+
+def gated_attention_weights(q, Kmat, g, scale):
+    """Figure 1(c) read literally for one query row: softmax weights times g_j, renormalised.
+
+    Used by the pins to show it equals the logit-bias form. q: [D]; Kmat: [n, D]; g: [n].
+    """
+    logits = scale * (np.asarray(Kmat, np.float64) @ np.asarray(q, np.float64))
+    w = np.exp(logits - logits.max())
+    w = w / w.sum()
+    wg = w * np.asarray(g, np.float64)
+    return wg / wg.sum()
+
+
+# --------------------------------------------------------------------------- whole path
+
+
+def prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, Hq, Hkv, scale,
+                    head_gain=None, unnormalised=False, question_gate_one=False):
+    """The gated path above layer L: score -> top-K (+question tail) -> gather -> attention.
+
+    aitualizate.com article, phases 2 and 3; thelatestinai.com page, Figure 1(a)-(c).
+    ``layers`` is a list of (Q, K, V) per above-L layer, already shaped by the kept count.
+    Returns a dict with every intermediate.
+    """
+    s = gate_scores(H, W1, b1, w2, b2)
+    return prefill_from_scores(H, s, seqlens, q_len, k, layers, Hq, Hkv, scale, head_gain,
+                               unnormalised, question_gate_one)
+
+
+def prefill_from_scores(H, s, seqlens, q_len, k, layers, Hq, Hkv, scale, head_gain=None,
+                        unnormalised=False, question_gate_one=False):
+    """The same path starting from given scores (select, gather, attention)."""
+    kept, cu = topk_select(s, seqlens, q_len, k)
+    Hk, pos, g, logg = gather(H, s, kept, seqlens, q_len, cu, question_gate_one)
+    outs = [gated_attention(Q, Kt, V, logg, pos, cu, Hq, Hkv, scale, head_gain, unnormalised)
+            for (Q, Kt, V) in layers]
+    return {"score": s, "kept": kept, "cu_kept": cu, "H_kept": Hk, "pos": pos, "g": g,
+            "logg": logg, "attn": outs}

@@ -1,0 +1,375 @@
+"""Pins for the CPU oracle: closed forms, textbook values, brute force and invariants.
+
+These tests tie the oracle to what the TokenGate pages and the mathematics fix, so that a
+plausible mistake in it (a dropped term, a wrong sign or index, a transposed operand, a
+wrong tie-break) fails at least one of them. CPU only.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import tg_inputs as ti
+from oracle import tg_oracle as orc
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+def _num(x):
+    return float(x) if not isinstance(x, str) else float(x.replace("nan", "nan"))
+
+
+# ----------------------------------------------------------------------------- score
+
+
+def test_gelu_matches_normal_cdf_table(golden_dir):
+    fx = _load(golden_dir, "gelu_normal_cdf.json")
+    for xs, phi in fx["phi"].items():
+        x = float(xs)
+        assert abs(orc.gelu(x) - x * phi) <= fx["tolerance_abs"], x
+
+
+def test_gelu_odd_part_identity():
+    # GELU(x) - GELU(-x) = x Phi(x) + x Phi(-x) = x for every x
+    x = np.linspace(-6, 6, 101)
+    assert np.max(np.abs(orc.gelu(x) - orc.gelu(-x) - x)) < 1e-14
+
+
+def test_score_one_hot_closed_form(golden_dir):
+    fx = _load(golden_dir, "score_onehot.json")
+    s = orc.gate_scores(np.array(fx["H"]), np.array(fx["W1"]), np.array(fx["b1"]),
+                        np.array(fx["w2"]), fx["b2"])
+    np.testing.assert_allclose(s, fx["expected"], rtol=0, atol=fx["tolerance_abs"])
+
+
+def _score_bruteforce(H, W1, b1, w2, b2):
+    out = []
+    for h in H:
+        acc = 0.0
+        for kk in range(len(W1)):
+            z = sum(float(W1[kk][j]) * float(h[j]) for j in range(len(h))) + float(b1[kk])
+            acc += float(w2[kk]) * 0.5 * z * (1.0 + math.erf(z / math.sqrt(2.0)))
+        out.append(acc + b2)
+    return np.array(out)
+
+
+def test_score_matches_per_token_loop_nonsquare():
+    g = np.random.default_rng(5)
+    n, d, dg = 7, 5, 3  # d != dg so a transposed W1 cannot pass
+    H = g.standard_normal((n, d))
+    W1 = g.standard_normal((dg, d))
+    b1 = g.uniform(-0.5, 0.5, dg)
+    w2 = g.standard_normal(dg)
+    b2 = 0.3
+    np.testing.assert_allclose(orc.gate_scores(H, W1, b1, w2, b2),
+                               _score_bruteforce(H, W1, b1, w2, b2), rtol=1e-12, atol=1e-12)
+
+
+def test_score_float32_independent_evaluation():
+    # an independent float32 evaluation (torch, exact-erf GELU) agrees within float32 error
+    wl = ti.scaled(ti.WORKLOADS["tiny_f32"], seqlens=(64,), q_len=(8,), k=(8,))
+    H = ti.hidden_states(wl)
+    W1, b1, w2, b2 = ti.gate_weights(wl, biased=True)
+    s64 = orc.gate_scores(H, W1, b1, w2, b2)
+    t = torch.nn.functional.gelu(torch.from_numpy(H) @ torch.from_numpy(W1).T
+                                 + torch.from_numpy(b1)) @ torch.from_numpy(w2) + b2
+    np.testing.assert_allclose(s64, t.numpy().astype(np.float64), rtol=0,
+                               atol=2e-5 * np.abs(s64).max())
+
+
+# ----------------------------------------------------------------------------- gate value
+
+
+def test_gate_value_special_values():
+    g, lg = orc.gate_value(np.array([0.0]))
+    assert g[0] == 0.5 and abs(lg[0] - math.log(0.5)) < 1e-15
+    s = np.linspace(-30, 30, 241)
+    g, lg = orc.gate_value(s)
+    assert np.all((g > 0) & (g < 1 + 1e-15))
+    np.testing.assert_allclose(g, 1.0 / (1.0 + np.exp(-s)), rtol=1e-14)
+    np.testing.assert_allclose(np.exp(lg), g, rtol=1e-14)
+    # log sigma(s) - log sigma(-s) = s
+    _, lgm = orc.gate_value(-s)
+    np.testing.assert_allclose(lg - lgm, s, rtol=0, atol=1e-12)
+
+
+def test_log_gate_is_finite_and_linear_far_left():
+    s = np.array([-50.0, -700.0, -1e4, 40.0, 800.0])
+    _, lg = orc.gate_value(s)
+    assert np.all(np.isfinite(lg))
+    np.testing.assert_allclose(lg[:3], s[:3], rtol=1e-15, atol=0)
+    assert lg[3] == pytest.approx(-math.exp(-40.0), rel=1e-12)
+    assert lg[4] == 0.0 or abs(lg[4]) < 1e-300
+
+
+# ----------------------------------------------------------------------------- select
+
+
+def _parse_scores(vals):
+    out = []
+    for v in vals:
+        out.append(float(v) if not isinstance(v, str) else float(v))
+    return np.array(out, dtype=np.float32)
+
+
+def test_topk_golden_ties(golden_dir):
+    fx = _load(golden_dir, "topk_ties.json")
+    s = _parse_scores(fx["scores"])
+    assert math.copysign(1.0, s[2]) < 0  # the fixture really holds a negative zero
+    for case in fx["cases"]:
+        kept, cu = orc.topk_select(s, fx["seqlens"], fx["q_len"], case["k"])
+        assert kept.tolist() == case["kept"], case
+        assert cu.tolist() == case["cu_kept"], case
+
+
+def _exhaustive_check(s, kept, seqlens, q_len, k):
+    start = 0
+    kept = set(int(x) for x in kept)
+    for n, q, kb in zip(seqlens, q_len, k):
+        n_ctx = n - q
+        ctx = range(start, start + n_ctx)
+        kept_ctx = [j for j in ctx if j in kept]
+        drop_ctx = [i for i in ctx if i not in kept]
+        assert len(kept_ctx) == min(max(kb, 0), n_ctx)
+        for j in range(start + n_ctx, start + n):
+            assert j in kept  # question tail always kept
+
+        def before(a, b):  # a ranks before b
+            sa, sb = s[a], s[b]
+            if np.isnan(sa) or np.isnan(sb):
+                return (not np.isnan(sa) and np.isnan(sb)) or (np.isnan(sa) and np.isnan(sb) and a < b)
+            return sa > sb or (sa == sb and a < b)
+
+        for j in kept_ctx:
+            for i in drop_ctx:
+                assert before(j, i), (j, i, s[j], s[i])
+        start += n
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_bruteforce_small_integer_ties(seed):
+    g = np.random.default_rng(seed)
+    B = int(g.integers(1, 4))
+    seqlens = [int(g.integers(1, 40)) for _ in range(B)]
+    q_len = [int(g.integers(0, n + 1)) for n in seqlens]
+    k = [int(g.integers(0, 45)) for _ in range(B)]
+    s = g.integers(0, 4, size=sum(seqlens)).astype(np.float32)  # heavy ties
+    s[g.random(s.size) < 0.05] = np.nan
+    s[g.random(s.size) < 0.05] = -0.0
+    kept, cu = orc.topk_select(s, seqlens, q_len, k)
+    assert np.all(np.diff(kept[cu[0]:cu[1]]) > 0)
+    for b in range(B):
+        seg = kept[cu[b]:cu[b + 1]]
+        assert np.all(np.diff(seg) > 0)
+        assert seg.size == orc.kept_count(seqlens[b], q_len[b], k[b])
+    _exhaustive_check(s, kept, seqlens, q_len, k)
+
+
+def test_topk_matches_full_stable_sort_by_python_sorted():
+    g = np.random.default_rng(11)
+    n, q, kk = 300, 20, 37
+    s = np.round(g.standard_normal(n) * 4) / 4  # ties
+    kept, _ = orc.topk_select(s.astype(np.float32), [n], [q], [kk])
+    ranked = sorted(range(n - q), key=lambda i: (-float(np.float32(s[i])), i))
+    expect = sorted(ranked[:kk]) + list(range(n - q, n))
+    assert kept.tolist() == expect
+
+
+def test_topk_degenerate_budgets():
+    s = np.arange(10, dtype=np.float32)
+    kept, cu = orc.topk_select(s, [10], [10], [5])  # question only: nothing to prune
+    assert kept.tolist() == list(range(10))
+    kept, cu = orc.topk_select(s, [10], [0], [3])  # no question
+    assert kept.tolist() == [7, 8, 9]
+    kept, cu = orc.topk_select(s, [10], [4], [-2])  # negative budget reads as 0
+    assert kept.tolist() == [6, 7, 8, 9]
+    kept, cu = orc.topk_select(np.zeros(0, np.float32), [], [], [])
+    assert kept.size == 0 and cu.tolist() == [0]
+
+
+# ----------------------------------------------------------------------------- gather
+
+
+def test_gather_positions_and_rows():
+    g = np.random.default_rng(2)
+    seqlens, q_len, k = [12, 7, 9], [3, 0, 9], [4, 2, 1]
+    H = g.standard_normal((sum(seqlens), 5)).astype(np.float32)
+    s = g.standard_normal(sum(seqlens)).astype(np.float32)
+    kept, cu = orc.topk_select(s, seqlens, q_len, k)
+    Hk, pos, gv, lg = orc.gather(H, s, kept, seqlens, q_len, cu)
+    starts = np.cumsum([0] + seqlens[:-1])
+    for r, j in enumerate(kept):
+        b = max(i for i in range(3) if starts[i] <= j)
+        assert pos[r] == j - starts[b]
+        assert np.array_equal(Hk[r].view(np.uint32), H[j].view(np.uint32))
+        assert gv[r] == pytest.approx(1 / (1 + math.exp(-float(s[j]))), rel=1e-14)
+    _, _, g1, l1 = orc.gather(H, s, kept, seqlens, q_len, cu, question_gate_one=True)
+    for b in range(3):
+        hi = cu[b + 1]
+        assert np.all(g1[hi - q_len[b]:hi] == 1.0) and np.all(l1[hi - q_len[b]:hi] == 0.0)
+        lo_ctx = hi - q_len[b]
+        np.testing.assert_array_equal(g1[cu[b]:lo_ctx], gv[cu[b]:lo_ctx])
+
+
+# ----------------------------------------------------------------------------- attention
+
+
+def _attn_bruteforce(Q, K, V, logg, pos, cu, Hq, Hkv, scale, gain=None, unnorm=False):
+    M, _, D = Q.shape
+    G = Hq // Hkv
+    O = np.zeros((M, Hq, D))
+    L = np.zeros((Hq, M))
+    for b in range(len(cu) - 1):
+        for i in range(cu[b], cu[b + 1]):
+            for h in range(Hq):
+                gh = 1.0 if gain is None else gain[h]
+                js = [j for j in range(cu[b], cu[b + 1]) if pos[j] <= pos[i]]
+                lo = [scale * sum(Q[i, h, t] * K[j, h // G, t] for t in range(D)) for j in js]
+                bias = [gh * (0.0 if logg is None else logg[j]) for j in js]
+                tot = [a + c for a, c in zip(lo, bias)] if not unnorm else lo
+                m = max(tot)
+                w = [math.exp(x - m) for x in tot]
+                z = sum(w)
+                L[h, i] = m + math.log(z)
+                for jj, j in enumerate(js):
+                    f = w[jj] / z * (math.exp(bias[jj]) if unnorm else 1.0)
+                    O[i, h, :] += f * V[j, h // G, :]
+    return O, L
+
+
+def test_attention_golden_two_keys(golden_dir):
+    fx = _load(golden_dir, "attention_two_keys.json")
+    Q, K, V = (np.array(fx[x]) for x in ("Q", "K", "V"))
+    lg = np.log(np.array(fx["g"]))
+    pos = np.array(fx["pos"])
+    cu = [0, 2]
+    tol = fx["tolerance_abs"]
+    for key, kw in (("normalised", {}), ("gain2", {"head_gain": [2.0]}),
+                    ("unnormalised", {"unnormalised": True})):
+        O, L = orc.gated_attention(Q, K, V, lg, pos, cu, 1, 1, fx["scale"], **kw)
+        np.testing.assert_allclose(O[:, 0, :], fx["expected"][key]["O"], rtol=0, atol=tol)
+        np.testing.assert_allclose(L[0], fx["expected"][key]["LSE"], rtol=0, atol=tol)
+
+
+@pytest.mark.parametrize("unnorm", [False, True])
+def test_attention_bruteforce_gqa_ragged_gain(unnorm):
+    g = np.random.default_rng(3)
+    cu = [0, 5, 6, 11]
+    M, Hq, Hkv, D = 11, 4, 2, 3
+    Q = g.standard_normal((M, Hq, D))
+    K = g.standard_normal((M, Hkv, D))
+    V = g.standard_normal((M, Hkv, D))
+    lg = np.log(g.uniform(0.05, 1, M))
+    pos = np.array([0, 3, 4, 9, 20, 7, 1, 2, 5, 6, 8])  # ascending within each sequence
+    gain = np.array([1.0, 0.5, 2.0, -1.0])
+    O, L = orc.gated_attention(Q, K, V, lg, pos, cu, Hq, Hkv, 0.7, gain, unnorm)
+    Ob, Lb = _attn_bruteforce(Q, K, V, lg, pos, cu, Hq, Hkv, 0.7, gain, unnorm)
+    np.testing.assert_allclose(O, Ob, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(L, Lb, rtol=1e-12, atol=1e-12)
+    rows = np.array([10, 0, 5, 3])
+    Os, Ls = orc.gated_attention(Q, K, V, lg, pos, cu, Hq, Hkv, 0.7, gain, unnorm, rows=rows)
+    np.testing.assert_allclose(Os, O[rows], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(Ls, L[:, rows], rtol=1e-13, atol=1e-13)
+
+
+def test_attention_g1_all_kept_is_textbook_causal_attention():
+    # g == 1 and K >= N - q keeps every token: ordinary causal attention (torch SDPA, float64)
+    g = np.random.default_rng(4)
+    N, q, Hq, Hkv, D = 40, 6, 4, 2, 8
+    s = g.standard_normal(N).astype(np.float32)
+    kept, cu = orc.topk_select(s, [N], [q], [N])
+    assert kept.tolist() == list(range(N))
+    Q = g.standard_normal((N, Hq, D))
+    K = g.standard_normal((N, Hkv, D))
+    V = g.standard_normal((N, Hkv, D))
+    scale = 1 / math.sqrt(D)
+    O, _ = orc.gated_attention(Q, K, V, None, np.arange(N), cu, Hq, Hkv, scale)
+    tq = torch.from_numpy(Q).permute(1, 0, 2)
+    tk = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+    tv = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=scale)
+    np.testing.assert_allclose(O, ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_invariants():
+    g = np.random.default_rng(8)
+    M, Hq, Hkv, D = 17, 2, 1, 4
+    Q = g.standard_normal((M, Hq, D))
+    K = g.standard_normal((M, Hkv, D))
+    V = g.standard_normal((M, Hkv, D))
+    pos = np.arange(M) * 2
+    cu = [0, M]
+    lg = np.log(g.uniform(0.1, 1, M))
+    O1, _ = orc.gated_attention(Q, K, V, None, pos, cu, Hq, Hkv, 0.5)
+    # constant g is a shift of every logit: same as g == 1
+    Oc, _ = orc.gated_attention(Q, K, V, np.full(M, math.log(0.3)), pos, cu, Hq, Hkv, 0.5)
+    np.testing.assert_allclose(Oc, O1, rtol=1e-12, atol=1e-12)
+    # the first kept row sees only itself: O = v0 (normalised), g0 v0 (unnormalised)
+    O, _ = orc.gated_attention(Q, K, V, lg, pos, cu, Hq, Hkv, 0.5)
+    np.testing.assert_allclose(O[0, 0], V[0, 0], rtol=0, atol=1e-15)
+    Ou, _ = orc.gated_attention(Q, K, V, lg, pos, cu, Hq, Hkv, 0.5, unnormalised=True)
+    np.testing.assert_allclose(Ou[0, 1], math.exp(lg[0]) * V[0, 0], rtol=1e-14)
+    # a key whose gate goes to zero is the same as removing that key
+    lz = lg.copy()
+    lz[5] = -1e4
+    Oz, _ = orc.gated_attention(Q, K, V, lz, pos, cu, Hq, Hkv, 0.5)
+    keep = np.array([i for i in range(M) if i != 5])
+    Or, _ = orc.gated_attention(Q[keep], K[keep], V[keep], lg[keep], pos[keep], [0, M - 1],
+                                Hq, Hkv, 0.5)
+    np.testing.assert_allclose(Oz[keep], Or, rtol=1e-12, atol=1e-12)
+    # logit bias == weight times g_j, renormalised (the literal reading of Figure 1(c))
+    for i in (3, 16):
+        w = orc.gated_attention_weights(Q[i, 0], K[: i + 1, 0], np.exp(lg[: i + 1]), 0.5)
+        np.testing.assert_allclose(w @ V[: i + 1, 0], O[i, 0], rtol=1e-12, atol=1e-12)
+        assert abs(w.sum() - 1.0) < 1e-12
+
+
+def test_dropped_tokens_do_not_matter():
+    # layers above L see only the kept tokens: perturbing dropped rows changes nothing
+    wl = ti.scaled(ti.WORKLOADS["tiny_f32"], seqlens=(96, 40), q_len=(8, 4), k=(16, 9))
+    H = ti.hidden_states(wl)
+    s = ti.rng(wl, "scores").standard_normal(wl.n_tok).astype(np.float32)
+    kept, cu = orc.topk_select(s, wl.seqlens, wl.q_len, wl.k)
+    H2 = H.copy()
+    dropped = np.setdiff1d(np.arange(wl.n_tok), kept)
+    H2[dropped] = 1e3
+    out1 = orc.prefill_from_scores(H, s, wl.seqlens, wl.q_len, wl.k, [], 4, 2, 0.125)
+    out2 = orc.prefill_from_scores(H2, s, wl.seqlens, wl.q_len, wl.k, [], 4, 2, 0.125)
+    assert np.array_equal(out1["H_kept"], out2["H_kept"])
+    Hk64 = out1["H_kept"].astype(np.float64)
+    layers = [ti.project_kept(wl, Hk64)]
+    a1 = orc.prefill_from_scores(H, s, wl.seqlens, wl.q_len, wl.k, layers, 4, 2, 0.125)["attn"]
+    a2 = orc.prefill_from_scores(H2, s, wl.seqlens, wl.q_len, wl.k, layers, 4, 2, 0.125)["attn"]
+    assert np.array_equal(a1[0][0], a2[0][0])
+
+
+def test_softmax_rows_sum_to_one():
+    g = np.random.default_rng(9)
+    M, D = 30, 5
+    Q = g.standard_normal((M, 1, D))
+    K = g.standard_normal((M, 1, D))
+    lg = np.log(g.uniform(0.01, 1, M))
+    # with V = identity-like one-hot columns the output rows are the weights themselves
+    V = np.zeros((M, 1, M))
+    V[np.arange(M), 0, np.arange(M)] = 1.0
+    Qp = np.concatenate([Q, np.zeros((M, 1, M - D))], axis=2)
+    Kp = np.concatenate([K, np.zeros((M, 1, M - D))], axis=2)
+    O, _ = orc.gated_attention(Qp, Kp, V, lg, np.arange(M), [0, M], 1, 1, 0.3)
+    P = O[:, 0, :]
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert np.all(np.triu(P, 1) == 0.0)  # causal
+
+
+def test_planted_spans_are_kept_when_salient():
+    wl = ti.scaled(ti.WORKLOADS["qwen3_32k"], seqlens=(4096,), q_len=(64,), k=(409,))
+    s = ti.stage_scores(wl)
+    m = ti.planted_mask(wl)
+    kept, _ = orc.topk_select(s, wl.seqlens, wl.q_len, wl.k)
+    frac = m[kept[:409]].mean()
+    assert frac > 0.8  # +3 sigma offsets dominate the kept set
