@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Throughput of the TokenGate gated-prefill hot path on B200.
+
+One step = the whole path over one synthetic batch: gate-MLP score of every token ->
+top-K with the question tail -> gather of the kept rows -> token-gated causal attention
+(one above-L layer), each through the C ABI of libtokengate. Default workload: N=32768
+tokens, question tail 128, K=2048 (2176 kept rows), d=2048, gate 2048->256->1, 16 query /
+8 KV heads, head_dim 128, bf16 (Qwen3-1.7B shapes; seeded synthetic data).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tokengate|reference]
+
+Prints ONE JSON line on rank 0. With N > 1 (torchrun) every rank runs an independent
+replica of the workload (the path needs no exchange between GPUs) and value = tokens of
+all ranks / max-over-ranks time. ``--impl reference`` times the CPU oracle instead, on a
+bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "gated-prefill tokens/s at N=32K,K=2K; gated-attn TFLOP/s and % of bf16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="tokengate", choices=["tokengate", "reference"])
+    ap.add_argument("--workload", default="qwen3_32k")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-full-ref", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) every 5 ms."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.error = repr(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def start(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._t.is_alive():
+            self._t.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml", "note": getattr(self, "error", "no samples")}
+        busy = [m for m, r in self.samples if not (r & 0x1)] or [m for m, _ in self.samples]
+        seen = 0
+        for _, r in self.samples:
+            seen |= r
+        names = [k for k, v in self.REASONS.items() if seen & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples), "source": "nvml 5 ms"}
+
+
+# --------------------------------------------------------------------------- oracle timing
+
+
+def oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_score_tok, n_attn_rows):
+    """Times the CPU oracle on a bounded sample of one step and scales it to the whole step.
+
+    Score: the first n_score_tok tokens (time x N / n_score_tok). Select and gather: full.
+    Attention: n_attn_rows query rows spread over the sequence, all heads (time x M / rows).
+    Returns (estimated seconds per step, description)."""
+    import numpy as np
+
+    import tg_inputs as ti
+    from oracle import tg_oracle as orc
+
+    W64, w64 = ti.widen(W1, wl.dtype), ti.widen(w2, wl.dtype)
+    t0 = time.perf_counter()
+    orc.gate_scores(ti.widen(H[:n_score_tok], wl.dtype), W64, b1, w64, b2)
+    t_score = (time.perf_counter() - t0) * wl.n_tok / n_score_tok
+    t0 = time.perf_counter()
+    kept, cu = orc.topk_select(s_full, wl.seqlens, wl.q_len, wl.k)
+    t_sel = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    _, pos, _, lg = orc.gather(H, s_full, kept, wl.seqlens, wl.q_len, cu)
+    t_gat = time.perf_counter() - t0
+    Q, K, V = (ti.widen(x, wl.dtype) for x in layer)
+    m = int(cu[-1])
+    rows = np.linspace(0, m - 1, n_attn_rows).astype(np.int64)
+    t0 = time.perf_counter()
+    orc.gated_attention(Q, K, V, lg, pos, cu, wl.Hq, wl.Hkv, 1.0 / math.sqrt(wl.D), rows=rows)
+    t_att = (time.perf_counter() - t0) * m / n_attn_rows
+    desc = (f"score on {n_score_tok} of {wl.n_tok} tokens (scaled), full select and gather, attention on "
+            f"{n_attn_rows} of {m} query rows x {wl.Hq} heads (scaled)")
+    return t_score + t_sel + t_gat + t_att, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------------------- main
+
+
+def kernel_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "learned_token_pruning_02_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel_key, src_hash):
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel_key)
+        if e and e.get("source_hash") == src_hash:
+            return e.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+def run_reference(args, wl):
+    import numpy as np
+
+    import tg_inputs as ti
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    H = ti.hidden_states(wl)
+    W1, b1, w2, b2 = ti.gate_weights(wl)
+    s_full = ti.stage_scores(wl) if wl.score_mode != "mlp" else np.random.default_rng(0).standard_normal(
+        wl.n_tok).astype(np.float32)
+    layer = ti.qkv(wl, 0)
+    # per-step sample sized so that warmup + steps end within about two minutes
+    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    n_tok, n_rows = 64, 4
+    est, _ = oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_tok, n_rows)
+    t0 = time.perf_counter()
+    oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_tok, n_rows)
+    wall = time.perf_counter() - t0
+    grow = max(1.0, min(64.0, budget / max(wall, 1e-3)))
+    n_tok, n_rows = int(min(wl.n_tok, n_tok * grow)), int(min(wl.m_tot, max(4, n_rows * grow)))
+    for _ in range(args.warmup):
+        oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_tok, n_rows)
+    ests = []
+    for _ in range(args.steps):
+        e, desc = oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_tok, n_rows)
+        ests.append(e)
+    t_step = sum(ests) / len(ests)
+    value = wl.n_tok / t_step
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl):
+    return {
+        "workload": f"{wl.name}: N={'+'.join(map(str, wl.seqlens))}, question tail {'+'.join(map(str, wl.q_len))}, "
+                    f"K={'+'.join(map(str, wl.k))}, d={wl.d}, gate {wl.d}->{wl.dg}->1 GELU, {wl.Hq}/{wl.Hkv} heads, "
+                    f"head_dim {wl.D}, {wl.n_layers} above-L layer(s), {wl.dtype}",
+        "global_batch": wl.B, "seq_len": max(wl.seqlens), "kept_rows": wl.m_tot,
+        "parallelism": "replicas (one independent workload per GPU)",
+        "l2": "flushed between timed steps (512 MiB memset)",
+    }
+
+
+def main():
+    args = parse()
+    import tg_inputs as ti
+
+    wl = ti.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import learned_token_pruning_02_b200 as tg
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    # ---------------- inputs (seeded, identical on every rank: weak-scaling replicas)
+    Hn = ti.hidden_states(wl)
+    W1n, b1n, w2n, b2 = ti.gate_weights(wl)
+    lay = [ti.qkv(wl, l) for l in range(wl.n_layers)]
+    H_host = bf(Hn).pin_memory()
+    qkv_host = [tuple(bf(x).pin_memory() for x in L) for L in lay]
+    H = H_host.to(dev)
+    W1, b1, w2 = bf(W1n).to(dev), torch.from_numpy(b1n).to(dev), bf(w2n).to(dev)
+    layers = [tuple(x.to(dev) for x in L) for L in qkv_host]
+    cu = tg.tg_kept_counts(wl.seqlens, wl.q_len, wl.k)
+    M = cu[-1]
+    scale = 1.0 / math.sqrt(wl.D)
+    score = torch.empty(wl.n_tok, device=dev, dtype=torch.float32)
+    kept = torch.empty(M, device=dev, dtype=torch.int32)
+    cu_dev = torch.empty(wl.B + 1, device=dev, dtype=torch.int32)
+    Hk = torch.empty(M, wl.d, device=dev, dtype=torch.bfloat16)
+    pos = torch.empty(M, device=dev, dtype=torch.int32)
+    g = torch.empty(M, device=dev, dtype=torch.float32)
+    logg = torch.empty(M, device=dev, dtype=torch.float32)
+    Os = [torch.empty_like(L[0]) for L in layers]
+    status = torch.zeros(1, device=dev, dtype=torch.int32)
+    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        tg.tg_score(H, W1, b1, w2, b2, score=score)
+        if ev:
+            ev[1].record(stream)
+        tg.tg_topk_select(score, wl.seqlens, wl.q_len, wl.k, kept_idx=kept, cu_kept_dev=cu_dev, dev_status=status)
+        if ev:
+            ev[2].record(stream)
+        tg.tg_gather(H, score, kept, wl.seqlens, wl.q_len, wl.k, H_kept=Hk, pos=pos, g=g, logg=logg,
+                     dev_status=status)
+        if ev:
+            ev[3].record(stream)
+        for li, (q, k, v) in enumerate(layers):
+            tg.tg_gated_attn_fwd(q, k, v, logg, pos, cu, scale, O=Os[li], want_lse=False, dev_status=status)
+        if ev:
+            ev[4].record(stream)
+
+    launches_per_step = 4 + (wl.n_layers - 1)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local).start()
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush, outside the timed events
+        torch.cuda._sleep(300_000)  # lets the host queue the step's launches ahead of the GPU
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    st_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    step_ms = st_ms.sum(axis=1)
+    t_total = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([t_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_total = float(t.item())
+    ms_per_step = t_total / args.steps
+    value = wl.n_tok * world * args.steps / (t_total / 1e3)
+    stage_ms = st_ms.mean(axis=0)
+    dev_status = int(status.item())
+
+    # ---------------- roofline of the dominant kernel
+    pk, pk_src = peaks()
+    flops_attn = 4.0 * wl.Hq * wl.D * sum(m * (m + 1) / 2 for m in np.diff(cu)) * wl.n_layers
+    attn_s = stage_ms[3] / 1e3 / wl.n_layers
+    attn_tflops = flops_attn / wl.n_layers / attn_s / 1e12
+    bytes_score = wl.n_tok * wl.d * 2 + wl.n_tok * 4 + wl.dg * wl.d * 2
+    score_gbs = bytes_score / (stage_ms[0] / 1e3) / 1e9
+    bytes_gather = M * wl.d * 2 * 2 + M * 4 * 4
+    bytes_select = (wl.n_tok - sum(wl.q_len)) * 4 + M * 4
+    dominant = int(np.argmax(stage_ms))
+    names = ["score", "select", "gather", "gated_attn"]
+    if dominant == 3:
+        roof = {"kernel": "gated_attn", "bound": "tensor", "achieved": attn_tflops, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": attn_tflops / pk["bf16_tflops"],
+                "traffic": traffic_from_profile("gated_attn", kernel_hash("tg_attn_tc.cu") if os.path.exists(
+                    os.path.join(ROOT, "learned_token_pruning_02_b200", "csrc", "tg_attn_tc.cu")) else "")}
+    else:
+        nm = names[dominant]
+        byts = [bytes_score, bytes_select, bytes_gather][dominant]
+        gbs = byts / (stage_ms[dominant] / 1e3) / 1e9
+        src = {"score": "tg_score_tc.cu", "select": "tg_select.cu", "gather": "tg_gather.cu"}[nm]
+        srcp = os.path.join(ROOT, "learned_token_pruning_02_b200", "csrc", src)
+        roof = {"kernel": nm, "bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"],
+                "traffic": traffic_from_profile(nm, kernel_hash(src) if os.path.exists(srcp) else "")}
+    roof["peak_source"] = f"{pk_src} ({'burst' if roof['bound'] == 'tensor' else 'copy'})"
+
+    # ---------------- end to end through the public API, host buffers in and out
+    e2e = None
+    if args.e2e_steps > 0:
+        O_host = [torch.empty(L[0].shape, dtype=torch.bfloat16).pin_memory() for L in layers]
+        kept_host = torch.empty(M, dtype=torch.int32).pin_memory()
+        out = {"score": score, "kept_idx": kept, "cu_kept_dev": cu_dev, "H_kept": Hk, "pos": pos, "g": g,
+               "logg": logg, "O": Os, "lse": [None] * len(layers)}
+
+        def e2e_step():
+            H.copy_(H_host, non_blocking=True)
+            for (q, k, v), (qh, kh, vh) in zip(layers, qkv_host):
+                q.copy_(qh, non_blocking=True)
+                k.copy_(kh, non_blocking=True)
+                v.copy_(vh, non_blocking=True)
+            tg.tg_prefill_above_L(H, W1, b1, w2, b2, wl.seqlens, wl.q_len, wl.k, layers, scale, out=out,
+                                  dev_status=status)
+            for o, oh in zip(Os, O_host):
+                oh.copy_(o, non_blocking=True)
+            kept_host.copy_(kept, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([t], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            t = float(tt.item())
+        h2d = H.numel() * 2 + sum(x.numel() * 2 for L in layers for x in L)
+        d2h = sum(o.numel() * 2 for o in Os) + M * 4
+        e2e = {"value": wl.n_tok * world * args.e2e_steps / (t / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": t / args.e2e_steps, "api": "tg_prefill_above_L", "steps": args.e2e_steps}
+
+    # ---------------- unpruned causal attention at the full length (reference point)
+    full_ref = None
+    if not args.no_full_ref and rank == 0:
+        n = max(wl.seqlens)
+        gq = torch.Generator(device=dev).manual_seed(7)
+        q = (torch.randn(n, wl.Hq, wl.D, device=dev, generator=gq) / math.sqrt(128)).to(torch.bfloat16)
+        k = (torch.randn(n, wl.Hkv, wl.D, device=dev, generator=gq) / math.sqrt(128)).to(torch.bfloat16)
+        v = (torch.randn(n, wl.Hkv, wl.D, device=dev, generator=gq) / math.sqrt(128)).to(torch.bfloat16)
+        p = torch.arange(n, device=dev, dtype=torch.int32)
+        o = torch.empty_like(q)
+        reps = 3
+        for _ in range(1):
+            tg.tg_gated_attn_fwd(q, k, v, None, p, [0, n], scale, O=o, want_lse=False)
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            tg.tg_gated_attn_fwd(q, k, v, None, p, [0, n], scale, O=o, want_lse=False)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ms = a0.elapsed_time(a1) / reps
+        fl = 4.0 * wl.Hq * wl.D * n * (n + 1) / 2
+        full_ref = {"n": n, "ms": ms, "tflops": fl / (ms / 1e3) / 1e12,
+                    "note": "unpruned causal attention over all N tokens (g == 1), same kernel"}
+        del q, k, v, o
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s_full = score.cpu().numpy()
+        est, desc = oracle_sample(wl, Hn, W1n, b1n, w2n, b2, s_full, lay[0], 8192, 256)
+        cpu = {"value": wl.n_tok / est, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc, "host_cpus": os.cpu_count()}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; Qwen3-1.7B shapes)",
+            "config": workload_config(wl),
+            "stages_us": {n: float(x * 1e3) for n, x in zip(names, stage_ms)},
+            "gated_attn_tflops": attn_tflops,
+            "gated_attn_frac_of_bf16_peak": attn_tflops / pk["bf16_tflops"],
+            "score_hbm_gbs": score_gbs,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "full_attention_reference": full_ref,
+            "device_status": dev_status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,184 @@
+/*
+ * tokengate.h - C ABI of the TokenGate gated-prefill hot path for NVIDIA B200 (sm_100a).
+ *
+ * The method (TokenGate: Adapting LLMs for Fast and Memory-Efficient Prefill with Learned
+ * Token Pruning): at a selection layer L a small gate MLP scores every token's hidden
+ * state; a top-K selector keeps K context tokens and always keeps the question tail; the
+ * kept hidden states travel upward with their gate values and original positions; every
+ * layer above L runs token-gated causal attention over the kept tokens only, each
+ * attention weight multiplied by its key's gate value g_j (row renormalised).
+ *
+ * Conventions shared by every entry point
+ *   - Memory: every buffer is owned by the caller. Pointers named "device" must be CUDA
+ *     device memory of the current device; "host" pointers are ordinary host memory that
+ *     is read before the call returns. No entry point allocates or frees memory.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All GPU work is enqueued asynchronously on it; nothing synchronises the host and no
+ *     device-to-host copy is made, so a chain of calls can be captured in a CUDA graph.
+ *   - Layout: tokens are packed back to back ("varlen", token-major). Sequence b occupies
+ *     rows [cu_seqlens[b], cu_seqlens[b+1]) of the hidden states and rows
+ *     [cu_kept[b], cu_kept[b+1]) of every kept-token tensor.
+ *   - Errors: argument problems are reported synchronously before anything is launched
+ *     (TG_ERR_INVALID_ARG / TG_ERR_UNSUPPORTED). A failed launch returns TG_ERR_CUDA.
+ *     Problems found by the kernels are OR-ed into the optional device status word
+ *     (int32, TG_DEV_* bits), which the caller zeroes beforehand and reads after a sync.
+ *     No kernel traps, asserts or waits without a bound. tg_last_error() describes the
+ *     most recent failure on the calling thread.
+ *   - dtype: TG_F32 means every floating-point tensor named "act" below is float32;
+ *     TG_BF16 means bfloat16. Biases, scores, gate values, LSE are always float32.
+ */
+#ifndef TOKENGATE_H
+#define TOKENGATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TG_OK = 0,
+  TG_ERR_INVALID_ARG = 1,   /* null pointer, negative size, inconsistent sizes */
+  TG_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes / alignment / GPU */
+  TG_ERR_WORKSPACE = 3,     /* reserved: no entry point needs a workspace */
+  TG_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  TG_ERR_DEVICE_CHECK = 5,  /* reserved for callers that map TG_DEV_* bits to a status */
+  TG_ERR_DEVICE_TIMEOUT = 6 /* reserved for callers that map TG_DEV_TIMEOUT to a status */
+} tg_status;
+
+typedef enum { TG_F32 = 0, TG_BF16 = 1 } tg_dtype;
+
+/* flags */
+#define TG_ATTN_UNNORMALISED (1u << 0) /* weight times g_j without renormalising the row */
+#define TG_QUESTION_GATE_ONE (1u << 1) /* question-tail rows get g = 1 (log g = 0)       */
+
+/* device status word bits */
+#define TG_DEV_NAN_SCORE (1 << 0)        /* a context score was NaN (ranked below -inf) */
+#define TG_DEV_POS_NOT_ASCENDING (1 << 1)/* kept positions not strictly ascending         */
+#define TG_DEV_TIMEOUT (1 << 2)          /* a bounded wait inside a kernel gave up        */
+#define TG_DEV_BAD_INDEX (1 << 3)        /* a kept index lay outside its own sequence     */
+
+/* Limits. A sequence's context (N - q) may hold up to TG_MAX_CTX tokens. */
+#define TG_MAX_CTX 262144
+
+/* Per-sequence description of a packed batch. All three arrays are HOST memory of length B.
+ * seqlens[b] = N_b >= 0 tokens; q_len[b] = question-tail length, 0 <= q_b <= N_b;
+ * k[b] = number of context tokens to keep (values < 0 read as 0, values > N_b - q_b keep
+ * the whole context). */
+typedef struct {
+  int32_t B;
+  const int32_t* seqlens;
+  const int32_t* q_len;
+  const int32_t* k;
+} tg_seqs;
+
+/* Human-readable name of a status code. */
+const char* tg_status_string(int32_t status);
+
+/* Description of the most recent failed call on this thread ("" if none). */
+const char* tg_last_error(void);
+
+/* ABI version, (major << 16) | minor. */
+int32_t tg_version(void);
+
+/* Kept-row offsets (host only, no GPU work). M_b = min(max(k_b, 0), N_b - q_b) + q_b: the
+ * K highest-scoring context tokens plus the whole question tail (aitualizate.com TokenGate
+ * article, phase 2: only the document part may be pruned, the question never is).
+ * cu_kept_host: HOST int32 [B+1], written with the exclusive prefix sums of M_b. */
+tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host);
+
+/* Gate MLP score of every token (aitualizate.com TokenGate article, phase 2: an MLP scores
+ * each token's post-attention residual state at layer L; thelatestinai.com TokenGate page,
+ * Figure 1(b)):   score[i] = w2 . GELU(W1 h_i + b1) + b2,  GELU with the exact erf.
+ *   H      device act [n_tok, d], row stride ldh elements (ldh >= d)
+ *   W1     device act [dg, d] row-major (output-major, like torch.nn.Linear.weight)
+ *   b1     device f32 [dg], or NULL for zero
+ *   w2     device act [dg]
+ *   b2     scalar
+ *   score  device f32 [n_tok] (written)
+ * Supported: dg in {64, 128, 256}; d % 64 == 0; ldh * sizeof(act) % 16 == 0; 16-byte
+ * aligned H and W1. bf16 runs on the tensor cores with fp32 accumulation; f32 runs on the
+ * CUDA cores in fp32. */
+tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, int32_t d,
+                   const void* W1, const float* b1, const void* w2, float b2, int32_t dg,
+                   float* score, void* stream);
+
+/* Top-K over each sequence's context with the question tail always kept (aitualizate.com
+ * TokenGate article, phase 2; thelatestinai.com TokenGate page, Figure 1(a)-(b)).
+ * Per sequence the min(k_b, N_b - q_b) context tokens with the largest scores are kept;
+ * equal scores keep the lower index; -0 equals +0; NaN ranks below -inf (and sets
+ * TG_DEV_NAN_SCORE). The kept context indices, ascending, are followed by the q_b tail
+ * indices. Exact and deterministic.
+ *   score       device f32 [sum N_b]
+ *   kept_idx    device int32 [sum M_b] (written): packed row indices into H / score
+ *   cu_kept_dev device int32 [B+1] (written) or NULL
+ *   dev_status  device int32 [1] or NULL
+ * Supported: N_b - q_b <= TG_MAX_CTX. */
+tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
+                         int32_t* cu_kept_dev, int32_t* dev_status, void* stream);
+
+/* Forward the kept hidden states with their gate values and positions (thelatestinai.com
+ * TokenGate page, Figure 1(b): the selector forwards the kept hidden states together with
+ * their importance scores; aitualizate.com article, phase 3).
+ *   H        device act [sum N_b, d], row stride ldh
+ *   score    device f32 [sum N_b]
+ *   kept_idx device int32 [sum M_b], packed indices as written by tg_topk_select
+ *   H_kept   device act [sum M_b, d] contiguous (written; a bit-exact copy of the rows)
+ *   pos      device int32 [sum M_b] (written): index of the row within its own sequence
+ *   g, logg  device f32 [sum M_b] (written): g = sigmoid(score), log g as a stable
+ *            log-sigmoid; with TG_QUESTION_GATE_ONE the tail rows get g = 1, log g = 0.
+ *            Either may be NULL.
+ * A kept index outside its sequence sets TG_DEV_BAD_INDEX and its row is left unwritten.
+ * Supported: d * sizeof(act) % 16 == 0, ldh * sizeof(act) % 16 == 0, 16-byte aligned. */
+tg_status tg_gather(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const float* score,
+                    const int32_t* kept_idx, const tg_seqs* seqs, uint32_t flags, void* H_kept,
+                    int32_t* pos, float* g, float* logg, int32_t* dev_status, void* stream);
+
+/* Token-gated causal attention over the kept tokens (thelatestinai.com TokenGate page,
+ * Figure 1(c): each attention weight is multiplied by its key's gate value g_j; read with
+ * the row renormalised this is log g_j added to the logit; aitualizate.com article: the
+ * score acts as a bias on the attention logits with a per-head gain). For sequence b,
+ * query row i and head h (KV head h / (Hq / Hkv)):
+ *   S_ij = softmax_scale * q_i . k_j + gain_h * log g_j   for pos_j <= pos_i (same sequence)
+ *   O_i  = sum_j softmax_j(S_ij) v_j ;  lse_i = logsumexp_j S_ij (natural log)
+ * With TG_ATTN_UNNORMALISED: O_i = sum_j softmax_j(softmax_scale q_i . k_j) g_j^gain_h v_j
+ * and lse is that of the unbiased logits.
+ *   Q            device act [sum M_b, Hq, D];  K, V device act [sum M_b, Hkv, D]
+ *   logg         device f32 [sum M_b], or NULL for g == 1
+ *   head_gain    device f32 [Hq], or NULL for gain 1
+ *   pos          device int32 [sum M_b]: must be strictly ascending inside each sequence
+ *                (as tg_gather writes them); otherwise TG_DEV_POS_NOT_ASCENDING is set.
+ *   cu_kept_host HOST int32 [B+1] kept-row offsets (tg_kept_counts)
+ *   O            device act [sum M_b, Hq, D] (written)
+ *   lse          device f32 [Hq, sum M_b] (written) or NULL
+ * Supported: D in {64, 128}; Hq % Hkv == 0; 16-byte aligned tensors. bf16 runs on the
+ * tensor cores (fp32 softmax and accumulation); f32 runs on the CUDA cores in fp32. */
+tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const void* V,
+                            const float* logg, const float* head_gain, const int32_t* pos,
+                            const int32_t* cu_kept_host, int32_t B, int32_t Hq, int32_t Hkv,
+                            int32_t D, float softmax_scale, uint32_t flags, void* O,
+                            float* lse, int32_t* dev_status, void* stream);
+
+/* The whole gated path above layer L (aitualizate.com TokenGate article, phases 2-3;
+ * thelatestinai.com TokenGate page, Figure 1(a)): tg_score -> tg_topk_select -> tg_gather
+ * -> tg_gated_attn_fwd for each of n_layers above-L layers, enqueued on one stream with no
+ * host synchronisation. Q, K, V, O, lse are HOST arrays of n_layers device pointers shaped
+ * as in tg_gated_attn_fwd (lse may be NULL, or hold NULL entries). The other arguments and
+ * outputs are those of the single steps; score, kept_idx, H_kept, pos, g, logg are all
+ * required here. */
+tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t d,
+                             const void* W1, const float* b1, const void* w2, float b2,
+                             int32_t dg, const tg_seqs* seqs, int32_t n_layers,
+                             const void* const* Q, const void* const* K, const void* const* V,
+                             int32_t Hq, int32_t Hkv, int32_t D, float softmax_scale,
+                             const float* head_gain, uint32_t flags, float* score,
+                             int32_t* kept_idx, int32_t* cu_kept_dev, void* H_kept, int32_t* pos,
+                             float* g, float* logg, void* const* O, float* const* lse,
+                             int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOKENGATE_H */

@@ -1,0 +1,251 @@
+"""TokenGate gated-prefill hot path for B200 (sm_100a): thin Python binding of libtokengate.
+
+Every function here marshals torch tensors into the C ABI declared in include/tokengate.h
+and calls it; all computation runs in the library's CUDA kernels. There is no CPU path:
+if the shared library is missing, or the tensors are not on a CUDA device, calls raise.
+
+Build the library in-tree with ``python -m learned_token_pruning_02_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtokengate.so")
+
+TG_F32, TG_BF16 = 0, 1
+TG_ATTN_UNNORMALISED = 1 << 0
+TG_QUESTION_GATE_ONE = 1 << 1
+TG_DEV_NAN_SCORE = 1 << 0
+TG_DEV_POS_NOT_ASCENDING = 1 << 1
+TG_DEV_TIMEOUT = 1 << 2
+TG_DEV_BAD_INDEX = 1 << 3
+TG_MAX_CTX = 262144
+
+EXPORTS = (
+    "tg_status_string", "tg_last_error", "tg_version", "tg_kept_counts", "tg_score",
+    "tg_topk_select", "tg_gather", "tg_gated_attn_fwd", "tg_prefill_above_L",
+)
+
+
+class TokenGateError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {msg}")
+        self.status = status
+
+
+class tg_seqs(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32),
+        ("seqlens", ctypes.POINTER(ctypes.c_int32)),
+        ("q_len", ctypes.POINTER(ctypes.c_int32)),
+        ("k", ctypes.POINTER(ctypes.c_int32)),
+    ]
+
+
+_VP = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_U32 = ctypes.c_uint32
+_SEQP = ctypes.POINTER(tg_seqs)
+_lib_handle = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtokengate.so (once). Raises if it has not been built."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libtokengate.so not found at {LIB_PATH}; build it with "
+            "`python -m learned_token_pruning_02_b200.build` (no CPU fallback exists)")
+    L = ctypes.CDLL(LIB_PATH)
+    L.tg_status_string.restype = ctypes.c_char_p
+    L.tg_status_string.argtypes = [_I32]
+    L.tg_last_error.restype = ctypes.c_char_p
+    L.tg_last_error.argtypes = []
+    L.tg_version.restype = _I32
+    L.tg_kept_counts.restype = _I32
+    L.tg_kept_counts.argtypes = [_SEQP, ctypes.POINTER(_I32)]
+    L.tg_score.restype = _I32
+    L.tg_score.argtypes = [_I32, _VP, _I64, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP]
+    L.tg_topk_select.restype = _I32
+    L.tg_topk_select.argtypes = [_VP, _SEQP, _VP, _VP, _VP, _VP]
+    L.tg_gather.restype = _I32
+    L.tg_gather.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _SEQP, _U32, _VP, _VP, _VP, _VP, _VP, _VP]
+    L.tg_gated_attn_fwd.restype = _I32
+    L.tg_gated_attn_fwd.argtypes = [_I32, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(_I32), _I32, _I32,
+                                    _I32, _I32, _F, _U32, _VP, _VP, _VP, _VP]
+    L.tg_prefill_above_L.restype = _I32
+    L.tg_prefill_above_L.argtypes = [
+        _I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _I32, _SEQP, _I32,
+        ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP),
+        _I32, _I32, _I32, _F, _VP, _U32, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+        ctypes.POINTER(_VP), ctypes.POINTER(_VP), _VP, _VP]
+    _lib_handle = L
+    return L
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        L = lib()
+        raise TokenGateError(fn, st, f"{L.tg_status_string(st).decode()}: {L.tg_last_error().decode()}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TG_BF16
+    if t.dtype == torch.float32:
+        return TG_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libtokengate works on CUDA tensors only (there is no CPU path)")
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+class Seqs:
+    """Host-side sequence description (keeps the int32 arrays alive for the call)."""
+
+    def __init__(self, seqlens, q_len, k):
+        n = len(seqlens)
+        assert len(q_len) == n and len(k) == n
+        self._arrs = [(ctypes.c_int32 * max(n, 1))(*[int(x) for x in a]) for a in (seqlens, q_len, k)]
+        self.s = tg_seqs(n, *[ctypes.cast(a, ctypes.POINTER(ctypes.c_int32)) for a in self._arrs])
+        self.B = n
+
+    def ref(self):
+        return ctypes.byref(self.s)
+
+
+def tg_kept_counts(seqlens, q_len, k) -> list:
+    """cu_kept offsets (host list of B+1 ints)."""
+    s = Seqs(seqlens, q_len, k)
+    out = (ctypes.c_int32 * (s.B + 1))()
+    _check("tg_kept_counts", lib().tg_kept_counts(s.ref(), out))
+    return list(out)
+
+
+def tg_score(H, W1, b1, w2, b2: float, score=None, stream=None):
+    """Gate-MLP score of every token: w2 . GELU(W1 h + b1) + b2 (float32 [n_tok])."""
+    _cuda(H, W1, b1, w2, score)
+    n_tok, d = H.shape
+    assert H.stride(1) == 1 and W1.is_contiguous() and w2.is_contiguous()
+    if score is None:
+        score = torch.empty(n_tok, device=H.device, dtype=torch.float32)
+    _check("tg_score", lib().tg_score(_dtype(H), _ptr(H), H.stride(0), n_tok, d, _ptr(W1), _ptr(b1), _ptr(w2),
+                                      float(b2), W1.shape[0], _ptr(score), _stream(stream)))
+    return score
+
+
+def tg_topk_select(score, seqlens, q_len, k, kept_idx=None, cu_kept_dev=None, dev_status=None, stream=None):
+    """Top-K context tokens per sequence plus the question tail (int32 kept_idx, cu_kept_dev)."""
+    _cuda(score, kept_idx, cu_kept_dev, dev_status)
+    s = Seqs(seqlens, q_len, k)
+    cu = tg_kept_counts(seqlens, q_len, k)
+    if kept_idx is None:
+        kept_idx = torch.empty(cu[-1], device=score.device, dtype=torch.int32)
+    if cu_kept_dev is None:
+        cu_kept_dev = torch.empty(s.B + 1, device=score.device, dtype=torch.int32)
+    _check("tg_topk_select", lib().tg_topk_select(_ptr(score), s.ref(), _ptr(kept_idx), _ptr(cu_kept_dev),
+                                                  _ptr(dev_status), _stream(stream)))
+    return kept_idx, cu_kept_dev
+
+
+def tg_gather(H, score, kept_idx, seqlens, q_len, k, flags=0, H_kept=None, pos=None, g=None, logg=None,
+              dev_status=None, stream=None):
+    """Kept rows of H with their positions and gate values: (H_kept, pos, g, logg)."""
+    _cuda(H, score, kept_idx, H_kept, pos, g, logg, dev_status)
+    s = Seqs(seqlens, q_len, k)
+    m = kept_idx.numel()
+    d = H.shape[1]
+    dev = H.device
+    H_kept = torch.empty(m, d, device=dev, dtype=H.dtype) if H_kept is None else H_kept
+    pos = torch.empty(m, device=dev, dtype=torch.int32) if pos is None else pos
+    g = torch.empty(m, device=dev, dtype=torch.float32) if g is None else g
+    logg = torch.empty(m, device=dev, dtype=torch.float32) if logg is None else logg
+    _check("tg_gather", lib().tg_gather(_dtype(H), _ptr(H), H.stride(0), d, _ptr(score), _ptr(kept_idx), s.ref(),
+                                        int(flags), _ptr(H_kept), _ptr(pos), _ptr(g), _ptr(logg), _ptr(dev_status),
+                                        _stream(stream)))
+    return H_kept, pos, g, logg
+
+
+def tg_gated_attn_fwd(Q, K, V, logg, pos, cu_kept, softmax_scale: float, head_gain=None, flags=0, O=None,
+                      lse=None, want_lse=True, dev_status=None, stream=None):
+    """Token-gated causal attention over the kept tokens: (O [M, Hq, D], lse [Hq, M] or None)."""
+    _cuda(Q, K, V, logg, pos, head_gain, O, lse, dev_status)
+    M, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    assert Q.is_contiguous() and K.is_contiguous() and V.is_contiguous()
+    cu = [int(x) for x in cu_kept]
+    B = len(cu) - 1
+    cu_arr = (ctypes.c_int32 * len(cu))(*cu)
+    O = torch.empty_like(Q) if O is None else O
+    if lse is None and want_lse:
+        lse = torch.empty(Hq, M, device=Q.device, dtype=torch.float32)
+    _check("tg_gated_attn_fwd", lib().tg_gated_attn_fwd(
+        _dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(logg), _ptr(head_gain), _ptr(pos), cu_arr, B, Hq, Hkv, D,
+        float(softmax_scale), int(flags), _ptr(O), _ptr(lse), _ptr(dev_status), _stream(stream)))
+    return O, lse
+
+
+def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_scale, head_gain=None, flags=0,
+                       want_lse=False, out=None, dev_status=None, stream=None):
+    """The whole gated path above layer L: score -> top-K -> gather -> gated attention per layer.
+
+    layers: list of (Q, K, V) device tensors shaped by the kept count. Returns a dict of the
+    outputs (score, kept_idx, cu_kept_dev, H_kept, pos, g, logg, O list, lse list). Pass
+    ``out`` (a dict from an earlier call) to reuse its buffers.
+    """
+    _cuda(H, W1, b1, w2, head_gain, dev_status)
+    s = Seqs(seqlens, q_len, k)
+    cu = tg_kept_counts(seqlens, q_len, k)
+    m = cu[-1]
+    n_tok, d = H.shape
+    dev = H.device
+    nl = len(layers)
+    Hq = layers[0][0].shape[1] if nl else 1
+    Hkv = layers[0][1].shape[1] if nl else 1
+    D = layers[0][0].shape[2] if nl else 64
+    if out is None:
+        out = {
+            "score": torch.empty(n_tok, device=dev, dtype=torch.float32),
+            "kept_idx": torch.empty(m, device=dev, dtype=torch.int32),
+            "cu_kept_dev": torch.empty(s.B + 1, device=dev, dtype=torch.int32),
+            "H_kept": torch.empty(m, d, device=dev, dtype=H.dtype),
+            "pos": torch.empty(m, device=dev, dtype=torch.int32),
+            "g": torch.empty(m, device=dev, dtype=torch.float32),
+            "logg": torch.empty(m, device=dev, dtype=torch.float32),
+            "O": [torch.empty_like(q) for (q, _, _) in layers],
+            "lse": [torch.empty(Hq, m, device=dev, dtype=torch.float32) if want_lse else None for _ in layers],
+        }
+    qa = (_VP * max(nl, 1))(*[t[0].data_ptr() for t in layers])
+    ka = (_VP * max(nl, 1))(*[t[1].data_ptr() for t in layers])
+    va = (_VP * max(nl, 1))(*[t[2].data_ptr() for t in layers])
+    oa = (_VP * max(nl, 1))(*[t.data_ptr() for t in out["O"]])
+    la = (_VP * max(nl, 1))(*[(t.data_ptr() if t is not None else None) for t in out["lse"]])
+    _check("tg_prefill_above_L", lib().tg_prefill_above_L(
+        _dtype(H), _ptr(H), H.stride(0), d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2), W1.shape[0], s.ref(), nl,
+        qa, ka, va, Hq, Hkv, D, float(softmax_scale), _ptr(head_gain), int(flags), _ptr(out["score"]),
+        _ptr(out["kept_idx"]), _ptr(out["cu_kept_dev"]), _ptr(out["H_kept"]), _ptr(out["pos"]), _ptr(out["g"]),
+        _ptr(out["logg"]), oa, la, _ptr(dev_status), _stream(stream)))
+    return out

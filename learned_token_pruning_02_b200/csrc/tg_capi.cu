@@ -1,0 +1,287 @@
+// C-ABI layer of libtokengate: argument validation, per-sequence descriptors, dispatch.
+// No entry point allocates memory or synchronises the host with the device.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <vector>
+
+#include "tg_internal.cuh"
+
+namespace tg {
+
+static thread_local char g_err[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+tg_status fail(tg_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+tg_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return TG_OK;
+  return fail(TG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Per-device capability cache: 0 = unknown, 1 = supported, -1 = not supported.
+static int g_dev_ok[64];
+static int g_dev_sms[64];
+
+tg_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(TG_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  if (g_dev_ok[dev] == 0) {
+    cudaDeviceProp p;
+    e = cudaGetDeviceProperties(&p, dev);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetDeviceProperties");
+    g_dev_ok[dev] = (p.major == 10) ? 1 : -1;
+    g_dev_sms[dev] = p.multiProcessorCount;
+  }
+  if (g_dev_ok[dev] < 0)
+    return fail(TG_ERR_UNSUPPORTED, "libtokengate is built for sm_100a (B200); device %d is not", dev);
+  return TG_OK;
+}
+
+int device_sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (dev >= 0 && dev < 64 && g_dev_sms[dev] > 0) ? g_dev_sms[dev] : 148;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static size_t esize(tg_dtype dt) { return dt == TG_BF16 ? 2 : 4; }
+
+static tg_status check_seqs(const tg_seqs* s, int64_t* n_tot, int64_t* m_tot) {
+  if (!s) return fail(TG_ERR_INVALID_ARG, "seqs is NULL");
+  if (s->B < 0) return fail(TG_ERR_INVALID_ARG, "seqs->B < 0");
+  if (s->B > 0 && (!s->seqlens || !s->q_len || !s->k))
+    return fail(TG_ERR_INVALID_ARG, "seqs arrays are NULL");
+  int64_t n = 0, m = 0;
+  for (int b = 0; b < s->B; ++b) {
+    int32_t N = s->seqlens[b], q = s->q_len[b];
+    if (N < 0 || q < 0 || q > N)
+      return fail(TG_ERR_INVALID_ARG, "sequence %d: need 0 <= q_len (%d) <= seqlen (%d)", b, q, N);
+    if (N - q > TG_MAX_CTX)
+      return fail(TG_ERR_UNSUPPORTED, "sequence %d: context %d exceeds TG_MAX_CTX", b, N - q);
+    int32_t kc = s->k[b] < 0 ? 0 : (s->k[b] > N - q ? N - q : s->k[b]);
+    n += N;
+    m += kc + q;
+  }
+  if (n > INT32_MAX) return fail(TG_ERR_UNSUPPORTED, "total tokens exceed int32 indexing");
+  if (n_tot) *n_tot = n;
+  if (m_tot) *m_tot = m;
+  return TG_OK;
+}
+
+static int32_t kept_rows(const tg_seqs* s, int b) {
+  int32_t N = s->seqlens[b], q = s->q_len[b];
+  int32_t kc = s->k[b] < 0 ? 0 : (s->k[b] > N - q ? N - q : s->k[b]);
+  return kc + q;
+}
+
+}  // namespace tg
+
+using namespace tg;
+
+extern "C" {
+
+const char* tg_status_string(int32_t st) {
+  switch (st) {
+    case TG_OK: return "TG_OK";
+    case TG_ERR_INVALID_ARG: return "TG_ERR_INVALID_ARG";
+    case TG_ERR_UNSUPPORTED: return "TG_ERR_UNSUPPORTED";
+    case TG_ERR_WORKSPACE: return "TG_ERR_WORKSPACE";
+    case TG_ERR_CUDA: return "TG_ERR_CUDA";
+    case TG_ERR_DEVICE_CHECK: return "TG_ERR_DEVICE_CHECK";
+    case TG_ERR_DEVICE_TIMEOUT: return "TG_ERR_DEVICE_TIMEOUT";
+    default: return "TG_ERR_UNKNOWN";
+  }
+}
+
+const char* tg_last_error(void) { return g_err; }
+
+int32_t tg_version(void) { return (1 << 16) | 0; }
+
+tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host) {
+  g_err[0] = 0;
+  tg_status st = check_seqs(seqs, nullptr, nullptr);
+  if (st != TG_OK) return st;
+  if (!cu_kept_host) return fail(TG_ERR_INVALID_ARG, "cu_kept_host is NULL");
+  int64_t acc = 0;
+  cu_kept_host[0] = 0;
+  for (int b = 0; b < seqs->B; ++b) {
+    acc += kept_rows(seqs, b);
+    cu_kept_host[b + 1] = (int32_t)acc;
+  }
+  return TG_OK;
+}
+
+tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, int32_t d,
+                   const void* W1, const float* b1, const void* w2, float b2, int32_t dg,
+                   float* score, void* stream) {
+  g_err[0] = 0;
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
+  if (n_tok < 0 || d <= 0 || dg <= 0 || ldh < d)
+    return fail(TG_ERR_INVALID_ARG, "need n_tok >= 0, d > 0, dg > 0, ldh >= d");
+  if (n_tok > INT32_MAX) return fail(TG_ERR_UNSUPPORTED, "n_tok exceeds int32 indexing");
+  if (n_tok == 0) return TG_OK;
+  if (!H || !W1 || !w2 || !score) return fail(TG_ERR_INVALID_ARG, "H, W1, w2 and score are required");
+  if (dg != 64 && dg != 128 && dg != 256) return fail(TG_ERR_UNSUPPORTED, "dg must be 64, 128 or 256");
+  if (d % 64) return fail(TG_ERR_UNSUPPORTED, "d must be a multiple of 64");
+  if (!aligned16(H) || !aligned16(W1) || (ldh * esize(dtype)) % 16)
+    return fail(TG_ERR_UNSUPPORTED, "H and W1 must be 16-byte aligned with 16-byte row strides");
+  tg_status st = check_device();
+  if (st != TG_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  return launch_score_simt(dtype, H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, s);
+}
+
+tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
+                         int32_t* cu_kept_dev, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  int64_t n_tot = 0, m_tot = 0;
+  tg_status st = check_seqs(seqs, &n_tot, &m_tot);
+  if (st != TG_OK) return st;
+  if (seqs->B == 0) return TG_OK;
+  if ((n_tot > 0 && !score) || (m_tot > 0 && !kept_idx))
+    return fail(TG_ERR_INVALID_ARG, "score and kept_idx are required");
+  st = check_device();
+  if (st != TG_OK) return st;
+  std::vector<SelSeq> d(seqs->B);
+  int64_t start = 0, off = 0;
+  for (int b = 0; b < seqs->B; ++b) {
+    int32_t N = seqs->seqlens[b], q = seqs->q_len[b];
+    int32_t m = kept_rows(seqs, b);
+    d[b] = SelSeq{(int32_t)start, N - q, q, m - q, (int32_t)off, b};
+    start += N;
+    off += m;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int b0 = 0; b0 < seqs->B; b0 += kMaxSeqPerLaunch) {
+    int nb = seqs->B - b0 < kMaxSeqPerLaunch ? seqs->B - b0 : kMaxSeqPerLaunch;
+    int nmax = 0;
+    for (int i = 0; i < nb; ++i) nmax = d[b0 + i].n_ctx > nmax ? d[b0 + i].n_ctx : nmax;
+    st = launch_select(score, d.data() + b0, nb, nmax, kept_idx, cu_kept_dev, dev_status, s);
+    if (st != TG_OK) return st;
+  }
+  return TG_OK;
+}
+
+tg_status tg_gather(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const float* score,
+                    const int32_t* kept_idx, const tg_seqs* seqs, uint32_t flags, void* H_kept,
+                    int32_t* pos, float* g, float* logg, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
+  int64_t n_tot = 0, m_tot = 0;
+  tg_status st = check_seqs(seqs, &n_tot, &m_tot);
+  if (st != TG_OK) return st;
+  if (d <= 0 || ldh < d) return fail(TG_ERR_INVALID_ARG, "need d > 0 and ldh >= d");
+  if (m_tot == 0) return TG_OK;
+  if (!H || !kept_idx || !H_kept || !pos || ((g || logg) && !score))
+    return fail(TG_ERR_INVALID_ARG, "H, kept_idx, H_kept, pos (and score for g/logg) are required");
+  if (!aligned16(H) || !aligned16(H_kept) || (ldh * esize(dtype)) % 16 || (d * esize(dtype)) % 16)
+    return fail(TG_ERR_UNSUPPORTED, "H/H_kept must be 16-byte aligned with 16-byte rows");
+  st = check_device();
+  if (st != TG_OK) return st;
+  std::vector<GatherSeq> v(seqs->B);
+  int64_t start = 0, off = 0;
+  for (int b = 0; b < seqs->B; ++b) {
+    int32_t m = kept_rows(seqs, b);
+    v[b] = GatherSeq{(int32_t)start, seqs->seqlens[b], seqs->q_len[b], (int32_t)off, m};
+    start += seqs->seqlens[b];
+    off += m;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int b0 = 0; b0 < seqs->B; b0 += kMaxSeqPerLaunch) {
+    int nb = seqs->B - b0 < kMaxSeqPerLaunch ? seqs->B - b0 : kMaxSeqPerLaunch;
+    int m_chunk = 0;
+    for (int i = 0; i < nb; ++i) m_chunk += v[b0 + i].m;
+    if (m_chunk == 0) continue;
+    st = launch_gather(dtype, H, ldh, d, score, kept_idx, v.data() + b0, nb, m_chunk, flags, H_kept,
+                       pos, g, logg, dev_status, s);
+    if (st != TG_OK) return st;
+  }
+  return TG_OK;
+}
+
+tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const void* V,
+                            const float* logg, const float* head_gain, const int32_t* pos,
+                            const int32_t* cu_kept_host, int32_t B, int32_t Hq, int32_t Hkv,
+                            int32_t D, float softmax_scale, uint32_t flags, void* O,
+                            float* lse, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return fail(TG_ERR_INVALID_ARG, "need B >= 0 and Hq, Hkv, D > 0");
+  if (B > 0 && !cu_kept_host) return fail(TG_ERR_INVALID_ARG, "cu_kept_host is NULL");
+  if (Hq % Hkv) return fail(TG_ERR_UNSUPPORTED, "Hq must be a multiple of Hkv");
+  if (D != 64 && D != 128) return fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128");
+  if (!(softmax_scale == softmax_scale)) return fail(TG_ERR_INVALID_ARG, "softmax_scale is NaN");
+  if (B == 0) return TG_OK;
+  if (cu_kept_host[0] != 0) return fail(TG_ERR_INVALID_ARG, "cu_kept_host[0] must be 0");
+  for (int b = 0; b < B; ++b)
+    if (cu_kept_host[b + 1] < cu_kept_host[b]) return fail(TG_ERR_INVALID_ARG, "cu_kept_host not monotone");
+  int64_t m_tot = cu_kept_host[B];
+  if (m_tot == 0) return TG_OK;
+  if (!Q || !K || !V || !pos || !O) return fail(TG_ERR_INVALID_ARG, "Q, K, V, pos and O are required");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(TG_ERR_UNSUPPORTED, "Q, K, V and O must be 16-byte aligned");
+  tg_status st = check_device();
+  if (st != TG_OK) return st;
+  AttnArgs a{dtype, Q, K, V, logg, head_gain, pos, Hq, Hkv, D, softmax_scale, flags, O, lse, dev_status, m_tot};
+  std::vector<AttnSeq> v(B);
+  for (int b = 0; b < B; ++b) v[b] = AttnSeq{cu_kept_host[b], cu_kept_host[b + 1] - cu_kept_host[b]};
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int b0 = 0; b0 < B; b0 += kMaxSeqPerLaunch) {
+    int nb = B - b0 < kMaxSeqPerLaunch ? B - b0 : kMaxSeqPerLaunch;
+    st = launch_attn_simt(a, v.data() + b0, nb, s);
+    if (st != TG_OK) return st;
+  }
+  return TG_OK;
+}
+
+tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t d,
+                             const void* W1, const float* b1, const void* w2, float b2,
+                             int32_t dg, const tg_seqs* seqs, int32_t n_layers,
+                             const void* const* Q, const void* const* K, const void* const* V,
+                             int32_t Hq, int32_t Hkv, int32_t D, float softmax_scale,
+                             const float* head_gain, uint32_t flags, float* score,
+                             int32_t* kept_idx, int32_t* cu_kept_dev, void* H_kept, int32_t* pos,
+                             float* g, float* logg, void* const* O, float* const* lse,
+                             int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  int64_t n_tot = 0, m_tot = 0;
+  tg_status st = check_seqs(seqs, &n_tot, &m_tot);
+  if (st != TG_OK) return st;
+  if (n_layers < 0) return fail(TG_ERR_INVALID_ARG, "n_layers < 0");
+  if (n_layers > 0 && (!Q || !K || !V || !O)) return fail(TG_ERR_INVALID_ARG, "Q/K/V/O arrays are required");
+  if (m_tot > 0 && (!score || !kept_idx || !H_kept || !pos || !g || !logg))
+    return fail(TG_ERR_INVALID_ARG, "score, kept_idx, H_kept, pos, g and logg are required");
+  std::vector<int32_t> cu(seqs->B + 1);
+  st = tg_kept_counts(seqs, cu.data());
+  if (st != TG_OK) return st;
+  st = tg_score(dtype, H, ldh, n_tot, d, W1, b1, w2, b2, dg, score, stream);
+  if (st != TG_OK) return st;
+  st = tg_topk_select(score, seqs, kept_idx, cu_kept_dev, dev_status, stream);
+  if (st != TG_OK) return st;
+  st = tg_gather(dtype, H, ldh, d, score, kept_idx, seqs, flags, H_kept, pos, g, logg, dev_status, stream);
+  if (st != TG_OK) return st;
+  for (int l = 0; l < n_layers; ++l) {
+    st = tg_gated_attn_fwd(dtype, Q[l], K[l], V[l], logg, head_gain, pos, cu.data(), seqs->B, Hq, Hkv, D,
+                           softmax_scale, flags, O[l], lse ? lse[l] : nullptr, dev_status, stream);
+    if (st != TG_OK) return st;
+  }
+  return TG_OK;
+}
+
+}  // extern "C"

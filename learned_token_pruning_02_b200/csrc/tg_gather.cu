@@ -1,0 +1,96 @@
+// Forward the kept hidden states, their original positions and gate values.
+//
+// TokenGate paper page (thelatestinai.com), Figure 1(b): the top-K selector forwards the
+// kept hidden states together with their importance scores; aitualizate.com article,
+// phase 3: layers above L receive only the kept tokens.
+//
+// Design (B200): a pure HBM copy. One warp moves one kept row with 16-byte vector loads
+// and stores (a 2048-wide bf16 row is 4 KB = 8 x 16 B per lane), all loads of a row issued
+// before its stores so each warp keeps 4 KB in flight. Lane 0 also writes pos = row index
+// within its sequence, g = sigmoid(score) and log g (stable log-sigmoid). Grid-stride over
+// rows with a grid of a few waves of the SM count.
+#include "tg_internal.cuh"
+
+namespace tg {
+namespace {
+
+struct GatherParams {
+  GatherSeq s[kMaxSeqPerLaunch];
+  int nseq;
+};
+
+constexpr int WARPS = 8;
+constexpr int MAXV = 8;  // 16-byte vectors per lane held in registers per pass
+
+__global__ void __launch_bounds__(WARPS * 32)
+    gather_kernel(const uint4* __restrict__ H, int64_t ldv, int nvec, const float* __restrict__ score,
+                  const int32_t* __restrict__ kept, uint32_t flags, uint4* __restrict__ Hk, int32_t* __restrict__ pos,
+                  float* __restrict__ g, float* __restrict__ logg, int32_t* __restrict__ dev_status, int m_chunk,
+                  const __grid_constant__ GatherParams p) {
+  const int lane = threadIdx.x & 31;
+  const int row0 = p.s[0].out_off;
+  for (int r = blockIdx.x * WARPS + (threadIdx.x >> 5); r < m_chunk; r += gridDim.x * WARPS) {
+    const int row = row0 + r;
+    int b = 0;
+    while (b + 1 < p.nseq && row >= p.s[b + 1].out_off) ++b;
+    const GatherSeq sq = p.s[b];
+    const int32_t j = __ldg(kept + row);
+    if (j < sq.start || j >= sq.start + sq.n) {
+      if (lane == 0 && dev_status) atomicOr(dev_status, TG_DEV_BAD_INDEX);
+      continue;
+    }
+    const uint4* src = H + (int64_t)j * ldv;
+    uint4* dst = Hk + (int64_t)row * nvec;
+    for (int v0 = 0; v0 < nvec; v0 += 32 * MAXV) {
+      uint4 buf[MAXV];
+#pragma unroll
+      for (int u = 0; u < MAXV; ++u) {
+        int v = v0 + u * 32 + lane;
+        if (v < nvec) buf[u] = __ldcs(src + v);
+      }
+#pragma unroll
+      for (int u = 0; u < MAXV; ++u) {
+        int v = v0 + u * 32 + lane;
+        if (v < nvec) __stcs(dst + v, buf[u]);
+      }
+    }
+    if (lane == 0) {
+      pos[row] = j - sq.start;
+      if (g || logg) {
+        const float s = __ldg(score + j);
+        float gv, lg;
+        if ((flags & TG_QUESTION_GATE_ONE) && (row - sq.out_off) >= sq.m - sq.q) {
+          gv = 1.f;
+          lg = 0.f;
+        } else {
+          const float e = expf(-fabsf(s));
+          gv = s >= 0.f ? 1.f / (1.f + e) : e / (1.f + e);
+          lg = s >= 0.f ? -log1pf(e) : s - log1pf(e);
+        }
+        if (g) g[row] = gv;
+        if (logg) logg[row] = lg;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const float* score, const int32_t* kept_idx,
+                        const GatherSeq* seqs, int nseq, int m_chunk, uint32_t flags, void* H_kept, int32_t* pos,
+                        float* g, float* logg, int32_t* dev_status, cudaStream_t st) {
+  GatherParams p = {};
+  for (int i = 0; i < nseq; ++i) p.s[i] = seqs[i];
+  p.nseq = nseq;
+  const int es = dt == TG_BF16 ? 2 : 4;
+  const int nvec = d * es / 16;
+  const int64_t ldv = ldh * es / 16;
+  int blocks = (m_chunk + WARPS - 1) / WARPS;
+  const int cap = device_sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  gather_kernel<<<blocks, WARPS * 32, 0, st>>>(static_cast<const uint4*>(H), ldv, nvec, score, kept_idx, flags,
+                                               static_cast<uint4*>(H_kept), pos, g, logg, dev_status, m_chunk, p);
+  return cuda_status(cudaGetLastError(), "gather launch");
+}
+
+}  // namespace tg

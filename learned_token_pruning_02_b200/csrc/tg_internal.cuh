@@ -1,0 +1,86 @@
+// Internal declarations shared by the CUDA translation units of libtokengate.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tokengate.h"
+
+namespace tg {
+
+constexpr int kMaxSeqPerLaunch = 64;  // per-sequence descriptors travel as kernel params
+
+// ----------------------------------------------------------------------------- error text
+void set_error(const char* fmt, ...);
+tg_status fail(tg_status st, const char* fmt, ...);
+tg_status cuda_status(cudaError_t e, const char* what);
+
+// Checks that the current device is a B200-class part (compute capability 10.x) once per
+// device; returns TG_ERR_UNSUPPORTED otherwise.
+tg_status check_device();
+int device_sm_count();
+
+// ----------------------------------------------------------------------------- launchers
+// Each returns TG_OK or TG_ERR_CUDA (argument checks happen in the C-ABI layer).
+
+tg_status launch_score_simt(tg_dtype dt, const void* H, int64_t ldh, int64_t n_tok, int d,
+                            const void* W1, const float* b1, const void* w2, float b2, int dg,
+                            float* score, cudaStream_t st);
+
+tg_status launch_score_tc(const void* H, int64_t ldh, int64_t n_tok, int d, const void* W1,
+                          const float* b1, const void* w2, float b2, int dg, float* score,
+                          cudaStream_t st);
+
+struct SelSeq {
+  int32_t start;    // packed row of the sequence's first token
+  int32_t n_ctx;    // context tokens N - q
+  int32_t q;        // question-tail tokens
+  int32_t kc;       // context tokens to keep, min(max(k,0), n_ctx)
+  int32_t out_off;  // first output row (cu_kept[b])
+  int32_t b;        // sequence index in the whole batch
+};
+
+tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_ctx_max,
+                        int32_t* kept_idx, int32_t* cu_kept_dev, int32_t* dev_status,
+                        cudaStream_t st);
+
+struct GatherSeq {
+  int32_t start;    // packed row of the sequence's first token
+  int32_t n;        // tokens N
+  int32_t q;        // question-tail tokens
+  int32_t out_off;  // cu_kept[b]
+  int32_t m;        // kept rows M_b
+};
+
+tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const float* score,
+                        const int32_t* kept_idx, const GatherSeq* seqs, int nseq, int m_chunk,
+                        uint32_t flags, void* H_kept, int32_t* pos, float* g, float* logg,
+                        int32_t* dev_status, cudaStream_t st);
+
+struct AttnSeq {
+  int32_t off;  // cu_kept[b]
+  int32_t m;    // kept rows M_b
+};
+
+struct AttnArgs {
+  tg_dtype dt;
+  const void* Q;
+  const void* K;
+  const void* V;
+  const float* logg;
+  const float* head_gain;
+  const int32_t* pos;
+  int Hq, Hkv, D;
+  float scale;
+  uint32_t flags;
+  void* O;
+  float* lse;
+  int32_t* dev_status;
+  int64_t m_tot;
+};
+
+tg_status launch_attn_simt(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);
+tg_status launch_attn_tc(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);
+
+}  // namespace tg

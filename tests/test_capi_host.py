@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared symbol, and
+rejects bad arguments synchronously (before any CUDA call). No GPU needed."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import learned_token_pruning_02_b200 as tg
+from oracle import tg_oracle as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(tg_[a-zA-Z0-9_]+)\s*\(", txt, re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(tg.LIB_PATH):
+        from learned_token_pruning_02_b200 import build
+        build.build()
+    return tg.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared_functions()
+    assert len(declared) >= 9, declared
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(tg.EXPORTS) == set(declared)
+
+
+def test_status_strings_and_version(L):
+    assert L.tg_status_string(0) == b"TG_OK"
+    assert L.tg_status_string(1) == b"TG_ERR_INVALID_ARG"
+    assert L.tg_status_string(4) == b"TG_ERR_CUDA"
+    assert L.tg_status_string(99) == b"TG_ERR_UNKNOWN"
+    assert L.tg_version() >> 16 == 1
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_kept_counts_match_oracle_rule(L, seed):
+    g = np.random.default_rng(seed)
+    B = int(g.integers(1, 9))
+    seqlens = g.integers(0, 5000, B)
+    q_len = np.array([g.integers(0, n + 1) for n in seqlens])
+    k = g.integers(-5, 6000, B)
+    cu = tg.tg_kept_counts(seqlens, q_len, k)
+    expect = np.concatenate([[0], np.cumsum([orc.kept_count(n, q, kk) for n, q, kk in zip(seqlens, q_len, k)])])
+    assert cu == expect.tolist()
+
+
+def test_kept_counts_rejects_bad_sequences(L):
+    with pytest.raises(tg.TokenGateError) as e:
+        tg.tg_kept_counts([10], [11], [3])
+    assert e.value.status == 1
+    with pytest.raises(tg.TokenGateError) as e:
+        tg.tg_kept_counts([-1], [0], [3])
+    assert e.value.status == 1
+    with pytest.raises(tg.TokenGateError) as e:
+        tg.tg_kept_counts([tg.TG_MAX_CTX + 10], [0], [3])
+    assert e.value.status == 2
+
+
+def _seqs(seqlens, q, k):
+    return tg.Seqs(seqlens, q, k)
+
+
+def test_argument_errors_are_synchronous(L):
+    V = ctypes.c_void_p
+    fake = V(0x1000)  # never dereferenced: every call below fails validation first
+    # tg_score: null H, bad dg, bad d, misaligned pointer
+    assert L.tg_score(1, None, 64, 10, 64, fake, None, fake, 0.0, 64, fake, None) == 1
+    assert L.tg_score(1, fake, 64, 10, 64, fake, None, fake, 0.0, 96, fake, None) == 2
+    assert L.tg_score(1, fake, 96, 10, 96, fake, None, fake, 0.0, 64, fake, None) == 2
+    assert L.tg_score(1, V(0x1002), 64, 10, 64, fake, None, fake, 0.0, 64, fake, None) == 2
+    assert L.tg_score(7, fake, 64, 10, 64, fake, None, fake, 0.0, 64, fake, None) == 1
+    assert L.tg_score(1, fake, 32, 10, 64, fake, None, fake, 0.0, 64, fake, None) == 1  # ldh < d
+    assert b"dg" in L.tg_last_error() or b"ldh" in L.tg_last_error()
+    # n_tok == 0 is a no-op that needs no device
+    assert L.tg_score(1, None, 64, 0, 64, None, None, None, 0.0, 64, None, None) == 0
+    # tg_topk_select: q > N, null outputs
+    s = _seqs([10], [11], [2])
+    assert L.tg_topk_select(fake, s.ref(), fake, None, None, None) == 1
+    s = _seqs([10], [2], [2])
+    assert L.tg_topk_select(None, s.ref(), fake, None, None, None) == 1
+    assert L.tg_topk_select(fake, None, fake, None, None, None) == 1
+    s0 = _seqs([], [], [])
+    assert L.tg_topk_select(None, s0.ref(), None, None, None, None) == 0
+    # tg_gather: misaligned row pitch, null outputs
+    s = _seqs([10], [2], [2])
+    assert L.tg_gather(1, fake, 65, 64, fake, fake, s.ref(), 0, fake, fake, None, None, None, None) == 2
+    assert L.tg_gather(1, fake, 64, 64, fake, fake, s.ref(), 0, None, fake, None, None, None, None) == 1
+    assert L.tg_gather(1, fake, 64, 64, None, fake, s.ref(), 0, fake, fake, fake, None, None, None) == 1
+    # tg_gated_attn_fwd: Hq % Hkv, D, null cu_kept, non-monotone offsets
+    cu = (ctypes.c_int32 * 2)(0, 8)
+    assert L.tg_gated_attn_fwd(1, fake, fake, fake, None, None, fake, cu, 1, 6, 4, 128, 0.1, 0, fake, None, None,
+                               None) == 2
+    assert L.tg_gated_attn_fwd(1, fake, fake, fake, None, None, fake, cu, 1, 8, 4, 96, 0.1, 0, fake, None, None,
+                               None) == 2
+    assert L.tg_gated_attn_fwd(1, fake, fake, fake, None, None, fake, None, 1, 8, 4, 128, 0.1, 0, fake, None, None,
+                               None) == 1
+    bad = (ctypes.c_int32 * 3)(0, 8, 4)
+    assert L.tg_gated_attn_fwd(1, fake, fake, fake, None, None, fake, bad, 2, 8, 4, 128, 0.1, 0, fake, None, None,
+                               None) == 1
+    assert L.tg_gated_attn_fwd(1, None, fake, fake, None, None, fake, cu, 1, 8, 4, 128, 0.1, 0, fake, None, None,
+                               None) == 1
+    assert L.tg_gated_attn_fwd(1, fake, fake, fake, None, None, fake, cu, 1, 8, 4, 128, float("nan"), 0, fake, None,
+                               None, None) == 1
+    # tg_prefill_above_L: missing outputs
+    s = _seqs([10], [2], [2])
+    arr = (V * 1)(fake.value)
+    assert L.tg_prefill_above_L(1, fake, 64, 64, fake, None, fake, 0.0, 64, s.ref(), 1, arr, arr, arr, 8, 4, 128,
+                                0.1, None, 0, None, fake, None, fake, fake, fake, fake, arr, None, None, None) == 1
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    H = torch.zeros(4, 64)
+    with pytest.raises(ValueError):
+        tg.tg_score(H, torch.zeros(64, 64), None, torch.zeros(64), 0.0)

@@ -1,0 +1,359 @@
+"""GPU parity of every step of the gated-prefill path against the CPU oracle.
+
+Bar: selected indices, gathered rows and positions bit-exact (select is compared with the
+oracle's top-K run on the GPU's own scores); scores, gate values and attention within the
+max-abs-relative tolerance 1e-4 (float32) / 2e-2 (bf16). Inputs are the seeded synthetic
+tensors of tg_inputs; every call goes through the C ABI (the ctypes binding)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import learned_token_pruning_02_b200 as tg
+import tg_inputs as ti
+from oracle import tg_oracle as orc
+from tg_testutil import TOL, bits, from_dev, max_abs_rel, to_dev
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU hosts too; every test here is gpu-marked
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+DEV = "cuda"
+
+
+def _stat():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+# ============================================================================ score
+
+
+def _score_case(wl, biased=False, rows=None, ldh_pad=0):
+    H = ti.hidden_states(wl)
+    W1, b1, w2, b2 = ti.gate_weights(wl, biased=biased)
+    Hd = to_dev(H, wl.dtype)
+    if ldh_pad:
+        big = torch.zeros(Hd.shape[0], Hd.shape[1] + ldh_pad, dtype=Hd.dtype, device=DEV)
+        big[:, : Hd.shape[1]] = Hd
+        Hd = big[:, : Hd.shape[1]]
+    s = tg.tg_score(Hd, to_dev(W1, wl.dtype), to_dev(b1, "f32"), to_dev(w2, wl.dtype), b2)
+    torch.cuda.synchronize()
+    s = from_dev(s)
+    H64, W64, w64 = ti.widen(H, wl.dtype), ti.widen(W1, wl.dtype), ti.widen(w2, wl.dtype)
+    if rows is None:
+        ref = orc.gate_scores(H64, W64, b1, w64, b2)
+        return s, ref
+    ref = orc.gate_scores(H64[rows], W64, b1, w64, b2)
+    return s[rows], ref
+
+
+@pytest.mark.parametrize("biased", [False, True])
+def test_score_tiny_f32(biased):
+    s, ref = _score_case(ti.WORKLOADS["tiny_f32"], biased)
+    assert max_abs_rel(s, ref) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("dg,d,n", [(256, 2048, 1000), (128, 512, 300), (64, 256, 129), (256, 1024, 1)])
+def test_score_bf16_small(dg, d, n):
+    wl = ti.scaled(ti.WORKLOADS["qwen3_8k"], seqlens=(n,), q_len=(0,), k=(0,), d=d, dg=dg)
+    s, ref = _score_case(wl, biased=True)
+    assert max_abs_rel(s, ref) <= TOL["bf16"]
+    assert max_abs_rel(s, ref) <= 1e-3  # bf16 inputs are exact; only fp32 accumulation differs
+
+
+def test_score_bf16_strided_rows():
+    wl = ti.scaled(ti.WORKLOADS["qwen3_8k"], seqlens=(777,), q_len=(0,), k=(0,), d=512)
+    s, ref = _score_case(wl, ldh_pad=64)
+    assert max_abs_rel(s, ref) <= TOL["bf16"]
+
+
+def test_score_bf16_full_32k_sampled():
+    wl = ti.WORKLOADS["qwen3_32k"]
+    g = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 127, 128, wl.n_tok - 1], g.integers(0, wl.n_tok, 500)]))
+    s, ref = _score_case(wl, rows=rows)
+    assert max_abs_rel(s, ref) <= TOL["bf16"]
+
+
+# ============================================================================ select
+
+
+def _select_check(s, seqlens, q_len, k):
+    sd = torch.from_numpy(np.ascontiguousarray(s, dtype=np.float32)).to(DEV)
+    st = _stat()
+    kept, cu = tg.tg_topk_select(sd, seqlens, q_len, k, dev_status=st)
+    torch.cuda.synchronize()
+    ref, ref_cu = orc.topk_select(s, seqlens, q_len, k)
+    assert cu.cpu().numpy().tolist() == ref_cu.tolist()
+    got = kept.cpu().numpy()
+    assert np.array_equal(got, ref.astype(np.int32))
+    return int(st.item())
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "qwen3_8k", "qwen3_32k", "qwen3_128k", "ragged4"])
+def test_select_stage_scores_bitexact(name):
+    wl = ti.WORKLOADS[name]
+    st = _select_check(ti.stage_scores(wl), wl.seqlens, wl.q_len, wl.k)
+    assert st == 0
+
+
+def test_select_on_gpu_mlp_scores_bitexact():
+    wl = ti.WORKLOADS["qwen3_8k"]
+    H = ti.hidden_states(wl)
+    W1, b1, w2, b2 = ti.gate_weights(wl)
+    s = tg.tg_score(to_dev(H, "bf16"), to_dev(W1, "bf16"), to_dev(b1, "f32"), to_dev(w2, "bf16"), b2)
+    torch.cuda.synchronize()
+    _select_check(s.cpu().numpy(), wl.seqlens, wl.q_len, wl.k)
+
+
+@pytest.mark.parametrize("case", [
+    ((1000,), (10,), (0,)),           # K = 0: only the question tail
+    ((1000,), (10,), (990,)),         # K = N - q: everything
+    ((1000,), (10,), (5000,)),        # K > N - q
+    ((1000,), (0,), (17,)),           # no question
+    ((64,), (64,), (8,)),             # question only
+    ((0, 5, 0), (0, 2, 0), (3, 1, 3)),  # empty sequences
+    ((1,), (0,), (1,)),
+    ((4097,), (1,), (4095,)),         # K = n_ctx - 1
+    ((262144,), (0,), (1000,)),  # the largest context: an 8-CTA cluster
+])
+def test_select_edge_cases(case):
+    seqlens, q_len, k = case
+    g = np.random.default_rng(sum(seqlens))
+    s = g.standard_normal(sum(seqlens)).astype(np.float32)
+    _select_check(s, seqlens, q_len, k)
+
+
+def test_select_ties_nan_negzero():
+    g = np.random.default_rng(1)
+    n = 50000
+    s = g.integers(-2, 3, n).astype(np.float32)  # 5 distinct values: huge tie groups
+    s[g.random(n) < 0.01] = np.nan
+    s[g.random(n) < 0.05] = -0.0
+    s[g.random(n) < 0.01] = -np.inf
+    for k in (1, 777, 20000, 49000):
+        st = _select_check(s, (n,), (100,), (k,))
+        assert st & tg.TG_DEV_NAN_SCORE
+    assert _select_check(np.zeros(3000, np.float32), (3000,), (0,), (1234,)) == 0  # all equal
+
+
+def test_select_many_sequences_chunks_launches():
+    g = np.random.default_rng(2)
+    B = 150  # more than the 64 descriptors one launch carries
+    seqlens = tuple(int(x) for x in g.integers(0, 3000, B))
+    q_len = tuple(int(g.integers(0, n + 1)) for n in seqlens)
+    k = tuple(int(x) for x in g.integers(0, 1500, B))
+    s = np.round(g.standard_normal(sum(seqlens)) * 8).astype(np.float32)
+    _select_check(s, seqlens, q_len, k)
+
+
+def test_select_batched_long_sequences():
+    g = np.random.default_rng(3)
+    seqlens = (131072,) * 6 + (70000,)
+    q_len = (256,) * 6 + (0,)
+    k = (4096, 1, 65536, 130000, 4096, 0, 69999)
+    s = ti.bf16_bits_to_f32(ti.f32_to_bf16_bits(g.standard_normal(sum(seqlens)).astype(np.float32)))
+    _select_check(s, seqlens, q_len, k)
+
+
+# ============================================================================ gather
+
+
+@pytest.mark.parametrize("name,flags", [("tiny_f32", 0), ("qwen3_32k", 0), ("ragged4", tg.TG_QUESTION_GATE_ONE)])
+def test_gather_bitexact(name, flags):
+    wl = ti.WORKLOADS[name]
+    H = ti.hidden_states(wl)
+    s = ti.stage_scores(wl)
+    kept, cu = orc.topk_select(s, wl.seqlens, wl.q_len, wl.k)
+    Hd = to_dev(H, wl.dtype)
+    sd = torch.from_numpy(s).to(DEV)
+    kd = torch.from_numpy(kept.astype(np.int32)).to(DEV)
+    st = _stat()
+    Hk, pos, g, lg = tg.tg_gather(Hd, sd, kd, wl.seqlens, wl.q_len, wl.k, flags=flags, dev_status=st)
+    torch.cuda.synchronize()
+    rHk, rpos, rg, rlg = orc.gather(H, s, kept, wl.seqlens, wl.q_len, cu, bool(flags & tg.TG_QUESTION_GATE_ONE))
+    assert np.array_equal(bits(Hk), np.ascontiguousarray(rHk).view(np.int16 if wl.dtype == "bf16" else np.int32))
+    assert np.array_equal(pos.cpu().numpy(), rpos.astype(np.int32))
+    assert max_abs_rel(from_dev(g), rg) <= 1e-6
+    np.testing.assert_allclose(from_dev(lg), rlg, rtol=2e-6, atol=2e-7)
+    assert st.item() == 0
+
+
+def test_gather_strided_and_bad_index_flag():
+    wl = ti.scaled(ti.WORKLOADS["qwen3_8k"], seqlens=(300, 200), q_len=(10, 20), k=(50, 40), d=512)
+    H = ti.hidden_states(wl)
+    s = ti.stage_scores(wl)
+    kept, cu = orc.topk_select(s, wl.seqlens, wl.q_len, wl.k)
+    base = torch.zeros(wl.n_tok, 640, dtype=torch.bfloat16, device=DEV)
+    base[:, :512] = to_dev(H, "bf16")
+    Hd = base[:, :512]
+    kd = torch.from_numpy(kept.astype(np.int32)).to(DEV)
+    Hk, pos, _, _ = tg.tg_gather(Hd, torch.from_numpy(s).to(DEV), kd, wl.seqlens, wl.q_len, wl.k)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(Hk), H[kept].view(np.int16))
+    bad = kd.clone()
+    bad[3] = 299 + 5  # row of the second sequence written into the first sequence's slot
+    st = _stat()
+    tg.tg_gather(Hd, torch.from_numpy(s).to(DEV), bad, wl.seqlens, wl.q_len, wl.k, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() & tg.TG_DEV_BAD_INDEX
+
+
+# ============================================================================ attention
+
+
+def _attn_case(wl, layer=0, rows=None, flags=0, gain=None, logg_none=False, m_rows=None):
+    m = wl.m_tot if m_rows is None else m_rows
+    cu = np.concatenate([[0], np.cumsum(wl.kept_rows())])
+    Q, K, V = ti.qkv(wl, layer, m)
+    lg = None if logg_none else ti.random_logg(wl, m, layer)
+    pos = np.concatenate([np.sort(np.random.default_rng(b).choice(n, size=int(cu[b + 1] - cu[b]), replace=False))
+                          for b, n in enumerate(wl.seqlens)]).astype(np.int32)
+    scale = 1.0 / math.sqrt(wl.D)
+    st = _stat()
+    O, lse = tg.tg_gated_attn_fwd(to_dev(Q, wl.dtype), to_dev(K, wl.dtype), to_dev(V, wl.dtype),
+                                  None if lg is None else torch.from_numpy(lg).to(DEV),
+                                  torch.from_numpy(pos).to(DEV), cu.tolist(), scale,
+                                  head_gain=None if gain is None else torch.tensor(gain, device=DEV),
+                                  flags=flags, dev_status=st)
+    torch.cuda.synchronize()
+    rO, rL = orc.gated_attention(ti.widen(Q, wl.dtype), ti.widen(K, wl.dtype), ti.widen(V, wl.dtype), lg, pos, cu,
+                                 wl.Hq, wl.Hkv, scale, gain, bool(flags & tg.TG_ATTN_UNNORMALISED), rows)
+    O, lse = from_dev(O), from_dev(lse)
+    if rows is not None:
+        O, lse = O[rows], lse[:, rows]
+    assert st.item() == 0
+    return O, lse, rO, rL
+
+
+@pytest.mark.parametrize("flags,gain", [(0, None), (tg.TG_ATTN_UNNORMALISED, None), (0, [1.0, 0.5, 2.0, -0.5])])
+def test_attention_tiny_f32(flags, gain):
+    wl = ti.WORKLOADS["tiny_f32"]
+    O, L, rO, rL = _attn_case(wl, flags=flags, gain=gain)
+    assert max_abs_rel(O, rO) <= TOL["f32"]
+    assert max_abs_rel(L, rL) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("name", ["qwen3_8k", "ragged4"])
+def test_attention_bf16_full(name):
+    wl = ti.WORKLOADS[name]
+    O, L, rO, rL = _attn_case(wl)
+    assert max_abs_rel(O, rO) <= TOL["bf16"]
+    assert max_abs_rel(L, rL) <= TOL["bf16"]
+
+
+def test_attention_bf16_32k_full():
+    wl = ti.WORKLOADS["qwen3_32k"]
+    O, L, rO, rL = _attn_case(wl)
+    assert max_abs_rel(O, rO) <= TOL["bf16"]
+    assert max_abs_rel(L, rL) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("layer", [0, 3])
+def test_attention_bf16_128k_sampled(layer):
+    wl = ti.WORKLOADS["qwen3_128k"]
+    g = np.random.default_rng(layer)
+    m = wl.m_tot
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, m - 1], g.integers(0, m, 256)]))
+    O, L, rO, rL = _attn_case(wl, layer=layer, rows=rows)
+    assert max_abs_rel(O, rO) <= TOL["bf16"]
+    assert max_abs_rel(L, rL) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("flags,gain", [(tg.TG_ATTN_UNNORMALISED, None), (0, [0.5] * 8 + [2.0] * 8)])
+def test_attention_bf16_flags(flags, gain):
+    wl = ti.scaled(ti.WORKLOADS["qwen3_8k"], seqlens=(2000, 700), q_len=(64, 30), k=(300, 500))
+    O, L, rO, rL = _attn_case(wl, flags=flags, gain=gain)
+    assert max_abs_rel(O, rO) <= TOL["bf16"]
+    assert max_abs_rel(L, rL) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(8, 8, 64), (16, 4, 128), (4, 2, 64)])
+def test_attention_bf16_head_layouts(Hq, Hkv, D):
+    wl = ti.scaled(ti.WORKLOADS["qwen3_8k"], seqlens=(1000, 301), q_len=(40, 1), k=(400, 129), Hq=Hq, Hkv=Hkv, D=D)
+    O, L, rO, rL = _attn_case(wl)
+    assert max_abs_rel(O, rO) <= TOL["bf16"]
+
+
+def test_attention_g1_all_kept_matches_torch_sdpa():
+    # g == 1 with every token kept is ordinary causal attention: a third opinion from torch
+    wl = ti.scaled(ti.WORKLOADS["qwen3_8k"], seqlens=(1000,), q_len=(0,), k=(1000,))
+    m = 1000
+    Q, K, V = ti.qkv(wl, 0, m)
+    q, k, v = (to_dev(x, "bf16") for x in (Q, K, V))
+    pos = torch.arange(m, dtype=torch.int32, device=DEV)
+    O, _ = tg.tg_gated_attn_fwd(q, k, v, None, pos, [0, m], 1 / math.sqrt(128))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.permute(1, 0, 2).float(), k.permute(1, 0, 2).float().repeat_interleave(2, 0),
+        v.permute(1, 0, 2).float().repeat_interleave(2, 0), is_causal=True, scale=1 / math.sqrt(128))
+    torch.cuda.synchronize()
+    assert max_abs_rel(from_dev(O), from_dev(ref.permute(1, 0, 2))) <= TOL["bf16"]
+
+
+def test_attention_non_ascending_positions_flagged():
+    wl = ti.scaled(ti.WORKLOADS["qwen3_8k"], seqlens=(300,), q_len=(0,), k=(300,))
+    Q, K, V = ti.qkv(wl, 0, 300)
+    pos = torch.arange(300, dtype=torch.int32, device=DEV)
+    pos[100] = 5
+    st = _stat()
+    tg.tg_gated_attn_fwd(to_dev(Q, "bf16"), to_dev(K, "bf16"), to_dev(V, "bf16"), None, pos, [0, 300], 0.1,
+                         dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() & tg.TG_DEV_POS_NOT_ASCENDING
+
+
+# ============================================================================ chain
+
+
+def _chain(wl, flags=0, layers_np=None):
+    H = ti.hidden_states(wl)
+    W1, b1, w2, b2 = ti.gate_weights(wl, biased=True)
+    scale = 1.0 / math.sqrt(wl.D)
+    ref = orc.prefill_above_L(H, ti.widen(W1, wl.dtype), b1, ti.widen(w2, wl.dtype), b2, wl.seqlens, wl.q_len,
+                              wl.k, [], wl.Hq, wl.Hkv, scale)
+    if layers_np is None:
+        if wl.dtype == "f32":
+            layers_np = [ti.project_kept(wl, ti.widen(ref["H_kept"], "f32"))]
+        else:
+            layers_np = [ti.qkv(wl, l) for l in range(wl.n_layers)]
+    layers = [tuple(to_dev(x, wl.dtype) for x in lyr) for lyr in layers_np]
+    st = _stat()
+    out = tg.tg_prefill_above_L(to_dev(H, wl.dtype), to_dev(W1, wl.dtype), to_dev(b1, "f32"), to_dev(w2, wl.dtype),
+                                b2, wl.seqlens, wl.q_len, wl.k, layers, scale, flags=flags, want_lse=True,
+                                dev_status=st)
+    torch.cuda.synchronize()
+    return H, ref, layers_np, out, st
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "qwen3_8k"])
+def test_chain_end_to_end(name):
+    wl = ti.WORKLOADS[name]
+    H, ref, layers_np, out, st = _chain(wl)
+    tol = TOL[wl.dtype]
+    s_gpu = out["score"].cpu().numpy()
+    assert max_abs_rel(s_gpu, ref["score"]) <= tol
+    # selection: bit-exact against the oracle's top-K run on the GPU's own scores
+    kept_o, cu_o = orc.topk_select(s_gpu, wl.seqlens, wl.q_len, wl.k)
+    assert np.array_equal(out["kept_idx"].cpu().numpy(), kept_o.astype(np.int32))
+    assert out["cu_kept_dev"].cpu().numpy().tolist() == cu_o.tolist()
+    Hk, pos, g, lg = orc.gather(H, s_gpu, kept_o, wl.seqlens, wl.q_len, cu_o)
+    assert np.array_equal(bits(out["H_kept"]), np.ascontiguousarray(Hk).view(np.int16 if wl.dtype == "bf16" else np.int32))
+    assert np.array_equal(out["pos"].cpu().numpy(), pos.astype(np.int32))
+    assert max_abs_rel(from_dev(out["g"]), g) <= 1e-6
+    for (Q, K, V), O, L in zip(layers_np, out["O"], out["lse"]):
+        rO, rL = orc.gated_attention(ti.widen(Q, wl.dtype), ti.widen(K, wl.dtype), ti.widen(V, wl.dtype), lg, pos,
+                                     cu_o, wl.Hq, wl.Hkv, 1.0 / math.sqrt(wl.D))
+        assert max_abs_rel(from_dev(O), rO) <= tol
+        assert max_abs_rel(from_dev(L), rL) <= tol
+    assert st.item() == 0
+
+
+def test_chain_deterministic():
+    wl = ti.WORKLOADS["ragged4"]
+    _, _, layers_np, out1, _ = _chain(wl)
+    _, _, _, out2, _ = _chain(wl, layers_np=layers_np)
+    for key in ("score", "kept_idx", "H_kept", "pos", "g", "logg"):
+        assert np.array_equal(bits(out1[key]), bits(out2[key])), key
+    assert np.array_equal(bits(out1["O"][0]), bits(out2["O"][0]))
