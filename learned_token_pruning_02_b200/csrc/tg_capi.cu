@@ -144,6 +144,7 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
   tg_status st = check_device();
   if (st != TG_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == TG_BF16) return launch_score_tc(H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, s);
   return launch_score_simt(dtype, H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, s);
 }
 
@@ -244,7 +245,7 @@ tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const 
   cudaStream_t s = (cudaStream_t)stream;
   for (int b0 = 0; b0 < B; b0 += kMaxSeqPerLaunch) {
     int nb = B - b0 < kMaxSeqPerLaunch ? B - b0 : kMaxSeqPerLaunch;
-    st = launch_attn_simt(a, v.data() + b0, nb, s);
+    st = (dtype == TG_BF16) ? launch_attn_tc(a, v.data() + b0, nb, s) : launch_attn_simt(a, v.data() + b0, nb, s);
     if (st != TG_OK) return st;
   }
   return TG_OK;

@@ -311,8 +311,8 @@ def _chain(wl, flags=0, layers_np=None):
     H = ti.hidden_states(wl)
     W1, b1, w2, b2 = ti.gate_weights(wl, biased=True)
     scale = 1.0 / math.sqrt(wl.D)
-    ref = orc.prefill_above_L(H, ti.widen(W1, wl.dtype), b1, ti.widen(w2, wl.dtype), b2, wl.seqlens, wl.q_len,
-                              wl.k, [], wl.Hq, wl.Hkv, scale)
+    ref = orc.prefill_above_L(ti.widen(H, wl.dtype), ti.widen(W1, wl.dtype), b1, ti.widen(w2, wl.dtype), b2,
+                              wl.seqlens, wl.q_len, wl.k, [], wl.Hq, wl.Hkv, scale)
     if layers_np is None:
         if wl.dtype == "f32":
             layers_np = [ti.project_kept(wl, ti.widen(ref["H_kept"], "f32"))]
