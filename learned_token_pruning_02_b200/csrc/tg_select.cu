@@ -256,13 +256,18 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
                         int32_t* cu_kept_dev, int32_t* dev_status, cudaStream_t st) {
   SelParams p = {};
   for (int i = 0; i < nseq; ++i) p.s[i] = seqs[i];
-  int R = 4;
-  while (R < 32 && (int64_t)NT * R < n_ctx_max) R *= 2;
-  int C = (int)((n_ctx_max + (int64_t)NT * R - 1) / ((int64_t)NT * R));
-  if (C < 1) C = 1;
-  if (C > 8) return fail(TG_ERR_UNSUPPORTED, "context of %d tokens exceeds the select capacity", n_ctx_max);
+  // Spread a sequence over up to 8 SMs (one cluster) so its scores stream in parallel, with
+  // at least 4 keys per thread; R keys per thread are held in registers.
+  int C = (int)((n_ctx_max + 4 * NT - 1) / (4 * NT));
+  C = C < 1 ? 1 : (C > 8 ? 8 : C);
+  int R = 1;
+  while (R < 32 && (int64_t)NT * R * C < n_ctx_max) R *= 2;
+  if ((int64_t)NT * R * C < n_ctx_max)
+    return fail(TG_ERR_UNSUPPORTED, "context of %d tokens exceeds the select capacity", n_ctx_max);
   p.C = C;
   switch (R) {
+    case 1: return launch_r<1>(score, p, nseq, kept_idx, cu_kept_dev, dev_status, st);
+    case 2: return launch_r<2>(score, p, nseq, kept_idx, cu_kept_dev, dev_status, st);
     case 4: return launch_r<4>(score, p, nseq, kept_idx, cu_kept_dev, dev_status, st);
     case 8: return launch_r<8>(score, p, nseq, kept_idx, cu_kept_dev, dev_status, st);
     case 16: return launch_r<16>(score, p, nseq, kept_idx, cu_kept_dev, dev_status, st);
