@@ -5,20 +5,23 @@
 // (aitualizate.com article: the score acts as a bias on the attention logits, with a
 // per-head gain). Causal on original positions, grouped KV heads (kv = h / (Hq/Hkv)).
 //
-// Design (B200, bf16 in, fp32 softmax and accumulation), one CTA per (sequence, 128-row
+// Design (B200, bf16 in, fp32 softmax and accumulation). One CTA per (sequence, 128-row
 // query tile, query head), launched longest causal row-range first so the block scheduler
-// packs the triangle like a longest-processing-time list schedule:
-//   * warp 0: TMA loads the Q tile once and K_j, V_j tiles (128 keys) into a 2-stage ring
-//     (128-byte swizzle; K and V have separate "full" barriers so S_j can start early).
-//   * warp 1 (one thread): tcgen05.mma. S_j = Q K_j^T (M=128, N=128, K=D) into one of two
-//     TMEM S buffers, then O += P_j V_j with P_j read straight from TMEM (A operand in
-//     tensor memory) and V_j from shared memory (N-contiguous operand). The issue order
-//     S_0, S_1, PV_0, S_2, PV_1, ... overlaps each softmax with the next QK^T.
-//   * warps 2-5: online softmax, one query row per thread: log2-domain logits
-//     scale*log2e*S + gain*log2e*log g_j (staged in shared memory per key tile), causal mask
-//     on the diagonal tile, running max/sum, O rescale in TMEM when the max moves, and P
-//     written back as packed bf16 into the S buffer it came from. The epilogue normalises
-//     O, writes it as bf16 and the row's log-sum-exp.
+// packs the triangle like a longest-processing-time list schedule. The key tiles of the CTA
+// are split into two interleaved chains (even and odd tiles), each with its own softmax
+// warpgroup, TMEM score buffer and TMEM output accumulator, so one group's exponentials
+// overlap the other group's matrix products:
+//   * warp 0: TMA loads Q once and K_j, V_j (128 keys) into the stage of chain j % 2, and
+//     stages the tile's per-key bias gain*log2(e)*log g_j in shared memory.
+//   * warp 1 (one thread): tcgen05.mma. S_j = Q K_j^T (M=128, N=128, K=D) into the chain's
+//     TMEM S buffer; O_c += P_j V_j with P_j read from TMEM (A operand in tensor memory) and
+//     V_j from shared memory (N-contiguous operand).
+//   * warps 2-5 (chain 0) and 6-9 (chain 1): one query row per thread. Pass 1 reads S and
+//     finds the row max of scale*log2(e)*S + bias (causal mask on the diagonal tile);
+//     pass 2 writes P = 2^(x - m) as packed bf16 into the same TMEM columns. The running
+//     max is only moved (and O rescaled in TMEM) when it grows by more than 8 (a factor
+//     256), which keeps every P <= 256 and the result exact after normalisation.
+//   * Chain 0's warps merge the two chains (max, sum, O) and write O (bf16) and the LSE.
 //   * The unnormalised variant multiplies P by g_j^gain before the PV product and sums the
 //     unbiased weights.
 //   * Every wait is bounded (about 2 s); on a timeout the CTA sets TG_DEV_TIMEOUT, drains
@@ -33,9 +36,10 @@ using namespace sm100;
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleSlack = 8.f;  // log2 units the running max may lag behind
 
 struct ATParams {
   int off[kMaxSeqPerLaunch];
@@ -52,13 +56,12 @@ struct ACfg {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = TILE_BYTES;  // + stage * 2 * TILE_BYTES
   static constexpr int V_OFF = 2 * TILE_BYTES;
-  static constexpr int STAGES = 2;
-  static constexpr int TAIL_OFF = TILE_BYTES * (1 + 2 * STAGES);
+  static constexpr int TAIL_OFF = TILE_BYTES * 5;
   static constexpr int TAIL = 4096;
   static constexpr int SMEM = 1024 + TAIL_OFF + TAIL;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BQ, BKV, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, true);
-  static constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256, 256+D)
+  static constexpr uint32_t TMEM_COLS = 512;  // S_c at [128c, 128c+128), O_c at [256 + Dc, 256 + D(c+1))
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -79,18 +82,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* tail = smem + C::TAIL_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   uint64_t* qfull = bars + 0;
-  uint64_t* kfull = bars + 1;   // [2]
-  uint64_t* vfull = bars + 3;   // [2]
-  uint64_t* empty = bars + 5;   // [2]
-  uint64_t* sfull = bars + 7;   // [2]
-  uint64_t* pready = bars + 9;  // [2]
-  uint64_t* pvdone = bars + 11;
-  uint64_t* drain = bars + 12;
-  uint64_t* bfull = bars + 13;  // [2] key-tile bias staged by the producer warp
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* kfull = bars + 1;    // [2] per chain/stage
+  uint64_t* vfull = bars + 3;    // [2]
+  uint64_t* empty = bars + 5;    // [2]
+  uint64_t* bfull = bars + 7;    // [2]
+  uint64_t* sfull = bars + 9;    // [2]
+  uint64_t* pready = bars + 11;  // [2]
+  uint64_t* pvdone = bars + 13;  // [2]
+  uint64_t* mlready = bars + 15;
+  uint64_t* drain = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* bias_s = reinterpret_cast<float*>(tail + 256);  // [2][128]
   float* gmul_s = bias_s + 2 * BKV;                      // [2][128]
+  float* ml_s = gmul_s + 2 * BKV;                        // [2][128]: chain-1 max and sum
 
   // ---- which (sequence, query tile, head) this CTA owns: longest row-ranges first
   const int h = blockIdx.x % Hq;
@@ -115,7 +120,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   const int off = p.off[b], m = p.m[b];
   const int nt = t + 1;  // key tiles 0..t (causal)
+  const int n0 = (nt + 1) >> 1, n1 = nt >> 1;  // key tiles in chain 0 (even) and chain 1 (odd)
   const int kvh = h / (Hq / Hkv);
+  const bool unnorm = (flags & TG_ATTN_UNNORMALISED) != 0;
+  const float gain2 = (gain ? gain[h] : 1.f) * kLog2e;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -124,11 +132,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&kfull[s], 1);
       mbar_init(&vfull[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&bfull[s], 32);
       mbar_init(&sfull[s], 1);
       mbar_init(&pready[s], 128);
-      mbar_init(&bfull[s], 32);
+      mbar_init(&pvdone[s], 1);
     }
-    mbar_init(pvdone, 1);
+    mbar_init(mlready, 128);
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -146,11 +155,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 256;
 
-  const bool unnorm = (flags & TG_ATTN_UNNORMALISED) != 0;
-  const float gain2 = (gain ? gain[h] : 1.f) * kLog2e;
-  if (warp == 0) {  // ------------------------------------------------ TMA producer warp
+  if (warp == 0) {  // ---------------------------------------------------- TMA producer warp
     int issued = 0;
     if (lane == 0) {
       mbar_arrive_expect_tx(qfull, C::TILE_BYTES);
@@ -158,32 +164,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_load_2d(smem + C::Q_OFF + bx * (BQ * 128), &tmQ, h * D + bx * 64, off + t * BQ, qfull);
     }
     for (int j = 0; j < nt; ++j) {
-      const int s = j & 1;
+      const int c = j & 1, u = j >> 1;
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1u, abort, dev_status);
+      if (lane == 0) ok = mbar_wait(&empty[c], (u & 1) ^ 1u, abort, dev_status);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       if (lane == 0) {
-        uint8_t* kb = smem + C::K_OFF + s * 2 * C::TILE_BYTES;
-        uint8_t* vb = smem + C::V_OFF + s * 2 * C::TILE_BYTES;
-        mbar_arrive_expect_tx(&kfull[s], C::TILE_BYTES);
+        uint8_t* kb = smem + C::K_OFF + c * 2 * C::TILE_BYTES;
+        uint8_t* vb = smem + C::V_OFF + c * 2 * C::TILE_BYTES;
+        mbar_arrive_expect_tx(&kfull[c], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_2d(kb + bx * (BKV * 128), &tmK, kvh * D + bx * 64, off + j * BKV, &kfull[s]);
-        mbar_arrive_expect_tx(&vfull[s], C::TILE_BYTES);
+          tma_load_2d(kb + bx * (BKV * 128), &tmK, kvh * D + bx * 64, off + j * BKV, &kfull[c]);
+        mbar_arrive_expect_tx(&vfull[c], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_2d(vb + bx * (BKV * 128), &tmV, kvh * D + bx * 64, off + j * BKV, &vfull[s]);
+          tma_load_2d(vb + bx * (BKV * 128), &tmV, kvh * D + bx * 64, off + j * BKV, &vfull[c]);
       }
       ++issued;
-      // per-key bias of this key tile (log2 domain), 4 keys per lane; the stage's slot is free
-      // because PV of the tile that used it last has completed (empty barrier above)
+      // per-key bias of this key tile (log2 domain), 4 keys per lane; the slot is free
+      // because the PV product of the chain's previous tile has completed (empty barrier)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int c = lane * 4 + e;
-        const int kl = j * BKV + c;
+        const int col = lane * 4 + e;
+        const int kl = j * BKV + col;
         const float bv = (logg && kl < m) ? gain2 * logg[off + kl] : 0.f;
-        bias_s[s * BKV + c] = unnorm ? 0.f : bv;
-        gmul_s[s * BKV + c] = unnorm ? ex2(bv) : 1.f;
+        bias_s[c * BKV + col] = unnorm ? 0.f : bv;
+        gmul_s[c * BKV + col] = unnorm ? ex2(bv) : 1.f;
       }
-      mbar_arrive(&bfull[s]);
+      mbar_arrive(&bfull[c]);
     }
     if (lane == 0 && *abort) {  // let the copies in flight land before the CTA can leave
       const uint64_t t0 = globaltimer_ns();
@@ -197,137 +203,178 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {  // ------------------------------------------------ MMA issuer
+  } else if (warp == 1) {  // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
       const uint32_t qa = smem_u32(smem + C::Q_OFF);
+      auto issue_s = [&](int j) -> bool {
+        const int c = j & 1, u = j >> 1;
+        if (!mbar_wait(&kfull[c], u & 1, abort, dev_status)) return false;
+        // the chain's S buffer still holds P of its previous tile until that PV completes
+        if (u > 0 && !mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status)) return false;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(smem + C::K_OFF + c * 2 * C::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          mma_ss(tmem + c * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK, kk > 0);
+        }
+        mma_commit(&sfull[c]);
+        return true;
+      };
       bool ok = mbar_wait(qfull, 0, abort, dev_status);
-      for (int j = 0; ok && j <= nt; ++j) {
-        if (j < nt) {
-          const int sb = j & 1;
-          if (j >= 2 && !mbar_wait(pvdone, (j - 2) & 1, abort, dev_status)) break;
-          if (!mbar_wait(&kfull[sb], (j >> 1) & 1, abort, dev_status)) break;
-          tc_fence_after();
-          const uint32_t ka = smem_u32(smem + C::K_OFF + sb * 2 * C::TILE_BYTES);
+      for (int j = 0; ok && j < 2 && j < nt; ++j) ok = issue_s(j);
+      for (int j = 0; ok && j < nt; ++j) {
+        const int c = j & 1, u = j >> 1;
+        if (!mbar_wait(&pready[c], u & 1, abort, dev_status) || !mbar_wait(&vfull[c], u & 1, abort, dev_status))
+          break;
+        tc_fence_after();
+        const uint32_t va = smem_u32(smem + C::V_OFF + c * 2 * C::TILE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-            mma_ss(tS + sb * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK, kk > 0);
-          }
-          mma_commit(&sfull[sb]);
-        }
-        if (j >= 1) {
-          const int jj = j - 1, pb = jj & 1;
-          if (!mbar_wait(&pready[pb], (jj >> 1) & 1, abort, dev_status)) break;
-          if (!mbar_wait(&vfull[pb], (jj >> 1) & 1, abort, dev_status)) break;
-          tc_fence_after();
-          const uint32_t va = smem_u32(smem + C::V_OFF + pb * 2 * C::TILE_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk)
-            mma_ts(tO, tS + pb * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024), C::IDESC_PV,
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(pvdone);
-          mma_commit(&empty[pb]);
-        }
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
+                 C::IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&pvdone[c]);
+        mma_commit(&empty[c]);
+        if (j + 2 < nt) ok = issue_s(j + 2);
       }
       mma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {
       }
     }
-  } else {  // ------------------------------------------------------------ softmax warps 2..5
+  } else {  // --------------------------------------------------------- softmax warpgroups
+    const int c = (warp - 2) >> 2;  // chain: 0 = warps 2-5 (even tiles), 1 = warps 6-9 (odd tiles)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // query row in the tile == TMEM lane
     const int il = t * BQ + r;     // row within the sequence
     const bool valid = il < m;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    if (h == 0 && valid && il > 0 && dev_status && pos[off + il - 1] >= pos[off + il])
+    const uint32_t tS = tmem + lane_base + c * BKV;
+    const uint32_t tO = tmem + lane_base + 256 + c * D;
+    if (c == 0 && h == 0 && valid && il > 0 && dev_status && pos[off + il - 1] >= pos[off + il])
       atomicOr(dev_status, TG_DEV_POS_NOT_ASCENDING);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      const int sb = j & 1;
+    const int n_mine = c == 0 ? n0 : n1;
+    for (int u = 0; u < n_mine; ++u) {
+      const int j = 2 * u + c;
       // warp-uniform waits: the tcgen05.ld/st below are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&bfull[sb], (j >> 1) & 1, abort, dev_status) &&
-                                       mbar_wait(&sfull[sb], (j >> 1) & 1, abort, dev_status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bfull[c], u & 1, abort, dev_status) &&
+                                       mbar_wait(&sfull[c], u & 1, abort, dev_status))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[BKV];
-#pragma unroll
-      for (int c = 0; c < BKV / 32; ++c)
-        tmem_ld32(tS + lane_base + sb * BKV + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-      tmem_wait_ld();
-      const float* bs = bias_s + sb * BKV;
+      const float* bs = bias_s + c * BKV;
       const bool diag = (j == t);
+      // pass 1: row max of the biased log2-domain logits
       float mx = -INFINITY;
+#pragma unroll 1
+      for (int ch = 0; ch < BKV / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tS + ch * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < BKV; ++c) {
-        float x = fmaf(__uint_as_float(sr[c]), qk_scale, bs[c]);
-        if (diag && c > r) x = -INFINITY;
-        sr[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
-      }
-      const float m_new = fmaxf(m_run, mx);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;  // a row whose keys are all -inf stays finite
-      const float alpha = ex2(m_run - m_use);
-      float sum = 0.f;
-      uint32_t pk[BKV / 2];
-      const float* gm = gmul_s + sb * BKV;
-#pragma unroll
-      for (int c = 0; c < BKV; c += 2) {
-        const float p0 = ex2(__uint_as_float(sr[c]) - m_use);
-        const float p1 = ex2(__uint_as_float(sr[c + 1]) - m_use);
-        sum += p0 + p1;
-        pk[c / 2] = unnorm ? pack_bf16(p0 * gm[c], p1 * gm[c + 1]) : pack_bf16(p0, p1);
-      }
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
-      if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(pvdone, (j - 1) & 1, abort, dev_status))) {
-          ok = false;
-          break;
+        for (int e = 0; e < 32; ++e) {
+          const int col = ch * 32 + e;
+          const float x = fmaf(__uint_as_float(v[e]), qk_scale, bs[col]);
+          mx = fmaxf(mx, (diag && col > r) ? -INFINITY : x);
         }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {  // rescale the running O in TMEM
+      }
+      const float m_cand = fmaxf(m_run, mx);
+      if (__any_sync(0xffffffffu, m_cand > m_run + kRescaleSlack)) {
+        const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_cand);  // 0 on the chain's first tile
+        if (u > 0) {  // rescale the chain's O once its previous PV product has landed
+          if (!__all_sync(0xffffffffu, mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(tO + lane_base + c0, o);
+            tmem_ld32(tO + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + lane_base + c0, o);
+            tmem_st32(tO + c0, o);
           }
           tmem_wait_st();
         }
+        l_run *= alpha;
+        m_run = m_cand;
       }
-      tmem_st32(tS + lane_base + sb * BKV, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + lane_base + sb * BKV + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&pready[sb]);
-    }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(pvdone, (nt - 1) & 1, abort, dev_status))) {
-      tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = O + ((int64_t)(off + il) * Hq + h) * D;
+      const float mb = m_run == -INFINITY ? 0.f : m_run;
+      const float* gm = gmul_s + c * BKV;
+      // pass 2: P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns
+      float sum = 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tO + lane_base + c0, o);
+      for (int ch = 0; ch < BKV / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tS + ch * 32, v);
         tmem_wait_ld();
-        uint32_t pkd[16];
+        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pkd[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+        for (int e = 0; e < 32; e += 2) {
+          const int col = ch * 32 + e;
+          float x0 = fmaf(__uint_as_float(v[e]), qk_scale, bs[col]);
+          float x1 = fmaf(__uint_as_float(v[e + 1]), qk_scale, bs[col + 1]);
+          if (diag && col > r) x0 = -INFINITY;
+          if (diag && col + 1 > r) x1 = -INFINITY;
+          const float p0 = ex2(x0 - mb), p1 = ex2(x1 - mb);
+          sum += p0 + p1;
+          pk[e >> 1] = unnorm ? pack_bf16(p0 * gm[col], p1 * gm[col + 1]) : pack_bf16(p0, p1);
         }
+        tmem_st16(tS + ch * 16, pk);
       }
-      if (valid && lse) lse[(int64_t)h * m_tot + off + il] = (m_run + __log2f(l_run)) * kLn2;
+      tmem_wait_st();
+      l_run += sum;
+      tc_fence_before();
+      mbar_arrive(&pready[c]);
+    }
+    if (c == 1) {  // hand the chain's max and sum to chain 0
+      ml_s[r] = ok ? m_run : -INFINITY;
+      ml_s[BKV + r] = ok ? l_run : 0.f;
+      mbar_arrive(mlready);
+    } else if (ok) {
+      const bool got = __all_sync(0xffffffffu, mbar_wait(mlready, 0, abort, dev_status) &&
+                                                   mbar_wait(&pvdone[0], (n0 - 1) & 1, abort, dev_status) &&
+                                                   (n1 == 0 || mbar_wait(&pvdone[1], (n1 - 1) & 1, abort, dev_status)));
+      if (got) {
+        tc_fence_after();
+        const float m1 = ml_s[r], l1 = ml_s[BKV + r];
+        const float mfin = fmaxf(m_run, m1);
+        const float mz = mfin == -INFINITY ? 0.f : mfin;
+        const float f0 = ex2(m_run - mz), f1 = n1 > 0 ? ex2(m1 - mz) : 0.f;
+        const float lt = l_run * f0 + l1 * f1;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float s0 = f0 * inv, s1 = f1 * inv;
+        __nv_bfloat16* orow = O + ((int64_t)(off + il) * Hq + h) * D;
+        const uint32_t tO1 = tmem + lane_base + 256 + D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(tO + c0, o0);
+          if (n1 > 0) tmem_ld32(tO1 + c0, o1);
+          tmem_wait_ld();
+          uint32_t pkd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float a0 = __uint_as_float(o0[2 * e]) * s0, a1 = __uint_as_float(o0[2 * e + 1]) * s0;
+            if (n1 > 0) {
+              a0 = fmaf(__uint_as_float(o1[2 * e]), s1, a0);
+              a1 = fmaf(__uint_as_float(o1[2 * e + 1]), s1, a1);
+            }
+            pkd[e] = pack_bf16(a0, a1);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+          }
+        }
+        if (valid && lse) lse[(int64_t)h * m_tot + off + il] = (mz + __log2f(lt)) * kLn2;
+      }
     }
   }
 

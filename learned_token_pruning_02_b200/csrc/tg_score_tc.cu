@@ -28,17 +28,20 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 224;  // warp 0: H loads, 1: MMA, 2-5: epilogue, 6: W1 loads
 
 template <int DG>
 struct Cfg {
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = DG * BK * 2;
-  static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = DG == 256 ? 4 : (DG == 128 ? 6 : 8);
+  static constexpr int A_BYTES = BM * BK * 2;  // one 128 x 64 slice of H
+  static constexpr int B_BYTES = DG * BK * 2;  // one dg x 64 slice of W1
+  // H streams from HBM through a deep ring (about 2 us of latency cover at full rate);
+  // W1 comes from L2 through a shallow one.
+  static constexpr int SA = DG == 64 ? 10 : 8;
+  static constexpr int SB = DG == 256 ? 2 : (DG == 128 ? 3 : 4);
+  static constexpr int RING = SA * A_BYTES + SB * B_BYTES;
   static constexpr int TMEM_COLS = 2 * DG;
-  static constexpr int TAIL = 2048;  // barriers, flags, b1/w2 copies
-  static constexpr int SMEM = 1024 + STAGES * STAGE + TAIL + 2 * DG * 4;
+  static constexpr int TAIL = 2048;  // barriers, flags
+  static constexpr int SMEM = 1024 + RING + TAIL + 2 * DG * 4;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, DG, false);
 };
 
@@ -50,10 +53,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   using C = Cfg<DG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* tail = smem + C::STAGES * C::STAGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tail);
-  uint64_t* empty = full + C::STAGES;
-  uint64_t* accf = empty + C::STAGES;
+  uint8_t* ringA = smem;
+  uint8_t* ringB = smem + C::SA * C::A_BYTES;
+  uint8_t* tail = smem + C::RING;
+  uint64_t* afull = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* aempty = afull + C::SA;
+  uint64_t* bfull = aempty + C::SA;
+  uint64_t* bempty = bfull + C::SB;
+  uint64_t* accf = bempty + C::SB;
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -63,9 +70,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < C::SA; ++s) {
+      mbar_init(&afull[s], 1);
+      mbar_init(&aempty[s], 1);
+    }
+    for (int s = 0; s < C::SB; ++s) {
+      mbar_init(&bfull[s], 1);
+      mbar_init(&bempty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&accf[a], 1);
@@ -79,7 +90,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tmH);
     prefetch_tmap(&tmW);
   }
-  if (warp >= 2) {
+  if (warp >= 2 && warp <= 5) {
     for (int u = threadIdx.x - 64; u < DG; u += 128) {
       b1s[u] = b1 ? b1[u] : 0.f;
       w2s[u] = __bfloat162float(w2[u]);
@@ -94,39 +105,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {  // TMA producer
+  if (warp == 0 || warp == 6) {
+    if (lane == 0) {  // TMA producers: warp 0 streams H, warp 6 streams W1
+      const bool isA = warp == 0;
+      const int NS = isA ? C::SA : C::SB;
+      uint64_t* full = isA ? afull : bfull;
+      uint64_t* empty = isA ? aempty : bempty;
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
       for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, dev_status)) break;
-          uint8_t* a = smem + stage * C::STAGE;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE);
-          tma_load_2d(a, &tmH, kb * BK, tile * BM, &full[stage]);
-          tma_load_2d(a + C::A_BYTES, &tmW, kb * BK, 0, &full[stage]);
+          if (isA) {
+            mbar_arrive_expect_tx(&full[stage], C::A_BYTES);
+            tma_load_2d(ringA + stage * C::A_BYTES, &tmH, kb * BK, tile * BM, &full[stage]);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
+            tma_load_2d(ringB + stage * C::B_BYTES, &tmW, kb * BK, 0, &full[stage]);
+          }
           ++issued;
-          if (++stage == C::STAGES) {
+          if (++stage == NS) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       if (*abort) {  // drain the copies still in flight before the CTA can leave
-        for (long n = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; n < issued; ++n) {
-          int s = (int)(n % C::STAGES);
-          uint32_t ph = (uint32_t)((n / C::STAGES) & 1);
+        for (long n = issued - NS < 0 ? 0 : issued - NS; n < issued; ++n) {
+          const int s2 = (int)(n % NS);
+          const uint32_t ph = (uint32_t)((n / NS) & 1);
           const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full[s], ph) && globaltimer_ns() - t0 < 1000000000ull) {
+          while (!mbar_try_wait(&full[s2], ph) && globaltimer_ns() - t0 < 1000000000ull) {
           }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {  // MMA issuer
-      int stage = 0;
-      uint32_t phase = 0;
+      int sa = 0, sb = 0;
+      uint32_t pa = 0, pb = 0;
       int it = 0;
       for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x, ++it) {
         const int acc = it & 1;
@@ -135,21 +153,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t d = tmem + acc * DG;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort, dev_status)) {
+          if (!mbar_wait(&afull[sa], pa, abort, dev_status) || !mbar_wait(&bfull[sb], pb, abort, dev_status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * C::STAGE);
-          const uint32_t b0 = a0 + C::A_BYTES;
+          const uint32_t a0 = smem_u32(ringA + sa * C::A_BYTES);
+          const uint32_t b0 = smem_u32(ringB + sb * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             mma_ss(d, sdesc_sw128(a0 + 32 * k, 16, 1024), sdesc_sw128(b0 + 32 * k, 16, 1024), C::IDESC,
                    (kb | k) != 0);
-          mma_commit(&empty[stage]);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
+          mma_commit(&aempty[sa]);
+          mma_commit(&bempty[sb]);
+          if (++sa == C::SA) {
+            sa = 0;
+            pa ^= 1u;
+          }
+          if (++sb == C::SB) {
+            sb = 0;
+            pb ^= 1u;
           }
         }
         if (!ok) break;
