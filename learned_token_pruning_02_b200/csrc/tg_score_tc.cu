@@ -3,21 +3,19 @@
 // TokenGate paper page (thelatestinai.com), Figure 1(b): a small scoring network scores
 // every hidden state at the selection layer; aitualizate.com article, phase 2.
 //
-// Design (B200, bf16 in, fp32 accumulate):
-//   * One CTA per SM, persistent over 128-token tiles. The whole hidden width dg (<= 256)
-//     is one UMMA N, so a tile is one 128 x dg accumulator in TMEM (fp32) and H is read
-//     from HBM exactly once. Two accumulators (2 x dg TMEM columns) let the epilogue of
-//     tile t overlap the MMAs of tile t+1.
-//   * Warp 0 streams 64-wide K slices of H (128 x 64) and W1 (dg x 64) with TMA into a ring
-//     of shared-memory stages in the 128-byte swizzle layout; W1 stays L2-resident.
-//   * Warp 1 (one thread) issues tcgen05.mma (M=128, N=dg, K=16) and releases each stage
-//     with tcgen05.commit; it also owns the TMEM allocation.
-//   * Warps 2-5 are the epilogue: each thread owns one token row, reads its dg fp32 values
-//     with tcgen05.ld, and reduces + b1 -> exact-erf GELU -> * w2 -> sum in registers, so
-//     the [n_tok, dg] hidden activation never leaves the SM. Only 4 bytes per token are
-//     written.
-//   * Every wait is bounded (about 2 s); on a timeout the kernel sets TG_DEV_TIMEOUT,
-//     drains its outstanding copies and MMAs, frees TMEM and returns.
+// Design (B200, bf16 in, fp32 accumulate). The whole hidden width dg (<= 256) is one UMMA N,
+// so the [n_tok, dg] activation lives only in TMEM and H is read from HBM exactly once.
+// W1 (dg x d) is re-read from L2 by every CTA, so each CTA multiplies one W1 slice into TWO
+// 128-token tiles (a 256-token pair) to halve the W1 bytes per flop:
+//   * warp 0 (one thread): TMA loads, per 64-wide K slice, H rows of both tiles and the W1
+//     slice into a ring of shared-memory stages (128-byte swizzle).
+//   * warp 1 (one thread): tcgen05.mma M=128, N=dg, K=16 for both tiles into two fp32 TMEM
+//     accumulators (2 x dg columns); releases stages with tcgen05.commit; owns TMEM.
+//   * warps 2-17: epilogue. Four warps cover the 128 TMEM lanes; four such groups split the
+//     work into (tile, half of the dg columns). Each thread reduces + b1 -> exact-erf GELU
+//     -> * w2 over its 128 columns in registers; the two halves meet in shared memory.
+//   * Persistent over tile pairs; every wait is bounded (about 2 s); on a timeout the kernel
+//     sets its abort flag, drains outstanding copies and MMAs, frees TMEM and returns.
 #include "tg_internal.cuh"
 #include "tg_sm100.cuh"
 
@@ -28,20 +26,18 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int NTHREADS = 224;  // warp 0: H loads, 1: MMA, 2-5: epilogue, 6: W1 loads
+constexpr int NEPI = 16;                      // epilogue warps
+constexpr int NTHREADS = 32 * (2 + NEPI);     // 576
 
 template <int DG>
 struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;  // one 128 x 64 slice of H
   static constexpr int B_BYTES = DG * BK * 2;  // one dg x 64 slice of W1
-  // H streams from HBM through a deep ring (about 2 us of latency cover at full rate);
-  // W1 comes from L2 through a shallow one.
-  static constexpr int SA = DG == 64 ? 10 : 8;
-  static constexpr int SB = DG == 256 ? 2 : (DG == 128 ? 3 : 4);
-  static constexpr int RING = SA * A_BYTES + SB * B_BYTES;
+  static constexpr int STAGE = 2 * A_BYTES + B_BYTES;
+  static constexpr int STAGES = DG == 256 ? 3 : (DG == 128 ? 4 : 5);
   static constexpr int TMEM_COLS = 2 * DG;
-  static constexpr int TAIL = 2048;  // barriers, flags
-  static constexpr int SMEM = 1024 + RING + TAIL + 2 * DG * 4;
+  static constexpr int TAIL = 1024;  // barriers, flags
+  static constexpr int SMEM = 1024 + STAGES * STAGE + TAIL + 2 * DG * 4 + 2 * BM * 4;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, DG, false);
 };
 
@@ -49,39 +45,33 @@ template <int DG>
 __global__ void __launch_bounds__(NTHREADS, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW,
                     const float* __restrict__ b1, const __nv_bfloat16* __restrict__ w2, float b2,
-                    float* __restrict__ score, int n_tok, int nk, int n_tiles, int32_t* __restrict__ dev_status) {
+                    float* __restrict__ score, int n_tok, int nk, int n_pairs, int32_t* __restrict__ dev_status) {
   using C = Cfg<DG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ringA = smem;
-  uint8_t* ringB = smem + C::SA * C::A_BYTES;
-  uint8_t* tail = smem + C::RING;
-  uint64_t* afull = reinterpret_cast<uint64_t*>(tail);
-  uint64_t* aempty = afull + C::SA;
-  uint64_t* bfull = aempty + C::SA;
-  uint64_t* bempty = bfull + C::SB;
-  uint64_t* accf = bempty + C::SB;
-  uint64_t* acce = accf + 2;
-  uint64_t* drain = acce + 2;
+  uint8_t* tail = smem + C::STAGES * C::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint64_t* acce = accf + 1;
+  uint64_t* half_ready = acce + 1;  // [2] one per tile of the pair
+  uint64_t* drain = half_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* b1s = reinterpret_cast<float*>(tail + C::TAIL);
   float* w2s = b1s + DG;
+  float* part = w2s + DG;  // [2][BM] partial sums of the upper column half
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::SA; ++s) {
-      mbar_init(&afull[s], 1);
-      mbar_init(&aempty[s], 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    for (int s = 0; s < C::SB; ++s) {
-      mbar_init(&bfull[s], 1);
-      mbar_init(&bempty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&accf[a], 1);
-      mbar_init(&acce[a], 4);
-    }
+    mbar_init(accf, 1);
+    mbar_init(acce, NEPI);
+    mbar_init(&half_ready[0], 128);
+    mbar_init(&half_ready[1], 128);
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -90,8 +80,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tmH);
     prefetch_tmap(&tmW);
   }
-  if (warp >= 2 && warp <= 5) {
-    for (int u = threadIdx.x - 64; u < DG; u += 128) {
+  if (warp >= 2) {
+    for (int u = threadIdx.x - 64; u < DG; u += 32 * NEPI) {
       b1s[u] = b1 ? b1[u] : 0.f;
       w2s[u] = __bfloat162float(w2[u]);
     }
@@ -105,36 +95,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 || warp == 6) {
-    if (lane == 0) {  // TMA producers: warp 0 streams H, warp 6 streams W1
-      const bool isA = warp == 0;
-      const int NS = isA ? C::SA : C::SB;
-      uint64_t* full = isA ? afull : bfull;
-      uint64_t* empty = isA ? aempty : bempty;
+  if (warp == 0) {
+    if (lane == 0) {  // ---------------------------------------------------- TMA producer
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
+      for (int pr = blockIdx.x; pr < n_pairs && !*abort; pr += gridDim.x) {
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, dev_status)) break;
-          if (isA) {
-            mbar_arrive_expect_tx(&full[stage], C::A_BYTES);
-            tma_load_2d(ringA + stage * C::A_BYTES, &tmH, kb * BK, tile * BM, &full[stage]);
-          } else {
-            mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
-            tma_load_2d(ringB + stage * C::B_BYTES, &tmW, kb * BK, 0, &full[stage]);
-          }
+          uint8_t* st = smem + stage * C::STAGE;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE);
+          tma_load_2d(st, &tmH, kb * BK, (2 * pr) * BM, &full[stage]);
+          tma_load_2d(st + C::A_BYTES, &tmH, kb * BK, (2 * pr + 1) * BM, &full[stage]);
+          tma_load_2d(st + 2 * C::A_BYTES, &tmW, kb * BK, 0, &full[stage]);
           ++issued;
-          if (++stage == NS) {
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       if (*abort) {  // drain the copies still in flight before the CTA can leave
-        for (long n = issued - NS < 0 ? 0 : issued - NS; n < issued; ++n) {
-          const int s2 = (int)(n % NS);
-          const uint32_t ph = (uint32_t)((n / NS) & 1);
+        for (long n = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; n < issued; ++n) {
+          const int s2 = (int)(n % C::STAGES);
+          const uint32_t ph = (uint32_t)((n / C::STAGES) & 1);
           const uint64_t t0 = globaltimer_ns();
           while (!mbar_try_wait(&full[s2], ph) && globaltimer_ns() - t0 < 1000000000ull) {
           }
@@ -142,41 +126,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {  // MMA issuer
-      int sa = 0, sb = 0;
-      uint32_t pa = 0, pb = 0;
+    if (lane == 0) {  // ------------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
       int it = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        if (!mbar_wait(&acce[acc], ((it >> 1) & 1) ^ 1u, abort, dev_status)) break;
+      for (int pr = blockIdx.x; pr < n_pairs && !*abort; pr += gridDim.x, ++it) {
+        if (!mbar_wait(acce, (it & 1) ^ 1u, abort, dev_status)) break;
         tc_fence_after();
-        const uint32_t d = tmem + acc * DG;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&afull[sa], pa, abort, dev_status) || !mbar_wait(&bfull[sb], pb, abort, dev_status)) {
+          if (!mbar_wait(&full[stage], phase, abort, dev_status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(ringA + sa * C::A_BYTES);
-          const uint32_t b0 = smem_u32(ringB + sb * C::B_BYTES);
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE);
+          const uint32_t a1 = a0 + C::A_BYTES;
+          const uint32_t b0 = a0 + 2 * C::A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            mma_ss(d, sdesc_sw128(a0 + 32 * k, 16, 1024), sdesc_sw128(b0 + 32 * k, 16, 1024), C::IDESC,
-                   (kb | k) != 0);
-          mma_commit(&aempty[sa]);
-          mma_commit(&bempty[sb]);
-          if (++sa == C::SA) {
-            sa = 0;
-            pa ^= 1u;
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t bd = sdesc_sw128(b0 + 32 * k, 16, 1024);
+            mma_ss(tmem, sdesc_sw128(a0 + 32 * k, 16, 1024), bd, C::IDESC, (kb | k) != 0);
+            mma_ss(tmem + DG, sdesc_sw128(a1 + 32 * k, 16, 1024), bd, C::IDESC, (kb | k) != 0);
           }
-          if (++sb == C::SB) {
-            sb = 0;
-            pb ^= 1u;
+          mma_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&accf[acc]);
+        mma_commit(accf);
       }
       // every MMA issued above completes before TMEM can be released
       mma_commit(drain);
@@ -184,34 +164,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {
       }
     }
-  } else {  // epilogue: warps 2..5, one token row per thread
-    const int q = warp & 3;
+  } else {  // ------------------------------------------- epilogue: warps 2..17
+    const int grp = (warp - 2) >> 2;  // 0..3
+    const int tile = grp >> 1, half = grp & 1;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
+    const int c_lo = half * (DG / 2);
     int it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
-      const int acc = it & 1;
+    for (int pr = blockIdx.x; pr < n_pairs; pr += gridDim.x, ++it) {
       // warp-uniform: the tcgen05.ld below is warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&accf[acc], (it >> 1) & 1, abort, dev_status))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(accf, it & 1, abort, dev_status))) break;
       tc_fence_after();
       float s = 0.f;
-      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + acc * DG;
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + tile * DG + c_lo;
 #pragma unroll 1
-      for (int c0 = 0; c0 < DG; c0 += 32) {
+      for (int c0 = 0; c0 < DG / 2; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(base + c0, v);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float z = __uint_as_float(v[j]) + b1s[c0 + j];
+          const float z = __uint_as_float(v[j]) + b1s[c_lo + c0 + j];
           const float gz = 0.5f * z * (1.f + erff(z * 0.70710678118654752f));
-          s = fmaf(gz, w2s[c0 + j], s);
+          s = fmaf(gz, w2s[c_lo + c0 + j], s);
         }
       }
       tc_fence_before();
+      bool ok = true;
+      if (half == 1) {
+        part[tile * BM + row] = s;
+        mbar_arrive(&half_ready[tile]);
+      } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(&half_ready[tile], it & 1, abort, dev_status));
+        const long r = (long)(2 * pr + tile) * BM + row;
+        if (ok && r < n_tok) score[r] = (s + part[tile * BM + row]) + b2;
+      }
+      // the accumulators (and the partial sums) are released only once this pair is fully
+      // consumed, so neither can be overwritten early
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[acc]);
-      const long r = (long)tile * BM + row;
-      if (r < n_tok) score[r] = s + b2;
+      if (lane == 0) mbar_arrive(acce);
+      if (!ok) break;
     }
   }
 
@@ -236,10 +228,11 @@ tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void
     attr_set = true;
   }
   const int n_tiles = (int)((n_tok + BM - 1) / BM);
+  const int n_pairs = (n_tiles + 1) / 2;
   int grid = device_sm_count();
-  if (grid > n_tiles) grid = n_tiles;
+  if (grid > n_pairs) grid = n_pairs;
   score_tc_kernel<DG><<<grid, NTHREADS, C::SMEM, st>>>(tmH, tmW, b1, static_cast<const __nv_bfloat16*>(w2), b2, score,
-                                                      (int)n_tok, d / BK, n_tiles, nullptr);
+                                                      (int)n_tok, d / BK, n_pairs, nullptr);
   return cuda_status(cudaGetLastError(), "tg_score: score_tc launch");
 }
 

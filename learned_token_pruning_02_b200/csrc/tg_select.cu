@@ -6,15 +6,18 @@
 //
 // Design (B200): one CTA of 1024 threads per sequence while its context fits in shared
 // memory (32768 keys = 128 KB), otherwise one thread-block cluster of up to 8 CTAs. The
-// scores are read from HBM exactly once and turned into order-preserving 32-bit keys held in
-// shared memory. An MSB-first radix select with 4-bit digits (8 passes) finds the K-th
-// largest key T without any atomics: every thread counts its keys per digit in four
-// registers of packed 8-bit counters, warps reduce the 16 counts with redux.sync, and warp
-// 0 sums the warps (and, in a cluster, the CTAs over distributed shared memory after a
-// hardware cluster barrier) and picks the digit. Keys > T are kept, and keys == T in index
-// order until K is reached (lower index wins ties). An ascending compaction uses warp
-// ballots and one block-wide scan per class. No workspace: the per-sequence descriptors
-// travel as kernel parameters; nothing spins.
+// scores are read from HBM exactly once (loads batched 8 deep per thread) into
+// order-preserving 32-bit keys in shared memory. An MSB-first radix select in three passes
+// finds the K-th largest key T:
+//   pass 0: sign + exponent (9 bits, 512 bins). Scores crowd into a few exponents, so
+//           lanes with the same bin are merged with match.any before one shared atomic;
+//   pass 1: the next 11 bits (2048 bins) of the keys in the chosen bin - nearly uniform;
+//   pass 2: the last 12 bits (4096 bins) of the few keys left.
+// In a cluster every CTA sums the cluster's histograms over distributed shared memory after
+// a hardware cluster barrier and scans them itself. Keys > T are kept, and keys == T in
+// index order until K is reached (lower index wins ties). An ascending compaction uses warp
+// ballots and block-wide scans. No workspace: the per-sequence descriptors travel as kernel
+// parameters; nothing spins.
 #include <cooperative_groups.h>
 
 #include "tg_internal.cuh"
@@ -26,6 +29,7 @@ namespace {
 
 constexpr int NT = 1024;
 constexpr int MAX_ROWS = 32;  // keys per thread: 32 x 1024 = 32768 keys per CTA
+constexpr int NB0 = 512, NB1 = 2048, NB2 = 4096;
 
 struct SelParams {
   SelSeq s[kMaxSeqPerLaunch];
@@ -42,17 +46,15 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive scan, in place, of n <= 1024 ints in shared memory; returns the total.
-__device__ __forceinline__ int block_scan_excl(int* a, int n, int* warp_sums) {
+// Inclusive block-wide scan of one int per thread; optionally returns the block total.
+__device__ __forceinline__ int block_scan_incl(int v, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int v = threadIdx.x < n ? a[threadIdx.x] : 0;
-  int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
   }
-  if (lane == 31) warp_sums[w] = x;
+  if (lane == 31) warp_sums[w] = v;
   __syncthreads();
   if (w == 0) {
     int s = warp_sums[lane];
@@ -64,10 +66,58 @@ __device__ __forceinline__ int block_scan_excl(int* a, int n, int* warp_sums) {
     warp_sums[lane] = s;
   }
   __syncthreads();
-  const int total = warp_sums[31];
-  if (threadIdx.x < n) a[threadIdx.x] = x - v + (w > 0 ? warp_sums[w - 1] : 0);
+  const int res = v + (w > 0 ? warp_sums[w - 1] : 0);
+  if (total) *total = warp_sums[31];
+  __syncthreads();
+  return res;
+}
+
+// Exclusive scan, in place, of n <= 1024 ints in shared memory; returns the total.
+__device__ __forceinline__ int block_scan_excl(int* a, int n, int* warp_sums) {
+  const int v = threadIdx.x < n ? a[threadIdx.x] : 0;
+  int total = 0;
+  const int incl = block_scan_incl(v, warp_sums, &total);
+  if (threadIdx.x < n) a[threadIdx.x] = incl - v;
   __syncthreads();
   return total;
+}
+
+// Finds, over the cluster's histograms h (nb bins, ascending digit order), the digit whose
+// bin holds the need-th largest key; writes it and the count of keys in higher bins.
+__device__ __forceinline__ void find_digit(const uint32_t* h, int nb, int need, cg::cluster_group& cluster, int C,
+                                           int rank, int* warp_sums, uint32_t* s_digit, int* s_above) {
+  const int bpt = nb >= NT ? nb / NT : 1;  // bins per thread, in descending order
+  const int first = threadIdx.x * bpt;
+  int cnt[4] = {0, 0, 0, 0};
+  if (first < nb) {
+    uint32_t part[8][4];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const uint32_t* rh = (r < C && r != rank) ? cluster.map_shared_rank(h, r) : h;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) part[r][e] = (r < C && e < bpt) ? rh[nb - 1 - (first + e)] : 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cnt[e] += (int)part[r][e];
+  }
+  const int local = cnt[0] + cnt[1] + cnt[2] + cnt[3];
+  const int incl = block_scan_incl(local, warp_sums, nullptr);
+  const int excl = incl - local;
+  if (first < nb && excl < need && need <= incl) {
+    int run = excl;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (e < bpt && run + cnt[e] >= need) {
+        *s_digit = (uint32_t)(nb - 1 - (first + e));
+        *s_above = run;
+        break;
+      }
+      run += cnt[e];
+    }
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -80,8 +130,9 @@ __global__ void __launch_bounds__(NT, 1)
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
 
   extern __shared__ uint32_t keys[];  // [R][NT]
-  __shared__ int wcnt[32][16];        // per-warp digit counts
-  __shared__ int cta_cnt[8][16];      // per-pass digit counts of this CTA (read by the cluster)
+  __shared__ uint32_t hist0[NB0];
+  __shared__ uint32_t hist1[NB1];
+  __shared__ uint32_t hist2[NB2];
   __shared__ int tab_a[32 * MAX_ROWS];
   __shared__ int tab_b[32 * MAX_ROWS];
   __shared__ int warp_sums[32];
@@ -100,92 +151,79 @@ __global__ void __launch_bounds__(NT, 1)
     return;
   }
 
-  // ---- load this CTA's slice once: element e = base + i * NT + tid, i < R
+  for (int e = tid; e < NB0; e += NT) hist0[e] = 0u;
+  for (int e = tid; e < NB1; e += NT) hist1[e] = 0u;
+  for (int e = tid; e < NB2; e += NT) hist2[e] = 0u;
+
+  // ---- load this CTA's slice once, 8 loads in flight per thread: element = base + i*NT + tid
   const int base = rank * (NT * R);
+  const int nvalid = sq.n_ctx - base - tid;  // key i of this thread exists iff i * NT < nvalid
   bool saw_nan = false;
-  for (int i = 0; i < R; ++i) {
-    const int idx = base + i * NT + tid;
-    uint32_t k = 0u;
-    if (idx < sq.n_ctx) {
-      k = order_key(__ldg(score + sq.start + idx));
-      saw_nan |= (k == 0u);
+#pragma unroll 1
+  for (int i0 = 0; i0 < R; i0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u;
+      v[u] = (i < R && i * NT < nvalid) ? __ldg(score + sq.start + base + i * NT + tid) : 0.f;
     }
-    keys[i * NT + tid] = k;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u;
+      if (i < R) {
+        const bool ok = i * NT < nvalid;
+        const uint32_t k = ok ? order_key(v[u]) : 0u;
+        saw_nan |= ok && k == 0u;
+        keys[i * NT + tid] = k;
+      }
+    }
   }
   if (saw_nan && dev_status) atomicOr(dev_status, TG_DEV_NAN_SCORE);
-  const int nvalid = sq.n_ctx - base - tid;  // key i of this thread exists iff i * NT < nvalid
   __syncthreads();
 
-  // ---- radix select, 4-bit digits, most significant first
-  uint32_t prefix = 0u, pmask = 0u;
-  int need = sq.kc;
-#pragma unroll 1
-  for (int pass = 0; pass < 8; ++pass) {
-    const int shift = 28 - 4 * pass;
-    uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;  // 16 packed 8-bit counters (<= 32 keys each)
-    for (int i = 0; i < R; ++i) {
-      if (i * NT >= nvalid) break;
-      const uint32_t k = keys[i * NT + tid];
-      if ((k & pmask) == prefix) {
-        const uint32_t d = (k >> shift) & 15u;
-        const uint32_t inc = 1u << ((d & 3u) * 8u);
-        const uint32_t q = d >> 2;
-        c0 += q == 0 ? inc : 0u;
-        c1 += q == 1 ? inc : 0u;
-        c2 += q == 2 ? inc : 0u;
-        c3 += q == 3 ? inc : 0u;
-      }
+  // ---- pass 0: sign + exponent, lanes with equal bins merged before the atomic
+  for (int i = 0; i < R; ++i) {
+    const bool ok = i * NT < nvalid;
+    const uint32_t act = __ballot_sync(0xffffffffu, ok);
+    if (ok) {
+      const uint32_t d = keys[i * NT + tid] >> 23;
+      const uint32_t grp = __match_any_sync(act, d);
+      if (lane == __ffs(grp) - 1) atomicAdd(&hist0[d], (uint32_t)__popc(grp));
     }
-    int mine = 0;  // lane d (< 16) keeps the warp's count of digit d
-#pragma unroll
-    for (int d = 0; d < 16; ++d) {
-      const uint32_t word = d < 4 ? c0 : (d < 8 ? c1 : (d < 12 ? c2 : c3));
-      const int v = (int)((word >> ((d & 3) * 8)) & 0xffu);
-      const int sum = (int)__reduce_add_sync(0xffffffffu, (unsigned)v);
-      if (lane == d) mine = sum;
-    }
-    if (lane < 16) wcnt[w][lane] = mine;
-    __syncthreads();
-    if (w == 0 && lane < 16) {
-      int tot = 0;
-#pragma unroll 8
-      for (int x = 0; x < 32; ++x) tot += wcnt[x][lane];
-      cta_cnt[pass][lane] = tot;
-    }
-    if (C > 1) cluster.sync();
-    else __syncthreads();
-    if (w == 0) {
-      // lane l holds the cluster-wide count of digit 15 - l (descending order)
-      int c = 0;
-      if (lane < 16) {
-        int part[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-          part[r] = r < C ? (r == rank ? cta_cnt[pass][15 - lane]
-                                       : cluster.map_shared_rank(&cta_cnt[pass][0], r)[15 - lane])
-                          : 0;
-#pragma unroll
-        for (int r = 0; r < 8; ++r) c += part[r];
-      }
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 16; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const int excl = incl - c;
-      if (lane < 16 && excl < need && need <= incl) {
-        s_digit = (uint32_t)(15 - lane);
-        s_above = excl;
-      }
-    }
-    __syncthreads();
-    prefix |= s_digit << shift;
-    pmask |= 15u << shift;
-    need -= s_above;
-    __syncthreads();
   }
-  const uint32_t T = prefix;  // the K-th largest key; `need` keys equal to T are kept
+  if (C > 1) cluster.sync();
+  else __syncthreads();
+  int need = sq.kc;
+  find_digit(hist0, NB0, need, cluster, C, rank, warp_sums, &s_digit, &s_above);
+  const uint32_t d0 = s_digit;
+  need -= s_above;
+  __syncthreads();
+
+  // ---- pass 1: the next 11 bits of keys in bin d0
+  for (int i = 0; i < R; ++i) {
+    if (i * NT >= nvalid) break;
+    const uint32_t k = keys[i * NT + tid];
+    if ((k >> 23) == d0) atomicAdd(&hist1[(k >> 12) & (NB1 - 1)], 1u);
+  }
+  if (C > 1) cluster.sync();
+  else __syncthreads();
+  find_digit(hist1, NB1, need, cluster, C, rank, warp_sums, &s_digit, &s_above);
+  const uint32_t p1 = (d0 << 11) | s_digit;  // key >> 12
+  need -= s_above;
+  __syncthreads();
+
+  // ---- pass 2: the last 12 bits
+  for (int i = 0; i < R; ++i) {
+    if (i * NT >= nvalid) break;
+    const uint32_t k = keys[i * NT + tid];
+    if ((k >> 12) == p1) atomicAdd(&hist2[k & (NB2 - 1)], 1u);
+  }
+  if (C > 1) cluster.sync();
+  else __syncthreads();
+  find_digit(hist2, NB2, need, cluster, C, rank, warp_sums, &s_digit, &s_above);
+  const uint32_t T = (p1 << 12) | s_digit;  // the K-th largest key; `need` keys equal to T are kept
+  need -= s_above;
+  __syncthreads();
 
   // ---- compaction in index order: per (row i, warp) counts, element = base + i*NT + w*32 + lane
   const uint32_t lt = (1u << lane) - 1u;
@@ -245,7 +283,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
   }
   if (overflow && dev_status) atomicOr(dev_status, TG_DEV_BAD_INDEX);
-  if (C > 1) cluster.sync();  // no CTA leaves while a peer may still read its counters
+  if (C > 1) cluster.sync();  // no CTA leaves while a peer may still read its shared memory
 }
 
 }  // namespace
