@@ -11,8 +11,9 @@
 // are split into two interleaved chains (even and odd tiles), each with its own softmax
 // warpgroup, TMEM score buffer and TMEM output accumulator, so one group's exponentials
 // overlap the other group's matrix products:
-//   * warp 0: TMA loads Q once and K_j, V_j (128 keys) into the stage of chain j % 2, and
-//     stages the tile's per-key bias gain*log2(e)*log g_j in shared memory.
+//   * warp 0: TMA loads Q once and K_j (128 keys) into a 3-deep ring, so the next products
+//     QK^T never wait on L2; warp 10 loads V_j into the stage of chain j % 2 and stages the
+//     tile's per-key bias gain*log2(e)*log g_j in shared memory.
 //   * warp 1 (one thread): tcgen05.mma. S_j = Q K_j^T (M=128, N=128, K=D) into the chain's
 //     TMEM S buffer; O_c += P_j V_j with P_j read from TMEM (A operand in tensor memory) and
 //     V_j from shared memory (N-contiguous operand).
@@ -36,7 +37,8 @@ using namespace sm100;
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 352;  // warp 0: Q/K loads, 1: MMA, 2-9: softmax, 10: V loads + bias
+constexpr int KS = 3;           // K ring depth
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleSlack = 8.f;  // log2 units the running max may lag behind
@@ -54,9 +56,9 @@ struct ACfg {
   static constexpr int TILE_BYTES = BQ * D * 2;  // one 128 x D bf16 tile
   static constexpr int NBOX = D / 64;            // 64-column boxes per tile
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = TILE_BYTES;  // + stage * 2 * TILE_BYTES
-  static constexpr int V_OFF = 2 * TILE_BYTES;
-  static constexpr int TAIL_OFF = TILE_BYTES * 5;
+  static constexpr int K_OFF = TILE_BYTES;               // KS stages
+  static constexpr int V_OFF = TILE_BYTES * (1 + KS);    // 2 stages (one per chain)
+  static constexpr int TAIL_OFF = TILE_BYTES * (3 + KS);
   static constexpr int TAIL = 4096;
   static constexpr int SMEM = 1024 + TAIL_OFF + TAIL;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BQ, BKV, false);
@@ -82,16 +84,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* tail = smem + C::TAIL_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   uint64_t* qfull = bars + 0;
-  uint64_t* kfull = bars + 1;    // [2] per chain/stage
-  uint64_t* vfull = bars + 3;    // [2]
-  uint64_t* empty = bars + 5;    // [2]
-  uint64_t* bfull = bars + 7;    // [2]
-  uint64_t* sfull = bars + 9;    // [2]
-  uint64_t* pready = bars + 11;  // [2]
-  uint64_t* pvdone = bars + 13;  // [2]
-  uint64_t* mlready = bars + 15;
-  uint64_t* drain = bars + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* kfull = bars + 1;    // [KS]
+  uint64_t* kempty = bars + 4;   // [KS]
+  uint64_t* vfull = bars + 7;    // [2] per chain
+  uint64_t* vempty = bars + 9;   // [2]
+  uint64_t* bfull = bars + 11;   // [2]
+  uint64_t* sfull = bars + 13;   // [2]
+  uint64_t* pready = bars + 15;  // [2]
+  uint64_t* pvdone = bars + 17;  // [2]
+  uint64_t* mlready = bars + 19;
+  uint64_t* drain = bars + 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* bias_s = reinterpret_cast<float*>(tail + 256);  // [2][128]
   float* gmul_s = bias_s + 2 * BKV;                      // [2][128]
@@ -128,10 +131,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(&kfull[s], 1);
+      mbar_init(&kempty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&vfull[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&vempty[s], 1);
       mbar_init(&bfull[s], 32);
       mbar_init(&sfull[s], 1);
       mbar_init(&pready[s], 128);
@@ -156,31 +162,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {  // ---------------------------------------------------- TMA producer warp
-    int issued = 0;
+  if (warp == 0) {  // ------------------------------------------------- Q and K producer
     if (lane == 0) {
       mbar_arrive_expect_tx(qfull, C::TILE_BYTES);
       for (int bx = 0; bx < C::NBOX; ++bx)
         tma_load_2d(smem + C::Q_OFF + bx * (BQ * 128), &tmQ, h * D + bx * 64, off + t * BQ, qfull);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % KS;
+        if (!mbar_wait(&kempty[s], ((j / KS) & 1) ^ 1u, abort, dev_status)) break;
+        uint8_t* kb = smem + C::K_OFF + s * C::TILE_BYTES;
+        mbar_arrive_expect_tx(&kfull[s], C::TILE_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_2d(kb + bx * (BKV * 128), &tmK, kvh * D + bx * 64, off + j * BKV, &kfull[s]);
+        ++issued;
+      }
+      if (*abort) {  // let the copies in flight land before the CTA can leave
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(qfull, 0) && globaltimer_ns() - t0 < 1000000000ull) {
+        }
+        for (int j = issued - KS < 0 ? 0 : issued - KS; j < issued; ++j) {
+          const uint64_t t1 = globaltimer_ns();
+          while (!mbar_try_wait(&kfull[j % KS], (j / KS) & 1) && globaltimer_ns() - t1 < 1000000000ull) {
+          }
+        }
+      }
     }
+  } else if (warp == 10) {  // ---------------------------------------- V producer + key bias
+    int issued = 0;
     for (int j = 0; j < nt; ++j) {
       const int c = j & 1, u = j >> 1;
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(&empty[c], (u & 1) ^ 1u, abort, dev_status);
+      if (lane == 0) ok = mbar_wait(&vempty[c], (u & 1) ^ 1u, abort, dev_status);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       if (lane == 0) {
-        uint8_t* kb = smem + C::K_OFF + c * 2 * C::TILE_BYTES;
-        uint8_t* vb = smem + C::V_OFF + c * 2 * C::TILE_BYTES;
-        mbar_arrive_expect_tx(&kfull[c], C::TILE_BYTES);
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_2d(kb + bx * (BKV * 128), &tmK, kvh * D + bx * 64, off + j * BKV, &kfull[c]);
+        uint8_t* vb = smem + C::V_OFF + c * C::TILE_BYTES;
         mbar_arrive_expect_tx(&vfull[c], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_2d(vb + bx * (BKV * 128), &tmV, kvh * D + bx * 64, off + j * BKV, &vfull[c]);
       }
       ++issued;
-      // per-key bias of this key tile (log2 domain), 4 keys per lane; the slot is free
-      // because the PV product of the chain's previous tile has completed (empty barrier)
+      // per-key bias of this key tile (log2 domain), 4 keys per lane; the chain's slot is
+      // free because the PV product of its previous tile has completed (vempty above)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int col = lane * 4 + e;
@@ -191,15 +214,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       mbar_arrive(&bfull[c]);
     }
-    if (lane == 0 && *abort) {  // let the copies in flight land before the CTA can leave
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(qfull, 0) && globaltimer_ns() - t0 < 1000000000ull) {
-      }
+    if (lane == 0 && *abort) {
       for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
-        const uint32_t ph = (j >> 1) & 1;
         const uint64_t t1 = globaltimer_ns();
-        while (!(mbar_try_wait(&kfull[j & 1], ph) && mbar_try_wait(&vfull[j & 1], ph)) &&
-               globaltimer_ns() - t1 < 1000000000ull) {
+        while (!mbar_try_wait(&vfull[j & 1], (j >> 1) & 1) && globaltimer_ns() - t1 < 1000000000ull) {
         }
       }
     }
@@ -207,18 +225,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       const uint32_t qa = smem_u32(smem + C::Q_OFF);
       auto issue_s = [&](int j) -> bool {
-        const int c = j & 1, u = j >> 1;
-        if (!mbar_wait(&kfull[c], u & 1, abort, dev_status)) return false;
+        const int c = j & 1, u = j >> 1, ks = j % KS;
+        if (!mbar_wait(&kfull[ks], (j / KS) & 1, abort, dev_status)) return false;
         // the chain's S buffer still holds P of its previous tile until that PV completes
         if (u > 0 && !mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status)) return false;
         tc_fence_after();
-        const uint32_t ka = smem_u32(smem + C::K_OFF + c * 2 * C::TILE_BYTES);
+        const uint32_t ka = smem_u32(smem + C::K_OFF + ks * C::TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
           mma_ss(tmem + c * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK, kk > 0);
         }
         mma_commit(&sfull[c]);
+        mma_commit(&kempty[ks]);
         return true;
       };
       bool ok = mbar_wait(qfull, 0, abort, dev_status);
@@ -228,13 +247,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&pready[c], u & 1, abort, dev_status) || !mbar_wait(&vfull[c], u & 1, abort, dev_status))
           break;
         tc_fence_after();
-        const uint32_t va = smem_u32(smem + C::V_OFF + c * 2 * C::TILE_BYTES);
+        const uint32_t va = smem_u32(smem + C::V_OFF + c * C::TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)
           mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
                  C::IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&pvdone[c]);
-        mma_commit(&empty[c]);
+        mma_commit(&vempty[c]);
         if (j + 2 < nt) ok = issue_s(j + 2);
       }
       mma_commit(drain);

@@ -6,7 +6,8 @@
 // Design (B200, bf16 in, fp32 accumulate). The whole hidden width dg (<= 256) is one UMMA N,
 // so the [n_tok, dg] activation lives only in TMEM and H is read from HBM exactly once.
 // W1 (dg x d) is re-read from L2 by every CTA, so each CTA multiplies one W1 slice into TWO
-// 128-token tiles (a 256-token pair) to halve the W1 bytes per flop:
+// 128-token tiles (a 256-token pair) to halve the W1 bytes per flop, and each CTA starts its
+// K loop at a different slice so the CTAs do not all hit the same L2 lines at once:
 //   * warp 0 (one thread): TMA loads, per 64-wide K slice, H rows of both tiles and the W1
 //     slice into a ring of shared-memory stages (128-byte swizzle).
 //   * warp 1 (one thread): tcgen05.mma M=128, N=dg, K=16 for both tiles into two fp32 TMEM
@@ -63,6 +64,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float* part = w2s + DG;  // [2][BM] partial sums of the upper column half
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kb0 = (int)(((long)blockIdx.x * nk) / gridDim.x);  // first K slice of this CTA
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -101,7 +103,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t phase = 0;
       long issued = 0;
       for (int pr = blockIdx.x; pr < n_pairs && !*abort; pr += gridDim.x) {
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int i = 0; i < nk; ++i) {
+          const int kb = (i + kb0) % nk;  // CTAs start at different W1 slices (spreads L2 hot spots)
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, dev_status)) break;
           uint8_t* st = smem + stage * C::STAGE;
           mbar_arrive_expect_tx(&full[stage], C::STAGE);
@@ -134,7 +137,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(acce, (it & 1) ^ 1u, abort, dev_status)) break;
         tc_fence_after();
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int i = 0; i < nk; ++i) {
           if (!mbar_wait(&full[stage], phase, abort, dev_status)) {
             ok = false;
             break;
@@ -146,8 +149,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t bd = sdesc_sw128(b0 + 32 * k, 16, 1024);
-            mma_ss(tmem, sdesc_sw128(a0 + 32 * k, 16, 1024), bd, C::IDESC, (kb | k) != 0);
-            mma_ss(tmem + DG, sdesc_sw128(a1 + 32 * k, 16, 1024), bd, C::IDESC, (kb | k) != 0);
+            mma_ss(tmem, sdesc_sw128(a0 + 32 * k, 16, 1024), bd, C::IDESC, (i | k) != 0);
+            mma_ss(tmem + DG, sdesc_sw128(a1 + 32 * k, 16, 1024), bd, C::IDESC, (i | k) != 0);
           }
           mma_commit(&empty[stage]);
           if (++stage == C::STAGES) {

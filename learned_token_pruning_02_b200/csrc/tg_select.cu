@@ -4,8 +4,8 @@
 // highest gate score, and only the document part of the prompt may be pruned. TokenGate
 // paper page (thelatestinai.com), Figure 1(a)-(b).
 //
-// Design (B200): one CTA of 1024 threads per sequence while its context fits in shared
-// memory (32768 keys = 128 KB), otherwise one thread-block cluster of up to 8 CTAs. The
+// Design (B200): one thread-block cluster of up to 8 CTAs (1024 threads each, about 4096
+// keys per CTA, at most 32768) per sequence. The
 // scores are read from HBM exactly once (loads batched 8 deep per thread) into
 // order-preserving 32-bit keys in shared memory. An MSB-first radix select in three passes
 // finds the K-th largest key T:
@@ -293,9 +293,12 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
   SelParams p = {};
   for (int i = 0; i < nseq; ++i) p.s[i] = seqs[i];
   const int per_cta = NT * MAX_ROWS;
-  int C = (n_ctx_max + per_cta - 1) / per_cta;
-  if (C < 1) C = 1;
-  if (C > 8) return fail(TG_ERR_UNSUPPORTED, "context of %d tokens exceeds the select capacity", n_ctx_max);
+  // about 4096 keys per CTA (up to 8 CTAs): the passes are instruction-bound, so a sequence
+  // is spread over several SMs rather than one
+  int C = (n_ctx_max + 4 * NT - 1) / (4 * NT);
+  C = C < 1 ? 1 : (C > 8 ? 8 : C);
+  if ((int64_t)C * per_cta < n_ctx_max)
+    return fail(TG_ERR_UNSUPPORTED, "context of %d tokens exceeds the select capacity", n_ctx_max);
   int rows = (n_ctx_max + NT * C - 1) / (NT * C);
   if (rows < 1) rows = 1;
   p.C = C;
