@@ -301,21 +301,26 @@ def main():
     flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream()
 
+    out = {"score": score, "kept_idx": kept, "cu_kept_dev": cu_dev, "H_kept": Hk, "pos": pos, "g": g,
+           "logg": logg, "O": Os, "lse": [None] * len(layers)}
+    chain = tg.PreparedChain(H, W1, b1, w2, b2, wl.seqlens, wl.q_len, wl.k, layers, scale, out, dev_status=status,
+                             stream=stream)
+
     def step(ev=None):
+        # the same four C-ABI calls tg_prefill_above_L makes, with events between them
         if ev:
             ev[0].record(stream)
-        tg.tg_score(H, W1, b1, w2, b2, score=score)
+        chain.score()
         if ev:
             ev[1].record(stream)
-        tg.tg_topk_select(score, wl.seqlens, wl.q_len, wl.k, kept_idx=kept, cu_kept_dev=cu_dev, dev_status=status)
+        chain.select()
         if ev:
             ev[2].record(stream)
-        tg.tg_gather(H, score, kept, wl.seqlens, wl.q_len, wl.k, H_kept=Hk, pos=pos, g=g, logg=logg,
-                     dev_status=status)
+        chain.gather()
         if ev:
             ev[3].record(stream)
-        for li, (q, k, v) in enumerate(layers):
-            tg.tg_gated_attn_fwd(q, k, v, logg, pos, cu, scale, O=Os[li], want_lse=False, dev_status=status)
+        for li in range(len(layers)):
+            chain.attention(li)
         if ev:
             ev[4].record(stream)
 
@@ -332,7 +337,7 @@ def main():
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.zero_()  # L2 flush, outside the timed events
-        torch.cuda._sleep(300_000)  # lets the host queue the step's launches ahead of the GPU
+        torch.cuda._sleep(200_000)  # keeps the host's launches ahead of the GPU (no idle gaps timed)
         step(evs[i])
     torch.cuda.synchronize()
     barrier()
@@ -381,9 +386,6 @@ def main():
     if args.e2e_steps > 0:
         O_host = [torch.empty(L[0].shape, dtype=torch.bfloat16).pin_memory() for L in layers]
         kept_host = torch.empty(M, dtype=torch.int32).pin_memory()
-        out = {"score": score, "kept_idx": kept, "cu_kept_dev": cu_dev, "H_kept": Hk, "pos": pos, "g": g,
-               "logg": logg, "O": Os, "lse": [None] * len(layers)}
-
         def e2e_step():
             H.copy_(H_host, non_blocking=True)
             for (q, k, v), (qh, kh, vh) in zip(layers, qkv_host):

@@ -17,9 +17,10 @@
 //   * warp 1 (one thread): tcgen05.mma. S_j = Q K_j^T (M=128, N=128, K=D) into the chain's
 //     TMEM S buffer; O_c += P_j V_j with P_j read from TMEM (A operand in tensor memory) and
 //     V_j from shared memory (N-contiguous operand).
-//   * warps 2-5 (chain 0) and 6-9 (chain 1): one query row per thread. Pass 1 reads S and
-//     finds the row max of scale*log2(e)*S + bias (causal mask on the diagonal tile);
-//     pass 2 writes P = 2^(x - m) as packed bf16 into the same TMEM columns. The running
+//   * warps 2-5 (chain 0) and 6-9 (chain 1): one query row per thread. The thread loads its
+//     whole S row from TMEM into registers, forms scale*log2(e)*S + bias (causal mask on the
+//     diagonal tile only), and writes P = 2^(x - m) back as packed bf16 into the same TMEM
+//     columns. The running
 //     max is only moved (and O rescaled in TMEM) when it grows by more than 8 (a factor
 //     256), which keeps every P <= 256 and the result exact after normalisation.
 //   * Chain 0's warps merge the two chains (max, sum, O) and write O (bf16) and the LSE.
@@ -224,37 +225,55 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {  // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t qa = smem_u32(smem + C::Q_OFF);
-      auto issue_s = [&](int j) -> bool {
-        const int c = j & 1, u = j >> 1, ks = j % KS;
-        if (!mbar_wait(&kfull[ks], (j / KS) & 1, abort, dev_status)) return false;
-        // the chain's S buffer still holds P of its previous tile until that PV completes
-        if (u > 0 && !mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status)) return false;
-        tc_fence_after();
-        const uint32_t ka = smem_u32(smem + C::K_OFF + ks * C::TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          mma_ss(tmem + c * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK, kk > 0);
-        }
-        mma_commit(&sfull[c]);
-        mma_commit(&kempty[ks]);
-        return true;
-      };
+      // Event loop: issue whichever product is ready, never blocking on one barrier while the
+      // other product could go. S_j needs K_j and the chain's S buffer (free once PV of the
+      // chain's previous tile completed); PV_j needs P_j and V_j. At most two S ahead of PV.
       bool ok = mbar_wait(qfull, 0, abort, dev_status);
-      for (int j = 0; ok && j < 2 && j < nt; ++j) ok = issue_s(j);
-      for (int j = 0; ok && j < nt; ++j) {
-        const int c = j & 1, u = j >> 1;
-        if (!mbar_wait(&pready[c], u & 1, abort, dev_status) || !mbar_wait(&vfull[c], u & 1, abort, dev_status))
-          break;
-        tc_fence_after();
-        const uint32_t va = smem_u32(smem + C::V_OFF + c * C::TILE_BYTES);
+      int next_s = 0, next_pv = 0;
+      uint64_t t_idle = globaltimer_ns();
+      while (ok && next_pv < nt) {
+        bool progressed = false;
+        if (next_pv < next_s) {
+          const int j = next_pv, c = j & 1, u = j >> 1;
+          if (mbar_try_wait(&pready[c], u & 1) && mbar_try_wait(&vfull[c], u & 1)) {
+            tc_fence_after();
+            const uint32_t va = smem_u32(smem + C::V_OFF + c * C::TILE_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)
-          mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
-                 C::IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&pvdone[c]);
-        mma_commit(&vempty[c]);
-        if (j + 2 < nt) ok = issue_s(j + 2);
+            for (int kk = 0; kk < BKV / 16; ++kk)
+              mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
+                     C::IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&pvdone[c]);
+            mma_commit(&vempty[c]);
+            ++next_pv;
+            progressed = true;
+          }
+        }
+        if (next_s < nt && next_s < next_pv + 2) {
+          const int j = next_s, c = j & 1, u = j >> 1, ks = j % KS;
+          if (mbar_try_wait(&kfull[ks], (j / KS) & 1) && (u == 0 || mbar_try_wait(&pvdone[c], (u - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t ka = smem_u32(smem + C::K_OFF + ks * C::TILE_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+              mma_ss(tmem + c * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK,
+                     kk > 0);
+            }
+            mma_commit(&sfull[c]);
+            mma_commit(&kempty[ks]);
+            ++next_s;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t_idle = globaltimer_ns();
+        } else if (*abort) {
+          ok = false;
+        } else if (globaltimer_ns() - t_idle > 2000000000ull) {
+          *abort = 1;
+          if (dev_status) atomicOr(dev_status, TG_DEV_TIMEOUT);
+          ok = false;
+        }
       }
       mma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
@@ -284,20 +303,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
-      const float* bs = bias_s + c * BKV;
-      const bool diag = (j == t);
-      // pass 1: row max of the biased log2-domain logits
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int ch = 0; ch < BKV / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tS + ch * 32, v);
-        tmem_wait_ld();
+      uint32_t sr[BKV];  // the whole S row of this thread, then P
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = ch * 32 + e;
-          const float x = fmaf(__uint_as_float(v[e]), qk_scale, bs[col]);
-          mx = fmaxf(mx, (diag && col > r) ? -INFINITY : x);
+      for (int ch = 0; ch < BKV / 32; ++ch)
+        tmem_ld32(tS + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
+      tmem_wait_ld();
+      const float4* bs4 = reinterpret_cast<const float4*>(bias_s + c * BKV);
+      float mx = -INFINITY;
+      if (j == t) {  // diagonal tile: causal mask (key column > query row)
+#pragma unroll
+        for (int q = 0; q < BKV / 4; ++q) {
+          const float4 bb = bs4[q];
+          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 4 * q + e;
+            const float x = col > r ? -INFINITY : fmaf(__uint_as_float(sr[col]), qk_scale, bv[e]);
+            sr[col] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < BKV / 4; ++q) {
+          const float4 bb = bs4[q];
+          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 4 * q + e;
+            const float x = fmaf(__uint_as_float(sr[col]), qk_scale, bv[e]);
+            sr[col] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
         }
       }
       const float m_cand = fmaxf(m_run, mx);
@@ -324,28 +361,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         m_run = m_cand;
       }
       const float mb = m_run == -INFINITY ? 0.f : m_run;
-      const float* gm = gmul_s + c * BKV;
-      // pass 2: P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns
+      // P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns
       float sum = 0.f;
-#pragma unroll 1
-      for (int ch = 0; ch < BKV / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tS + ch * 32, v);
-        tmem_wait_ld();
-        uint32_t pk[16];
+      uint32_t pk[BKV / 2];
+      if (unnorm) {
+        const float4* gm4 = reinterpret_cast<const float4*>(gmul_s + c * BKV);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int col = ch * 32 + e;
-          float x0 = fmaf(__uint_as_float(v[e]), qk_scale, bs[col]);
-          float x1 = fmaf(__uint_as_float(v[e + 1]), qk_scale, bs[col + 1]);
-          if (diag && col > r) x0 = -INFINITY;
-          if (diag && col + 1 > r) x1 = -INFINITY;
-          const float p0 = ex2(x0 - mb), p1 = ex2(x1 - mb);
-          sum += p0 + p1;
-          pk[e >> 1] = unnorm ? pack_bf16(p0 * gm[col], p1 * gm[col + 1]) : pack_bf16(p0, p1);
+        for (int q = 0; q < BKV / 4; ++q) {
+          const float4 gg = gm4[q];
+          const float p0 = ex2(__uint_as_float(sr[4 * q]) - mb), p1 = ex2(__uint_as_float(sr[4 * q + 1]) - mb);
+          const float p2 = ex2(__uint_as_float(sr[4 * q + 2]) - mb), p3 = ex2(__uint_as_float(sr[4 * q + 3]) - mb);
+          sum += (p0 + p1) + (p2 + p3);
+          pk[2 * q] = pack_bf16(p0 * gg.x, p1 * gg.y);
+          pk[2 * q + 1] = pack_bf16(p2 * gg.z, p3 * gg.w);
         }
-        tmem_st16(tS + ch * 16, pk);
+      } else {
+#pragma unroll
+        for (int e = 0; e < BKV; e += 2) {
+          const float p0 = ex2(__uint_as_float(sr[e]) - mb), p1 = ex2(__uint_as_float(sr[e + 1]) - mb);
+          sum += p0 + p1;
+          pk[e >> 1] = pack_bf16(p0, p1);
+        }
       }
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       l_run += sum;
       tc_fence_before();
