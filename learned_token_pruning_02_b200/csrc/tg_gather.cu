@@ -19,7 +19,7 @@ struct GatherParams {
   int nseq;
 };
 
-constexpr int WARPS = 8;
+constexpr int WARPS = 4;
 constexpr int MAXV = 8;  // 16-byte vectors per lane held in registers per pass
 
 __global__ void __launch_bounds__(WARPS * 32)
@@ -39,25 +39,26 @@ __global__ void __launch_bounds__(WARPS * 32)
       if (lane == 0 && dev_status) atomicOr(dev_status, TG_DEV_BAD_INDEX);
       continue;
     }
+    // the score load goes out together with the row loads (one round trip, not two)
+    const float s = (lane == 0 && (g || logg)) ? __ldg(score + j) : 0.f;
     const uint4* src = H + (int64_t)j * ldv;
     uint4* dst = Hk + (int64_t)row * nvec;
     for (int v0 = 0; v0 < nvec; v0 += 32 * MAXV) {
       uint4 buf[MAXV];
 #pragma unroll
       for (int u = 0; u < MAXV; ++u) {
-        int v = v0 + u * 32 + lane;
+        const int v = v0 + u * 32 + lane;
         if (v < nvec) buf[u] = __ldcs(src + v);
       }
 #pragma unroll
       for (int u = 0; u < MAXV; ++u) {
-        int v = v0 + u * 32 + lane;
+        const int v = v0 + u * 32 + lane;
         if (v < nvec) __stcs(dst + v, buf[u]);
       }
     }
     if (lane == 0) {
       pos[row] = j - sq.start;
       if (g || logg) {
-        const float s = __ldg(score + j);
         float gv, lg;
         if ((flags & TG_QUESTION_GATE_ONE) && (row - sq.out_off) >= sq.m - sq.q) {
           gv = 1.f;
@@ -86,7 +87,7 @@ tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const fl
   const int nvec = d * es / 16;
   const int64_t ldv = ldh * es / 16;
   int blocks = (m_chunk + WARPS - 1) / WARPS;
-  const int cap = device_sm_count() * 8;
+  const int cap = device_sm_count() * 16;
   if (blocks > cap) blocks = cap;
   gather_kernel<<<blocks, WARPS * 32, 0, st>>>(static_cast<const uint4*>(H), ldv, nvec, score, kept_idx, flags,
                                                static_cast<uint4*>(H_kept), pos, g, logg, dev_status, m_chunk, p);

@@ -4,19 +4,17 @@
 // highest gate score, and only the document part of the prompt may be pruned. TokenGate
 // paper page (thelatestinai.com), Figure 1(a)-(b).
 //
-// Design (B200): one thread-block cluster of up to 8 CTAs (1024 threads each, about 4096
-// keys per CTA, at most 32768) per sequence. The
-// scores are read from HBM exactly once (loads batched 8 deep per thread) into
-// order-preserving 32-bit keys in shared memory. An MSB-first radix select in three passes
-// finds the K-th largest key T:
-//   pass 0: sign + exponent (9 bits, 512 bins). Scores crowd into a few exponents, so
-//           lanes with the same bin are merged with match.any before one shared atomic;
-//   pass 1: the next 11 bits (2048 bins) of the keys in the chosen bin - nearly uniform;
-//   pass 2: the last 12 bits (4096 bins) of the few keys left.
-// In a cluster every CTA sums the cluster's histograms over distributed shared memory after
-// a hardware cluster barrier and scans them itself. Keys > T are kept, and keys == T in
-// index order until K is reached (lower index wins ties). An ascending compaction uses warp
-// ballots and block-wide scans. No workspace: the per-sequence descriptors travel as kernel
+// Design (B200): one thread-block cluster of 1-8 CTAs (1024 threads each, up to 8192 keys
+// per CTA below 64K keys, at most 32768) per sequence. The scores are read from HBM exactly
+// once (loads batched 8 deep per thread) into order-preserving 32-bit keys in shared
+// memory. An MSB-first radix select with 8-bit digits (4 passes, 256 bins) finds the K-th
+// largest key T. Pass 0 (sign + 7 exponent bits) sees scores crowded into a few bins, so
+// lanes with the same bin are merged with match.any before one shared atomic; later passes
+// only count keys that still match the prefix. After a hardware cluster barrier 64 threads
+// of every CTA sum the cluster's 256-bin histograms with 16-byte distributed-shared-memory
+// loads and pick the digit. Keys > T are kept, and keys == T in index order until K is
+// reached (lower index wins ties). An ascending compaction uses warp ballots and
+// block-wide scans. No workspace: the per-sequence descriptors travel as kernel
 // parameters; nothing spins.
 #include <cooperative_groups.h>
 
@@ -29,7 +27,7 @@ namespace {
 
 constexpr int NT = 1024;
 constexpr int MAX_ROWS = 32;  // keys per thread: 32 x 1024 = 32768 keys per CTA
-constexpr int NB0 = 512, NB1 = 2048, NB2 = 4096;
+constexpr int NB = 256;  // bins per pass (8-bit digits)
 
 struct SelParams {
   SelSeq s[kMaxSeqPerLaunch];
@@ -82,35 +80,50 @@ __device__ __forceinline__ int block_scan_excl(int* a, int n, int* warp_sums) {
   return total;
 }
 
-// Finds, over the cluster's histograms h (nb bins, ascending digit order), the digit whose
+// Finds, over the cluster's 256-bin histograms h (ascending digit order), the digit whose
 // bin holds the need-th largest key; writes it and the count of keys in higher bins.
-__device__ __forceinline__ void find_digit(const uint32_t* h, int nb, int need, cg::cluster_group& cluster, int C,
-                                           int rank, int* warp_sums, uint32_t* s_digit, int* s_above) {
-  const int bpt = nb >= NT ? nb / NT : 1;  // bins per thread, in descending order
-  const int first = threadIdx.x * bpt;
+// Threads 0..63 each own 4 bins (descending) and read them from every CTA with one 16-byte
+// load per CTA.
+__device__ __forceinline__ void find_digit(const uint32_t* h, int need, cg::cluster_group& cluster, int C, int rank,
+                                           int* warp_sums, uint32_t* s_digit, int* s_above) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   int cnt[4] = {0, 0, 0, 0};
-  if (first < nb) {
-    uint32_t part[8][4];
+  if (tid < NB / 4) {
+    const int lo = NB - 4 * (tid + 1);  // bins lo..lo+3; this thread's order is lo+3, lo+2, lo+1, lo
+    uint4 part[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const uint32_t* rh = (r < C && r != rank) ? cluster.map_shared_rank(h, r) : h;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) part[r][e] = (r < C && e < bpt) ? rh[nb - 1 - (first + e)] : 0u;
+      part[r] = r < C ? *reinterpret_cast<const uint4*>(rh + lo) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) cnt[e] += (int)part[r][e];
+    for (int r = 0; r < 8; ++r) {
+      cnt[0] += (int)part[r].w;
+      cnt[1] += (int)part[r].z;
+      cnt[2] += (int)part[r].y;
+      cnt[3] += (int)part[r].x;
+    }
   }
+  // inclusive scan over threads 0..63 (two warps) of their 4-bin totals
   const int local = cnt[0] + cnt[1] + cnt[2] + cnt[3];
-  const int incl = block_scan_incl(local, warp_sums, nullptr);
+  int incl = local;
+  if (w < 2) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[w] = incl;
+  }
+  __syncthreads();
+  if (w == 1) incl += warp_sums[0];
   const int excl = incl - local;
-  if (first < nb && excl < need && need <= incl) {
+  if (tid < NB / 4 && excl < need && need <= incl) {
     int run = excl;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if (e < bpt && run + cnt[e] >= need) {
-        *s_digit = (uint32_t)(nb - 1 - (first + e));
+      if (run + cnt[e] >= need) {
+        *s_digit = (uint32_t)(NB - 1 - (4 * tid + e));
         *s_above = run;
         break;
       }
@@ -130,9 +143,7 @@ __global__ void __launch_bounds__(NT, 1)
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
 
   extern __shared__ uint32_t keys[];  // [R][NT]
-  __shared__ uint32_t hist0[NB0];
-  __shared__ uint32_t hist1[NB1];
-  __shared__ uint32_t hist2[NB2];
+  __shared__ __align__(16) uint32_t hist[4][NB];  // one per pass (read by the cluster)
   __shared__ int tab_a[32 * MAX_ROWS];
   __shared__ int tab_b[32 * MAX_ROWS];
   __shared__ int warp_sums[32];
@@ -151,9 +162,7 @@ __global__ void __launch_bounds__(NT, 1)
     return;
   }
 
-  for (int e = tid; e < NB0; e += NT) hist0[e] = 0u;
-  for (int e = tid; e < NB1; e += NT) hist1[e] = 0u;
-  for (int e = tid; e < NB2; e += NT) hist2[e] = 0u;
+  for (int e = tid; e < 4 * NB; e += NT) (&hist[0][0])[e] = 0u;
 
   // ---- load this CTA's slice once, 8 loads in flight per thread: element = base + i*NT + tid
   const int base = rank * (NT * R);
@@ -181,49 +190,40 @@ __global__ void __launch_bounds__(NT, 1)
   if (saw_nan && dev_status) atomicOr(dev_status, TG_DEV_NAN_SCORE);
   __syncthreads();
 
-  // ---- pass 0: sign + exponent, lanes with equal bins merged before the atomic
+  // ---- pass 0: sign + 7 exponent bits; lanes with equal bins merged before the atomic
   for (int i = 0; i < R; ++i) {
     const bool ok = i * NT < nvalid;
     const uint32_t act = __ballot_sync(0xffffffffu, ok);
     if (ok) {
-      const uint32_t d = keys[i * NT + tid] >> 23;
+      const uint32_t d = keys[i * NT + tid] >> 24;
       const uint32_t grp = __match_any_sync(act, d);
-      if (lane == __ffs(grp) - 1) atomicAdd(&hist0[d], (uint32_t)__popc(grp));
+      if (lane == __ffs(grp) - 1) atomicAdd(&hist[0][d], (uint32_t)__popc(grp));
     }
   }
   if (C > 1) cluster.sync();
   else __syncthreads();
   int need = sq.kc;
-  find_digit(hist0, NB0, need, cluster, C, rank, warp_sums, &s_digit, &s_above);
-  const uint32_t d0 = s_digit;
+  find_digit(hist[0], need, cluster, C, rank, warp_sums, &s_digit, &s_above);
+  uint32_t prefix = s_digit;  // key >> 24
   need -= s_above;
   __syncthreads();
-
-  // ---- pass 1: the next 11 bits of keys in bin d0
-  for (int i = 0; i < R; ++i) {
-    if (i * NT >= nvalid) break;
-    const uint32_t k = keys[i * NT + tid];
-    if ((k >> 23) == d0) atomicAdd(&hist1[(k >> 12) & (NB1 - 1)], 1u);
+  // ---- passes 1-3: the next byte of the keys that still match the prefix
+#pragma unroll 1
+  for (int pass = 1; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = 0; i < R; ++i) {
+      if (i * NT >= nvalid) break;
+      const uint32_t k = keys[i * NT + tid];
+      if ((k >> (shift + 8)) == prefix) atomicAdd(&hist[pass][(k >> shift) & (NB - 1)], 1u);
+    }
+    if (C > 1) cluster.sync();
+    else __syncthreads();
+    find_digit(hist[pass], need, cluster, C, rank, warp_sums, &s_digit, &s_above);
+    prefix = (prefix << 8) | s_digit;
+    need -= s_above;
+    __syncthreads();
   }
-  if (C > 1) cluster.sync();
-  else __syncthreads();
-  find_digit(hist1, NB1, need, cluster, C, rank, warp_sums, &s_digit, &s_above);
-  const uint32_t p1 = (d0 << 11) | s_digit;  // key >> 12
-  need -= s_above;
-  __syncthreads();
-
-  // ---- pass 2: the last 12 bits
-  for (int i = 0; i < R; ++i) {
-    if (i * NT >= nvalid) break;
-    const uint32_t k = keys[i * NT + tid];
-    if ((k >> 12) == p1) atomicAdd(&hist2[k & (NB2 - 1)], 1u);
-  }
-  if (C > 1) cluster.sync();
-  else __syncthreads();
-  find_digit(hist2, NB2, need, cluster, C, rank, warp_sums, &s_digit, &s_above);
-  const uint32_t T = (p1 << 12) | s_digit;  // the K-th largest key; `need` keys equal to T are kept
-  need -= s_above;
-  __syncthreads();
+  const uint32_t T = prefix;  // the K-th largest key; `need` keys equal to T are kept
 
   // ---- compaction in index order: per (row i, warp) counts, element = base + i*NT + w*32 + lane
   const uint32_t lt = (1u << lane) - 1u;
@@ -293,9 +293,9 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
   SelParams p = {};
   for (int i = 0; i < nseq; ++i) p.s[i] = seqs[i];
   const int per_cta = NT * MAX_ROWS;
-  // about 4096 keys per CTA (up to 8 CTAs): the passes are instruction-bound, so a sequence
+  // about 8192 keys per CTA (up to 8 CTAs): the passes are instruction-bound, so a sequence
   // is spread over several SMs rather than one
-  int C = (n_ctx_max + 4 * NT - 1) / (4 * NT);
+  int C = (n_ctx_max + 8 * NT - 1) / (8 * NT);
   C = C < 1 ? 1 : (C > 8 ? 8 : C);
   if ((int64_t)C * per_cta < n_ctx_max)
     return fail(TG_ERR_UNSUPPORTED, "context of %d tokens exceeds the select capacity", n_ctx_max);
