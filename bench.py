@@ -259,6 +259,7 @@ def main():
     import torch.distributed as dist
 
     import learned_token_pruning_02_b200 as tg
+    from learned_token_pruning_02_b200 import replicas
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -344,11 +345,7 @@ def main():
     clk = clocks.stop()
     st_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
     step_ms = st_ms.sum(axis=1)
-    t_total = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([t_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_total = float(t.item())
+    t_total = replicas.max_over_ranks(float(step_ms.sum()), device=dev)
     ms_per_step = t_total / args.steps
     value = wl.n_tok * world * args.steps / (t_total / 1e3)
     stage_ms = st_ms.mean(axis=0)
@@ -410,11 +407,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        t = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([t], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t = float(tt.item())
+        t = replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
         h2d = H.numel() * 2 + sum(x.numel() * 2 for L in layers for x in L)
         d2h = sum(o.numel() * 2 for o in Os) + M * 4
         e2e = {"value": wl.n_tok * world * args.e2e_steps / (t / 1e3), "unit": "tokens/s",
