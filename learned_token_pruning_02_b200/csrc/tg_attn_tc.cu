@@ -12,12 +12,12 @@
 // warpgroup, TMEM score buffer and TMEM output accumulator, so one group's exponentials
 // overlap the other group's matrix products:
 //   * warp 0: TMA loads Q once and K_j (128 keys) into a 3-deep ring, so the next products
-//     QK^T never wait on L2; warp 10 loads V_j into the stage of chain j % 2 and stages the
+//     QK^T never wait on L2; warp 2 loads V_j into the stage of chain j % 2 and stages the
 //     tile's per-key bias gain*log2(e)*log g_j in shared memory.
 //   * warp 1 (one thread): tcgen05.mma. S_j = Q K_j^T (M=128, N=128, K=D) into the chain's
 //     TMEM S buffer; O_c += P_j V_j with P_j read from TMEM (A operand in tensor memory) and
 //     V_j from shared memory (N-contiguous operand).
-//   * warps 2-5 (chain 0) and 6-9 (chain 1): one query row per thread. The thread loads its
+//   * warps 4-7 (chain 0) and 8-11 (chain 1): one query row per thread. The thread loads its
 //     whole S row from TMEM into registers, forms scale*log2(e)*S + bias (causal mask on the
 //     diagonal tile only), and writes P = 2^(x - m) back as packed bf16 into the same TMEM
 //     columns. The running
@@ -38,7 +38,7 @@ using namespace sm100;
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int NTHREADS = 352;  // warp 0: Q/K loads, 1: MMA, 2-9: softmax, 10: V loads + bias
+constexpr int NTHREADS = 384;  // warp 0: Q/K loads, 1: MMA, 2: V loads + bias, 3: idle, 4-11: softmax
 constexpr int KS = 3;           // K ring depth
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 10) {  // ---------------------------------------- V producer + key bias
+  } else if (warp == 2) {  // ----------------------------------------- V producer + key bias
     int issued = 0;
     for (int j = 0; j < nt; ++j) {
       const int c = j & 1, u = j >> 1;
@@ -280,8 +280,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {
       }
     }
-  } else {  // --------------------------------------------------------- softmax warpgroups
-    const int c = (warp - 2) >> 2;  // chain: 0 = warps 2-5 (even tiles), 1 = warps 6-9 (odd tiles)
+  } else if (warp >= 4) {  // ------------------------------------------- softmax warpgroups
+    const int c = (warp - 4) >> 2;  // chain: 0 = warps 4-7 (even tiles), 1 = warps 8-11 (odd tiles)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // query row in the tile == TMEM lane
     const int il = t * BQ + r;     // row within the sequence
@@ -303,90 +303,106 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
-      uint32_t sr[BKV];  // the whole S row of this thread, then P
-#pragma unroll
-      for (int ch = 0; ch < BKV / 32; ++ch)
-        tmem_ld32(tS + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
-      tmem_wait_ld();
       const float4* bs4 = reinterpret_cast<const float4*>(bias_s + c * BKV);
-      float mx = -INFINITY;
-      if (j == t) {  // diagonal tile: causal mask (key column > query row)
+      const float2 qk2 = make_float2(qk_scale, qk_scale);
+      const bool diag = (j == t);
+      // pass 1: row max of the log2-domain logits scale*log2(e)*S + bias (causal mask on the
+      // diagonal tile), 32 columns per TMEM load, 8 independent max chains
+      float m8[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+      for (int ch = 0; ch < BKV / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tS + ch * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < BKV / 4; ++q) {
-          const float4 bb = bs4[q];
-          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = 4 * q + e;
-            const float x = col > r ? -INFINITY : fmaf(__uint_as_float(sr[col]), qk_scale, bv[e]);
-            sr[col] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
+        for (int q = 0; q < 8; ++q) {
+          const float4 bb = bs4[ch * 8 + q];
+          float2 x0 = __ffma2_rn(make_float2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])), qk2,
+                                 make_float2(bb.x, bb.y));
+          float2 x1 = __ffma2_rn(make_float2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), qk2,
+                                 make_float2(bb.z, bb.w));
+          if (diag) {
+            const int col = ch * 32 + 4 * q;
+            if (col > r) x0.x = -INFINITY;
+            if (col + 1 > r) x0.y = -INFINITY;
+            if (col + 2 > r) x1.x = -INFINITY;
+            if (col + 3 > r) x1.y = -INFINITY;
           }
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < BKV / 4; ++q) {
-          const float4 bb = bs4[q];
-          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = 4 * q + e;
-            const float x = fmaf(__uint_as_float(sr[col]), qk_scale, bv[e]);
-            sr[col] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
-          }
+          m8[q] = fmaxf(m8[q], fmaxf(fmaxf(x0.x, x0.y), fmaxf(x1.x, x1.y)));
         }
       }
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float m_cand = fmaxf(m_run, mx);
-      if (__any_sync(0xffffffffu, m_cand > m_run + kRescaleSlack)) {
-        const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_cand);  // 0 on the chain's first tile
-        if (u > 0) {  // rescale the chain's O once its previous PV product has landed
-          if (!__all_sync(0xffffffffu, mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + c0, o);
-          }
-          tmem_wait_st();
-        }
-        l_run *= alpha;
+      // lazy rescale: move the running max only when it grows by more than the slack
+      const bool resc = __any_sync(0xffffffffu, m_cand > m_run + kRescaleSlack);
+      float alpha = 1.f;
+      if (resc) {
+        alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_cand);  // 0 on the chain's first tile
         m_run = m_cand;
       }
       const float mb = m_run == -INFINITY ? 0.f : m_run;
-      // P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns
-      float sum = 0.f;
-      uint32_t pk[BKV / 2];
-      if (unnorm) {
-        const float4* gm4 = reinterpret_cast<const float4*>(gmul_s + c * BKV);
+      // pass 2: P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns
+      // (P chunk ch lands on columns 16ch..16ch+15, all already read)
+      const float2 nm = make_float2(-mb, -mb);
+      const float4* gm4 = reinterpret_cast<const float4*>(gmul_s + c * BKV);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll 1
+      for (int ch = 0; ch < BKV / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tS + ch * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < BKV / 4; ++q) {
-          const float4 gg = gm4[q];
-          const float p0 = ex2(__uint_as_float(sr[4 * q]) - mb), p1 = ex2(__uint_as_float(sr[4 * q + 1]) - mb);
-          const float p2 = ex2(__uint_as_float(sr[4 * q + 2]) - mb), p3 = ex2(__uint_as_float(sr[4 * q + 3]) - mb);
-          sum += (p0 + p1) + (p2 + p3);
-          pk[2 * q] = pack_bf16(p0 * gg.x, p1 * gg.y);
-          pk[2 * q + 1] = pack_bf16(p2 * gg.z, p3 * gg.w);
+        for (int q = 0; q < 8; ++q) {
+          const float4 bb = bs4[ch * 8 + q];
+          float2 x0 = __ffma2_rn(make_float2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])), qk2,
+                                 make_float2(bb.x, bb.y));
+          float2 x1 = __ffma2_rn(make_float2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), qk2,
+                                 make_float2(bb.z, bb.w));
+          if (diag) {
+            const int col = ch * 32 + 4 * q;
+            if (col > r) x0.x = -INFINITY;
+            if (col + 1 > r) x0.y = -INFINITY;
+            if (col + 2 > r) x1.x = -INFINITY;
+            if (col + 3 > r) x1.y = -INFINITY;
+          }
+          const float2 d0 = __fadd2_rn(x0, nm), d1 = __fadd2_rn(x1, nm);
+          float2 p0 = make_float2(ex2(d0.x), ex2(d0.y)), p1 = make_float2(ex2(d1.x), ex2(d1.y));
+          acc[(2 * q) & 3] = __fadd2_rn(acc[(2 * q) & 3], p0);
+          acc[(2 * q + 1) & 3] = __fadd2_rn(acc[(2 * q + 1) & 3], p1);
+          if (unnorm) {
+            const float4 gg = gm4[ch * 8 + q];
+            p0 = __fmul2_rn(p0, make_float2(gg.x, gg.y));
+            p1 = __fmul2_rn(p1, make_float2(gg.z, gg.w));
+          }
+          pk[2 * q] = pack_bf16(p0.x, p0.y);
+          pk[2 * q + 1] = pack_bf16(p1.x, p1.y);
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < BKV; e += 2) {
-          const float p0 = ex2(__uint_as_float(sr[e]) - mb), p1 = ex2(__uint_as_float(sr[e + 1]) - mb);
-          sum += p0 + p1;
-          pk[e >> 1] = pack_bf16(p0, p1);
-        }
+        tmem_st16(tS + ch * 16, pk);
       }
-      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 s4 = __fadd2_rn(s01, s23);
+      const float sum = s4.x + s4.y;
       tmem_wait_st();
-      l_run += sum;
+      if (resc && u > 0) {  // rescale the chain's O once its previous PV product has landed
+        if (!__all_sync(0xffffffffu, mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + c0, o);
+        }
+        tmem_wait_st();
+      }
+      l_run = l_run * alpha + sum;
       tc_fence_before();
       mbar_arrive(&pready[c]);
     }
