@@ -72,7 +72,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int D>
+template <int D, bool UNNORM>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const float* __restrict__ logg,
@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int nt = t + 1;  // key tiles 0..t (causal)
   const int n0 = (nt + 1) >> 1, n1 = nt >> 1;  // key tiles in chain 0 (even) and chain 1 (odd)
   const int kvh = h / (Hq / Hkv);
-  const bool unnorm = (flags & TG_ATTN_UNNORMALISED) != 0;
+  constexpr bool unnorm = UNNORM;
   const float gain2 = (gain ? gain[h] : 1.f) * kLog2e;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -303,32 +303,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
-      const float4* bs4 = reinterpret_cast<const float4*>(bias_s + c * BKV);
-      const float2 qk2 = make_float2(qk_scale, qk_scale);
-      const bool diag = (j == t);
-      // pass 1: row max of the log2-domain logits scale*log2(e)*S + bias (causal mask on the
-      // diagonal tile), 32 columns per TMEM load, 8 independent max chains
-      float m8[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-      for (int ch = 0; ch < BKV / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tS + ch * 32, v);
-        tmem_wait_ld();
+      uint32_t sr[BKV];  // the whole S row of this thread, then the logits
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 bb = bs4[ch * 8 + q];
-          float2 x0 = __ffma2_rn(make_float2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])), qk2,
-                                 make_float2(bb.x, bb.y));
-          float2 x1 = __ffma2_rn(make_float2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), qk2,
-                                 make_float2(bb.z, bb.w));
-          if (diag) {
-            const int col = ch * 32 + 4 * q;
-            if (col > r) x0.x = -INFINITY;
-            if (col + 1 > r) x0.y = -INFINITY;
-            if (col + 2 > r) x1.x = -INFINITY;
-            if (col + 3 > r) x1.y = -INFINITY;
+      for (int ch = 0; ch < BKV / 32; ++ch)
+        tmem_ld32(tS + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
+      tmem_wait_ld();
+      const float4* bs4 = reinterpret_cast<const float4*>(bias_s + c * BKV);
+      // log2-domain logits scale*log2(e)*S + bias; causal mask on the diagonal tile only;
+      // the row max runs as 8 independent chains
+      float m8[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (j == t) {
+#pragma unroll
+        for (int q = 0; q < BKV / 4; ++q) {
+          const float4 bb = bs4[q];
+          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 4 * q + e;
+            const float x = col > r ? -INFINITY : fmaf(__uint_as_float(sr[col]), qk_scale, bv[e]);
+            sr[col] = __float_as_uint(x);
+            m8[col & 7] = fmaxf(m8[col & 7], x);
           }
-          m8[q] = fmaxf(m8[q], fmaxf(fmaxf(x0.x, x0.y), fmaxf(x1.x, x1.y)));
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < BKV / 4; ++q) {
+          const float4 bb = bs4[q];
+          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 4 * q + e;
+            const float x = fmaf(__uint_as_float(sr[col]), qk_scale, bv[e]);
+            sr[col] = __float_as_uint(x);
+            m8[col & 7] = fmaxf(m8[col & 7], x);
+          }
         }
       }
       const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
@@ -342,48 +350,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         m_run = m_cand;
       }
       const float mb = m_run == -INFINITY ? 0.f : m_run;
-      // pass 2: P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns
-      // (P chunk ch lands on columns 16ch..16ch+15, all already read)
-      const float2 nm = make_float2(-mb, -mb);
-      const float4* gm4 = reinterpret_cast<const float4*>(gmul_s + c * BKV);
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll 1
-      for (int ch = 0; ch < BKV / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tS + ch * 32, v);
-        tmem_wait_ld();
-        uint32_t pk[16];
+      // P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[BKV / 2];
+      if constexpr (UNNORM) {
+        const float4* gm4 = reinterpret_cast<const float4*>(gmul_s + c * BKV);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 bb = bs4[ch * 8 + q];
-          float2 x0 = __ffma2_rn(make_float2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])), qk2,
-                                 make_float2(bb.x, bb.y));
-          float2 x1 = __ffma2_rn(make_float2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), qk2,
-                                 make_float2(bb.z, bb.w));
-          if (diag) {
-            const int col = ch * 32 + 4 * q;
-            if (col > r) x0.x = -INFINITY;
-            if (col + 1 > r) x0.y = -INFINITY;
-            if (col + 2 > r) x1.x = -INFINITY;
-            if (col + 3 > r) x1.y = -INFINITY;
-          }
-          const float2 d0 = __fadd2_rn(x0, nm), d1 = __fadd2_rn(x1, nm);
-          float2 p0 = make_float2(ex2(d0.x), ex2(d0.y)), p1 = make_float2(ex2(d1.x), ex2(d1.y));
-          acc[(2 * q) & 3] = __fadd2_rn(acc[(2 * q) & 3], p0);
-          acc[(2 * q + 1) & 3] = __fadd2_rn(acc[(2 * q + 1) & 3], p1);
-          if (unnorm) {
-            const float4 gg = gm4[ch * 8 + q];
-            p0 = __fmul2_rn(p0, make_float2(gg.x, gg.y));
-            p1 = __fmul2_rn(p1, make_float2(gg.z, gg.w));
-          }
-          pk[2 * q] = pack_bf16(p0.x, p0.y);
-          pk[2 * q + 1] = pack_bf16(p1.x, p1.y);
+        for (int q = 0; q < BKV / 4; ++q) {
+          const float4 gg = gm4[q];
+          const float p0 = ex2(__uint_as_float(sr[4 * q]) - mb), p1 = ex2(__uint_as_float(sr[4 * q + 1]) - mb);
+          const float p2 = ex2(__uint_as_float(sr[4 * q + 2]) - mb), p3 = ex2(__uint_as_float(sr[4 * q + 3]) - mb);
+          s4[0] += p0;
+          s4[1] += p1;
+          s4[2] += p2;
+          s4[3] += p3;
+          pk[2 * q] = pack_bf16(p0 * gg.x, p1 * gg.y);
+          pk[2 * q + 1] = pack_bf16(p2 * gg.z, p3 * gg.w);
         }
-        tmem_st16(tS + ch * 16, pk);
+      } else {
+#pragma unroll
+        for (int e = 0; e < BKV; e += 2) {
+          const float p0 = ex2(__uint_as_float(sr[e]) - mb), p1 = ex2(__uint_as_float(sr[e + 1]) - mb);
+          s4[(e >> 1) & 3] += p0 + p1;
+          pk[e >> 1] = pack_bf16(p0, p1);
+        }
       }
-      const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
-      const float2 s4 = __fadd2_rn(s01, s23);
-      const float sum = s4.x + s4.y;
+      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       if (resc && u > 0) {  // rescale the chain's O once its previous PV product has landed
         if (!__all_sync(0xffffffffu, mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status))) {
@@ -478,16 +472,17 @@ tg_status launch_d(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_
       !make_tmap_bf16_2d(&tk, a.K, (uint64_t)a.m_tot, (uint64_t)a.Hkv * D, (uint64_t)a.Hkv * D, BKV, 64) ||
       !make_tmap_bf16_2d(&tv, a.V, (uint64_t)a.m_tot, (uint64_t)a.Hkv * D, (uint64_t)a.Hkv * D, BKV, 64))
     return fail(TG_ERR_CUDA, "tg_gated_attn_fwd: building the TMA tensor maps failed");
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const bool un = (a.flags & TG_ATTN_UNNORMALISED) != 0;
+  auto kern = un ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
+  static bool attr_set[2] = {false, false};
+  if (!attr_set[un]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_fwd: cudaFuncSetAttribute");
-    attr_set = true;
+    attr_set[un] = true;
   }
   const int grid = units * a.Hq;
-  attn_tc_kernel<D><<<grid, NTHREADS, C::SMEM, st>>>(tq, tk, tv, a.logg, a.head_gain, a.pos,
-                                                     static_cast<__nv_bfloat16*>(a.O), a.lse, a.m_tot, a.Hq, a.Hkv,
-                                                     a.scale * kLog2e, a.flags, a.dev_status, p);
+  kern<<<grid, NTHREADS, C::SMEM, st>>>(tq, tk, tv, a.logg, a.head_gain, a.pos, static_cast<__nv_bfloat16*>(a.O),
+                                        a.lse, a.m_tot, a.Hq, a.Hkv, a.scale * kLog2e, a.flags, a.dev_status, p);
   return cuda_status(cudaGetLastError(), "tg_gated_attn_fwd: attn_tc launch");
 }
 
