@@ -60,7 +60,7 @@ struct ACfg {
   static constexpr int K_OFF = TILE_BYTES;               // KS stages
   static constexpr int V_OFF = TILE_BYTES * (1 + KS);    // 2 stages (one per chain)
   static constexpr int TAIL_OFF = TILE_BYTES * (3 + KS);
-  static constexpr int TAIL = 4096;
+  static constexpr int TAIL = 8192;  // barriers (256 B), bias and gate multipliers (2 KB), chain max/sum (2 KB)
   static constexpr int SMEM = 1024 + TAIL_OFF + TAIL;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BQ, BKV, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, true);
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* bias_s = reinterpret_cast<float*>(tail + 256);  // [2][128]
   float* gmul_s = bias_s + 2 * BKV;                      // [2][128]
-  float* ml_s = gmul_s + 2 * BKV;                        // [2][128]: chain-1 max and sum
+  float* ml_s = gmul_s + 2 * BKV;                        // [2 chains][max, sum][128]
 
   // ---- which (sequence, query tile, head) this CTA owns: longest row-ranges first
   const int h = blockIdx.x % Hq;
@@ -144,15 +144,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&pready[s], 128);
       mbar_init(&pvdone[s], 1);
     }
-    mbar_init(mlready, 128);
+    mbar_init(mlready, 256);
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
+    // Q and the first key tiles go out before the CTA-wide sync (their ring slots start free)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    mbar_arrive_expect_tx(qfull, C::TILE_BYTES);
+    for (int bx = 0; bx < C::NBOX; ++bx)
+      tma_load_2d(smem + C::Q_OFF + bx * (BQ * 128), &tmQ, h * D + bx * 64, off + t * BQ, qfull);
+    for (int j = 0; j < KS && j < nt; ++j) {
+      uint8_t* kb = smem + C::K_OFF + j * C::TILE_BYTES;
+      mbar_arrive_expect_tx(&kfull[j], C::TILE_BYTES);
+      for (int bx = 0; bx < C::NBOX; ++bx)
+        tma_load_2d(kb + bx * (BKV * 128), &tmK, kvh * D + bx * 64, off + j * BKV, &kfull[j]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -165,11 +173,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp == 0) {  // ------------------------------------------------- Q and K producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(qfull, C::TILE_BYTES);
-      for (int bx = 0; bx < C::NBOX; ++bx)
-        tma_load_2d(smem + C::Q_OFF + bx * (BQ * 128), &tmQ, h * D + bx * 64, off + t * BQ, qfull);
-      int issued = 0;
-      for (int j = 0; j < nt; ++j) {
+      int issued = KS < nt ? KS : nt;
+      for (int j = issued; j < nt; ++j) {
         const int s = j % KS;
         if (!mbar_wait(&kempty[s], ((j / KS) & 1) ^ 1u, abort, dev_status)) break;
         uint8_t* kb = smem + C::K_OFF + s * C::TILE_BYTES;
@@ -189,44 +194,50 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 2) {  // ----------------------------------------- V producer + key bias
-    int issued = 0;
-    for (int j = 0; j < nt; ++j) {
-      const int c = j & 1, u = j >> 1;
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(&vempty[c], (u & 1) ^ 1u, abort, dev_status);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      if (lane == 0) {
+  } else if (warp == 2) {  // ------------------------------------------------- V producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int c = j & 1, u = j >> 1;
+        if (!mbar_wait(&vempty[c], (u & 1) ^ 1u, abort, dev_status)) break;
         uint8_t* vb = smem + C::V_OFF + c * C::TILE_BYTES;
         mbar_arrive_expect_tx(&vfull[c], C::TILE_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_2d(vb + bx * (BKV * 128), &tmV, kvh * D + bx * 64, off + j * BKV, &vfull[c]);
+        ++issued;
       }
-      ++issued;
-      // per-key bias of this key tile (log2 domain), 4 keys per lane; the chain's slot is
-      // free because the PV product of its previous tile has completed (vempty above)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = lane * 4 + e;
-        const int kl = j * BKV + col;
-        const float bv = (logg && kl < m) ? gain2 * logg[off + kl] : 0.f;
-        bias_s[c * BKV + col] = unnorm ? 0.f : bv;
-        gmul_s[c * BKV + col] = unnorm ? ex2(bv) : 1.f;
-      }
-      mbar_arrive(&bfull[c]);
-    }
-    if (lane == 0 && *abort) {
-      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
-        const uint64_t t1 = globaltimer_ns();
-        while (!mbar_try_wait(&vfull[j & 1], (j >> 1) & 1) && globaltimer_ns() - t1 < 1000000000ull) {
+      if (*abort) {
+        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
+          const uint64_t t1 = globaltimer_ns();
+          while (!mbar_try_wait(&vfull[j & 1], (j >> 1) & 1) && globaltimer_ns() - t1 < 1000000000ull) {
+          }
         }
       }
+    }
+  } else if (warp == 3) {  // ---------------------------------------------- key-bias stager
+    // Per-key bias of key tile j (log2 domain), 4 keys per lane, staged in the chain's slot as
+    // soon as the chain's previous softmax has read it; the log g loads go out first.
+    for (int j = 0; j < nt; ++j) {
+      const int c = j & 1, u = j >> 1;
+      float bv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kl = j * BKV + lane * 4 + e;
+        bv[e] = (logg && kl < m) ? gain2 * logg[off + kl] : 0.f;
+      }
+      if (u > 0 && !__all_sync(0xffffffffu, mbar_wait(&pready[c], (u - 1) & 1, abort, dev_status))) break;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bias_s[c * BKV + lane * 4 + e] = unnorm ? 0.f : bv[e];
+        gmul_s[c * BKV + lane * 4 + e] = unnorm ? ex2(bv[e]) : 1.f;
+      }
+      mbar_arrive(&bfull[c]);
     }
   } else if (warp == 1) {  // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t qa = smem_u32(smem + C::Q_OFF);
-      // Event loop: issue whichever product is ready, never blocking on one barrier while the
-      // other product could go. S_j needs K_j and the chain's S buffer (free once PV of the
+      // Event loop: issue whichever product is ready, polling with non-blocking test_wait so
+      // it never sleeps on one barrier while the other product could go. S_j needs K_j and the chain's S buffer (free once PV of the
       // chain's previous tile completed); PV_j needs P_j and V_j. At most two S ahead of PV.
       bool ok = mbar_wait(qfull, 0, abort, dev_status);
       int next_s = 0, next_pv = 0;
@@ -235,7 +246,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool progressed = false;
         if (next_pv < next_s) {
           const int j = next_pv, c = j & 1, u = j >> 1;
-          if (mbar_try_wait(&pready[c], u & 1) && mbar_try_wait(&vfull[c], u & 1)) {
+          if (mbar_test(&pready[c], u & 1) && mbar_test(&vfull[c], u & 1)) {
             tc_fence_after();
             const uint32_t va = smem_u32(smem + C::V_OFF + c * C::TILE_BYTES);
 #pragma unroll
@@ -250,7 +261,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         if (next_s < nt && next_s < next_pv + 2) {
           const int j = next_s, c = j & 1, u = j >> 1, ks = j % KS;
-          if (mbar_try_wait(&kfull[ks], (j / KS) & 1) && (u == 0 || mbar_try_wait(&pvdone[c], (u - 1) & 1))) {
+          if (mbar_test(&kfull[ks], (j / KS) & 1) && (u == 0 || mbar_test(&pvdone[c], (u - 1) & 1))) {
             tc_fence_after();
             const uint32_t ka = smem_u32(smem + C::K_OFF + ks * C::TILE_BYTES);
 #pragma unroll
@@ -400,49 +411,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_before();
       mbar_arrive(&pready[c]);
     }
-    if (c == 1) {  // hand the chain's max and sum to chain 0
-      ml_s[r] = ok ? m_run : -INFINITY;
-      ml_s[BKV + r] = ok ? l_run : 0.f;
-      mbar_arrive(mlready);
-    } else if (ok) {
-      const bool got = __all_sync(0xffffffffu, mbar_wait(mlready, 0, abort, dev_status) &&
-                                                   mbar_wait(&pvdone[0], (n0 - 1) & 1, abort, dev_status) &&
-                                                   (n1 == 0 || mbar_wait(&pvdone[1], (n1 - 1) & 1, abort, dev_status)));
-      if (got) {
-        tc_fence_after();
-        const float m1 = ml_s[r], l1 = ml_s[BKV + r];
-        const float mfin = fmaxf(m_run, m1);
-        const float mz = mfin == -INFINITY ? 0.f : mfin;
-        const float f0 = ex2(m_run - mz), f1 = n1 > 0 ? ex2(m1 - mz) : 0.f;
-        const float lt = l_run * f0 + l1 * f1;
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        const float s0 = f0 * inv, s1 = f1 * inv;
-        __nv_bfloat16* orow = O + ((int64_t)(off + il) * Hq + h) * D;
-        const uint32_t tO1 = tmem + lane_base + 256 + D;
+    // Merge the two chains: both warpgroups publish their (max, sum), then each writes half of
+    // the head dimension of O from both accumulators; chain 0 also writes the LSE.
+    ml_s[c * 2 * BKV + r] = ok ? m_run : -INFINITY;
+    ml_s[c * 2 * BKV + BKV + r] = ok ? l_run : 0.f;
+    mbar_arrive(mlready);
+    const bool got = ok && __all_sync(0xffffffffu, mbar_wait(mlready, 0, abort, dev_status) &&
+                                                       mbar_wait(&pvdone[0], (n0 - 1) & 1, abort, dev_status) &&
+                                                       (n1 == 0 || mbar_wait(&pvdone[1], (n1 - 1) & 1, abort, dev_status)));
+    if (got) {
+      tc_fence_after();
+      const float m0 = ml_s[r], l0 = ml_s[BKV + r];
+      const float m1 = ml_s[2 * BKV + r], l1 = ml_s[3 * BKV + r];
+      const float mfin = fmaxf(m0, m1);
+      const float mz = mfin == -INFINITY ? 0.f : mfin;
+      const float f0 = ex2(m0 - mz), f1 = n1 > 0 ? ex2(m1 - mz) : 0.f;
+      const float lt = l0 * f0 + l1 * f1;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float s0 = f0 * inv, s1 = f1 * inv;
+      __nv_bfloat16* orow = O + ((int64_t)(off + il) * Hq + h) * D;
+      const uint32_t tO0 = tmem + lane_base + 256, tO1 = tmem + lane_base + 256 + D;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o0[32], o1[32];
-          tmem_ld32(tO + c0, o0);
-          if (n1 > 0) tmem_ld32(tO1 + c0, o1);
-          tmem_wait_ld();
-          uint32_t pkd[16];
+      for (int c0 = c * (D / 2); c0 < (c + 1) * (D / 2); c0 += 32) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tO0 + c0, o0);
+        if (n1 > 0) tmem_ld32(tO1 + c0, o1);
+        tmem_wait_ld();
+        uint32_t pkd[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float a0 = __uint_as_float(o0[2 * e]) * s0, a1 = __uint_as_float(o0[2 * e + 1]) * s0;
-            if (n1 > 0) {
-              a0 = fmaf(__uint_as_float(o1[2 * e]), s1, a0);
-              a1 = fmaf(__uint_as_float(o1[2 * e + 1]), s1, a1);
-            }
-            pkd[e] = pack_bf16(a0, a1);
+        for (int e = 0; e < 16; ++e) {
+          float a0 = __uint_as_float(o0[2 * e]) * s0, a1 = __uint_as_float(o0[2 * e + 1]) * s0;
+          if (n1 > 0) {
+            a0 = fmaf(__uint_as_float(o1[2 * e]), s1, a0);
+            a1 = fmaf(__uint_as_float(o1[2 * e + 1]), s1, a1);
           }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
-          }
+          pkd[e] = pack_bf16(a0, a1);
         }
-        if (valid && lse) lse[(int64_t)h * m_tot + off + il] = (mz + __log2f(lt)) * kLn2;
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+        }
       }
+      if (c == 0 && valid && lse) lse[(int64_t)h * m_tot + off + il] = (mz + __log2f(lt)) * kLn2;
     }
   }
 
