@@ -325,29 +325,44 @@ def main():
         if ev:
             ev[4].record(stream)
 
-    launches_per_step = 4 + (wl.n_layers - 1)
+    launches_per_step = 4 + (wl.n_layers - 1)  # score, select, gather, attention per layer
 
     for _ in range(args.warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # Timed region A (the metric): whole steps, events only at step boundaries, so the
+    # kernels of a step chain with programmatic dependent launch as they do for a user.
+    ev_a = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     clocks = ClockSampler(local).start()
     barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.zero_()  # L2 flush, outside the timed events
         torch.cuda._sleep(200_000)  # keeps the host's launches ahead of the GPU (no idle gaps timed)
+        ev_a[i][0].record(stream)
+        chain()
+        ev_a[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = np.array([e[0].elapsed_time(e[1]) for e in ev_a])
+    t_total = replicas.max_over_ranks(float(step_ms.sum()), device=dev)
+    ms_per_step = t_total / args.steps
+    value = wl.n_tok * world * args.steps / (t_total / 1e3)
+    # Timed region B (the per-kernel durations behind the roofline): the same steps with an
+    # event between kernels (which also serialises them, so their sum exceeds region A's step).
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        torch.cuda._sleep(200_000)
         step(evs[i])
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     st_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
-    step_ms = st_ms.sum(axis=1)
-    t_total = replicas.max_over_ranks(float(step_ms.sum()), device=dev)
-    ms_per_step = t_total / args.steps
-    value = wl.n_tok * world * args.steps / (t_total / 1e3)
     stage_ms = st_ms.mean(axis=0)
     dev_status = int(status.item())
 
@@ -461,7 +476,8 @@ def main():
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": 2 * launches_per_step * args.steps,  # timed regions A and B together
+            "stages_sum_us": float(stage_ms.sum() * 1e3),
             "clocks": clk,
             "full_attention_reference": full_ref,
             "device_status": dev_status,

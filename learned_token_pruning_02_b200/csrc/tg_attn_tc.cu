@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
+    griddep_wait();  // inputs written by the previous kernel are visible from here on
     // Q and the first key tiles go out before the CTA-wide sync (their ring slots start free)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
@@ -169,6 +170,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_launch_dependents();  // the next kernel may start its prologue
+  griddep_wait();               // (a no-op once thread 0's wait has returned)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {  // ------------------------------------------------- Q and K producer
@@ -492,9 +495,18 @@ tg_status launch_d(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_
     attr_set[un] = true;
   }
   const int grid = units * a.Hq;
-  kern<<<grid, NTHREADS, C::SMEM, st>>>(tq, tk, tv, a.logg, a.head_gain, a.pos, static_cast<__nv_bfloat16*>(a.O),
-                                        a.lse, a.m_tot, a.Hq, a.Hkv, a.scale * kLog2e, a.flags, a.dev_status, p);
-  return cuda_status(cudaGetLastError(), "tg_gated_attn_fwd: attn_tc launch");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = (size_t)C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, a.logg, a.head_gain, a.pos,
+                                        static_cast<__nv_bfloat16*>(a.O), a.lse, a.m_tot, a.Hq, a.Hkv,
+                                        a.scale * kLog2e, a.flags, a.dev_status, p),
+                     "tg_gated_attn_fwd: attn_tc launch");
 }
 
 }  // namespace

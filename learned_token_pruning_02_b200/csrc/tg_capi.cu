@@ -1,6 +1,7 @@
 // C-ABI layer of libtokengate: argument validation, per-sequence descriptors, dispatch.
 // No entry point allocates memory or synchronises the host with the device.
 #include <stdarg.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -57,6 +58,15 @@ int device_sm_count() {
   int dev = 0;
   cudaGetDevice(&dev);
   return (dev >= 0 && dev < 64 && g_dev_sms[dev] > 0) ? g_dev_sms[dev] : 148;
+}
+
+bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("TG_DISABLE_PDL");
+    v = (e && e[0] && e[0] != '0') ? 0 : 1;
+  }
+  return v == 1;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

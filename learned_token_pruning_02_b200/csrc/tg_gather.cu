@@ -10,6 +10,7 @@
 // within its sequence, g = sigmoid(score) and log g (stable log-sigmoid). Grid-stride over
 // rows with a grid of a few waves of the SM count.
 #include "tg_internal.cuh"
+#include "tg_sm100.cuh"
 
 namespace tg {
 namespace {
@@ -29,6 +30,8 @@ __global__ void __launch_bounds__(WARPS * 32)
                   const __grid_constant__ GatherParams p) {
   const int lane = threadIdx.x & 31;
   const int row0 = p.s[0].out_off;
+  sm100::griddep_launch_dependents();  // the next kernel may start its prologue
+  sm100::griddep_wait();               // the kept indices of the previous kernel are visible
   for (int r = blockIdx.x * WARPS + (threadIdx.x >> 5); r < m_chunk; r += gridDim.x * WARPS) {
     const int row = row0 + r;
     int b = 0;
@@ -89,9 +92,16 @@ tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const fl
   int blocks = (m_chunk + WARPS - 1) / WARPS;
   const int cap = device_sm_count() * 16;
   if (blocks > cap) blocks = cap;
-  gather_kernel<<<blocks, WARPS * 32, 0, st>>>(static_cast<const uint4*>(H), ldv, nvec, score, kept_idx, flags,
-                                               static_cast<uint4*>(H_kept), pos, g, logg, dev_status, m_chunk, p);
-  return cuda_status(cudaGetLastError(), "gather launch");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(WARPS * 32);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, gather_kernel, static_cast<const uint4*>(H), ldv, nvec, score, kept_idx,
+                                        flags, static_cast<uint4*>(H_kept), pos, g, logg, dev_status, m_chunk, p),
+                     "gather launch");
 }
 
 }  // namespace tg

@@ -21,6 +21,17 @@ tg_status cuda_status(cudaError_t e, const char* what);
 tg_status check_device();
 int device_sm_count();
 
+// Launch attribute for programmatic dependent launch (the tensor-core chain kernels start
+// their prologue while the previous kernel drains; each waits on griddepcontrol.wait before
+// its first global memory access). TG_DISABLE_PDL=1 in the environment turns it off.
+bool pdl_enabled();
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  return a;
+}
+
 // ----------------------------------------------------------------------------- launchers
 // Each returns TG_OK or TG_ERR_CUDA (argument checks happen in the C-ABI layer).
 

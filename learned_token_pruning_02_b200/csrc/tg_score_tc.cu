@@ -89,15 +89,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tmH);
     prefetch_tmap(&tmW);
   }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  griddep_launch_dependents();  // the next kernel may start its prologue
+  griddep_wait();               // the previous kernel's results are visible from here on
   if (warp >= 2) {
     for (int u = threadIdx.x - 64; u < DG; u += 32 * NEPI) {
       b1s[u] = b1 ? b1[u] : 0.f;
       w2s[u] = __bfloat162float(w2[u]);
     }
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish_pair();
   }
   tc_fence_before();
   cluster_sync_all();  // barriers of both CTAs initialised, TMEM of the pair allocated
@@ -247,13 +249,14 @@ tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void
   cfg.blockDim = dim3(NTHREADS);
   cfg.dynamicSmemBytes = (size_t)C::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cuda_status(cudaLaunchKernelEx(&cfg, score_tc_kernel<DG>, tmH, tmW, b1,
                                         static_cast<const __nv_bfloat16*>(w2), b2, score, (int)n_tok, d / BK,
                                         n_tiles, (int32_t*)nullptr),

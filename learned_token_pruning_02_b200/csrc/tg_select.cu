@@ -19,6 +19,7 @@
 #include <cooperative_groups.h>
 
 #include "tg_internal.cuh"
+#include "tg_sm100.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -87,6 +88,8 @@ __device__ __forceinline__ int block_scan_excl(int* a, int n, int* warp_sums) {
 __device__ __forceinline__ void find_digit(const uint32_t* h, int need, cg::cluster_group& cluster, int C, int rank,
                                            int* warp_sums, uint32_t* s_digit, int* s_above) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  sm100::griddep_launch_dependents();  // the next kernel may start its prologue
+  sm100::griddep_wait();               // the scores of the previous kernel are visible from here on
   int cnt[4] = {0, 0, 0, 0};
   if (tid < NB / 4) {
     const int lo = NB - 4 * (tid + 1);  // bins lo..lo+3; this thread's order is lo+3, lo+2, lo+1, lo
@@ -314,13 +317,14 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
   cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = (size_t)rows * NT * 4;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cuda_status(cudaLaunchKernelEx(&cfg, select_kernel, score, kept_idx, cu_kept_dev, dev_status, p),
                      "select launch");
 }

@@ -30,6 +30,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// ----------------------------------------------------------------------------- launch chaining
+// Programmatic dependent launch: a kernel lets the next kernel of the stream start its
+// prologue early, and waits for the previous kernel's results before touching memory.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
