@@ -241,46 +241,36 @@ __global__ void __launch_bounds__(NT, 1)
     }
   }
   __syncthreads();
-  const int gt_tot = block_scan_excl(tab_a, 32 * R, warp_sums);
-  const int eq_tot = block_scan_excl(tab_b, 32 * R, warp_sums);  // exclusive offsets of equal keys
+  const int gt_tot = block_scan_excl(tab_a, 32 * R, warp_sums);  // exclusive offsets of keys > T
+  const int eq_tot = block_scan_excl(tab_b, 32 * R, warp_sums);  // exclusive offsets of keys == T
   if (tid == 0) {
     cta_tot[0] = gt_tot;
     cta_tot[1] = eq_tot;
   }
-  int eq_before = 0, sel_before = 0;
+  // Keys before this CTA in index order: gt_before keys > T and eq_before keys == T.
+  int eq_before = 0, gt_before = 0;
   if (C > 1) {
     cluster.sync();
     for (int r = 0; r < rank; ++r) {
       const int* rc = cluster.map_shared_rank(cta_tot, r);
-      const int g_r = rc[0], e_r = rc[1];
-      int take = need - eq_before;
-      take = take < 0 ? 0 : (take > e_r ? e_r : take);
-      sel_before += g_r + take;
-      eq_before += e_r;
+      gt_before += rc[0];
+      eq_before += rc[1];
     }
   }
-  // selected: key > T, or key == T with global rank among equal keys < need
-  for (int i = 0; i < R; ++i) {
-    const uint32_t k = keys[i * NT + tid];
-    const bool v = i * NT < nvalid;
-    const bool eq = v && k == T;
-    const uint32_t be = __ballot_sync(0xffffffffu, eq);
-    const bool sel = (v && k > T) || (eq && eq_before + tab_b[i * 32 + w] + __popc(be & lt) < need);
-    const uint32_t bs = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) tab_a[i * 32 + w] = __popc(bs);
-  }
-  __syncthreads();
-  block_scan_excl(tab_a, 32 * R, warp_sums);
+  // A kept key's output slot is the number of kept keys before it: GT(p) + min(EQ(p), need),
+  // where GT(p) and EQ(p) count the keys > T and == T before position p (equal keys are kept
+  // in index order while their rank is below `need`).
   bool overflow = false;
   for (int i = 0; i < R; ++i) {
     const uint32_t k = keys[i * NT + tid];
     const bool v = i * NT < nvalid;
-    const bool eq = v && k == T;
+    const bool gt = v && k > T, eq = v && k == T;
+    const uint32_t bg = __ballot_sync(0xffffffffu, gt);
     const uint32_t be = __ballot_sync(0xffffffffu, eq);
-    const bool sel = (v && k > T) || (eq && eq_before + tab_b[i * 32 + w] + __popc(be & lt) < need);
-    const uint32_t bs = __ballot_sync(0xffffffffu, sel);
-    if (sel) {
-      const int o = sel_before + tab_a[i * 32 + w] + __popc(bs & lt);  // rank among kept context tokens
+    const int GT = gt_before + tab_a[i * 32 + w] + __popc(bg & lt);
+    const int EQ = eq_before + tab_b[i * 32 + w] + __popc(be & lt);
+    if (gt || (eq && EQ < need)) {
+      const int o = GT + (EQ < need ? EQ : need);  // rank among kept context tokens
       if (o < sq.kc) kept[sq.out_off + o] = sq.start + base + i * NT + tid;
       else overflow = true;  // cannot happen for a correct threshold; never write past the slot
     }
