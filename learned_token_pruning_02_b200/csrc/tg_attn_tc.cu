@@ -500,7 +500,7 @@ tg_status launch_d(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_
   cfg.blockDim = dim3(NTHREADS);
   cfg.dynamicSmemBytes = (size_t)C::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cudaLaunchAttribute attr[1] = {pdl_attribute(PDL_ATTN)};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, a.logg, a.head_gain, a.pos,

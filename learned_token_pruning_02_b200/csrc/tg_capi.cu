@@ -60,13 +60,14 @@ int device_sm_count() {
   return (dev >= 0 && dev < 64 && g_dev_sms[dev] > 0) ? g_dev_sms[dev] : 148;
 }
 
-bool pdl_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("TG_DISABLE_PDL");
-    v = (e && e[0] && e[0] != '0') ? 0 : 1;
+bool pdl_enabled(int kernel_id) {
+  static int mask = -1;
+  if (mask < 0) {
+    const char* off = getenv("TG_DISABLE_PDL");
+    const char* m = getenv("TG_PDL_MASK");
+    mask = (off && off[0] && off[0] != '0') ? 0 : (m ? atoi(m) : 15);
   }
-  return v == 1;
+  return (mask & kernel_id) != 0;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -96,7 +96,7 @@ tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const fl
   cfg.gridDim = dim3((unsigned)blocks);
   cfg.blockDim = dim3(WARPS * 32);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cudaLaunchAttribute attr[1] = {pdl_attribute(PDL_GATHER)};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, gather_kernel, static_cast<const uint4*>(H), ldv, nvec, score, kept_idx,

@@ -24,11 +24,13 @@ int device_sm_count();
 // Launch attribute for programmatic dependent launch (the tensor-core chain kernels start
 // their prologue while the previous kernel drains; each waits on griddepcontrol.wait before
 // its first global memory access). TG_DISABLE_PDL=1 in the environment turns it off.
-bool pdl_enabled();
-inline cudaLaunchAttribute pdl_attribute() {
+// kernel ids for the launch-chaining mask
+enum { PDL_SCORE = 1, PDL_SELECT = 2, PDL_GATHER = 4, PDL_ATTN = 8 };
+bool pdl_enabled(int kernel_id);
+inline cudaLaunchAttribute pdl_attribute(int kernel_id) {
   cudaLaunchAttribute a;
   a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  a.val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  a.val.programmaticStreamSerializationAllowed = pdl_enabled(kernel_id) ? 1 : 0;
   return a;
 }
 

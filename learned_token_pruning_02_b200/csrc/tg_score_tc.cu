@@ -254,7 +254,7 @@ tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1] = pdl_attribute();
+  attr[1] = pdl_attribute(PDL_SCORE);
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cuda_status(cudaLaunchKernelEx(&cfg, score_tc_kernel<DG>, tmH, tmW, b1,

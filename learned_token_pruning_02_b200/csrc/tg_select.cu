@@ -88,8 +88,6 @@ __device__ __forceinline__ int block_scan_excl(int* a, int n, int* warp_sums) {
 __device__ __forceinline__ void find_digit(const uint32_t* h, int need, cg::cluster_group& cluster, int C, int rank,
                                            int* warp_sums, uint32_t* s_digit, int* s_above) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  sm100::griddep_launch_dependents();  // the next kernel may start its prologue
-  sm100::griddep_wait();               // the scores of the previous kernel are visible from here on
   int cnt[4] = {0, 0, 0, 0};
   if (tid < NB / 4) {
     const int lo = NB - 4 * (tid + 1);  // bins lo..lo+3; this thread's order is lo+3, lo+2, lo+1, lo
@@ -154,6 +152,9 @@ __global__ void __launch_bounds__(NT, 1)
   __shared__ uint32_t s_digit;
   __shared__ int s_above;
 
+  sm100::griddep_launch_dependents();  // the next kernel may start its prologue
+  sm100::griddep_wait();  // the scores of the previous kernel are visible from here on, and no
+                          // kernel before it still reads kept or cu_kept
   if (rank == 0 && tid == 0 && cu_kept_dev) {
     if (sq.b == 0) cu_kept_dev[0] = 0;
     cu_kept_dev[sq.b + 1] = sq.out_off + sq.kc + sq.q;
@@ -312,7 +313,7 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
   attr[0].val.clusterDim.x = (unsigned)C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1] = pdl_attribute();
+  attr[1] = pdl_attribute(PDL_SELECT);
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cuda_status(cudaLaunchKernelEx(&cfg, select_kernel, score, kept_idx, cu_kept_dev, dev_status, p),

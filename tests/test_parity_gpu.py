@@ -357,3 +357,40 @@ def test_chain_deterministic():
     for key in ("score", "kept_idx", "H_kept", "pos", "g", "logg"):
         assert np.array_equal(bits(out1[key]), bits(out2[key])), key
     assert np.array_equal(bits(out1["O"][0]), bits(out2["O"][0]))
+
+
+def test_chain_back_to_back():
+    """Repeated launches of the whole chain on one stream, without host synchronisation.
+
+    The chain's kernels may start while their predecessor drains (launch chaining), so a
+    read placed before the wait on the previous kernel would see stale or partial data.
+    Each step's scores and kept rows are copied out on the stream; every step must select
+    exactly the oracle's top-K of its own scores, and a run of steps with no copies between
+    them must end with bit-identical outputs.
+    """
+    wl = ti.WORKLOADS["qwen3_8k"]
+    H = to_dev(ti.hidden_states(wl), wl.dtype)
+    W1n, b1n, w2n, b2 = ti.gate_weights(wl, biased=True)
+    W1, b1, w2 = to_dev(W1n, wl.dtype), to_dev(b1n, "f32"), to_dev(w2n, wl.dtype)
+    layers = [tuple(to_dev(x, wl.dtype) for x in ti.qkv(wl, 0))]
+    scale = 1.0 / math.sqrt(wl.D)
+    out = tg.tg_prefill_above_L(H, W1, b1, w2, b2, wl.seqlens, wl.q_len, wl.k, layers, scale)
+    torch.cuda.synchronize()
+    ref = {key: bits(out[key]) for key in ("score", "kept_idx", "H_kept", "pos", "logg")}
+    ref_O = bits(out["O"][0])
+    st = _stat()
+    chain = tg.PreparedChain(H, W1, b1, w2, b2, wl.seqlens, wl.q_len, wl.k, layers, scale, out, dev_status=st)
+    copies = []
+    for _ in range(12):
+        chain()
+        copies.append((out["score"].clone(), out["kept_idx"].clone()))
+    for _ in range(12):
+        chain()
+    torch.cuda.synchronize()
+    for s, kept in copies:
+        kept_o, _ = orc.topk_select(s.cpu().numpy(), wl.seqlens, wl.q_len, wl.k)
+        assert np.array_equal(kept.cpu().numpy(), kept_o.astype(np.int32))
+    for key, val in ref.items():
+        assert np.array_equal(bits(out[key]), val), key
+    assert np.array_equal(bits(out["O"][0]), ref_O)
+    assert st.item() == 0
