@@ -170,10 +170,19 @@ def blas_threads():
 # --------------------------------------------------------------------------- main
 
 
-def kernel_hash(*names):
+KERNEL_SRC = {"score": "tg_score_tc.cu", "select": "tg_select.cu", "gather": "tg_gather.cu",
+              "gated_attn": "tg_attn_tc.cu"}
+
+
+def kernel_hash(kernel_key):
+    """Hash of the sources a kernel is built from (its .cu and the shared device headers);
+    DRAM counters recorded under profiles/ apply only while this hash is unchanged."""
     h = hashlib.sha256()
-    for n in names:
-        with open(os.path.join(ROOT, "learned_token_pruning_02_b200", "csrc", n), "rb") as f:
+    for n in (KERNEL_SRC[kernel_key], "tg_sm100.cuh", "tg_internal.cuh"):
+        p = os.path.join(ROOT, "learned_token_pruning_02_b200", "csrc", n)
+        if not os.path.exists(p):
+            return ""
+        with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
@@ -375,22 +384,25 @@ def main():
     score_gbs = bytes_score / (stage_ms[0] / 1e3) / 1e9
     bytes_gather = M * wl.d * 2 * 2 + M * 4 * 4
     bytes_select = (wl.n_tok - sum(wl.q_len)) * 4 + M * 4
-    dominant = int(np.argmax(stage_ms))
     names = ["score", "select", "gather", "gated_attn"]
-    if dominant == 3:
-        roof = {"kernel": "gated_attn", "bound": "tensor", "achieved": attn_tflops, "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": attn_tflops / pk["bf16_tflops"],
-                "traffic": traffic_from_profile("gated_attn", kernel_hash("tg_attn_tc.cu") if os.path.exists(
-                    os.path.join(ROOT, "learned_token_pruning_02_b200", "csrc", "tg_attn_tc.cu")) else "")}
-    else:
-        nm = names[dominant]
-        byts = [bytes_score, bytes_select, bytes_gather][dominant]
-        gbs = byts / (stage_ms[dominant] / 1e3) / 1e9
-        src = {"score": "tg_score_tc.cu", "select": "tg_select.cu", "gather": "tg_gather.cu"}[nm]
-        srcp = os.path.join(ROOT, "learned_token_pruning_02_b200", "csrc", src)
-        roof = {"kernel": nm, "bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / pk["hbm_gbs"],
-                "traffic": traffic_from_profile(nm, kernel_hash(src) if os.path.exists(srcp) else "")}
+    per_kernel = {}
+    for i, nm in enumerate(names):
+        t_s = stage_ms[i] / 1e3
+        if nm == "gated_attn":
+            ach = attn_tflops
+            e = {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                 "algorithmic": flops_attn / wl.n_layers}
+        else:
+            byts = [bytes_score, bytes_select, bytes_gather][i]
+            ach = byts / t_s / 1e9
+            e = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s", "algorithmic": byts}
+        e["frac"] = e["achieved"] / e["peak"]
+        e["us"] = stage_ms[i] * 1e3 / (wl.n_layers if nm == "gated_attn" else 1)
+        e["traffic"] = traffic_from_profile(nm, kernel_hash(nm))
+        per_kernel[nm] = e
+    dominant = names[int(np.argmax(stage_ms))]
+    roof = {"kernel": dominant}
+    roof.update({k: per_kernel[dominant][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")})
     roof["peak_source"] = f"{pk_src} ({'burst' if roof['bound'] == 'tensor' else 'copy'})"
 
     # ---------------- end to end through the public API, host buffers in and out
@@ -474,6 +486,7 @@ def main():
             "gated_attn_frac_of_bf16_peak": attn_tflops / pk["bf16_tflops"],
             "score_hbm_gbs": score_gbs,
             "roofline": roof,
+            "kernels": per_kernel,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 2 * launches_per_step * args.steps,  # timed regions A and B together
