@@ -139,6 +139,18 @@ def test_select_ties_nan_negzero():
     assert _select_check(np.zeros(3000, np.float32), (3000,), (0,), (1234,)) == 0  # all equal
 
 
+def test_select_crowded_threshold_bin():
+    """Distinct scores that share their sign, exponent and top mantissa bits fill one bin of
+    the first histogram pass beyond the candidate buffer, so the selection narrows the bin
+    with passes over all keys before it resolves the threshold among few candidates."""
+    g = np.random.default_rng(5)
+    for n, ks in ((60000, (1, 3000, 25000, 59000)), (200000, (4096, 150000))):
+        s = (1.0 + 0.125 * g.random(n)).astype(np.float32)  # every key has the same top 12 bits
+        s[g.random(n) < 0.3] = np.float32(1.0625)              # plus one large tie group inside it
+        for k in ks:
+            assert _select_check(s, (n,), (64,), (k,)) == 0
+
+
 def test_select_many_sequences_chunks_launches():
     g = np.random.default_rng(2)
     B = 150  # more than the 64 descriptors one launch carries
