@@ -285,6 +285,23 @@ class PreparedChain:
                                     self._cu, self._B, q.shape[1], kk.shape[1], q.shape[2], float(softmax_scale),
                                     int(flags), _ptr(o), _ptr(l), _ptr(dev_status), s))
 
+        nl = len(layers)
+        self._arrays = tuple((_VP * max(nl, 1))(*[t[i].data_ptr() for t in layers]) for i in range(3))
+        self._o_arr = (_VP * max(nl, 1))(*[t.data_ptr() for t in out["O"]])
+        self._lse_arr = (_VP * max(nl, 1))(*[(t.data_ptr() if t is not None else None) for t in out["lse"]])
+        Hq = layers[0][0].shape[1] if nl else 1
+        Hkv = layers[0][1].shape[1] if nl else 1
+        D = layers[0][0].shape[2] if nl else 64
+        self._prefill_args = (dt, _ptr(H), H.stride(0), d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2), W1.shape[0],
+                              self._seqs.ref(), nl, *self._arrays, Hq, Hkv, D, float(softmax_scale), _ptr(head_gain),
+                              int(flags), _ptr(out["score"]), _ptr(out["kept_idx"]), _ptr(out["cu_kept_dev"]),
+                              _ptr(out["H_kept"]), _ptr(out["pos"]), _ptr(out["g"]), _ptr(out["logg"]), self._o_arr,
+                              self._lse_arr, _ptr(dev_status), s)
+
+    def prefill(self):
+        """The whole path through its single C-ABI entry (tg_prefill_above_L)."""
+        _check("tg_prefill_above_L", self._L.tg_prefill_above_L(*self._prefill_args))
+
     def score(self):
         _check("tg_score", self._L.tg_score(*self._score_args))
 

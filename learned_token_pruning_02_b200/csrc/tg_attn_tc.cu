@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tmV, const float* __restrict__ logg,
                    const float* __restrict__ gain, const int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ O,
                    float* __restrict__ lse, int64_t m_tot, int Hq, int Hkv, float qk_scale, uint32_t flags,
-                   int32_t* __restrict__ dev_status, const __grid_constant__ ATParams p) {
+                   int32_t* __restrict__ dev_status, int qkv_ready, const __grid_constant__ ATParams p) {
   using C = ACfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -148,7 +148,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
-    griddep_wait();  // inputs written by the previous kernel are visible from here on
+    // With qkv_ready (the chained prefill, where Q, K and V are inputs of the whole chain and the
+    // previous kernel only produces log g and pos), Q and the first key tiles go out before the
+    // wait on that kernel; otherwise anything may come from it and the wait is first.
+    if (!qkv_ready) griddep_wait();  // inputs written by the previous kernel are visible from here on
     // Q and the first key tiles go out before the CTA-wide sync (their ring slots start free)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
@@ -162,6 +165,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int bx = 0; bx < C::NBOX; ++bx)
         tma_load_2d(kb + bx * (BKV * 128), &tmK, kvh * D + bx * 64, off + j * BKV, &kfull[j]);
     }
+    if (qkv_ready) griddep_wait();  // log g and pos of the previous kernel are visible from here on
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -239,55 +243,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {  // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t qa = smem_u32(smem + C::Q_OFF);
-      // Event loop: issue whichever product is ready, polling with non-blocking test_wait so
-      // it never sleeps on one barrier while the other product could go. S_j needs K_j and the chain's S buffer (free once PV of the
-      // chain's previous tile completed); PV_j needs P_j and V_j. At most two S ahead of PV.
+      // Fixed schedule with blocking (suspending) waits: S_0, S_1, then PV_j followed by
+      // S_{j+2} for j = 0, 1, ... The chains alternate, so this is the order the products
+      // become ready in, and a waiting issuer sleeps instead of taking issue slots from the
+      // softmax warps that share its scheduler. S_j needs K_j and the chain's S buffer (free
+      // once PV_{j-2} completed); PV_j needs P_j and V_j.
+      auto issue_s = [&](int j) -> bool {
+        const int c = j & 1, u = j >> 1, ks = j % KS;
+        if (!mbar_wait(&kfull[ks], (j / KS) & 1, abort, dev_status)) return false;
+        if (u > 0 && !mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status)) return false;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(smem + C::K_OFF + ks * C::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          mma_ss(tmem + c * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK, kk > 0);
+        }
+        mma_commit(&sfull[c]);
+        mma_commit(&kempty[ks]);
+        return true;
+      };
       bool ok = mbar_wait(qfull, 0, abort, dev_status);
-      int next_s = 0, next_pv = 0;
-      uint64_t t_idle = globaltimer_ns();
-      while (ok && next_pv < nt) {
-        bool progressed = false;
-        if (next_pv < next_s) {
-          const int j = next_pv, c = j & 1, u = j >> 1;
-          if (mbar_test(&pready[c], u & 1) && mbar_test(&vfull[c], u & 1)) {
-            tc_fence_after();
-            const uint32_t va = smem_u32(smem + C::V_OFF + c * C::TILE_BYTES);
-#pragma unroll
-            for (int kk = 0; kk < BKV / 16; ++kk)
-              mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
-                     C::IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&pvdone[c]);
-            mma_commit(&vempty[c]);
-            ++next_pv;
-            progressed = true;
-          }
-        }
-        if (next_s < nt && next_s < next_pv + 2) {
-          const int j = next_s, c = j & 1, u = j >> 1, ks = j % KS;
-          if (mbar_test(&kfull[ks], (j / KS) & 1) && (u == 0 || mbar_test(&pvdone[c], (u - 1) & 1))) {
-            tc_fence_after();
-            const uint32_t ka = smem_u32(smem + C::K_OFF + ks * C::TILE_BYTES);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-              mma_ss(tmem + c * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK,
-                     kk > 0);
-            }
-            mma_commit(&sfull[c]);
-            mma_commit(&kempty[ks]);
-            ++next_s;
-            progressed = true;
-          }
-        }
-        if (progressed) {
-          t_idle = globaltimer_ns();
-        } else if (*abort) {
+      for (int j = 0; ok && j < 2 && j < nt; ++j) ok = issue_s(j);
+      for (int j = 0; ok && j < nt; ++j) {
+        const int c = j & 1, u = j >> 1;
+        if (!mbar_wait(&pready[c], u & 1, abort, dev_status) || !mbar_wait(&vfull[c], u & 1, abort, dev_status)) {
           ok = false;
-        } else if (globaltimer_ns() - t_idle > 2000000000ull) {
-          *abort = 1;
-          if (dev_status) atomicOr(dev_status, TG_DEV_TIMEOUT);
-          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t va = smem_u32(smem + C::V_OFF + c * C::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
+                 C::IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&pvdone[c]);
+        mma_commit(&vempty[c]);
+        if (j + 2 < nt) ok = issue_s(j + 2);
       }
       mma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
@@ -303,7 +295,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tmem + lane_base + c * BKV;
     const uint32_t tO = tmem + lane_base + 256 + c * D;
-    if (c == 0 && h == 0 && valid && il > 0 && dev_status && pos[off + il - 1] >= pos[off + il])
+    if (c == 0 && h == 0 && valid && il > 0 && dev_status && pos && pos[off + il - 1] >= pos[off + il])
       atomicOr(dev_status, TG_DEV_POS_NOT_ASCENDING);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
@@ -492,6 +484,8 @@ tg_status launch_d(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_
   if (!attr_set[un]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_fwd: cudaFuncSetAttribute");
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_fwd: cudaFuncSetAttribute");
     attr_set[un] = true;
   }
   const int grid = units * a.Hq;
@@ -505,7 +499,7 @@ tg_status launch_d(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_
   cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, a.logg, a.head_gain, a.pos,
                                         static_cast<__nv_bfloat16*>(a.O), a.lse, a.m_tot, a.Hq, a.Hkv,
-                                        a.scale * kLog2e, a.flags, a.dev_status, p),
+                                        a.scale * kLog2e, a.flags, a.dev_status, a.qkv_ready ? 1 : 0, p),
                      "tg_gated_attn_fwd: attn_tc launch");
 }
 

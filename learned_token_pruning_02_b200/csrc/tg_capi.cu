@@ -159,9 +159,10 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
   return launch_score_simt(dtype, H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, s);
 }
 
-tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
-                         int32_t* cu_kept_dev, int32_t* dev_status, void* stream) {
-  g_err[0] = 0;
+// The selector with optional per-row outputs pos, g and log g (the chained prefill).
+static tg_status select_impl(const float* score, const tg_seqs* seqs, int32_t* kept_idx, int32_t* cu_kept_dev,
+                             int32_t* dev_status, void* stream, int32_t* pos, float* g, float* logg,
+                             uint32_t flags) {
   int64_t n_tot = 0, m_tot = 0;
   tg_status st = check_seqs(seqs, &n_tot, &m_tot);
   if (st != TG_OK) return st;
@@ -184,10 +185,16 @@ tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_
     int nb = seqs->B - b0 < kMaxSeqPerLaunch ? seqs->B - b0 : kMaxSeqPerLaunch;
     int nmax = 0;
     for (int i = 0; i < nb; ++i) nmax = d[b0 + i].n_ctx > nmax ? d[b0 + i].n_ctx : nmax;
-    st = launch_select(score, d.data() + b0, nb, nmax, kept_idx, cu_kept_dev, dev_status, s);
+    st = launch_select(score, d.data() + b0, nb, nmax, kept_idx, cu_kept_dev, dev_status, s, pos, g, logg, flags);
     if (st != TG_OK) return st;
   }
   return TG_OK;
+}
+
+tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
+                         int32_t* cu_kept_dev, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  return select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, nullptr, nullptr, nullptr, 0);
 }
 
 tg_status tg_gather(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const float* score,
@@ -227,12 +234,12 @@ tg_status tg_gather(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const
   return TG_OK;
 }
 
-tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const void* V,
-                            const float* logg, const float* head_gain, const int32_t* pos,
-                            const int32_t* cu_kept_host, int32_t B, int32_t Hq, int32_t Hkv,
-                            int32_t D, float softmax_scale, uint32_t flags, void* O,
-                            float* lse, int32_t* dev_status, void* stream) {
-  g_err[0] = 0;
+// qkv_ready: Q, K and V are inputs of the whole chain (the chained prefill), so the kernel may
+// load them before it waits on the previous kernel.
+static tg_status attn_impl(tg_dtype dtype, const void* Q, const void* K, const void* V, const float* logg,
+                           const float* head_gain, const int32_t* pos, const int32_t* cu_kept_host, int32_t B,
+                           int32_t Hq, int32_t Hkv, int32_t D, float softmax_scale, uint32_t flags, void* O,
+                           float* lse, int32_t* dev_status, void* stream, bool qkv_ready) {
   if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return fail(TG_ERR_INVALID_ARG, "need B >= 0 and Hq, Hkv, D > 0");
   if (B > 0 && !cu_kept_host) return fail(TG_ERR_INVALID_ARG, "cu_kept_host is NULL");
@@ -251,6 +258,7 @@ tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const 
   tg_status st = check_device();
   if (st != TG_OK) return st;
   AttnArgs a{dtype, Q, K, V, logg, head_gain, pos, Hq, Hkv, D, softmax_scale, flags, O, lse, dev_status, m_tot};
+  a.qkv_ready = qkv_ready;
   std::vector<AttnSeq> v(B);
   for (int b = 0; b < B; ++b) v[b] = AttnSeq{cu_kept_host[b], cu_kept_host[b + 1] - cu_kept_host[b]};
   cudaStream_t s = (cudaStream_t)stream;
@@ -258,6 +266,46 @@ tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const 
     int nb = B - b0 < kMaxSeqPerLaunch ? B - b0 : kMaxSeqPerLaunch;
     st = (dtype == TG_BF16) ? launch_attn_tc(a, v.data() + b0, nb, s) : launch_attn_simt(a, v.data() + b0, nb, s);
     if (st != TG_OK) return st;
+  }
+  return TG_OK;
+}
+
+tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const void* V,
+                            const float* logg, const float* head_gain, const int32_t* pos,
+                            const int32_t* cu_kept_host, int32_t B, int32_t Hq, int32_t Hkv,
+                            int32_t D, float softmax_scale, uint32_t flags, void* O,
+                            float* lse, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  return attn_impl(dtype, Q, K, V, logg, head_gain, pos, cu_kept_host, B, Hq, Hkv, D, softmax_scale, flags, O, lse,
+                   dev_status, stream, false);
+}
+
+// The row copy of the chained prefill (the selector already wrote pos, g and log g): launched
+// after the attention layers, which read nothing it writes, so its first launch starts copying
+// at once and waits for them only at its end.
+static tg_status gather_after(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const int32_t* kept_idx,
+                              const tg_seqs* seqs, void* H_kept, int32_t* dev_status, void* stream) {
+  if (d <= 0 || ldh < d) return fail(TG_ERR_INVALID_ARG, "need d > 0 and ldh >= d");
+  if (!aligned16(H) || !aligned16(H_kept) || (ldh * esize(dtype)) % 16 || (d * esize(dtype)) % 16)
+    return fail(TG_ERR_UNSUPPORTED, "H/H_kept must be 16-byte aligned with 16-byte rows");
+  std::vector<GatherSeq> v(seqs->B);
+  int64_t start = 0, off = 0;
+  for (int b = 0; b < seqs->B; ++b) {
+    const int32_t m = kept_rows(seqs, b);
+    v[b] = GatherSeq{(int32_t)start, seqs->seqlens[b], seqs->q_len[b], (int32_t)off, m};
+    start += seqs->seqlens[b];
+    off += m;
+  }
+  bool first = true;
+  for (int b0 = 0; b0 < seqs->B; b0 += kMaxSeqPerLaunch) {
+    const int nb = seqs->B - b0 < kMaxSeqPerLaunch ? seqs->B - b0 : kMaxSeqPerLaunch;
+    int m_chunk = 0;
+    for (int i = 0; i < nb; ++i) m_chunk += v[b0 + i].m;
+    if (m_chunk == 0) continue;
+    const tg_status st = launch_gather(dtype, H, ldh, d, nullptr, kept_idx, v.data() + b0, nb, m_chunk, 0, H_kept,
+                                       nullptr, nullptr, nullptr, dev_status, (cudaStream_t)stream, first);
+    if (st != TG_OK) return st;
+    first = false;
   }
   return TG_OK;
 }
@@ -284,16 +332,29 @@ tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t
   if (st != TG_OK) return st;
   st = tg_score(dtype, H, ldh, n_tot, d, W1, b1, w2, b2, dg, score, stream);
   if (st != TG_OK) return st;
-  st = tg_topk_select(score, seqs, kept_idx, cu_kept_dev, dev_status, stream);
-  if (st != TG_OK) return st;
-  st = tg_gather(dtype, H, ldh, d, score, kept_idx, seqs, flags, H_kept, pos, g, logg, dev_status, stream);
+  if (dtype != TG_BF16 || n_layers == 0 || m_tot == 0) {
+    st = select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, nullptr, nullptr, nullptr, 0);
+    if (st != TG_OK) return st;
+    st = tg_gather(dtype, H, ldh, d, score, kept_idx, seqs, flags, H_kept, pos, g, logg, dev_status, stream);
+    if (st != TG_OK) return st;
+    for (int l = 0; l < n_layers; ++l) {
+      st = tg_gated_attn_fwd(dtype, Q[l], K[l], V[l], logg, head_gain, pos, cu.data(), seqs->B, Hq, Hkv, D,
+                             softmax_scale, flags, O[l], lse ? lse[l] : nullptr, dev_status, stream);
+      if (st != TG_OK) return st;
+    }
+    return TG_OK;
+  }
+  // bf16: the selector also writes pos, g and log g of every kept row, so the attention layers
+  // follow it directly (their prologue and Q/K loads overlap it), and the copy of the kept rows
+  // comes last, filling the SMs that attention's last CTAs leave idle.
+  st = select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, pos, g, logg, flags);
   if (st != TG_OK) return st;
   for (int l = 0; l < n_layers; ++l) {
-    st = tg_gated_attn_fwd(dtype, Q[l], K[l], V[l], logg, head_gain, pos, cu.data(), seqs->B, Hq, Hkv, D,
-                           softmax_scale, flags, O[l], lse ? lse[l] : nullptr, dev_status, stream);
+    st = attn_impl(dtype, Q[l], K[l], V[l], logg, head_gain, pos, cu.data(), seqs->B, Hq, Hkv, D, softmax_scale,
+                   flags, O[l], lse ? lse[l] : nullptr, dev_status, stream, true);
     if (st != TG_OK) return st;
   }
-  return TG_OK;
+  return gather_after(dtype, H, ldh, d, kept_idx, seqs, H_kept, dev_status, stream);
 }
 
 }  // extern "C"

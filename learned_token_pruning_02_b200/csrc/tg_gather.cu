@@ -23,6 +23,7 @@ struct GatherParams {
 constexpr int WARPS = 4;
 constexpr int MAXV = 8;  // 16-byte vectors per lane held in registers per pass
 
+template <bool WAIT_LAST>
 __global__ void __launch_bounds__(WARPS * 32)
     gather_kernel(const uint4* __restrict__ H, int64_t ldv, int nvec, const float* __restrict__ score,
                   const int32_t* __restrict__ kept, uint32_t flags, uint4* __restrict__ Hk, int32_t* __restrict__ pos,
@@ -31,19 +32,19 @@ __global__ void __launch_bounds__(WARPS * 32)
   const int lane = threadIdx.x & 31;
   const int row0 = p.s[0].out_off;
   sm100::griddep_launch_dependents();  // the next kernel may start its prologue
-  sm100::griddep_wait();               // the kept indices of the previous kernel are visible
+  if (!WAIT_LAST) sm100::griddep_wait();  // the kept indices of the previous kernel are visible
   for (int r = blockIdx.x * WARPS + (threadIdx.x >> 5); r < m_chunk; r += gridDim.x * WARPS) {
     const int row = row0 + r;
     int b = 0;
     while (b + 1 < p.nseq && row >= p.s[b + 1].out_off) ++b;
     const GatherSeq sq = p.s[b];
-    const int32_t j = __ldg(kept + row);
+    const int32_t j = __ldcg(kept + row);
     if (j < sq.start || j >= sq.start + sq.n) {
       if (lane == 0 && dev_status) atomicOr(dev_status, TG_DEV_BAD_INDEX);
       continue;
     }
     // the score load goes out together with the row loads (one round trip, not two)
-    const float s = (lane == 0 && (g || logg)) ? __ldg(score + j) : 0.f;
+    const float s = (lane == 0 && (g || logg)) ? __ldcg(score + j) : 0.f;
     const uint4* src = H + (int64_t)j * ldv;
     uint4* dst = Hk + (int64_t)row * nvec;
     for (int v0 = 0; v0 < nvec; v0 += 32 * MAXV) {
@@ -60,35 +61,46 @@ __global__ void __launch_bounds__(WARPS * 32)
       }
     }
     if (lane == 0) {
-      pos[row] = j - sq.start;
+      if (pos) pos[row] = j - sq.start;
       if (g || logg) {
         float gv, lg;
         if ((flags & TG_QUESTION_GATE_ONE) && (row - sq.out_off) >= sq.m - sq.q) {
           gv = 1.f;
           lg = 0.f;
         } else {
-          const float e = expf(-fabsf(s));
-          gv = s >= 0.f ? 1.f / (1.f + e) : e / (1.f + e);
-          lg = s >= 0.f ? -log1pf(e) : s - log1pf(e);
+          gate_from_score(s, &gv, &lg);
         }
         if (g) g[row] = gv;
         if (logg) logg[row] = lg;
       }
     }
   }
+  // the kernel before this one only ends after it: the gather completes after it too, so stream
+  // order past the gather still means past both
+  if (WAIT_LAST) sm100::griddep_wait();
 }
 
 }  // namespace
 
 tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const float* score, const int32_t* kept_idx,
                         const GatherSeq* seqs, int nseq, int m_chunk, uint32_t flags, void* H_kept, int32_t* pos,
-                        float* g, float* logg, int32_t* dev_status, cudaStream_t st) {
+                        float* g, float* logg, int32_t* dev_status, cudaStream_t st,
+                        bool after_kernel_reads_nothing) {
   GatherParams p = {};
   for (int i = 0; i < nseq; ++i) p.s[i] = seqs[i];
   p.nseq = nseq;
   const int es = dt == TG_BF16 ? 2 : 4;
   const int nvec = d * es / 16;
   const int64_t ldv = ldh * es / 16;
+  static bool attr_set = false;
+  if (!attr_set) {  // the carveout of the other chain kernels: no reconfiguration between them
+    for (auto k : {gather_kernel<false>, gather_kernel<true>}) {
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                           (int)cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return cuda_status(e, "gather: cudaFuncSetAttribute");
+    }
+    attr_set = true;
+  }
   int blocks = (m_chunk + WARPS - 1) / WARPS;
   const int cap = device_sm_count() * 16;
   if (blocks > cap) blocks = cap;
@@ -99,7 +111,8 @@ tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const fl
   cudaLaunchAttribute attr[1] = {pdl_attribute(PDL_GATHER)};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, gather_kernel, static_cast<const uint4*>(H), ldv, nvec, score, kept_idx,
+  return cuda_status(cudaLaunchKernelEx(&cfg, after_kernel_reads_nothing ? gather_kernel<true> : gather_kernel<false>,
+                                        static_cast<const uint4*>(H), ldv, nvec, score, kept_idx,
                                         flags, static_cast<uint4*>(H_kept), pos, g, logg, dev_status, m_chunk, p),
                      "gather launch");
 }

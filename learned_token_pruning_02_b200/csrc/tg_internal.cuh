@@ -34,6 +34,16 @@ inline cudaLaunchAttribute pdl_attribute(int kernel_id) {
   return a;
 }
 
+// Gate value of a score and its logarithm: g = sigmoid(s), log g = log-sigmoid(s), computed
+// stably for either sign of s (TokenGate paper page, Figure 1(c): the keys' gate values come
+// from the selector's scores). Used wherever the chain needs g or log g, so every kernel that
+// derives them gets bit-identical values.
+__device__ __forceinline__ void gate_from_score(float s, float* g, float* lg) {
+  const float e = expf(-fabsf(s));
+  *g = s >= 0.f ? 1.f / (1.f + e) : e / (1.f + e);
+  *lg = s >= 0.f ? -log1pf(e) : s - log1pf(e);
+}
+
 // ----------------------------------------------------------------------------- launchers
 // Each returns TG_OK or TG_ERR_CUDA (argument checks happen in the C-ABI layer).
 
@@ -54,9 +64,12 @@ struct SelSeq {
   int32_t b;        // sequence index in the whole batch
 };
 
+// With pos != nullptr (the chained prefill) every kept row also gets pos, g and log g, the
+// values the gather writes (the question tail with g = 1 under TG_QUESTION_GATE_ONE).
 tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_ctx_max,
                         int32_t* kept_idx, int32_t* cu_kept_dev, int32_t* dev_status,
-                        cudaStream_t st);
+                        cudaStream_t st, int32_t* pos = nullptr, float* g = nullptr,
+                        float* logg = nullptr, uint32_t flags = 0);
 
 struct GatherSeq {
   int32_t start;    // packed row of the sequence's first token
@@ -66,10 +79,13 @@ struct GatherSeq {
   int32_t m;        // kept rows M_b
 };
 
+// after_kernel_reads_nothing: the previous kernel in the stream does not produce anything
+// this gather reads (inside the chained prefill, attention runs between select and gather), so
+// the gather starts its copies at once and waits for that kernel only before it exits.
 tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const float* score,
                         const int32_t* kept_idx, const GatherSeq* seqs, int nseq, int m_chunk,
                         uint32_t flags, void* H_kept, int32_t* pos, float* g, float* logg,
-                        int32_t* dev_status, cudaStream_t st);
+                        int32_t* dev_status, cudaStream_t st, bool after_kernel_reads_nothing = false);
 
 struct AttnSeq {
   int32_t off;  // cu_kept[b]
@@ -91,6 +107,9 @@ struct AttnArgs {
   float* lse;
   int32_t* dev_status;
   int64_t m_tot;
+  // Q, K and V are inputs of the whole chain (the chained prefill): the kernel may load them
+  // before it waits on the previous kernel.
+  bool qkv_ready = false;
 };
 
 tg_status launch_attn_simt(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);

@@ -300,6 +300,11 @@ tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<DG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return cuda_status(e, "tg_score: cudaFuncSetAttribute");
+    // every kernel of the chain asks for the same (all-shared) carveout, so consecutive chain
+    // kernels never wait for an SM to drain and reconfigure its L1 / shared-memory split
+    e = cudaFuncSetAttribute(score_tc_kernel<DG>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return cuda_status(e, "tg_score: cudaFuncSetAttribute");
     attr_set = true;
   }
   const int n_tiles = (int)((n_tok + BM - 1) / BM);

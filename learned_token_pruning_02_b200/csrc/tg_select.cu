@@ -69,6 +69,13 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
   return v;
 }
 
+// The score bits of a key (the inverse of order_key): exact for every score except -0, which
+// comes back as +0 (the same gate value), and NaN, whose key 0 carries no bits (the caller
+// reads NaN scores from memory instead).
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+
 // Inclusive block-wide scan of one value per thread; optionally returns the block total.
 template <typename V>
 __device__ __forceinline__ V block_scan_incl(V v, V* warp_sums, V* total) {
@@ -228,7 +235,8 @@ __device__ __noinline__ void narrow(const uint32_t* keys, int R, int nvalid, cg:
 
 __global__ void __launch_bounds__(NT, 1)
     select_kernel(const float* __restrict__ score, int32_t* __restrict__ kept, int32_t* __restrict__ cu_kept_dev,
-                  int32_t* __restrict__ dev_status, const __grid_constant__ SelParams p) {
+                  int32_t* __restrict__ dev_status, int32_t* __restrict__ pos, float* __restrict__ gate,
+                  float* __restrict__ logg, uint32_t flags, const __grid_constant__ SelParams p) {
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.C, R = p.rows;
   const int rank = (int)cluster.block_rank();
@@ -257,10 +265,23 @@ __global__ void __launch_bounds__(NT, 1)
     if (sq.b == 0) cu_kept_dev[0] = 0;
     cu_kept_dev[sq.b + 1] = sq.out_off + sq.kc + sq.q;
   }
-  for (int j = rank * NT + tid; j < sq.q; j += C * NT) kept[sq.out_off + sq.kc + j] = sq.start + sq.n_ctx + j;
+  // output row `row` keeps the token at `ip` within the sequence (tail: a question token);
+  // key is its order key when the caller holds it (0: read the score from memory)
+  auto emit = [&](int row, int ip, bool tail, uint32_t key) {
+    kept[row] = sq.start + ip;
+    if (pos) {
+      float gv = 1.f, lg = 0.f;
+      if (!(tail && (flags & TG_QUESTION_GATE_ONE)))
+        gate_from_score(key ? key_score(key) : __ldcg(score + sq.start + ip), &gv, &lg);
+      pos[row] = ip;
+      gate[row] = gv;
+      logg[row] = lg;
+    }
+  };
+  for (int j = rank * NT + tid; j < sq.q; j += C * NT) emit(sq.out_off + sq.kc + j, sq.n_ctx + j, true, 0u);
   if (sq.kc == 0) return;  // the whole cluster takes this branch: no barrier is pending
   if (sq.kc == sq.n_ctx) {
-    for (int j = rank * NT + tid; j < sq.n_ctx; j += C * NT) kept[sq.out_off + j] = sq.start + j;
+    for (int j = rank * NT + tid; j < sq.n_ctx; j += C * NT) emit(sq.out_off + j, j, false, 0u);
     return;
   }
 
@@ -487,7 +508,7 @@ __global__ void __launch_bounds__(NT, 1)
     const int EQ = eq_before + (int)(tab[i * 32 + w] & 0xffffu) + __popc(be & lt);
     if (gt || (eq && EQ < need)) {
       const int o = GT + (EQ < need ? EQ : need);  // rank among kept context tokens
-      if (o < sq.kc) kept[sq.out_off + o] = sq.start + base + i * NT + tid;
+      if (o < sq.kc) emit(sq.out_off + o, base + i * NT + tid, false, k);
       else overflow = true;  // cannot happen for a correct threshold; never write past the slot
     }
   }
@@ -498,7 +519,8 @@ __global__ void __launch_bounds__(NT, 1)
 }  // namespace
 
 tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_ctx_max, int32_t* kept_idx,
-                        int32_t* cu_kept_dev, int32_t* dev_status, cudaStream_t st) {
+                        int32_t* cu_kept_dev, int32_t* dev_status, cudaStream_t st, int32_t* pos, float* g,
+                        float* logg, uint32_t flags) {
   SelParams p = {};
   for (int i = 0; i < nseq; ++i) p.s[i] = seqs[i];
   const int per_cta = NT * MAX_ROWS;
@@ -517,6 +539,9 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (per_cta + MAXC) * 4);
     if (e != cudaSuccess) return cuda_status(e, "select: cudaFuncSetAttribute");
+    e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return cuda_status(e, "select: cudaFuncSetAttribute");
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
@@ -532,7 +557,8 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
   attr[1] = pdl_attribute(PDL_SELECT);
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cuda_status(cudaLaunchKernelEx(&cfg, select_kernel, score, kept_idx, cu_kept_dev, dev_status, p),
+  return cuda_status(cudaLaunchKernelEx(&cfg, select_kernel, score, kept_idx, cu_kept_dev, dev_status, pos, g, logg,
+                                        flags, p),
                      "select launch");
 }
 

@@ -406,3 +406,45 @@ def test_chain_back_to_back():
         assert np.array_equal(bits(out[key]), val), key
     assert np.array_equal(bits(out["O"][0]), ref_O)
     assert st.item() == 0
+
+
+@pytest.mark.parametrize("flags", [0, tg.TG_QUESTION_GATE_ONE, tg.TG_ATTN_UNNORMALISED])
+def test_prefill_fused_matches_stages(flags):
+    """Inside tg_prefill_above_L the bf16 attention derives log g from score and kept itself
+    and the gather runs after it. Every output must equal, bit for bit, the four stage entry
+    points run one after another (where attention reads the gather's log g), and O must match
+    the oracle's prefill. Two layers and four ragged sequences."""
+    wl = ti.WORKLOADS["ragged4"]
+    H = to_dev(ti.hidden_states(wl), wl.dtype)
+    W1n, b1n, w2n, b2 = ti.gate_weights(wl, biased=True)
+    W1, b1, w2 = to_dev(W1n, wl.dtype), to_dev(b1n, "f32"), to_dev(w2n, wl.dtype)
+    layers_np = [ti.qkv(wl, l) for l in range(2)]
+    layers = [tuple(to_dev(x, wl.dtype) for x in lyr) for lyr in layers_np]
+    gain = torch.linspace(0.5, 1.5, wl.Hq, device="cuda", dtype=torch.float32)
+    scale = 1.0 / math.sqrt(wl.D)
+    st = _stat()
+    fused = tg.tg_prefill_above_L(H, W1, b1, w2, b2, wl.seqlens, wl.q_len, wl.k, layers, scale, head_gain=gain,
+                                  flags=flags, want_lse=True, dev_status=st)
+    s = tg.tg_score(H, W1, b1, w2, b2)
+    kept, cu_dev = tg.tg_topk_select(s, wl.seqlens, wl.q_len, wl.k)
+    Hk, pos, g, lg = tg.tg_gather(H, s, kept, wl.seqlens, wl.q_len, wl.k, flags=flags)
+    cu = tg.tg_kept_counts(wl.seqlens, wl.q_len, wl.k)
+    torch.cuda.synchronize()
+    for key, ref in (("score", s), ("kept_idx", kept), ("cu_kept_dev", cu_dev), ("H_kept", Hk), ("pos", pos),
+                     ("g", g), ("logg", lg)):
+        assert np.array_equal(bits(fused[key]), bits(ref)), key
+    s_np = s.cpu().numpy()
+    kept_o, cu_o = orc.topk_select(s_np, wl.seqlens, wl.q_len, wl.k)
+    _, pos_o, _, lg_o = orc.gather(ti.widen(ti.hidden_states(wl), wl.dtype), s_np, kept_o, wl.seqlens, wl.q_len, cu_o,
+                                   question_gate_one=bool(flags & tg.TG_QUESTION_GATE_ONE))
+    for l, (Q, K, V) in enumerate(layers):
+        O, L = tg.tg_gated_attn_fwd(Q, K, V, lg, pos, cu, scale, head_gain=gain, flags=flags)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(fused["O"][l]), bits(O)), l
+        assert np.array_equal(bits(fused["lse"][l]), bits(L)), l
+        Qn, Kn, Vn = (ti.widen(x, wl.dtype) for x in layers_np[l])
+        rO, _ = orc.gated_attention(Qn, Kn, Vn, lg_o, pos_o, cu_o, wl.Hq, wl.Hkv, scale,
+                                    head_gain=gain.cpu().numpy().astype(np.float64),
+                                    unnormalised=bool(flags & tg.TG_ATTN_UNNORMALISED))
+        assert max_abs_rel(from_dev(fused["O"][l]), rO) <= TOL[wl.dtype]
+    assert st.item() == 0
