@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-full-ref", action="store_true")
+    ap.add_argument("--no-bw", action="store_true", help="skip the byte-heavy select/gather instances")
+    ap.add_argument("--bw-only", action="store_true", help="run only the byte-heavy select/gather instances")
+    ap.add_argument("--bw-reps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -200,6 +203,61 @@ def traffic_from_profile(kernel_key, src_hash):
     return None
 
 
+def bandwidth_instances(tg, torch, dev, peak_gbs, reps):
+    """Select and gather on byte-heavy shapes, with the same kernels and entry points, to show
+    their bandwidth where the bench workload is latency-bound: select over 64 sequences of
+    131072 seeded N(0,1) scores (question tail 256, K=4096 each; 33.5 MB read) and a gather of
+    65536 of 131072 rows of d=2048 bf16 (537 MB moved). L2 is flushed before every launch; each
+    launch is timed alone with CUDA events on its stream."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20260)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            torch.cuda._sleep(100_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        return sum(ts) / len(ts)
+
+    out = {"l2": "flushed before every launch (512 MiB memset)", "peak_gbs": peak_gbs}
+    B, N, q, K = 64, 131072, 256, 4096
+    seqlens, q_len, k = (N,) * B, (q,) * B, (K,) * B
+    sc = torch.randn(B * N, device=dev, generator=gen, dtype=torch.float32)
+    m_tot = tg.tg_kept_counts(seqlens, q_len, k)[-1]
+    kept = torch.empty(m_tot, device=dev, dtype=torch.int32)
+    cu_dev = torch.empty(B + 1, device=dev, dtype=torch.int32)
+    t = timed(lambda: tg.tg_topk_select(sc, seqlens, q_len, k, kept_idx=kept, cu_kept_dev=cu_dev))
+    byts = B * (N - q) * 4 + m_tot * 4
+    out["select"] = {"shape": f"{B} sequences x {N} tokens, question tail {q}, K={K}", "bytes": byts,
+                     "us": t * 1e6, "gbs": byts / t / 1e9, "frac": byts / t / 1e9 / peak_gbs}
+    del sc, kept
+    N, d, q = 131072, 2048, 256
+    K = 65536 - q
+    H = torch.randn(N, d, device=dev, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+    s1 = torch.randn(N, device=dev, generator=gen, dtype=torch.float32)
+    kept, _ = tg.tg_topk_select(s1, (N,), (q,), (K,))
+    M = kept.numel()
+    Hk = torch.empty(M, d, device=dev, dtype=torch.bfloat16)
+    pos = torch.empty(M, device=dev, dtype=torch.int32)
+    g = torch.empty(M, device=dev, dtype=torch.float32)
+    lg = torch.empty(M, device=dev, dtype=torch.float32)
+    t = timed(lambda: tg.tg_gather(H, s1, kept, (N,), (q,), (K,), H_kept=Hk, pos=pos, g=g, logg=lg))
+    byts = 2 * M * d * 2 + 16 * M
+    out["gather"] = {"shape": f"{M} of {N} rows, d={d} bf16", "bytes": byts, "us": t * 1e6,
+                     "gbs": byts / t / 1e9, "frac": byts / t / 1e9 / peak_gbs}
+    return out
+
+
 def run_reference(args, wl):
     import numpy as np
 
@@ -283,6 +341,15 @@ def main():
     def barrier():
         if world > 1:
             dist.barrier()
+
+    if args.bw_only:
+        pk, _ = peaks()
+        bw = bandwidth_instances(tg, torch, dev, pk["hbm_gbs"], args.bw_reps)
+        if rank == 0:
+            print(json.dumps({"bandwidth_instances": bw}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     def bf(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
@@ -472,6 +539,12 @@ def main():
                     "note": "unpruned causal attention over all N tokens (g == 1), same kernel"}
         del q, k, v, o
 
+    # ---------------- byte-heavy select/gather instances (bandwidth evidence)
+    bw = None
+    if not args.no_bw:
+        barrier()
+        bw = bandwidth_instances(tg, torch, dev, pk["hbm_gbs"], args.bw_reps)
+
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -498,6 +571,7 @@ def main():
             "stages_sum_us": float(stage_ms.sum() * 1e3),
             "clocks": clk,
             "full_attention_reference": full_ref,
+            "bandwidth_instances": bw,
             "device_status": dev_status,
         }
         print(json.dumps(line), flush=True)
