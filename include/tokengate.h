@@ -161,12 +161,16 @@ tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const 
                             float* lse, int32_t* dev_status, void* stream);
 
 /* The whole gated path above layer L (aitualizate.com TokenGate article, phases 2-3;
- * thelatestinai.com TokenGate page, Figure 1(a)): tg_score -> tg_topk_select -> tg_gather
- * -> tg_gated_attn_fwd for each of n_layers above-L layers, enqueued on one stream with no
- * host synchronisation. Q, K, V, O, lse are HOST arrays of n_layers device pointers shaped
- * as in tg_gated_attn_fwd (lse may be NULL, or hold NULL entries). The other arguments and
- * outputs are those of the single steps; score, kept_idx, H_kept, pos, g, logg are all
- * required here. */
+ * thelatestinai.com TokenGate page, Figure 1(a)): the results of tg_score -> tg_topk_select
+ * -> tg_gather -> tg_gated_attn_fwd for each of n_layers above-L layers, enqueued on one
+ * stream with no host synchronisation. Q, K, V, O, lse are HOST arrays of n_layers device
+ * pointers shaped as in tg_gated_attn_fwd (lse may be NULL, or hold NULL entries). The other
+ * arguments and outputs are those of the single steps; score, kept_idx, H_kept, pos, g, logg
+ * are all required here. Every output is bit-identical to running the single steps in that
+ * order. For bf16 with n_layers >= 1 the kernels run in another order: the selector also
+ * writes pos, g and log g, the attention layers follow it, and the copy of the kept rows into
+ * H_kept comes last (it overlaps the attention's tail). Q, K and V must therefore not alias
+ * any output of this call. */
 tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t d,
                              const void* W1, const float* b1, const void* w2, float b2,
                              int32_t dg, const tg_seqs* seqs, int32_t n_layers,
