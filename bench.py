@@ -258,6 +258,48 @@ def bandwidth_instances(tg, torch, dev, peak_gbs, reps):
     return out
 
 
+def split_select_times(tg, torch, dev, reps):
+    """The sequence-split selection's two device steps for one 131072-token sequence cut into 8
+    blocks, K=4096: one rank's top-k candidates of its 16352-token block, and the merge of the
+    8 x 4096 gathered candidates (the all-gather between devices is not part of this run)."""
+    from learned_token_pruning_02_b200 import split
+
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20261)
+    world, n_ctx, q, k = 8, 131072 - 256, 256, 4096
+    s = torch.randn(n_ctx + q, device=dev, generator=gen, dtype=torch.float32)
+    lo, hi = split.block_bounds(n_ctx, world, 0)
+    counts = split.candidate_counts(n_ctx, world, k)
+    cs = torch.empty(world * k, device=dev, dtype=torch.float32)
+    ci = torch.empty(world * k, device=dev, dtype=torch.int32)
+    for r in range(world):
+        a, b = split.block_bounds(n_ctx, world, r)
+        tg.tg_topk_candidates(s[a:b], k, base=a, cand_score=cs[r * k:(r + 1) * k], cand_idx=ci[r * k:(r + 1) * k])
+    kept = torch.empty(k + q, device=dev, dtype=torch.int32)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(reps):
+            torch.cuda._sleep(100_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1) * 1e3
+        return tot / reps
+
+    c_us = timed(lambda: tg.tg_topk_candidates(s[lo:hi], k, base=lo, cand_score=cs[:k], cand_idx=ci[:k]))
+    m_us = timed(lambda: tg.tg_topk_merge(cs, ci, k, n_ctx, q, kept_idx=kept))
+    whole, _ = tg.tg_topk_select(s, (n_ctx + q,), (q,), (k,))
+    torch.cuda.synchronize()
+    return {"shape": f"{n_ctx + q} tokens (question tail {q}) over {world} blocks, K={k}",
+            "candidates_us": c_us, "merge_us": m_us, "equals_whole_sequence_select": bool(torch.equal(kept, whole))}
+
+
 def run_reference(args, wl):
     import numpy as np
 
@@ -585,6 +627,8 @@ def main():
         barrier()
         bw = bandwidth_instances(tg, torch, dev, pk["hbm_gbs"], args.bw_reps)
 
+    split_t = split_select_times(tg, torch, dev, 20) if not args.no_bw else None
+
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -614,6 +658,7 @@ def main():
             "full_attention_reference": full_ref,
             "bandwidth_instances": bw,
             "graph_replay": graph,
+            "split_select": split_t,
             "device_status": dev_status,
         }
         print(json.dumps(line), flush=True)

@@ -118,6 +118,26 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
 tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
                          int32_t* cu_kept_dev, int32_t* dev_status, void* stream);
 
+/* Sequence-split selection across devices, step 1 (one contiguous block of a sequence's
+ * context per device; the merge below is step 2). The min(k, n) tokens of the block with the
+ * largest scores, ordered by position, as candidates: cand_idx = base + position in the block
+ * and cand_score = that token's score (bit for bit). Every token of the sequence's top-k that
+ * lies in this block is among them. Same order and ties as tg_topk_select.
+ *   score       device f32 [n]: the block's scores
+ *   cand_score  device f32 [min(k, n)] (written);  cand_idx device int32 [min(k, n)] (written)
+ * Supported: n <= TG_MAX_CTX. NaN scores set TG_DEV_NAN_SCORE. */
+tg_status tg_topk_candidates(const float* score, int32_t n, int32_t k, int32_t base, float* cand_score,
+                             int32_t* cand_idx, int32_t* dev_status, void* stream);
+
+/* Step 2: the top-k among the candidates of all blocks, concatenated in block order (so
+ * position order is index order and ties keep the lower index), followed by the q question-
+ * tail indices q_start .. q_start+q-1. The result equals tg_topk_select over the whole
+ * sequence. Candidates must all be real: a block with fewer than k tokens contributes fewer.
+ *   kept_idx  device int32 [min(k, n_cand) + q] (written), ascending context indices first
+ * Supported: n_cand <= TG_MAX_CTX. */
+tg_status tg_topk_merge(const float* cand_score, const int32_t* cand_idx, int32_t n_cand, int32_t k,
+                        int32_t q_start, int32_t q, int32_t* kept_idx, int32_t* dev_status, void* stream);
+
 /* Forward the kept hidden states with their gate values and positions (thelatestinai.com
  * TokenGate page, Figure 1(b): the selector forwards the kept hidden states together with
  * their importance scores; aitualizate.com article, phase 3).

@@ -28,6 +28,8 @@ TG_MAX_CTX = 262144
 EXPORTS = (
     "tg_status_string", "tg_last_error", "tg_version", "tg_kept_counts", "tg_score",
     "tg_topk_select", "tg_gather", "tg_gated_attn_fwd", "tg_prefill_above_L",
+    "tg_topk_candidates",
+    "tg_topk_merge",
 )
 
 
@@ -76,6 +78,10 @@ def lib() -> ctypes.CDLL:
     L.tg_score.argtypes = [_I32, _VP, _I64, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP]
     L.tg_topk_select.restype = _I32
     L.tg_topk_select.argtypes = [_VP, _SEQP, _VP, _VP, _VP, _VP]
+    L.tg_topk_candidates.restype = _I32
+    L.tg_topk_candidates.argtypes = [_VP, _I32, _I32, _I32, _VP, _VP, _VP, _VP]
+    L.tg_topk_merge.restype = _I32
+    L.tg_topk_merge.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _VP, _VP, _VP]
     L.tg_gather.restype = _I32
     L.tg_gather.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _SEQP, _U32, _VP, _VP, _VP, _VP, _VP, _VP]
     L.tg_gated_attn_fwd.restype = _I32
@@ -169,6 +175,32 @@ def tg_topk_select(score, seqlens, q_len, k, kept_idx=None, cu_kept_dev=None, de
     _check("tg_topk_select", lib().tg_topk_select(_ptr(score), s.ref(), _ptr(kept_idx), _ptr(cu_kept_dev),
                                                   _ptr(dev_status), _stream(stream)))
     return kept_idx, cu_kept_dev
+
+
+def tg_topk_candidates(score, k: int, base: int = 0, cand_score=None, cand_idx=None, dev_status=None, stream=None):
+    """Top-k of one block of a sequence's context as (cand_score, cand_idx = base + position)."""
+    _cuda(score, cand_score, cand_idx, dev_status)
+    n = score.numel()
+    kc = min(int(k), n)
+    if cand_score is None:
+        cand_score = torch.empty(kc, device=score.device, dtype=torch.float32)
+    if cand_idx is None:
+        cand_idx = torch.empty(kc, device=score.device, dtype=torch.int32)
+    _check("tg_topk_candidates", lib().tg_topk_candidates(_ptr(score), n, int(k), int(base), _ptr(cand_score),
+                                                          _ptr(cand_idx), _ptr(dev_status), _stream(stream)))
+    return cand_score, cand_idx
+
+
+def tg_topk_merge(cand_score, cand_idx, k: int, q_start: int, q: int, kept_idx=None, dev_status=None, stream=None):
+    """Top-k of candidates concatenated in block order, then the question tail q_start..q_start+q-1."""
+    _cuda(cand_score, cand_idx, kept_idx, dev_status)
+    n = cand_score.numel()
+    m = min(int(k), n) + int(q)
+    if kept_idx is None:
+        kept_idx = torch.empty(m, device=cand_score.device, dtype=torch.int32)
+    _check("tg_topk_merge", lib().tg_topk_merge(_ptr(cand_score), _ptr(cand_idx), n, int(k), int(q_start), int(q),
+                                                _ptr(kept_idx), _ptr(dev_status), _stream(stream)))
+    return kept_idx
 
 
 def tg_gather(H, score, kept_idx, seqlens, q_len, k, flags=0, H_kept=None, pos=None, g=None, logg=None,

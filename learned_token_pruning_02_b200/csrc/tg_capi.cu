@@ -176,7 +176,7 @@ static tg_status select_impl(const float* score, const tg_seqs* seqs, int32_t* k
   for (int b = 0; b < seqs->B; ++b) {
     int32_t N = seqs->seqlens[b], q = seqs->q_len[b];
     int32_t m = kept_rows(seqs, b);
-    d[b] = SelSeq{(int32_t)start, N - q, q, m - q, (int32_t)off, b};
+    d[b] = SelSeq{(int32_t)start, N - q, q, m - q, (int32_t)off, b, (int32_t)(start + N - q), (int32_t)start};
     start += N;
     off += m;
   }
@@ -195,6 +195,37 @@ tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_
                          int32_t* cu_kept_dev, int32_t* dev_status, void* stream) {
   g_err[0] = 0;
   return select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, nullptr, nullptr, nullptr, 0);
+}
+
+tg_status tg_topk_candidates(const float* score, int32_t n, int32_t k, int32_t base, float* cand_score,
+                             int32_t* cand_idx, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  if (n < 0 || k < 0 || base < 0) return fail(TG_ERR_INVALID_ARG, "need n, k, base >= 0");
+  if (n > TG_MAX_CTX) return fail(TG_ERR_UNSUPPORTED, "block of %d tokens exceeds TG_MAX_CTX", n);
+  const int32_t kc = k < n ? k : n;
+  if (kc == 0) return TG_OK;
+  if (!score || !cand_score || !cand_idx) return fail(TG_ERR_INVALID_ARG, "score, cand_score and cand_idx are required");
+  tg_status st = check_device();
+  if (st != TG_OK) return st;
+  const SelSeq d{0, n, 0, kc, 0, 0, n, base};
+  return launch_select(score, &d, 1, n, cand_idx, nullptr, dev_status, (cudaStream_t)stream, nullptr, nullptr,
+                       nullptr, 0, nullptr, cand_score);
+}
+
+tg_status tg_topk_merge(const float* cand_score, const int32_t* cand_idx, int32_t n_cand, int32_t k,
+                        int32_t q_start, int32_t q, int32_t* kept_idx, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  if (n_cand < 0 || k < 0 || q < 0 || q_start < 0) return fail(TG_ERR_INVALID_ARG, "need n_cand, k, q, q_start >= 0");
+  if (n_cand > TG_MAX_CTX) return fail(TG_ERR_UNSUPPORTED, "%d candidates exceed TG_MAX_CTX", n_cand);
+  const int32_t kc = k < n_cand ? k : n_cand;
+  if (kc + q == 0) return TG_OK;
+  if (!kept_idx || (n_cand > 0 && (!cand_score || !cand_idx)))
+    return fail(TG_ERR_INVALID_ARG, "kept_idx (and cand_score, cand_idx) are required");
+  tg_status st = check_device();
+  if (st != TG_OK) return st;
+  const SelSeq d{0, n_cand, q, kc, 0, 0, q_start, 0};
+  return launch_select(cand_score, &d, 1, n_cand, kept_idx, nullptr, dev_status, (cudaStream_t)stream, nullptr,
+                       nullptr, nullptr, 0, cand_idx, nullptr);
 }
 
 tg_status tg_gather(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const float* score,

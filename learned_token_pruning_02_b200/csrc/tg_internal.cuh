@@ -62,14 +62,20 @@ struct SelSeq {
   int32_t kc;       // context tokens to keep, min(max(k,0), n_ctx)
   int32_t out_off;  // first output row (cu_kept[b])
   int32_t b;        // sequence index in the whole batch
+  int32_t tail;     // index written for the first question-tail token (normally start + n_ctx)
+  int32_t wbase;    // index written for context position 0 (normally start)
 };
 
 // With pos != nullptr (the chained prefill) every kept row also gets pos, g and log g, the
 // values the gather writes (the question tail with g = 1 under TG_QUESTION_GATE_ONE).
+// With idxmap != nullptr a kept context position p writes idxmap[start + p] instead of
+// start + p, and with kept_score != nullptr each kept context row also gets its score (the
+// split selection across devices: candidates, then their merge).
 tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_ctx_max,
                         int32_t* kept_idx, int32_t* cu_kept_dev, int32_t* dev_status,
                         cudaStream_t st, int32_t* pos = nullptr, float* g = nullptr,
-                        float* logg = nullptr, uint32_t flags = 0);
+                        float* logg = nullptr, uint32_t flags = 0, const int32_t* idxmap = nullptr,
+                        float* kept_score = nullptr);
 
 struct GatherSeq {
   int32_t start;    // packed row of the sequence's first token

@@ -236,7 +236,8 @@ __device__ __noinline__ void narrow(const uint32_t* keys, int R, int nvalid, cg:
 __global__ void __launch_bounds__(NT, 1)
     select_kernel(const float* __restrict__ score, int32_t* __restrict__ kept, int32_t* __restrict__ cu_kept_dev,
                   int32_t* __restrict__ dev_status, int32_t* __restrict__ pos, float* __restrict__ gate,
-                  float* __restrict__ logg, uint32_t flags, const __grid_constant__ SelParams p) {
+                  float* __restrict__ logg, uint32_t flags, const int32_t* __restrict__ idxmap,
+                  float* __restrict__ kept_score, const __grid_constant__ SelParams p) {
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.C, R = p.rows;
   const int rank = (int)cluster.block_rank();
@@ -268,7 +269,8 @@ __global__ void __launch_bounds__(NT, 1)
   // output row `row` keeps the token at `ip` within the sequence (tail: a question token);
   // key is its order key when the caller holds it (0: read the score from memory)
   auto emit = [&](int row, int ip, bool tail, uint32_t key) {
-    kept[row] = sq.start + ip;
+    kept[row] = tail ? sq.tail + (ip - sq.n_ctx) : (idxmap ? __ldcg(idxmap + sq.start + ip) : sq.wbase + ip);
+    if (kept_score && !tail) kept_score[row] = key ? key_score(key) : __ldcg(score + sq.start + ip);
     if (pos) {
       float gv = 1.f, lg = 0.f;
       if (!(tail && (flags & TG_QUESTION_GATE_ONE)))
@@ -280,8 +282,14 @@ __global__ void __launch_bounds__(NT, 1)
   };
   for (int j = rank * NT + tid; j < sq.q; j += C * NT) emit(sq.out_off + sq.kc + j, sq.n_ctx + j, true, 0u);
   if (sq.kc == 0) return;  // the whole cluster takes this branch: no barrier is pending
-  if (sq.kc == sq.n_ctx) {
-    for (int j = rank * NT + tid; j < sq.n_ctx; j += C * NT) emit(sq.out_off + j, j, false, 0u);
+  if (sq.kc == sq.n_ctx) {  // every context token is kept; NaN scores are still reported
+    bool nan = false;
+    for (int j = rank * NT + tid; j < sq.n_ctx; j += C * NT) {
+      const float v = __ldcg(score + sq.start + j);
+      nan |= v != v;
+      emit(sq.out_off + j, j, false, 0u);
+    }
+    if (nan && dev_status) atomicOr(dev_status, TG_DEV_NAN_SCORE);
     return;
   }
 
@@ -520,7 +528,7 @@ __global__ void __launch_bounds__(NT, 1)
 
 tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_ctx_max, int32_t* kept_idx,
                         int32_t* cu_kept_dev, int32_t* dev_status, cudaStream_t st, int32_t* pos, float* g,
-                        float* logg, uint32_t flags) {
+                        float* logg, uint32_t flags, const int32_t* idxmap, float* kept_score) {
   SelParams p = {};
   for (int i = 0; i < nseq; ++i) p.s[i] = seqs[i];
   const int per_cta = NT * MAX_ROWS;
@@ -566,7 +574,7 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cuda_status(cudaLaunchKernelEx(&cfg, select_kernel, score, kept_idx, cu_kept_dev, dev_status, pos, g, logg,
-                                        flags, p),
+                                        flags, idxmap, kept_score, p),
                      "select launch");
 }
 

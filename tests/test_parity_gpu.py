@@ -137,6 +137,9 @@ def test_select_ties_nan_negzero():
         st = _select_check(s, (n,), (100,), (k,))
         assert st & tg.TG_DEV_NAN_SCORE
     assert _select_check(np.zeros(3000, np.float32), (3000,), (0,), (1234,)) == 0  # all equal
+    s = g.standard_normal(600).astype(np.float32)
+    s[[5, 77]] = np.nan
+    assert _select_check(s, (600,), (10,), (590,)) & tg.TG_DEV_NAN_SCORE  # every context token kept
 
 
 def test_select_crowded_threshold_bin():
