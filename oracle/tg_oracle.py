@@ -24,6 +24,10 @@ leave a step open, the reading taken is stated in the function's docstring:
     "unnormalised" variant multiplies the weight by g_j without renormalising;
   * causal mask on original positions (key allowed iff pos_j <= pos_i, same sequence);
     grouped KV heads map query head h to KV head h // (Hq / Hkv).
+  * above-L projections (not on the pages, which stop at "layers above L process the kept
+    tokens"): Q/K/V = kept rows times one stacked projection matrix, with rotary position
+    embedding on Q and K at each kept token's original position, rotate-half pairing
+    (i, i + D/2) and inverse frequencies theta^(-2i/D).
 
 Every function is pinned by tests/test_oracle_pins.py against closed forms, textbook
 values, brute force and invariants. Parity is unpinned for nothing in this file.
@@ -250,3 +254,38 @@ def prefill_from_scores(H, s, seqlens, q_len, k, layers, Hq, Hkv, scale, head_ga
             for (Q, Kt, V) in layers]
     return {"score": s, "kept": kept, "cu_kept": cu, "H_kept": Hk, "pos": pos, "g": g,
             "logg": logg, "attn": outs}
+
+
+# --------------------------------------------------------------------------- above L: projections
+
+
+def rope(x, pos, theta):
+    """Rotary position embedding of x [M, H, D] at integer positions pos [M].
+
+    Rotate-half pairing: for i < D/2 with angle a = pos * theta**(-2 i / D),
+    y[i] = x[i] cos a - x[i + D/2] sin a and y[i + D/2] = x[i + D/2] cos a + x[i] sin a.
+    The pages give no projection or rotary details; this is the plainest reading of "original
+    position ids" for the layers above L. theta <= 0 means no rotation.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if theta <= 0:
+        return x.copy()
+    D = x.shape[-1]
+    half = D // 2
+    inv = float(theta) ** (-2.0 * np.arange(half, dtype=np.float64) / D)
+    a = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]  # [M, D/2]
+    c, s = np.cos(a)[:, None, :], np.sin(a)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def qkv_rope(Hk, W, pos, Hq, Hkv, D, theta):
+    """Q, K, V of the kept rows: X = Hk W^T with W [(Hq + 2 Hkv) D, d] (output-major, like
+    torch.nn.Linear.weight), split into Q [M, Hq, D], K [M, Hkv, D], V [M, Hkv, D]; Q and K
+    rotated by rope() at pos. float64."""
+    X = np.asarray(Hk, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T
+    M = X.shape[0]
+    Q = X[:, : Hq * D].reshape(M, Hq, D)
+    K = X[:, Hq * D: (Hq + Hkv) * D].reshape(M, Hkv, D)
+    V = X[:, (Hq + Hkv) * D:].reshape(M, Hkv, D)
+    return rope(Q, pos, theta), rope(K, pos, theta), V

@@ -373,3 +373,47 @@ def test_planted_spans_are_kept_when_salient():
     kept, _ = orc.topk_select(s, wl.seqlens, wl.q_len, wl.k)
     frac = m[kept[:409]].mean()
     assert frac > 0.8  # +3 sigma offsets dominate the kept set
+
+
+# ---------------------------------------------------------------- rotary embedding / QKV projection
+
+
+def test_rope_hand_values_fix_pairing_and_frequencies():
+    # D = 4: pairs (0, 2) and (1, 3); frequencies theta^0 = 1 and theta^(-1/2) = 0.01 for theta 1e4
+    x = np.array([[[1.0, 2.0, 3.0, 4.0]]])
+    y = orc.rope(x, [1], 1.0e4)[0, 0]
+    c1, s1, c2, s2 = math.cos(1.0), math.sin(1.0), math.cos(0.01), math.sin(0.01)
+    want = [1 * c1 - 3 * s1, 2 * c2 - 4 * s2, 3 * c1 + 1 * s1, 4 * c2 + 2 * s2]
+    assert np.allclose(y, want, rtol=0, atol=1e-15)
+
+
+def test_rope_identity_norm_and_relative_position():
+    g = np.random.default_rng(3)
+    x = g.standard_normal((5, 3, 16))
+    assert np.array_equal(orc.rope(x, [0] * 5, 1.0e6), x)  # position 0 rotates nothing
+    assert np.array_equal(orc.rope(x, [7] * 5, 0.0), x)    # theta <= 0: no rotation
+    y = orc.rope(x, [3, 100, 4097, 65535, 131071], 1.0e6)
+    n0 = x[..., :8] ** 2 + x[..., 8:] ** 2
+    n1 = y[..., :8] ** 2 + y[..., 8:] ** 2
+    assert np.allclose(n0, n1, rtol=1e-12)                # each pair keeps its length
+    q, k = g.standard_normal((1, 1, 16)), g.standard_normal((1, 1, 16))
+    for m, n, t in ((5, 2, 11), (1000, 10, 777), (0, 0, 4096)):
+        d0 = np.sum(orc.rope(q, [m], 1.0e4) * orc.rope(k, [n], 1.0e4))
+        d1 = np.sum(orc.rope(q, [m + t], 1.0e4) * orc.rope(k, [n + t], 1.0e4))
+        assert abs(d0 - d1) < 1e-9                        # depends on m - n only
+
+
+def test_qkv_rope_split_and_projection():
+    g = np.random.default_rng(4)
+    M, d, Hq, Hkv, D = 6, 32, 4, 2, 8
+    Hk = g.standard_normal((M, d))
+    W = g.standard_normal(((Hq + 2 * Hkv) * D, d))
+    pos = np.array([0, 1, 2, 50, 51, 9])
+    Q, K, V = orc.qkv_rope(Hk, W, pos, Hq, Hkv, D, 1.0e4)
+    X = np.array([[sum(Hk[i, c] * W[o, c] for c in range(d)) for o in range(W.shape[0])] for i in range(M)])
+    assert np.allclose(V, X[:, (Hq + Hkv) * D:].reshape(M, Hkv, D), atol=1e-12)  # V is not rotated
+    assert np.allclose(Q[0], X[0, : Hq * D].reshape(Hq, D), atol=1e-12)          # row at position 0
+    q3 = X[3, : Hq * D].reshape(1, Hq, D)
+    assert np.allclose(Q[3], orc.rope(q3, [50], 1.0e4)[0], atol=1e-12)
+    k4 = X[4, Hq * D: (Hq + Hkv) * D].reshape(1, Hkv, D)
+    assert np.allclose(K[4], orc.rope(k4, [51], 1.0e4)[0], atol=1e-12)

@@ -451,3 +451,41 @@ def test_prefill_fused_matches_stages(flags):
                                     unnormalised=bool(flags & tg.TG_ATTN_UNNORMALISED))
         assert max_abs_rel(from_dev(fused["O"][l]), rO) <= TOL[wl.dtype]
     assert st.item() == 0
+
+
+def test_prefill_many_sequences_chunked():
+    """More sequences than one launch carries: the chained prefill splits the selector, the
+    attention layers and the trailing row copy into several launches each. Every output must
+    equal the stage-by-stage results bit for bit (bf16, small shapes, two layers)."""
+    g = np.random.default_rng(11)
+    B, d, dg, Hq, Hkv, D = 70, 256, 64, 4, 2, 64
+    seqlens = tuple(int(x) for x in g.integers(1, 400, B))
+    q_len = tuple(int(g.integers(0, min(n, 40) + 1)) for n in seqlens)
+    k = tuple(int(x) for x in g.integers(0, 200, B))
+    n_tot = sum(seqlens)
+    H = to_dev(ti.f32_to_bf16_bits((g.standard_normal((n_tot, d)) / 4).astype(np.float32)), "bf16")
+    W1 = to_dev(ti.f32_to_bf16_bits((g.standard_normal((dg, d)) / 16).astype(np.float32)), "bf16")
+    w2 = to_dev(ti.f32_to_bf16_bits((g.standard_normal(dg) / 8).astype(np.float32)), "bf16")
+    b1 = to_dev((g.standard_normal(dg) / 10).astype(np.float32), "f32")
+    cu = tg.tg_kept_counts(seqlens, q_len, k)
+    M = cu[-1]
+    layers = [tuple(to_dev(ti.f32_to_bf16_bits((g.standard_normal((M, h, D)) / math.sqrt(D)).astype(np.float32)), "bf16")
+                    for h in (Hq, Hkv, Hkv)) for _ in range(2)]
+    scale = 1.0 / math.sqrt(D)
+    st = _stat()
+    fused = tg.tg_prefill_above_L(H, W1, b1, w2, 0.05, seqlens, q_len, k, layers, scale, want_lse=True, dev_status=st)
+    s = tg.tg_score(H, W1, b1, w2, 0.05)
+    kept, cu_dev = tg.tg_topk_select(s, seqlens, q_len, k)
+    Hk, pos, gv, lg = tg.tg_gather(H, s, kept, seqlens, q_len, k)
+    torch.cuda.synchronize()
+    for key, ref in (("score", s), ("kept_idx", kept), ("cu_kept_dev", cu_dev), ("H_kept", Hk), ("pos", pos),
+                     ("g", gv), ("logg", lg)):
+        assert np.array_equal(bits(fused[key]), bits(ref)), key
+    for l, (Q, K, V) in enumerate(layers):
+        O, L = tg.tg_gated_attn_fwd(Q, K, V, lg, pos, cu, scale)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(fused["O"][l]), bits(O)), l
+        assert np.array_equal(bits(fused["lse"][l]), bits(L)), l
+    kept_o, _ = orc.topk_select(s.cpu().numpy(), seqlens, q_len, k)
+    assert np.array_equal(kept.cpu().numpy(), kept_o.astype(np.int32))
+    assert st.item() == 0
