@@ -258,6 +258,39 @@ def bandwidth_instances(tg, torch, dev, peak_gbs, reps):
     return out
 
 
+def qkv_rope_time(tg, torch, dev, Hk, pos, Hq, Hkv, D, peak_tflops, reps):
+    """Projection of the bench workload's kept rows to Q/K/V with rotary embedding at their
+    original positions (a seeded N(0, 1/d) stacked projection, theta 1e6), L2 flushed before
+    every launch."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20262)
+    M, d = Hk.shape
+    N = (Hq + 2 * Hkv) * D
+    W = (torch.randn(N, d, device=dev, generator=gen) / d ** 0.5).to(torch.bfloat16)
+    Q = torch.empty(M, Hq, D, device=dev, dtype=torch.bfloat16)
+    K = torch.empty(M, Hkv, D, device=dev, dtype=torch.bfloat16)
+    V = torch.empty(M, Hkv, D, device=dev, dtype=torch.bfloat16)
+    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+    run = lambda: tg.tg_qkv_rope(Hk, W, pos, Hq, Hkv, D, 1.0e6, Q=Q, K=K, V=V)
+    run()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(reps):
+        flush.zero_()
+        torch.cuda._sleep(100_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1) / 1e3
+    t = tot / reps
+    flops = 2.0 * M * N * d
+    return {"shape": f"M={M} kept rows x d={d} -> {Hq}/{Hkv} heads x D={D}, rotary at original positions",
+            "us": t * 1e6, "tflops": flops / t / 1e12, "frac": flops / t / 1e12 / peak_tflops}
+
+
 def split_select_times(tg, torch, dev, reps):
     """The sequence-split selection's two device steps for one 131072-token sequence cut into 8
     blocks, K=4096: one rank's top-k candidates of its 16352-token block, and the merge of the
@@ -628,6 +661,7 @@ def main():
         bw = bandwidth_instances(tg, torch, dev, pk["hbm_gbs"], args.bw_reps)
 
     split_t = split_select_times(tg, torch, dev, 20) if not args.no_bw else None
+    qkv_t = qkv_rope_time(tg, torch, dev, Hk, pos, wl.Hq, wl.Hkv, wl.D, pk["bf16_tflops"], 20) if not args.no_bw else None
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -659,6 +693,7 @@ def main():
             "bandwidth_instances": bw,
             "graph_replay": graph,
             "split_select": split_t,
+            "qkv_rope": qkv_t,
             "device_status": dev_status,
         }
         print(json.dumps(line), flush=True)

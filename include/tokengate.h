@@ -118,6 +118,23 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
 tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
                          int32_t* cu_kept_dev, int32_t* dev_status, void* stream);
 
+/* Projection of the kept rows for a layer above L (aitualizate.com TokenGate article,
+ * phase 3: those layers process only the kept tokens, at their original positions). The
+ * pages give no projection or rotary details; the reading implemented:
+ *   X = H_kept W_qkv^T split into Q [M, Hq, D], K [M, Hkv, D], V [M, Hkv, D];
+ *   Q and K rotated at pos: for i < D/2, angle a = pos * rope_theta^(-2i/D),
+ *   y[i] = x[i] cos a - x[i+D/2] sin a,  y[i+D/2] = x[i+D/2] cos a + x[i] sin a.
+ *   H_kept   device bf16 [M, d] row-major (tg_gather's output)
+ *   W_qkv    device bf16 [(Hq + 2 Hkv) D, d] row-major (output-major, like nn.Linear.weight)
+ *   pos      device int32 [M] original positions (tg_gather's output); unused if rope_theta <= 0
+ *   Q, K, V  device bf16 (written)
+ * rope_theta <= 0: no rotation. bf16 only, on the tensor cores (fp32 accumulation; the angle
+ * is reduced in double, so positions up to TG_MAX_CTX keep their accuracy).
+ * Supported: d % 64 == 0; D in {64, 128}; (Hq + 2 Hkv) D % 256 == 0; 16-byte aligned tensors. */
+tg_status tg_qkv_rope(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W_qkv,
+                      const int32_t* pos, int32_t Hq, int32_t Hkv, int32_t D, float rope_theta, void* Q, void* K,
+                      void* V, int32_t* dev_status, void* stream);
+
 /* Sequence-split selection across devices, step 1 (one contiguous block of a sequence's
  * context per device; the merge below is step 2). The min(k, n) tokens of the block with the
  * largest scores, ordered by position, as candidates: cand_idx = base + position in the block

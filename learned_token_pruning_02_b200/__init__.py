@@ -28,6 +28,7 @@ TG_MAX_CTX = 262144
 EXPORTS = (
     "tg_status_string", "tg_last_error", "tg_version", "tg_kept_counts", "tg_score",
     "tg_topk_select", "tg_gather", "tg_gated_attn_fwd", "tg_prefill_above_L",
+    "tg_qkv_rope",
     "tg_topk_candidates",
     "tg_topk_merge",
 )
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.tg_score.argtypes = [_I32, _VP, _I64, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP]
     L.tg_topk_select.restype = _I32
     L.tg_topk_select.argtypes = [_VP, _SEQP, _VP, _VP, _VP, _VP]
+    L.tg_qkv_rope.restype = _I32
+    L.tg_qkv_rope.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _I32, _I32, _I32, _F, _VP, _VP, _VP, _VP, _VP]
     L.tg_topk_candidates.restype = _I32
     L.tg_topk_candidates.argtypes = [_VP, _I32, _I32, _I32, _VP, _VP, _VP, _VP]
     L.tg_topk_merge.restype = _I32
@@ -175,6 +178,21 @@ def tg_topk_select(score, seqlens, q_len, k, kept_idx=None, cu_kept_dev=None, de
     _check("tg_topk_select", lib().tg_topk_select(_ptr(score), s.ref(), _ptr(kept_idx), _ptr(cu_kept_dev),
                                                   _ptr(dev_status), _stream(stream)))
     return kept_idx, cu_kept_dev
+
+
+def tg_qkv_rope(H_kept, W_qkv, pos, Hq: int, Hkv: int, D: int, rope_theta: float, Q=None, K=None, V=None,
+                dev_status=None, stream=None):
+    """Q, K, V of the kept rows (bf16), Q and K rotated at their original positions: (Q, K, V)."""
+    _cuda(H_kept, W_qkv, pos, Q, K, V, dev_status)
+    M, d = H_kept.shape
+    dev = H_kept.device
+    Q = torch.empty(M, Hq, D, device=dev, dtype=torch.bfloat16) if Q is None else Q
+    K = torch.empty(M, Hkv, D, device=dev, dtype=torch.bfloat16) if K is None else K
+    V = torch.empty(M, Hkv, D, device=dev, dtype=torch.bfloat16) if V is None else V
+    _check("tg_qkv_rope", lib().tg_qkv_rope(_dtype(H_kept), _ptr(H_kept), M, d, _ptr(W_qkv), _ptr(pos), Hq, Hkv, D,
+                                            float(rope_theta), _ptr(Q), _ptr(K), _ptr(V), _ptr(dev_status),
+                                            _stream(stream)))
+    return Q, K, V
 
 
 def tg_topk_candidates(score, k: int, base: int = 0, cand_score=None, cand_idx=None, dev_status=None, stream=None):

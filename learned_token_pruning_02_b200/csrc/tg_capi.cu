@@ -65,7 +65,7 @@ bool pdl_enabled(int kernel_id) {
   if (mask < 0) {
     const char* off = getenv("TG_DISABLE_PDL");
     const char* m = getenv("TG_PDL_MASK");
-    mask = (off && off[0] && off[0] != '0') ? 0 : (m ? atoi(m) : 15);
+    mask = (off && off[0] && off[0] != '0') ? 0 : (m ? atoi(m) : 31);
   }
   return (mask & kernel_id) != 0;
 }
@@ -195,6 +195,27 @@ tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_
                          int32_t* cu_kept_dev, int32_t* dev_status, void* stream) {
   g_err[0] = 0;
   return select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, nullptr, nullptr, nullptr, 0);
+}
+
+tg_status tg_qkv_rope(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W_qkv,
+                      const int32_t* pos, int32_t Hq, int32_t Hkv, int32_t D, float rope_theta, void* Q, void* K,
+                      void* V, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  if (dtype != TG_BF16) return fail(TG_ERR_UNSUPPORTED, "tg_qkv_rope runs on bf16 only");
+  if (M < 0 || d <= 0 || Hq <= 0 || Hkv <= 0) return fail(TG_ERR_INVALID_ARG, "need M >= 0 and d, Hq, Hkv > 0");
+  if (M > INT32_MAX) return fail(TG_ERR_UNSUPPORTED, "M too large");
+  if (d % 64) return fail(TG_ERR_UNSUPPORTED, "d must be a multiple of 64");
+  if (D != 64 && D != 128) return fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128");
+  if (((int64_t)(Hq + 2 * Hkv) * D) % 256) return fail(TG_ERR_UNSUPPORTED, "(Hq + 2 Hkv) * D must be a multiple of 256");
+  if (!(rope_theta == rope_theta)) return fail(TG_ERR_INVALID_ARG, "rope_theta is NaN");
+  if (M == 0) return TG_OK;
+  if (!H_kept || !W_qkv || !Q || !K || !V || (rope_theta > 0.f && !pos))
+    return fail(TG_ERR_INVALID_ARG, "H_kept, W_qkv, Q, K, V (and pos when rope_theta > 0) are required");
+  if (!aligned16(H_kept) || !aligned16(W_qkv) || !aligned16(Q) || !aligned16(K) || !aligned16(V))
+    return fail(TG_ERR_UNSUPPORTED, "H_kept, W_qkv, Q, K and V must be 16-byte aligned");
+  tg_status st = check_device();
+  if (st != TG_OK) return st;
+  return launch_qkv_rope(H_kept, M, d, W_qkv, pos, Hq, Hkv, D, rope_theta, Q, K, V, dev_status, (cudaStream_t)stream);
 }
 
 tg_status tg_topk_candidates(const float* score, int32_t n, int32_t k, int32_t base, float* cand_score,

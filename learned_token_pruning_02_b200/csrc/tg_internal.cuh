@@ -25,7 +25,7 @@ int device_sm_count();
 // their prologue while the previous kernel drains; each waits on griddepcontrol.wait before
 // its first global memory access). TG_DISABLE_PDL=1 in the environment turns it off.
 // kernel ids for the launch-chaining mask
-enum { PDL_SCORE = 1, PDL_SELECT = 2, PDL_GATHER = 4, PDL_ATTN = 8 };
+enum { PDL_SCORE = 1, PDL_SELECT = 2, PDL_GATHER = 4, PDL_ATTN = 8, PDL_QKV = 16 };
 bool pdl_enabled(int kernel_id);
 inline cudaLaunchAttribute pdl_attribute(int kernel_id) {
   cudaLaunchAttribute a;
@@ -117,6 +117,10 @@ struct AttnArgs {
   // before it waits on the previous kernel.
   bool qkv_ready = false;
 };
+
+// Q/K/V = H_kept W^T with rotary embedding of Q and K at pos (bf16, tensor cores).
+tg_status launch_qkv_rope(const void* Hk, int64_t M, int d, const void* W, const int32_t* pos, int Hq, int Hkv,
+                          int D, float theta, void* Q, void* K, void* V, int32_t* dev_status, cudaStream_t st);
 
 tg_status launch_attn_simt(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);
 tg_status launch_attn_tc(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);

@@ -1,0 +1,39 @@
+"""Projection of the kept rows to Q/K/V with rotary embedding at original positions
+(tg_qkv_rope) against the oracle's qkv_rope, within the bf16 tolerance. Cases cover two heads
+per 128-column half (D = 64), the Qwen3-1.7B shapes, positions near 128K tokens (angles of
+about 1e5 radians before reduction) and no rotation."""
+import numpy as np
+import pytest
+import torch
+
+import learned_token_pruning_02_b200 as tg
+import tg_inputs as ti
+from oracle import tg_oracle as orc
+from tg_testutil import TOL, from_dev, max_abs_rel, to_dev
+
+pytestmark = pytest.mark.gpu
+
+CASES = [  # (M, d, Hq, Hkv, D, theta, max position)
+    (300, 256, 4, 2, 64, 1.0e4, 3000),
+    (1088, 2048, 16, 8, 128, 1.0e6, 8192),
+    (256, 256, 2, 1, 128, 1.0e4, 131072),
+    (200, 512, 2, 1, 128, 0.0, 1000),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_qkv_rope_matches_oracle(case):
+    M, d, Hq, Hkv, D, theta, pmax = case
+    g = np.random.default_rng(M + d + D)
+    Hk = ti.f32_to_bf16_bits((g.standard_normal((M, d)) / 2).astype(np.float32))
+    W = ti.f32_to_bf16_bits((g.standard_normal(((Hq + 2 * Hkv) * D, d)) / np.sqrt(d)).astype(np.float32))
+    pos = np.sort(g.choice(pmax, size=M, replace=M > pmax)).astype(np.int32)
+    st = torch.zeros(1, device="cuda", dtype=torch.int32)
+    Q, K, V = tg.tg_qkv_rope(to_dev(Hk, "bf16"), to_dev(W, "bf16"), torch.from_numpy(pos).cuda(), Hq, Hkv, D, theta,
+                             dev_status=st)
+    torch.cuda.synchronize()
+    rQ, rK, rV = orc.qkv_rope(ti.widen(Hk, "bf16"), ti.widen(W, "bf16"), pos, Hq, Hkv, D, theta)
+    for got, ref, name in ((Q, rQ, "Q"), (K, rK, "K"), (V, rV, "V")):
+        err = max_abs_rel(from_dev(got), ref)
+        assert err <= TOL["bf16"], (name, err)
+    assert st.item() == 0
