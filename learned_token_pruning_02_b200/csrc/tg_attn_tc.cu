@@ -480,13 +480,13 @@ tg_status launch_d(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_
     return fail(TG_ERR_CUDA, "tg_gated_attn_fwd: building the TMA tensor maps failed");
   const bool un = (a.flags & TG_ATTN_UNNORMALISED) != 0;
   auto kern = un ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
-  static bool attr_set[2] = {false, false};
-  if (!attr_set[un]) {
+  const int slot = D == 64 ? (un ? ATTR_ATTN64_UN : ATTR_ATTN64) : (un ? ATTR_ATTN128_UN : ATTR_ATTN128);
+  if (attrs_needed(slot)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_fwd: cudaFuncSetAttribute");
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_fwd: cudaFuncSetAttribute");
-    attr_set[un] = true;
+    mark_attrs_set(slot);
   }
   const int grid = units * a.Hq;
   cudaLaunchConfig_t cfg = {};

@@ -54,6 +54,24 @@ tg_status check_device() {
   return TG_OK;
 }
 
+static bool g_attr_set[ATTR_SLOTS][64];
+
+static int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (dev >= 0 && dev < 64) ? dev : -1;
+}
+
+bool attrs_needed(int slot) {
+  const int dev = current_device();
+  return dev < 0 || !g_attr_set[slot][dev];
+}
+
+void mark_attrs_set(int slot) {
+  const int dev = current_device();
+  if (dev >= 0) g_attr_set[slot][dev] = true;
+}
+
 int device_sm_count() {
   int dev = 0;
   cudaGetDevice(&dev);

@@ -92,14 +92,13 @@ tg_status launch_gather(tg_dtype dt, const void* H, int64_t ldh, int d, const fl
   const int es = dt == TG_BF16 ? 2 : 4;
   const int nvec = d * es / 16;
   const int64_t ldv = ldh * es / 16;
-  static bool attr_set = false;
-  if (!attr_set) {  // the carveout of the other chain kernels: no reconfiguration between them
+  if (attrs_needed(ATTR_GATHER)) {  // the carveout of the other chain kernels: no reconfiguration between them
     for (auto k : {gather_kernel<false>, gather_kernel<true>}) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
                                            (int)cudaSharedmemCarveoutMaxShared);
       if (e != cudaSuccess) return cuda_status(e, "gather: cudaFuncSetAttribute");
     }
-    attr_set = true;
+    mark_attrs_set(ATTR_GATHER);
   }
   int blocks = (m_chunk + WARPS - 1) / WARPS;
   const int cap = device_sm_count() * 16;

@@ -21,6 +21,19 @@ tg_status cuda_status(cudaError_t e, const char* what);
 tg_status check_device();
 int device_sm_count();
 
+// Function attributes (shared-memory size, carveout) apply per device. True until
+// mark_attrs_set(slot) is called on the current device; slots name the launchers.
+// Template kernels take one slot per instantiation (score: dg 64/128/256; attention: D 64/128
+// times the normalised / unnormalised form).
+enum {
+  ATTR_SCORE64 = 0, ATTR_SCORE128, ATTR_SCORE256,
+  ATTR_SELECT, ATTR_GATHER,
+  ATTR_ATTN64, ATTR_ATTN64_UN, ATTR_ATTN128, ATTR_ATTN128_UN,
+  ATTR_QKV, ATTR_SLOTS
+};
+bool attrs_needed(int slot);
+void mark_attrs_set(int slot);
+
 // Launch attribute for programmatic dependent launch (the tensor-core chain kernels start
 // their prologue while the previous kernel drains; each waits on griddepcontrol.wait before
 // its first global memory access). TG_DISABLE_PDL=1 in the environment turns it off.

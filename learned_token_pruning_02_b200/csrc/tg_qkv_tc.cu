@@ -292,11 +292,10 @@ tg_status launch_qkv_rope(const void* Hk, int64_t M, int d, const void* W, const
   if (!make_tmap_bf16_2d(&tmA, Hk, (uint64_t)M, (uint64_t)d, (uint64_t)d, BM, BK) ||
       !make_tmap_bf16_2d(&tmW, W, (uint64_t)N, (uint64_t)d, (uint64_t)d, BN, BK))
     return fail(TG_ERR_CUDA, "tg_qkv_rope: building the TMA tensor maps failed");
-  static bool attr_set = false;
-  if (!attr_set) {
+  if (attrs_needed(ATTR_QKV)) {
     cudaError_t e = cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return cuda_status(e, "tg_qkv_rope: cudaFuncSetAttribute");
-    attr_set = true;
+    mark_attrs_set(ATTR_QKV);
   }
   int ctas = device_sm_count();
   if (ctas > p.tiles) ctas = p.tiles;

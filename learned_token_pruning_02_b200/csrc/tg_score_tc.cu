@@ -296,8 +296,8 @@ tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void
   if (!make_tmap_bf16_2d(&tmH, H, (uint64_t)n_tok, (uint64_t)d, (uint64_t)ldh, BM, BK) ||
       !make_tmap_bf16_2d(&tmW, W1, (uint64_t)DG, (uint64_t)d, (uint64_t)d, DG, BK))
     return fail(TG_ERR_CUDA, "tg_score: building the TMA tensor maps failed");
-  static bool attr_set = false;
-  if (!attr_set) {
+  constexpr int slot = DG == 64 ? ATTR_SCORE64 : (DG == 128 ? ATTR_SCORE128 : ATTR_SCORE256);
+  if (attrs_needed(slot)) {
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<DG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return cuda_status(e, "tg_score: cudaFuncSetAttribute");
     // every kernel of the chain asks for the same (all-shared) carveout, so consecutive chain
@@ -305,7 +305,7 @@ tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void
     e = cudaFuncSetAttribute(score_tc_kernel<DG>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_status(e, "tg_score: cudaFuncSetAttribute");
-    attr_set = true;
+    mark_attrs_set(slot);
   }
   const int n_tiles = (int)((n_tok + BM - 1) / BM);
   int ctas = device_sm_count();

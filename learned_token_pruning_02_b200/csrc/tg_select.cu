@@ -550,15 +550,14 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
   if (rows < 1) rows = 1;
   p.C = C;
   p.rows = rows;
-  static bool attr_set = false;
-  if (!attr_set) {
+  if (attrs_needed(ATTR_SELECT)) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (per_cta + MAXC) * 4);
     if (e != cudaSuccess) return cuda_status(e, "select: cudaFuncSetAttribute");
     e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_status(e, "select: cudaFuncSetAttribute");
-    attr_set = true;
+    mark_attrs_set(ATTR_SELECT);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(nseq * C));
