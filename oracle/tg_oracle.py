@@ -24,6 +24,9 @@ leave a step open, the reading taken is stated in the function's docstring:
     "unnormalised" variant multiplies the weight by g_j without renormalising;
   * causal mask on original positions (key allowed iff pos_j <= pos_i, same sequence);
     grouped KV heads map query head h to KV head h // (Hq / Hkv).
+  * gradients of the attention (for training the selector end to end): the derivative of
+    the normalised form above with the per-head gain held constant; the score gradient
+    goes through log g = log-sigmoid(s).
   * above-L projections (not on the pages, which stop at "layers above L process the kept
     tokens"): Q/K/V = kept rows times one stacked projection matrix, with rotary position
     embedding on Q and K at each kept token's original position, rotate-half pairing
@@ -215,6 +218,64 @@ def gated_attention(Q, K, V, logg, pos, cu_kept, Hq, Hkv, scale, head_gain=None,
                 O[sel, h, :] = P @ V[lo:hi, kv, :]
             LSE[h, sel] = (m + np.log(l))[:, 0]
     return O, LSE
+
+
+def gated_attention_bwd(Q, K, V, logg, pos, cu_kept, Hq, Hkv, scale, dO, head_gain=None):
+    """Gradients of the (normalised) token-gated attention with respect to Q, K, V and log g.
+
+    thelatestinai.com page, Figure 1(c): the gated attention is what lets the selector train
+    end to end; aitualizate.com article, "Cómo consigue entrenar una selección top-K": the
+    score is a bias on the logits, so its gradient is that of an additive logit bias. This is
+    the derivative of gated_attention() written out per sequence and query head, with
+    S = scale Q K^T + gain_h log g^T (masked), P = softmax rows, O = P V, and upstream dO:
+        dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(dP * P)),
+        dQ = scale dS K,  dK = scale dS^T Q,  d log g_j = sum_h gain_h sum_i dS_ij.
+    Query heads of one KV group add into that KV head's dK, dV. The per-head gain is a
+    constant here (no gradient). Returns float64 (dQ [M, Hq, D], dK [M, Hkv, D],
+    dV [M, Hkv, D], dlogg [M]).
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    M, _, D = Q.shape
+    G = Hq // Hkv
+    assert Hq % Hkv == 0 and K.shape[1] == Hkv and dO.shape == Q.shape
+    pos = np.asarray(pos, dtype=np.int64)
+    lg = np.zeros(M) if logg is None else np.asarray(logg, dtype=np.float64)
+    gain = np.ones(Hq) if head_gain is None else np.asarray(head_gain, dtype=np.float64)
+    cu = np.asarray(cu_kept, dtype=np.int64)
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    dlogg = np.zeros(M)
+    for b in range(cu.size - 1):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        if hi == lo:
+            continue
+        allowed = pos[lo:hi][None, :] <= pos[lo:hi][:, None]
+        for h in range(Hq):
+            kv = h // G
+            Qh, Kh, Vh, dOh = Q[lo:hi, h, :], K[lo:hi, kv, :], V[lo:hi, kv, :], dO[lo:hi, h, :]
+            S = np.where(allowed, scale * (Qh @ Kh.T) + gain[h] * lg[lo:hi][None, :], -np.inf)
+            P = np.exp(S - S.max(axis=1, keepdims=True))
+            P = P / P.sum(axis=1, keepdims=True)
+            dP = dOh @ Vh.T
+            dS = P * (dP - (dP * P).sum(axis=1, keepdims=True))
+            dQ[lo:hi, h, :] = scale * (dS @ Kh)
+            dK[lo:hi, kv, :] += scale * (dS.T @ Qh)
+            dV[lo:hi, kv, :] += P.T @ dOh
+            dlogg[lo:hi] += gain[h] * dS.sum(axis=0)
+    return dQ, dK, dV, dlogg
+
+
+def gate_score_grad(dlogg, logg):
+    """Gradient with respect to the selector's score, given the gradient with respect to log g.
+
+    With g = sigmoid(s) (the reading of gate_value), d log g / ds = 1 - g = -expm1(log g),
+    which is exact where g is close to 1. Rows whose log g was fixed to 0 (question tail with
+    the gate forced to one) get zero."""
+    return np.asarray(dlogg, np.float64) * -np.expm1(np.asarray(logg, np.float64))
 
 
 def gated_attention_weights(q, Kmat, g, scale):

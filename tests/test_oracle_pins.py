@@ -417,3 +417,99 @@ def test_qkv_rope_split_and_projection():
     assert np.allclose(Q[3], orc.rope(q3, [50], 1.0e4)[0], atol=1e-12)
     k4 = X[4, Hq * D: (Hq + Hkv) * D].reshape(1, Hkv, D)
     assert np.allclose(K[4], orc.rope(k4, [51], 1.0e4)[0], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- attention backward
+
+
+def _bwd_case(seed, lens=(5, 7), Hq=4, Hkv=2, D=8, gain=True):
+    g = np.random.default_rng(seed)
+    M = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    pos = np.concatenate([np.sort(g.choice(3 * n, n, replace=False)) for n in lens]).astype(np.int64)
+    Q, K, V = g.standard_normal((M, Hq, D)), g.standard_normal((M, Hkv, D)), g.standard_normal((M, Hkv, D))
+    logg = orc.gate_value(g.standard_normal(M) * 2)[1]
+    dO = g.standard_normal((M, Hq, D))
+    hg = g.uniform(0.5, 1.5, Hq) if gain else None
+    return Q, K, V, logg, pos, cu, Hq, Hkv, 1.0 / math.sqrt(D), dO, hg
+
+
+def _loss(Q, K, V, logg, pos, cu, Hq, Hkv, scale, dO, hg):
+    O, _ = orc.gated_attention(Q, K, V, logg, pos, cu, Hq, Hkv, scale, head_gain=hg)
+    return float((O * dO).sum())
+
+
+def test_attention_bwd_matches_central_differences():
+    # every input element perturbed on its own: a wrong sign, scale, transposition or GQA
+    # accumulation in the backward shows up as an O(1) mismatch against the forward's slopes
+    case = _bwd_case(1)
+    Q, K, V, logg, pos, cu, Hq, Hkv, scale, dO, hg = case
+    dQ, dK, dV, dl = orc.gated_attention_bwd(Q, K, V, logg, pos, cu, Hq, Hkv, scale, dO, head_gain=hg)
+    eps = 1e-6
+    for name, X, dX in (("Q", Q, dQ), ("K", K, dK), ("V", V, dV), ("logg", logg, dl)):
+        fd = np.zeros_like(X)
+        for idx in np.ndindex(X.shape):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[idx] += eps
+            Xm[idx] -= eps
+            args = {"Q": Q, "K": K, "V": V, "logg": logg}
+            ap, am = dict(args, **{name: Xp}), dict(args, **{name: Xm})
+            lp = _loss(ap["Q"], ap["K"], ap["V"], ap["logg"], pos, cu, Hq, Hkv, scale, dO, hg)
+            lm = _loss(am["Q"], am["K"], am["V"], am["logg"], pos, cu, Hq, Hkv, scale, dO, hg)
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert np.max(np.abs(fd - dX)) <= 1e-6 * max(1.0, np.max(np.abs(dX))), name
+
+
+def test_attention_bwd_matches_torch_autograd():
+    # torch's own differentiation of a direct torch statement of the forward (float64, CPU)
+    Q, K, V, logg, pos, cu, Hq, Hkv, scale, dO, hg = _bwd_case(2, lens=(17, 1, 23), Hq=8, Hkv=2, D=16)
+    tQ, tK, tV, tl = (torch.tensor(x, requires_grad=True) for x in (Q, K, V, logg))
+    G = Hq // Hkv
+    loss = 0.0
+    for b in range(len(cu) - 1):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        mask = torch.tensor(pos[lo:hi][None, :] <= pos[lo:hi][:, None])
+        for h in range(Hq):
+            S = scale * tQ[lo:hi, h] @ tK[lo:hi, h // G].T + float(hg[h]) * tl[lo:hi][None, :]
+            P = torch.softmax(S.masked_fill(~mask, float("-inf")), dim=1)
+            loss = loss + (P @ tV[lo:hi, h // G] * torch.tensor(dO[lo:hi, h])).sum()
+    loss.backward()
+    ref = orc.gated_attention_bwd(Q, K, V, logg, pos, cu, Hq, Hkv, scale, dO, head_gain=hg)
+    for got, t in zip(ref, (tQ, tK, tV, tl)):
+        np.testing.assert_allclose(got, t.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_bwd_invariants():
+    Q, K, V, logg, pos, cu, Hq, Hkv, scale, dO, hg = _bwd_case(3, lens=(9, 12, 1), Hq=6, Hkv=3, D=4)
+    dQ, dK, dV, dl = orc.gated_attention_bwd(Q, K, V, logg, pos, cu, Hq, Hkv, scale, dO, head_gain=hg)
+    # each row's dS sums to zero (softmax is shift invariant), so d log g sums to zero per sequence
+    for b in range(len(cu) - 1):
+        assert abs(dl[cu[b]:cu[b + 1]].sum()) <= 1e-12 * max(1.0, np.abs(dl).max())
+    # a constant added to log g within a sequence changes nothing, gradients included
+    shifted = logg + np.where(np.arange(len(logg)) < cu[1], 3.0, -2.0)
+    for a, b in zip((dQ, dK, dV, dl),
+                    orc.gated_attention_bwd(Q, K, V, shifted, pos, cu, Hq, Hkv, scale, dO, head_gain=hg)):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-12)
+    # the first row of a sequence sees only itself: P = 1, so its dQ is 0 and dV_0 gets dO_0
+    first = _bwd_case(4, lens=(1,), Hq=2, Hkv=1, D=4)
+    fq, fk, fv, fl = orc.gated_attention_bwd(*first[:9], first[9], head_gain=first[10])
+    assert np.all(fq == 0) and np.all(fl == 0)
+    np.testing.assert_allclose(fv[0, 0], first[9][0].sum(axis=0), rtol=1e-14)
+
+
+def test_gate_score_grad_matches_central_differences():
+    # through the gate map: d/ds of the attention loss with log g = log-sigmoid(s)
+    Q, K, V, _, pos, cu, Hq, Hkv, scale, dO, hg = _bwd_case(5)
+    s = np.random.default_rng(6).standard_normal(len(pos)) * 3
+    logg = orc.gate_value(s)[1]
+    dl = orc.gated_attention_bwd(Q, K, V, logg, pos, cu, Hq, Hkv, scale, dO, head_gain=hg)[3]
+    ds = orc.gate_score_grad(dl, logg)
+    eps = 1e-6
+    for j in range(len(s)):
+        sp, sm = s.copy(), s.copy()
+        sp[j] += eps
+        sm[j] -= eps
+        fd = (_loss(Q, K, V, orc.gate_value(sp)[1], pos, cu, Hq, Hkv, scale, dO, hg)
+              - _loss(Q, K, V, orc.gate_value(sm)[1], pos, cu, Hq, Hkv, scale, dO, hg)) / (2 * eps)
+        assert abs(fd - ds[j]) <= 1e-6 * max(1.0, np.abs(ds).max()), j
+    assert orc.gate_score_grad(np.array([5.0]), np.array([0.0]))[0] == 0.0
