@@ -291,6 +291,47 @@ def qkv_rope_time(tg, torch, dev, Hk, pos, Hq, Hkv, D, peak_tflops, reps):
             "us": t * 1e6, "tflops": flops / t / 1e12, "frac": flops / t / 1e12 / peak_tflops}
 
 
+def attn_bwd_time(tg, torch, dev, Q, K, V, logg, pos, cu, scale, peak_tflops, reps):
+    """Gradients of the gated attention for the bench workload's kept set (one above-L layer's
+    Q/K/V, the chain's own log g and positions, a seeded N(0, 1) upstream dO): the forward gives
+    O and lse, then the two backward kernels are timed together, L2 flushed before each run.
+    Algorithmic work: the five products of the backward (S recomputed, dP, dV, dK, dQ), each
+    2 D flop per visible (query, key) pair and head."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20263)
+    Hq, D = Q.shape[1], Q.shape[2]
+    m = cu[-1]
+    O, lse = tg.tg_gated_attn_fwd(Q, K, V, logg, pos, cu, scale)
+    dO = torch.randn(Q.shape, device=dev, generator=gen).to(torch.bfloat16)
+    bufs = dict(dQ=torch.empty(Q.shape, device=dev), dK=torch.empty(K.shape, device=dev),
+                dV=torch.empty(V.shape, device=dev), dlogg=torch.empty(m, device=dev),
+                dscore=torch.empty(m, device=dev))
+    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+    run = lambda: tg.tg_gated_attn_bwd(Q, K, V, logg, pos, cu, O, lse, dO, scale, want_dscore=True, **bufs)
+    run()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(reps):
+        flush.zero_()
+        torch.cuda._sleep(100_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1) / 1e3
+    t = tot / reps
+    pairs = sum((b - a) * (b - a + 1) // 2 for a, b in zip(cu[:-1], cu[1:]))
+    flops = 10.0 * Hq * D * pairs
+    fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 FMA lanes x 2 flop x max SM clock
+    return {"shape": f"M={m} kept rows in {len(cu) - 1} sequence(s), {Hq}/{K.shape[1]} heads, D={D}, bf16 in, f32 gradients",
+            "us": t * 1e6, "tflops": flops / t / 1e12, "bound": "alu", "fp32_fma_peak_tflops": fma_peak,
+            "frac_of_fp32_fma_peak": flops / t / 1e12 / fma_peak,
+            "frac_of_bf16_peak": flops / t / 1e12 / peak_tflops,
+            "note": "CUDA-core fp32 kernels (dK/dV per key tile, dQ per query tile)"}
+
+
 def split_select_times(tg, torch, dev, reps):
     """The sequence-split selection's two device steps for one 131072-token sequence cut into 8
     blocks, K=4096: one rank's top-k candidates of its 16352-token block, and the merge of the
@@ -662,6 +703,8 @@ def main():
 
     split_t = split_select_times(tg, torch, dev, 20) if not args.no_bw else None
     qkv_t = qkv_rope_time(tg, torch, dev, Hk, pos, wl.Hq, wl.Hkv, wl.D, pk["bf16_tflops"], 20) if not args.no_bw else None
+    bwd_t = (attn_bwd_time(tg, torch, dev, *layers[0], logg, pos, list(cu), scale, pk["bf16_tflops"], 5)
+             if not args.no_bw else None)
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -694,6 +737,7 @@ def main():
             "graph_replay": graph,
             "split_select": split_t,
             "qkv_rope": qkv_t,
+            "gated_attn_bwd": bwd_t,
             "device_status": dev_status,
         }
         print(json.dumps(line), flush=True)

@@ -197,6 +197,35 @@ tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const 
                             int32_t D, float softmax_scale, uint32_t flags, void* O,
                             float* lse, int32_t* dev_status, void* stream);
 
+/* Gradients of tg_gated_attn_fwd in its normalised form (thelatestinai.com TokenGate page,
+ * Figure 1(c): the gated attention lets the top-K selector train end to end; aitualizate.com
+ * article: the score is a bias on the logits, so its gradient is that of an additive bias).
+ * With S, P, O and lse as in the forward and the upstream gradient dO, per sequence and head:
+ *   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(dO * O)),
+ *   dQ = scale dS K,  dK = scale dS^T Q  (the query heads of a KV group add into its dK, dV),
+ *   dlogg_j  = sum_h gain_h sum_i dS_ij,
+ *   dscore_j = dlogg_j * (1 - g_j) = dlogg_j * -expm1(logg_j)  (g = sigmoid(score)).
+ * The per-head gain is treated as a constant (no gradient for it).
+ *   Q, K, V, logg, head_gain, pos, cu_kept_host, B, Hq, Hkv, D, softmax_scale: as given to
+ *                the forward (pos strictly ascending inside each sequence; a violation sets
+ *                TG_DEV_POS_NOT_ASCENDING)
+ *   O            device act [sum M_b, Hq, D]: the forward's output
+ *   lse          device f32 [Hq, sum M_b]: the forward's lse (required)
+ *   dO           device act [sum M_b, Hq, D]
+ *   dQ           device f32 [sum M_b, Hq, D] (written)
+ *   dK, dV       device f32 [sum M_b, Hkv, D] (written)
+ *   dlogg        device f32 [sum M_b] (written) or NULL
+ *   dscore       device f32 [sum M_b] (written) or NULL; needs logg
+ * Arithmetic is fp32 for both dtypes; no workspace; results are deterministic.
+ * Supported: D in {64, 128}; Hq % Hkv == 0; 16-byte aligned Q, K, V, dO, dQ, dK, dV;
+ * flags without TG_ATTN_UNNORMALISED (TG_ERR_UNSUPPORTED otherwise). */
+tg_status tg_gated_attn_bwd(tg_dtype dtype, const void* Q, const void* K, const void* V,
+                            const float* logg, const float* head_gain, const int32_t* pos,
+                            const int32_t* cu_kept_host, int32_t B, int32_t Hq, int32_t Hkv,
+                            int32_t D, float softmax_scale, uint32_t flags, const void* O,
+                            const float* lse, const void* dO, float* dQ, float* dK, float* dV,
+                            float* dlogg, float* dscore, int32_t* dev_status, void* stream);
+
 /* The whole gated path above layer L (aitualizate.com TokenGate article, phases 2-3;
  * thelatestinai.com TokenGate page, Figure 1(a)): the results of tg_score -> tg_topk_select
  * -> tg_gather -> tg_gated_attn_fwd for each of n_layers above-L layers, enqueued on one

@@ -31,6 +31,7 @@ EXPORTS = (
     "tg_qkv_rope",
     "tg_topk_candidates",
     "tg_topk_merge",
+    "tg_gated_attn_bwd",
 )
 
 
@@ -90,6 +91,9 @@ def lib() -> ctypes.CDLL:
     L.tg_gated_attn_fwd.restype = _I32
     L.tg_gated_attn_fwd.argtypes = [_I32, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(_I32), _I32, _I32,
                                     _I32, _I32, _F, _U32, _VP, _VP, _VP, _VP]
+    L.tg_gated_attn_bwd.restype = _I32
+    L.tg_gated_attn_bwd.argtypes = [_I32, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(_I32), _I32, _I32,
+                                    _I32, _I32, _F, _U32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]
     L.tg_prefill_above_L.restype = _I32
     L.tg_prefill_above_L.argtypes = [
         _I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _I32, _SEQP, _I32,
@@ -256,6 +260,36 @@ def tg_gated_attn_fwd(Q, K, V, logg, pos, cu_kept, softmax_scale: float, head_ga
         _dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(logg), _ptr(head_gain), _ptr(pos), cu_arr, B, Hq, Hkv, D,
         float(softmax_scale), int(flags), _ptr(O), _ptr(lse), _ptr(dev_status), _stream(stream)))
     return O, lse
+
+
+def tg_gated_attn_bwd(Q, K, V, logg, pos, cu_kept, O, lse, dO, softmax_scale: float, head_gain=None, flags=0,
+                      want_dlogg=True, want_dscore=False, dQ=None, dK=None, dV=None, dlogg=None, dscore=None,
+                      dev_status=None, stream=None):
+    """Gradients of the gated attention (normalised form) from the forward's O and lse and the
+    upstream dO: (dQ [M, Hq, D], dK [M, Hkv, D], dV [M, Hkv, D], dlogg [M] or None,
+    dscore [M] or None), all float32."""
+    _cuda(Q, K, V, logg, pos, O, lse, dO, head_gain, dQ, dK, dV, dlogg, dscore, dev_status)
+    M, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    for t in (Q, K, V, O, dO):
+        assert t.is_contiguous() and t.dtype == Q.dtype
+    cu = [int(x) for x in cu_kept]
+    B = len(cu) - 1
+    cu_arr = (ctypes.c_int32 * len(cu))(*cu)
+    dev = Q.device
+    f32 = torch.float32
+    dQ = torch.empty(M, Hq, D, device=dev, dtype=f32) if dQ is None else dQ
+    dK = torch.empty(M, Hkv, D, device=dev, dtype=f32) if dK is None else dK
+    dV = torch.empty(M, Hkv, D, device=dev, dtype=f32) if dV is None else dV
+    if dlogg is None and want_dlogg:
+        dlogg = torch.empty(M, device=dev, dtype=f32)
+    if dscore is None and want_dscore:
+        dscore = torch.empty(M, device=dev, dtype=f32)
+    _check("tg_gated_attn_bwd", lib().tg_gated_attn_bwd(
+        _dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(logg), _ptr(head_gain), _ptr(pos), cu_arr, B, Hq, Hkv, D,
+        float(softmax_scale), int(flags), _ptr(O), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dlogg),
+        _ptr(dscore), _ptr(dev_status), _stream(stream)))
+    return dQ, dK, dV, dlogg, dscore
 
 
 def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_scale, head_gain=None, flags=0,

@@ -350,6 +350,47 @@ tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const 
                    dev_status, stream, false);
 }
 
+tg_status tg_gated_attn_bwd(tg_dtype dtype, const void* Q, const void* K, const void* V,
+                            const float* logg, const float* head_gain, const int32_t* pos,
+                            const int32_t* cu_kept_host, int32_t B, int32_t Hq, int32_t Hkv,
+                            int32_t D, float softmax_scale, uint32_t flags, const void* O,
+                            const float* lse, const void* dO, float* dQ, float* dK, float* dV,
+                            float* dlogg, float* dscore, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return fail(TG_ERR_INVALID_ARG, "need B >= 0 and Hq, Hkv, D > 0");
+  if (B > 0 && !cu_kept_host) return fail(TG_ERR_INVALID_ARG, "cu_kept_host is NULL");
+  if (Hq % Hkv) return fail(TG_ERR_UNSUPPORTED, "Hq must be a multiple of Hkv");
+  if (D != 64 && D != 128) return fail(TG_ERR_UNSUPPORTED, "D must be 64 or 128");
+  if (flags & TG_ATTN_UNNORMALISED)
+    return fail(TG_ERR_UNSUPPORTED, "the backward covers the normalised form only");
+  if (!(softmax_scale == softmax_scale)) return fail(TG_ERR_INVALID_ARG, "softmax_scale is NaN");
+  if (dscore && !logg) return fail(TG_ERR_INVALID_ARG, "dscore needs logg");
+  if (B == 0) return TG_OK;
+  if (cu_kept_host[0] != 0) return fail(TG_ERR_INVALID_ARG, "cu_kept_host[0] must be 0");
+  for (int b = 0; b < B; ++b)
+    if (cu_kept_host[b + 1] < cu_kept_host[b]) return fail(TG_ERR_INVALID_ARG, "cu_kept_host not monotone");
+  const int64_t m_tot = cu_kept_host[B];
+  if (m_tot == 0) return TG_OK;
+  if (!Q || !K || !V || !pos || !O || !lse || !dO || !dQ || !dK || !dV)
+    return fail(TG_ERR_INVALID_ARG, "Q, K, V, pos, O, lse, dO, dQ, dK and dV are required");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) || !aligned16(dK) ||
+      !aligned16(dV))
+    return fail(TG_ERR_UNSUPPORTED, "Q, K, V, dO, dQ, dK and dV must be 16-byte aligned");
+  tg_status st = check_device();
+  if (st != TG_OK) return st;
+  AttnBwdArgs a{dtype, Q, K, V, O, dO, logg, head_gain, pos, lse, Hq, Hkv, D, softmax_scale,
+                dQ, dK, dV, dlogg, dscore, dev_status, m_tot};
+  std::vector<AttnSeq> v(B);
+  for (int b = 0; b < B; ++b) v[b] = AttnSeq{cu_kept_host[b], cu_kept_host[b + 1] - cu_kept_host[b]};
+  for (int b0 = 0; b0 < B; b0 += kMaxSeqPerLaunch) {
+    const int nb = B - b0 < kMaxSeqPerLaunch ? B - b0 : kMaxSeqPerLaunch;
+    st = launch_attn_bwd(a, v.data() + b0, nb, (cudaStream_t)stream);
+    if (st != TG_OK) return st;
+  }
+  return TG_OK;
+}
+
 // The row copy of the chained prefill (the selector already wrote pos, g and log g): launched
 // after the attention layers, which read nothing it writes, so its first launch starts copying
 // at once and waits for them only at its end.
