@@ -324,12 +324,10 @@ def attn_bwd_time(tg, torch, dev, Q, K, V, logg, pos, cu, scale, peak_tflops, re
     t = tot / reps
     pairs = sum((b - a) * (b - a + 1) // 2 for a, b in zip(cu[:-1], cu[1:]))
     flops = 10.0 * Hq * D * pairs
-    fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 FMA lanes x 2 flop x max SM clock
     return {"shape": f"M={m} kept rows in {len(cu) - 1} sequence(s), {Hq}/{K.shape[1]} heads, D={D}, bf16 in, f32 gradients",
-            "us": t * 1e6, "tflops": flops / t / 1e12, "bound": "alu", "fp32_fma_peak_tflops": fma_peak,
-            "frac_of_fp32_fma_peak": flops / t / 1e12 / fma_peak,
-            "frac_of_bf16_peak": flops / t / 1e12 / peak_tflops,
-            "note": "CUDA-core fp32 kernels (dK/dV per key tile, dQ per query tile)"}
+            "us": t * 1e6, "tflops": flops / t / 1e12, "bound": "tensor", "peak": peak_tflops,
+            "frac": flops / t / 1e12 / peak_tflops,
+            "note": "warp-level mma.sync m16n8k16 kernels (dK/dV per 64-key tile, dQ per 64-query tile)"}
 
 
 def split_select_times(tg, torch, dev, reps):

@@ -30,7 +30,7 @@ enum {
   ATTR_SELECT, ATTR_GATHER,
   ATTR_ATTN64, ATTR_ATTN64_UN, ATTR_ATTN128, ATTR_ATTN128_UN,
   ATTR_QKV,
-  ATTR_BWD,  // 4 slots: (f32, bf16) x (D 64, 128), both backward kernels
+  ATTR_BWD,  // 4 slots: CUDA-core (f32) D 64, 128, then tensor-core (bf16) D 64, 128
   ATTR_SLOTS = ATTR_BWD + 4
 };
 bool attrs_needed(int slot);
