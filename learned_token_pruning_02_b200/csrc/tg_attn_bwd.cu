@@ -29,7 +29,7 @@
 #include <cooperative_groups.h>
 #include <math.h>
 
-#include "tg_internal.cuh"
+#include "tg_attn_bwd.cuh"
 #include "tg_sm100.cuh"
 
 namespace cg = cooperative_groups;
@@ -384,9 +384,57 @@ template <int D>
 struct MSmem {
   static constexpr int SH = D + 8;  // padded row stride in bf16 elements (16-byte pad)
   static constexpr int OWN = MT * SH, STR = ST * SH;
-  // two own tiles, two streamed tiles (bf16), then 6 vectors of 64 32-bit values
-  static constexpr int BYTES = (2 * OWN + 2 * STR) * 2 + 6 * MT * 4;
+  // two own tiles, two buffers of three streamed tiles (bf16), then 8 vectors of 64 32-bit values
+  static constexpr int BYTES = (2 * OWN + 6 * STR) * 2 + 8 * MT * 4;
 };
+
+// 16-byte and 4-byte asynchronous copies global -> shared; a copy with ok == false reads
+// nothing and writes zeros (src must still be a valid address)
+__device__ __forceinline__ void cp16(void* dst, const void* src, bool ok) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sm100::smem_u32(dst)), "l"(src),
+               "r"(ok ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp4(void* dst, const void* src, bool ok) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(sm100::smem_u32(dst)), "l"(src),
+               "r"(ok ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// every group but the most recent one has landed (for this thread's copies)
+__device__ __forceinline__ void cp_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// rows [0, nvalid) of a tile of `rows` rows (row r at src + r * stride) into a padded bf16
+// tile with asynchronous copies; rows past nvalid become zeros
+template <int D>
+__device__ __forceinline__ void cp_tile(const __nv_bfloat16* __restrict__ src, int64_t stride, int rows, int nvalid,
+                                        __nv_bfloat16* dst) {
+  constexpr int VPR = D / 8, SH = D + 8;
+  for (int v = threadIdx.x; v < rows * VPR; v += NTM) {
+    const int r = v / VPR, c = (v % VPR) * 8;
+    const bool ok = r < nvalid;
+    cp16(dst + r * SH + c, src + (ok ? r : 0) * stride + c, ok);
+  }
+}
+
+// rowsum(dO * O) of `rows` rows, both from padded shared tiles
+template <int D>
+__device__ __forceinline__ void row_dot_smem(int rows, const __nv_bfloat16* dOs, const __nv_bfloat16* Os, float* dv) {
+  constexpr int SH = D + 8;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int r = w; r < rows; r += NTM / 32) {
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dOs + r * SH + c * 64 + 2 * lane));
+      const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Os + r * SH + c * 64 + 2 * lane));
+      s = fmaf(a.x, o.x, fmaf(a.y, o.y, s));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) dv[r] = s;
+  }
+}
 
 __device__ __forceinline__ void ldsm4(const __nv_bfloat16* p, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -429,19 +477,6 @@ __device__ __forceinline__ const __nv_bfloat16* frag_bn(const __nv_bfloat16* t, 
   return t + (r0 + (l & 7) + (l >> 4) * 8) * SH + c0 + ((l >> 3) & 1) * 8;
 }
 
-// rows [0, nvalid) of a tile of `rows` rows (row r at src + r * stride) into a padded bf16
-// tile; rows past nvalid become zeros
-template <int D>
-__device__ __forceinline__ void load_bf16_tile(const __nv_bfloat16* __restrict__ src, int64_t stride, int rows,
-                                               int nvalid, __nv_bfloat16* dst) {
-  constexpr int VPR = D / 8, SH = MSmem<D>::SH;
-  for (int v = threadIdx.x; v < rows * VPR; v += NTM) {
-    const int r = v / VPR, c = (v % VPR) * 8;
-    const uint4 x = r < nvalid ? __ldg(reinterpret_cast<const uint4*>(src + r * stride + c)) : make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint4*>(dst + r * SH + c) = x;
-  }
-}
-
 // rowsum(dO * O) of `rows` rows: dO from its padded shared tile, O from global memory
 template <int D>
 __device__ __forceinline__ void row_dot_bf16(const __nv_bfloat16* __restrict__ O, int64_t stride, int rows, int nvalid,
@@ -474,14 +509,11 @@ __global__ void __launch_bounds__(NTM)
   extern __shared__ __align__(16) unsigned char smraw[];
   __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smraw);
   __nv_bfloat16* Vs = Ks + S_::OWN;
-  __nv_bfloat16* Qs = Vs + S_::OWN;
-  __nv_bfloat16* dOs = Qs + S_::STR;
-  float* lse_s = reinterpret_cast<float*>(dOs + S_::STR);  // [ST]
-  float* dv = lse_s + MT;                                   // [ST]
-  float* bias = dv + MT;                                    // [MT]
-  float* dl_s = bias + MT;                                  // [MT]
-  int* posq = reinterpret_cast<int*>(dl_s + MT);            // [ST]
-  int* posk = posq + MT;                                    // [MT]
+  __nv_bfloat16* stream0 = Vs + S_::OWN;  // buffer b: Q, dO, O tiles at stream0 + 3 b STR
+  float* lse_b = reinterpret_cast<float*>(stream0 + 6 * S_::STR);  // [2][ST]
+  int* posq_b = reinterpret_cast<int*>(lse_b + 2 * ST);            // [2][ST]
+  float* dv = reinterpret_cast<float*>(posq_b + 2 * ST);           // [ST]
+  float* dl_s = dv + MT;                                           // [MT]
 
   const int C = p.C;
   const int unit = blockIdx.x / C, rank = blockIdx.x % C;
@@ -491,97 +523,120 @@ __global__ void __launch_bounds__(NTM)
   const int t = unit - p.tiles[b];  // key tile: tile 0 has the most query steps below it
   const int k0 = t * MT;
   const int kvalid = min(MT, sq.m - k0);
-  const int nsteps = (sq.m + ST - 1) / ST;  // query steps of the sequence; this tile starts at k0 / ST
+  const int qs0 = k0 / ST;                        // first query step at or below the diagonal
+  const int nq = (sq.m + ST - 1) / ST - qs0;      // query steps per head
   const int G = Hq / Hkv;
+  const int total = G * nq;                       // (head, query step) pairs of a KV head
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t4 = lane & 3;
   const int kr0 = 16 * w + g, kr1 = kr0 + 8;  // this thread's key rows within the tile
+  const int pk0 = kr0 < kvalid ? pos[sq.off + k0 + kr0] : INT_MAX;
+  const int pk1 = kr1 < kvalid ? pos[sq.off + k0 + kr1] : INT_MAX;
+  const float lg0 = (logg && kr0 < kvalid) ? __ldg(logg + sq.off + k0 + kr0) : 0.f;
+  const float lg1 = (logg && kr1 < kvalid) ? __ldg(logg + sq.off + k0 + kr1) : 0.f;
 
-  if (tid < MT) posk[tid] = tid < kvalid ? pos[sq.off + k0 + tid] : INT_MAX;
+  // step n of KV head kvh: head kvh * G + n / nq, query rows from (qs0 + n % nq) * ST
+  auto issue = [&](int kvh, int n, int buf) {
+    const int h = kvh * G + n / nq;
+    const int q0 = (qs0 + n % nq) * ST;
+    const int qvalid = min(ST, sq.m - q0);
+    const int64_t qrow = ((int64_t)(sq.off + q0) * Hq + h) * D;
+    __nv_bfloat16* base = stream0 + 3 * buf * S_::STR;
+    cp_tile<D>(Q + qrow, (int64_t)Hq * D, ST, qvalid, base);
+    cp_tile<D>(dO + qrow, (int64_t)Hq * D, ST, qvalid, base + S_::STR);
+    cp_tile<D>(O + qrow, (int64_t)Hq * D, ST, qvalid, base + 2 * S_::STR);
+    if (tid < ST) {
+      const bool ok = tid < qvalid;
+      const int64_t row = sq.off + q0 + (ok ? tid : 0);
+      cp4(lse_b + buf * ST + tid, lse + (int64_t)h * m_tot + row, ok);
+      cp4(posq_b + buf * ST + tid, pos + row, ok);
+    }
+  };
+
   float dl0 = 0.f, dl1 = 0.f;
   for (int kvh = rank; kvh < Hkv; kvh += C) {
-    __syncthreads();  // the previous KV head's readers are done with Ks and Vs
-    load_bf16_tile<D>(K + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, MT, kvalid, Ks);
-    load_bf16_tile<D>(V + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, MT, kvalid, Vs);
+    __syncthreads();  // the previous KV head's readers are done with every tile
+    cp_tile<D>(K + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, MT, kvalid, Ks);
+    cp_tile<D>(V + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, MT, kvalid, Vs);
+    issue(kvh, 0, 0);
+    cp_commit();
     float aK[NN][4], aV[NN][4];
 #pragma unroll
     for (int n = 0; n < NN; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) aK[n][e] = aV[n][e] = 0.f;
-    for (int hh = 0; hh < G; ++hh) {
-      const int h = kvh * G + hh;
+    for (int n = 0; n < total; ++n) {
+      const int buf = n & 1;
+      if (n + 1 < total) issue(kvh, n + 1, buf ^ 1);  // its buffer was released at the end of step n - 1
+      cp_commit();
+      cp_wait_prev();
+      __syncthreads();  // step n's tiles have landed for every thread
+      const int h = kvh * G + n / nq;
       const float gh = gain ? __ldg(gain + h) : 1.f;
-      for (int qs = k0 / ST; qs < nsteps; ++qs) {
-        const int q0 = qs * ST;
-        const int qvalid = min(ST, sq.m - q0);
-        __syncthreads();  // the previous step's readers are done with Qs, dOs and the vectors
-        if (tid < MT) bias[tid] = (logg && tid < kvalid) ? gh * __ldg(logg + sq.off + k0 + tid) : 0.f;
-        if (tid < ST) {
-          posq[tid] = tid < qvalid ? pos[sq.off + q0 + tid] : INT_MIN;
-          lse_s[tid] = tid < qvalid ? __ldg(lse + (int64_t)h * m_tot + sq.off + q0 + tid) : 0.f;
-        }
-        const int64_t qrow = ((int64_t)(sq.off + q0) * Hq + h) * D;
-        load_bf16_tile<D>(Q + qrow, (int64_t)Hq * D, ST, qvalid, Qs);
-        load_bf16_tile<D>(dO + qrow, (int64_t)Hq * D, ST, qvalid, dOs);
-        __syncthreads();
-        row_dot_bf16<D>(O + qrow, (int64_t)Hq * D, ST, qvalid, dOs, dv);
-        // S^T (keys x queries) = K Q^T and dP^T = V dO^T, 16 x 32 per warp
-        float sT[4][4], pT[4][4];
+      const int qvalid = min(ST, sq.m - (qs0 + n % nq) * ST);
+      const __nv_bfloat16* Qs = stream0 + 3 * buf * S_::STR;
+      const __nv_bfloat16* dOs = Qs + S_::STR;
+      const float* lse_s = lse_b + buf * ST;
+      const int* posq = posq_b + buf * ST;
+      row_dot_smem<D>(ST, dOs, dOs + S_::STR, dv);
+      // S^T (keys x queries) = K Q^T and dP^T = V dO^T, 16 x 32 per warp
+      float sT[4][4], pT[4][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sT[j][e] = pT[j][e] = 0.f;
+        for (int e = 0; e < 4; ++e) sT[j][e] = pT[j][e] = 0.f;
 #pragma unroll
-        for (int kd = 0; kd < D / 16; ++kd) {
-          uint32_t ak[4], av[4];
-          ldsm4(frag_a<SH>(Ks, 16 * w, 16 * kd), ak);
-          ldsm4(frag_a<SH>(Vs, 16 * w, 16 * kd), av);
+      for (int kd = 0; kd < D / 16; ++kd) {
+        uint32_t ak[4], av[4];
+        ldsm4(frag_a<SH>(Ks, 16 * w, 16 * kd), ak);
+        ldsm4(frag_a<SH>(Vs, 16 * w, 16 * kd), av);
 #pragma unroll
-          for (int np = 0; np < 2; ++np) {
-            uint32_t bq[4], bo[4];
-            ldsm4(frag_bn<SH>(Qs, 16 * np, 16 * kd), bq);
-            ldsm4(frag_bn<SH>(dOs, 16 * np, 16 * kd), bo);
-            mma16816(sT[2 * np], ak, bq[0], bq[1]);
-            mma16816(sT[2 * np + 1], ak, bq[2], bq[3]);
-            mma16816(pT[2 * np], av, bo[0], bo[1]);
-            mma16816(pT[2 * np + 1], av, bo[2], bo[3]);
-          }
-        }
-        __syncthreads();  // dv is complete
-        // P^T and dS^T in place: rows kr0 / kr1 (keys), columns 8j + 2t4 + {0, 1} (queries)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int kr = e < 2 ? kr0 : kr1, qc = 8 * j + 2 * t4 + (e & 1);
-            const bool vis = posk[kr] <= posq[qc];
-            const float pv = vis ? expf(fmaf(scale, sT[j][e], bias[kr] - lse_s[qc])) : 0.f;
-            const float ds = pv * (pT[j][e] - dv[qc]);
-            sT[j][e] = pv;
-            pT[j][e] = ds;
-            if (e < 2) dl0 = fmaf(gh, ds, dl0);
-            else dl1 = fmaf(gh, ds, dl1);
-          }
-        // dV += P^T dO and dK += dS^T Q: k runs over the 32 queries (two steps of 16)
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const uint32_t ap[4] = {pack_bf16(sT[2 * kk][0], sT[2 * kk][1]), pack_bf16(sT[2 * kk][2], sT[2 * kk][3]),
-                                  pack_bf16(sT[2 * kk + 1][0], sT[2 * kk + 1][1]),
-                                  pack_bf16(sT[2 * kk + 1][2], sT[2 * kk + 1][3])};
-          const uint32_t as[4] = {pack_bf16(pT[2 * kk][0], pT[2 * kk][1]), pack_bf16(pT[2 * kk][2], pT[2 * kk][3]),
-                                  pack_bf16(pT[2 * kk + 1][0], pT[2 * kk + 1][1]),
-                                  pack_bf16(pT[2 * kk + 1][2], pT[2 * kk + 1][3])};
-#pragma unroll
-          for (int u = 0; u < D / 16; ++u) {
-            uint32_t bo[4], bq[4];
-            ldsm4t(frag_a<SH>(dOs, 16 * kk, 16 * u), bo);
-            ldsm4t(frag_a<SH>(Qs, 16 * kk, 16 * u), bq);
-            mma16816(aV[2 * u], ap, bo[0], bo[1]);
-            mma16816(aV[2 * u + 1], ap, bo[2], bo[3]);
-            mma16816(aK[2 * u], as, bq[0], bq[1]);
-            mma16816(aK[2 * u + 1], as, bq[2], bq[3]);
-          }
+        for (int np = 0; np < 2; ++np) {
+          uint32_t bq[4], bo[4];
+          ldsm4(frag_bn<SH>(Qs, 16 * np, 16 * kd), bq);
+          ldsm4(frag_bn<SH>(dOs, 16 * np, 16 * kd), bo);
+          mma16816(sT[2 * np], ak, bq[0], bq[1]);
+          mma16816(sT[2 * np + 1], ak, bq[2], bq[3]);
+          mma16816(pT[2 * np], av, bo[0], bo[1]);
+          mma16816(pT[2 * np + 1], av, bo[2], bo[3]);
         }
       }
+      __syncthreads();  // dv is complete
+      // P^T and dS^T in place: rows kr0 / kr1 (keys), columns 8j + 2t4 + {0, 1} (queries)
+      const float b0 = gh * lg0, b1 = gh * lg1;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int qc = 8 * j + 2 * t4 + (e & 1);
+          const bool vis = qc < qvalid && (e < 2 ? pk0 : pk1) <= posq[qc];
+          const float pv = vis ? expf(fmaf(scale, sT[j][e], (e < 2 ? b0 : b1) - lse_s[qc])) : 0.f;
+          const float ds = pv * (pT[j][e] - dv[qc]);
+          sT[j][e] = pv;
+          pT[j][e] = ds;
+          if (e < 2) dl0 = fmaf(gh, ds, dl0);
+          else dl1 = fmaf(gh, ds, dl1);
+        }
+      // dV += P^T dO and dK += dS^T Q: k runs over the 32 queries (two steps of 16)
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        const uint32_t ap[4] = {pack_bf16(sT[2 * kk][0], sT[2 * kk][1]), pack_bf16(sT[2 * kk][2], sT[2 * kk][3]),
+                                pack_bf16(sT[2 * kk + 1][0], sT[2 * kk + 1][1]),
+                                pack_bf16(sT[2 * kk + 1][2], sT[2 * kk + 1][3])};
+        const uint32_t as[4] = {pack_bf16(pT[2 * kk][0], pT[2 * kk][1]), pack_bf16(pT[2 * kk][2], pT[2 * kk][3]),
+                                pack_bf16(pT[2 * kk + 1][0], pT[2 * kk + 1][1]),
+                                pack_bf16(pT[2 * kk + 1][2], pT[2 * kk + 1][3])};
+#pragma unroll
+        for (int u = 0; u < D / 16; ++u) {
+          uint32_t bo[4], bq[4];
+          ldsm4t(frag_a<SH>(dOs, 16 * kk, 16 * u), bo);
+          ldsm4t(frag_a<SH>(Qs, 16 * kk, 16 * u), bq);
+          mma16816(aV[2 * u], ap, bo[0], bo[1]);
+          mma16816(aV[2 * u + 1], ap, bo[2], bo[3]);
+          mma16816(aK[2 * u], as, bq[0], bq[1]);
+          mma16816(aK[2 * u + 1], as, bq[2], bq[3]);
+        }
+      }
+      __syncthreads();  // every read of this buffer is done: step n + 2 may refill it
     }
     // rows kr0 / kr1 of dK (scaled) and dV for this KV head, columns 8n + 2t4 + {0, 1}
 #pragma unroll
@@ -643,13 +698,12 @@ __global__ void __launch_bounds__(NTM)
   extern __shared__ __align__(16) unsigned char smraw[];
   __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smraw);
   __nv_bfloat16* dOs = Qs + S_::OWN;
-  __nv_bfloat16* Ks = dOs + S_::OWN;
-  __nv_bfloat16* Vs = Ks + S_::STR;
-  float* lse_s = reinterpret_cast<float*>(Vs + S_::STR);  // [MT]
-  float* dv = lse_s + MT;                                  // [MT]
-  float* bias = dv + MT;                                   // [ST]
-  int* posq = reinterpret_cast<int*>(bias + 2 * MT);       // [MT]
-  int* posk = posq + MT;                                   // [ST]
+  __nv_bfloat16* stream0 = dOs + S_::OWN;  // buffer b: K, V tiles at stream0 + 2 b STR
+  float* lse_s = reinterpret_cast<float*>(stream0 + 6 * S_::STR);  // [MT]
+  float* dv = lse_s + MT;                                          // [MT]
+  int* posq = reinterpret_cast<int*>(dv + MT);                     // [MT]
+  float* lgk_b = reinterpret_cast<float*>(posq + MT);              // [2][ST] log g of the keys
+  int* posk_b = reinterpret_cast<int*>(lgk_b + 2 * ST);            // [2][ST]
 
   const int unit = blockIdx.x, h = blockIdx.y;
   int b = 0;
@@ -672,11 +726,25 @@ __global__ void __launch_bounds__(NTM)
     if (ok && h == 0 && q0 + tid > 0 && dev_status && pos[sq.off + q0 + tid - 1] >= posq[tid])
       atomicOr(dev_status, TG_DEV_POS_NOT_ASCENDING);
   }
+  // key step ks: keys from ks * ST, their K and V rows, log g and positions
+  auto issue = [&](int ks, int buf) {
+    const int k0 = ks * ST;
+    const int kvalid = min(ST, sq.m - k0);
+    __nv_bfloat16* base = stream0 + 2 * buf * S_::STR;
+    cp_tile<D>(K + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, ST, kvalid, base);
+    cp_tile<D>(V + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, ST, kvalid, base + S_::STR);
+    if (tid < ST) {
+      const bool ok = tid < kvalid;
+      const int64_t row = sq.off + k0 + (ok ? tid : 0);
+      cp4(lgk_b + buf * ST + tid, logg ? logg + row : reinterpret_cast<const float*>(pos + row), ok && logg);
+      cp4(posk_b + buf * ST + tid, pos + row, ok);
+    }
+  };
   const int64_t qrow = ((int64_t)(sq.off + q0) * Hq + h) * D;
-  load_bf16_tile<D>(Q + qrow, (int64_t)Hq * D, MT, qvalid, Qs);
-  load_bf16_tile<D>(dO + qrow, (int64_t)Hq * D, MT, qvalid, dOs);
-  __syncthreads();
-  row_dot_bf16<D>(O + qrow, (int64_t)Hq * D, MT, qvalid, dOs, dv);
+  cp_tile<D>(Q + qrow, (int64_t)Hq * D, MT, qvalid, Qs);
+  cp_tile<D>(dO + qrow, (int64_t)Hq * D, MT, qvalid, dOs);
+  issue(0, 0);
+  cp_commit();
   float aQ[NN][4];
 #pragma unroll
   for (int n = 0; n < NN; ++n)
@@ -684,17 +752,17 @@ __global__ void __launch_bounds__(NTM)
     for (int e = 0; e < 4; ++e) aQ[n][e] = 0.f;
   const int nks = (q0 + qvalid - 1) / ST + 1;  // key steps up to the tile's last row
   for (int ks = 0; ks < nks; ++ks) {
-    const int k0 = ks * ST;
-    const int kvalid = min(ST, sq.m - k0);
-    __syncthreads();  // the previous step's readers are done with Ks, Vs and the key vectors
-    if (tid < ST) {
-      const bool ok = tid < kvalid;
-      bias[tid] = (logg && ok) ? gh * __ldg(logg + sq.off + k0 + tid) : 0.f;
-      posk[tid] = ok ? pos[sq.off + k0 + tid] : INT_MAX;
-    }
-    load_bf16_tile<D>(K + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, ST, kvalid, Ks);
-    load_bf16_tile<D>(V + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, ST, kvalid, Vs);
-    __syncthreads();
+    const int buf = ks & 1;
+    if (ks + 1 < nks) issue(ks + 1, buf ^ 1);  // its buffer was released at the end of step ks - 1
+    cp_commit();
+    cp_wait_prev();
+    __syncthreads();  // step ks's tiles (and, at ks = 0, Q and dO) have landed for every thread
+    if (ks == 0) row_dot_bf16<D>(O + qrow, (int64_t)Hq * D, MT, qvalid, dOs, dv);
+    const int kvalid = min(ST, sq.m - ks * ST);
+    const __nv_bfloat16* Ks = stream0 + 2 * buf * S_::STR;
+    const __nv_bfloat16* Vs = Ks + S_::STR;
+    const float* lgk = lgk_b + buf * ST;
+    const int* posk = posk_b + buf * ST;
     // S = Q K^T and dP = dO V^T, 16 x 32 per warp
     float sc[4][4], dp[4][4];
 #pragma unroll
@@ -717,14 +785,15 @@ __global__ void __launch_bounds__(NTM)
         mma16816(dp[2 * np + 1], ao, bv[2], bv[3]);
       }
     }
+    __syncthreads();  // dv is complete (written at ks = 0)
     // dS in place: rows qr0 / qr1 (queries), columns 8j + 2t4 + {0, 1} (keys)
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int qr = e < 2 ? qr0 : qr1, kc = 8 * j + 2 * t4 + (e & 1);
-        const bool vis = posk[kc] <= posq[qr];
-        const float pv = vis ? expf(fmaf(scale, sc[j][e], bias[kc] - lse_s[qr])) : 0.f;
+        const bool vis = kc < kvalid && posk[kc] <= posq[qr];
+        const float pv = vis ? expf(fmaf(scale, sc[j][e], gh * lgk[kc] - lse_s[qr])) : 0.f;
         dp[j][e] = pv * (dp[j][e] - dv[qr]);
       }
     // dQ += dS K: k runs over the 32 keys (two steps of 16)
@@ -741,6 +810,7 @@ __global__ void __launch_bounds__(NTM)
         mma16816(aQ[2 * u + 1], as, bk[2], bk[3]);
       }
     }
+    __syncthreads();  // every read of this buffer is done: step ks + 2 may refill it
   }
 #pragma unroll
   for (int n = 0; n < NN; ++n) {

@@ -7,6 +7,7 @@
 
 #include <vector>
 
+#include "tg_attn_bwd.cuh"
 #include "tg_internal.cuh"
 
 namespace tg {
@@ -54,7 +55,7 @@ tg_status check_device() {
   return TG_OK;
 }
 
-static bool g_attr_set[ATTR_SLOTS][64];
+static bool g_attr_set[ATTR_ALL][64];  // the forward path's slots, then the backward's
 
 static int current_device() {
   int dev = 0;

@@ -29,9 +29,7 @@ enum {
   ATTR_SCORE64 = 0, ATTR_SCORE128, ATTR_SCORE256,
   ATTR_SELECT, ATTR_GATHER,
   ATTR_ATTN64, ATTR_ATTN64_UN, ATTR_ATTN128, ATTR_ATTN128_UN,
-  ATTR_QKV,
-  ATTR_BWD,  // 4 slots: CUDA-core (f32) D 64, 128, then tensor-core (bf16) D 64, 128
-  ATTR_SLOTS = ATTR_BWD + 4
+  ATTR_QKV, ATTR_SLOTS
 };
 bool attrs_needed(int slot);
 void mark_attrs_set(int slot);
@@ -138,31 +136,6 @@ tg_status launch_qkv_rope(const void* Hk, int64_t M, int d, const void* W, const
                           int D, float theta, void* Q, void* K, void* V, int32_t* dev_status, cudaStream_t st);
 
 tg_status launch_attn_simt(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);
-
-// Gradients of the gated attention (normalised form): dQ, dK, dV (f32) and optionally d log g,
-// d score (f32), from the forward's inputs, O and lse and the upstream dO.
-struct AttnBwdArgs {
-  tg_dtype dt;
-  const void* Q;
-  const void* K;
-  const void* V;
-  const void* O;
-  const void* dO;
-  const float* logg;
-  const float* head_gain;
-  const int32_t* pos;
-  const float* lse;
-  int Hq, Hkv, D;
-  float scale;
-  float* dQ;
-  float* dK;
-  float* dV;
-  float* dlogg;
-  float* dscore;
-  int32_t* dev_status;
-  int64_t m_tot;
-};
-tg_status launch_attn_bwd(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);
 tg_status launch_attn_tc(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);
 
 }  // namespace tg
