@@ -384,8 +384,11 @@ template <int D>
 struct MSmem {
   static constexpr int SH = D + 8;  // padded row stride in bf16 elements (16-byte pad)
   static constexpr int OWN = MT * SH, STR = ST * SH;
-  // two own tiles, two buffers of three streamed tiles (bf16), then 8 vectors of 64 32-bit values
-  static constexpr int BYTES = (2 * OWN + 6 * STR) * 2 + 8 * MT * 4;
+  // dK/dV kernel: two own tiles, two buffers of three streamed tiles (Q, dO, O), then vectors;
+  // dQ kernel: two own tiles, two buffers of two streamed tiles (K, V), then vectors
+  static constexpr int VEC = 6 * MT * 4;  // up to 6 vectors of 64 32-bit values
+  static constexpr int BYTES_DKDV = (2 * OWN + 6 * STR) * 2 + VEC;
+  static constexpr int BYTES_DQ = (2 * OWN + 4 * STR) * 2 + VEC;
 };
 
 // 16-byte and 4-byte asynchronous copies global -> shared; a copy with ok == false reads
@@ -699,7 +702,7 @@ __global__ void __launch_bounds__(NTM)
   __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smraw);
   __nv_bfloat16* dOs = Qs + S_::OWN;
   __nv_bfloat16* stream0 = dOs + S_::OWN;  // buffer b: K, V tiles at stream0 + 2 b STR
-  float* lse_s = reinterpret_cast<float*>(stream0 + 6 * S_::STR);  // [MT]
+  float* lse_s = reinterpret_cast<float*>(stream0 + 4 * S_::STR);  // [MT]
   float* dv = lse_s + MT;                                          // [MT]
   int* posq = reinterpret_cast<int*>(dv + MT);                     // [MT]
   float* lgk_b = reinterpret_cast<float*>(posq + MT);              // [2][ST] log g of the keys
@@ -879,15 +882,14 @@ template <int D>
 tg_status launch_mma(const AttnBwdArgs& a, const BwdParams& p0, cudaStream_t st) {
   BwdParams p = p0;
   const int units = p.tiles[p.nseq];
-  constexpr int SMEM = MSmem<D>::BYTES;
+  constexpr int SMEM_DKDV = MSmem<D>::BYTES_DKDV, SMEM_DQ = MSmem<D>::BYTES_DQ;
   auto kdkdv = attn_bwd_dkdv_mma<D>;
   auto kdq = attn_bwd_dq_mma<D>;
   const int slot = ATTR_BWD + 2 + (D == 128 ? 1 : 0);
   if (attrs_needed(slot)) {
-    for (const void* k : {(const void*)kdkdv, (const void*)kdq}) {
-      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-      if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: cudaFuncSetAttribute");
-    }
+    cudaError_t e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DKDV);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DQ);
+    if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: cudaFuncSetAttribute");
     mark_attrs_set(slot);
   }
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.Q);
@@ -900,7 +902,7 @@ tg_status launch_mma(const AttnBwdArgs& a, const BwdParams& p0, cudaStream_t st)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(units * p.C));
   cfg.blockDim = dim3(NTM);
-  cfg.dynamicSmemBytes = (size_t)SMEM;
+  cfg.dynamicSmemBytes = (size_t)SMEM_DKDV;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -916,7 +918,7 @@ tg_status launch_mma(const AttnBwdArgs& a, const BwdParams& p0, cudaStream_t st)
   cudaLaunchConfig_t cq = {};
   cq.gridDim = dim3((unsigned)units, (unsigned)a.Hq);
   cq.blockDim = dim3(NTM);
-  cq.dynamicSmemBytes = (size_t)SMEM;
+  cq.dynamicSmemBytes = (size_t)SMEM_DQ;
   cq.stream = st;
   e = cudaLaunchKernelEx(&cq, kdq, q, k, v, o, dO, a.logg, a.head_gain, a.pos, a.lse, a.scale, a.Hq, a.Hkv, a.m_tot,
                          a.dQ, a.dev_status, p);
