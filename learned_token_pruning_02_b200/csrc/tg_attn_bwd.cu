@@ -387,7 +387,8 @@ struct MSmem {
   // dK/dV kernel: two own tiles, two buffers of three streamed tiles (Q, dO, O), then vectors;
   // dQ kernel: two own tiles, two buffers of two streamed tiles (K, V), then vectors
   static constexpr int VEC = 6 * MT * 4;  // up to 6 vectors of 64 32-bit values
-  static constexpr int BYTES_DKDV = (2 * OWN + 6 * STR) * 2 + VEC;
+  // dK/dV kernel with NWG warp groups: each group has its own two buffers and 5 vectors of 32
+  static constexpr int bytes_dkdv(int nwg) { return (2 * OWN + nwg * 6 * STR) * 2 + (nwg * 5 * ST + MT) * 4; }
   static constexpr int BYTES_DQ = (2 * OWN + 4 * STR) * 2 + VEC;
 };
 
@@ -404,28 +405,32 @@ __device__ __forceinline__ void cp4(void* dst, const void* src, bool ok) {
                : "memory");
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 // every group but the most recent one has landed (for this thread's copies)
 __device__ __forceinline__ void cp_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // rows [0, nvalid) of a tile of `rows` rows (row r at src + r * stride) into a padded bf16
 // tile with asynchronous copies; rows past nvalid become zeros
+// (lt: this thread's index among the nthr threads that share the copy)
 template <int D>
 __device__ __forceinline__ void cp_tile(const __nv_bfloat16* __restrict__ src, int64_t stride, int rows, int nvalid,
-                                        __nv_bfloat16* dst) {
+                                        __nv_bfloat16* dst, int lt = threadIdx.x, int nthr = NTM) {
   constexpr int VPR = D / 8, SH = D + 8;
-  for (int v = threadIdx.x; v < rows * VPR; v += NTM) {
+  for (int v = lt; v < rows * VPR; v += nthr) {
     const int r = v / VPR, c = (v % VPR) * 8;
     const bool ok = r < nvalid;
     cp16(dst + r * SH + c, src + (ok ? r : 0) * stride + c, ok);
   }
 }
 
-// rowsum(dO * O) of `rows` rows, both from padded shared tiles
+// rowsum(dO * O) of `rows` rows, both from padded shared tiles, by the 4 warps of one group
+// (wl: this warp's index in the group)
 template <int D>
-__device__ __forceinline__ void row_dot_smem(int rows, const __nv_bfloat16* dOs, const __nv_bfloat16* Os, float* dv) {
+__device__ __forceinline__ void row_dot_smem(int rows, const __nv_bfloat16* dOs, const __nv_bfloat16* Os, float* dv,
+                                             int wl) {
   constexpr int SH = D + 8;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  for (int r = w; r < rows; r += NTM / 32) {
+  const int lane = threadIdx.x & 31;
+  for (int r = wl; r < rows; r += NTM / 32) {
     float s = 0.f;
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
@@ -499,8 +504,15 @@ __device__ __forceinline__ void row_dot_bf16(const __nv_bfloat16* __restrict__ O
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(NTM)
+// bar.sync on a named barrier shared by the 4 warps of one warp group
+__device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+
+// NWG warp groups of 4 warps share the 64-key tile; group grp takes the query heads
+// grp, grp + NWG, ... of the KV group, so each warp's chain of steps is G / NWG heads long.
+// A group synchronises on its own named barrier (1 + grp); its dK / dV are added to group 0's
+// through shared memory at the end of each KV head, in a fixed order.
+template <int D, int NWG>
+__global__ void __launch_bounds__(NTM * NWG, 1)
     attn_bwd_dkdv_mma(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                       const __nv_bfloat16* __restrict__ V, const __nv_bfloat16* __restrict__ O,
                       const __nv_bfloat16* __restrict__ dO, const float* __restrict__ logg,
@@ -510,13 +522,17 @@ __global__ void __launch_bounds__(NTM)
   using S_ = MSmem<D>;
   constexpr int SH = S_::SH, NN = D / 8;  // n-tiles of 8 across the head dimension
   extern __shared__ __align__(16) unsigned char smraw[];
+  const int tid = threadIdx.x, grp = tid >> 7, lt = tid & (NTM - 1);
+  const int lane = tid & 31, wl = (tid >> 5) & 3, g = lane >> 2, t4 = lane & 3;
   __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smraw);
   __nv_bfloat16* Vs = Ks + S_::OWN;
-  __nv_bfloat16* stream0 = Vs + S_::OWN;  // buffer b: Q, dO, O tiles at stream0 + 3 b STR
-  float* lse_b = reinterpret_cast<float*>(stream0 + 6 * S_::STR);  // [2][ST]
-  int* posq_b = reinterpret_cast<int*>(lse_b + 2 * ST);            // [2][ST]
-  float* dv = reinterpret_cast<float*>(posq_b + 2 * ST);           // [ST]
-  float* dl_s = dv + MT;                                           // [MT]
+  // group grp, buffer b: Q, dO, O tiles at stream0 + (2 grp + b) 3 STR
+  __nv_bfloat16* stream0 = Vs + S_::OWN;
+  float* vec0 = reinterpret_cast<float*>(stream0 + NWG * 6 * S_::STR);
+  float* lse_b = vec0 + grp * 5 * ST;                    // [2][ST] this group's
+  int* posq_b = reinterpret_cast<int*>(lse_b + 2 * ST);  // [2][ST]
+  float* dv = lse_b + 4 * ST;                            // [ST]
+  float* dl_s = vec0 + NWG * 5 * ST;                     // [MT]
 
   const int C = p.C;
   const int unit = blockIdx.x / C, rank = blockIdx.x % C;
@@ -526,40 +542,44 @@ __global__ void __launch_bounds__(NTM)
   const int t = unit - p.tiles[b];  // key tile: tile 0 has the most query steps below it
   const int k0 = t * MT;
   const int kvalid = min(MT, sq.m - k0);
-  const int qs0 = k0 / ST;                        // first query step at or below the diagonal
-  const int nq = (sq.m + ST - 1) / ST - qs0;      // query steps per head
+  const int qs0 = k0 / ST;                    // first query step at or below the diagonal
+  const int nq = (sq.m + ST - 1) / ST - qs0;  // query steps per head
   const int G = Hq / Hkv;
-  const int total = G * nq;                       // (head, query step) pairs of a KV head
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t4 = lane & 3;
-  const int kr0 = 16 * w + g, kr1 = kr0 + 8;  // this thread's key rows within the tile
+  const int nh = (G - grp + NWG - 1) / NWG;   // heads of this group (NWG <= G: at least 1)
+  const int total = nh * nq;                  // (head, query step) pairs of this group per KV head
+  const int kr0 = 16 * wl + g, kr1 = kr0 + 8;  // this thread's key rows within the tile
   const int pk0 = kr0 < kvalid ? pos[sq.off + k0 + kr0] : INT_MAX;
   const int pk1 = kr1 < kvalid ? pos[sq.off + k0 + kr1] : INT_MAX;
   const float lg0 = (logg && kr0 < kvalid) ? __ldg(logg + sq.off + k0 + kr0) : 0.f;
   const float lg1 = (logg && kr1 < kvalid) ? __ldg(logg + sq.off + k0 + kr1) : 0.f;
 
-  // step n of KV head kvh: head kvh * G + n / nq, query rows from (qs0 + n % nq) * ST
+  // step n of this group for KV head kvh: head kvh G + grp + NWG (n / nq), query rows from
+  // (qs0 + n % nq) ST
   auto issue = [&](int kvh, int n, int buf) {
-    const int h = kvh * G + n / nq;
+    const int h = kvh * G + grp + NWG * (n / nq);
     const int q0 = (qs0 + n % nq) * ST;
     const int qvalid = min(ST, sq.m - q0);
     const int64_t qrow = ((int64_t)(sq.off + q0) * Hq + h) * D;
-    __nv_bfloat16* base = stream0 + 3 * buf * S_::STR;
-    cp_tile<D>(Q + qrow, (int64_t)Hq * D, ST, qvalid, base);
-    cp_tile<D>(dO + qrow, (int64_t)Hq * D, ST, qvalid, base + S_::STR);
-    cp_tile<D>(O + qrow, (int64_t)Hq * D, ST, qvalid, base + 2 * S_::STR);
-    if (tid < ST) {
-      const bool ok = tid < qvalid;
-      const int64_t row = sq.off + q0 + (ok ? tid : 0);
-      cp4(lse_b + buf * ST + tid, lse + (int64_t)h * m_tot + row, ok);
-      cp4(posq_b + buf * ST + tid, pos + row, ok);
+    __nv_bfloat16* base = stream0 + (2 * grp + buf) * 3 * S_::STR;
+    cp_tile<D>(Q + qrow, (int64_t)Hq * D, ST, qvalid, base, lt, NTM);
+    cp_tile<D>(dO + qrow, (int64_t)Hq * D, ST, qvalid, base + S_::STR, lt, NTM);
+    cp_tile<D>(O + qrow, (int64_t)Hq * D, ST, qvalid, base + 2 * S_::STR, lt, NTM);
+    if (lt < ST) {
+      const bool ok = lt < qvalid;
+      const int64_t row = sq.off + q0 + (ok ? lt : 0);
+      cp4(lse_b + buf * ST + lt, lse + (int64_t)h * m_tot + row, ok);
+      cp4(posq_b + buf * ST + lt, pos + row, ok);
     }
   };
 
   float dl0 = 0.f, dl1 = 0.f;
   for (int kvh = rank; kvh < Hkv; kvh += C) {
-    __syncthreads();  // the previous KV head's readers are done with every tile
-    cp_tile<D>(K + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, MT, kvalid, Ks);
-    cp_tile<D>(V + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, MT, kvalid, Vs);
+    __syncthreads();  // every group is done with the previous KV head (tiles and reduction)
+    cp_tile<D>(K + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, MT, kvalid, Ks, tid, NTM * NWG);
+    cp_tile<D>(V + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, MT, kvalid, Vs, tid, NTM * NWG);
+    cp_commit();
+    cp_wait_all();
+    __syncthreads();  // K and V have landed for every thread of both groups
     issue(kvh, 0, 0);
     cp_commit();
     float aK[NN][4], aV[NN][4];
@@ -572,15 +592,15 @@ __global__ void __launch_bounds__(NTM)
       if (n + 1 < total) issue(kvh, n + 1, buf ^ 1);  // its buffer was released at the end of step n - 1
       cp_commit();
       cp_wait_prev();
-      __syncthreads();  // step n's tiles have landed for every thread
-      const int h = kvh * G + n / nq;
+      group_sync(1 + grp);  // step n's tiles have landed for every thread of the group
+      const int h = kvh * G + grp + NWG * (n / nq);
       const float gh = gain ? __ldg(gain + h) : 1.f;
       const int qvalid = min(ST, sq.m - (qs0 + n % nq) * ST);
-      const __nv_bfloat16* Qs = stream0 + 3 * buf * S_::STR;
+      const __nv_bfloat16* Qs = stream0 + (2 * grp + buf) * 3 * S_::STR;
       const __nv_bfloat16* dOs = Qs + S_::STR;
       const float* lse_s = lse_b + buf * ST;
       const int* posq = posq_b + buf * ST;
-      row_dot_smem<D>(ST, dOs, dOs + S_::STR, dv);
+      row_dot_smem<D>(ST, dOs, dOs + S_::STR, dv, wl);
       // S^T (keys x queries) = K Q^T and dP^T = V dO^T, 16 x 32 per warp
       float sT[4][4], pT[4][4];
 #pragma unroll
@@ -590,8 +610,8 @@ __global__ void __launch_bounds__(NTM)
 #pragma unroll
       for (int kd = 0; kd < D / 16; ++kd) {
         uint32_t ak[4], av[4];
-        ldsm4(frag_a<SH>(Ks, 16 * w, 16 * kd), ak);
-        ldsm4(frag_a<SH>(Vs, 16 * w, 16 * kd), av);
+        ldsm4(frag_a<SH>(Ks, 16 * wl, 16 * kd), ak);
+        ldsm4(frag_a<SH>(Vs, 16 * wl, 16 * kd), av);
 #pragma unroll
         for (int np = 0; np < 2; ++np) {
           uint32_t bq[4], bo[4];
@@ -603,7 +623,7 @@ __global__ void __launch_bounds__(NTM)
           mma16816(pT[2 * np + 1], av, bo[2], bo[3]);
         }
       }
-      __syncthreads();  // dv is complete
+      group_sync(1 + grp);  // dv is complete
       // P^T and dS^T in place: rows kr0 / kr1 (keys), columns 8j + 2t4 + {0, 1} (queries)
       const float b0 = gh * lg0, b1 = gh * lg1;
 #pragma unroll
@@ -639,32 +659,77 @@ __global__ void __launch_bounds__(NTM)
           mma16816(aK[2 * u + 1], as, bq[2], bq[3]);
         }
       }
-      __syncthreads();  // every read of this buffer is done: step n + 2 may refill it
+      group_sync(1 + grp);  // every read of this buffer is done: step n + 2 may refill it
+    }
+    // group 1's dK / dV go through shared memory (the stream buffers, now idle) into group 0's
+    if (NWG > 1) {
+      float* red = reinterpret_cast<float*>(stream0);  // [2][MT][D]: dK, then dV
+      __syncthreads();  // both groups are done with their stream buffers
+      if (grp == 1) {
+#pragma unroll
+        for (int n = 0; n < NN; ++n) {
+          const int c = 8 * n + 2 * t4;
+          *reinterpret_cast<float2*>(red + kr0 * D + c) = make_float2(aK[n][0], aK[n][1]);
+          *reinterpret_cast<float2*>(red + kr1 * D + c) = make_float2(aK[n][2], aK[n][3]);
+          *reinterpret_cast<float2*>(red + (MT + kr0) * D + c) = make_float2(aV[n][0], aV[n][1]);
+          *reinterpret_cast<float2*>(red + (MT + kr1) * D + c) = make_float2(aV[n][2], aV[n][3]);
+        }
+      }
+      __syncthreads();
+      if (grp == 0) {
+#pragma unroll
+        for (int n = 0; n < NN; ++n) {
+          const int c = 8 * n + 2 * t4;
+          const float2 k0v = *reinterpret_cast<const float2*>(red + kr0 * D + c);
+          const float2 k1v = *reinterpret_cast<const float2*>(red + kr1 * D + c);
+          const float2 v0v = *reinterpret_cast<const float2*>(red + (MT + kr0) * D + c);
+          const float2 v1v = *reinterpret_cast<const float2*>(red + (MT + kr1) * D + c);
+          aK[n][0] += k0v.x;
+          aK[n][1] += k0v.y;
+          aK[n][2] += k1v.x;
+          aK[n][3] += k1v.y;
+          aV[n][0] += v0v.x;
+          aV[n][1] += v0v.y;
+          aV[n][2] += v1v.x;
+          aV[n][3] += v1v.y;
+        }
+      }
     }
     // rows kr0 / kr1 of dK (scaled) and dV for this KV head, columns 8n + 2t4 + {0, 1}
+    if (grp == 0) {
 #pragma unroll
-    for (int n = 0; n < NN; ++n) {
-      const int c = 8 * n + 2 * t4;
-      if (kr0 < kvalid) {
-        const int64_t r = ((int64_t)(sq.off + k0 + kr0) * Hkv + kvh) * D + c;
-        *reinterpret_cast<float2*>(dK + r) = make_float2(scale * aK[n][0], scale * aK[n][1]);
-        *reinterpret_cast<float2*>(dV + r) = make_float2(aV[n][0], aV[n][1]);
-      }
-      if (kr1 < kvalid) {
-        const int64_t r = ((int64_t)(sq.off + k0 + kr1) * Hkv + kvh) * D + c;
-        *reinterpret_cast<float2*>(dK + r) = make_float2(scale * aK[n][2], scale * aK[n][3]);
-        *reinterpret_cast<float2*>(dV + r) = make_float2(aV[n][2], aV[n][3]);
+      for (int n = 0; n < NN; ++n) {
+        const int c = 8 * n + 2 * t4;
+        if (kr0 < kvalid) {
+          const int64_t r = ((int64_t)(sq.off + k0 + kr0) * Hkv + kvh) * D + c;
+          *reinterpret_cast<float2*>(dK + r) = make_float2(scale * aK[n][0], scale * aK[n][1]);
+          *reinterpret_cast<float2*>(dV + r) = make_float2(aV[n][0], aV[n][1]);
+        }
+        if (kr1 < kvalid) {
+          const int64_t r = ((int64_t)(sq.off + k0 + kr1) * Hkv + kvh) * D + c;
+          *reinterpret_cast<float2*>(dK + r) = make_float2(scale * aK[n][2], scale * aK[n][3]);
+          *reinterpret_cast<float2*>(dV + r) = make_float2(aV[n][2], aV[n][3]);
+        }
       }
     }
   }
-  // d log g: the quad holding a key row adds its columns, then the cluster adds its KV heads
+  // d log g: the quad holding a key row adds its columns, the groups add in order, then the
+  // cluster adds its KV heads
   dl0 += __shfl_xor_sync(0xffffffffu, dl0, 1);
   dl0 += __shfl_xor_sync(0xffffffffu, dl0, 2);
   dl1 += __shfl_xor_sync(0xffffffffu, dl1, 1);
   dl1 += __shfl_xor_sync(0xffffffffu, dl1, 2);
-  if (t4 == 0) {
+  __syncthreads();  // dl_s may alias nothing in use, but keep the groups' writes ordered
+  if (grp == 0 && t4 == 0) {
     dl_s[kr0] = dl0;
     dl_s[kr1] = dl1;
+  }
+  if (NWG > 1) {
+    __syncthreads();
+    if (grp == 1 && t4 == 0) {
+      dl_s[kr0] += dl0;
+      dl_s[kr1] += dl1;
+    }
   }
   if (C > 1) {
     cg::cluster_group cluster = cg::this_cluster();
@@ -878,14 +943,15 @@ tg_status launch_td(const AttnBwdArgs& a, const BwdParams& p0, cudaStream_t st) 
   return cuda_status(e, "tg_gated_attn_bwd: dQ launch");
 }
 
-template <int D>
+template <int D, int NWG>
 tg_status launch_mma(const AttnBwdArgs& a, const BwdParams& p0, cudaStream_t st) {
   BwdParams p = p0;
   const int units = p.tiles[p.nseq];
-  constexpr int SMEM_DKDV = MSmem<D>::BYTES_DKDV, SMEM_DQ = MSmem<D>::BYTES_DQ;
-  auto kdkdv = attn_bwd_dkdv_mma<D>;
+  constexpr int SMEM_DKDV = MSmem<D>::bytes_dkdv(NWG), SMEM_DQ = MSmem<D>::BYTES_DQ;
+  static_assert(SMEM_DKDV <= 227 * 1024, "shared memory budget");
+  auto kdkdv = attn_bwd_dkdv_mma<D, NWG>;
   auto kdq = attn_bwd_dq_mma<D>;
-  const int slot = ATTR_BWD + 2 + (D == 128 ? 1 : 0);
+  const int slot = ATTR_BWD + 2 + (D == 128 ? 2 : 0) + (NWG - 1);
   if (attrs_needed(slot)) {
     cudaError_t e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DKDV);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DQ);
@@ -901,7 +967,7 @@ tg_status launch_mma(const AttnBwdArgs& a, const BwdParams& p0, cudaStream_t st)
   p.C = a.Hkv < MAXC ? a.Hkv : MAXC;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(units * p.C));
-  cfg.blockDim = dim3(NTM);
+  cfg.blockDim = dim3(NTM * NWG);
   cfg.dynamicSmemBytes = (size_t)SMEM_DKDV;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -938,7 +1004,12 @@ tg_status launch_attn_bwd(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, c
     p.tiles[i + 1] = p.tiles[i] + (seqs[i].m + tile - 1) / tile;
   }
   if (p.tiles[nseq] == 0) return TG_OK;
-  if (a.dt == TG_BF16) return a.D == 64 ? launch_mma<64>(a, p, st) : launch_mma<128>(a, p, st);
+  if (a.dt == TG_BF16) {
+    // two warp groups share a key tile when its KV group has at least two query heads
+    const bool two = a.Hq / a.Hkv >= 2;
+    if (a.D == 64) return two ? launch_mma<64, 2>(a, p, st) : launch_mma<64, 1>(a, p, st);
+    return two ? launch_mma<128, 2>(a, p, st) : launch_mma<128, 1>(a, p, st);
+  }
   return a.D == 64 ? launch_td<float, 64>(a, p, st) : launch_td<float, 128>(a, p, st);
 }
 

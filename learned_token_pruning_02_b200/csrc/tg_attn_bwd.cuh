@@ -6,8 +6,9 @@
 namespace tg {
 
 // Function-attribute slots of the backward's kernels (after the forward path's slots):
-// CUDA-core (f32) D 64, 128, then tensor-core (bf16) D 64, 128.
-enum { ATTR_BWD = ATTR_SLOTS, ATTR_ALL = ATTR_BWD + 4 };
+// CUDA-core (f32) D 64, 128, then tensor-core (bf16) D 64 and 128, each with one or two warp
+// groups in the dK/dV kernel.
+enum { ATTR_BWD = ATTR_SLOTS, ATTR_ALL = ATTR_BWD + 6 };
 
 // Gradients of the gated attention (normalised form): dQ, dK, dV (f32) and optionally d log g,
 // d score (f32), from the forward's inputs, O and lse and the upstream dO.
