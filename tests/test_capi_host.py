@@ -128,3 +128,42 @@ def test_binding_refuses_cpu_tensors(L):
     H = torch.zeros(4, 64)
     with pytest.raises(ValueError):
         tg.tg_score(H, torch.zeros(64, 64), None, torch.zeros(64), 0.0)
+
+
+def test_argument_errors_of_the_next_entry_points(L):
+    """The projection, the split selection and the attention backward validate before any CUDA
+    call too: each bad argument below returns its status with nothing launched."""
+    V = ctypes.c_void_p
+    fake = V(0x1000)
+    # tg_qkv_rope: f32, d not a multiple of 64, D, (Hq + 2 Hkv) D not a multiple of 256, NaN theta
+    assert L.tg_qkv_rope(0, fake, 8, 128, fake, fake, 16, 8, 128, 1e6, fake, fake, fake, None, None) == 2
+    assert L.tg_qkv_rope(1, fake, 8, 96, fake, fake, 16, 8, 128, 1e6, fake, fake, fake, None, None) == 2
+    assert L.tg_qkv_rope(1, fake, 8, 128, fake, fake, 16, 8, 96, 1e6, fake, fake, fake, None, None) == 2
+    assert L.tg_qkv_rope(1, fake, 8, 128, fake, fake, 1, 1, 64, 1e6, fake, fake, fake, None, None) == 2
+    assert L.tg_qkv_rope(1, fake, 8, 128, fake, fake, 16, 8, 128, float("nan"), fake, fake, fake, None, None) == 1
+    assert L.tg_qkv_rope(1, fake, 8, 128, fake, None, 16, 8, 128, 1e6, fake, fake, fake, None, None) == 1  # no pos
+    assert L.tg_qkv_rope(1, None, 0, 128, None, None, 16, 8, 128, 1e6, None, None, None, None, None) == 0  # M = 0
+    # tg_topk_candidates / tg_topk_merge: negative sizes, oversize blocks, missing outputs
+    assert L.tg_topk_candidates(fake, -1, 4, 0, fake, fake, None, None) == 1
+    assert L.tg_topk_candidates(fake, tg.TG_MAX_CTX + 1, 4, 0, fake, fake, None, None) == 2
+    assert L.tg_topk_candidates(fake, 100, 4, 0, None, fake, None, None) == 1
+    assert L.tg_topk_candidates(None, 100, 0, 0, None, None, None, None) == 0  # k = 0 keeps nothing
+    assert L.tg_topk_merge(fake, fake, -1, 4, 0, 0, fake, None, None) == 1
+    assert L.tg_topk_merge(fake, fake, tg.TG_MAX_CTX + 1, 4, 0, 0, fake, None, None) == 2
+    assert L.tg_topk_merge(fake, fake, 100, 4, 0, 0, None, None, None) == 1
+    # tg_gated_attn_bwd: unnormalised form, D, Hq % Hkv, d score without log g, missing lse
+    cu = (ctypes.c_int32 * 2)(0, 8)
+    args = lambda **kw: [kw.get(n, d) for n, d in (
+        ("dtype", 1), ("Q", fake), ("K", fake), ("V", fake), ("logg", fake), ("gain", None), ("pos", fake),
+        ("cu", cu), ("B", 1), ("Hq", 8), ("Hkv", 4), ("D", 128), ("scale", 0.1), ("flags", 0), ("O", fake),
+        ("lse", fake), ("dO", fake), ("dQ", fake), ("dK", fake), ("dV", fake), ("dlogg", None), ("dscore", None),
+        ("st", None), ("stream", None))]
+    assert L.tg_gated_attn_bwd(*args(flags=tg.TG_ATTN_UNNORMALISED)) == 2
+    assert L.tg_gated_attn_bwd(*args(D=96)) == 2
+    assert L.tg_gated_attn_bwd(*args(Hq=6)) == 2
+    assert L.tg_gated_attn_bwd(*args(logg=None, dscore=fake)) == 1
+    assert L.tg_gated_attn_bwd(*args(lse=None)) == 1
+    assert L.tg_gated_attn_bwd(*args(dK=V(0x1004))) == 2  # misaligned
+    assert L.tg_gated_attn_bwd(*args(scale=float("nan"))) == 1
+    assert L.tg_gated_attn_bwd(*args(dtype=7)) == 1
+    assert L.tg_gated_attn_bwd(*args(cu=(ctypes.c_int32 * 2)(0, 0))) == 0  # no rows: nothing to do
