@@ -369,12 +369,15 @@ __global__ void __launch_bounds__(NT, 2)
 // distinct banks; a transposed B (k along rows of the stored tile) comes from ldmatrix.trans.
 // P and dS are rounded to bf16 for the products that consume them, as the forward does with P.
 //
-//   attn_bwd_dkdv_mma: 64-key tile per CTA (4 warps x 16 keys), clustered over the KV heads
-//     like the CUDA-core kernel. Per 32-query step: S^T = K Q^T and dP^T = V dO^T
+//   attn_bwd_dkdv_mma: 64-key tile per CTA, clustered over the KV heads like the CUDA-core
+//     kernel. One or two warp groups of 4 warps x 16 keys; with two, each takes every other
+//     query head of the KV group. Per 32-query step: S^T = K Q^T and dP^T = V dO^T
 //     (16 x 32 per warp), then P^T and dS^T in registers, then dV += P^T dO and
 //     dK += dS^T Q (16 x D per warp).
 //   attn_bwd_dq_mma: 64-query tile per CTA (4 warps x 16 rows) and head. Per 32-key step:
 //     S = Q K^T, dP = dO V^T, dS in registers, dQ += dS K.
+//   The streamed tiles (and their per-row vectors) are double-buffered with cp.async, so the
+//   next step's copies fly while the current step computes.
 
 constexpr int MT = 64;   // rows of a CTA's own tile (keys in dkdv, queries in dq)
 constexpr int ST = 32;   // rows of the streamed tile (queries in dkdv, keys in dq)
