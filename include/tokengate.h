@@ -79,7 +79,9 @@ const char* tg_status_string(int32_t status);
 /* Description of the most recent failed call on this thread ("" if none). */
 const char* tg_last_error(void);
 
-/* ABI version, (major << 16) | minor. */
+/* ABI version, (major << 16) | minor. 1.0: the gated-prefill path (tg_score, tg_topk_select,
+ * tg_gather, tg_gated_attn_fwd, tg_prefill_above_L and the helpers). 1.1 adds tg_qkv_rope,
+ * tg_topk_candidates, tg_topk_merge and tg_gated_attn_bwd; nothing of 1.0 changed. */
 int32_t tg_version(void);
 
 /* Kept-row offsets (host only, no GPU work). M_b = min(max(k_b, 0), N_b - q_b) + q_b: the

@@ -141,7 +141,7 @@ const char* tg_status_string(int32_t st) {
 
 const char* tg_last_error(void) { return g_err; }
 
-int32_t tg_version(void) { return (1 << 16) | 0; }
+int32_t tg_version(void) { return (1 << 16) | 1; }
 
 tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host) {
   g_err[0] = 0;

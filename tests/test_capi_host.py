@@ -45,6 +45,7 @@ def test_status_strings_and_version(L):
     assert L.tg_status_string(4) == b"TG_ERR_CUDA"
     assert L.tg_status_string(99) == b"TG_ERR_UNKNOWN"
     assert L.tg_version() >> 16 == 1
+    assert L.tg_version() & 0xffff >= 1  # the projection, split selection and backward
 
 
 @pytest.mark.parametrize("seed", range(5))
