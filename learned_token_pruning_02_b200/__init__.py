@@ -122,6 +122,18 @@ def _dtype(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
 
 
+def _want(dtype, **named):
+    """Side tensors (scores, gates, positions, indices, status words, gradients) must have the
+    library's fixed dtype and be contiguous: the C ABI reads them as plain arrays."""
+    for name, t in named.items():
+        if t is None:
+            continue
+        if t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
 def _cuda(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:
@@ -160,6 +172,7 @@ def tg_kept_counts(seqlens, q_len, k) -> list:
 
 def tg_score(H, W1, b1, w2, b2: float, score=None, stream=None):
     """Gate-MLP score of every token: w2 . GELU(W1 h + b1) + b2 (float32 [n_tok])."""
+    _want(torch.float32, b1=b1, score=score)
     _cuda(H, W1, b1, w2, score)
     n_tok, d = H.shape
     assert H.stride(1) == 1 and W1.is_contiguous() and w2.is_contiguous()
@@ -172,6 +185,8 @@ def tg_score(H, W1, b1, w2, b2: float, score=None, stream=None):
 
 def tg_topk_select(score, seqlens, q_len, k, kept_idx=None, cu_kept_dev=None, dev_status=None, stream=None):
     """Top-K context tokens per sequence plus the question tail (int32 kept_idx, cu_kept_dev)."""
+    _want(torch.float32, score=score)
+    _want(torch.int32, kept_idx=kept_idx, cu_kept_dev=cu_kept_dev, dev_status=dev_status)
     _cuda(score, kept_idx, cu_kept_dev, dev_status)
     s = Seqs(seqlens, q_len, k)
     cu = tg_kept_counts(seqlens, q_len, k)
@@ -187,6 +202,7 @@ def tg_topk_select(score, seqlens, q_len, k, kept_idx=None, cu_kept_dev=None, de
 def tg_qkv_rope(H_kept, W_qkv, pos, Hq: int, Hkv: int, D: int, rope_theta: float, Q=None, K=None, V=None,
                 dev_status=None, stream=None):
     """Q, K, V of the kept rows (bf16), Q and K rotated at their original positions: (Q, K, V)."""
+    _want(torch.int32, pos=pos, dev_status=dev_status)
     _cuda(H_kept, W_qkv, pos, Q, K, V, dev_status)
     M, d = H_kept.shape
     dev = H_kept.device
@@ -201,6 +217,8 @@ def tg_qkv_rope(H_kept, W_qkv, pos, Hq: int, Hkv: int, D: int, rope_theta: float
 
 def tg_topk_candidates(score, k: int, base: int = 0, cand_score=None, cand_idx=None, dev_status=None, stream=None):
     """Top-k of one block of a sequence's context as (cand_score, cand_idx = base + position)."""
+    _want(torch.float32, score=score, cand_score=cand_score)
+    _want(torch.int32, cand_idx=cand_idx, dev_status=dev_status)
     _cuda(score, cand_score, cand_idx, dev_status)
     n = score.numel()
     kc = min(int(k), n)
@@ -215,6 +233,8 @@ def tg_topk_candidates(score, k: int, base: int = 0, cand_score=None, cand_idx=N
 
 def tg_topk_merge(cand_score, cand_idx, k: int, q_start: int, q: int, kept_idx=None, dev_status=None, stream=None):
     """Top-k of candidates concatenated in block order, then the question tail q_start..q_start+q-1."""
+    _want(torch.float32, cand_score=cand_score)
+    _want(torch.int32, cand_idx=cand_idx, kept_idx=kept_idx, dev_status=dev_status)
     _cuda(cand_score, cand_idx, kept_idx, dev_status)
     n = cand_score.numel()
     m = min(int(k), n) + int(q)
@@ -228,6 +248,8 @@ def tg_topk_merge(cand_score, cand_idx, k: int, q_start: int, q: int, kept_idx=N
 def tg_gather(H, score, kept_idx, seqlens, q_len, k, flags=0, H_kept=None, pos=None, g=None, logg=None,
               dev_status=None, stream=None):
     """Kept rows of H with their positions and gate values: (H_kept, pos, g, logg)."""
+    _want(torch.float32, score=score, g=g, logg=logg)
+    _want(torch.int32, kept_idx=kept_idx, pos=pos, dev_status=dev_status)
     _cuda(H, score, kept_idx, H_kept, pos, g, logg, dev_status)
     s = Seqs(seqlens, q_len, k)
     m = kept_idx.numel()
@@ -246,6 +268,8 @@ def tg_gather(H, score, kept_idx, seqlens, q_len, k, flags=0, H_kept=None, pos=N
 def tg_gated_attn_fwd(Q, K, V, logg, pos, cu_kept, softmax_scale: float, head_gain=None, flags=0, O=None,
                       lse=None, want_lse=True, dev_status=None, stream=None):
     """Token-gated causal attention over the kept tokens: (O [M, Hq, D], lse [Hq, M] or None)."""
+    _want(torch.float32, logg=logg, head_gain=head_gain, lse=lse)
+    _want(torch.int32, pos=pos, dev_status=dev_status)
     _cuda(Q, K, V, logg, pos, head_gain, O, lse, dev_status)
     M, Hq, D = Q.shape
     Hkv = K.shape[1]
@@ -268,6 +292,8 @@ def tg_gated_attn_bwd(Q, K, V, logg, pos, cu_kept, O, lse, dO, softmax_scale: fl
     """Gradients of the gated attention (normalised form) from the forward's O and lse and the
     upstream dO: (dQ [M, Hq, D], dK [M, Hkv, D], dV [M, Hkv, D], dlogg [M] or None,
     dscore [M] or None), all float32."""
+    _want(torch.float32, logg=logg, lse=lse, head_gain=head_gain, dQ=dQ, dK=dK, dV=dV, dlogg=dlogg, dscore=dscore)
+    _want(torch.int32, pos=pos, dev_status=dev_status)
     _cuda(Q, K, V, logg, pos, O, lse, dO, head_gain, dQ, dK, dV, dlogg, dscore, dev_status)
     M, Hq, D = Q.shape
     Hkv = K.shape[1]
@@ -300,6 +326,8 @@ def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_sca
     outputs (score, kept_idx, cu_kept_dev, H_kept, pos, g, logg, O list, lse list). Pass
     ``out`` (a dict from an earlier call) to reuse its buffers.
     """
+    _want(torch.float32, b1=b1, head_gain=head_gain)
+    _want(torch.int32, dev_status=dev_status)
     _cuda(H, W1, b1, w2, head_gain, dev_status)
     s = Seqs(seqlens, q_len, k)
     cu = tg_kept_counts(seqlens, q_len, k)
@@ -322,6 +350,7 @@ def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_sca
             "O": [torch.empty_like(q) for (q, _, _) in layers],
             "lse": [torch.empty(Hq, m, device=dev, dtype=torch.float32) if want_lse else None for _ in layers],
         }
+    _check_out(out)
     qa = (_VP * max(nl, 1))(*[t[0].data_ptr() for t in layers])
     ka = (_VP * max(nl, 1))(*[t[1].data_ptr() for t in layers])
     va = (_VP * max(nl, 1))(*[t[2].data_ptr() for t in layers])
@@ -335,6 +364,14 @@ def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_sca
     return out
 
 
+def _check_out(out):
+    """The output buffers of the chain have the library's fixed dtypes and are contiguous."""
+    _want(torch.float32, score=out["score"], g=out["g"], logg=out["logg"])
+    _want(torch.int32, kept_idx=out["kept_idx"], cu_kept_dev=out["cu_kept_dev"], pos=out["pos"])
+    for i, t in enumerate(out["lse"]):
+        _want(torch.float32, **{f"lse[{i}]": t})
+
+
 class PreparedChain:
     """The gated path with every C-ABI argument marshalled once, for repeated launches.
 
@@ -345,6 +382,9 @@ class PreparedChain:
 
     def __init__(self, H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_scale, out, head_gain=None, flags=0,
                  dev_status=None, stream=None):
+        _want(torch.float32, b1=b1, head_gain=head_gain)
+        _want(torch.int32, dev_status=dev_status)
+        _check_out(out)
         _cuda(H, W1, b1, w2, head_gain, dev_status)
         self._L = lib()
         self._seqs = Seqs(seqlens, q_len, k)

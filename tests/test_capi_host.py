@@ -168,3 +168,29 @@ def test_argument_errors_of_the_next_entry_points(L):
     assert L.tg_gated_attn_bwd(*args(scale=float("nan"))) == 1
     assert L.tg_gated_attn_bwd(*args(dtype=7)) == 1
     assert L.tg_gated_attn_bwd(*args(cu=(ctypes.c_int32 * 2)(0, 0))) == 0  # no rows: nothing to do
+
+
+def test_binding_refuses_wrong_side_dtypes():
+    """Scores, gates, positions, indices, status words and gradients have fixed dtypes and must
+    be contiguous; the binding rejects anything else before it touches a device."""
+    import torch
+    f64, i64 = torch.float64, torch.int64
+    Q = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    K = V = torch.zeros(4, 1, 64, dtype=torch.bfloat16)
+    pos = torch.arange(4, dtype=torch.int32)
+    with pytest.raises(TypeError, match="logg"):
+        tg.tg_gated_attn_fwd(Q, K, V, torch.zeros(4, dtype=f64), pos, [0, 4], 0.1)
+    with pytest.raises(TypeError, match="pos"):
+        tg.tg_gated_attn_fwd(Q, K, V, None, pos.to(i64), [0, 4], 0.1)
+    with pytest.raises(TypeError, match="score"):
+        tg.tg_topk_select(torch.zeros(10, dtype=f64), (10,), (2,), (3,))
+    with pytest.raises(TypeError, match="kept_idx"):
+        tg.tg_gather(torch.zeros(10, 64, dtype=torch.bfloat16), torch.zeros(10), torch.zeros(5, dtype=i64),
+                     (10,), (2,), (3,))
+    with pytest.raises(TypeError, match="cand_idx"):
+        tg.tg_topk_merge(torch.zeros(8), torch.zeros(8, dtype=i64), 4, 8, 2)
+    with pytest.raises(ValueError, match="lse must be contiguous"):
+        tg.tg_gated_attn_bwd(Q, K, V, None, pos, [0, 4], Q, torch.zeros(4, 2).t(), Q, 0.1)
+    with pytest.raises(TypeError, match="dQ"):
+        tg.tg_gated_attn_bwd(Q, K, V, None, pos, [0, 4], Q, torch.zeros(2, 4), Q, 0.1,
+                             dQ=torch.zeros(4, 2, 64, dtype=torch.bfloat16))
