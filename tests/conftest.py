@@ -12,11 +12,6 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (sm_100a) and the built library")
 
 
-def pytest_collection_modifyitems(config, items):
-    # keep collection order stable; the no-allocation test file sorts last by name
-    pass
-
-
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
