@@ -196,6 +196,27 @@ def test_gather_bitexact(name, flags):
     assert st.item() == 0
 
 
+def test_gather_ignores_dropped_rows():
+    """Layers above L see only the kept tokens: with the scores held fixed, the rows the
+    selector dropped can hold anything without changing the gathered rows, positions or gate
+    values, bit for bit."""
+    wl = ti.WORKLOADS["qwen3_8k"]
+    H = ti.hidden_states(wl)
+    s = ti.stage_scores(wl)
+    kept, cu = orc.topk_select(s, wl.seqlens, wl.q_len, wl.k)
+    H2 = H.copy()
+    dropped = np.setdiff1d(np.arange(H.shape[0]), kept)
+    assert dropped.size > 0
+    H2[dropped] = ti.f32_to_bf16_bits(np.array([1000.0], dtype=np.float32))[0]
+    sd = torch.from_numpy(s).to(DEV)
+    kd = torch.from_numpy(kept.astype(np.int32)).to(DEV)
+    a = tg.tg_gather(to_dev(H, wl.dtype), sd, kd, wl.seqlens, wl.q_len, wl.k)
+    b = tg.tg_gather(to_dev(H2, wl.dtype), sd, kd, wl.seqlens, wl.q_len, wl.k)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert np.array_equal(bits(x), bits(y))
+
+
 def test_gather_strided_and_bad_index_flag():
     wl = ti.scaled(ti.WORKLOADS["qwen3_8k"], seqlens=(300, 200), q_len=(10, 20), k=(50, 40), d=512)
     H = ti.hidden_states(wl)
