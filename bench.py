@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-full-ref", action="store_true")
+    ap.add_argument("--no-other", action="store_true", help="skip the other configurations' throughput")
     ap.add_argument("--no-bw", action="store_true", help="skip the byte-heavy select/gather instances")
     ap.add_argument("--bw-only", action="store_true", help="run only the byte-heavy select/gather instances")
     ap.add_argument("--bw-reps", type=int, default=20)
@@ -128,36 +129,30 @@ class ClockSampler:
 # --------------------------------------------------------------------------- oracle timing
 
 
-def oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_score_tok, n_attn_rows):
-    """Times the CPU oracle on a bounded sample of one step and scales it to the whole step.
+def oracle_step(wl, H, W1, b1, w2, b2, layers):
+    """One whole step of the CPU oracle on the workload, timed (wall clock, host cores).
 
-    Score: the first n_score_tok tokens (time x N / n_score_tok). Select and gather: full.
-    Attention: n_attn_rows query rows spread over the sequence, all heads (time x M / rows).
-    Returns (estimated seconds per step, description)."""
+    The step starts from the stored input bytes (bf16 bits widened exactly to float64, as the
+    oracle consumes them): gate-MLP scores of every token, top-K with the question tail on those
+    scores, gather, and gated attention over every kept query row, every head and every above-L
+    layer. Returns (seconds, description)."""
     import numpy as np
 
     import tg_inputs as ti
     from oracle import tg_oracle as orc
 
-    W64, w64 = ti.widen(W1, wl.dtype), ti.widen(w2, wl.dtype)
     t0 = time.perf_counter()
-    orc.gate_scores(ti.widen(H[:n_score_tok], wl.dtype), W64, b1, w64, b2)
-    t_score = (time.perf_counter() - t0) * wl.n_tok / n_score_tok
-    t0 = time.perf_counter()
-    kept, cu = orc.topk_select(s_full, wl.seqlens, wl.q_len, wl.k)
-    t_sel = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    _, pos, _, lg = orc.gather(H, s_full, kept, wl.seqlens, wl.q_len, cu)
-    t_gat = time.perf_counter() - t0
-    Q, K, V = (ti.widen(x, wl.dtype) for x in layer)
-    m = int(cu[-1])
-    rows = np.linspace(0, m - 1, n_attn_rows).astype(np.int64)
-    t0 = time.perf_counter()
-    orc.gated_attention(Q, K, V, lg, pos, cu, wl.Hq, wl.Hkv, 1.0 / math.sqrt(wl.D), rows=rows)
-    t_att = (time.perf_counter() - t0) * m / n_attn_rows
-    desc = (f"score on {n_score_tok} of {wl.n_tok} tokens (scaled), full select and gather, attention on "
-            f"{n_attn_rows} of {m} query rows x {wl.Hq} heads (scaled)")
-    return t_score + t_sel + t_gat + t_att, desc
+    s = orc.gate_scores(ti.widen(H, wl.dtype), ti.widen(W1, wl.dtype), b1, ti.widen(w2, wl.dtype), b2)
+    kept, cu = orc.topk_select(s, wl.seqlens, wl.q_len, wl.k)
+    _, pos, _, lg = orc.gather(H, s, kept, wl.seqlens, wl.q_len, cu)
+    for (Q, K, V) in layers:
+        orc.gated_attention(ti.widen(Q, wl.dtype), ti.widen(K, wl.dtype), ti.widen(V, wl.dtype), lg, pos, cu,
+                            wl.Hq, wl.Hkv, 1.0 / math.sqrt(wl.D))
+    dt = time.perf_counter() - t0
+    m = int(np.asarray(cu)[-1])
+    desc = (f"full step: scores of all {wl.n_tok} tokens, select, gather, attention over all {m} kept rows x "
+            f"{wl.Hq} heads x {len(layers)} layer(s), float64 NumPy from the stored input bytes")
+    return dt, desc
 
 
 def blas_threads():
@@ -373,8 +368,9 @@ def split_select_times(tg, torch, dev, reps):
 
 
 def run_reference(args, wl):
-    import numpy as np
-
+    """The oracle arm: whole oracle steps on the host cores (rank 0 only). Warm-up and timed
+    steps are full steps; if the requested count would run past about three minutes, fewer steps
+    are timed and the line says how many (the per-step time is measured, never extrapolated)."""
     import tg_inputs as ti
 
     rank = int(os.environ.get("RANK", "0"))
@@ -382,36 +378,30 @@ def run_reference(args, wl):
         return 0
     H = ti.hidden_states(wl)
     W1, b1, w2, b2 = ti.gate_weights(wl)
-    s_full = ti.stage_scores(wl) if wl.score_mode != "mlp" else np.random.default_rng(0).standard_normal(
-        wl.n_tok).astype(np.float32)
-    layer = ti.qkv(wl, 0)
-    # per-step sample sized so that warmup + steps end within about two minutes
-    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
-    n_tok, n_rows = 64, 4
-    est, _ = oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_tok, n_rows)
-    t0 = time.perf_counter()
-    oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_tok, n_rows)
-    wall = time.perf_counter() - t0
-    grow = max(1.0, min(64.0, budget / max(wall, 1e-3)))
-    n_tok, n_rows = int(min(wl.n_tok, n_tok * grow)), int(min(wl.m_tot, max(4, n_rows * grow)))
-    for _ in range(args.warmup):
-        oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_tok, n_rows)
-    ests = []
-    for _ in range(args.steps):
-        e, desc = oracle_sample(wl, H, W1, b1, w2, b2, s_full, layer, n_tok, n_rows)
-        ests.append(e)
-    t_step = sum(ests) / len(ests)
+    layers = [ti.qkv(wl, l) for l in range(wl.n_layers)]
+    t_first, desc = oracle_step(wl, H, W1, b1, w2, b2, layers)  # the first warm-up step sizes the run
+    budget = 180.0
+    fit = max(1, int((budget - t_first) / max(t_first, 1e-3)))
+    warm = min(max(args.warmup - 1, 0), max(0, fit - args.steps))
+    steps = max(1, min(args.steps, fit - warm))
+    for _ in range(warm):
+        oracle_step(wl, H, W1, b1, w2, b2, layers)
+    ts = [oracle_step(wl, H, W1, b1, w2, b2, layers)[0] for _ in range(steps)]
+    t_step = sum(ts) / len(ts)
     value = wl.n_tok / t_step
     cores = blas_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "steps": steps, "warmup": 1 + warm, "ms_per_step": t_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
+    if steps != args.steps or 1 + warm != args.warmup:
+        line["note"] = (f"{args.steps} steps after {args.warmup} warm-up steps were asked for; {steps} full steps "
+                        f"after {1 + warm} warm-up step(s) fit the time budget and were timed")
     print(json.dumps(line), flush=True)
     return 0
 
@@ -423,8 +413,151 @@ def workload_config(wl):
                     f"head_dim {wl.D}, {wl.n_layers} above-L layer(s), {wl.dtype}",
         "global_batch": wl.B, "seq_len": max(wl.seqlens), "kept_rows": wl.m_tot,
         "parallelism": "replicas (one independent workload per GPU)",
-        "l2": "flushed between timed steps (512 MiB memset)",
+        "l2": "flushed between timed steps (512 MiB memset, then a 256 MiB read sweep that evicts its dirty lines)",
     }
+
+
+class L2Flush:
+    """Leaves L2 holding only clean lines of an unrelated buffer: a 512 MiB memset, then a read of
+    256 MiB more (a reduction), so the next kernel's reads neither hit in L2 nor wait behind the
+    write-back of dirty lines."""
+
+    def __init__(self, torch, dev):
+        self.w = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+        self.r = torch.zeros(64 << 20, device=dev, dtype=torch.float32)
+        self.acc = torch.zeros((), device=dev, dtype=torch.float32)
+
+    def __call__(self):
+        self.w.zero_()
+        self.acc.add_(self.r.sum())
+
+
+class ChainBench:
+    """Device buffers and the prepared C-ABI arguments of one workload's whole chain."""
+
+    def __init__(self, tg, torch, np, dev, wl, stream):
+        import tg_inputs as ti
+
+        def bf(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+        self.wl = wl
+        self.Hn = ti.hidden_states(wl)
+        self.W1n, self.b1n, self.w2n, self.b2 = ti.gate_weights(wl)
+        self.lay = [ti.qkv(wl, l) for l in range(wl.n_layers)]
+        self.H_host = bf(self.Hn).pin_memory()
+        self.qkv_host = [tuple(bf(x).pin_memory() for x in L) for L in self.lay]
+        self.H = self.H_host.to(dev)
+        self.W1, self.b1, self.w2 = bf(self.W1n).to(dev), torch.from_numpy(self.b1n).to(dev), bf(self.w2n).to(dev)
+        self.layers = [tuple(x.to(dev) for x in L) for L in self.qkv_host]
+        self.cu = tg.tg_kept_counts(wl.seqlens, wl.q_len, wl.k)
+        M = self.M = self.cu[-1]
+        self.scale = 1.0 / math.sqrt(wl.D)
+        f32, i32 = torch.float32, torch.int32
+        self.out = {"score": torch.empty(wl.n_tok, device=dev, dtype=f32),
+                    "kept_idx": torch.empty(M, device=dev, dtype=i32),
+                    "cu_kept_dev": torch.empty(wl.B + 1, device=dev, dtype=i32),
+                    "H_kept": torch.empty(M, wl.d, device=dev, dtype=torch.bfloat16),
+                    "pos": torch.empty(M, device=dev, dtype=i32), "g": torch.empty(M, device=dev, dtype=f32),
+                    "logg": torch.empty(M, device=dev, dtype=f32),
+                    "O": [torch.empty_like(L[0]) for L in self.layers], "lse": [None] * len(self.layers)}
+        self.status = torch.zeros(1, device=dev, dtype=i32)
+        self.stream = stream
+        self.chain = tg.PreparedChain(self.H, self.W1, self.b1, self.w2, self.b2, wl.seqlens, wl.q_len, wl.k,
+                                      self.layers, self.scale, self.out, dev_status=self.status, stream=stream)
+
+    def stages(self, ev=None):
+        """The four stage entry points one after another, with an event between kernels."""
+        c, st = self.chain, self.stream
+        if ev:
+            ev[0].record(st)
+        c.score()
+        if ev:
+            ev[1].record(st)
+        c.select()
+        if ev:
+            ev[2].record(st)
+        c.gather()
+        if ev:
+            ev[3].record(st)
+        for li in range(len(self.layers)):
+            c.attention(li)
+        if ev:
+            ev[4].record(st)
+
+    def measure(self, torch, np, steps, warmup, flush, barrier):
+        """Region A: whole steps through tg_prefill_above_L, events at step boundaries only (the
+        metric). Region B: the stage entry points with events between kernels (per-kernel times)."""
+        for _ in range(warmup):
+            flush()
+            self.stages()
+            flush()
+            self.chain.prefill()
+        torch.cuda.synchronize()
+        st = self.stream
+        ev_a = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush()  # outside the timed events
+            torch.cuda._sleep(200_000)  # keeps the host's launches ahead of the GPU (no idle gaps timed)
+            ev_a[i][0].record(st)
+            self.chain.prefill()
+            ev_a[i][1].record(st)
+        torch.cuda.synchronize()
+        barrier()
+        step_ms = np.array([e[0].elapsed_time(e[1]) for e in ev_a])
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush()
+            torch.cuda._sleep(200_000)
+            self.stages(evs[i])
+        torch.cuda.synchronize()
+        barrier()
+        st_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)])
+        return step_ms, st_ms.mean(axis=0)
+
+    def per_kernel(self, np, stage_ms, pk):
+        wl, cu, M = self.wl, self.cu, self.M
+        flops_attn = 4.0 * wl.Hq * wl.D * sum(m * (m + 1) / 2 for m in np.diff(cu))
+        bytes_score = wl.n_tok * wl.d * 2 + wl.n_tok * 4 + wl.dg * wl.d * 2
+        bytes_gather = M * wl.d * 2 * 2 + M * 4 * 4
+        bytes_select = (wl.n_tok - sum(wl.q_len)) * 4 + M * 4
+        out = {}
+        for i, nm in enumerate(("score", "select", "gather", "gated_attn")):
+            t_s = stage_ms[i] / 1e3 / (wl.n_layers if nm == "gated_attn" else 1)
+            if nm == "gated_attn":
+                e = {"bound": "tensor", "achieved": flops_attn / t_s / 1e12, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "algorithmic": flops_attn}
+            else:
+                byts = {"score": bytes_score, "select": bytes_select, "gather": bytes_gather}[nm]
+                e = {"bound": "hbm", "achieved": byts / t_s / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "algorithmic": byts}
+            e["frac"] = e["achieved"] / e["peak"]
+            e["us"] = t_s * 1e6
+            out[nm] = e
+        return out
+
+
+def other_workload(tg, torch, np, dev, name, steps, warmup, flush, pk):
+    """Throughput of another configuration through the same entry point (rank 0 only)."""
+    import tg_inputs as ti
+
+    wl = ti.WORKLOADS[name]
+    cb = ChainBench(tg, torch, np, dev, wl, torch.cuda.current_stream())
+    step_ms, stage_ms = cb.measure(torch, np, steps, warmup, flush, lambda: None)
+    ms = float(step_ms.mean())
+    kern = cb.per_kernel(np, stage_ms, pk)
+    res = {"config": workload_config(wl)["workload"], "steps": steps, "warmup": warmup, "ms_per_step": ms,
+           "value": wl.n_tok / (ms / 1e3), "unit": "tokens/s",
+           "stages_us": {n: float(x * 1e3) for n, x in zip(("score", "select", "gather", "gated_attn"), stage_ms)},
+           "kernels": {k: {kk: v[kk] for kk in ("achieved", "unit", "frac", "us")} for k, v in kern.items()},
+           "device_status": int(cb.status.item())}
+    del cb
+    torch.cuda.empty_cache()
+    return res
 
 
 def main():
@@ -465,127 +598,30 @@ def main():
             dist.destroy_process_group()
         return 0
 
-    def bf(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
-
     # ---------------- inputs (seeded, identical on every rank: weak-scaling replicas)
-    Hn = ti.hidden_states(wl)
-    W1n, b1n, w2n, b2 = ti.gate_weights(wl)
-    lay = [ti.qkv(wl, l) for l in range(wl.n_layers)]
-    H_host = bf(Hn).pin_memory()
-    qkv_host = [tuple(bf(x).pin_memory() for x in L) for L in lay]
-    H = H_host.to(dev)
-    W1, b1, w2 = bf(W1n).to(dev), torch.from_numpy(b1n).to(dev), bf(w2n).to(dev)
-    layers = [tuple(x.to(dev) for x in L) for L in qkv_host]
-    cu = tg.tg_kept_counts(wl.seqlens, wl.q_len, wl.k)
-    M = cu[-1]
-    scale = 1.0 / math.sqrt(wl.D)
-    score = torch.empty(wl.n_tok, device=dev, dtype=torch.float32)
-    kept = torch.empty(M, device=dev, dtype=torch.int32)
-    cu_dev = torch.empty(wl.B + 1, device=dev, dtype=torch.int32)
-    Hk = torch.empty(M, wl.d, device=dev, dtype=torch.bfloat16)
-    pos = torch.empty(M, device=dev, dtype=torch.int32)
-    g = torch.empty(M, device=dev, dtype=torch.float32)
-    logg = torch.empty(M, device=dev, dtype=torch.float32)
-    Os = [torch.empty_like(L[0]) for L in layers]
-    status = torch.zeros(1, device=dev, dtype=torch.int32)
-    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream()
-
-    out = {"score": score, "kept_idx": kept, "cu_kept_dev": cu_dev, "H_kept": Hk, "pos": pos, "g": g,
-           "logg": logg, "O": Os, "lse": [None] * len(layers)}
-    chain = tg.PreparedChain(H, W1, b1, w2, b2, wl.seqlens, wl.q_len, wl.k, layers, scale, out, dev_status=status,
-                             stream=stream)
-
-    def step(ev=None):
-        # the four stage entry points one after another, with events between them (inside
-        # tg_prefill_above_L the bf16 attention derives log g from score and kept itself and the
-        # gather runs last; the kernels are the same)
-        if ev:
-            ev[0].record(stream)
-        chain.score()
-        if ev:
-            ev[1].record(stream)
-        chain.select()
-        if ev:
-            ev[2].record(stream)
-        chain.gather()
-        if ev:
-            ev[3].record(stream)
-        for li in range(len(layers)):
-            chain.attention(li)
-        if ev:
-            ev[4].record(stream)
-
+    cb = ChainBench(tg, torch, np, dev, wl, stream)
+    flush = L2Flush(torch, dev)
+    H, W1, b1, w2, b2, layers, out = cb.H, cb.W1, cb.b1, cb.w2, cb.b2, cb.layers, cb.out
+    M, cu, scale, status = cb.M, cb.cu, cb.scale, cb.status
     launches_per_step = 4 + (wl.n_layers - 1)  # score, select, gather, attention per layer
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-        flush.zero_()
-        chain.prefill()
-    torch.cuda.synchronize()
-
-    # Timed region A (the metric): whole steps through the path's single C-ABI entry
-    # (tg_prefill_above_L), events only at step boundaries, so the kernels of a step chain with
-    # programmatic dependent launch as they do for a user.
-    ev_a = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     clocks = ClockSampler(local).start()
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()  # L2 flush, outside the timed events
-        torch.cuda._sleep(200_000)  # keeps the host's launches ahead of the GPU (no idle gaps timed)
-        ev_a[i][0].record(stream)
-        chain.prefill()
-        ev_a[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    step_ms = np.array([e[0].elapsed_time(e[1]) for e in ev_a])
+    step_ms, stage_ms = cb.measure(torch, np, args.steps, args.warmup, flush, barrier)
+    clk = clocks.stop()
     t_total = replicas.max_over_ranks(float(step_ms.sum()), device=dev)
     ms_per_step = t_total / args.steps
     value = wl.n_tok * world * args.steps / (t_total / 1e3)
-    # Timed region B (the per-kernel durations behind the roofline): the same steps with an
-    # event between kernels (which also serialises them, so their sum exceeds region A's step).
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        torch.cuda._sleep(200_000)
-        step(evs[i])
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    st_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
-    stage_ms = st_ms.mean(axis=0)
     dev_status = int(status.item())
 
     # ---------------- roofline of the dominant kernel
     pk, pk_src = peaks()
-    flops_attn = 4.0 * wl.Hq * wl.D * sum(m * (m + 1) / 2 for m in np.diff(cu)) * wl.n_layers
-    attn_s = stage_ms[3] / 1e3 / wl.n_layers
-    attn_tflops = flops_attn / wl.n_layers / attn_s / 1e12
-    bytes_score = wl.n_tok * wl.d * 2 + wl.n_tok * 4 + wl.dg * wl.d * 2
-    score_gbs = bytes_score / (stage_ms[0] / 1e3) / 1e9
-    bytes_gather = M * wl.d * 2 * 2 + M * 4 * 4
-    bytes_select = (wl.n_tok - sum(wl.q_len)) * 4 + M * 4
+    per_kernel = cb.per_kernel(np, stage_ms, pk)
     names = ["score", "select", "gather", "gated_attn"]
-    per_kernel = {}
-    for i, nm in enumerate(names):
-        t_s = stage_ms[i] / 1e3
-        if nm == "gated_attn":
-            ach = attn_tflops
-            e = {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                 "algorithmic": flops_attn / wl.n_layers}
-        else:
-            byts = [bytes_score, bytes_select, bytes_gather][i]
-            ach = byts / t_s / 1e9
-            e = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s", "algorithmic": byts}
-        e["frac"] = e["achieved"] / e["peak"]
-        e["us"] = stage_ms[i] * 1e3 / (wl.n_layers if nm == "gated_attn" else 1)
-        e["traffic"] = traffic_from_profile(nm, kernel_hash(nm))
-        per_kernel[nm] = e
+    for nm in names:
+        per_kernel[nm]["traffic"] = traffic_from_profile(nm, kernel_hash(nm))
+    attn_tflops = per_kernel["gated_attn"]["achieved"]
+    score_gbs = per_kernel["score"]["achieved"]
     dominant = names[int(np.argmax(stage_ms))]
     roof = {"kernel": dominant}
     roof.update({k: per_kernel[dominant][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")})
@@ -594,11 +630,14 @@ def main():
     # ---------------- end to end through the public API, host buffers in and out
     e2e = None
     if args.e2e_steps > 0:
+        Os = out["O"]
+        kept = out["kept_idx"]
         O_host = [torch.empty(L[0].shape, dtype=torch.bfloat16).pin_memory() for L in layers]
         kept_host = torch.empty(M, dtype=torch.int32).pin_memory()
+
         def e2e_step():
-            H.copy_(H_host, non_blocking=True)
-            for (q, k, v), (qh, kh, vh) in zip(layers, qkv_host):
+            H.copy_(cb.H_host, non_blocking=True)
+            for (q, k, v), (qh, kh, vh) in zip(layers, cb.qkv_host):
                 q.copy_(qh, non_blocking=True)
                 k.copy_(kh, non_blocking=True)
                 v.copy_(vh, non_blocking=True)
@@ -638,8 +677,7 @@ def main():
         p = torch.arange(n, device=dev, dtype=torch.int32)
         o = torch.empty_like(q)
         reps = 3
-        for _ in range(1):
-            tg.tg_gated_attn_fwd(q, k, v, None, p, [0, n], scale, O=o, want_lse=False)
+        tg.tg_gated_attn_fwd(q, k, v, None, p, [0, n], scale, O=o, want_lse=False)
         torch.cuda.synchronize()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
@@ -668,12 +706,12 @@ def main():
                 g_chain.prefill()
         torch.cuda.synchronize()
         for _ in range(args.warmup):
-            flush.zero_()
+            flush()
             cg.replay()
         torch.cuda.synchronize()
         ev_g = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             torch.cuda._sleep(200_000)
             ev_g[i][0].record(stream)
             cg.replay()
@@ -700,17 +738,25 @@ def main():
         bw = bandwidth_instances(tg, torch, dev, pk["hbm_gbs"], args.bw_reps)
 
     split_t = split_select_times(tg, torch, dev, 20) if not args.no_bw else None
-    qkv_t = qkv_rope_time(tg, torch, dev, Hk, pos, wl.Hq, wl.Hkv, wl.D, pk["bf16_tflops"], 20) if not args.no_bw else None
-    bwd_t = (attn_bwd_time(tg, torch, dev, *layers[0], logg, pos, list(cu), scale, pk["bf16_tflops"], 5)
+    qkv_t = (qkv_rope_time(tg, torch, dev, out["H_kept"], out["pos"], wl.Hq, wl.Hkv, wl.D, pk["bf16_tflops"], 20)
+             if not args.no_bw else None)
+    bwd_t = (attn_bwd_time(tg, torch, dev, *layers[0], out["logg"], out["pos"], list(cu), scale, pk["bf16_tflops"], 5)
              if not args.no_bw else None)
 
-    # ---------------- CPU oracle baseline (rank 0, N = 1 only)
+    # ---------------- the other configurations, through the same entry point (rank 0)
+    others = None
+    if rank == 0 and not args.no_other:
+        others = {}
+        for name in ("qwen3_8k", "qwen3_128k", "ragged4"):
+            if name != wl.name:
+                others[name] = other_workload(tg, torch, np, dev, name, 20, 3, flush, pk)
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1 only): one whole oracle step
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s_full = score.cpu().numpy()
-        est, desc = oracle_sample(wl, Hn, W1n, b1n, w2n, b2, s_full, lay[0], 8192, 256)
-        cpu = {"value": wl.n_tok / est, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": desc, "host_cpus": os.cpu_count()}
+        t_cpu, desc = oracle_step(wl, cb.Hn, cb.W1n, cb.b1n, cb.w2n, cb.b2, cb.lay)
+        cpu = {"value": wl.n_tok / t_cpu, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc, "seconds": t_cpu, "host_cpus": os.cpu_count()}
 
     if rank == 0:
         line = {
@@ -731,6 +777,7 @@ def main():
             "stages_sum_us": float(stage_ms.sum() * 1e3),
             "clocks": clk,
             "full_attention_reference": full_ref,
+            "other_workloads": others,
             "bandwidth_instances": bw,
             "graph_replay": graph,
             "split_select": split_t,

@@ -81,8 +81,18 @@ const char* tg_last_error(void);
 
 /* ABI version, (major << 16) | minor. 1.0: the gated-prefill path (tg_score, tg_topk_select,
  * tg_gather, tg_gated_attn_fwd, tg_prefill_above_L and the helpers). 1.1 adds tg_qkv_rope,
- * tg_topk_candidates, tg_topk_merge and tg_gated_attn_bwd; nothing of 1.0 changed. */
+ * tg_topk_candidates, tg_topk_merge and tg_gated_attn_bwd. 1.2 gives tg_score a device
+ * status word (its last argument before the stream) and adds tg_set_test_wait_probe. */
 int32_t tg_version(void);
+
+/* Test hook for the bounded waits, off by default (limit_ns = 0). With limit_ns > 0, every
+ * tensor-core kernel this calling thread launches afterwards (tg_score, tg_gated_attn_fwd,
+ * tg_qkv_rope and the chain's kernels, bf16) first waits, with that limit, on a barrier that
+ * nothing signals, before it issues any copy or product. The wait runs out, the kernel ORs
+ * TG_DEV_TIMEOUT into its status word, does none of its work (its outputs are left as they
+ * were) and returns; the context stays usable. Only for tests of the timeout path; set 0 to
+ * restore normal operation. limit_ns < 0 -> TG_ERR_INVALID_ARG. */
+tg_status tg_set_test_wait_probe(int64_t limit_ns);
 
 /* Kept-row offsets (host only, no GPU work). M_b = min(max(k_b, 0), N_b - q_b) + q_b: the
  * K highest-scoring context tokens plus the whole question tail (aitualizate.com TokenGate
@@ -99,12 +109,14 @@ tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host);
  *   w2     device act [dg]
  *   b2     scalar
  *   score  device f32 [n_tok] (written)
+ *   dev_status device int32 [1] or NULL: a wait of the bf16 kernel that gave up sets
+ *          TG_DEV_TIMEOUT (the scores of the tiles it did not finish are then unwritten)
  * Supported: dg in {64, 128, 256}; d % 64 == 0; ldh * sizeof(act) % 16 == 0; 16-byte
  * aligned H and W1. bf16 runs on the tensor cores with fp32 accumulation; f32 runs on the
  * CUDA cores in fp32. */
 tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, int32_t d,
                    const void* W1, const float* b1, const void* w2, float b2, int32_t dg,
-                   float* score, void* stream);
+                   float* score, int32_t* dev_status, void* stream);
 
 /* Top-K over each sequence's context with the question tail always kept (aitualizate.com
  * TokenGate article, phase 2; thelatestinai.com TokenGate page, Figure 1(a)-(b)).
@@ -116,6 +128,9 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
  *   kept_idx    device int32 [sum M_b] (written): packed row indices into H / score
  *   cu_kept_dev device int32 [B+1] (written) or NULL
  *   dev_status  device int32 [1] or NULL
+ * No workspace is needed: per-sequence descriptors travel as kernel parameters and each
+ * sequence's histogram lives in the shared memory of its thread-block cluster (so
+ * TG_ERR_WORKSPACE is never returned).
  * Supported: N_b - q_b <= TG_MAX_CTX. */
 tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
                          int32_t* cu_kept_dev, int32_t* dev_status, void* stream);

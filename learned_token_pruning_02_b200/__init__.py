@@ -32,6 +32,7 @@ EXPORTS = (
     "tg_topk_candidates",
     "tg_topk_merge",
     "tg_gated_attn_bwd",
+    "tg_set_test_wait_probe",
 )
 
 
@@ -77,7 +78,9 @@ def lib() -> ctypes.CDLL:
     L.tg_kept_counts.restype = _I32
     L.tg_kept_counts.argtypes = [_SEQP, ctypes.POINTER(_I32)]
     L.tg_score.restype = _I32
-    L.tg_score.argtypes = [_I32, _VP, _I64, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP]
+    L.tg_score.argtypes = [_I32, _VP, _I64, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP, _VP]
+    L.tg_set_test_wait_probe.restype = _I32
+    L.tg_set_test_wait_probe.argtypes = [_I64]
     L.tg_topk_select.restype = _I32
     L.tg_topk_select.argtypes = [_VP, _SEQP, _VP, _VP, _VP, _VP]
     L.tg_qkv_rope.restype = _I32
@@ -134,6 +137,22 @@ def _want(dtype, **named):
             raise ValueError(f"{name} must be contiguous")
 
 
+def _contig(**named):
+    for name, t in named.items():
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def _shape(name, t, want):
+    if tuple(t.shape) != tuple(want):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(want)}")
+
+
+def _len_at_least(name, t, n):
+    if t is not None and t.numel() < n:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs at least {n}")
+
+
 def _cuda(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:
@@ -170,17 +189,25 @@ def tg_kept_counts(seqlens, q_len, k) -> list:
     return list(out)
 
 
-def tg_score(H, W1, b1, w2, b2: float, score=None, stream=None):
+def tg_score(H, W1, b1, w2, b2: float, score=None, dev_status=None, stream=None):
     """Gate-MLP score of every token: w2 . GELU(W1 h + b1) + b2 (float32 [n_tok])."""
     _want(torch.float32, b1=b1, score=score)
-    _cuda(H, W1, b1, w2, score)
+    _want(torch.int32, dev_status=dev_status)
+    _cuda(H, W1, b1, w2, score, dev_status)
     n_tok, d = H.shape
     assert H.stride(1) == 1 and W1.is_contiguous() and w2.is_contiguous()
     if score is None:
         score = torch.empty(n_tok, device=H.device, dtype=torch.float32)
     _check("tg_score", lib().tg_score(_dtype(H), _ptr(H), H.stride(0), n_tok, d, _ptr(W1), _ptr(b1), _ptr(w2),
-                                      float(b2), W1.shape[0], _ptr(score), _stream(stream)))
+                                      float(b2), W1.shape[0], _ptr(score), _ptr(dev_status), _stream(stream)))
     return score
+
+
+def tg_set_test_wait_probe(limit_ns: int):
+    """Test hook (off by default): with limit_ns > 0 every tensor-core kernel launched afterwards
+    by this thread waits that long on a barrier nothing signals, records TG_DEV_TIMEOUT and skips
+    its work. 0 restores normal operation."""
+    _check("tg_set_test_wait_probe", lib().tg_set_test_wait_probe(int(limit_ns)))
 
 
 def tg_topk_select(score, seqlens, q_len, k, kept_idx=None, cu_kept_dev=None, dev_status=None, stream=None):
@@ -203,9 +230,18 @@ def tg_qkv_rope(H_kept, W_qkv, pos, Hq: int, Hkv: int, D: int, rope_theta: float
                 dev_status=None, stream=None):
     """Q, K, V of the kept rows (bf16), Q and K rotated at their original positions: (Q, K, V)."""
     _want(torch.int32, pos=pos, dev_status=dev_status)
-    _cuda(H_kept, W_qkv, pos, Q, K, V, dev_status)
     M, d = H_kept.shape
+    _contig(H_kept=H_kept, W_qkv=W_qkv)
+    _shape("W_qkv", W_qkv, ((Hq + 2 * Hkv) * D, d))
+    if rope_theta > 0:
+        if pos is None or pos.numel() < M:
+            raise ValueError(f"pos must hold at least M = {M} positions when rope_theta > 0")
     dev = H_kept.device
+    for name, t, h in (("Q", Q, Hq), ("K", K, Hkv), ("V", V, Hkv)):
+        if t is not None:
+            _shape(name, t, (M, h, D))
+            _contig(**{name: t})
+    _cuda(H_kept, W_qkv, pos, Q, K, V, dev_status)
     Q = torch.empty(M, Hq, D, device=dev, dtype=torch.bfloat16) if Q is None else Q
     K = torch.empty(M, Hkv, D, device=dev, dtype=torch.bfloat16) if K is None else K
     V = torch.empty(M, Hkv, D, device=dev, dtype=torch.bfloat16) if V is None else V
@@ -294,13 +330,32 @@ def tg_gated_attn_bwd(Q, K, V, logg, pos, cu_kept, O, lse, dO, softmax_scale: fl
     dscore [M] or None), all float32."""
     _want(torch.float32, logg=logg, lse=lse, head_gain=head_gain, dQ=dQ, dK=dK, dV=dV, dlogg=dlogg, dscore=dscore)
     _want(torch.int32, pos=pos, dev_status=dev_status)
-    _cuda(Q, K, V, logg, pos, O, lse, dO, head_gain, dQ, dK, dV, dlogg, dscore, dev_status)
     M, Hq, D = Q.shape
     Hkv = K.shape[1]
-    for t in (Q, K, V, O, dO):
-        assert t.is_contiguous() and t.dtype == Q.dtype
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O), ("dO", dO)):
+        _contig(**{name: t})
+        if t.dtype != Q.dtype:
+            raise TypeError(f"{name} must have Q's dtype {Q.dtype}")
     cu = [int(x) for x in cu_kept]
     B = len(cu) - 1
+    if B >= 0 and cu and cu[-1] != M:
+        raise ValueError(f"cu_kept[-1] = {cu[-1]} must equal the row count of Q ({M})")
+    _shape("K", K, (M, Hkv, D))
+    _shape("V", V, (M, Hkv, D))
+    _shape("O", O, (M, Hq, D))
+    _shape("dO", dO, (M, Hq, D))
+    if lse is not None:
+        _shape("lse", lse, (Hq, M))
+    _len_at_least("pos", pos, M)
+    _len_at_least("logg", logg, M)
+    _len_at_least("head_gain", head_gain, Hq)
+    for name, t, h in (("dQ", dQ, Hq), ("dK", dK, Hkv), ("dV", dV, Hkv)):
+        if t is not None:
+            _shape(name, t, (M, h, D))
+    for name, t in (("dlogg", dlogg), ("dscore", dscore)):
+        if t is not None:
+            _shape(name, t, (M,))
+    _cuda(Q, K, V, logg, pos, O, lse, dO, head_gain, dQ, dK, dV, dlogg, dscore, dev_status)
     cu_arr = (ctypes.c_int32 * len(cu))(*cu)
     dev = Q.device
     f32 = torch.float32
@@ -397,7 +452,7 @@ class PreparedChain:
         n_tok, d = H.shape
         s = self._stream
         self._score_args = (dt, _ptr(H), H.stride(0), n_tok, d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2),
-                            W1.shape[0], _ptr(out["score"]), s)
+                            W1.shape[0], _ptr(out["score"]), _ptr(dev_status), s)
         self._select_args = (_ptr(out["score"]), self._seqs.ref(), _ptr(out["kept_idx"]), _ptr(out["cu_kept_dev"]),
                              _ptr(dev_status), s)
         self._gather_args = (dt, _ptr(H), H.stride(0), d, _ptr(out["score"]), _ptr(out["kept_idx"]), self._seqs.ref(),

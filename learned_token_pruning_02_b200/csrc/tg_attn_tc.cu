@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tmV, const float* __restrict__ logg,
                    const float* __restrict__ gain, const int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ O,
                    float* __restrict__ lse, int64_t m_tot, int Hq, int Hkv, float qk_scale, uint32_t flags,
-                   int32_t* __restrict__ dev_status, int qkv_ready, const __grid_constant__ ATParams p) {
+                   int32_t* __restrict__ dev_status, int qkv_ready, uint64_t probe_ns,
+                   const __grid_constant__ ATParams p) {
   using C = ACfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -95,7 +96,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* pvdone = bars + 17;  // [2]
   uint64_t* mlready = bars + 19;
   uint64_t* drain = bars + 20;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  uint64_t* probe = bars + 21;  // test hook: a barrier nothing signals
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* bias_s = reinterpret_cast<float*>(tail + 256);  // [2][128]
   float* gmul_s = bias_s + 2 * BKV;                      // [2][128]
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
+    wait_probe(probe, probe_ns, abort, dev_status);  // no-op unless a test asked for it
     // With qkv_ready (the chained prefill, where Q, K and V are inputs of the whole chain and the
     // previous kernel only produces log g and pos), Q and the first key tiles go out before the
     // wait on that kernel; otherwise anything may come from it and the wait is first.
@@ -156,10 +159,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
-    mbar_arrive_expect_tx(qfull, C::TILE_BYTES);
-    for (int bx = 0; bx < C::NBOX; ++bx)
-      tma_load_2d(smem + C::Q_OFF + bx * (BQ * 128), &tmQ, h * D + bx * 64, off + t * BQ, qfull);
-    for (int j = 0; j < KS && j < nt; ++j) {
+    if (!*abort) {
+      mbar_arrive_expect_tx(qfull, C::TILE_BYTES);
+      for (int bx = 0; bx < C::NBOX; ++bx)
+        tma_load_2d(smem + C::Q_OFF + bx * (BQ * 128), &tmQ, h * D + bx * 64, off + t * BQ, qfull);
+    }
+    for (int j = 0; j < KS && j < nt && !*abort; ++j) {
       uint8_t* kb = smem + C::K_OFF + j * C::TILE_BYTES;
       mbar_arrive_expect_tx(&kfull[j], C::TILE_BYTES);
       for (int bx = 0; bx < C::NBOX; ++bx)
@@ -177,8 +182,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   griddep_launch_dependents();  // the next kernel may start its prologue
   griddep_wait();               // (a no-op once thread 0's wait has returned)
   const uint32_t tmem = *tmem_slot;
+  const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
 
-  if (warp == 0) {  // ------------------------------------------------- Q and K producer
+  if (skip) {
+  } else if (warp == 0) {  // ------------------------------------------ Q and K producer
     if (lane == 0) {
       int issued = KS < nt ? KS : nt;
       for (int j = issued; j < nt; ++j) {
@@ -499,7 +506,8 @@ tg_status launch_d(const AttnArgs& a, const AttnSeq* seqs, int nseq, cudaStream_
   cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, a.logg, a.head_gain, a.pos,
                                         static_cast<__nv_bfloat16*>(a.O), a.lse, a.m_tot, a.Hq, a.Hkv,
-                                        a.scale * kLog2e, a.flags, a.dev_status, a.qkv_ready ? 1 : 0, p),
+                                        a.scale * kLog2e, a.flags, a.dev_status, a.qkv_ready ? 1 : 0,
+                                        wait_probe_ns(), p),
                      "tg_gated_attn_fwd: attn_tc launch");
 }
 

@@ -13,6 +13,9 @@
 namespace tg {
 
 static thread_local char g_err[512] = "";
+static thread_local uint64_t g_wait_probe_ns = 0;  // test hook of the bounded waits (0 = off)
+
+uint64_t wait_probe_ns() { return g_wait_probe_ns; }
 
 void set_error(const char* fmt, ...) {
   va_list ap;
@@ -141,7 +144,14 @@ const char* tg_status_string(int32_t st) {
 
 const char* tg_last_error(void) { return g_err; }
 
-int32_t tg_version(void) { return (1 << 16) | 1; }
+int32_t tg_version(void) { return (1 << 16) | 2; }
+
+tg_status tg_set_test_wait_probe(int64_t limit_ns) {
+  g_err[0] = 0;
+  if (limit_ns < 0) return fail(TG_ERR_INVALID_ARG, "limit_ns < 0");
+  g_wait_probe_ns = (uint64_t)limit_ns;
+  return TG_OK;
+}
 
 tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host) {
   g_err[0] = 0;
@@ -159,7 +169,7 @@ tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host) {
 
 tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, int32_t d,
                    const void* W1, const float* b1, const void* w2, float b2, int32_t dg,
-                   float* score, void* stream) {
+                   float* score, int32_t* dev_status, void* stream) {
   g_err[0] = 0;
   if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
   if (n_tok < 0 || d <= 0 || dg <= 0 || ldh < d)
@@ -174,7 +184,7 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
   tg_status st = check_device();
   if (st != TG_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  if (dtype == TG_BF16) return launch_score_tc(H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, s);
+  if (dtype == TG_BF16) return launch_score_tc(H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, dev_status, s);
   return launch_score_simt(dtype, H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, s);
 }
 
@@ -442,7 +452,7 @@ tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t
   std::vector<int32_t> cu(seqs->B + 1);
   st = tg_kept_counts(seqs, cu.data());
   if (st != TG_OK) return st;
-  st = tg_score(dtype, H, ldh, n_tot, d, W1, b1, w2, b2, dg, score, stream);
+  st = tg_score(dtype, H, ldh, n_tot, d, W1, b1, w2, b2, dg, score, dev_status, stream);
   if (st != TG_OK) return st;
   if (dtype != TG_BF16 || n_layers == 0 || m_tot == 0) {
     st = select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, nullptr, nullptr, nullptr, 0);

@@ -21,6 +21,11 @@ tg_status cuda_status(cudaError_t e, const char* what);
 tg_status check_device();
 int device_sm_count();
 
+// Limit of the test-only wait probe of the tensor-core kernels on this thread (0 = off; set by
+// tg_set_test_wait_probe). A kernel given a non-zero limit waits that long on a barrier that
+// nothing signals, records TG_DEV_TIMEOUT and skips all of its work.
+uint64_t wait_probe_ns();
+
 // Function attributes (shared-memory size, carveout) apply per device. True until
 // mark_attrs_set(slot) is called on the current device; slots name the launchers.
 // Template kernels take one slot per instantiation (score: dg 64/128/256; attention: D 64/128
@@ -66,7 +71,7 @@ tg_status launch_score_simt(tg_dtype dt, const void* H, int64_t ldh, int64_t n_t
 
 tg_status launch_score_tc(const void* H, int64_t ldh, int64_t n_tok, int d, const void* W1,
                           const float* b1, const void* w2, float b2, int dg, float* score,
-                          cudaStream_t st);
+                          int32_t* dev_status, cudaStream_t st);
 
 struct SelSeq {
   int32_t start;    // packed row of the sequence's first token

@@ -56,7 +56,7 @@ struct QKVParams {
 __global__ void __launch_bounds__(NTHREADS, 1)
     qkv_rope_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ Qo, __nv_bfloat16* __restrict__ Ko,
-                    __nv_bfloat16* __restrict__ Vo, int32_t* __restrict__ dev_status,
+                    __nv_bfloat16* __restrict__ Vo, int32_t* __restrict__ dev_status, uint64_t probe_ns,
                     const __grid_constant__ QKVParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -69,7 +69,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* accf = wempty + WS;                         // [2] accumulator complete
   uint64_t* acce = accf + 2;                            // [2] accumulator consumed
   uint64_t* drain = acce + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* probe = drain + 1;  // test hook: a barrier nothing signals
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(probe + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
+    wait_probe(probe, probe_ns, abort, dev_status);  // no-op unless a test asked for it
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
@@ -105,8 +107,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int nk = p.nk;
+  const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
 
-  if (warp == 0 || warp == WPROD) {
+  if (skip) {
+  } else if (warp == 0 || warp == WPROD) {
     if (lane == 0) {  // ------------------------------------ TMA producers: H_kept (warp 0), W (warp 10)
       const bool is_a = warp == 0;
       const int depth = is_a ? AS : WS;
@@ -193,7 +197,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       const int gm = (tile / p.tiles_n) * BM + r;
       const bool valid = gm < p.M;
-      const double pr = valid ? (double)pos[gm] : 0.0;
+      const double pr = (valid && p.rotate) ? (double)pos[gm] : 0.0;  // pos may be NULL without rotation
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * BN + half * 128;
       const int cbase = (tile % p.tiles_n) * BN + half * 128;  // first output column of this half
 #pragma unroll 1
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 
   // every product has completed before TMEM is released
-  if (warp == 1) {
+  if (warp == 1 && !skip) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {
     }
@@ -308,7 +312,8 @@ tg_status launch_qkv_rope(const void* Hk, int64_t M, int d, const void* W, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, qkv_rope_kernel, tmA, tmW, pos, static_cast<__nv_bfloat16*>(Q),
-                                        static_cast<__nv_bfloat16*>(K), static_cast<__nv_bfloat16*>(V), dev_status, p),
+                                        static_cast<__nv_bfloat16*>(K), static_cast<__nv_bfloat16*>(V), dev_status,
+                                        wait_probe_ns(), p),
                      "tg_qkv_rope: launch");
 }
 

@@ -45,7 +45,9 @@ def test_status_strings_and_version(L):
     assert L.tg_status_string(4) == b"TG_ERR_CUDA"
     assert L.tg_status_string(99) == b"TG_ERR_UNKNOWN"
     assert L.tg_version() >> 16 == 1
-    assert L.tg_version() & 0xffff >= 1  # the projection, split selection and backward
+    assert L.tg_version() & 0xffff >= 2  # 1.1: projection, split selection, backward; 1.2: score status
+    assert L.tg_set_test_wait_probe(-1) == 1
+    assert L.tg_set_test_wait_probe(0) == 0
 
 
 @pytest.mark.parametrize("seed", range(5))
@@ -80,15 +82,15 @@ def test_argument_errors_are_synchronous(L):
     V = ctypes.c_void_p
     fake = V(0x1000)  # never dereferenced: every call below fails validation first
     # tg_score: null H, bad dg, bad d, misaligned pointer
-    assert L.tg_score(1, None, 64, 10, 64, fake, None, fake, 0.0, 64, fake, None) == 1
-    assert L.tg_score(1, fake, 64, 10, 64, fake, None, fake, 0.0, 96, fake, None) == 2
-    assert L.tg_score(1, fake, 96, 10, 96, fake, None, fake, 0.0, 64, fake, None) == 2
-    assert L.tg_score(1, V(0x1002), 64, 10, 64, fake, None, fake, 0.0, 64, fake, None) == 2
-    assert L.tg_score(7, fake, 64, 10, 64, fake, None, fake, 0.0, 64, fake, None) == 1
-    assert L.tg_score(1, fake, 32, 10, 64, fake, None, fake, 0.0, 64, fake, None) == 1  # ldh < d
+    assert L.tg_score(1, None, 64, 10, 64, fake, None, fake, 0.0, 64, fake, None, None) == 1
+    assert L.tg_score(1, fake, 64, 10, 64, fake, None, fake, 0.0, 96, fake, None, None) == 2
+    assert L.tg_score(1, fake, 96, 10, 96, fake, None, fake, 0.0, 64, fake, None, None) == 2
+    assert L.tg_score(1, V(0x1002), 64, 10, 64, fake, None, fake, 0.0, 64, fake, None, None) == 2
+    assert L.tg_score(7, fake, 64, 10, 64, fake, None, fake, 0.0, 64, fake, None, None) == 1
+    assert L.tg_score(1, fake, 32, 10, 64, fake, None, fake, 0.0, 64, fake, None, None) == 1  # ldh < d
     assert b"dg" in L.tg_last_error() or b"ldh" in L.tg_last_error()
     # n_tok == 0 is a no-op that needs no device
-    assert L.tg_score(1, None, 64, 0, 64, None, None, None, 0.0, 64, None, None) == 0
+    assert L.tg_score(1, None, 64, 0, 64, None, None, None, 0.0, 64, None, None, None) == 0
     # tg_topk_select: q > N, null outputs
     s = _seqs([10], [11], [2])
     assert L.tg_topk_select(fake, s.ref(), fake, None, None, None) == 1
@@ -194,3 +196,74 @@ def test_binding_refuses_wrong_side_dtypes():
     with pytest.raises(TypeError, match="dQ"):
         tg.tg_gated_attn_bwd(Q, K, V, None, pos, [0, 4], Q, torch.zeros(2, 4), Q, 0.1,
                              dQ=torch.zeros(4, 2, 64, dtype=torch.bfloat16))
+
+
+def test_binding_checks_projection_shapes():
+    """tg_qkv_rope builds its TMA maps from M, d and the head counts, so a short W_qkv or a
+    strided H_kept would be read wrongly on the device: the binding refuses them first."""
+    import torch
+    bf = torch.bfloat16
+    M, d, Hq, Hkv, D = 8, 128, 2, 1, 64
+    Hk = torch.zeros(M, d, dtype=bf)
+    W = torch.zeros((Hq + 2 * Hkv) * D, d, dtype=bf)
+    pos = torch.arange(M, dtype=torch.int32)
+    with pytest.raises(ValueError, match="W_qkv has shape"):
+        tg.tg_qkv_rope(Hk, W[:-1], pos, Hq, Hkv, D, 1e4)
+    with pytest.raises(ValueError, match="H_kept must be contiguous"):
+        tg.tg_qkv_rope(torch.zeros(M, 2 * d, dtype=bf)[:, ::2], W, pos, Hq, Hkv, D, 1e4)
+    with pytest.raises(ValueError, match="W_qkv must be contiguous"):
+        tg.tg_qkv_rope(Hk, torch.zeros(d, (Hq + 2 * Hkv) * D, dtype=bf).t(), pos, Hq, Hkv, D, 1e4)
+    with pytest.raises(ValueError, match="pos must hold"):
+        tg.tg_qkv_rope(Hk, W, pos[:M - 1], Hq, Hkv, D, 1e4)
+    with pytest.raises(ValueError, match="pos must hold"):
+        tg.tg_qkv_rope(Hk, W, None, Hq, Hkv, D, 1e4)
+    with pytest.raises(ValueError, match="Q has shape"):
+        tg.tg_qkv_rope(Hk, W, pos, Hq, Hkv, D, 1e4, Q=torch.zeros(M, Hq + 1, D, dtype=bf))
+    with pytest.raises(ValueError, match="V has shape"):
+        tg.tg_qkv_rope(Hk, W, pos, Hq, Hkv, D, 1e4, V=torch.zeros(M - 1, Hkv, D, dtype=bf))
+    # without rotation pos is not needed: the call gets as far as the device check
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        tg.tg_qkv_rope(Hk, W, None, Hq, Hkv, D, 0.0)
+
+
+def test_binding_checks_backward_shapes():
+    """tg_gated_attn_bwd indexes lse as [Hq, M] and writes dK/dV rows up to cu_kept[-1]: every
+    shape that would send it out of bounds is refused before the call."""
+    import torch
+    bf, f32 = torch.bfloat16, torch.float32
+    M, Hq, Hkv, D = 6, 4, 2, 64
+    Q = torch.zeros(M, Hq, D, dtype=bf)
+    K = torch.zeros(M, Hkv, D, dtype=bf)
+    pos = torch.arange(M, dtype=torch.int32)
+    lse = torch.zeros(Hq, M, dtype=f32)
+    logg = torch.zeros(M, dtype=f32)
+
+    def call(**kw):
+        a = dict(Q=Q, K=K, V=K, logg=logg, pos=pos, cu_kept=[0, M], O=Q, lse=lse, dO=Q, softmax_scale=0.1)
+        a.update(kw)
+        return tg.tg_gated_attn_bwd(**a)
+
+    with pytest.raises(ValueError, match="cu_kept"):
+        call(cu_kept=[0, M - 1])
+    with pytest.raises(ValueError, match="cu_kept"):
+        call(cu_kept=[0, 2, M + 1])
+    with pytest.raises(ValueError, match="lse has shape"):
+        call(lse=torch.zeros(Hq, M - 1, dtype=f32))
+    with pytest.raises(ValueError, match="pos holds"):
+        call(pos=pos[:M - 1])
+    with pytest.raises(ValueError, match="logg holds"):
+        call(logg=logg[:M - 2])
+    with pytest.raises(ValueError, match="V has shape"):
+        call(V=torch.zeros(M, Hkv + 1, D, dtype=bf))
+    with pytest.raises(ValueError, match="O has shape"):
+        call(O=torch.zeros(M, Hq, D // 2, dtype=bf))
+    with pytest.raises(ValueError, match="dO has shape"):
+        call(dO=torch.zeros(M - 1, Hq, D, dtype=bf))
+    with pytest.raises(ValueError, match="dK has shape"):
+        call(dK=torch.zeros(M, Hq, D, dtype=f32))
+    with pytest.raises(ValueError, match="dlogg has shape"):
+        call(dlogg=torch.zeros(M + 1, dtype=f32))
+    with pytest.raises(ValueError, match="head_gain holds"):
+        call(head_gain=torch.ones(Hq - 1, dtype=f32))
+    with pytest.raises(ValueError, match="CUDA tensors only"):  # well-formed: stops at the device check
+        call()

@@ -37,3 +37,22 @@ def test_qkv_rope_matches_oracle(case):
         err = max_abs_rel(from_dev(got), ref)
         assert err <= TOL["bf16"], (name, err)
     assert st.item() == 0
+
+
+def test_qkv_no_rotation_without_positions():
+    """rope_theta = 0 needs no positions: pos=None (a NULL pointer through the C ABI) gives the
+    plain projection, equal to the oracle's and bit-identical to the same call with positions."""
+    M, d, Hq, Hkv, D = 333, 256, 4, 2, 64
+    g = np.random.default_rng(5)
+    Hk = ti.f32_to_bf16_bits((g.standard_normal((M, d)) / 2).astype(np.float32))
+    W = ti.f32_to_bf16_bits((g.standard_normal(((Hq + 2 * Hkv) * D, d)) / np.sqrt(d)).astype(np.float32))
+    st = torch.zeros(1, device="cuda", dtype=torch.int32)
+    Hd, Wd = to_dev(Hk, "bf16"), to_dev(W, "bf16")
+    Q, K, V = tg.tg_qkv_rope(Hd, Wd, None, Hq, Hkv, D, 0.0, dev_status=st)
+    Q2, K2, V2 = tg.tg_qkv_rope(Hd, Wd, torch.arange(M, dtype=torch.int32, device="cuda"), Hq, Hkv, D, 0.0)
+    torch.cuda.synchronize()
+    rQ, rK, rV = orc.qkv_rope(ti.widen(Hk, "bf16"), ti.widen(W, "bf16"), np.zeros(M, np.int64), Hq, Hkv, D, 0.0)
+    for got, again, ref in ((Q, Q2, rQ), (K, K2, rK), (V, V2, rV)):
+        assert max_abs_rel(from_dev(got), ref) <= TOL["bf16"]
+        assert torch.equal(got, again)
+    assert st.item() == 0
