@@ -37,6 +37,13 @@ namespace cg = cooperative_groups;
 namespace tg {
 namespace {
 
+// A key whose gate value is exactly 0 (log g = -inf) is masked for every head gain (gain * -inf
+// would give NaN for a zero gain), as in the forward.
+__device__ __forceinline__ float key_bias(float gain, float lg) { return lg == -INFINITY ? -INFINITY : gain * lg; }
+// A query row whose visible keys are all masked has lse = -inf in the forward; reading it as +inf
+// makes every weight exp(s - lse) of the row 0 instead of NaN.
+__device__ __forceinline__ float lse_or_inf(float l) { return l == -INFINITY ? INFINITY : l; }
+
 constexpr int BT = 32;    // rows per tile (queries or keys)
 constexpr int NT = 256;   // threads per CTA
 constexpr int MAXC = 8;   // CTAs per cluster (KV heads split over them)
@@ -200,9 +207,9 @@ __global__ void __launch_bounds__(NT, 2)
         const int qvalid = min(BT, sq.m - q0);
         __syncthreads();  // the previous tile's readers are done with Qs, dOs, Ss, dPs, bias
         if (tid < BT) {
-          bias[tid] = (logg && tid < kvalid) ? gh * __ldg(logg + sq.off + k0 + tid) : 0.f;
+          bias[tid] = (logg && tid < kvalid) ? key_bias(gh, __ldg(logg + sq.off + k0 + tid)) : 0.f;
           posq[tid] = tid < qvalid ? pos[sq.off + q0 + tid] : INT_MIN;
-          lse_s[tid] = tid < qvalid ? __ldg(lse + (int64_t)h * m_tot + sq.off + q0 + tid) : 0.f;
+          lse_s[tid] = tid < qvalid ? lse_or_inf(__ldg(lse + (int64_t)h * m_tot + sq.off + q0 + tid)) : 0.f;
         }
         const int64_t qrow = ((int64_t)(sq.off + q0) * Hq + h) * D;
         load_tile<T, D>(Q + qrow, (int64_t)Hq * D, qvalid, Qs);
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(NT, 2)
   if (tid < BT) {
     const bool ok = tid < qvalid;
     posq[tid] = ok ? pos[sq.off + q0 + tid] : INT_MIN;
-    lse_s[tid] = ok ? __ldg(lse + (int64_t)h * m_tot + sq.off + q0 + tid) : 0.f;
+    lse_s[tid] = ok ? lse_or_inf(__ldg(lse + (int64_t)h * m_tot + sq.off + q0 + tid)) : 0.f;
     // the positions must rise strictly inside a sequence (row order is the causal order)
     if (ok && h == 0 && q0 + tid > 0 && dev_status && pos[sq.off + q0 + tid - 1] >= posq[tid])
       atomicOr(dev_status, TG_DEV_POS_NOT_ASCENDING);
@@ -324,7 +331,7 @@ __global__ void __launch_bounds__(NT, 2)
     __syncthreads();  // the previous key tile's readers are done with Ks, Vs, Ss, dPs, bias
     if (tid < BT) {
       const bool ok = tid < kvalid;
-      bias[tid] = (logg && ok) ? gh * __ldg(logg + sq.off + k0 + tid) : 0.f;
+      bias[tid] = (logg && ok) ? key_bias(gh, __ldg(logg + sq.off + k0 + tid)) : 0.f;
       posk[tid] = ok ? pos[sq.off + k0 + tid] : INT_MAX;
     }
     load_tile<T, D>(K + ((int64_t)(sq.off + k0) * Hkv + kvh) * D, (int64_t)Hkv * D, kvalid, Ks);
@@ -628,14 +635,14 @@ __global__ void __launch_bounds__(NTM * NWG, 1)
       }
       group_sync(1 + grp);  // dv is complete
       // P^T and dS^T in place: rows kr0 / kr1 (keys), columns 8j + 2t4 + {0, 1} (queries)
-      const float b0 = gh * lg0, b1 = gh * lg1;
+      const float b0 = key_bias(gh, lg0), b1 = key_bias(gh, lg1);
 #pragma unroll
       for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int qc = 8 * j + 2 * t4 + (e & 1);
           const bool vis = qc < qvalid && (e < 2 ? pk0 : pk1) <= posq[qc];
-          const float pv = vis ? expf(fmaf(scale, sT[j][e], (e < 2 ? b0 : b1) - lse_s[qc])) : 0.f;
+          const float pv = vis ? expf(fmaf(scale, sT[j][e], (e < 2 ? b0 : b1) - lse_or_inf(lse_s[qc]))) : 0.f;
           const float ds = pv * (pT[j][e] - dv[qc]);
           sT[j][e] = pv;
           pT[j][e] = ds;
@@ -792,7 +799,7 @@ __global__ void __launch_bounds__(NTM)
   if (tid < MT) {
     const bool ok = tid < qvalid;
     posq[tid] = ok ? pos[sq.off + q0 + tid] : INT_MIN;
-    lse_s[tid] = ok ? __ldg(lse + (int64_t)h * m_tot + sq.off + q0 + tid) : 0.f;
+    lse_s[tid] = ok ? lse_or_inf(__ldg(lse + (int64_t)h * m_tot + sq.off + q0 + tid)) : 0.f;
     // the positions must rise strictly inside a sequence (row order is the causal order)
     if (ok && h == 0 && q0 + tid > 0 && dev_status && pos[sq.off + q0 + tid - 1] >= posq[tid])
       atomicOr(dev_status, TG_DEV_POS_NOT_ASCENDING);
@@ -864,7 +871,7 @@ __global__ void __launch_bounds__(NTM)
       for (int e = 0; e < 4; ++e) {
         const int qr = e < 2 ? qr0 : qr1, kc = 8 * j + 2 * t4 + (e & 1);
         const bool vis = kc < kvalid && posk[kc] <= posq[qr];
-        const float pv = vis ? expf(fmaf(scale, sc[j][e], gh * lgk[kc] - lse_s[qr])) : 0.f;
+        const float pv = vis ? expf(fmaf(scale, sc[j][e], key_bias(gh, lgk[kc]) - lse_s[qr])) : 0.f;
         dp[j][e] = pv * (dp[j][e] - dv[qr]);
       }
     // dQ += dS K: k runs over the 32 keys (two steps of 16)

@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(WARPS * 32)
     for (int e = 0; e < EPL; ++e) dot = fmaf(qv[e], ldf(K, (j * Hkv + kv) * D + lane * EPL + e), dot);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    const float b2 = logg ? gain2 * logg[j] : 0.f;  // gain * log2(g_j)
+    const float lgj = logg ? logg[j] : 0.f;
+    const float b2 = lgj == -INFINITY ? -INFINITY : gain2 * lgj;  // gain * log2(g_j); g = 0 closes the key
     const float s2 = unnorm ? dot : dot + b2;
     if (s2 == -INFINITY) continue;
     const float mn = fmaxf(m, s2);

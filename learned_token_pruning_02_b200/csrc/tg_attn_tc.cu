@@ -72,6 +72,38 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of arguments on the FMA pipe, so that part of a tile's exponentials leave the
+// MUFU unit (which has a sixteenth of the FMA pipe's lanes). Cody-Waite range reduction:
+// x = n + f with n = round(x) (taken from the low mantissa bits of x + 1.5 * 2^23) and
+// f in [-1/2, 1/2]; 2^f from a cubic fitted here by minimising the maximum relative error on
+// [-1/2, 1/2] (iteratively reweighted least squares; max relative error 7.5e-5, far below the
+// bf16 rounding that P gets before the PV product); 2^n is added to the exponent field with
+// one integer multiply-add. Arguments are clamped to >= -125 so that the exponent stays
+// normal: such a weight is 2^-125 instead of 0, which no fp32 sum of 128 terms can notice.
+constexpr float kExpC0 = 0.99992806f, kExpC1 = 0.69326097f, kExpC2 = 0.24261114f, kExpC3 = 0.05517167f;
+constexpr float kRoundMagic = 12582912.f;  // 1.5 * 2^23
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  const float2 xc = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  const float2 t = __fadd2_rn(xc, make_float2(kRoundMagic, kRoundMagic));
+  const float2 n = __fadd2_rn(t, make_float2(-kRoundMagic, -kRoundMagic));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), xc);
+  float2 q = __ffma2_rn(f, make_float2(kExpC3, kExpC3), make_float2(kExpC2, kExpC2));
+  q = __ffma2_rn(q, f, make_float2(kExpC1, kExpC1));
+  q = __ffma2_rn(q, f, make_float2(kExpC0, kExpC0));
+  // the low 9 bits of t hold n (two's complement); times 2^23 they land in the exponent field
+  return make_float2(__uint_as_float(__float_as_uint(t.x) * 8388608u + __float_as_uint(q.x)),
+                     __uint_as_float(__float_as_uint(t.y) * 8388608u + __float_as_uint(q.y)));
+}
+
+// Which pairs of a 128-key row take the FMA-pipe exponential: kPolyOf8 of every 8 pairs.
+constexpr int kPolyOf8 = 3;
+
 template <int D, bool UNNORM>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -183,7 +215,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   griddep_wait();               // (a no-op once thread 0's wait has returned)
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
-
+  if (warp < 4) {
   if (skip) {
   } else if (warp == 0) {  // ------------------------------------------ Q and K producer
     if (lane == 0) {
@@ -237,7 +269,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int kl = j * BKV + lane * 4 + e;
-        bv[e] = (logg && kl < m) ? gain2 * logg[off + kl] : 0.f;
+        const float lg = (logg && kl < m) ? logg[off + kl] : 0.f;
+        bv[e] = lg == -INFINITY ? -INFINITY : gain2 * lg;  // g = 0 closes the key whatever the gain
       }
       if (u > 0 && !__all_sync(0xffffffffu, mbar_wait(&pready[c], (u - 1) & 1, abort, dev_status))) break;
 #pragma unroll
@@ -247,18 +280,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       mbar_arrive(&bfull[c]);
     }
-  } else if (warp == 1) {  // ------------------------------------------------ MMA issuer
+  } else {  // warp 1 ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t qa = smem_u32(smem + C::Q_OFF);
       // Fixed schedule with blocking (suspending) waits: S_0, S_1, then PV_j followed by
       // S_{j+2} for j = 0, 1, ... The chains alternate, so this is the order the products
       // become ready in, and a waiting issuer sleeps instead of taking issue slots from the
-      // softmax warps that share its scheduler. S_j needs K_j and the chain's S buffer (free
-      // once PV_{j-2} completed); PV_j needs P_j and V_j.
+      // softmax warps that share its scheduler. PV_j needs P_j and V_j; S_{j+2} needs K_{j+2}
+      // and overwrites the TMEM columns PV_j reads P_j from, which is safe without waiting for
+      // PV_j to complete: the MMAs one thread issues execute in issue order, so S_{j+2} writes
+      // only after PV_j has read its operand, and the tensor pipe never drains between them.
       auto issue_s = [&](int j) -> bool {
-        const int c = j & 1, u = j >> 1, ks = j % KS;
+        const int c = j & 1, ks = j % KS;
         if (!mbar_wait(&kfull[ks], (j / KS) & 1, abort, dev_status)) return false;
-        if (u > 0 && !mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status)) return false;
         tc_fence_after();
         const uint32_t ka = smem_u32(smem + C::K_OFF + ks * C::TILE_BYTES);
 #pragma unroll
@@ -293,7 +327,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {
       }
     }
-  } else if (warp >= 4) {  // ------------------------------------------- softmax warpgroups
+  }
+  } else if (!skip) {  // ----------------------------------------------- softmax warpgroups
     const int c = (warp - 4) >> 2;  // chain: 0 = warps 4-7 (even tiles), 1 = warps 8-11 (odd tiles)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // query row in the tile == TMEM lane
@@ -321,39 +356,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int ch = 0; ch < BKV / 32; ++ch)
         tmem_ld32(tS + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
       tmem_wait_ld();
+      float* x = reinterpret_cast<float*>(sr);
       const float4* bs4 = reinterpret_cast<const float4*>(bias_s + c * BKV);
-      // log2-domain logits scale*log2(e)*S + bias; causal mask on the diagonal tile only;
-      // the row max runs as 8 independent chains
-      float m8[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      const float2 qs2 = make_float2(qk_scale, qk_scale);
+      // log2-domain logits scale*log2(e)*S + bias in pairs; causal mask on the diagonal tile only
+#pragma unroll
+      for (int q = 0; q < BKV / 4; ++q) {
+        const float4 bb = bs4[q];
+        const float2 v0 = __ffma2_rn(make_float2(x[4 * q], x[4 * q + 1]), qs2, make_float2(bb.x, bb.y));
+        const float2 v1 = __ffma2_rn(make_float2(x[4 * q + 2], x[4 * q + 3]), qs2, make_float2(bb.z, bb.w));
+        x[4 * q] = v0.x;
+        x[4 * q + 1] = v0.y;
+        x[4 * q + 2] = v1.x;
+        x[4 * q + 3] = v1.y;
+      }
       if (j == t) {
 #pragma unroll
-        for (int q = 0; q < BKV / 4; ++q) {
-          const float4 bb = bs4[q];
-          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = 4 * q + e;
-            const float x = col > r ? -INFINITY : fmaf(__uint_as_float(sr[col]), qk_scale, bv[e]);
-            sr[col] = __float_as_uint(x);
-            m8[col & 7] = fmaxf(m8[col & 7], x);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < BKV / 4; ++q) {
-          const float4 bb = bs4[q];
-          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = 4 * q + e;
-            const float x = fmaf(__uint_as_float(sr[col]), qk_scale, bv[e]);
-            sr[col] = __float_as_uint(x);
-            m8[col & 7] = fmaxf(m8[col & 7], x);
-          }
-        }
+        for (int col = 0; col < BKV; ++col)
+          if (col > r) x[col] = -INFINITY;
       }
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      // row max with three-input max, four independent chains
+      float ma = -INFINITY, mbx = -INFINITY, mc = -INFINITY, md = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < BKV / 8; ++q) {
+        ma = max3(ma, x[8 * q], x[8 * q + 1]);
+        mbx = max3(mbx, x[8 * q + 2], x[8 * q + 3]);
+        mc = max3(mc, x[8 * q + 4], x[8 * q + 5]);
+        md = max3(md, x[8 * q + 6], x[8 * q + 7]);
+      }
+      const float mx = max3(ma, mbx, fmaxf(mc, md));
       const float m_cand = fmaxf(m_run, mx);
       // lazy rescale: move the running max only when it grows by more than the slack
       const bool resc = __any_sync(0xffffffffu, m_cand > m_run + kRescaleSlack);
@@ -363,34 +394,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         m_run = m_cand;
       }
       const float mb = m_run == -INFINITY ? 0.f : m_run;
-      // P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 nm2 = make_float2(-mb, -mb);
+      // P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns, 32 columns
+      // (64 keys) at a time so the first store overlaps the second half's arithmetic
+      float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
       uint32_t pk[BKV / 2];
-      if constexpr (UNNORM) {
-        const float4* gm4 = reinterpret_cast<const float4*>(gmul_s + c * BKV);
 #pragma unroll
-        for (int q = 0; q < BKV / 4; ++q) {
-          const float4 gg = gm4[q];
-          const float p0 = ex2(__uint_as_float(sr[4 * q]) - mb), p1 = ex2(__uint_as_float(sr[4 * q + 1]) - mb);
-          const float p2 = ex2(__uint_as_float(sr[4 * q + 2]) - mb), p3 = ex2(__uint_as_float(sr[4 * q + 3]) - mb);
-          s4[0] += p0;
-          s4[1] += p1;
-          s4[2] += p2;
-          s4[3] += p3;
-          pk[2 * q] = pack_bf16(p0 * gg.x, p1 * gg.y);
-          pk[2 * q + 1] = pack_bf16(p2 * gg.z, p3 * gg.w);
-        }
-      } else {
+      for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
-        for (int e = 0; e < BKV; e += 2) {
-          const float p0 = ex2(__uint_as_float(sr[e]) - mb), p1 = ex2(__uint_as_float(sr[e + 1]) - mb);
-          s4[(e >> 1) & 3] += p0 + p1;
-          pk[e >> 1] = pack_bf16(p0, p1);
+        for (int q = h2 * (BKV / 4); q < (h2 + 1) * (BKV / 4); ++q) {
+          const float2 d = __fadd2_rn(make_float2(x[2 * q], x[2 * q + 1]), nm2);
+          float2 pr;
+          if constexpr (UNNORM) {
+            pr = make_float2(ex2(d.x), ex2(d.y));
+            const float2 gg = *reinterpret_cast<const float2*>(gmul_s + c * BKV + 2 * q);
+            if (q & 1) sb = __fadd2_rn(sb, pr); else sa = __fadd2_rn(sa, pr);
+            pr = __fmul2_rn(pr, gg);
+          } else {
+            if (j != t && (q & 7) >= 8 - kPolyOf8) pr = exp2_fma2(d);
+            else pr = make_float2(ex2(d.x), ex2(d.y));
+            if (q & 1) sb = __fadd2_rn(sb, pr); else sa = __fadd2_rn(sa, pr);
+          }
+          pk[q] = pack_bf16(pr.x, pr.y);
         }
+        tmem_st32(tS + h2 * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[h2 * 32]));
       }
-      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      const float2 s2 = __fadd2_rn(sa, sb);
+      const float sum = s2.x + s2.y;
       tmem_wait_st();
       if (resc && u > 0) {  // rescale the chain's O once its previous PV product has landed
         if (!__all_sync(0xffffffffu, mbar_wait(&pvdone[c], (u - 1) & 1, abort, dev_status))) {

@@ -205,19 +205,31 @@ def gated_attention(Q, K, V, logg, pos, cu_kept, Hq, Hkv, scale, head_gain=None,
         for h in range(Hq):
             kv = h // G
             logits = scale * (Q[r, h, :] @ K[lo:hi, kv, :].T)
-            bias = gain[h] * lg[lo:hi]
+            bias = _key_bias(gain[h], lg[lo:hi])
             S = logits if unnormalised else logits + bias[None, :]
-            S = np.where(allowed, S, -np.inf)
+            S = np.where(allowed & (bias > -np.inf)[None, :], S, -np.inf)
             m = S.max(axis=1, keepdims=True)
+            m = np.where(np.isfinite(m), m, 0.0)
             P = np.exp(S - m)
             l = P.sum(axis=1, keepdims=True)
-            P = P / l
+            P = P / np.where(l > 0, l, 1.0)
             if unnormalised:
                 O[sel, h, :] = P @ (np.exp(bias)[:, None] * V[lo:hi, kv, :])
             else:
                 O[sel, h, :] = P @ V[lo:hi, kv, :]
-            LSE[h, sel] = (m + np.log(l))[:, 0]
+            with np.errstate(divide="ignore"):
+                LSE[h, sel] = (m + np.log(l))[:, 0]
     return O, LSE
+
+
+def _key_bias(gain, lg):
+    """gain * log g per key, where a key whose gate value is exactly 0 (log g = -inf) stays at
+    -inf for every gain: a zero gate closes the key (Figure 1(c) multiplies its weight by 0),
+    and 0 * -inf must not turn it into NaN. A query row whose visible keys are all closed has
+    all-zero weights: O = 0 and LSE = -inf."""
+    lg = np.asarray(lg, dtype=np.float64)
+    with np.errstate(invalid="ignore"):
+        return np.where(lg == -np.inf, -np.inf, gain * lg)
 
 
 def gated_attention_bwd(Q, K, V, logg, pos, cu_kept, Hq, Hkv, scale, dO, head_gain=None):
@@ -257,9 +269,12 @@ def gated_attention_bwd(Q, K, V, logg, pos, cu_kept, Hq, Hkv, scale, dO, head_ga
         for h in range(Hq):
             kv = h // G
             Qh, Kh, Vh, dOh = Q[lo:hi, h, :], K[lo:hi, kv, :], V[lo:hi, kv, :], dO[lo:hi, h, :]
-            S = np.where(allowed, scale * (Qh @ Kh.T) + gain[h] * lg[lo:hi][None, :], -np.inf)
-            P = np.exp(S - S.max(axis=1, keepdims=True))
-            P = P / P.sum(axis=1, keepdims=True)
+            bias = _key_bias(gain[h], lg[lo:hi])
+            S = np.where(allowed & (bias > -np.inf)[None, :], scale * (Qh @ Kh.T) + bias[None, :], -np.inf)
+            mx = S.max(axis=1, keepdims=True)
+            P = np.exp(S - np.where(np.isfinite(mx), mx, 0.0))
+            l = P.sum(axis=1, keepdims=True)
+            P = P / np.where(l > 0, l, 1.0)
             dP = dOh @ Vh.T
             dS = P * (dP - (dP * P).sum(axis=1, keepdims=True))
             dQ[lo:hi, h, :] = scale * (dS @ Kh)

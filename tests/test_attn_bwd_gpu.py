@@ -146,3 +146,34 @@ def test_attn_bwd_rejects_unsupported():
         tg.tg_gated_attn_bwd(dev(c["Q"]), dev(c["K"]), dev(c["V"]), None, dev(c["pos"]), c["cu"].tolist(),
                              dev(O.astype(np.float32)), dev(lse.astype(np.float32)), dev(c["dO"]), c["scale"],
                              want_dscore=True)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_closed_gates_forward_and_backward(dtype):
+    """Keys with gate value exactly 0 (log g = -inf) are masked whatever the head gain, a gain
+    of 0 included; the first rows of a sequence, whose visible keys are all closed, get O = 0,
+    LSE = -inf and zero gradients. Forward and backward against the oracle, no NaN anywhere."""
+    c = _make(31, [300, 77], 4, 2, 128 if dtype == "bf16" else 64, dtype, True, True)
+    lg = c["logg"].copy()
+    lg[[0, 1, 7, 150, 299, 300, 340]] = -np.inf
+    c["logg"] = lg
+    c["hg"] = np.array([0.0, 1.0, 0.7, 0.0], np.float32)
+    O, lse, grads = _oracle(c)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dev = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    Og, Lg = tg.tg_gated_attn_fwd(to_dev(c["Q"], dtype), to_dev(c["K"], dtype), to_dev(c["V"], dtype), dev(lg),
+                                  dev(c["pos"]), c["cu"].tolist(), c["scale"], head_gain=dev(c["hg"]), dev_status=st)
+    torch.cuda.synchronize()
+    Ogn, Lgn = from_dev(Og), from_dev(Lg)
+    assert not np.isnan(Ogn).any() and not np.isnan(Lgn).any()
+    assert max_abs_rel(Ogn, O) <= TOL[dtype]
+    fin = np.isfinite(lse)
+    assert np.array_equal(np.isfinite(Lgn), fin)
+    assert max_abs_rel(Lgn[fin], lse[fin]) <= TOL[dtype]
+    got = _run(c, O, lse, st)
+    torch.cuda.synchronize()
+    for t in got:
+        if t is not None:
+            assert not torch.isnan(t).any()
+    _check(c, got, grads)
+    assert st.item() == 0

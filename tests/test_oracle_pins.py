@@ -513,3 +513,45 @@ def test_gate_score_grad_matches_central_differences():
               - _loss(Q, K, V, orc.gate_value(sm)[1], pos, cu, Hq, Hkv, scale, dO, hg)) / (2 * eps)
         assert abs(fd - ds[j]) <= 1e-6 * max(1.0, np.abs(ds).max()), j
     assert orc.gate_score_grad(np.array([5.0]), np.array([0.0]))[0] == 0.0
+
+
+def test_attention_closed_gate_is_a_removed_key_for_every_gain():
+    """A key with gate value exactly 0 (log g = -inf) contributes nothing, whatever the head's
+    gain, including a gain of 0 (where gain * log g would be 0 * -inf): it equals the sequence
+    with that key removed, for the biased and the unnormalised form. A query row whose visible
+    keys are all closed has all-zero weights: O = 0, LSE = -inf, and zero gradients."""
+    g = np.random.default_rng(21)
+    M, Hq, Hkv, D = 11, 3, 1, 4
+    Q, K, V = g.standard_normal((M, Hq, D)), g.standard_normal((M, Hkv, D)), g.standard_normal((M, Hkv, D))
+    pos = np.arange(M) * 3
+    lg = np.log(g.uniform(0.1, 1, M))
+    lg[4] = -np.inf
+    gain = np.array([0.0, 1.0, 2.5])
+    keep = np.array([i for i in range(M) if i != 4])
+    for unnorm in (False, True):
+        O, L = orc.gated_attention(Q, K, V, lg, pos, [0, M], Hq, Hkv, 0.5, head_gain=gain, unnormalised=unnorm)
+        Or, Lr = orc.gated_attention(Q[keep], K[keep], V[keep], lg[keep], pos[keep], [0, M - 1], Hq, Hkv, 0.5,
+                                     head_gain=gain, unnormalised=unnorm)
+        assert np.isfinite(O).all()
+        np.testing.assert_allclose(O[keep], Or, rtol=1e-12, atol=1e-13)
+        if not unnorm:  # the removed key's own row still sees the keys before it
+            np.testing.assert_allclose(L[:, keep], Lr, rtol=1e-12, atol=1e-13)
+    # gain 0 with open gates is plain causal attention (bias 0)
+    O0, _ = orc.gated_attention(Q, K, V, lg, pos, [0, M], Hq, Hkv, 0.5, head_gain=gain)
+    P0, _ = orc.gated_attention(Q[keep], K[keep], V[keep], None, pos[keep], [0, M - 1], Hq, Hkv, 0.5)
+    np.testing.assert_allclose(O0[keep, 0], P0[:, 0], rtol=1e-12, atol=1e-13)
+    # the first two rows with closed gates: row 0 and row 1 see only closed keys
+    lz = lg.copy()
+    lz[:2] = -np.inf
+    O, L = orc.gated_attention(Q, K, V, lz, pos, [0, M], Hq, Hkv, 0.5, head_gain=gain)
+    assert np.all(O[:2] == 0) and np.all(L[:, :2] == -np.inf)
+    dO = g.standard_normal((M, Hq, D))
+    dQ, dK, dV, dl = orc.gated_attention_bwd(Q, K, V, lz, pos, [0, M], Hq, Hkv, 0.5, dO, head_gain=gain)
+    for t in (dQ, dK, dV, dl):
+        assert np.isfinite(t).all()
+    assert np.all(dQ[:2] == 0) and np.all(dl[:2] == 0)
+    # away from the closed rows the gradient is that of the sequence without those keys' weight
+    dQr, dKr, dVr, dlr = orc.gated_attention_bwd(Q[2:], K[2:], V[2:], lz[2:], pos[2:], [0, M - 2], Hq, Hkv, 0.5,
+                                                 dO[2:], head_gain=gain)
+    np.testing.assert_allclose(dQ[2:], dQr, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dK[2:], dKr, rtol=1e-10, atol=1e-12)
