@@ -82,7 +82,8 @@ const char* tg_last_error(void);
 /* ABI version, (major << 16) | minor. 1.0: the gated-prefill path (tg_score, tg_topk_select,
  * tg_gather, tg_gated_attn_fwd, tg_prefill_above_L and the helpers). 1.1 adds tg_qkv_rope,
  * tg_topk_candidates, tg_topk_merge and tg_gated_attn_bwd. 1.2 gives tg_score a device
- * status word (its last argument before the stream) and adds tg_set_test_wait_probe. */
+ * status word (its last argument before the stream) and a temperature (after b2, also in
+ * tg_prefill_above_L), and adds tg_set_test_wait_probe. */
 int32_t tg_version(void);
 
 /* Test hook for the bounded waits, off by default (limit_ns = 0). With limit_ns > 0, every
@@ -102,12 +103,18 @@ tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host);
 
 /* Gate MLP score of every token (aitualizate.com TokenGate article, phase 2: an MLP scores
  * each token's post-attention residual state at layer L; thelatestinai.com TokenGate page,
- * Figure 1(b)):   score[i] = w2 . GELU(W1 h_i + b1) + b2,  GELU with the exact erf.
+ * Figure 1(b)):   score[i] = (w2 . GELU(W1 h_i + b1) + b2) / temperature,  GELU with the
+ * exact erf. The temperature is a reading of the gate temperature that the thelatestinai.com
+ * TokenGate page names in its Figure 7 caption (Eq. 7) without printing a formula: it
+ * divides the score, so the gate value is g = sigmoid(s / temperature) and the
+ * top-K selection (an order statistic) is the same for every temperature > 0. Pass 1 for the
+ * plain score.
  *   H      device act [n_tok, d], row stride ldh elements (ldh >= d)
  *   W1     device act [dg, d] row-major (output-major, like torch.nn.Linear.weight)
  *   b1     device f32 [dg], or NULL for zero
  *   w2     device act [dg]
  *   b2     scalar
+ *   temperature  > 0 and finite (else TG_ERR_INVALID_ARG)
  *   score  device f32 [n_tok] (written)
  *   dev_status device int32 [1] or NULL: a wait of the bf16 kernel that gave up sets
  *          TG_DEV_TIMEOUT (the scores of the tiles it did not finish are then unwritten)
@@ -115,8 +122,8 @@ tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host);
  * aligned H and W1. bf16 runs on the tensor cores with fp32 accumulation; f32 runs on the
  * CUDA cores in fp32. */
 tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, int32_t d,
-                   const void* W1, const float* b1, const void* w2, float b2, int32_t dg,
-                   float* score, int32_t* dev_status, void* stream);
+                   const void* W1, const float* b1, const void* w2, float b2, float temperature,
+                   int32_t dg, float* score, int32_t* dev_status, void* stream);
 
 /* Top-K over each sequence's context with the question tail always kept (aitualizate.com
  * TokenGate article, phase 2; thelatestinai.com TokenGate page, Figure 1(a)-(b)).
@@ -256,7 +263,7 @@ tg_status tg_gated_attn_bwd(tg_dtype dtype, const void* Q, const void* K, const 
  * any output of this call. */
 tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t d,
                              const void* W1, const float* b1, const void* w2, float b2,
-                             int32_t dg, const tg_seqs* seqs, int32_t n_layers,
+                             float temperature, int32_t dg, const tg_seqs* seqs, int32_t n_layers,
                              const void* const* Q, const void* const* K, const void* const* V,
                              int32_t Hq, int32_t Hkv, int32_t D, float softmax_scale,
                              const float* head_gain, uint32_t flags, float* score,

@@ -78,7 +78,7 @@ def lib() -> ctypes.CDLL:
     L.tg_kept_counts.restype = _I32
     L.tg_kept_counts.argtypes = [_SEQP, ctypes.POINTER(_I32)]
     L.tg_score.restype = _I32
-    L.tg_score.argtypes = [_I32, _VP, _I64, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP, _VP]
+    L.tg_score.argtypes = [_I32, _VP, _I64, _I64, _I32, _VP, _VP, _VP, _F, _F, _I32, _VP, _VP, _VP]
     L.tg_set_test_wait_probe.restype = _I32
     L.tg_set_test_wait_probe.argtypes = [_I64]
     L.tg_topk_select.restype = _I32
@@ -99,7 +99,7 @@ def lib() -> ctypes.CDLL:
                                     _I32, _I32, _F, _U32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]
     L.tg_prefill_above_L.restype = _I32
     L.tg_prefill_above_L.argtypes = [
-        _I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _I32, _SEQP, _I32,
+        _I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _F, _I32, _SEQP, _I32,
         ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP),
         _I32, _I32, _I32, _F, _VP, _U32, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
         ctypes.POINTER(_VP), ctypes.POINTER(_VP), _VP, _VP]
@@ -189,8 +189,8 @@ def tg_kept_counts(seqlens, q_len, k) -> list:
     return list(out)
 
 
-def tg_score(H, W1, b1, w2, b2: float, score=None, dev_status=None, stream=None):
-    """Gate-MLP score of every token: w2 . GELU(W1 h + b1) + b2 (float32 [n_tok])."""
+def tg_score(H, W1, b1, w2, b2: float, score=None, dev_status=None, stream=None, temperature: float = 1.0):
+    """Gate-MLP score of every token: (w2 . GELU(W1 h + b1) + b2) / temperature (float32 [n_tok])."""
     _want(torch.float32, b1=b1, score=score)
     _want(torch.int32, dev_status=dev_status)
     _cuda(H, W1, b1, w2, score, dev_status)
@@ -199,7 +199,8 @@ def tg_score(H, W1, b1, w2, b2: float, score=None, dev_status=None, stream=None)
     if score is None:
         score = torch.empty(n_tok, device=H.device, dtype=torch.float32)
     _check("tg_score", lib().tg_score(_dtype(H), _ptr(H), H.stride(0), n_tok, d, _ptr(W1), _ptr(b1), _ptr(w2),
-                                      float(b2), W1.shape[0], _ptr(score), _ptr(dev_status), _stream(stream)))
+                                      float(b2), float(temperature), W1.shape[0], _ptr(score), _ptr(dev_status),
+                                      _stream(stream)))
     return score
 
 
@@ -374,7 +375,7 @@ def tg_gated_attn_bwd(Q, K, V, logg, pos, cu_kept, O, lse, dO, softmax_scale: fl
 
 
 def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_scale, head_gain=None, flags=0,
-                       want_lse=False, out=None, dev_status=None, stream=None):
+                       want_lse=False, out=None, dev_status=None, stream=None, temperature: float = 1.0):
     """The whole gated path above layer L: score -> top-K -> gather -> gated attention per layer.
 
     layers: list of (Q, K, V) device tensors shaped by the kept count. Returns a dict of the
@@ -412,7 +413,8 @@ def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_sca
     oa = (_VP * max(nl, 1))(*[t.data_ptr() for t in out["O"]])
     la = (_VP * max(nl, 1))(*[(t.data_ptr() if t is not None else None) for t in out["lse"]])
     _check("tg_prefill_above_L", lib().tg_prefill_above_L(
-        _dtype(H), _ptr(H), H.stride(0), d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2), W1.shape[0], s.ref(), nl,
+        _dtype(H), _ptr(H), H.stride(0), d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2), float(temperature), W1.shape[0],
+        s.ref(), nl,
         qa, ka, va, Hq, Hkv, D, float(softmax_scale), _ptr(head_gain), int(flags), _ptr(out["score"]),
         _ptr(out["kept_idx"]), _ptr(out["cu_kept_dev"]), _ptr(out["H_kept"]), _ptr(out["pos"]), _ptr(out["g"]),
         _ptr(out["logg"]), oa, la, _ptr(dev_status), _stream(stream)))
@@ -436,7 +438,7 @@ class PreparedChain:
     """
 
     def __init__(self, H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_scale, out, head_gain=None, flags=0,
-                 dev_status=None, stream=None):
+                 dev_status=None, stream=None, temperature: float = 1.0):
         _want(torch.float32, b1=b1, head_gain=head_gain)
         _want(torch.int32, dev_status=dev_status)
         _check_out(out)
@@ -452,7 +454,7 @@ class PreparedChain:
         n_tok, d = H.shape
         s = self._stream
         self._score_args = (dt, _ptr(H), H.stride(0), n_tok, d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2),
-                            W1.shape[0], _ptr(out["score"]), _ptr(dev_status), s)
+                            float(temperature), W1.shape[0], _ptr(out["score"]), _ptr(dev_status), s)
         self._select_args = (_ptr(out["score"]), self._seqs.ref(), _ptr(out["kept_idx"]), _ptr(out["cu_kept_dev"]),
                              _ptr(dev_status), s)
         self._gather_args = (dt, _ptr(H), H.stride(0), d, _ptr(out["score"]), _ptr(out["kept_idx"]), self._seqs.ref(),
@@ -471,7 +473,8 @@ class PreparedChain:
         Hq = layers[0][0].shape[1] if nl else 1
         Hkv = layers[0][1].shape[1] if nl else 1
         D = layers[0][0].shape[2] if nl else 64
-        self._prefill_args = (dt, _ptr(H), H.stride(0), d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2), W1.shape[0],
+        self._prefill_args = (dt, _ptr(H), H.stride(0), d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2), float(temperature),
+                              W1.shape[0],
                               self._seqs.ref(), nl, *self._arrays, Hq, Hkv, D, float(softmax_scale), _ptr(head_gain),
                               int(flags), _ptr(out["score"]), _ptr(out["kept_idx"]), _ptr(out["cu_kept_dev"]),
                               _ptr(out["H_kept"]), _ptr(out["pos"]), _ptr(out["g"]), _ptr(out["logg"]), self._o_arr,

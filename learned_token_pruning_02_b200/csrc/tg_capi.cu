@@ -168,9 +168,11 @@ tg_status tg_kept_counts(const tg_seqs* seqs, int32_t* cu_kept_host) {
 }
 
 tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, int32_t d,
-                   const void* W1, const float* b1, const void* w2, float b2, int32_t dg,
-                   float* score, int32_t* dev_status, void* stream) {
+                   const void* W1, const float* b1, const void* w2, float b2, float temperature,
+                   int32_t dg, float* score, int32_t* dev_status, void* stream) {
   g_err[0] = 0;
+  if (!(temperature > 0.f) || temperature == INFINITY)
+    return fail(TG_ERR_INVALID_ARG, "temperature must be positive and finite");
   if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
   if (n_tok < 0 || d <= 0 || dg <= 0 || ldh < d)
     return fail(TG_ERR_INVALID_ARG, "need n_tok >= 0, d > 0, dg > 0, ldh >= d");
@@ -184,8 +186,9 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
   tg_status st = check_device();
   if (st != TG_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  if (dtype == TG_BF16) return launch_score_tc(H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, dev_status, s);
-  return launch_score_simt(dtype, H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, s);
+  const float inv_t = (float)(1.0 / (double)temperature);
+  if (dtype == TG_BF16) return launch_score_tc(H, ldh, n_tok, d, W1, b1, w2, b2, inv_t, dg, score, dev_status, s);
+  return launch_score_simt(dtype, H, ldh, n_tok, d, W1, b1, w2, b2, inv_t, dg, score, s);
 }
 
 // The selector with optional per-row outputs pos, g and log g (the chained prefill).
@@ -434,7 +437,7 @@ static tg_status gather_after(tg_dtype dtype, const void* H, int64_t ldh, int32_
 
 tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t d,
                              const void* W1, const float* b1, const void* w2, float b2,
-                             int32_t dg, const tg_seqs* seqs, int32_t n_layers,
+                             float temperature, int32_t dg, const tg_seqs* seqs, int32_t n_layers,
                              const void* const* Q, const void* const* K, const void* const* V,
                              int32_t Hq, int32_t Hkv, int32_t D, float softmax_scale,
                              const float* head_gain, uint32_t flags, float* score,
@@ -452,7 +455,7 @@ tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t
   std::vector<int32_t> cu(seqs->B + 1);
   st = tg_kept_counts(seqs, cu.data());
   if (st != TG_OK) return st;
-  st = tg_score(dtype, H, ldh, n_tot, d, W1, b1, w2, b2, dg, score, dev_status, stream);
+  st = tg_score(dtype, H, ldh, n_tot, d, W1, b1, w2, b2, temperature, dg, score, dev_status, stream);
   if (st != TG_OK) return st;
   if (dtype != TG_BF16 || n_layers == 0 || m_tot == 0) {
     st = select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, nullptr, nullptr, nullptr, 0);

@@ -65,12 +65,13 @@ __device__ __forceinline__ void gate_from_score(float s, float* g, float* lg) {
 // ----------------------------------------------------------------------------- launchers
 // Each returns TG_OK or TG_ERR_CUDA (argument checks happen in the C-ABI layer).
 
+// inv_t = 1 / temperature multiplies the score (exactly 1 for the plain score).
 tg_status launch_score_simt(tg_dtype dt, const void* H, int64_t ldh, int64_t n_tok, int d,
-                            const void* W1, const float* b1, const void* w2, float b2, int dg,
+                            const void* W1, const float* b1, const void* w2, float b2, float inv_t, int dg,
                             float* score, cudaStream_t st);
 
 tg_status launch_score_tc(const void* H, int64_t ldh, int64_t n_tok, int d, const void* W1,
-                          const float* b1, const void* w2, float b2, int dg, float* score,
+                          const float* b1, const void* w2, float b2, float inv_t, int dg, float* score,
                           int32_t* dev_status, cudaStream_t st);
 
 struct SelSeq {

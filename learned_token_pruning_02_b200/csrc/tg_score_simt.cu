@@ -1,4 +1,4 @@
-// Gate-MLP score on the CUDA cores (fp32 arithmetic): score = w2 . GELU(W1 h + b1) + b2.
+// Gate-MLP score on the CUDA cores (fp32 arithmetic): score = (w2 . GELU(W1 h + b1) + b2) / temperature.
 // Used for float32 inputs, where the 1e-4 tolerance rules out TF32 tensor-core math.
 // TokenGate paper page (thelatestinai.com), Figure 1(b): a small scoring network scores
 // every hidden state at the selection layer.
@@ -17,7 +17,7 @@ __device__ __forceinline__ float ld_act(const __nv_bfloat16* p, int64_t i) { ret
 template <typename T, int DG>
 __global__ void __launch_bounds__(NT) score_simt_kernel(const T* __restrict__ H, int64_t ldh, int n_tok, int d,
                                                         const T* __restrict__ W1, const float* __restrict__ b1,
-                                                        const T* __restrict__ w2, float b2, float* __restrict__ score) {
+                                                        const T* __restrict__ w2, float b2, float inv_t, float* __restrict__ score) {
   constexpr int CPT = DG / 32;  // hidden units per thread
   __shared__ float hs[TM][TK + 1];
   __shared__ float ws[DG][TK + 1];
@@ -69,29 +69,30 @@ __global__ void __launch_bounds__(NT) score_simt_kernel(const T* __restrict__ H,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     int64_t t = tok0 + ty * 4 + i;
-    if (tx == 0 && t < n_tok) score[t] = part + b2;
+    if (tx == 0 && t < n_tok) score[t] = (part + b2) * inv_t;
   }
 }
 
 template <typename T>
 tg_status launch_t(const void* H, int64_t ldh, int64_t n_tok, int d, const void* W1, const float* b1,
-                   const void* w2, float b2, int dg, float* score, cudaStream_t st) {
+                   const void* w2, float b2, float inv_t, int dg, float* score, cudaStream_t st) {
   dim3 grid((unsigned)((n_tok + TM - 1) / TM));
   const T* h = static_cast<const T*>(H);
   const T* w = static_cast<const T*>(W1);
   const T* v = static_cast<const T*>(w2);
-  if (dg == 64) score_simt_kernel<T, 64><<<grid, NT, 0, st>>>(h, ldh, (int)n_tok, d, w, b1, v, b2, score);
-  else if (dg == 128) score_simt_kernel<T, 128><<<grid, NT, 0, st>>>(h, ldh, (int)n_tok, d, w, b1, v, b2, score);
-  else score_simt_kernel<T, 256><<<grid, NT, 0, st>>>(h, ldh, (int)n_tok, d, w, b1, v, b2, score);
+  if (dg == 64) score_simt_kernel<T, 64><<<grid, NT, 0, st>>>(h, ldh, (int)n_tok, d, w, b1, v, b2, inv_t, score);
+  else if (dg == 128) score_simt_kernel<T, 128><<<grid, NT, 0, st>>>(h, ldh, (int)n_tok, d, w, b1, v, b2, inv_t, score);
+  else score_simt_kernel<T, 256><<<grid, NT, 0, st>>>(h, ldh, (int)n_tok, d, w, b1, v, b2, inv_t, score);
   return cuda_status(cudaGetLastError(), "score_simt launch");
 }
 
 }  // namespace
 
 tg_status launch_score_simt(tg_dtype dt, const void* H, int64_t ldh, int64_t n_tok, int d, const void* W1,
-                            const float* b1, const void* w2, float b2, int dg, float* score, cudaStream_t st) {
-  if (dt == TG_BF16) return launch_t<__nv_bfloat16>(H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, st);
-  return launch_t<float>(H, ldh, n_tok, d, W1, b1, w2, b2, dg, score, st);
+                            const float* b1, const void* w2, float b2, float inv_t, int dg, float* score,
+                            cudaStream_t st) {
+  if (dt == TG_BF16) return launch_t<__nv_bfloat16>(H, ldh, n_tok, d, W1, b1, w2, b2, inv_t, dg, score, st);
+  return launch_t<float>(H, ldh, n_tok, d, W1, b1, w2, b2, inv_t, dg, score, st);
 }
 
 }  // namespace tg

@@ -51,15 +51,18 @@ def gelu(z):
     return 0.5 * z * (1.0 + erf(z / np.sqrt(2.0)))
 
 
-def gate_scores(H, W1, b1, w2, b2):
+def gate_scores(H, W1, b1, w2, b2, temperature=1.0):
     """One scalar importance score per token from its hidden state at layer L.
 
-    aitualizate.com article, phase 2 ("una pequeña red neuronal multicapa ... asigna una
-    puntuación individual a cada token"); thelatestinai.com page, Figure 1(b) ("scores each
-    hidden state with a small scoring network"). The network is d -> dg -> 1 with GELU:
-        s_i = w2 . GELU(W1 h_i + b1) + b2
+    aitualizate.com article, phase 2 (a small multilayer network gives every token its own
+    score); thelatestinai.com page, Figure 1(b) (a small scoring network scores each hidden
+    state). The network is d -> dg -> 1 with GELU:
+        s_i = (w2 . GELU(W1 h_i + b1) + b2) / temperature
     H: [n, d]; W1: [dg, d] (output-major, like nn.Linear); b1: [dg] or None; w2: [dg];
     b2: scalar. The hidden layer is kept at full precision (no rounding between layers).
+    The temperature is a reading: the thelatestinai.com page names a gate temperature in its
+    Figure 7 caption (Eq. 7) but prints no formula; here it divides the score, so the gate
+    value becomes sigmoid(s / temperature) and the selected set does not depend on it.
     """
     H = np.asarray(H, dtype=np.float64)
     W1 = np.asarray(W1, dtype=np.float64)
@@ -67,7 +70,7 @@ def gate_scores(H, W1, b1, w2, b2):
     z = H @ W1.T
     if b1 is not None:
         z = z + np.asarray(b1, dtype=np.float64)[None, :]
-    return gelu(z) @ w2 + float(b2)
+    return (gelu(z) @ w2 + float(b2)) / float(temperature)
 
 
 def gate_value(s):
@@ -99,9 +102,9 @@ def kept_count(n, q, k):
 def topk_select(s, seqlens, q_len, k):
     """Top-K over the context part of each packed sequence; the question tail is always kept.
 
-    aitualizate.com article, phase 2 ("un selector top-K conserva los K tokens con mayor
-    puntuación") and the restriction that only the document may be pruned ("la pregunta
-    nunca se elimina"); thelatestinai.com page, Figure 1(a) ("the gate module keeps K").
+    aitualizate.com article, phase 2 (a top-K selector keeps the K tokens with the highest
+    scores) and the restriction that only the document may be pruned (the question is never
+    removed); thelatestinai.com page, Figure 1(a) (the gate module keeps K tokens).
 
     Per sequence b (packed at offset start_b): the context positions are [0, N_b - q_b),
     the question tail is [N_b - q_b, N_b). The context is fully sorted by (score
@@ -138,8 +141,8 @@ def topk_select(s, seqlens, q_len, k):
 def gather(H, s, kept, seqlens, q_len, cu_kept, question_gate_one=False):
     """Kept hidden states with their gate values and original positions.
 
-    thelatestinai.com page, Figure 1(b) ("forwards the kept hidden states together with
-    their importance scores"); aitualizate.com article, phase 3 (layers above L receive only
+    thelatestinai.com page, Figure 1(b) (the kept hidden states travel on with their
+    importance scores); aitualizate.com article, phase 3 (layers above L receive only
     the kept tokens). pos is each kept row's index within its own sequence (the original
     position id the causal mask uses). With ``question_gate_one`` the question-tail rows get
     g = 1, log g = 0 instead of their own gate value.

@@ -82,15 +82,18 @@ def test_argument_errors_are_synchronous(L):
     V = ctypes.c_void_p
     fake = V(0x1000)  # never dereferenced: every call below fails validation first
     # tg_score: null H, bad dg, bad d, misaligned pointer
-    assert L.tg_score(1, None, 64, 10, 64, fake, None, fake, 0.0, 64, fake, None, None) == 1
-    assert L.tg_score(1, fake, 64, 10, 64, fake, None, fake, 0.0, 96, fake, None, None) == 2
-    assert L.tg_score(1, fake, 96, 10, 96, fake, None, fake, 0.0, 64, fake, None, None) == 2
-    assert L.tg_score(1, V(0x1002), 64, 10, 64, fake, None, fake, 0.0, 64, fake, None, None) == 2
-    assert L.tg_score(7, fake, 64, 10, 64, fake, None, fake, 0.0, 64, fake, None, None) == 1
-    assert L.tg_score(1, fake, 32, 10, 64, fake, None, fake, 0.0, 64, fake, None, None) == 1  # ldh < d
+    assert L.tg_score(1, None, 64, 10, 64, fake, None, fake, 0.0, 1.0, 64, fake, None, None) == 1
+    assert L.tg_score(1, fake, 64, 10, 64, fake, None, fake, 0.0, 1.0, 96, fake, None, None) == 2
+    assert L.tg_score(1, fake, 96, 10, 96, fake, None, fake, 0.0, 1.0, 64, fake, None, None) == 2
+    assert L.tg_score(1, V(0x1002), 64, 10, 64, fake, None, fake, 0.0, 1.0, 64, fake, None, None) == 2
+    assert L.tg_score(7, fake, 64, 10, 64, fake, None, fake, 0.0, 1.0, 64, fake, None, None) == 1
+    assert L.tg_score(1, fake, 32, 10, 64, fake, None, fake, 0.0, 1.0, 64, fake, None, None) == 1  # ldh < d
     assert b"dg" in L.tg_last_error() or b"ldh" in L.tg_last_error()
+    for bad_t in (0.0, -1.0, float("inf"), float("nan")):  # the temperature must be positive and finite
+        assert L.tg_score(1, fake, 64, 10, 64, fake, None, fake, 0.0, bad_t, 64, fake, None, None) == 1
+        assert b"temperature" in L.tg_last_error()
     # n_tok == 0 is a no-op that needs no device
-    assert L.tg_score(1, None, 64, 0, 64, None, None, None, 0.0, 64, None, None, None) == 0
+    assert L.tg_score(1, None, 64, 0, 64, None, None, None, 0.0, 1.0, 64, None, None, None) == 0
     # tg_topk_select: q > N, null outputs
     s = _seqs([10], [11], [2])
     assert L.tg_topk_select(fake, s.ref(), fake, None, None, None) == 1
@@ -122,7 +125,7 @@ def test_argument_errors_are_synchronous(L):
     # tg_prefill_above_L: missing outputs
     s = _seqs([10], [2], [2])
     arr = (V * 1)(fake.value)
-    assert L.tg_prefill_above_L(1, fake, 64, 64, fake, None, fake, 0.0, 64, s.ref(), 1, arr, arr, arr, 8, 4, 128,
+    assert L.tg_prefill_above_L(1, fake, 64, 64, fake, None, fake, 0.0, 1.0, 64, s.ref(), 1, arr, arr, arr, 8, 4, 128,
                                 0.1, None, 0, None, fake, None, fake, fake, fake, fake, arr, None, None, None) == 1
 
 

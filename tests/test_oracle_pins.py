@@ -555,3 +555,27 @@ def test_attention_closed_gate_is_a_removed_key_for_every_gain():
                                                  dO[2:], head_gain=gain)
     np.testing.assert_allclose(dQ[2:], dQr, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(dK[2:], dKr, rtol=1e-10, atol=1e-12)
+
+
+def test_score_temperature_golden_and_selection_invariance(golden_dir):
+    """The gate temperature (a reading: it divides the score) against the hand-derived one-hot
+    case, and the property that makes it a temperature: the kept set is the same for every
+    temperature > 0, while g = sigmoid(s / T) flattens towards 1/2 as T grows."""
+    fx = _load(golden_dir, "score_onehot.json")
+    tc = fx["temperature_case"]
+    s = orc.gate_scores(np.array(fx["H"]), np.array(fx["W1"]), np.array(fx["b1"]), np.array(fx["w2"]), fx["b2"],
+                        temperature=tc["temperature"])
+    np.testing.assert_allclose(s, tc["expected"], rtol=0, atol=tc["tolerance_abs"])
+    wl = ti.scaled(ti.WORKLOADS["tiny_f32"], seqlens=(300, 77), q_len=(20, 5), k=(40, 30))
+    H = ti.hidden_states(wl)
+    W1, b1, w2, b2 = ti.gate_weights(wl, biased=True)
+    base = orc.gate_scores(H, W1, b1, w2, b2)
+    kept1, _ = orc.topk_select(base, wl.seqlens, wl.q_len, wl.k)
+    spread = []
+    for T in (0.05, 0.7, 3.0, 40.0):
+        sT = orc.gate_scores(H, W1, b1, w2, b2, temperature=T)
+        keptT, _ = orc.topk_select(sT, wl.seqlens, wl.q_len, wl.k)
+        assert np.array_equal(keptT, kept1)
+        g, _ = orc.gate_value(sT)
+        spread.append(float(np.max(np.abs(g - 0.5))))
+    assert spread == sorted(spread, reverse=True) and spread[-1] < 0.05

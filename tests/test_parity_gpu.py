@@ -569,3 +569,34 @@ def test_benchmarked_chain_matches_oracle(name):
                                      wl.Hq, wl.Hkv, scale, rows=qrows)
         assert max_abs_rel(from_dev(out["O"][l])[qrows], rO) <= TOL["bf16"], l
         assert max_abs_rel(from_dev(out["lse"][l])[:, qrows], rL) <= TOL["bf16"], l
+
+
+@pytest.mark.parametrize("name,T", [("tiny_f32", 0.37), ("qwen3_8k", 2.5)])
+def test_score_temperature_and_chain(name, T):
+    """The gate temperature divides the score (g = sigmoid(s / T)): tg_score against the oracle
+    with the same temperature, and the chained prefill with it, whose kept set equals the one
+    at temperature 1 and whose gate values follow the divided scores."""
+    wl = ti.WORKLOADS[name]
+    if name == "qwen3_8k":
+        wl = ti.scaled(wl, seqlens=(3000,), q_len=(40,), k=(500,))
+    H = ti.hidden_states(wl)
+    W1, b1, w2, b2 = ti.gate_weights(wl, biased=True)
+    Hd, W1d, b1d, w2d = to_dev(H, wl.dtype), to_dev(W1, wl.dtype), to_dev(b1, "f32"), to_dev(w2, wl.dtype)
+    s = tg.tg_score(Hd, W1d, b1d, w2d, b2, temperature=T)
+    s1 = tg.tg_score(Hd, W1d, b1d, w2d, b2)
+    torch.cuda.synchronize()
+    ref = orc.gate_scores(ti.widen(H, wl.dtype), ti.widen(W1, wl.dtype), b1, ti.widen(w2, wl.dtype), b2, temperature=T)
+    assert max_abs_rel(from_dev(s), ref) <= TOL[wl.dtype]
+    M = tg.tg_kept_counts(wl.seqlens, wl.q_len, wl.k)[-1]
+    layers = [tuple(to_dev(x, wl.dtype) for x in (ti.qkv(wl, 0, M) if wl.dtype == "bf16" else
+                                                   ti.project_kept(wl, np.zeros((M, wl.d)))))]
+    st = _stat()
+    out = tg.tg_prefill_above_L(Hd, W1d, b1d, w2d, b2, wl.seqlens, wl.q_len, wl.k, layers, 1.0 / math.sqrt(wl.D),
+                                dev_status=st, temperature=T)
+    torch.cuda.synchronize()
+    kept1, _ = orc.topk_select(s1.cpu().numpy(), wl.seqlens, wl.q_len, wl.k)
+    assert np.array_equal(out["kept_idx"].cpu().numpy(), kept1.astype(np.int32))
+    sT = out["score"].cpu().numpy()
+    _, _, gref, _ = orc.gather(H, sT, kept1, wl.seqlens, wl.q_len, tg.tg_kept_counts(wl.seqlens, wl.q_len, wl.k))
+    assert max_abs_rel(from_dev(out["g"]), gref) <= 1e-6
+    assert st.item() == 0
