@@ -296,6 +296,37 @@ def gate_score_grad(dlogg, logg):
     return np.asarray(dlogg, np.float64) * -np.expm1(np.asarray(logg, np.float64))
 
 
+def gelu_grad(z):
+    """Derivative of the exact-erf GELU: d/dz [z Phi(z)] = Phi(z) + z phi(z), with Phi the standard
+    normal CDF and phi its density."""
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * (1.0 + erf(z / np.sqrt(2.0))) + z * np.exp(-0.5 * z * z) / np.sqrt(2.0 * np.pi)
+
+
+def gate_mlp_grad(H, W1, b1, w2, dscore, temperature=1.0):
+    """Gradients of the gate network's parameters from the score gradient of each row.
+
+    The last link of the end-to-end training path (thelatestinai.com page, Figure 1(c): the
+    gated attention lets the top-K selector learn; aitualizate.com article, section on how the
+    top-K selection is trained): with s_i = (w2 . GELU(W1 h_i + b1) + b2) / T (gate_scores) and
+    upstream gradients dscore_i (tg_gated_attn_bwd's d score, for the kept rows h_i), the
+    chain rule gives, per row, z = W1 h + b1, a = GELU(z), ds' = dscore / T, and
+        dw2 = sum_i ds'_i a_i,   db2 = sum_i ds'_i,
+        dz_i = ds'_i w2 * GELU'(z_i),   db1 = sum_i dz_i,   dW1 = sum_i dz_i h_i^T.
+    H: [M, d]; W1: [dg, d]; b1: [dg] or None; w2: [dg]; dscore: [M]. float64 throughout.
+    Returns (dW1 [dg, d], db1 [dg], dw2 [dg], db2 scalar).
+    """
+    H = np.asarray(H, dtype=np.float64)
+    W1 = np.asarray(W1, dtype=np.float64)
+    w2 = np.asarray(w2, dtype=np.float64).reshape(-1)
+    ds = np.asarray(dscore, dtype=np.float64).reshape(-1) / float(temperature)
+    z = H @ W1.T
+    if b1 is not None:
+        z = z + np.asarray(b1, dtype=np.float64)[None, :]
+    dz = ds[:, None] * w2[None, :] * gelu_grad(z)
+    return dz.T @ H, dz.sum(axis=0), gelu(z).T @ ds, float(ds.sum())
+
+
 def gated_attention_weights(q, Kmat, g, scale):
     """Figure 1(c) read literally for one query row: softmax weights times g_j, renormalised.
 

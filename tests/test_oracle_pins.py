@@ -579,3 +579,49 @@ def test_score_temperature_golden_and_selection_invariance(golden_dir):
         g, _ = orc.gate_value(sT)
         spread.append(float(np.max(np.abs(g - 0.5))))
     assert spread == sorted(spread, reverse=True) and spread[-1] < 0.05
+
+
+def test_gelu_grad_matches_central_differences():
+    z = np.linspace(-7, 7, 281)
+    h = 1e-6
+    fd = (orc.gelu(z + h) - orc.gelu(z - h)) / (2 * h)
+    np.testing.assert_allclose(orc.gelu_grad(z), fd, rtol=0, atol=1e-8)
+    assert orc.gelu_grad(0.0) == 0.5  # Phi(0) + 0
+
+
+def test_gate_mlp_grad_matches_central_differences_and_autograd():
+    """dW1, db1, dw2, db2 of L = sum_i dscore_i s_i against central differences of gate_scores
+    (every element of a small case with d != dg and a temperature) and torch autograd of a
+    direct torch statement of the score network (float64)."""
+    import torch
+    g = np.random.default_rng(12)
+    M, d, dg, T = 7, 5, 3, 1.7
+    H = g.standard_normal((M, d))
+    W1 = g.standard_normal((dg, d)) * 0.7
+    b1 = g.standard_normal(dg) * 0.3
+    w2 = g.standard_normal(dg)
+    b2 = 0.2
+    ds = g.standard_normal(M)
+    dW1, db1, dw2, db2 = orc.gate_mlp_grad(H, W1, b1, w2, ds, temperature=T)
+    loss = lambda W1_, b1_, w2_, b2_: float(ds @ orc.gate_scores(H, W1_, b1_, w2_, b2_, temperature=T))
+    h = 1e-6
+    for arr, grad, name in ((W1, dW1, "W1"), (b1, db1, "b1"), (w2, dw2, "w2")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            up, dn = arr.copy(), arr.copy()
+            up[idx] += h
+            dn[idx] -= h
+            args_up = {"W1": (up, b1, w2), "b1": (W1, up, w2), "w2": (W1, b1, up)}[name]
+            args_dn = {"W1": (dn, b1, w2), "b1": (W1, dn, w2), "w2": (W1, b1, dn)}[name]
+            fd[idx] = (loss(*args_up, b2) - loss(*args_dn, b2)) / (2 * h)
+        np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-8, err_msg=name)
+    assert abs(db2 - (loss(W1, b1, w2, b2 + h) - loss(W1, b1, w2, b2 - h)) / (2 * h)) < 1e-8
+    tH = torch.tensor(H)
+    tW = torch.tensor(W1, requires_grad=True)
+    tb = torch.tensor(b1, requires_grad=True)
+    tw = torch.tensor(w2, requires_grad=True)
+    tb2 = torch.tensor(b2, dtype=torch.float64, requires_grad=True)
+    s = (torch.nn.functional.gelu(tH @ tW.T + tb) @ tw + tb2) / T
+    (torch.tensor(ds) * s).sum().backward()
+    for t, r in ((tW, dW1), (tb, db1), (tw, dw2), (tb2, db2)):
+        np.testing.assert_allclose(t.grad.numpy(), r, rtol=1e-12, atol=1e-14)
