@@ -41,7 +41,7 @@ typedef enum {
   TG_OK = 0,
   TG_ERR_INVALID_ARG = 1,   /* null pointer, negative size, inconsistent sizes */
   TG_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes / alignment / GPU */
-  TG_ERR_WORKSPACE = 3,     /* reserved: no entry point needs a workspace */
+  TG_ERR_WORKSPACE = 3,     /* the workspace is missing, too small or misaligned */
   TG_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
   TG_ERR_DEVICE_CHECK = 5,  /* reserved for callers that map TG_DEV_* bits to a status */
   TG_ERR_DEVICE_TIMEOUT = 6 /* reserved for callers that map TG_DEV_TIMEOUT to a status */
@@ -83,7 +83,8 @@ const char* tg_last_error(void);
  * tg_gather, tg_gated_attn_fwd, tg_prefill_above_L and the helpers). 1.1 adds tg_qkv_rope,
  * tg_topk_candidates, tg_topk_merge and tg_gated_attn_bwd. 1.2 gives tg_score a device
  * status word (its last argument before the stream) and a temperature (after b2, also in
- * tg_prefill_above_L), and adds tg_set_test_wait_probe. */
+ * tg_prefill_above_L), and adds tg_set_test_wait_probe, tg_gate_mlp_bwd and its
+ * workspace query. */
 int32_t tg_version(void);
 
 /* Test hook for the bounded waits, off by default (limit_ns = 0). With limit_ns > 0, every
@@ -136,8 +137,7 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
  *   cu_kept_dev device int32 [B+1] (written) or NULL
  *   dev_status  device int32 [1] or NULL
  * No workspace is needed: per-sequence descriptors travel as kernel parameters and each
- * sequence's histogram lives in the shared memory of its thread-block cluster (so
- * TG_ERR_WORKSPACE is never returned).
+ * sequence's histogram lives in the shared memory of its thread-block cluster.
  * Supported: N_b - q_b <= TG_MAX_CTX. */
 tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
                          int32_t* cu_kept_dev, int32_t* dev_status, void* stream);
@@ -249,6 +249,33 @@ tg_status tg_gated_attn_bwd(tg_dtype dtype, const void* Q, const void* K, const 
                             int32_t D, float softmax_scale, uint32_t flags, const void* O,
                             const float* lse, const void* dO, float* dQ, float* dK, float* dV,
                             float* dlogg, float* dscore, int32_t* dev_status, void* stream);
+
+/* Workspace bytes tg_gate_mlp_bwd needs for M kept rows (0 when M <= 0 or the shape is
+ * unsupported). Host only; depends on the current device's SM count. */
+size_t tg_gate_mlp_bwd_workspace_size(int64_t M, int32_t d, int32_t dg);
+
+/* Gradients of the gate network's parameters from the score gradient of the kept rows: the last
+ * link of end-to-end selector training (thelatestinai.com TokenGate page, Figure 1(c): the
+ * gated attention lets the top-K selector learn; aitualizate.com article, section on training
+ * the top-K selection). With s = (w2 . GELU(W1 h + b1) + b2) / temperature (tg_score) and
+ * dscore from tg_gated_attn_bwd, per kept row h: z = W1 h + b1, ds' = dscore / temperature,
+ *   dw2 = sum ds' GELU(z),  db2 = sum ds',  u = ds' w2 * GELU'(z),  db1 = sum u,  dW1 = sum u h^T.
+ *   H_kept   device act [M, d] contiguous (tg_gather's output; rows the top-K dropped get no
+ *            gradient through the selection)
+ *   W1, b1, w2, temperature, dg: as given to tg_score (b1 may be NULL)
+ *   dscore   device f32 [M]
+ *   dW1      device f32 [dg, d] (written, required); db1, dw2 device f32 [dg] and db2 device f32
+ *            [1] (written, each may be NULL)
+ *   ws       device workspace of at least tg_gate_mlp_bwd_workspace_size(M, d, dg) bytes,
+ *            256-byte aligned (TG_ERR_WORKSPACE otherwise); owned by the caller, contents need
+ *            no initialisation and are overwritten
+ * Arithmetic is fp32 on the CUDA cores; results are deterministic (fixed reduction orders).
+ * M = 0 writes zero gradients. Supported: d % 64 == 0, dg % 64 == 0, 16-byte aligned H_kept,
+ * W1 and dW1. */
+tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W1,
+                          const float* b1, const void* w2, float temperature, int32_t dg,
+                          const float* dscore, float* dW1, float* db1, float* dw2, float* db2,
+                          void* ws, size_t ws_bytes, void* stream);
 
 /* The whole gated path above layer L (aitualizate.com TokenGate article, phases 2-3;
  * thelatestinai.com TokenGate page, Figure 1(a)): the results of tg_score -> tg_topk_select

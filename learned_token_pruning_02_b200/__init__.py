@@ -33,6 +33,8 @@ EXPORTS = (
     "tg_topk_merge",
     "tg_gated_attn_bwd",
     "tg_set_test_wait_probe",
+    "tg_gate_mlp_bwd_workspace_size",
+    "tg_gate_mlp_bwd",
 )
 
 
@@ -79,6 +81,11 @@ def lib() -> ctypes.CDLL:
     L.tg_kept_counts.argtypes = [_SEQP, ctypes.POINTER(_I32)]
     L.tg_score.restype = _I32
     L.tg_score.argtypes = [_I32, _VP, _I64, _I64, _I32, _VP, _VP, _VP, _F, _F, _I32, _VP, _VP, _VP]
+    L.tg_gate_mlp_bwd_workspace_size.restype = ctypes.c_size_t
+    L.tg_gate_mlp_bwd_workspace_size.argtypes = [_I64, _I32, _I32]
+    L.tg_gate_mlp_bwd.restype = _I32
+    L.tg_gate_mlp_bwd.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP, _VP, _VP, _VP, _VP,
+                                  ctypes.c_size_t, _VP]
     L.tg_set_test_wait_probe.restype = _I32
     L.tg_set_test_wait_probe.argtypes = [_I64]
     L.tg_topk_select.restype = _I32
@@ -372,6 +379,38 @@ def tg_gated_attn_bwd(Q, K, V, logg, pos, cu_kept, O, lse, dO, softmax_scale: fl
         float(softmax_scale), int(flags), _ptr(O), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dlogg),
         _ptr(dscore), _ptr(dev_status), _stream(stream)))
     return dQ, dK, dV, dlogg, dscore
+
+
+def tg_gate_mlp_bwd(H_kept, W1, b1, w2, dscore, temperature: float = 1.0, dW1=None, db1=None, dw2=None, db2=None,
+                    ws=None, stream=None):
+    """Gradients of the gate network's parameters from d score of the kept rows:
+    (dW1 [dg, d], db1 [dg], dw2 [dg], db2 [1]), all float32. ``ws`` is a uint8 device buffer of
+    at least tg_gate_mlp_bwd_workspace_size bytes (allocated here when not given)."""
+    _want(torch.float32, b1=b1, dscore=dscore, dW1=dW1, db1=db1, dw2=dw2, db2=db2)
+    M, d = H_kept.shape
+    dg = W1.shape[0]
+    _contig(H_kept=H_kept, W1=W1, w2=w2)
+    _shape("W1", W1, (dg, d))
+    _len_at_least("dscore", dscore, M)
+    if dW1 is not None:
+        _shape("dW1", dW1, (dg, d))
+    for name, t in (("b1", b1), ("db1", db1), ("dw2", dw2)):
+        if t is not None:
+            _shape(name, t, (dg,))
+    _cuda(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, ws)
+    dev = H_kept.device
+    f32 = torch.float32
+    dW1 = torch.empty(dg, d, device=dev, dtype=f32) if dW1 is None else dW1
+    db1 = torch.empty(dg, device=dev, dtype=f32) if db1 is None else db1
+    dw2 = torch.empty(dg, device=dev, dtype=f32) if dw2 is None else dw2
+    db2 = torch.empty(1, device=dev, dtype=f32) if db2 is None else db2
+    need = lib().tg_gate_mlp_bwd_workspace_size(M, d, dg)
+    if ws is None:
+        ws = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
+    _check("tg_gate_mlp_bwd", lib().tg_gate_mlp_bwd(
+        _dtype(H_kept), _ptr(H_kept), M, d, _ptr(W1), _ptr(b1), _ptr(w2), float(temperature), dg, _ptr(dscore),
+        _ptr(dW1), _ptr(db1), _ptr(dw2), _ptr(db2), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return dW1, db1, dw2, db2
 
 
 def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_scale, head_gain=None, flags=0,

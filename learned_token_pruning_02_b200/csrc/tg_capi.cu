@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "tg_attn_bwd.cuh"
+#include "tg_gate_bwd.cuh"
 #include "tg_internal.cuh"
 
 namespace tg {
@@ -403,6 +404,50 @@ tg_status tg_gated_attn_bwd(tg_dtype dtype, const void* Q, const void* K, const 
     if (st != TG_OK) return st;
   }
   return TG_OK;
+}
+
+static tg_status gate_bwd_check(tg_dtype dtype, int64_t M, int32_t d, int32_t dg, float temperature) {
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
+  if (M < 0 || d <= 0 || dg <= 0) return fail(TG_ERR_INVALID_ARG, "need M >= 0 and d, dg > 0");
+  if (M > INT32_MAX) return fail(TG_ERR_UNSUPPORTED, "M exceeds int32 indexing");
+  if (d % 64 || dg % 64) return fail(TG_ERR_UNSUPPORTED, "d and dg must be multiples of 64");
+  if (!(temperature > 0.f) || temperature == INFINITY)
+    return fail(TG_ERR_INVALID_ARG, "temperature must be positive and finite");
+  return TG_OK;
+}
+
+size_t tg_gate_mlp_bwd_workspace_size(int64_t M, int32_t d, int32_t dg) {
+  if (M <= 0 || d <= 0 || dg <= 0 || d % 64 || dg % 64) return 0;
+  return (size_t)gate_bwd_plan(M, d, dg, device_sm_count()).bytes;
+}
+
+tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W1,
+                          const float* b1, const void* w2, float temperature, int32_t dg, const float* dscore,
+                          float* dW1, float* db1, float* dw2, float* db2, void* ws, size_t ws_bytes,
+                          void* stream) {
+  g_err[0] = 0;
+  tg_status st = gate_bwd_check(dtype, M, d, dg, temperature);
+  if (st != TG_OK) return st;
+  if (!dW1) return fail(TG_ERR_INVALID_ARG, "dW1 is required");
+  if (M == 0) {  // no rows: every gradient is zero
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(dW1, 0, (size_t)dg * d * 4, s);
+    if (e == cudaSuccess && db1) e = cudaMemsetAsync(db1, 0, (size_t)dg * 4, s);
+    if (e == cudaSuccess && dw2) e = cudaMemsetAsync(dw2, 0, (size_t)dg * 4, s);
+    if (e == cudaSuccess && db2) e = cudaMemsetAsync(db2, 0, 4, s);
+    return cuda_status(e, "tg_gate_mlp_bwd: zeroing the gradients");
+  }
+  if (!H_kept || !W1 || !w2 || !dscore) return fail(TG_ERR_INVALID_ARG, "H_kept, W1, w2 and dscore are required");
+  if (!aligned16(H_kept) || !aligned16(W1) || !aligned16(dW1))
+    return fail(TG_ERR_UNSUPPORTED, "H_kept, W1 and dW1 must be 16-byte aligned");
+  const GateBwdPlan p = gate_bwd_plan(M, d, dg, device_sm_count());
+  if (!ws || ws_bytes < (size_t)p.bytes || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(TG_ERR_WORKSPACE, "the workspace needs %lld bytes at a 256-byte aligned address",
+                (long long)p.bytes);
+  st = check_device();
+  if (st != TG_OK) return st;
+  return launch_gate_bwd(dtype, H_kept, M, d, W1, b1, w2, (float)(1.0 / (double)temperature), dg, dscore, dW1, db1,
+                         dw2, db2, ws, p, (cudaStream_t)stream);
 }
 
 // The row copy of the chained prefill (the selector already wrote pos, g and log g): launched

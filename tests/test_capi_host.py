@@ -270,3 +270,28 @@ def test_binding_checks_backward_shapes():
         call(head_gain=torch.ones(Hq - 1, dtype=f32))
     with pytest.raises(ValueError, match="CUDA tensors only"):  # well-formed: stops at the device check
         call()
+
+
+def test_gate_mlp_bwd_arguments_and_workspace(L):
+    """tg_gate_mlp_bwd checks its shapes, temperature and workspace before any CUDA call."""
+    V = ctypes.c_void_p
+    fake, ws = V(0x1000), V(0x10000)
+    need = L.tg_gate_mlp_bwd_workspace_size(2176, 2048, 256)
+    assert need >= 2176 * 256 * 4
+    assert L.tg_gate_mlp_bwd_workspace_size(0, 2048, 256) == 0
+    assert L.tg_gate_mlp_bwd_workspace_size(100, 2000, 256) == 0  # d not a multiple of 64
+    args = lambda **kw: [kw.get(n, v) for n, v in (
+        ("dt", 1), ("H", fake), ("M", 2176), ("d", 2048), ("W1", fake), ("b1", None), ("w2", fake), ("T", 1.0),
+        ("dg", 256), ("ds", fake), ("dW1", fake), ("db1", None), ("dw2", None), ("db2", None), ("ws", ws),
+        ("wsb", need), ("stream", None))]
+    assert L.tg_gate_mlp_bwd(*args(d=2000)) == 2
+    assert L.tg_gate_mlp_bwd(*args(dg=100)) == 2
+    assert L.tg_gate_mlp_bwd(*args(T=0.0)) == 1
+    assert L.tg_gate_mlp_bwd(*args(dt=5)) == 1
+    assert L.tg_gate_mlp_bwd(*args(dW1=None)) == 1
+    assert L.tg_gate_mlp_bwd(*args(ds=None)) == 1
+    assert L.tg_gate_mlp_bwd(*args(H=V(0x1008))) == 2  # misaligned
+    assert L.tg_gate_mlp_bwd(*args(wsb=need - 1)) == 3
+    assert L.tg_gate_mlp_bwd(*args(ws=None)) == 3
+    assert L.tg_gate_mlp_bwd(*args(ws=V(0x10080))) == 3  # workspace not 256-byte aligned
+    assert b"workspace" in L.tg_last_error()
