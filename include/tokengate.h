@@ -84,7 +84,7 @@ const char* tg_last_error(void);
  * tg_topk_candidates, tg_topk_merge and tg_gated_attn_bwd. 1.2 gives tg_score a device
  * status word (its last argument before the stream) and a temperature (after b2, also in
  * tg_prefill_above_L), and adds tg_set_test_wait_probe, tg_gate_mlp_bwd and its
- * workspace query. */
+ * workspace query, and tg_prefill_projected. */
 int32_t tg_version(void);
 
 /* Test hook for the bounded waits, off by default (limit_ns = 0). With limit_ns > 0, every
@@ -297,6 +297,29 @@ tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t
                              int32_t* kept_idx, int32_t* cu_kept_dev, void* H_kept, int32_t* pos,
                              float* g, float* logg, void* const* O, float* const* lse,
                              int32_t* dev_status, void* stream);
+
+/* The gated path above layer L with each layer's own projections (aitualizate.com TokenGate
+ * article, phase 3: the layers above L work on the kept tokens only, at their original
+ * positions, and dropped tokens leave no key/value entries behind; thelatestinai.com TokenGate
+ * page, Figure 1(a)). tg_score -> tg_topk_select -> kept rows (H_kept) -> for each layer l:
+ * tg_qkv_rope(H_kept, W_qkv[l], pos, rope_theta) into Q[l], K_cache[l], V_cache[l] ->
+ * tg_gated_attn_fwd into O[l], lse[l]. K_cache[l] and V_cache[l] [sum M_b, Hkv, D] are the
+ * layer's key/value cache, holding the kept rows only. The pages print no projection; each
+ * layer here projects the same kept rows with its own matrix (the reading of tg_qkv_rope).
+ *   W_qkv, Q, K_cache, V_cache, O, lse: HOST arrays of n_layers device pointers (lse may be
+ *            NULL or hold NULL entries); shapes as in tg_qkv_rope and tg_gated_attn_fwd
+ *   the other arguments: as in tg_prefill_above_L (score, kept_idx, H_kept, pos, g, logg
+ *            required)
+ * bf16 only. Every output equals running those entry points one after another. No host
+ * synchronisation; the buffers of one layer must not alias another layer's or the chain's. */
+tg_status tg_prefill_projected(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const void* W1,
+                               const float* b1, const void* w2, float b2, float temperature, int32_t dg,
+                               const tg_seqs* seqs, int32_t n_layers, const void* const* W_qkv,
+                               float rope_theta, int32_t Hq, int32_t Hkv, int32_t D, float softmax_scale,
+                               const float* head_gain, uint32_t flags, float* score, int32_t* kept_idx,
+                               int32_t* cu_kept_dev, void* H_kept, int32_t* pos, float* g, float* logg,
+                               void* const* Q, void* const* K_cache, void* const* V_cache, void* const* O,
+                               float* const* lse, int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

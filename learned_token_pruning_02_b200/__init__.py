@@ -35,6 +35,7 @@ EXPORTS = (
     "tg_set_test_wait_probe",
     "tg_gate_mlp_bwd_workspace_size",
     "tg_gate_mlp_bwd",
+    "tg_prefill_projected",
 )
 
 
@@ -86,6 +87,12 @@ def lib() -> ctypes.CDLL:
     L.tg_gate_mlp_bwd.restype = _I32
     L.tg_gate_mlp_bwd.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP, _VP, _VP, _VP, _VP,
                                   ctypes.c_size_t, _VP]
+    L.tg_prefill_projected.restype = _I32
+    L.tg_prefill_projected.argtypes = [
+        _I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _F, _I32, _SEQP, _I32, ctypes.POINTER(_VP), _F,
+        _I32, _I32, _I32, _F, _VP, _U32, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+        ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP),
+        _VP, _VP]
     L.tg_set_test_wait_probe.restype = _I32
     L.tg_set_test_wait_probe.argtypes = [_I64]
     L.tg_topk_select.restype = _I32
@@ -457,6 +464,52 @@ def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_sca
         qa, ka, va, Hq, Hkv, D, float(softmax_scale), _ptr(head_gain), int(flags), _ptr(out["score"]),
         _ptr(out["kept_idx"]), _ptr(out["cu_kept_dev"]), _ptr(out["H_kept"]), _ptr(out["pos"]), _ptr(out["g"]),
         _ptr(out["logg"]), oa, la, _ptr(dev_status), _stream(stream)))
+    return out
+
+
+def tg_prefill_projected(H, W1, b1, w2, b2, seqlens, q_len, k, W_qkv, rope_theta, Hq, Hkv, D, softmax_scale,
+                         head_gain=None, flags=0, want_lse=False, out=None, dev_status=None, stream=None,
+                         temperature: float = 1.0):
+    """The gated path with each above-L layer's own projections: score -> top-K -> kept rows ->
+    per layer Q/K/V (rotary at original positions; K and V are the layer's kept-only cache) ->
+    gated attention. W_qkv: list of [(Hq + 2 Hkv) D, d] bf16 matrices. Returns a dict with score,
+    kept_idx, cu_kept_dev, H_kept, pos, g, logg and per-layer lists Q, K_cache, V_cache, O, lse."""
+    _want(torch.float32, b1=b1, head_gain=head_gain)
+    _want(torch.int32, dev_status=dev_status)
+    n_tok, d = H.shape
+    for i, W in enumerate(W_qkv):
+        _contig(**{f"W_qkv[{i}]": W})
+        _shape(f"W_qkv[{i}]", W, ((Hq + 2 * Hkv) * D, d))
+    _cuda(H, W1, b1, w2, head_gain, dev_status, *W_qkv)
+    s = Seqs(seqlens, q_len, k)
+    cu = tg_kept_counts(seqlens, q_len, k)
+    m = cu[-1]
+    dev = H.device
+    nl = len(W_qkv)
+    bf = torch.bfloat16
+    if out is None:
+        out = {
+            "score": torch.empty(n_tok, device=dev, dtype=torch.float32),
+            "kept_idx": torch.empty(m, device=dev, dtype=torch.int32),
+            "cu_kept_dev": torch.empty(s.B + 1, device=dev, dtype=torch.int32),
+            "H_kept": torch.empty(m, d, device=dev, dtype=H.dtype),
+            "pos": torch.empty(m, device=dev, dtype=torch.int32),
+            "g": torch.empty(m, device=dev, dtype=torch.float32),
+            "logg": torch.empty(m, device=dev, dtype=torch.float32),
+            "Q": [torch.empty(m, Hq, D, device=dev, dtype=bf) for _ in range(nl)],
+            "K_cache": [torch.empty(m, Hkv, D, device=dev, dtype=bf) for _ in range(nl)],
+            "V_cache": [torch.empty(m, Hkv, D, device=dev, dtype=bf) for _ in range(nl)],
+            "O": [torch.empty(m, Hq, D, device=dev, dtype=bf) for _ in range(nl)],
+            "lse": [torch.empty(Hq, m, device=dev, dtype=torch.float32) if want_lse else None for _ in range(nl)],
+        }
+    _check_out(out)
+    arr = lambda ts: (_VP * max(nl, 1))(*[(t.data_ptr() if t is not None else None) for t in ts])
+    _check("tg_prefill_projected", lib().tg_prefill_projected(
+        _dtype(H), _ptr(H), H.stride(0), d, _ptr(W1), _ptr(b1), _ptr(w2), float(b2), float(temperature), W1.shape[0],
+        s.ref(), nl, arr(W_qkv), float(rope_theta), Hq, Hkv, D, float(softmax_scale), _ptr(head_gain), int(flags),
+        _ptr(out["score"]), _ptr(out["kept_idx"]), _ptr(out["cu_kept_dev"]), _ptr(out["H_kept"]), _ptr(out["pos"]),
+        _ptr(out["g"]), _ptr(out["logg"]), arr(out["Q"]), arr(out["K_cache"]), arr(out["V_cache"]), arr(out["O"]),
+        arr(out["lse"]), _ptr(dev_status), _stream(stream)))
     return out
 
 

@@ -453,8 +453,9 @@ tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t
 // The row copy of the chained prefill (the selector already wrote pos, g and log g): launched
 // after the attention layers, which read nothing it writes, so its first launch starts copying
 // at once and waits for them only at its end.
-static tg_status gather_after(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const int32_t* kept_idx,
-                              const tg_seqs* seqs, void* H_kept, int32_t* dev_status, void* stream) {
+static tg_status gather_rows(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const int32_t* kept_idx,
+                             const tg_seqs* seqs, void* H_kept, int32_t* dev_status, void* stream,
+                             bool after_kernel_reads_nothing) {
   if (d <= 0 || ldh < d) return fail(TG_ERR_INVALID_ARG, "need d > 0 and ldh >= d");
   if (!aligned16(H) || !aligned16(H_kept) || (ldh * esize(dtype)) % 16 || (d * esize(dtype)) % 16)
     return fail(TG_ERR_UNSUPPORTED, "H/H_kept must be 16-byte aligned with 16-byte rows");
@@ -466,7 +467,7 @@ static tg_status gather_after(tg_dtype dtype, const void* H, int64_t ldh, int32_
     start += seqs->seqlens[b];
     off += m;
   }
-  bool first = true;
+  bool first = after_kernel_reads_nothing;
   for (int b0 = 0; b0 < seqs->B; b0 += kMaxSeqPerLaunch) {
     const int nb = seqs->B - b0 < kMaxSeqPerLaunch ? seqs->B - b0 : kMaxSeqPerLaunch;
     int m_chunk = 0;
@@ -524,7 +525,50 @@ tg_status tg_prefill_above_L(tg_dtype dtype, const void* H, int64_t ldh, int32_t
                    flags, O[l], lse ? lse[l] : nullptr, dev_status, stream, true);
     if (st != TG_OK) return st;
   }
-  return gather_after(dtype, H, ldh, d, kept_idx, seqs, H_kept, dev_status, stream);
+  return gather_rows(dtype, H, ldh, d, kept_idx, seqs, H_kept, dev_status, stream, true);
+}
+
+tg_status tg_prefill_projected(tg_dtype dtype, const void* H, int64_t ldh, int32_t d, const void* W1,
+                               const float* b1, const void* w2, float b2, float temperature, int32_t dg,
+                               const tg_seqs* seqs, int32_t n_layers, const void* const* W_qkv, float rope_theta,
+                               int32_t Hq, int32_t Hkv, int32_t D, float softmax_scale, const float* head_gain,
+                               uint32_t flags, float* score, int32_t* kept_idx, int32_t* cu_kept_dev, void* H_kept,
+                               int32_t* pos, float* g, float* logg, void* const* Q, void* const* K_cache,
+                               void* const* V_cache, void* const* O, float* const* lse, int32_t* dev_status,
+                               void* stream) {
+  g_err[0] = 0;
+  if (dtype != TG_BF16) return fail(TG_ERR_UNSUPPORTED, "tg_prefill_projected runs on bf16 only");
+  int64_t n_tot = 0, m_tot = 0;
+  tg_status st = check_seqs(seqs, &n_tot, &m_tot);
+  if (st != TG_OK) return st;
+  if (n_layers < 0) return fail(TG_ERR_INVALID_ARG, "n_layers < 0");
+  if (n_layers > 0 && (!W_qkv || !Q || !K_cache || !V_cache || !O))
+    return fail(TG_ERR_INVALID_ARG, "W_qkv, Q, K_cache, V_cache and O arrays are required");
+  if (m_tot > 0 && (!score || !kept_idx || !H_kept || !pos || !g || !logg))
+    return fail(TG_ERR_INVALID_ARG, "score, kept_idx, H_kept, pos, g and logg are required");
+  if (!(rope_theta == rope_theta)) return fail(TG_ERR_INVALID_ARG, "rope_theta is NaN");
+  for (int l = 0; l < n_layers; ++l)
+    if (!W_qkv[l] || !Q[l] || !K_cache[l] || !V_cache[l] || !O[l])
+      return fail(TG_ERR_INVALID_ARG, "layer %d: W_qkv, Q, K_cache, V_cache and O are required", l);
+  std::vector<int32_t> cu(seqs->B + 1);
+  st = tg_kept_counts(seqs, cu.data());
+  if (st != TG_OK) return st;
+  st = tg_score(dtype, H, ldh, n_tot, d, W1, b1, w2, b2, temperature, dg, score, dev_status, stream);
+  if (st != TG_OK) return st;
+  // the selector writes pos, g and log g; the row copy follows it (the projections read H_kept)
+  st = select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, pos, g, logg, flags);
+  if (st != TG_OK || m_tot == 0) return st;
+  st = gather_rows(dtype, H, ldh, d, kept_idx, seqs, H_kept, dev_status, stream, false);
+  if (st != TG_OK) return st;
+  for (int l = 0; l < n_layers; ++l) {
+    st = tg_qkv_rope(dtype, H_kept, m_tot, d, W_qkv[l], pos, Hq, Hkv, D, rope_theta, Q[l], K_cache[l], V_cache[l],
+                     dev_status, stream);
+    if (st != TG_OK) return st;
+    st = attn_impl(dtype, Q[l], K_cache[l], V_cache[l], logg, head_gain, pos, cu.data(), seqs->B, Hq, Hkv, D,
+                   softmax_scale, flags, O[l], lse ? lse[l] : nullptr, dev_status, stream, false);
+    if (st != TG_OK) return st;
+  }
+  return TG_OK;
 }
 
 }  // extern "C"

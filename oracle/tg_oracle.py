@@ -399,3 +399,25 @@ def qkv_rope(Hk, W, pos, Hq, Hkv, D, theta):
     K = X[:, Hq * D: (Hq + Hkv) * D].reshape(M, Hkv, D)
     V = X[:, (Hq + Hkv) * D:].reshape(M, Hkv, D)
     return rope(Q, pos, theta), rope(K, pos, theta), V
+
+
+def prefill_projected(H, W1, b1, w2, b2, seqlens, q_len, k, W_qkv, theta, Hq, Hkv, D, scale,
+                      head_gain=None, temperature=1.0):
+    """The gated path above layer L with each layer's own projections of the kept rows:
+    score -> top-K (+question tail) -> kept rows -> per layer qkv_rope -> gated attention.
+
+    aitualizate.com article, phase 3 (the layers above L work on the kept tokens only, at their
+    original positions, and keep no key/value entries for dropped tokens); thelatestinai.com
+    page, Figure 1(a). Returns the intermediates and, per layer, (Q, K, V, O, LSE); K and V of a
+    layer are its key/value cache, kept rows only.
+    """
+    s = gate_scores(H, W1, b1, w2, b2, temperature)
+    kept, cu = topk_select(s, seqlens, q_len, k)
+    Hk, pos, g, logg = gather(H, s, kept, seqlens, q_len, cu)
+    layers = []
+    for W in W_qkv:
+        Q, K, V = qkv_rope(Hk, W, pos, Hq, Hkv, D, theta)
+        O, L = gated_attention(Q, K, V, logg, pos, cu, Hq, Hkv, scale, head_gain)
+        layers.append((Q, K, V, O, L))
+    return {"score": s, "kept": kept, "cu_kept": cu, "H_kept": Hk, "pos": pos, "g": g, "logg": logg,
+            "layers": layers}

@@ -625,3 +625,32 @@ def test_gate_mlp_grad_matches_central_differences_and_autograd():
     (torch.tensor(ds) * s).sum().backward()
     for t, r in ((tW, dW1), (tb, db1), (tw, dw2), (tb2, db2)):
         np.testing.assert_allclose(t.grad.numpy(), r, rtol=1e-12, atol=1e-14)
+
+
+def test_prefill_projected_is_the_composition_of_its_steps():
+    """The projected chain is the selection path followed, per layer, by the projection of the
+    kept rows and attention over them: K/V of dropped tokens never exist (a perturbed dropped row
+    changes nothing), and the layer outputs equal qkv_rope + gated_attention on the kept rows."""
+    wl = ti.scaled(ti.WORKLOADS["tiny_f32"], seqlens=(80, 50), q_len=(8, 4), k=(20, 9))
+    H = ti.hidden_states(wl).astype(np.float64)
+    W1, b1, w2, b2 = ti.gate_weights(wl, biased=True)
+    g = np.random.default_rng(2)
+    Ws = [g.standard_normal(((wl.Hq + 2 * wl.Hkv) * wl.D, wl.d)) / math.sqrt(wl.d) for _ in range(2)]
+    r = orc.prefill_projected(H, W1, b1, w2, b2, wl.seqlens, wl.q_len, wl.k, Ws, 1e4, wl.Hq, wl.Hkv, wl.D, 0.125)
+    for W, (Q, K, V, O, L) in zip(Ws, r["layers"]):
+        Q2, K2, V2 = orc.qkv_rope(H[r["kept"]], W, r["pos"], wl.Hq, wl.Hkv, wl.D, 1e4)
+        np.testing.assert_array_equal(K, K2)
+        O2, _ = orc.gated_attention(Q2, K2, V2, r["logg"], r["pos"], r["cu_kept"], wl.Hq, wl.Hkv, 0.125)
+        np.testing.assert_allclose(O, O2, rtol=0, atol=1e-14)
+    dropped = np.setdiff1d(np.arange(sum(wl.seqlens)), r["kept"])
+    H2 = H.copy()
+    H2[dropped[:5]] += 0.0  # same scores: perturb only rows whose scores stay below the threshold
+    s = orc.gate_scores(H, W1, b1, w2, b2)
+    order = np.argsort(s[dropped])[:3]  # the lowest-scoring dropped rows, pushed further down
+    H2 = H.copy()
+    for i in dropped[order]:
+        H2[i] = H[i] * 0.5
+    r2 = orc.prefill_projected(H2, W1, b1, w2, b2, wl.seqlens, wl.q_len, wl.k, Ws, 1e4, wl.Hq, wl.Hkv, wl.D, 0.125)
+    if np.array_equal(r2["kept"], r["kept"]):
+        for a, b in zip(r["layers"], r2["layers"]):
+            np.testing.assert_array_equal(a[3], b[3])
