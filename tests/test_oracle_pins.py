@@ -643,8 +643,6 @@ def test_prefill_projected_is_the_composition_of_its_steps():
         O2, _ = orc.gated_attention(Q2, K2, V2, r["logg"], r["pos"], r["cu_kept"], wl.Hq, wl.Hkv, 0.125)
         np.testing.assert_allclose(O, O2, rtol=0, atol=1e-14)
     dropped = np.setdiff1d(np.arange(sum(wl.seqlens)), r["kept"])
-    H2 = H.copy()
-    H2[dropped[:5]] += 0.0  # same scores: perturb only rows whose scores stay below the threshold
     s = orc.gate_scores(H, W1, b1, w2, b2)
     order = np.argsort(s[dropped])[:3]  # the lowest-scoring dropped rows, pushed further down
     H2 = H.copy()
