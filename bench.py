@@ -325,6 +325,63 @@ def attn_bwd_time(tg, torch, dev, Q, K, V, logg, pos, cu, scale, peak_tflops, re
             "note": "warp-level mma.sync m16n8k16 kernels (dK/dV per 64-key tile, dQ per 64-query tile)"}
 
 
+def projected_chain_time(tg, torch, dev, cb, flush, reps):
+    """The path with the above-L layer's own projection (tg_prefill_projected): score, top-K, kept
+    rows, Q/K/V with rotary embedding at original positions into a kept-only K/V cache (a seeded
+    N(0, 1/d) stacked projection, theta 1e6), gated attention; L2 flushed before each step."""
+    wl = cb.wl
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20264)
+    W = (torch.randn((wl.Hq + 2 * wl.Hkv) * wl.D, wl.d, device=dev, generator=gen) / wl.d ** 0.5).to(torch.bfloat16)
+    run = lambda o: tg.tg_prefill_projected(cb.H, cb.W1, cb.b1, cb.w2, cb.b2, wl.seqlens, wl.q_len, wl.k, [W], 1.0e6,
+                                            wl.Hq, wl.Hkv, wl.D, cb.scale, out=o)
+    out = run(None)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ts = []
+    for _ in range(reps):
+        flush()
+        torch.cuda._sleep(200_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run(out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = sum(ts) / len(ts)
+    return {"value": wl.n_tok / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "note": "score + select + kept-row copy + Q/K/V projection with rotary embedding + gated attention, "
+                    "one above-L layer, through tg_prefill_projected (bound Python call per step)"}
+
+
+def gate_bwd_time(tg, torch, dev, cb, reps):
+    """Gradients of the gate network from d score of the bench workload's kept rows (seeded
+    N(0, 0.01) d score): two fp32 CUDA-core GEMM passes (recompute z, then u^T H) and a reduction."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20265)
+    Hk = cb.out["H_kept"]
+    M, d = Hk.shape
+    dg = cb.W1.shape[0]
+    ds = torch.randn(M, device=dev, generator=gen) * 0.01
+    bufs = dict(dW1=torch.empty(dg, d, device=dev), db1=torch.empty(dg, device=dev), dw2=torch.empty(dg, device=dev),
+                db2=torch.empty(1, device=dev),
+                ws=torch.empty(tg.lib().tg_gate_mlp_bwd_workspace_size(M, d, dg), device=dev, dtype=torch.uint8))
+    run = lambda: tg.tg_gate_mlp_bwd(Hk, cb.W1, cb.b1, cb.w2, ds, **bufs)
+    run()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / reps / 1e3
+    flops = 4.0 * M * d * dg
+    return {"shape": f"M={M} kept rows, d={d}, dg={dg}", "us": t * 1e6, "tflops": flops / t / 1e12,
+            "note": "fp32 CUDA-core kernels (z recomputed, then dW1 = u^T H over row splits), back to back, L2 warm"}
+
+
 def split_select_times(tg, torch, dev, reps):
     """The sequence-split selection's two device steps for one 131072-token sequence cut into 8
     blocks, K=4096: one rank's top-k candidates of its 16352-token block, and the merge of the
@@ -743,6 +800,9 @@ def main():
     bwd_t = (attn_bwd_time(tg, torch, dev, *layers[0], out["logg"], out["pos"], list(cu), scale, pk["bf16_tflops"], 5)
              if not args.no_bw else None)
 
+    proj_t = projected_chain_time(tg, torch, dev, cb, flush, 20) if not args.no_bw else None
+    gbwd_t = gate_bwd_time(tg, torch, dev, cb, 20) if not args.no_bw else None
+
     # ---------------- the other configurations, through the same entry point (rank 0)
     others = None
     if rank == 0 and not args.no_other:
@@ -783,6 +843,8 @@ def main():
             "split_select": split_t,
             "qkv_rope": qkv_t,
             "gated_attn_bwd": bwd_t,
+            "projected_chain": proj_t,
+            "gate_mlp_bwd": gbwd_t,
             "device_status": dev_status,
         }
         print(json.dumps(line), flush=True)
