@@ -89,10 +89,10 @@ struct Cfg {
 
 template <int DG>
 __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
-    score_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmHt,
-                    const __grid_constant__ CUtensorMap tmW, const float* __restrict__ b1,
-                    const __nv_bfloat16* __restrict__ w2, float b2, float inv_t, float* __restrict__ score, int n_tok, int nk,
-                    int rows_cta, int tail_rows, int32_t* __restrict__ dev_status, uint64_t probe_ns) {
+    score_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW,
+                    const float* __restrict__ b1, const __nv_bfloat16* __restrict__ w2, float b2, float inv_t,
+                    float* __restrict__ score, int n_tok, int nk, int n_tiles, int32_t* __restrict__ dev_status,
+                    uint64_t probe_ns) {
   using C = Cfg<DG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -137,7 +137,6 @@ __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmH);
-    prefetch_tmap(&tmHt);
     prefetch_tmap(&tmW);
   }
   if (warp == 1) {
@@ -158,14 +157,6 @@ __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int kb0 = (int)(((long)blockIdx.x * nk) / gridDim.x);  // first K slice of this CTA
-  // This CTA's rows: one contiguous run [r0, r0 + rows_cta) (the same length for every CTA but
-  // the last), so each SM streams the same number of H bytes. The run is cut into 128-row tiles;
-  // a shorter last tile (tail_rows) is loaded with its own box height (tmHt) and the
-  // accumulator rows past it are computed from stale shared memory and discarded.
-  const int r0 = blockIdx.x * rows_cta;
-  const int my_rows = min(rows_cta, n_tok - r0);
-  const int n_full = rows_cta / BM;
-  const int my_tiles = min(n_full + (tail_rows > 0 ? 1 : 0), (my_rows + BM - 1) / BM);
   const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
 
   if (skip) {
@@ -181,16 +172,13 @@ __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
-      for (int tile = 0; tile < my_tiles && !*abort; ++tile) {
-        const int y = is_h ? r0 + tile * BM : 0;
-        const bool part = is_h && tile == n_full;  // the short last tile of the run
-        const CUtensorMap* tmt = part ? &tmHt : tm;
-        const int tbytes = part ? tail_rows * BK * 2 : bytes;
+      for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
+        const int y = is_h ? tile * BM : 0;
         for (int i = 0; i < nk; ++i) {
           const int kb = (i + kb0) % nk;
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, dev_status)) break;
-          mbar_arrive_expect_tx(&full[stage], tbytes);
-          tma_load_2d(ring + stage * bytes, tmt, kb * BK, y, &full[stage]);
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(ring + stage * bytes, tm, kb * BK, y, &full[stage]);
           ++issued;
           if (++stage == depth) {
             stage = 0;
@@ -213,7 +201,7 @@ __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
       int hs = 0, ws = 0;
       uint32_t hph = 0, wph = 0;
       int it = 0;
-      for (int tile = 0; tile < my_tiles && !*abort; ++tile, ++it) {
+      for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         if (!mbar_wait(&acce[acc], ((it >> 1) & 1) ^ 1u, abort, dev_status)) break;
         tc_fence_after();
@@ -253,7 +241,7 @@ __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
     const int row = q * 32 + lane;
     const int c_lo = grp * C::CW;
     int it = 0;
-    for (int tile = 0; tile < my_tiles; ++tile, ++it) {
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       // warp-uniform: the tcgen05.ld below is warp-collective
       if (!__all_sync(0xffffffffu, mbar_wait(&accf[acc], (it >> 1) & 1, abort, dev_status))) break;
@@ -281,11 +269,10 @@ __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
         mbar_arrive(&half_ready[acc]);
       } else {
         ok = __all_sync(0xffffffffu, mbar_wait(&half_ready[acc], (it >> 1) & 1, abort, dev_status));
-        const int rl = tile * BM + row;  // row within this CTA's run
-        const long r = (long)r0 + rl;
+        const long r = (long)tile * BM + row;
 #pragma unroll
         for (int g = 1; g < C::NGRP; ++g) s += part[((g - 1) * 2 + acc) * BM + row];
-        if (ok && rl < my_rows) score[r] = (s + b2) * inv_t;
+        if (ok && r < n_tok) score[r] = (s + b2) * inv_t;
       }
       // the accumulator (and this buffer's partial sums) is released only once fully consumed
       __syncwarp();
@@ -310,17 +297,8 @@ template <int DG>
 tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void* W1, const float* b1, const void* w2,
                     float b2, float inv_t, float* score, int32_t* dev_status, cudaStream_t st) {
   using C = Cfg<DG>;
-  // Rows per CTA: the n_tok rows cut into equal contiguous runs, one per CTA (at most one CTA
-  // per SM and per 128 rows), so every SM streams the same number of H bytes.
-  const int sms = device_sm_count();
-  const int64_t tiles = (n_tok + BM - 1) / BM;
-  int ctas = (int)(tiles < sms ? tiles : sms);
-  const int rows_cta = (int)((n_tok + ctas - 1) / ctas);
-  ctas = (int)((n_tok + rows_cta - 1) / rows_cta);
-  const int tail_rows = rows_cta % BM;
-  CUtensorMap tmH, tmHt, tmW;
+  CUtensorMap tmH, tmW;
   if (!make_tmap_bf16_2d(&tmH, H, (uint64_t)n_tok, (uint64_t)d, (uint64_t)ldh, BM, BK) ||
-      !make_tmap_bf16_2d(&tmHt, H, (uint64_t)n_tok, (uint64_t)d, (uint64_t)ldh, tail_rows > 0 ? tail_rows : BM, BK) ||
       !make_tmap_bf16_2d(&tmW, W1, (uint64_t)DG, (uint64_t)d, (uint64_t)d, DG, BK))
     return fail(TG_ERR_CUDA, "tg_score: building the TMA tensor maps failed");
   constexpr int slot = DG == 64 ? ATTR_SCORE64 : (DG == 128 ? ATTR_SCORE128 : ATTR_SCORE256);
@@ -334,6 +312,9 @@ tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void
     if (e != cudaSuccess) return cuda_status(e, "tg_score: cudaFuncSetAttribute");
     mark_attrs_set(slot);
   }
+  const int n_tiles = (int)((n_tok + BM - 1) / BM);
+  int ctas = device_sm_count();
+  if (ctas > n_tiles) ctas = n_tiles;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)ctas);
   cfg.blockDim = dim3(C::NTHREADS);
@@ -342,9 +323,9 @@ tg_status launch_dg(const void* H, int64_t ldh, int64_t n_tok, int d, const void
   cudaLaunchAttribute attr[1] = {pdl_attribute(PDL_SCORE)};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, score_tc_kernel<DG>, tmH, tmHt, tmW, b1,
+  return cuda_status(cudaLaunchKernelEx(&cfg, score_tc_kernel<DG>, tmH, tmW, b1,
                                         static_cast<const __nv_bfloat16*>(w2), b2, inv_t, score, (int)n_tok, d / BK,
-                                        rows_cta, tail_rows, dev_status, wait_probe_ns()),
+                                        n_tiles, dev_status, wait_probe_ns()),
                      "tg_score: score_tc launch");
 }
 
