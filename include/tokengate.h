@@ -277,6 +277,31 @@ tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t
                           const float* dscore, float* dW1, float* db1, float* dw2, float* db2,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the fixed device scratch array behind tg_gate_mlp_bwd_noalloc (16 MiB). */
+#define TG_GATE_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* tg_gate_mlp_bwd for callers that cannot allocate device memory. The pages have no counterpart
+ * of this entry point; it exists for callers such as a serving or training runtime that plans
+ * all device memory up front and forbids allocations once it runs, a plugin hosted by a
+ * framework whose allocator it cannot reach, or a latency-critical loop where cudaMalloc (which
+ * may synchronise the device) is not allowed. The arguments and results are those of
+ * tg_gate_mlp_bwd without ws / ws_bytes: the working memory is a fixed array of
+ * TG_GATE_NOALLOC_SCRATCH_BYTES inside this library, which every GPU that loads the library
+ * holds until the process exits. Nothing here calls cudaMalloc, cudaFree or any allocating
+ * routine.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress
+ *     with that device current); make that first call before any stream capture.
+ *   - Shapes whose working memory exceeds the array (tg_gate_mlp_bwd_workspace_size(M, d, dg) >
+ *     TG_GATE_NOALLOC_SCRATCH_BYTES; at d = 2048, dg = 256 that is well above 4096 kept rows)
+ *     return TG_ERR_UNSUPPORTED before anything is launched.
+ *   - Every call on a device shares the one array, which keeps the last call's contents; no part
+ *     of it needs clearing (each call writes every byte it reads). Calls whose GPU work overlaps
+ *     (different streams, or a stream that does not order them) race on the array: order them. */
+tg_status tg_gate_mlp_bwd_noalloc(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d,
+                                  const void* W1, const float* b1, const void* w2, float temperature,
+                                  int32_t dg, const float* dscore, float* dW1, float* db1,
+                                  float* dw2, float* db2, void* stream);
+
 /* The whole gated path above layer L (aitualizate.com TokenGate article, phases 2-3;
  * thelatestinai.com TokenGate page, Figure 1(a)): the results of tg_score -> tg_topk_select
  * -> tg_gather -> tg_gated_attn_fwd for each of n_layers above-L layers, enqueued on one

@@ -36,6 +36,7 @@ EXPORTS = (
     "tg_gate_mlp_bwd_workspace_size",
     "tg_gate_mlp_bwd",
     "tg_prefill_projected",
+    "tg_gate_mlp_bwd_noalloc",
 )
 
 
@@ -93,6 +94,9 @@ def lib() -> ctypes.CDLL:
         _I32, _I32, _I32, _F, _VP, _U32, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
         ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP),
         _VP, _VP]
+    L.tg_gate_mlp_bwd_noalloc.restype = _I32
+    L.tg_gate_mlp_bwd_noalloc.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP, _VP, _VP, _VP,
+                                          _VP]
     L.tg_set_test_wait_probe.restype = _I32
     L.tg_set_test_wait_probe.argtypes = [_I64]
     L.tg_topk_select.restype = _I32
@@ -417,6 +421,24 @@ def tg_gate_mlp_bwd(H_kept, W1, b1, w2, dscore, temperature: float = 1.0, dW1=No
     _check("tg_gate_mlp_bwd", lib().tg_gate_mlp_bwd(
         _dtype(H_kept), _ptr(H_kept), M, d, _ptr(W1), _ptr(b1), _ptr(w2), float(temperature), dg, _ptr(dscore),
         _ptr(dW1), _ptr(db1), _ptr(dw2), _ptr(db2), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return dW1, db1, dw2, db2
+
+
+def tg_gate_mlp_bwd_noalloc(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, temperature: float = 1.0, stream=None):
+    """tg_gate_mlp_bwd for callers that cannot allocate: the library's fixed scratch array takes
+    the place of the workspace, and every output buffer is the caller's (nothing is allocated
+    here either). Calls on one device share the array: do not let them overlap on the GPU."""
+    _want(torch.float32, b1=b1, dscore=dscore, dW1=dW1, db1=db1, dw2=dw2, db2=db2)
+    M, d = H_kept.shape
+    dg = W1.shape[0]
+    _contig(H_kept=H_kept, W1=W1, w2=w2)
+    _shape("W1", W1, (dg, d))
+    _shape("dW1", dW1, (dg, d))
+    _len_at_least("dscore", dscore, M)
+    _cuda(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2)
+    _check("tg_gate_mlp_bwd_noalloc", lib().tg_gate_mlp_bwd_noalloc(
+        _dtype(H_kept), _ptr(H_kept), M, d, _ptr(W1), _ptr(b1), _ptr(w2), float(temperature), dg, _ptr(dscore),
+        _ptr(dW1), _ptr(db1), _ptr(dw2), _ptr(db2), _stream(stream)))
     return dW1, db1, dw2, db2
 
 

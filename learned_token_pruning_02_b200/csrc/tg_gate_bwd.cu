@@ -18,6 +18,8 @@
 //   * reduce: sums the partial blocks, the tile column sums and ds' in a fixed order.
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "tg_gate_bwd.cuh"
 
 namespace tg {
@@ -203,7 +205,30 @@ __global__ void __launch_bounds__(NT) gate_bwd_reduce_kernel(const float* __rest
 
 int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
+// Scratch of tg_gate_mlp_bwd_noalloc: a fixed device array of this library, present on every GPU
+// that loads it until the process exits, shared by every call of that entry point on the device.
+static __device__ __align__(256) unsigned char g_gate_scratch[TG_GATE_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_gate_scratch per device (the array's name in host code is only a host
+// stand-in for the symbol, never a device address), looked up on a device's first call.
+std::atomic<void*> g_gate_scratch_addr[64];
+
 }  // namespace
+
+tg_status gate_bwd_fixed_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "tg_gate_mlp_bwd_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(TG_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  void* p = g_gate_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    e = cudaGetSymbolAddress(&p, g_gate_scratch);  // the current device is `dev`
+    if (e != cudaSuccess) return cuda_status(e, "tg_gate_mlp_bwd_noalloc: cudaGetSymbolAddress of the scratch");
+    g_gate_scratch_addr[dev].store(p, std::memory_order_release);
+  }
+  *ptr = p;
+  return TG_OK;
+}
 
 GateBwdPlan gate_bwd_plan(int64_t M, int d, int dg, int sms) {
   GateBwdPlan p;
