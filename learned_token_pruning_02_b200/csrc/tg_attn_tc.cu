@@ -103,7 +103,7 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 }
 
 // Which pairs of a 128-key row take the FMA-pipe exponential: kPolyOf8 of every 8 pairs.
-constexpr int kPolyOf8 = 3;
+constexpr int kPolyOf8 = 0;
 
 // Work item w of the longest-first list: query tile t of sequence b, query head h. Items are
 // ordered by the length of their causal key range (tile index) descending, sequences in order
@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* probe = bars + 21;   // test hook: a barrier nothing signals
   uint64_t* qempty = bars + 22;  // the item's last S product read Q: the next Q may load
   uint64_t* oempty = bars + 23;  // the item's merge read both O accumulators: the next PV may write
+  uint64_t* phalf = bars + 26;   // [2] the first 64 keys of the chain's P are in TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* bias_s = reinterpret_cast<float*>(tail + 256);  // [2][128]
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bfull[s], 32);
       mbar_init(&sfull[s], 1);
       mbar_init(&pready[s], 128);
+      mbar_init(&phalf[s], 128);
       mbar_init(&pvdone[s], 1);
     }
     mbar_init(mlready, 256);
@@ -233,6 +235,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
 
+  if (warp < 4) {
+  regs_dec<64>();
   if (skip) {
   } else if (warp == 0) {  // ------------------------------------------ Q and K producer
     if (lane == 0) {
@@ -373,7 +377,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (ok && nt <= 2) mma_commit(qempty);  // every S product of the item is issued
         for (int j = 0; ok && j < nt; ++j) {
           const int c = j & 1;
-          if (!mbar_wait(&pready[c], pc[c] & 1, abort, dev_status) ||
+          if (!mbar_wait(&phalf[c], pc[c] & 1, abort, dev_status) ||
               !mbar_wait(&vfull[c], pc[c] & 1, abort, dev_status) ||
               (j == 0 && k > 0 && !mbar_wait(oempty, (k - 1) & 1, abort, dev_status))) {
             ok = false;
@@ -382,9 +386,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tc_fence_after();
           const uint32_t va = smem_u32(smem + C::V_OFF + c * C::TILE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk)
+          for (int kk = 0; kk < BKV / 32; ++kk)  // keys 0-63: their P is in TMEM
             mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
                    C::IDESC_PV, (j >= 2 || kk > 0) ? 1u : 0u);
+          if (!mbar_wait(&pready[c], pc[c] & 1, abort, dev_status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = BKV / 32; kk < BKV / 16; ++kk)  // keys 64-127
+            mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
+                   C::IDESC_PV, 1u);
           mma_commit(&pvdone[c]);
           mma_commit(&vempty[c]);
           ++pc[c];
@@ -399,7 +412,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {
       }
     }
-  } else {  // ------------------------------------------------------------ softmax warpgroups
+  }
+  } else if (!skip) {  // ----------------------------------------------------- softmax warpgroups
+    regs_inc<216>();
     const int c = (warp - 4) >> 2;  // chain: 0 = warps 4-7 (even tiles), 1 = warps 8-11 (odd tiles)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // query row in the tile == TMEM lane
@@ -471,6 +486,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_cand);  // 0 on the chain's first tile
           m_run = m_cand;
         }
+        if (resc && u > 0) {  // rescale the chain's O once its previous PV product has landed
+          if (!__all_sync(0xffffffffu, mbar_wait(&pvdone[c], (nc - 1) & 1, abort, dev_status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + c0, o);
+          }
+          tmem_wait_st();
+        }
         const float mb = m_run == -INFINITY ? 0.f : m_run;
         const float2 nm2 = make_float2(-mb, -mb);
         // P = 2^(x - m) as packed bf16 into the first half of the same TMEM columns, 32 columns
@@ -496,27 +528,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pk[q] = pack_bf16(pr.x, pr.y);
           }
           tmem_st32(tS + h2 * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[h2 * 32]));
+          if (h2 == 0) {  // the first 64 keys' P may go into the tensor core already
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&phalf[c]);
+          }
         }
         const float2 s2 = __fadd2_rn(sa, sb);
         const float sum = s2.x + s2.y;
         tmem_wait_st();
-        if (resc && u > 0) {  // rescale the chain's O once its previous PV product has landed
-          if (!__all_sync(0xffffffffu, mbar_wait(&pvdone[c], (nc - 1) & 1, abort, dev_status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + c0, o);
-          }
-          tmem_wait_st();
-        }
         l_run = l_run * alpha + sum;
         tc_fence_before();
         mbar_arrive(&pready[c]);
