@@ -207,14 +207,14 @@ def bandwidth_instances(tg, torch, dev, peak_gbs, reps):
     gen = torch.Generator(device=dev)
     gen.manual_seed(20260)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+    flush = L2Flush(torch, dev)
 
     def timed(fn):
         fn()
         torch.cuda.synchronize()
         ts = []
         for _ in range(reps):
-            flush.zero_()
+            flush()
             torch.cuda._sleep(100_000)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -224,7 +224,7 @@ def bandwidth_instances(tg, torch, dev, peak_gbs, reps):
             ts.append(e0.elapsed_time(e1) / 1e3)
         return sum(ts) / len(ts)
 
-    out = {"l2": "flushed before every launch (512 MiB memset)", "peak_gbs": peak_gbs}
+    out = {"l2": "flushed before every launch (512 MiB memset, then a 256 MiB read sweep)", "peak_gbs": peak_gbs}
     B, N, q, K = 64, 131072, 256, 4096
     seqlens, q_len, k = (N,) * B, (q,) * B, (K,) * B
     sc = torch.randn(B * N, device=dev, generator=gen, dtype=torch.float32)
@@ -265,14 +265,14 @@ def qkv_rope_time(tg, torch, dev, Hk, pos, Hq, Hkv, D, peak_tflops, reps):
     Q = torch.empty(M, Hq, D, device=dev, dtype=torch.bfloat16)
     K = torch.empty(M, Hkv, D, device=dev, dtype=torch.bfloat16)
     V = torch.empty(M, Hkv, D, device=dev, dtype=torch.bfloat16)
-    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+    flush = L2Flush(torch, dev)
     stream = torch.cuda.current_stream()
     run = lambda: tg.tg_qkv_rope(Hk, W, pos, Hq, Hkv, D, 1.0e6, Q=Q, K=K, V=V)
     run()
     torch.cuda.synchronize()
     tot = 0.0
     for _ in range(reps):
-        flush.zero_()
+        flush()
         torch.cuda._sleep(100_000)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -301,14 +301,14 @@ def attn_bwd_time(tg, torch, dev, Q, K, V, logg, pos, cu, scale, peak_tflops, re
     bufs = dict(dQ=torch.empty(Q.shape, device=dev), dK=torch.empty(K.shape, device=dev),
                 dV=torch.empty(V.shape, device=dev), dlogg=torch.empty(m, device=dev),
                 dscore=torch.empty(m, device=dev))
-    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+    flush = L2Flush(torch, dev)
     stream = torch.cuda.current_stream()
     run = lambda: tg.tg_gated_attn_bwd(Q, K, V, logg, pos, cu, O, lse, dO, scale, want_dscore=True, **bufs)
     run()
     torch.cuda.synchronize()
     tot = 0.0
     for _ in range(reps):
-        flush.zero_()
+        flush()
         torch.cuda._sleep(100_000)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
