@@ -5,25 +5,31 @@
 // (aitualizate.com article: the score acts as a bias on the attention logits, with a
 // per-head gain). Causal on original positions, grouped KV heads (kv = h / (Hq/Hkv)).
 //
-// Design (B200, bf16 in, fp32 softmax and accumulation). One CTA per (sequence, 128-row
-// query tile, query head), launched longest causal row-range first so the block scheduler
-// packs the triangle like a longest-processing-time list schedule. The key tiles of the CTA
-// are split into two interleaved chains (even and odd tiles), each with its own softmax
-// warpgroup, TMEM score buffer and TMEM output accumulator, so one group's exponentials
-// overlap the other group's matrix products:
-//   * warp 0: TMA loads Q once and K_j (128 keys) into a 3-deep ring, so the next products
-//     QK^T never wait on L2; warp 2 loads V_j into the stage of chain j % 2 and stages the
-//     tile's per-key bias gain*log2(e)*log g_j in shared memory.
-//   * warp 1 (one thread): tcgen05.mma. S_j = Q K_j^T (M=128, N=128, K=D) into the chain's
-//     TMEM S buffer; O_c += P_j V_j with P_j read from TMEM (A operand in tensor memory) and
-//     V_j from shared memory (N-contiguous operand).
+// Design (B200, bf16 in, fp32 softmax and accumulation). A persistent grid, one CTA per SM (a CTA
+// holds all 512 TMEM columns), walks work items (sequence, 128-row query tile, query head) from a
+// list ordered by causal key range, longest first; CTA i takes items i, 2G-1-i, 2G+i, ... so each
+// long item is paired with a short one. The key tiles of an item are split into two interleaved
+// chains (even and odd tiles), each with its own softmax warpgroup, TMEM score buffer and TMEM
+// output accumulator, so one group's exponentials overlap the other group's matrix products:
+//   * warp 0: TMA loads each item's Q (as soon as the previous item's last S product has read
+//     the old one) and the key tiles K_j (128 keys) into a 3-deep ring that runs across items;
+//     warp 2 loads V_j into the stage of chain j % 2; warp 3 stages each tile's per-key bias
+//     gain*log2(e)*log g_j in shared memory (a key with g = 0 is closed whatever the gain).
+//   * warp 1 (one thread): tcgen05.mma. S_j = Q K_j^T (M=128, N=128, K=D) into the chain's TMEM
+//     S buffer; O_c += P_j V_j with P_j read from TMEM (A operand in tensor memory) and V_j from
+//     shared memory (N-contiguous operand), in two halves of 64 keys so the first half enters the
+//     tensor core while the softmax computes the second. S_{j+2} is issued right after PV_j: the
+//     MMAs of one thread execute in issue order, so it overwrites P_j only after PV_j read it.
 //   * warps 4-7 (chain 0) and 8-11 (chain 1): one query row per thread. The thread loads its
-//     whole S row from TMEM into registers, forms scale*log2(e)*S + bias (causal mask on the
-//     diagonal tile only), and writes P = 2^(x - m) back as packed bf16 into the same TMEM
-//     columns. The running
-//     max is only moved (and O rescaled in TMEM) when it grows by more than 8 (a factor
-//     256), which keeps every P <= 256 and the result exact after normalisation.
-//   * Chain 0's warps merge the two chains (max, sum, O) and write O (bf16) and the LSE.
+//     whole S row from TMEM into registers, forms scale*log2(e)*S + bias in pairs (causal mask
+//     on the diagonal tile only), takes the row max with three-input max, and writes
+//     P = 2^(x - m) back as packed bf16 into the same TMEM columns. The running max is only
+//     moved (and O rescaled in TMEM, before the exponentials) when it grows by more than 8 (a
+//     factor 256), which keeps every P <= 256 and the result exact after normalisation.
+//   * Both warpgroups merge the two chains (max, sum, O), each writing half of the head
+//     dimension of O (bf16); chain 0 also writes the LSE. The next item's Q load and first S
+//     products overlap the merge; its first PV products wait until the merge has read O.
+//   * The loader/issuer warpgroup gives registers to the softmax warpgroups (setmaxnreg).
 //   * The unnormalised variant multiplies P by g_j^gain before the PV product and sums the
 //     unbiased weights.
 //   * Every wait is bounded (about 2 s); on a timeout the CTA sets TG_DEV_TIMEOUT, drains
@@ -79,31 +85,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair of arguments on the FMA pipe, so that part of a tile's exponentials leave the
-// MUFU unit (which has a sixteenth of the FMA pipe's lanes). Cody-Waite range reduction:
-// x = n + f with n = round(x) (taken from the low mantissa bits of x + 1.5 * 2^23) and
-// f in [-1/2, 1/2]; 2^f from a cubic fitted here by minimising the maximum relative error on
-// [-1/2, 1/2] (iteratively reweighted least squares; max relative error 7.5e-5, far below the
-// bf16 rounding that P gets before the PV product); 2^n is added to the exponent field with
-// one integer multiply-add. Arguments are clamped to >= -125 so that the exponent stays
-// normal: such a weight is 2^-125 instead of 0, which no fp32 sum of 128 terms can notice.
-constexpr float kExpC0 = 0.99992806f, kExpC1 = 0.69326097f, kExpC2 = 0.24261114f, kExpC3 = 0.05517167f;
-constexpr float kRoundMagic = 12582912.f;  // 1.5 * 2^23
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  const float2 xc = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
-  const float2 t = __fadd2_rn(xc, make_float2(kRoundMagic, kRoundMagic));
-  const float2 n = __fadd2_rn(t, make_float2(-kRoundMagic, -kRoundMagic));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), xc);
-  float2 q = __ffma2_rn(f, make_float2(kExpC3, kExpC3), make_float2(kExpC2, kExpC2));
-  q = __ffma2_rn(q, f, make_float2(kExpC1, kExpC1));
-  q = __ffma2_rn(q, f, make_float2(kExpC0, kExpC0));
-  // the low 9 bits of t hold n (two's complement); times 2^23 they land in the exponent field
-  return make_float2(__uint_as_float(__float_as_uint(t.x) * 8388608u + __float_as_uint(q.x)),
-                     __uint_as_float(__float_as_uint(t.y) * 8388608u + __float_as_uint(q.y)));
-}
-
-// Which pairs of a 128-key row take the FMA-pipe exponential: kPolyOf8 of every 8 pairs.
-constexpr int kPolyOf8 = 0;
 
 // Work item w of the longest-first list: query tile t of sequence b, query head h. Items are
 // ordered by the length of their causal key range (tile index) descending, sequences in order
@@ -235,6 +216,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
 
+  // Register split: the loader / issuer warpgroup (warps 0-3) gives registers to the two softmax
+  // warpgroups, which hold a whole 128-key row per thread. 128 x 64 + 256 x 216 = 63488 does not
+  // exceed the launch's 384 x 168 = 64512, and the 13312 registers released cover the 12288 taken.
   if (warp < 4) {
   regs_dec<64>();
   if (skip) {
@@ -521,8 +505,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               if (q & 1) sb = __fadd2_rn(sb, pr); else sa = __fadd2_rn(sa, pr);
               pr = __fmul2_rn(pr, gg);
             } else {
-              if (j != t && (q & 7) >= 8 - kPolyOf8) pr = exp2_fma2(d);
-              else pr = make_float2(ex2(d.x), ex2(d.y));
+              pr = make_float2(ex2(d.x), ex2(d.y));
               if (q & 1) sb = __fadd2_rn(sb, pr); else sa = __fadd2_rn(sa, pr);
             }
             pk[q] = pack_bf16(pr.x, pr.y);
