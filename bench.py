@@ -191,7 +191,7 @@ def traffic_from_profile(kernel_key, src_hash):
         with open(p) as f:
             d = json.load(f)
         e = d.get(kernel_key)
-        if e and e.get("source_hash") == src_hash:
+        if isinstance(e, dict) and e.get("source_hash") == src_hash:
             return e.get("bytes_per_launch")
     except Exception:
         pass
