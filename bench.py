@@ -289,7 +289,7 @@ def qkv_rope_time(tg, torch, dev, Hk, pos, Hq, Hkv, D, peak_tflops, reps):
 def attn_bwd_time(tg, torch, dev, Q, K, V, logg, pos, cu, scale, peak_tflops, reps):
     """Gradients of the gated attention for the bench workload's kept set (one above-L layer's
     Q/K/V, the chain's own log g and positions, a seeded N(0, 1) upstream dO): the forward gives
-    O and lse, then the two backward kernels are timed together, L2 flushed before each run.
+    O and lse, then the backward's four kernels are timed together, L2 flushed before each run.
     Algorithmic work: the five products of the backward (S recomputed, dP, dV, dK, dQ), each
     2 D flop per visible (query, key) pair and head."""
     gen = torch.Generator(device=dev)
@@ -322,7 +322,7 @@ def attn_bwd_time(tg, torch, dev, Q, K, V, logg, pos, cu, scale, peak_tflops, re
     return {"shape": f"M={m} kept rows in {len(cu) - 1} sequence(s), {Hq}/{K.shape[1]} heads, D={D}, bf16 in, f32 gradients",
             "us": t * 1e6, "tflops": flops / t / 1e12, "bound": "tensor", "peak": peak_tflops,
             "frac": flops / t / 1e12 / peak_tflops,
-            "note": "warp-level mma.sync m16n8k16 kernels (dK/dV per 64-key tile, dQ per 64-query tile)"}
+            "note": "tcgen05 kernels: rowsum(dO*O) pre-pass, dK/dV per (128-key tile, KV head) cluster, d log g sum, dQ per (128-query tile, head)"}
 
 
 def projected_chain_time(tg, torch, dev, cb, flush, reps):

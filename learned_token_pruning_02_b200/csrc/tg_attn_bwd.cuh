@@ -6,9 +6,8 @@
 namespace tg {
 
 // Function-attribute slots of the backward's kernels (after the forward path's slots):
-// CUDA-core (f32) D 64, 128, then tensor-core (bf16) D 64 and 128, each with one or two warp
-// groups in the dK/dV kernel.
-enum { ATTR_BWD = ATTR_SLOTS, ATTR_ALL = ATTR_BWD + 6 };
+// CUDA-core (f32) D 64, 128, then tensor-core (bf16) D 64, 128.
+enum { ATTR_BWD = ATTR_SLOTS, ATTR_ALL = ATTR_BWD + 4 };
 
 // Gradients of the gated attention (normalised form): dQ, dK, dV (f32) and optionally d log g,
 // d score (f32), from the forward's inputs, O and lse and the upstream dO.
@@ -34,5 +33,7 @@ struct AttnBwdArgs {
   int64_t m_tot;
 };
 tg_status launch_attn_bwd(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);
+// bf16 on the tensor cores (tcgen05); called by launch_attn_bwd
+tg_status launch_attn_bwd_tc(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st);
 
 }  // namespace tg

@@ -1,0 +1,958 @@
+// Gradients of the token-gated causal attention on the 5th-generation tensor cores (bf16 in,
+// fp32 softmax arithmetic and accumulation).
+//
+// TokenGate paper page (thelatestinai.com), Figure 1(c): the gated attention is what lets the
+// top-K selector train end to end; aitualizate.com article ("Cómo consigue entrenar una
+// selección top-K"): the score enters the attention logits as a bias, so its gradient is that
+// of an additive logit bias. Per sequence, query head h and KV head h / (Hq / Hkv), with
+// S = scale Q K^T + gain_h log g^T (causal), P = exp(S - lse), Dv_i = rowsum(dO_i * O_i):
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - Dv),  dQ = scale dS K,  dK = scale dS^T Q,
+//   d log g_j = sum_h gain_h sum_i dS_ij,  d score_j = d log g_j * -expm1(log g_j).
+//
+// Four launches per group of sequences; no workspace, no atomics, deterministic results:
+//   1. bwd_prep_kernel: Dv of every (row, query head), written into element 0 of that row's dQ
+//      vector. Only the dQ kernel (launch 4) overwrites it, after reading it.
+//   2. attn_bwd_dkdv_tc: per (128-key tile, KV head) a cluster of C = min(G, 8) CTAs
+//      (G = Hq / Hkv); rank r takes the query heads r, r + C, ... of the KV group and walks
+//      the query tiles at or after the key tile. Per step (query tile, head):
+//        S^T = K Q^T and dP^T = V dO^T  (M = 128 keys, N = 128 queries, both operands K-major
+//        as stored) into TMEM; two epilogue warpgroups (one key row per thread, 64 queries
+//        each) form P^T and dS^T in fp32 and write them back as packed bf16 into the columns
+//        they read; dV += P^T dO and dK += dS^T Q take that bf16 A operand from TMEM and dO, Q
+//        from shared memory as N-contiguous (MN-major) B operands.
+//      The products of one thread execute in issue order, so S^T_{n+1} is issued right after
+//      dV_n (it overwrites P^T_n only after dV_n read it) and dP^T_{n+1} after dK_n.
+//      The cluster adds its CTAs' dK, dV and per-key d log g partials in rank order through
+//      distributed shared memory; rank 0 stores the KV head's d log g partial in element 1
+//      of the dQ vector (key row, query head kvh).
+//   3. bwd_dlogg_kernel: d log g = the sum of those partials over the KV heads, in order, and
+//      d score.
+//   4. attn_bwd_dq_tc: per (128-query tile, head), walking the key tiles up to the diagonal:
+//      S = Q K^T (two TMEM buffers, so S_{j+1} is formed while the epilogue works on tile j),
+//      dP = dO V^T, dS written as bf16 into dP's columns, dQ += dS K (K as an MN-major B).
+// Work items are ordered by the length of their chain, longest first, so the hardware's
+// in-order dispatch of CTAs balances the causal triangle.
+// Masks use the kept-row index on the diagonal tile (positions ascend inside a sequence; a
+// violation is flagged by the pre-pass), the same rule as the forward. Key rows past the
+// sequence get a -inf bias and query rows past it lse = +inf, so their weights are exactly 0.
+// Every wait is bounded (about 2 s); on a timeout the CTA sets TG_DEV_TIMEOUT, drains its
+// copies and products, frees TMEM and returns without writing results.
+#include "tg_attn_bwd.cuh"
+#include "tg_sm100.cuh"
+
+namespace tg {
+namespace {
+
+using namespace sm100;
+
+constexpr int BT = 128;        // rows of every tile (keys or queries)
+constexpr int NTHREADS = 384;  // warp 0: TMA, 1: MMA + TMEM, 2: idle, 3: vector stager, 4-11: epilogue
+constexpr int MAXC = 8;        // CTAs per cluster of the dK/dV kernel
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int SMEM_LIMIT = 227 * 1024;
+
+struct TcParams {
+  int off[kMaxSeqPerLaunch];
+  int m[kMaxSeqPerLaunch];
+  int nt[kMaxSeqPerLaunch];  // ceil(m / 128)
+  int nseq;
+  int tmax;
+  int C;  // CTAs per cluster of the dK/dV kernel
+};
+
+__device__ __forceinline__ float key_bias(float gain2, float lg) { return lg == -INFINITY ? -INFINITY : gain2 * lg; }
+__device__ __forceinline__ float lse_or_inf(float l) { return l == -INFINITY ? INFINITY : l; }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Entries (sequence, L) with 1 <= L <= nt[b] whose length is at least L
+__device__ __forceinline__ int count_ge(int L, const TcParams& p) {
+  int c = 0;
+  for (int s = 0; s < p.nseq; ++s) c += max(0, p.nt[s] - L + 1);
+  return c;
+}
+
+// The w-th entry of the list of every (sequence b, chain length L), 1 <= L <= nt[b], ordered
+// by L descending and by sequence within one L.
+__device__ __forceinline__ void decode_len(int w, const TcParams& p, int& b, int& L) {
+  int lo = 1, hi = p.tmax;  // the largest L with count_ge(L) > w
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (count_ge(mid, p) > w) lo = mid; else hi = mid - 1;
+  }
+  L = lo;
+  int r = w - count_ge(L + 1, p);
+  b = 0;
+  for (int s = 0; s < p.nseq; ++s)
+    if (p.nt[s] >= L) {
+      if (r == 0) {
+        b = s;
+        return;
+      }
+      --r;
+    }
+}
+
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// Barrier over the first `nthreads` threads arriving at named barrier `id`, returning whether
+// any of them passed a nonzero `pred`.
+__device__ __forceinline__ int bar_red_or(int id, int nthreads, int pred) {
+  int r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.s32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"(pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r;
+}
+
+// Bounded wait for copies still in flight after an abort (the CTA may not exit before they land).
+__device__ __forceinline__ void settle(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < 1000000000ull) {
+  }
+}
+
+// ------------------------------------------------------------------ 1. Dv = rowsum(dO * O)
+// One warp per (row, query head) of rows [r0, r1); the result goes to dQ[row, h, 0]. Warps of
+// head 0 also check that positions ascend inside each sequence.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ O,
+                                                       const __nv_bfloat16* __restrict__ dO,
+                                                       const int32_t* __restrict__ pos, float* __restrict__ dQ,
+                                                       int r0, int r1, int Hq, int32_t* __restrict__ dev_status,
+                                                       const __grid_constant__ TcParams p) {
+  constexpr int E = D / 32;  // elements per lane
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t row = r0 + w / Hq;
+  const int h = (int)(w % Hq);
+  if (row >= r1) return;
+  const int64_t base = (row * Hq + h) * D + lane * E;
+  float s = 0.f;
+  if constexpr (E == 4) {
+    const uint2 a = *reinterpret_cast<const uint2*>(dO + base);
+    const uint2 o = *reinterpret_cast<const uint2*>(O + base);
+    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
+    const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
+    const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
+    const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
+    s = fmaf(a0.x, o0.x, fmaf(a0.y, o0.y, fmaf(a1.x, o1.x, a1.y * o1.y)));
+  } else {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dO + base));
+    const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(O + base));
+    s = fmaf(a.x, o.x, a.y * o.y);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) {
+    dQ[(row * Hq + h) * D] = s;
+    if (h == 0 && dev_status) {
+      bool start = false;
+      for (int i = 0; i < p.nseq; ++i) start |= p.off[i] == row;
+      if (!start && pos[row - 1] >= pos[row]) atomicOr(dev_status, TG_DEV_POS_NOT_ASCENDING);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ 2. dK, dV (and d log g partials)
+template <int D>
+struct KCfg {
+  static constexpr int TILE = BT * D * 2;  // one 128 x D bf16 tile (D / 64 boxes of 128 rows x 128 bytes)
+  static constexpr int NBOX = D / 64;
+  static constexpr int K_OFF = 0, V_OFF = TILE;
+  static constexpr int Q_OFF = 2 * TILE;  // stage s: Q at Q_OFF + 2 s TILE, dO right after it
+  static constexpr int TAIL_OFF = 6 * TILE;
+  static constexpr int TAIL = 256 + 4 * BT * 4 + 2 * BT * 4;  // barriers, [2 stages][-lse2, -Dv][128], dl [2][128]
+  static constexpr int SMEM = 1024 + TAIL_OFF + TAIL;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BT, BT, false);
+  static constexpr uint32_t IDESC_G = idesc_bf16_f32(BT, D, true);
+  // TMEM columns: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D)
+  static constexpr uint32_t T_DV = 256, T_DK = 256 + D;
+  static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
+  static_assert(4 * TILE >= 2 * BT * D * 4, "the Q / dO stages hold the fp32 dK, dV partials at the end");
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                     const float* __restrict__ logg, const float* __restrict__ gain, const float* __restrict__ lse,
+                     float* __restrict__ dQ, float* __restrict__ dK, float* __restrict__ dV, int64_t m_tot, int Hq,
+                     int Hkv, float qk_scale2, float scale, int want_dl, int32_t* __restrict__ dev_status,
+                     uint64_t probe_ns, const __grid_constant__ TcParams p) {
+  using C = KCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* tail = smem + C::TAIL_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* kvfull = bars + 0;
+  uint64_t* qfull = bars + 1;    // [2] Q and dO of a stage landed
+  uint64_t* qempty = bars + 3;   // [2] the stage's last product (dK) read them
+  uint64_t* vfull = bars + 5;    // [2] the stage's per-query vectors are staged
+  uint64_t* vempty = bars + 7;   // [2] both epilogue warpgroups read them
+  uint64_t* sfull = bars + 9;    // S^T landed
+  uint64_t* dpfull = bars + 10;  // dP^T landed
+  uint64_t* pready = bars + 11;  // [2] a warpgroup's half of P^T is in TMEM
+  uint64_t* dsready = bars + 13; // [2] a warpgroup's half of dS^T is in TMEM
+  uint64_t* accdone = bars + 15;
+  uint64_t* drain = bars + 16;
+  uint64_t* probe = bars + 17;   // test hook: a barrier nothing signals
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* vec_s = reinterpret_cast<float*>(tail + 256);  // [2 stages][-lse * log2(e), -Dv][128]
+  float* dl_s = vec_s + 4 * BT;                         // [2 warpgroups][128]
+
+  const int G = Hq / Hkv, Cn = p.C;
+  const int rank = (int)(blockIdx.x % (unsigned)Cn);
+  const int kvh = (int)((blockIdx.x / (unsigned)Cn) % (unsigned)Hkv);
+  int b, L;
+  decode_len((int)(blockIdx.x / (unsigned)(Cn * Hkv)), p, b, L);
+  const int off = p.off[b], m = p.m[b];
+  const int kt = p.nt[b] - L;                 // this key tile; query tiles kt .. nt-1 see it
+  const int nh = (G - rank + Cn - 1) / Cn;    // query heads kvh G + rank + i C, i < nh
+  const int N = nh * L;                       // steps (head, query tile)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kvfull, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qempty[s], 1);
+      mbar_init(&vfull[s], 32);
+      mbar_init(&vempty[s], 256);
+      mbar_init(&pready[s], 128);
+      mbar_init(&dsready[s], 128);
+    }
+    mbar_init(sfull, 1);
+    mbar_init(dpfull, 1);
+    mbar_init(accdone, 1);
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+    wait_probe(probe, probe_ns, abort, dev_status);  // no-op unless a test asked for it
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmdO);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
+  bool wrote = false;        // this thread's dK / dV / d log g partials are in shared memory
+
+  // The loader / issuer warpgroup gives registers to the epilogue warpgroups:
+  // 128 x 64 + 256 x 216 = 63488 <= the launch's 384 x 168 = 64512.
+  if (warp < 4) {
+    regs_dec<64>();
+    if (skip) {
+    } else if (warp == 0) {  // -------------------------------------------------- TMA producer
+      if (lane == 0) {
+        int issued = 0;
+        mbar_arrive_expect_tx(kvfull, 2 * C::TILE);
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          tma_load_2d(smem + C::K_OFF + bx * (BT * 128), &tmK, kvh * D + bx * 64, off + kt * BT, kvfull);
+          tma_load_2d(smem + C::V_OFF + bx * (BT * 128), &tmV, kvh * D + bx * 64, off + kt * BT, kvfull);
+        }
+        for (int n = 0; n < N; ++n) {
+          const int s = n & 1;
+          if (n >= 2 && !mbar_wait(&qempty[s], ((n >> 1) - 1) & 1, abort, dev_status)) break;
+          const int h = kvh * G + rank + (n / L) * Cn, qt = kt + n % L;
+          uint8_t* qb = smem + C::Q_OFF + s * 2 * C::TILE;
+          mbar_arrive_expect_tx(&qfull[s], 2 * C::TILE);
+          for (int bx = 0; bx < C::NBOX; ++bx) {
+            tma_load_2d(qb + bx * (BT * 128), &tmQ, h * D + bx * 64, off + qt * BT, &qfull[s]);
+            tma_load_2d(qb + C::TILE + bx * (BT * 128), &tmdO, h * D + bx * 64, off + qt * BT, &qfull[s]);
+          }
+          ++issued;
+        }
+        if (*abort) {  // let the copies in flight land before the CTA can leave
+          settle(kvfull, 0);
+          for (int n = issued - 2 < 0 ? 0 : issued - 2; n < issued; ++n) settle(&qfull[n & 1], (n >> 1) & 1);
+        }
+      }
+    } else if (warp == 1) {  // ------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t ka = smem_u32(smem + C::K_OFF), va = smem_u32(smem + C::V_OFF);
+        auto qa = [&](int n) { return smem_u32(smem + C::Q_OFF + (n & 1) * 2 * C::TILE); };
+        auto issue_ss = [&](uint32_t d, uint32_t a, uint32_t bq) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+            mma_ss(d, sdesc_sw128(a + o, 16, 1024), sdesc_sw128(bq + o, 16, 1024), C::IDESC_S, kk > 0);
+          }
+        };
+        bool ok = mbar_wait(kvfull, 0, abort, dev_status) && mbar_wait(&qfull[0], 0, abort, dev_status);
+        if (ok) {
+          tc_fence_after();
+          issue_ss(tmem + 0, ka, qa(0));  // S^T_0 = K Q_0^T
+          mma_commit(sfull);
+          issue_ss(tmem + 128, va, qa(0) + C::TILE);  // dP^T_0 = V dO_0^T
+          mma_commit(dpfull);
+        }
+        for (int n = 0; ok && n < N; ++n) {
+          const uint32_t ph = n & 1;
+          const uint32_t q_a = qa(n), do_a = q_a + C::TILE;
+          // dV += P^T dO in the two query halves, each as soon as its P^T is in TMEM
+          for (int c = 0; c < 2; ++c) {
+            if (!mbar_wait(&pready[c], ph, abort, dev_status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = 4 * c + k4;
+              mma_ts(tmem + C::T_DV, tmem + c * 64 + k4 * 8, sdesc_sw128(do_a + kk * 2048, BT * 128, 1024),
+                     C::IDESC_G, (n > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          if (n + 1 < N) {  // S^T_{n+1}: overwrites P^T_n only after dV_n read it (issue order)
+            if (!mbar_wait(&qfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, dev_status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_ss(tmem + 0, ka, qa(n + 1));
+            mma_commit(sfull);
+          }
+          for (int c = 0; c < 2; ++c) {  // dK += dS^T Q
+            if (!mbar_wait(&dsready[c], ph, abort, dev_status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = 4 * c + k4;
+              mma_ts(tmem + C::T_DK, tmem + 128 + c * 64 + k4 * 8, sdesc_sw128(q_a + kk * 2048, BT * 128, 1024),
+                     C::IDESC_G, (n > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&qempty[n & 1]);  // the stage's Q and dO are no longer read
+          if (n + 1 < N) {             // dP^T_{n+1}: overwrites dS^T_n only after dK_n read it
+            issue_ss(tmem + 128, va, qa(n + 1) + C::TILE);
+            mma_commit(dpfull);
+          }
+        }
+        if (ok) mma_commit(accdone);
+        mma_commit(drain);
+        settle(drain, 0);
+      }
+    } else if (warp == 3) {  // ----------------------------------- per-query vectors stager
+      // -lse * log2(e) (-inf for rows past the sequence, whose lse reads as +inf) and -Dv of
+      // the step's 128 queries, 4 per lane, into the stage's slots.
+      for (int n = 0; n < N; ++n) {
+        const int s = n & 1;
+        const int h = kvh * G + rank + (n / L) * Cn, qt = kt + n % L;
+        float nl[4], nd[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int q = qt * BT + lane * 4 + e;
+          const bool v = q < m;
+          nl[e] = v ? -lse_or_inf(lse[(int64_t)h * m_tot + off + q]) * kLog2e : -INFINITY;
+          nd[e] = v ? -dQ[((int64_t)(off + q) * Hq + h) * D] : 0.f;
+        }
+        if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&vempty[s], ((n >> 1) - 1) & 1, abort, dev_status))) break;
+        *reinterpret_cast<float4*>(vec_s + s * 2 * BT + lane * 4) = make_float4(nl[0], nl[1], nl[2], nl[3]);
+        *reinterpret_cast<float4*>(vec_s + s * 2 * BT + BT + lane * 4) = make_float4(nd[0], nd[1], nd[2], nd[3]);
+        mbar_arrive(&vfull[s]);
+      }
+    }
+  } else if (!skip) {  // ------------------------------------------------------ epilogue
+    regs_inc<216>();
+    const int c = (warp - 4) >> 2;  // query half: 0 = queries 0-63 (warps 4-7), 1 = 64-127 (warps 8-11)
+    const int q4 = warp & 3;
+    const int kr = q4 * 32 + lane;  // key row in the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tmem + lane_base + c * 64, tP = tmem + lane_base + 128 + c * 64;
+    const int kl = kt * BT + kr;
+    const bool kvalid = kl < m;
+    const float lgk = (logg && kvalid) ? logg[off + kl] : 0.f;
+    const float2 qs2 = make_float2(qk_scale2, qk_scale2);
+    float dl = 0.f, racc = 0.f, gh = 1.f, bias2 = 0.f;
+    bool ok = true;
+    for (int n = 0; n < N; ++n) {
+      const int s = n & 1;
+      const int qt = kt + n % L;
+      if (n % L == 0) {  // a new query head
+        dl = fmaf(gh, racc, dl);
+        racc = 0.f;
+        gh = gain ? gain[kvh * G + rank + (n / L) * Cn] : 1.f;
+        bias2 = kvalid ? key_bias(gh * kLog2e, lgk) : -INFINITY;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&vfull[s], (n >> 1) & 1, abort, dev_status) &&
+                                       mbar_wait(sfull, n & 1, abort, dev_status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t xr[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&xr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&xr[32]));
+      tmem_wait_ld();
+      float* x = reinterpret_cast<float*>(xr);
+      const float* nl = vec_s + s * 2 * BT + c * 64;
+      const float2 bb = make_float2(bias2, bias2);
+      const bool diag = qt == kt;
+      uint32_t pk[32];
+      // P^T = 2^(scale log2(e) S^T + bias - lse log2(e)); on the diagonal tile query < key is masked
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        float2 v = __ffma2_rn(make_float2(x[2 * q], x[2 * q + 1]), qs2, bb);
+        v = __fadd2_rn(v, *reinterpret_cast<const float2*>(nl + 2 * q));
+        if (diag) {
+          if (c * 64 + 2 * q < kr) v.x = -INFINITY;
+          if (c * 64 + 2 * q + 1 < kr) v.y = -INFINITY;
+        }
+        x[2 * q] = ex2(v.x);
+        x[2 * q + 1] = ex2(v.y);
+        pk[q] = pack_bf16(x[2 * q], x[2 * q + 1]);
+      }
+      tmem_st32(tS, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&pready[c]);
+      if (!__all_sync(0xffffffffu, mbar_wait(dpfull, n & 1, abort, dev_status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t yr[64];
+      tmem_ld32(tP, *reinterpret_cast<uint32_t(*)[32]>(&yr[0]));
+      tmem_ld32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&yr[32]));
+      tmem_wait_ld();
+      const float* y = reinterpret_cast<const float*>(yr);
+      const float* nd = vec_s + s * 2 * BT + BT + c * 64;
+      float2 ra = make_float2(0.f, 0.f), rb = make_float2(0.f, 0.f);
+      // dS^T = P^T * (dP^T - Dv), with the fp32 P^T
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const float2 d = __fadd2_rn(make_float2(y[2 * q], y[2 * q + 1]), *reinterpret_cast<const float2*>(nd + 2 * q));
+        const float2 ds = __fmul2_rn(make_float2(x[2 * q], x[2 * q + 1]), d);
+        if (q & 1) rb = __fadd2_rn(rb, ds); else ra = __fadd2_rn(ra, ds);
+        pk[q] = pack_bf16(ds.x, ds.y);
+      }
+      tmem_st32(tP, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&dsready[c]);
+      mbar_arrive(&vempty[s]);
+      racc += (ra.x + ra.y) + (rb.x + rb.y);
+    }
+    dl = fmaf(gh, racc, dl);
+    if (ok && __all_sync(0xffffffffu, mbar_wait(accdone, 0, abort, dev_status))) {
+      tc_fence_after();
+      // this CTA's dV and dK (fp32) into the freed Q / dO stages: [2][128 rows][D], each row's
+      // 16-byte slots permuted by row % 8 so a warp's stores (one row per lane) hit distinct banks
+      float* red = reinterpret_cast<float*>(smem + C::Q_OFF);
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+#pragma unroll 1
+        for (int col0 = c * (D / 2); col0 < (c + 1) * (D / 2); col0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + (t ? C::T_DK : C::T_DV) + col0, v);
+          tmem_wait_ld();
+          float4* rowp = reinterpret_cast<float4*>(red + (t * BT + kr) * D);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            rowp[((col0 >> 2) + i) ^ (kr & 7)] =
+                make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                            __uint_as_float(v[4 * i + 3]));
+        }
+      }
+      dl_s[c * BT + kr] = dl;
+      wrote = true;
+    }
+  }
+
+  // ------------------------------------------------------------ cluster reduction of dK, dV
+  // Every CTA of the cluster reaches here (all waits above are bounded). A CTA that could not
+  // finish publishes a nonzero flag; then nobody in the cluster writes results.
+  const int bad = __syncthreads_or(!skip && warp >= 4 && !wrote) || skip;
+  if (threadIdx.x == 0) *abort = bad ? 1 : 0;
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();
+  int any_bad = 0;
+  for (int q = 0; q < Cn; ++q) any_bad |= ld_cluster_s32(mapa_rank(smem_u32(const_cast<int*>(abort)), (uint32_t)q));
+  if (!any_bad) {
+    const float* red = reinterpret_cast<const float*>(smem + C::Q_OFF);
+    constexpr int D4 = D / 4;
+    const int c4a = rank * D4 / Cn, w4 = (rank + 1) * D4 / Cn - c4a;  // this rank's 16-byte columns
+    const int total = 2 * BT * w4;
+    for (int idx = threadIdx.x; idx < total; idx += NTHREADS) {
+      const int t = idx / (BT * w4), rem = idx - t * BT * w4;
+      const int row = rem / w4, c4 = c4a + rem % w4;
+      const int kl = kt * BT + row;
+      if (kl >= m) continue;
+      const uint32_t la = smem_u32(red + (t * BT + row) * D + ((c4 ^ (row & 7)) << 2));
+      float4 acc = ld_cluster_f4(mapa_rank(la, 0));
+      for (int q = 1; q < Cn; ++q) {
+        const float4 v = ld_cluster_f4(mapa_rank(la, (uint32_t)q));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      if (t == 1) acc = make_float4(acc.x * scale, acc.y * scale, acc.z * scale, acc.w * scale);
+      float* out = (t ? dK : dV) + ((int64_t)(off + kl) * Hkv + kvh) * D + c4 * 4;
+      *reinterpret_cast<float4*>(out) = acc;
+    }
+    if (want_dl && rank == 0 && threadIdx.x < BT) {
+      const int row = threadIdx.x, kl = kt * BT + row;
+      if (kl < m) {
+        float s = 0.f;
+        for (int q = 0; q < Cn; ++q)
+          s += ld_cluster_f32(mapa_rank(smem_u32(dl_s + row), (uint32_t)q)) +
+               ld_cluster_f32(mapa_rank(smem_u32(dl_s + BT + row), (uint32_t)q));
+        dQ[((int64_t)(off + kl) * Hq + kvh) * D + 1] = s;
+      }
+    }
+  }
+  __syncwarp();
+  cluster_sync_all();  // no CTA leaves while another still reads its shared memory
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ 3. d log g and d score
+__global__ void __launch_bounds__(256) bwd_dlogg_kernel(const float* __restrict__ dQ, const float* __restrict__ logg,
+                                                        float* __restrict__ dlogg, float* __restrict__ dscore, int r0,
+                                                        int r1, int Hq, int Hkv, int D) {
+  const int64_t row = r0 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= r1) return;
+  float s = 0.f;
+  for (int kvh = 0; kvh < Hkv; ++kvh) s += dQ[(row * Hq + kvh) * D + 1];
+  if (dlogg) dlogg[row] = s;
+  if (dscore) dscore[row] = s * -expm1f(logg[row]);
+}
+
+// ------------------------------------------------------------------ 4. dQ
+template <int D>
+struct QCfg {
+  static constexpr int TILE = BT * D * 2;
+  static constexpr int NBOX = D / 64;
+  static constexpr int KSL = 3;  // K ring: K_j is read by S_j and, a step later, by dQ_j
+  static constexpr int Q_OFF = 0, DO_OFF = TILE, K_OFF = 2 * TILE, V_OFF = (2 + KSL) * TILE;
+  static constexpr int TAIL_OFF = (4 + KSL) * TILE;
+  static constexpr int TAIL = 256 + 2 * BT * 4;  // barriers, key bias [2][128]
+  static constexpr int SMEM = 1024 + TAIL_OFF + TAIL;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BT, BT, false);
+  static constexpr uint32_t IDESC_G = idesc_bf16_f32(BT, D, true);
+  // TMEM columns: S buffers [0, 128) and [128, 256), dP [256, 384), dQ [384, 384 + D)
+  static constexpr uint32_t T_DP = 256, T_DQ = 384;
+  static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
+  static_assert(2 * TILE == BT * D * 4, "the Q and dO tiles hold the fp32 dQ tile at the end");
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                   const float* __restrict__ logg, const float* __restrict__ gain, const float* __restrict__ lse,
+                   float* __restrict__ dQ, int64_t m_tot, int Hq, int Hkv, float qk_scale2, float scale,
+                   int32_t* __restrict__ dev_status, uint64_t probe_ns, const __grid_constant__ TcParams p) {
+  using C = QCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* tail = smem + C::TAIL_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* qfull = bars + 0;
+  uint64_t* kfull = bars + 1;    // [3]
+  uint64_t* kempty = bars + 4;   // [3]
+  uint64_t* vfull = bars + 7;    // [2]
+  uint64_t* vempty = bars + 9;   // [2]
+  uint64_t* sfull = bars + 11;   // [2] per S buffer
+  uint64_t* dpfull = bars + 13;
+  uint64_t* dsready = bars + 14; // [2] per epilogue warpgroup
+  uint64_t* bfull = bars + 16;   // [2] key bias slots
+  uint64_t* bempty = bars + 18;  // [2]
+  uint64_t* accdone = bars + 20;
+  uint64_t* drain = bars + 21;
+  uint64_t* probe = bars + 22;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* bias_s = reinterpret_cast<float*>(tail + 256);  // [2][128]
+
+  const int G = Hq / Hkv;
+  const int h = (int)(blockIdx.x % (unsigned)Hq), kvh = h / G;
+  int b, L;
+  decode_len((int)(blockIdx.x / (unsigned)Hq), p, b, L);
+  const int off = p.off[b], m = p.m[b];
+  const int qt = L - 1;  // this query tile; key tiles 0 .. qt
+  const int N = L;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qfull, 1);
+    for (int s = 0; s < C::KSL; ++s) {
+      mbar_init(&kfull[s], 1);
+      mbar_init(&kempty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&vfull[s], 1);
+      mbar_init(&vempty[s], 1);
+      mbar_init(&sfull[s], 1);
+      mbar_init(&dsready[s], 128);
+      mbar_init(&bfull[s], 32);
+      mbar_init(&bempty[s], 256);
+    }
+    mbar_init(dpfull, 1);
+    mbar_init(accdone, 1);
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+    wait_probe(probe, probe_ns, abort, dev_status);
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmdO);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = *abort;
+
+  if (warp < 4) {
+    regs_dec<64>();
+    if (skip) {
+    } else if (warp == 0) {  // -------------------------------------------------- TMA producer
+      if (lane == 0) {
+        int nk = 0, nv = 0;
+        mbar_arrive_expect_tx(qfull, 2 * C::TILE);
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          tma_load_2d(smem + C::Q_OFF + bx * (BT * 128), &tmQ, h * D + bx * 64, off + qt * BT, qfull);
+          tma_load_2d(smem + C::DO_OFF + bx * (BT * 128), &tmdO, h * D + bx * 64, off + qt * BT, qfull);
+        }
+        for (int j = 0; j < N; ++j) {  // K_j and V_j in the order the products need them
+          const int ks = j % C::KSL;
+          if (j >= C::KSL && !mbar_wait(&kempty[ks], ((j / C::KSL) - 1) & 1, abort, dev_status)) break;
+          mbar_arrive_expect_tx(&kfull[ks], C::TILE);
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_2d(smem + C::K_OFF + ks * C::TILE + bx * (BT * 128), &tmK, kvh * D + bx * 64, off + j * BT,
+                        &kfull[ks]);
+          ++nk;
+          const int vs = j & 1;
+          if (j >= 2 && !mbar_wait(&vempty[vs], ((j >> 1) - 1) & 1, abort, dev_status)) break;
+          mbar_arrive_expect_tx(&vfull[vs], C::TILE);
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_2d(smem + C::V_OFF + vs * C::TILE + bx * (BT * 128), &tmV, kvh * D + bx * 64, off + j * BT,
+                        &vfull[vs]);
+          ++nv;
+        }
+        if (*abort) {
+          settle(qfull, 0);
+          for (int j = nk - C::KSL < 0 ? 0 : nk - C::KSL; j < nk; ++j) settle(&kfull[j % C::KSL], (j / C::KSL) & 1);
+          for (int j = nv - 2 < 0 ? 0 : nv - 2; j < nv; ++j) settle(&vfull[j & 1], (j >> 1) & 1);
+        }
+      }
+    } else if (warp == 1) {  // ------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t qa = smem_u32(smem + C::Q_OFF), doa = smem_u32(smem + C::DO_OFF);
+        auto ka = [&](int j) { return smem_u32(smem + C::K_OFF + (j % C::KSL) * C::TILE); };
+        auto issue_ss = [&](uint32_t d, uint32_t a, uint32_t bk) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+            mma_ss(d, sdesc_sw128(a + o, 16, 1024), sdesc_sw128(bk + o, 16, 1024), C::IDESC_S, kk > 0);
+          }
+        };
+        auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T into buffer j % 2
+          if (!mbar_wait(&kfull[j % C::KSL], (j / C::KSL) & 1, abort, dev_status)) return false;
+          tc_fence_after();
+          issue_ss(tmem + (j & 1) * 128, qa, ka(j));
+          mma_commit(&sfull[j & 1]);
+          return true;
+        };
+        auto issue_dp = [&](int j) -> bool {  // dP_j = dO V_j^T
+          if (!mbar_wait(&vfull[j & 1], (j >> 1) & 1, abort, dev_status)) return false;
+          tc_fence_after();
+          issue_ss(tmem + C::T_DP, doa, smem_u32(smem + C::V_OFF + (j & 1) * C::TILE));
+          mma_commit(dpfull);
+          mma_commit(&vempty[j & 1]);
+          return true;
+        };
+        bool ok = mbar_wait(qfull, 0, abort, dev_status);
+        ok = ok && issue_s(0) && issue_dp(0) && (N < 2 || issue_s(1));
+        for (int j = 0; ok && j < N; ++j) {
+          const uint32_t k_a = ka(j);
+          for (int c = 0; c < 2; ++c) {  // dQ += dS K_j, each key half as soon as its dS is in TMEM
+            if (!mbar_wait(&dsready[c], j & 1, abort, dev_status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = 4 * c + k4;
+              mma_ts(tmem + C::T_DQ, tmem + C::T_DP + c * 64 + k4 * 8, sdesc_sw128(k_a + kk * 2048, BT * 128, 1024),
+                     C::IDESC_G, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&kempty[j % C::KSL]);
+          // dP_{j+1} overwrites dS_j only after dQ_j read it; S_{j+2} reuses S_j's buffer, which
+          // the epilogue finished reading before it wrote dS_j
+          if (j + 1 < N) ok = issue_dp(j + 1);
+          if (ok && j + 2 < N) ok = issue_s(j + 2);
+        }
+        if (ok) mma_commit(accdone);
+        mma_commit(drain);
+        settle(drain, 0);
+      }
+    } else if (warp == 3) {  // ------------------------------------------- key bias stager
+      const float gain2 = (gain ? gain[h] : 1.f) * kLog2e;
+      for (int j = 0; j < N; ++j) {
+        const int bs = j & 1;
+        float bv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int kl = j * BT + lane * 4 + e;
+          bv[e] = kl < m ? (logg ? key_bias(gain2, logg[off + kl]) : 0.f) : -INFINITY;
+        }
+        if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bempty[bs], ((j >> 1) - 1) & 1, abort, dev_status))) break;
+        *reinterpret_cast<float4*>(bias_s + bs * BT + lane * 4) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+        mbar_arrive(&bfull[bs]);
+      }
+    }
+  } else if (!skip) {  // ------------------------------------------------------ epilogue
+    regs_inc<216>();
+    const int c = (warp - 4) >> 2;  // key half: 0 = keys 0-63 (warps 4-7), 1 = 64-127 (warps 8-11)
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;  // query row in the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tP = tmem + lane_base + C::T_DP + c * 64;
+    const int il = qt * BT + r;
+    const bool valid = il < m;
+    const float nlse2 = valid ? -lse_or_inf(lse[(int64_t)h * m_tot + off + il]) * kLog2e : -INFINITY;
+    const float ndv = valid ? -dQ[((int64_t)(off + il) * Hq + h) * D] : 0.f;  // read before any dQ write below
+    const float2 qs2 = make_float2(qk_scale2, qk_scale2), nl2 = make_float2(nlse2, nlse2), nd2 = make_float2(ndv, ndv);
+    bool ok = true;
+    for (int j = 0; j < N; ++j) {
+      const int bs = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bfull[bs], (j >> 1) & 1, abort, dev_status) &&
+                                       mbar_wait(&sfull[j & 1], (j >> 1) & 1, abort, dev_status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tS = tmem + lane_base + (j & 1) * 128 + c * 64;
+      uint32_t xr[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&xr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&xr[32]));
+      tmem_wait_ld();
+      float* x = reinterpret_cast<float*>(xr);
+      const float* bb = bias_s + bs * BT + c * 64;
+      const bool diag = j == qt;
+      // P = 2^(scale log2(e) S + bias - lse log2(e)); on the diagonal tile key > query is masked
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        float2 v = __ffma2_rn(make_float2(x[2 * q], x[2 * q + 1]), qs2, *reinterpret_cast<const float2*>(bb + 2 * q));
+        v = __fadd2_rn(v, nl2);
+        if (diag) {
+          if (c * 64 + 2 * q > r) v.x = -INFINITY;
+          if (c * 64 + 2 * q + 1 > r) v.y = -INFINITY;
+        }
+        x[2 * q] = ex2(v.x);
+        x[2 * q + 1] = ex2(v.y);
+      }
+      mbar_arrive(&bempty[bs]);
+      if (!__all_sync(0xffffffffu, mbar_wait(dpfull, j & 1, abort, dev_status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t yr[64];
+      tmem_ld32(tP, *reinterpret_cast<uint32_t(*)[32]>(&yr[0]));
+      tmem_ld32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&yr[32]));
+      tmem_wait_ld();
+      const float* y = reinterpret_cast<const float*>(yr);
+      uint32_t pk[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const float2 d = __fadd2_rn(make_float2(y[2 * q], y[2 * q + 1]), nd2);
+        const float2 ds = __fmul2_rn(make_float2(x[2 * q], x[2 * q + 1]), d);
+        pk[q] = pack_bf16(ds.x, ds.y);
+      }
+      tmem_st32(tP, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&dsready[c]);
+    }
+    ok = ok && __all_sync(0xffffffffu, mbar_wait(accdone, 0, abort, dev_status));
+    if (ok) {
+      tc_fence_after();
+      // the dQ tile (fp32) into the Q and dO tiles' space, then coalesced row stores
+      float* stg = reinterpret_cast<float*>(smem + C::Q_OFF);
+#pragma unroll 1
+      for (int col0 = c * (D / 2); col0 < (c + 1) * (D / 2); col0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + C::T_DQ + col0, v);
+        tmem_wait_ld();
+        float4* rowp = reinterpret_cast<float4*>(stg + r * D);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          rowp[((col0 >> 2) + i) ^ (r & 7)] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                          __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+      }
+    }
+    // both warpgroups: every Dv read above is done and the staged tile is complete
+    const bool all_ok = bar_red_or(1, 256, !ok) == 0;
+    if (all_ok) {
+      constexpr int D4 = D / 4;
+      const float* stg = reinterpret_cast<const float*>(smem + C::Q_OFF);
+      for (int idx = threadIdx.x - 128; idx < BT * D4; idx += 256) {
+        const int row = idx / D4, c4 = idx % D4;
+        const int i2 = qt * BT + row;
+        if (i2 >= m) continue;
+        const float4 v = *reinterpret_cast<const float4*>(stg + row * D + ((c4 ^ (row & 7)) << 2));
+        *reinterpret_cast<float4*>(dQ + ((int64_t)(off + i2) * Hq + h) * D + c4 * 4) =
+            make_float4(v.x * scale, v.y * scale, v.z * scale, v.w * scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+tg_status launch_tc_d(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st) {
+  using KC = KCfg<D>;
+  using QC = QCfg<D>;
+  TcParams p = {};
+  p.nseq = nseq;
+  int units = 0, tmax = 0;
+  for (int i = 0; i < nseq; ++i) {
+    p.off[i] = seqs[i].off;
+    p.m[i] = seqs[i].m;
+    p.nt[i] = (seqs[i].m + BT - 1) / BT;
+    units += p.nt[i];
+    tmax = p.nt[i] > tmax ? p.nt[i] : tmax;
+  }
+  p.tmax = tmax;
+  if (units == 0) return TG_OK;
+  const int r0 = seqs[0].off, r1 = seqs[nseq - 1].off + seqs[nseq - 1].m;
+  const int G = a.Hq / a.Hkv;
+  p.C = G < MAXC ? G : MAXC;
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap_bf16_2d(&tq, a.Q, (uint64_t)a.m_tot, (uint64_t)a.Hq * D, (uint64_t)a.Hq * D, BT, 64) ||
+      !make_tmap_bf16_2d(&tdo, a.dO, (uint64_t)a.m_tot, (uint64_t)a.Hq * D, (uint64_t)a.Hq * D, BT, 64) ||
+      !make_tmap_bf16_2d(&tk, a.K, (uint64_t)a.m_tot, (uint64_t)a.Hkv * D, (uint64_t)a.Hkv * D, BT, 64) ||
+      !make_tmap_bf16_2d(&tv, a.V, (uint64_t)a.m_tot, (uint64_t)a.Hkv * D, (uint64_t)a.Hkv * D, BT, 64))
+    return fail(TG_ERR_CUDA, "tg_gated_attn_bwd: building the TMA tensor maps failed");
+
+  auto kdkdv = attn_bwd_dkdv_tc<D>;
+  auto kdq = attn_bwd_dq_tc<D>;
+  const int slot = ATTR_BWD + 2 + (D == 128 ? 1 : 0);
+  if (attrs_needed(slot)) {
+    cudaError_t e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, KC::SMEM);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, QC::SMEM);
+    if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: cudaFuncSetAttribute");
+    mark_attrs_set(slot);
+  }
+  const __nv_bfloat16* O = static_cast<const __nv_bfloat16*>(a.O);
+  const __nv_bfloat16* dO = static_cast<const __nv_bfloat16*>(a.dO);
+  const uint64_t probe = wait_probe_ns();
+  const float qk2 = a.scale * kLog2e;
+
+  // 1. Dv into dQ[., ., 0]
+  const int64_t warps = (int64_t)(r1 - r0) * a.Hq;
+  bwd_prep_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(O, dO, a.pos, a.dQ, r0, r1, a.Hq, a.dev_status, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: prep launch");
+
+  // 2. dK, dV: clusters of C CTAs over the query heads of one (key tile, KV head)
+  const int want_dl = (a.dlogg || a.dscore) ? 1 : 0;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units * a.Hkv * p.C));
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = (size_t)KC::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kdkdv, tq, tk, tv, tdo, a.logg, a.head_gain, a.lse, a.dQ, a.dK, a.dV, a.m_tot, a.Hq,
+                           a.Hkv, qk2, a.scale, want_dl, a.dev_status, probe, p);
+    if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: dK/dV launch");
+  }
+
+  // 3. d log g, d score
+  if (want_dl) {
+    bwd_dlogg_kernel<<<(unsigned)((r1 - r0 + 255) / 256), 256, 0, st>>>(a.dQ, a.logg, a.dlogg, a.dscore, r0, r1, a.Hq,
+                                                                         a.Hkv, D);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: d log g launch");
+  }
+
+  // 4. dQ: one CTA per (query tile, head), longest chains first
+  {
+    cudaLaunchConfig_t cq = {};
+    cq.gridDim = dim3((unsigned)(units * a.Hq));
+    cq.blockDim = dim3(NTHREADS);
+    cq.dynamicSmemBytes = (size_t)QC::SMEM;
+    cq.stream = st;
+    e = cudaLaunchKernelEx(&cq, kdq, tq, tk, tv, tdo, a.logg, a.head_gain, a.lse, a.dQ, a.m_tot, a.Hq, a.Hkv, qk2,
+                           a.scale, a.dev_status, probe, p);
+  }
+  return cuda_status(e, "tg_gated_attn_bwd: dQ launch");
+}
+
+}  // namespace
+
+tg_status launch_attn_bwd_tc(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaStream_t st) {
+  return a.D == 64 ? launch_tc_d<64>(a, seqs, nseq, st) : launch_tc_d<128>(a, seqs, nseq, st);
+}
+
+}  // namespace tg
