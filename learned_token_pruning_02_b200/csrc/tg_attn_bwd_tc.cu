@@ -12,19 +12,19 @@
 // Four launches per group of sequences; no workspace, no atomics, deterministic results:
 //   1. bwd_prep_kernel: Dv of every (row, query head), written into element 0 of that row's dQ
 //      vector. Only the dQ kernel (launch 4) overwrites it, after reading it.
-//   2. attn_bwd_dkdv_tc: per (128-key tile, KV head) a cluster of C = min(G, 8) CTAs
-//      (G = Hq / Hkv); rank r takes the query heads r, r + C, ... of the KV group and walks
-//      the query tiles at or after the key tile. Per step (query tile, head):
-//        S^T = K Q^T and dP^T = V dO^T  (M = 128 keys, N = 128 queries, both operands K-major
-//        as stored) into TMEM; two epilogue warpgroups (one key row per thread, 64 queries
-//        each) form P^T and dS^T in fp32 and write them back as packed bf16 into the columns
-//        they read; dV += P^T dO and dK += dS^T Q take that bf16 A operand from TMEM and dO, Q
-//        from shared memory as N-contiguous (MN-major) B operands.
-//      The products of one thread execute in issue order, so S^T_{n+1} is issued right after
-//      dV_n (it overwrites P^T_n only after dV_n read it) and dP^T_{n+1} after dK_n.
-//      The cluster adds its CTAs' dK, dV and per-key d log g partials in rank order through
-//      distributed shared memory; rank 0 stores the KV head's d log g partial in element 1
-//      of the dQ vector (key row, query head kvh).
+//   2. attn_bwd_dkdv_tc: per (128-key tile, KV head) one CTA, or a cluster of two CTAs when
+//      the KV group has an even number G of query heads (each CTA takes every other head);
+//      every CTA walks the query tiles at or after its key tile. Per step (query tile, head):
+//        S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, both operands K-major as
+//        stored) take turns in one 128-column TMEM region: dP^T_n is issued as soon as the two
+//        epilogue warpgroups (one key row per thread, 64 queries each) hold S^T_n in registers,
+//        and S^T_{n+1} as soon as they hold dP^T_n. They write P^T and dS^T as packed bf16 into
+//        TMEM regions of their own; dV += P^T dO and dK += dS^T Q take that A operand from TMEM
+//        and dO, Q from shared memory as N-contiguous (MN-major) B operands.
+//      A cluster's two partial dK, dV (and d log g) are added in rank order: each CTA owns half
+//      of the columns, the other CTA bulk-copies its staged partial of them into the owner's
+//      shared memory, and the owner stores the sums; rank 0 stores the KV head's d log g
+//      partial in element 1 of the dQ vector (key row, query head kvh).
 //   3. bwd_dlogg_kernel: d log g = the sum of those partials over the KV heads, in order, and
 //      d score.
 //   4. attn_bwd_dq_tc: per (128-query tile, head), walking the key tiles up to the diagonal:
@@ -47,7 +47,7 @@ using namespace sm100;
 
 constexpr int BT = 128;        // rows of every tile (keys or queries)
 constexpr int NTHREADS = 384;  // warp 0: TMA, 1: MMA + TMEM, 2: idle, 3: vector stager, 4-11: epilogue
-constexpr int MAXC = 8;        // CTAs per cluster of the dK/dV kernel
+constexpr int MAXC = 2;        // CTAs per cluster of the dK/dV kernel
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int SMEM_LIMIT = 227 * 1024;
 
@@ -104,19 +104,6 @@ __device__ __forceinline__ uint32_t mapa_rank(uint32_t local, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
-}
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
 }
 __device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
   int v;
@@ -197,8 +184,9 @@ struct KCfg {
   static constexpr int SMEM = 1024 + TAIL_OFF + TAIL;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BT, BT, false);
   static constexpr uint32_t IDESC_G = idesc_bf16_f32(BT, D, true);
-  // TMEM columns: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D)
-  static constexpr uint32_t T_DV = 256, T_DK = 256 + D;
+  // TMEM columns: region A [0, 128) holds S^T_n and then dP^T_n, P^T [128, 192) and dS^T
+  // [192, 256) (bf16, 32 columns per query half), dV [256, 256 + D), dK [256 + D, 256 + 2D)
+  static constexpr uint32_t T_P = 128, T_DS = 192, T_DV = 256, T_DK = 256 + D;
   static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
   static_assert(4 * TILE >= 2 * BT * D * 4, "the Q / dO stages hold the fp32 dK, dV partials at the end");
 };
@@ -221,14 +209,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* qempty = bars + 3;   // [2] the stage's last product (dK) read them
   uint64_t* vfull = bars + 5;    // [2] the stage's per-query vectors are staged
   uint64_t* vempty = bars + 7;   // [2] both epilogue warpgroups read them
-  uint64_t* sfull = bars + 9;    // S^T landed
-  uint64_t* dpfull = bars + 10;  // dP^T landed
+  uint64_t* sfull = bars + 9;    // S^T landed in region A
+  uint64_t* dpfull = bars + 10;  // dP^T landed in region A
   uint64_t* pready = bars + 11;  // [2] a warpgroup's half of P^T is in TMEM
   uint64_t* dsready = bars + 13; // [2] a warpgroup's half of dS^T is in TMEM
   uint64_t* accdone = bars + 15;
   uint64_t* drain = bars + 16;
   uint64_t* probe = bars + 17;   // test hook: a barrier nothing signals
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* xbar = bars + 19;    // the peer's partials of this CTA's columns landed
+  uint64_t* sfree = bars + 20;   // the epilogue holds S^T in registers: dP^T may overwrite region A
+  uint64_t* afree = bars + 21;   // the epilogue holds dP^T in registers: the next S^T may overwrite A
+  uint64_t* pfree = bars + 22;   // dV read P^T: the next P^T may overwrite it
+  uint64_t* dsfree = bars + 23;  // dK read dS^T: the next dS^T may overwrite it
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* vec_s = reinterpret_cast<float*>(tail + 256);  // [2 stages][-lse * log2(e), -Dv][128]
   float* dl_s = vec_s + 4 * BT;                         // [2 warpgroups][128]
@@ -240,7 +233,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   decode_len((int)(blockIdx.x / (unsigned)(Cn * Hkv)), p, b, L);
   const int off = p.off[b], m = p.m[b];
   const int kt = p.nt[b] - L;                 // this key tile; query tiles kt .. nt-1 see it
-  const int nh = (G - rank + Cn - 1) / Cn;    // query heads kvh G + rank + i C, i < nh
+  const int nh = G / Cn;                      // query heads kvh G + rank + i C, i < nh
   const int N = nh * L;                       // steps (head, query tile)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -258,6 +251,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(dpfull, 1);
     mbar_init(accdone, 1);
     mbar_init(drain, 1);
+    mbar_init(xbar, 1);
+    mbar_init(sfree, 256);
+    mbar_init(afree, 256);
+    mbar_init(pfree, 1);
+    mbar_init(dsfree, 1);
     *abort = 0;
     fence_barrier_init();
     wait_probe(probe, probe_ns, abort, dev_status);  // no-op unless a test asked for it
@@ -275,7 +273,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
-  bool wrote = false;        // this thread's dK / dV / d log g partials are in shared memory
+  bool done = false;         // this epilogue thread's accumulators are final
+  float dl = 0.f;            // this thread's d log g partial (its key row, its query half)
 
   // The loader / issuer warpgroup gives registers to the epilogue warpgroups:
   // 128 x 64 + 256 x 216 = 63488 <= the launch's 384 x 168 = 64512.
@@ -318,17 +317,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mma_ss(d, sdesc_sw128(a + o, 16, 1024), sdesc_sw128(bq + o, 16, 1024), C::IDESC_S, kk > 0);
           }
         };
+        // Program per step n: dP^T_n into region A once the epilogue holds S^T_n, dV_n once P^T_n
+        // is in TMEM, S^T_{n+1} into A once the epilogue holds dP^T_n, dK_n once dS^T_n is in TMEM.
         bool ok = mbar_wait(kvfull, 0, abort, dev_status) && mbar_wait(&qfull[0], 0, abort, dev_status);
         if (ok) {
           tc_fence_after();
           issue_ss(tmem + 0, ka, qa(0));  // S^T_0 = K Q_0^T
           mma_commit(sfull);
-          issue_ss(tmem + 128, va, qa(0) + C::TILE);  // dP^T_0 = V dO_0^T
-          mma_commit(dpfull);
         }
         for (int n = 0; ok && n < N; ++n) {
           const uint32_t ph = n & 1;
           const uint32_t q_a = qa(n), do_a = q_a + C::TILE;
+          if (!mbar_wait(sfree, ph, abort, dev_status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_ss(tmem + 0, va, do_a);  // dP^T_n = V dO_n^T
+          mma_commit(dpfull);
           // dV += P^T dO in the two query halves, each as soon as its P^T is in TMEM
           for (int c = 0; c < 2; ++c) {
             if (!mbar_wait(&pready[c], ph, abort, dev_status)) {
@@ -339,13 +345,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const int kk = 4 * c + k4;
-              mma_ts(tmem + C::T_DV, tmem + c * 64 + k4 * 8, sdesc_sw128(do_a + kk * 2048, BT * 128, 1024),
+              mma_ts(tmem + C::T_DV, tmem + C::T_P + c * 32 + k4 * 8, sdesc_sw128(do_a + kk * 2048, BT * 128, 1024),
                      C::IDESC_G, (n > 0 || kk > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
-          if (n + 1 < N) {  // S^T_{n+1}: overwrites P^T_n only after dV_n read it (issue order)
-            if (!mbar_wait(&qfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, dev_status)) {
+          mma_commit(pfree);
+          if (n + 1 < N) {  // S^T_{n+1} = K Q_{n+1}^T into region A
+            if (!mbar_wait(afree, ph, abort, dev_status) ||
+                !mbar_wait(&qfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, dev_status)) {
               ok = false;
               break;
             }
@@ -362,16 +370,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const int kk = 4 * c + k4;
-              mma_ts(tmem + C::T_DK, tmem + 128 + c * 64 + k4 * 8, sdesc_sw128(q_a + kk * 2048, BT * 128, 1024),
+              mma_ts(tmem + C::T_DK, tmem + C::T_DS + c * 32 + k4 * 8, sdesc_sw128(q_a + kk * 2048, BT * 128, 1024),
                      C::IDESC_G, (n > 0 || kk > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
+          mma_commit(dsfree);
           mma_commit(&qempty[n & 1]);  // the stage's Q and dO are no longer read
-          if (n + 1 < N) {             // dP^T_{n+1}: overwrites dS^T_n only after dK_n read it
-            issue_ss(tmem + 128, va, qa(n + 1) + C::TILE);
-            mma_commit(dpfull);
-          }
         }
         if (ok) mma_commit(accdone);
         mma_commit(drain);
@@ -403,12 +408,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q4 = warp & 3;
     const int kr = q4 * 32 + lane;  // key row in the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tS = tmem + lane_base + c * 64, tP = tmem + lane_base + 128 + c * 64;
+    const uint32_t tA = tmem + lane_base + c * 64;  // this half of region A (S^T, then dP^T)
+    const uint32_t tPo = tmem + lane_base + C::T_P + c * 32, tDSo = tmem + lane_base + C::T_DS + c * 32;
     const int kl = kt * BT + kr;
     const bool kvalid = kl < m;
     const float lgk = (logg && kvalid) ? logg[off + kl] : 0.f;
     const float2 qs2 = make_float2(qk_scale2, qk_scale2);
-    float dl = 0.f, racc = 0.f, gh = 1.f, bias2 = 0.f;
+    float racc = 0.f, gh = 1.f, bias2 = 0.f;
     bool ok = true;
     for (int n = 0; n < N; ++n) {
       const int s = n & 1;
@@ -426,28 +432,56 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_after();
       uint32_t xr[64];
-      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&xr[0]));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&xr[32]));
+      tmem_ld32(tA, *reinterpret_cast<uint32_t(*)[32]>(&xr[0]));
+      tmem_ld32(tA + 32, *reinterpret_cast<uint32_t(*)[32]>(&xr[32]));
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(sfree);  // region A may receive dP^T_n
       float* x = reinterpret_cast<float*>(xr);
-      const float* nl = vec_s + s * 2 * BT + c * 64;
+      const float4* nl4 = reinterpret_cast<const float4*>(vec_s + s * 2 * BT + c * 64);
       const float2 bb = make_float2(bias2, bias2);
-      const bool diag = qt == kt;
       uint32_t pk[32];
       // P^T = 2^(scale log2(e) S^T + bias - lse log2(e)); on the diagonal tile query < key is masked
+      // (a separate loop, so the other tiles carry no mask arithmetic)
+      if (qt == kt) {
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        float2 v = __ffma2_rn(make_float2(x[2 * q], x[2 * q + 1]), qs2, bb);
-        v = __fadd2_rn(v, *reinterpret_cast<const float2*>(nl + 2 * q));
-        if (diag) {
-          if (c * 64 + 2 * q < kr) v.x = -INFINITY;
-          if (c * 64 + 2 * q + 1 < kr) v.y = -INFINITY;
+        for (int q = 0; q < 16; ++q) {
+          const float4 l4 = nl4[q];
+          float2 v0 = __fadd2_rn(__ffma2_rn(make_float2(x[4 * q], x[4 * q + 1]), qs2, bb), make_float2(l4.x, l4.y));
+          float2 v1 = __fadd2_rn(__ffma2_rn(make_float2(x[4 * q + 2], x[4 * q + 3]), qs2, bb), make_float2(l4.z, l4.w));
+          const int q0 = c * 64 + 4 * q;
+          if (q0 < kr) v0.x = -INFINITY;
+          if (q0 + 1 < kr) v0.y = -INFINITY;
+          if (q0 + 2 < kr) v1.x = -INFINITY;
+          if (q0 + 3 < kr) v1.y = -INFINITY;
+          x[4 * q] = ex2(v0.x);
+          x[4 * q + 1] = ex2(v0.y);
+          x[4 * q + 2] = ex2(v1.x);
+          x[4 * q + 3] = ex2(v1.y);
+          pk[2 * q] = pack_bf16(x[4 * q], x[4 * q + 1]);
+          pk[2 * q + 1] = pack_bf16(x[4 * q + 2], x[4 * q + 3]);
         }
-        x[2 * q] = ex2(v.x);
-        x[2 * q + 1] = ex2(v.y);
-        pk[q] = pack_bf16(x[2 * q], x[2 * q + 1]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float4 l4 = nl4[q];
+          const float2 v0 = __fadd2_rn(__ffma2_rn(make_float2(x[4 * q], x[4 * q + 1]), qs2, bb), make_float2(l4.x, l4.y));
+          const float2 v1 =
+              __fadd2_rn(__ffma2_rn(make_float2(x[4 * q + 2], x[4 * q + 3]), qs2, bb), make_float2(l4.z, l4.w));
+          x[4 * q] = ex2(v0.x);
+          x[4 * q + 1] = ex2(v0.y);
+          x[4 * q + 2] = ex2(v1.x);
+          x[4 * q + 3] = ex2(v1.y);
+          pk[2 * q] = pack_bf16(x[4 * q], x[4 * q + 1]);
+          pk[2 * q + 1] = pack_bf16(x[4 * q + 2], x[4 * q + 3]);
+        }
       }
-      tmem_st32(tS, pk);
+      if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(pfree, (n - 1) & 1, abort, dev_status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st32(tPo, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&pready[c]);
@@ -457,99 +491,140 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_after();
       uint32_t yr[64];
-      tmem_ld32(tP, *reinterpret_cast<uint32_t(*)[32]>(&yr[0]));
-      tmem_ld32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&yr[32]));
+      tmem_ld32(tA, *reinterpret_cast<uint32_t(*)[32]>(&yr[0]));
+      tmem_ld32(tA + 32, *reinterpret_cast<uint32_t(*)[32]>(&yr[32]));
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(afree);  // region A may receive S^T_{n+1}
       const float* y = reinterpret_cast<const float*>(yr);
-      const float* nd = vec_s + s * 2 * BT + BT + c * 64;
+      const float4* nd4 = reinterpret_cast<const float4*>(vec_s + s * 2 * BT + BT + c * 64);
       float2 ra = make_float2(0.f, 0.f), rb = make_float2(0.f, 0.f);
       // dS^T = P^T * (dP^T - Dv), with the fp32 P^T
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const float2 d = __fadd2_rn(make_float2(y[2 * q], y[2 * q + 1]), *reinterpret_cast<const float2*>(nd + 2 * q));
-        const float2 ds = __fmul2_rn(make_float2(x[2 * q], x[2 * q + 1]), d);
-        if (q & 1) rb = __fadd2_rn(rb, ds); else ra = __fadd2_rn(ra, ds);
-        pk[q] = pack_bf16(ds.x, ds.y);
+      for (int q = 0; q < 16; ++q) {
+        const float4 d4 = nd4[q];
+        const float2 s0 = __fmul2_rn(make_float2(x[4 * q], x[4 * q + 1]),
+                                     __fadd2_rn(make_float2(y[4 * q], y[4 * q + 1]), make_float2(d4.x, d4.y)));
+        const float2 s1 = __fmul2_rn(make_float2(x[4 * q + 2], x[4 * q + 3]),
+                                     __fadd2_rn(make_float2(y[4 * q + 2], y[4 * q + 3]), make_float2(d4.z, d4.w)));
+        ra = __fadd2_rn(ra, s0);
+        rb = __fadd2_rn(rb, s1);
+        pk[2 * q] = pack_bf16(s0.x, s0.y);
+        pk[2 * q + 1] = pack_bf16(s1.x, s1.y);
       }
-      tmem_st32(tP, pk);
+      mbar_arrive(&vempty[s]);
+      if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(dsfree, (n - 1) & 1, abort, dev_status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st32(tDSo, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&dsready[c]);
-      mbar_arrive(&vempty[s]);
       racc += (ra.x + ra.y) + (rb.x + rb.y);
     }
     dl = fmaf(gh, racc, dl);
-    if (ok && __all_sync(0xffffffffu, mbar_wait(accdone, 0, abort, dev_status))) {
+    done = ok && __all_sync(0xffffffffu, mbar_wait(accdone, 0, abort, dev_status));
+    dl_s[c * BT + kr] = dl;
+    fence_proxy_async_smem();  // a bulk copy may read dl_s
+
+    // ---------------------------------------------------------- cluster reduction of dK, dV
+    // With C = 2, rank r owns the columns [r D/2, (r + 1) D/2) of dK and dV: those of its
+    // epilogue warpgroup r. Each warpgroup stages its half of dV and dK (fp32, [tensor][128
+    // rows][D/2], 16-byte slots of a row permuted by row % 8) in the freed Q / dO stages. After
+    // barrier 1 (every CTA of the pair has finished its products and copies and armed its receive
+    // barrier) the other warpgroup bulk-copies its stage into the owner's freed K / V tiles, and
+    // rank 1 its d log g partials into rank 0's freed per-query vector slots. The owner adds the
+    // two partials in rank order and stores the sums with consecutive threads on consecutive 16
+    // bytes of a row; rank 0 does the same for d log g. Barrier 2 keeps every CTA alive until the
+    // copies that read its shared memory have landed. With C = 1 every column is owned. Every CTA
+    // reaches both barriers (all waits above are bounded); a CTA that could not finish publishes
+    // a nonzero flag and then its peer neither copies nor writes results. The other warps take
+    // part in the same CTA and cluster barriers below the role branches.
+    const int bad = __syncthreads_or(!done);  // also publishes dl_s
+    constexpr int H4 = D / 8;   // 16-byte slots of a half row
+    constexpr int LH4 = D == 128 ? 4 : 3;
+    constexpr uint32_t STAGE_BYTES = 2 * BT * (D / 2) * 4;
+    float* stage = reinterpret_cast<float*>(smem + C::Q_OFF) + c * (2 * BT * (D / 2));
+    const float* rx = reinterpret_cast<const float*>(smem + C::K_OFF);  // the peer's stage of this half
+    const float* dl_rx = vec_s;                                         // rank 0: rank 1's dl_s
+    const int tw = threadIdx.x & 127;  // thread index in the warpgroup
+    const int64_t ostride = (int64_t)Hkv * D;
+    const int64_t obase = ((int64_t)(off + kt * BT) * Hkv + kvh) * D + c * (D / 2);  // row 0 of the tile, this half
+    const bool owner = Cn == 1 || c == rank;
+    if (!bad) {
       tc_fence_after();
-      // this CTA's dV and dK (fp32) into the freed Q / dO stages: [2][128 rows][D], each row's
-      // 16-byte slots permuted by row % 8 so a warp's stores (one row per lane) hit distinct banks
-      float* red = reinterpret_cast<float*>(smem + C::Q_OFF);
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-#pragma unroll 1
-        for (int col0 = c * (D / 2); col0 < (c + 1) * (D / 2); col0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + (t ? C::T_DK : C::T_DV) + col0, v);
-          tmem_wait_ld();
-          float4* rowp = reinterpret_cast<float4*>(red + (t * BT + kr) * D);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            rowp[((col0 >> 2) + i) ^ (kr & 7)] =
+      for (int t = 0; t < 2; ++t) {
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t v[16];
+          tmem_ld16(tmem + lane_base + (t ? C::T_DK : C::T_DV) + c * (D / 2) + ch * 16, v);
+          tmem_wait_ld();
+          float* row = stage + (t * BT + kr) * (D / 2);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(row + (((ch * 4 + i) ^ (kr & 7)) << 2)) =
                 make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
                             __uint_as_float(v[4 * i + 3]));
         }
       }
-      dl_s[c * BT + kr] = dl;
-      wrote = true;
+      if (!owner) fence_proxy_async_smem();  // the stage is read by a bulk copy
+      if (Cn == 2 && owner && tw == 0)
+        mbar_arrive_expect_tx(xbar, STAGE_BYTES + (rank == 0 && want_dl ? 2 * BT * 4 : 0));
     }
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();
+    tc_fence_after();
+    int any_bad = 0;
+    for (int q = 0; q < Cn; ++q) any_bad |= ld_cluster_s32(mapa_rank(smem_u32(const_cast<int*>(abort)), (uint32_t)q));
+    if (!any_bad && !owner && tw == 0) {
+      const uint32_t peer = (uint32_t)(1 - rank);
+      const uint32_t pbar = mapa_rank(smem_u32(xbar), peer);
+      bulk_copy_to_cluster(mapa_rank(smem_u32(rx), peer), smem_u32(stage), STAGE_BYTES, pbar);
+      if (rank == 1 && want_dl) bulk_copy_to_cluster(mapa_rank(smem_u32(dl_rx), peer), smem_u32(dl_s), 2 * BT * 4, pbar);
+      bulk_commit_group();
+    }
+    if (!any_bad && owner && (Cn == 1 || __all_sync(0xffffffffu, mbar_wait(xbar, 0, abort, dev_status)))) {
+      if (Cn == 1) named_bar_sync(1 + c, 128);  // the warpgroup's stage is complete
+#pragma unroll 4
+      for (int i = tw; i < 2 * BT * H4; i += 128) {
+        const int t = i >> (7 + LH4), r = (i >> LH4) & (BT - 1), x = i & (H4 - 1);
+        if (kt * BT + r >= m) continue;
+        const int o = (t * BT + r) * (D / 2) + ((x ^ (r & 7)) << 2);
+        float4 a = *reinterpret_cast<const float4*>(stage + o);
+        if (Cn == 2) {
+          const float4 pp = *reinterpret_cast<const float4*>(rx + o);
+          a = rank == 0 ? make_float4(a.x + pp.x, a.y + pp.y, a.z + pp.z, a.w + pp.w)
+                        : make_float4(pp.x + a.x, pp.y + a.y, pp.z + a.z, pp.w + a.w);
+        }
+        const float f = t ? scale : 1.f;
+        *reinterpret_cast<float4*>((t ? dK : dV) + obase + r * ostride + x * 4) =
+            make_float4(a.x * f, a.y * f, a.z * f, a.w * f);
+      }
+      if (want_dl && rank == 0 && c == 0 && kvalid) {
+        float sdl = dl_s[kr] + dl_s[BT + kr];
+        if (Cn == 2) sdl += dl_rx[kr] + dl_rx[BT + kr];
+        dQ[((int64_t)(off + kl) * Hq + kvh) * D + 1] = sdl;
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();  // the copies that read this CTA's shared memory have landed
   }
-
-  // ------------------------------------------------------------ cluster reduction of dK, dV
-  // Every CTA of the cluster reaches here (all waits above are bounded). A CTA that could not
-  // finish publishes a nonzero flag; then nobody in the cluster writes results.
-  const int bad = __syncthreads_or(!skip && warp >= 4 && !wrote) || skip;
-  if (threadIdx.x == 0) *abort = bad ? 1 : 0;
+  if (warp < 4 || skip) {  // the same barriers for the loader / issuer warps (and all warps on skip)
+    const int bad = __syncthreads_or(skip ? 1 : 0);
+    if (threadIdx.x == 0) *abort = bad ? 1 : 0;
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();
+    __syncwarp();
+    cluster_sync_all();
+  }
   tc_fence_before();
-  __syncwarp();
-  cluster_sync_all();
-  int any_bad = 0;
-  for (int q = 0; q < Cn; ++q) any_bad |= ld_cluster_s32(mapa_rank(smem_u32(const_cast<int*>(abort)), (uint32_t)q));
-  if (!any_bad) {
-    const float* red = reinterpret_cast<const float*>(smem + C::Q_OFF);
-    constexpr int D4 = D / 4;
-    const int c4a = rank * D4 / Cn, w4 = (rank + 1) * D4 / Cn - c4a;  // this rank's 16-byte columns
-    const int total = 2 * BT * w4;
-    for (int idx = threadIdx.x; idx < total; idx += NTHREADS) {
-      const int t = idx / (BT * w4), rem = idx - t * BT * w4;
-      const int row = rem / w4, c4 = c4a + rem % w4;
-      const int kl = kt * BT + row;
-      if (kl >= m) continue;
-      const uint32_t la = smem_u32(red + (t * BT + row) * D + ((c4 ^ (row & 7)) << 2));
-      float4 acc = ld_cluster_f4(mapa_rank(la, 0));
-      for (int q = 1; q < Cn; ++q) {
-        const float4 v = ld_cluster_f4(mapa_rank(la, (uint32_t)q));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
-      if (t == 1) acc = make_float4(acc.x * scale, acc.y * scale, acc.z * scale, acc.w * scale);
-      float* out = (t ? dK : dV) + ((int64_t)(off + kl) * Hkv + kvh) * D + c4 * 4;
-      *reinterpret_cast<float4*>(out) = acc;
-    }
-    if (want_dl && rank == 0 && threadIdx.x < BT) {
-      const int row = threadIdx.x, kl = kt * BT + row;
-      if (kl < m) {
-        float s = 0.f;
-        for (int q = 0; q < Cn; ++q)
-          s += ld_cluster_f32(mapa_rank(smem_u32(dl_s + row), (uint32_t)q)) +
-               ld_cluster_f32(mapa_rank(smem_u32(dl_s + BT + row), (uint32_t)q));
-        dQ[((int64_t)(off + kl) * Hq + kvh) * D + 1] = s;
-      }
-    }
-  }
-  __syncwarp();
-  cluster_sync_all();  // no CTA leaves while another still reads its shared memory
+  __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
@@ -657,8 +732,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;
 
+  // The loader / issuer warpgroup gives registers to the epilogue warpgroups:
+  // 128 x 80 + 256 x 208 = 63488 <= the launch's 384 x 168 = 64512.
   if (warp < 4) {
-    regs_dec<64>();
+    regs_dec<80>();
     if (skip) {
     } else if (warp == 0) {  // -------------------------------------------------- TMA producer
       if (lane == 0) {
@@ -760,7 +837,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (!skip) {  // ------------------------------------------------------ epilogue
-    regs_inc<216>();
+    regs_inc<208>();
     const int c = (warp - 4) >> 2;  // key half: 0 = keys 0-63 (warps 4-7), 1 = 64-127 (warps 8-11)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // query row in the tile == TMEM lane
@@ -786,19 +863,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&xr[32]));
       tmem_wait_ld();
       float* x = reinterpret_cast<float*>(xr);
-      const float* bb = bias_s + bs * BT + c * 64;
-      const bool diag = j == qt;
+      const float4* bb4 = reinterpret_cast<const float4*>(bias_s + bs * BT + c * 64);
       // P = 2^(scale log2(e) S + bias - lse log2(e)); on the diagonal tile key > query is masked
+      // (a separate loop, so the other tiles carry no mask arithmetic)
+      if (j == qt) {
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        float2 v = __ffma2_rn(make_float2(x[2 * q], x[2 * q + 1]), qs2, *reinterpret_cast<const float2*>(bb + 2 * q));
-        v = __fadd2_rn(v, nl2);
-        if (diag) {
-          if (c * 64 + 2 * q > r) v.x = -INFINITY;
-          if (c * 64 + 2 * q + 1 > r) v.y = -INFINITY;
+        for (int q = 0; q < 16; ++q) {
+          const float4 b4 = bb4[q];
+          float2 v0 = __fadd2_rn(__ffma2_rn(make_float2(x[4 * q], x[4 * q + 1]), qs2, make_float2(b4.x, b4.y)), nl2);
+          float2 v1 = __fadd2_rn(__ffma2_rn(make_float2(x[4 * q + 2], x[4 * q + 3]), qs2, make_float2(b4.z, b4.w)), nl2);
+          const int k0 = c * 64 + 4 * q;
+          if (k0 > r) v0.x = -INFINITY;
+          if (k0 + 1 > r) v0.y = -INFINITY;
+          if (k0 + 2 > r) v1.x = -INFINITY;
+          if (k0 + 3 > r) v1.y = -INFINITY;
+          x[4 * q] = ex2(v0.x);
+          x[4 * q + 1] = ex2(v0.y);
+          x[4 * q + 2] = ex2(v1.x);
+          x[4 * q + 3] = ex2(v1.y);
         }
-        x[2 * q] = ex2(v.x);
-        x[2 * q + 1] = ex2(v.y);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float4 b4 = bb4[q];
+          const float2 v0 =
+              __fadd2_rn(__ffma2_rn(make_float2(x[4 * q], x[4 * q + 1]), qs2, make_float2(b4.x, b4.y)), nl2);
+          const float2 v1 =
+              __fadd2_rn(__ffma2_rn(make_float2(x[4 * q + 2], x[4 * q + 3]), qs2, make_float2(b4.z, b4.w)), nl2);
+          x[4 * q] = ex2(v0.x);
+          x[4 * q + 1] = ex2(v0.y);
+          x[4 * q + 2] = ex2(v1.x);
+          x[4 * q + 3] = ex2(v1.y);
+        }
       }
       mbar_arrive(&bempty[bs]);
       if (!__all_sync(0xffffffffu, mbar_wait(dpfull, j & 1, abort, dev_status))) {
@@ -879,7 +975,7 @@ tg_status launch_tc_d(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaS
   if (units == 0) return TG_OK;
   const int r0 = seqs[0].off, r1 = seqs[nseq - 1].off + seqs[nseq - 1].m;
   const int G = a.Hq / a.Hkv;
-  p.C = G < MAXC ? G : MAXC;
+  p.C = G % MAXC == 0 ? MAXC : 1;  // an even number of query heads per KV head: two CTAs split them
 
   CUtensorMap tq, tk, tv, tdo;
   if (!make_tmap_bf16_2d(&tq, a.Q, (uint64_t)a.m_tot, (uint64_t)a.Hq * D, (uint64_t)a.Hq * D, BT, 64) ||

@@ -4,8 +4,9 @@ dtype (max-abs-relative 1e-4 for f32, 2e-2 for bf16).
 
 Cases cover ragged tiles and empty sequences, more KV heads than a cluster holds (16), one KV
 head (no cluster), no gate (log g absent), per-head gains, 70 sequences (two launches), the
-ragged kept counts of the four-sequence workload, and the Qwen3-1.7B shapes at N=32K, K=2K
-chained after the library's own forward. O and lse fed to the backward come from the oracle's
+ragged kept counts of the four-sequence workload, 8, 6 and 1 query heads per KV head in bf16
+(the dK/dV clusters of 8, 2 and 1 CTAs), and the Qwen3-1.7B shapes at N=32K, K=2K chained after
+the library's own forward. O and lse fed to the backward come from the oracle's
 forward (or from the library's forward in the chained case); the oracle recomputes everything
 from Q, K, V, log g and dO."""
 import math
@@ -80,6 +81,9 @@ CASES = {  # name: (seed, lens, Hq, Hkv, D, dtype, gain, with_logg)
     "bf16_qwen3_1000_rows": (5, [1000], 16, 8, 128, "bf16", True, True),
     "bf16_four_ragged": (6, [320, 456, 288, 384], 16, 8, 128, "bf16", False, True),
     "bf16_d64": (7, [130, 64], 8, 2, 64, "bf16", True, True),
+    "bf16_eight_heads_per_kv": (12, [300], 16, 2, 128, "bf16", True, True),
+    "bf16_six_heads_per_kv_d64": (13, [200, 77], 12, 2, 64, "bf16", True, True),
+    "bf16_no_grouping": (14, [150, 0, 129], 4, 4, 128, "bf16", False, True),
 }
 
 
