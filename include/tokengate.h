@@ -89,7 +89,7 @@ int32_t tg_version(void);
 
 /* Test hook for the bounded waits, off by default (limit_ns = 0). With limit_ns > 0, every
  * tensor-core kernel this calling thread launches afterwards (tg_score, tg_gated_attn_fwd,
- * tg_qkv_rope and the chain's kernels, bf16) first waits, with that limit, on a barrier that
+ * tg_qkv_rope, tg_gated_attn_bwd and the chain's kernels, bf16) first waits, with that limit, on a barrier that
  * nothing signals, before it issues any copy or product. The wait runs out, the kernel ORs
  * TG_DEV_TIMEOUT into its status word, does none of its work (its outputs are left as they
  * were) and returns; the context stays usable. Only for tests of the timeout path; set 0 to
@@ -240,7 +240,12 @@ tg_status tg_gated_attn_fwd(tg_dtype dtype, const void* Q, const void* K, const 
  *   dK, dV       device f32 [sum M_b, Hkv, D] (written)
  *   dlogg        device f32 [sum M_b] (written) or NULL
  *   dscore       device f32 [sum M_b] (written) or NULL; needs logg
- * Arithmetic is fp32 for both dtypes; no workspace; results are deterministic.
+ *   dev_status   device int32 [1] or NULL: TG_DEV_POS_NOT_ASCENDING as above; a wait of the
+ *                bf16 kernels that gave up sets TG_DEV_TIMEOUT (the gradients are then invalid)
+ * f32 runs on the CUDA cores in fp32. bf16 runs its five products on the tensor cores with fp32
+ * accumulation (P and dS rounded to bf16 as operands, as the forward rounds P); softmax,
+ * rowsum(dO * O) and d log g are fp32. dQ also holds intermediate values until the call's last
+ * kernel writes it. No workspace; results are deterministic.
  * Supported: D in {64, 128}; Hq % Hkv == 0; 16-byte aligned Q, K, V, dO, dQ, dK, dV;
  * flags without TG_ATTN_UNNORMALISED (TG_ERR_UNSUPPORTED otherwise). */
 tg_status tg_gated_attn_bwd(tg_dtype dtype, const void* Q, const void* K, const void* V,

@@ -77,6 +77,42 @@ def test_waits_run_out_and_the_context_stays_usable():
     assert st0.item() == 0
 
 
+def test_backward_waits_run_out_and_the_context_stays_usable():
+    """tg_gated_attn_bwd (bf16): with the hook on, its tensor-core kernels time out, record
+    TG_DEV_TIMEOUT and write neither dK nor dV; with the hook off the same call matches the oracle."""
+    g = np.random.default_rng(5)
+    M, Hq, Hkv, D = 300, 4, 2, 64
+    scale = 1.0 / math.sqrt(D)
+    bits = lambda *shape: ti.f32_to_bf16_bits(g.standard_normal(shape).astype(np.float32))
+    Q, K, V, dO = bits(M, Hq, D), bits(M, Hkv, D), bits(M, Hkv, D), bits(M, Hq, D)
+    logg = np.log(g.uniform(0.05, 1.0, M)).astype(np.float32)
+    pos = np.arange(M, dtype=np.int32) * 2
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    Qd, Kd, Vd, dOd = (to_dev(x, "bf16") for x in (Q, K, V, dO))
+    lg, ps = dev(logg), dev(pos)
+    O, lse = tg.tg_gated_attn_fwd(Qd, Kd, Vd, lg, ps, [0, M], scale)
+    sent = lambda shape: torch.full(shape, 5.0, device="cuda")
+    bufs = dict(dQ=sent((M, Hq, D)), dK=sent((M, Hkv, D)), dV=sent((M, Hkv, D)), dlogg=sent((M,)))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        tg.tg_set_test_wait_probe(PROBE_NS)
+        tg.tg_gated_attn_bwd(Qd, Kd, Vd, lg, ps, [0, M], O, lse, dOd, scale, dev_status=st, **bufs)
+        torch.cuda.synchronize()
+    finally:
+        tg.tg_set_test_wait_probe(0)
+    assert st.item() & tg.TG_DEV_TIMEOUT, st.item()
+    assert torch.equal(bufs["dK"], sent((M, Hkv, D))) and torch.equal(bufs["dV"], sent((M, Hkv, D)))
+
+    st0 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = tg.tg_gated_attn_bwd(Qd, Kd, Vd, lg, ps, [0, M], O, lse, dOd, scale, dev_status=st0)
+    torch.cuda.synchronize()
+    w = lambda a: ti.widen(a, "bf16")
+    ref = orc.gated_attention_bwd(w(Q), w(K), w(V), logg, pos, [0, M], Hq, Hkv, scale, w(dO))
+    for x, r in zip(got[:4], ref):
+        assert max_abs_rel(from_dev(x), r) <= TOL["bf16"]
+    assert st0.item() == 0
+
+
 def test_probe_off_by_default_and_thread_local():
     """The hook is per host thread: another thread's setting does not reach this one."""
     import threading
