@@ -131,43 +131,55 @@ __device__ __forceinline__ void settle(uint64_t* bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------ 1. Dv = rowsum(dO * O)
-// One warp per (row, query head) of rows [r0, r1); the result goes to dQ[row, h, 0]. Warps of
-// head 0 also check that positions ascend inside each sequence.
+// Vectors (row, query head) of rows [r0, r1) are contiguous D-element runs of O and dO. A warp
+// takes 4 * 32 / (D / 8) consecutive ones: each lane loads 16 bytes of a vector per load, all
+// eight loads (four of dO, four of O) in flight before the first use; the D / 8 lanes of a
+// vector add their parts with shuffles and the first writes Dv to dQ[row, h, 0]. The lanes that
+// write a head-0 vector also check that positions ascend inside each sequence.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ O,
                                                        const __nv_bfloat16* __restrict__ dO,
                                                        const int32_t* __restrict__ pos, float* __restrict__ dQ,
                                                        int r0, int r1, int Hq, int32_t* __restrict__ dev_status,
                                                        const __grid_constant__ TcParams p) {
-  constexpr int E = D / 32;  // elements per lane
+  constexpr int LPV = D / 8;     // lanes per vector (16 bytes each)
+  constexpr int VPL = 32 / LPV;  // vectors per load instruction of the warp
+  constexpr int NL = 4;          // loads per tensor per lane
+  griddep_wait();  // O and dO come from earlier work on the stream
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
-  const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t row = r0 + w / Hq;
-  const int h = (int)(w % Hq);
-  if (row >= r1) return;
-  const int64_t base = (row * Hq + h) * D + lane * E;
-  float s = 0.f;
-  if constexpr (E == 4) {
-    const uint2 a = *reinterpret_cast<const uint2*>(dO + base);
-    const uint2 o = *reinterpret_cast<const uint2*>(O + base);
-    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
-    const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
-    const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
-    const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
-    s = fmaf(a0.x, o0.x, fmaf(a0.y, o0.y, fmaf(a1.x, o1.x, a1.y * o1.y)));
-  } else {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dO + base));
-    const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(O + base));
-    s = fmaf(a.x, o.x, a.y * o.y);
+  const int64_t v_end = (int64_t)r1 * Hq;
+  const int64_t vw = (int64_t)r0 * Hq + ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (VPL * NL);
+  uint4 a[NL], o[NL];
+#pragma unroll
+  for (int j = 0; j < NL; ++j) {
+    const int64_t v = vw + j * VPL + lane / LPV;
+    const int64_t e = v * D + (lane % LPV) * 8;
+    a[j] = v < v_end ? *reinterpret_cast<const uint4*>(dO + e) : make_uint4(0, 0, 0, 0);
+    o[j] = v < v_end ? *reinterpret_cast<const uint4*>(O + e) : make_uint4(0, 0, 0, 0);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) {
-    dQ[(row * Hq + h) * D] = s;
-    if (h == 0 && dev_status) {
-      bool start = false;
-      for (int i = 0; i < p.nseq; ++i) start |= p.off[i] == row;
-      if (!start && pos[row - 1] >= pos[row]) atomicOr(dev_status, TG_DEV_POS_NOT_ASCENDING);
+  for (int j = 0; j < NL; ++j) {
+    const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a[j]);
+    const uint32_t* ow = reinterpret_cast<const uint32_t*>(&o[j]);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[i]));
+      const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[i]));
+      s = fmaf(x.x, y.x, fmaf(x.y, y.y, s));
+    }
+#pragma unroll
+    for (int m = LPV / 2; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+    const int64_t v = vw + j * VPL + lane / LPV;
+    if (lane % LPV == 0 && v < v_end) {
+      dQ[v * D] = s;
+      const int64_t row = v / Hq;
+      if (v % Hq == 0 && dev_status) {
+        bool start = false;
+        for (int i = 0; i < p.nseq; ++i) start |= p.off[i] == row;
+        if (!start && pos[row - 1] >= pos[row]) atomicOr(dev_status, TG_DEV_POS_NOT_ASCENDING);
+      }
     }
   }
 }
@@ -271,6 +283,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_launch_dependents();  // the next kernel may start its prologue
+  griddep_wait();               // what earlier kernels wrote is visible from here on
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
   bool done = false;         // this epilogue thread's accumulators are final
@@ -633,6 +647,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 __global__ void __launch_bounds__(256) bwd_dlogg_kernel(const float* __restrict__ dQ, const float* __restrict__ logg,
                                                         float* __restrict__ dlogg, float* __restrict__ dscore, int r0,
                                                         int r1, int Hq, int Hkv, int D) {
+  griddep_launch_dependents();  // the dQ kernel may start its prologue
+  griddep_wait();               // the dK/dV kernel's partials are visible from here on
   const int64_t row = r0 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= r1) return;
   float s = 0.f;
@@ -729,6 +745,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_launch_dependents();  // the next kernel may start its prologue
+  griddep_wait();               // what earlier kernels wrote is visible from here on
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;
 
@@ -998,10 +1016,18 @@ tg_status launch_tc_d(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaS
   const uint64_t probe = wait_probe_ns();
   const float qk2 = a.scale * kLog2e;
 
-  // 1. Dv into dQ[., ., 0]
-  const int64_t warps = (int64_t)(r1 - r0) * a.Hq;
-  bwd_prep_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(O, dO, a.pos, a.dQ, r0, r1, a.Hq, a.dev_status, p);
-  cudaError_t e = cudaGetLastError();
+  // Every launch may start early (programmatic dependent launch): each kernel waits on the
+  // previous one before it touches memory that kernel or earlier work writes.
+  cudaLaunchAttribute pdl[1] = {pdl_attribute(PDL_BWD)};
+  // 1. Dv into dQ[., ., 0]: warps of 4 * 32 / (D / 8) vectors
+  const int64_t nvec = (int64_t)(r1 - r0) * a.Hq, per_block = 8 * 4 * (32 / (D / 8));
+  cudaLaunchConfig_t cp = {};
+  cp.gridDim = dim3((unsigned)((nvec + per_block - 1) / per_block));
+  cp.blockDim = dim3(256);
+  cp.stream = st;
+  cp.attrs = pdl;
+  cp.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cp, bwd_prep_kernel<D>, O, dO, a.pos, a.dQ, r0, r1, a.Hq, a.dev_status, p);
   if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: prep launch");
 
   // 2. dK, dV: clusters of C CTAs over the query heads of one (key tile, KV head)
@@ -1012,13 +1038,14 @@ tg_status launch_tc_d(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaS
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = (size_t)KC::SMEM;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)p.C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl[0];
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kdkdv, tq, tk, tv, tdo, a.logg, a.head_gain, a.lse, a.dQ, a.dK, a.dV, a.m_tot, a.Hq,
                            a.Hkv, qk2, a.scale, want_dl, a.dev_status, probe, p);
     if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: dK/dV launch");
@@ -1026,9 +1053,13 @@ tg_status launch_tc_d(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaS
 
   // 3. d log g, d score
   if (want_dl) {
-    bwd_dlogg_kernel<<<(unsigned)((r1 - r0 + 255) / 256), 256, 0, st>>>(a.dQ, a.logg, a.dlogg, a.dscore, r0, r1, a.Hq,
-                                                                         a.Hkv, D);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cl = {};
+    cl.gridDim = dim3((unsigned)((r1 - r0 + 255) / 256));
+    cl.blockDim = dim3(256);
+    cl.stream = st;
+    cl.attrs = pdl;
+    cl.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cl, bwd_dlogg_kernel, (const float*)a.dQ, a.logg, a.dlogg, a.dscore, r0, r1, a.Hq, a.Hkv, D);
     if (e != cudaSuccess) return cuda_status(e, "tg_gated_attn_bwd: d log g launch");
   }
 
@@ -1039,6 +1070,8 @@ tg_status launch_tc_d(const AttnBwdArgs& a, const AttnSeq* seqs, int nseq, cudaS
     cq.blockDim = dim3(NTHREADS);
     cq.dynamicSmemBytes = (size_t)QC::SMEM;
     cq.stream = st;
+    cq.attrs = pdl;
+    cq.numAttrs = 1;
     e = cudaLaunchKernelEx(&cq, kdq, tq, tk, tv, tdo, a.logg, a.head_gain, a.lse, a.dQ, a.m_tot, a.Hq, a.Hkv, qk2,
                            a.scale, a.dev_status, probe, p);
   }

@@ -88,7 +88,7 @@ bool pdl_enabled(int kernel_id) {
   if (mask < 0) {
     const char* off = getenv("TG_DISABLE_PDL");
     const char* m = getenv("TG_PDL_MASK");
-    mask = (off && off[0] && off[0] != '0') ? 0 : (m ? atoi(m) : 31);
+    mask = (off && off[0] && off[0] != '0') ? 0 : (m ? atoi(m) : 63);
   }
   return (mask & kernel_id) != 0;
 }
