@@ -283,8 +283,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The pre-pass waited for all earlier work on the stream, and this grid starts only after every
+  // pre-pass block has done so: Q, K, V, dO, lse and log g may be read at once, and the outputs
+  // written. Only the per-query stager reads what the pre-pass writes (Dv), after its wait.
   griddep_launch_dependents();  // the next kernel may start its prologue
-  griddep_wait();               // what earlier kernels wrote is visible from here on
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;  // only the test probe sets it this early: nothing was issued
   bool done = false;         // this epilogue thread's accumulators are final
@@ -399,6 +401,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else if (warp == 3) {  // ----------------------------------- per-query vectors stager
       // -lse * log2(e) (-inf for rows past the sequence, whose lse reads as +inf) and -Dv of
       // the step's 128 queries, 4 per lane, into the stage's slots.
+      griddep_wait();  // Dv of the pre-pass is visible from here on
       for (int n = 0; n < N; ++n) {
         const int s = n & 1;
         const int h = kvh * G + rank + (n / L) * Cn, qt = kt + n % L;
@@ -426,7 +429,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tPo = tmem + lane_base + C::T_P + c * 32, tDSo = tmem + lane_base + C::T_DS + c * 32;
     const int kl = kt * BT + kr;
     const bool kvalid = kl < m;
-    const float lgk = (logg && kvalid) ? logg[off + kl] : 0.f;
+    const float lgk = (logg && kvalid) ? __ldcg(logg + off + kl) : 0.f;
     const float2 qs2 = make_float2(qk_scale2, qk_scale2);
     float racc = 0.f, gh = 1.f, bias2 = 0.f;
     bool ok = true;
@@ -436,7 +439,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (n % L == 0) {  // a new query head
         dl = fmaf(gh, racc, dl);
         racc = 0.f;
-        gh = gain ? gain[kvh * G + rank + (n / L) * Cn] : 1.f;
+        gh = gain ? __ldcg(gain + kvh * G + rank + (n / L) * Cn) : 1.f;
         bias2 = kvalid ? key_bias(gh * kLog2e, lgk) : -INFINITY;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&vfull[s], (n >> 1) & 1, abort, dev_status) &&
@@ -745,8 +748,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_launch_dependents();  // the next kernel may start its prologue
-  griddep_wait();               // what earlier kernels wrote is visible from here on
+  // The tiles (Q, dO, K, V) and the per-key bias are inputs of the call, complete before the
+  // pre-pass passed its wait; only the epilogue reads (Dv) and writes (dQ) memory that the
+  // kernels before this one write, after its wait.
+  griddep_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort;
 
@@ -840,14 +845,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         settle(drain, 0);
       }
     } else if (warp == 3) {  // ------------------------------------------- key bias stager
-      const float gain2 = (gain ? gain[h] : 1.f) * kLog2e;
+      const float gain2 = (gain ? __ldcg(gain + h) : 1.f) * kLog2e;
       for (int j = 0; j < N; ++j) {
         const int bs = j & 1;
         float bv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int kl = j * BT + lane * 4 + e;
-          bv[e] = kl < m ? (logg ? key_bias(gain2, logg[off + kl]) : 0.f) : -INFINITY;
+          bv[e] = kl < m ? (logg ? key_bias(gain2, __ldcg(logg + off + kl)) : 0.f) : -INFINITY;
         }
         if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bempty[bs], ((j >> 1) - 1) & 1, abort, dev_status))) break;
         *reinterpret_cast<float4*>(bias_s + bs * BT + lane * 4) = make_float4(bv[0], bv[1], bv[2], bv[3]);
@@ -863,7 +868,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tP = tmem + lane_base + C::T_DP + c * 64;
     const int il = qt * BT + r;
     const bool valid = il < m;
-    const float nlse2 = valid ? -lse_or_inf(lse[(int64_t)h * m_tot + off + il]) * kLog2e : -INFINITY;
+    const float nlse2 = valid ? -lse_or_inf(__ldcg(lse + (int64_t)h * m_tot + off + il)) * kLog2e : -INFINITY;
+    griddep_wait();  // Dv, and the d log g partials in dQ, are final from here on
     const float ndv = valid ? -dQ[((int64_t)(off + il) * Hq + h) * D] : 0.f;  // read before any dQ write below
     const float2 qs2 = make_float2(qk_scale2, qk_scale2), nl2 = make_float2(nlse2, nlse2), nd2 = make_float2(ndv, ndv);
     bool ok = true;
