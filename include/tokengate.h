@@ -89,7 +89,8 @@ int32_t tg_version(void);
 
 /* Test hook for the bounded waits, off by default (limit_ns = 0). With limit_ns > 0, every
  * tensor-core kernel this calling thread launches afterwards (tg_score, tg_gated_attn_fwd,
- * tg_qkv_rope, tg_gated_attn_bwd and the chain's kernels, bf16) first waits, with that limit, on a barrier that
+ * tg_qkv_rope, tg_gated_attn_bwd, the tensor-core kernels of tg_gate_mlp_bwd and the chain's
+ * kernels, bf16) first waits, with that limit, on a barrier that
  * nothing signals, before it issues any copy or product. The wait runs out, the kernel ORs
  * TG_DEV_TIMEOUT into its status word, does none of its work (its outputs are left as they
  * were) and returns; the context stays usable. Only for tests of the timeout path; set 0 to
@@ -274,13 +275,19 @@ size_t tg_gate_mlp_bwd_workspace_size(int64_t M, int32_t d, int32_t dg);
  *   ws       device workspace of at least tg_gate_mlp_bwd_workspace_size(M, d, dg) bytes,
  *            256-byte aligned (TG_ERR_WORKSPACE otherwise); owned by the caller, contents need
  *            no initialisation and are overwritten
- * Arithmetic is fp32 on the CUDA cores; results are deterministic (fixed reduction orders).
- * M = 0 writes zero gradients. Supported: d % 64 == 0, dg % 64 == 0, 16-byte aligned H_kept,
- * W1 and dW1. */
+ *   dev_status device int32 [1] or NULL: a wait of the bf16 tensor-core kernels that gave up
+ *            ORs in TG_DEV_TIMEOUT, and their last kernel then writes none of the outputs (it also
+ *            writes none when the word already holds TG_DEV_TIMEOUT); with NULL a timed-out call
+ *            leaves invalid gradients. The CUDA-core kernels do not wait and never set it.
+ * Arithmetic: bf16 with dg % 128 == 0 and d % 128 == 0 runs on the 5th-generation tensor cores
+ * (z = H W1^T and dW1 = u^T H with fp32 accumulation; u is rounded to bf16 as the second
+ * product's operand, db1, dw2 and db2 add fp32 values); every other shape, and f32, is fp32 on the
+ * CUDA cores. Results are deterministic (fixed reduction orders). M = 0 writes zero gradients.
+ * Supported: d % 64 == 0, dg % 64 == 0, 16-byte aligned H_kept, W1 and dW1. */
 tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W1,
                           const float* b1, const void* w2, float temperature, int32_t dg,
                           const float* dscore, float* dW1, float* db1, float* dw2, float* db2,
-                          void* ws, size_t ws_bytes, void* stream);
+                          void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* Size of the fixed device scratch array behind tg_gate_mlp_bwd_noalloc (16 MiB). */
 #define TG_GATE_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -305,7 +312,7 @@ tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t
 tg_status tg_gate_mlp_bwd_noalloc(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d,
                                   const void* W1, const float* b1, const void* w2, float temperature,
                                   int32_t dg, const float* dscore, float* dW1, float* db1,
-                                  float* dw2, float* db2, void* stream);
+                                  float* dw2, float* db2, int32_t* dev_status, void* stream);
 
 /* The whole gated path above layer L (aitualizate.com TokenGate article, phases 2-3;
  * thelatestinai.com TokenGate page, Figure 1(a)): the results of tg_score -> tg_topk_select

@@ -87,7 +87,7 @@ def lib() -> ctypes.CDLL:
     L.tg_gate_mlp_bwd_workspace_size.argtypes = [_I64, _I32, _I32]
     L.tg_gate_mlp_bwd.restype = _I32
     L.tg_gate_mlp_bwd.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP, _VP, _VP, _VP, _VP,
-                                  ctypes.c_size_t, _VP]
+                                  ctypes.c_size_t, _VP, _VP]
     L.tg_prefill_projected.restype = _I32
     L.tg_prefill_projected.argtypes = [
         _I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _F, _I32, _SEQP, _I32, ctypes.POINTER(_VP), _F,
@@ -96,7 +96,7 @@ def lib() -> ctypes.CDLL:
         _VP, _VP]
     L.tg_gate_mlp_bwd_noalloc.restype = _I32
     L.tg_gate_mlp_bwd_noalloc.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _VP, _F, _I32, _VP, _VP, _VP, _VP, _VP,
-                                          _VP]
+                                          _VP, _VP]
     L.tg_set_test_wait_probe.restype = _I32
     L.tg_set_test_wait_probe.argtypes = [_I64]
     L.tg_topk_select.restype = _I32
@@ -393,11 +393,13 @@ def tg_gated_attn_bwd(Q, K, V, logg, pos, cu_kept, O, lse, dO, softmax_scale: fl
 
 
 def tg_gate_mlp_bwd(H_kept, W1, b1, w2, dscore, temperature: float = 1.0, dW1=None, db1=None, dw2=None, db2=None,
-                    ws=None, stream=None):
+                    ws=None, dev_status=None, stream=None):
     """Gradients of the gate network's parameters from d score of the kept rows:
     (dW1 [dg, d], db1 [dg], dw2 [dg], db2 [1]), all float32. ``ws`` is a uint8 device buffer of
-    at least tg_gate_mlp_bwd_workspace_size bytes (allocated here when not given)."""
+    at least tg_gate_mlp_bwd_workspace_size bytes (allocated here when not given);
+    ``dev_status`` an int32 device word that a timed-out wait ORs TG_DEV_TIMEOUT into."""
     _want(torch.float32, b1=b1, dscore=dscore, dW1=dW1, db1=db1, dw2=dw2, db2=db2)
+    _want(torch.int32, dev_status=dev_status)
     M, d = H_kept.shape
     dg = W1.shape[0]
     _contig(H_kept=H_kept, W1=W1, w2=w2)
@@ -408,7 +410,7 @@ def tg_gate_mlp_bwd(H_kept, W1, b1, w2, dscore, temperature: float = 1.0, dW1=No
     for name, t in (("b1", b1), ("db1", db1), ("dw2", dw2)):
         if t is not None:
             _shape(name, t, (dg,))
-    _cuda(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, ws)
+    _cuda(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, ws, dev_status)
     dev = H_kept.device
     f32 = torch.float32
     dW1 = torch.empty(dg, d, device=dev, dtype=f32) if dW1 is None else dW1
@@ -420,11 +422,13 @@ def tg_gate_mlp_bwd(H_kept, W1, b1, w2, dscore, temperature: float = 1.0, dW1=No
         ws = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
     _check("tg_gate_mlp_bwd", lib().tg_gate_mlp_bwd(
         _dtype(H_kept), _ptr(H_kept), M, d, _ptr(W1), _ptr(b1), _ptr(w2), float(temperature), dg, _ptr(dscore),
-        _ptr(dW1), _ptr(db1), _ptr(dw2), _ptr(db2), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+        _ptr(dW1), _ptr(db1), _ptr(dw2), _ptr(db2), _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status),
+        _stream(stream)))
     return dW1, db1, dw2, db2
 
 
-def tg_gate_mlp_bwd_noalloc(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, temperature: float = 1.0, stream=None):
+def tg_gate_mlp_bwd_noalloc(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, temperature: float = 1.0,
+                            dev_status=None, stream=None):
     """tg_gate_mlp_bwd for callers that cannot allocate: the library's fixed scratch array takes
     the place of the workspace, and every output buffer is the caller's (nothing is allocated
     here either). Calls on one device share the array: do not let them overlap on the GPU."""
@@ -435,10 +439,11 @@ def tg_gate_mlp_bwd_noalloc(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, temp
     _shape("W1", W1, (dg, d))
     _shape("dW1", dW1, (dg, d))
     _len_at_least("dscore", dscore, M)
-    _cuda(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2)
+    _want(torch.int32, dev_status=dev_status)
+    _cuda(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, dev_status)
     _check("tg_gate_mlp_bwd_noalloc", lib().tg_gate_mlp_bwd_noalloc(
         _dtype(H_kept), _ptr(H_kept), M, d, _ptr(W1), _ptr(b1), _ptr(w2), float(temperature), dg, _ptr(dscore),
-        _ptr(dW1), _ptr(db1), _ptr(dw2), _ptr(db2), _stream(stream)))
+        _ptr(dW1), _ptr(db1), _ptr(dw2), _ptr(db2), _ptr(dev_status), _stream(stream)))
     return dW1, db1, dw2, db2
 
 

@@ -424,7 +424,7 @@ size_t tg_gate_mlp_bwd_workspace_size(int64_t M, int32_t d, int32_t dg) {
 tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W1,
                           const float* b1, const void* w2, float temperature, int32_t dg, const float* dscore,
                           float* dW1, float* db1, float* dw2, float* db2, void* ws, size_t ws_bytes,
-                          void* stream) {
+                          int32_t* dev_status, void* stream) {
   g_err[0] = 0;
   tg_status st = gate_bwd_check(dtype, M, d, dg, temperature);
   if (st != TG_OK) return st;
@@ -440,25 +440,27 @@ tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t
   if (!H_kept || !W1 || !w2 || !dscore) return fail(TG_ERR_INVALID_ARG, "H_kept, W1, w2 and dscore are required");
   if (!aligned16(H_kept) || !aligned16(W1) || !aligned16(dW1))
     return fail(TG_ERR_UNSUPPORTED, "H_kept, W1 and dW1 must be 16-byte aligned");
-  const GateBwdPlan p = gate_bwd_plan(M, d, dg, device_sm_count());
+  const int sms = device_sm_count();
+  const GateBwdPlan p = gate_bwd_plan(M, d, dg, sms);
   if (!ws || ws_bytes < (size_t)p.bytes || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(TG_ERR_WORKSPACE, "the workspace needs %lld bytes at a 256-byte aligned address",
                 (long long)p.bytes);
   st = check_device();
   if (st != TG_OK) return st;
   return launch_gate_bwd(dtype, H_kept, M, d, W1, b1, w2, (float)(1.0 / (double)temperature), dg, dscore, dW1, db1,
-                         dw2, db2, ws, p, (cudaStream_t)stream);
+                         dw2, db2, ws, p, sms, dev_status, (cudaStream_t)stream);
 }
 
 tg_status tg_gate_mlp_bwd_noalloc(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W1,
                                   const float* b1, const void* w2, float temperature, int32_t dg,
                                   const float* dscore, float* dW1, float* db1, float* dw2, float* db2,
-                                  void* stream) {
+                                  int32_t* dev_status, void* stream) {
   g_err[0] = 0;
   tg_status st = gate_bwd_check(dtype, M, d, dg, temperature);
   if (st != TG_OK) return st;
   if (M > 0) {
-    const GateBwdPlan p = gate_bwd_plan(M, d, dg, device_sm_count());
+    const int sms = device_sm_count();
+    const GateBwdPlan p = gate_bwd_plan(M, d, dg, sms);
     if (p.bytes > (int64_t)TG_GATE_NOALLOC_SCRATCH_BYTES)
       return fail(TG_ERR_UNSUPPORTED,
                   "tg_gate_mlp_bwd_noalloc: M=%lld, d=%d, dg=%d need %lld bytes of scratch, more than the fixed "
@@ -474,11 +476,11 @@ tg_status tg_gate_mlp_bwd_noalloc(tg_dtype dtype, const void* H_kept, int64_t M,
     st = gate_bwd_fixed_scratch(&scratch);
     if (st != TG_OK) return st;
     return launch_gate_bwd(dtype, H_kept, M, d, W1, b1, w2, (float)(1.0 / (double)temperature), dg, dscore, dW1,
-                           db1, dw2, db2, scratch, p, (cudaStream_t)stream);
+                           db1, dw2, db2, scratch, p, sms, dev_status, (cudaStream_t)stream);
   }
   // no rows: the workspace entry point writes the zero gradients without touching any workspace
   return tg_gate_mlp_bwd(dtype, H_kept, M, d, W1, b1, w2, temperature, dg, dscore, dW1, db1, dw2, db2, nullptr, 0,
-                         stream);
+                         dev_status, stream);
 }
 
 // The row copy of the chained prefill (the selector already wrote pos, g and log g): launched

@@ -8,7 +8,8 @@
 //   dW1 = sum_rows u h^T,  db1 = sum_rows u,  dw2 = sum_rows ds' GELU(z),  db2 = sum_rows ds'.
 //
 // Three kernels, fp32 arithmetic on the CUDA cores, deterministic (fixed reduction orders, no
-// atomics), with a caller-provided workspace:
+// atomics), with a caller-provided workspace; f32 operands, and bf16 shapes the tensor-core
+// kernels (csrc/tg_gate_bwd_tc.cu: dg and d multiples of 128) do not take:
 //   * rows:   one CTA per (64-row tile, 64-column block of dg) forms z = H W1^T + b1 in fp32
 //             from bf16/f32 operands staged through shared memory (k-major, so each thread reads
 //             its 4 rows and 4 columns as two 16-byte words), then u into the workspace and the
@@ -243,12 +244,19 @@ GateBwdPlan gate_bwd_plan(int64_t M, int d, int dg, int sms) {
   p.off_part = align256(M * (int64_t)dg * 4);
   p.off_w = p.off_part + align256(2 * (int64_t)p.n_tiles * dg * 4);
   p.bytes = p.off_w + (splits > 1 ? align256((int64_t)splits * dg * d * 4) : 0);
+  if (gate_bwd_tc_shape(M, d, dg)) {
+    gate_bwd_tc_plan(p, M, d, dg, sms);
+    if (p.tc_bytes > p.bytes) p.bytes = p.tc_bytes;
+  }
   return p;
 }
 
 tg_status launch_gate_bwd(tg_dtype dt, const void* H, int64_t M, int d, const void* W1, const float* b1,
                           const void* w2, float inv_t, int dg, const float* dscore, float* dW1, float* db1,
-                          float* dw2, float* db2, void* ws, const GateBwdPlan& p, cudaStream_t st) {
+                          float* dw2, float* db2, void* ws, const GateBwdPlan& p, int sms, int32_t* dev_status,
+                          cudaStream_t st) {
+  if (dt == TG_BF16 && p.tc)
+    return launch_gate_bwd_tc(H, M, d, W1, b1, w2, inv_t, dg, dscore, dW1, db1, dw2, db2, ws, p, sms, dev_status, st);
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* U = reinterpret_cast<float*>(base);
   float* part_db1 = reinterpret_cast<float*>(base + p.off_part);

@@ -1,0 +1,514 @@
+// Gradients of the gate network's parameters on the 5th-generation tensor cores (bf16 H, W1, w2).
+//
+// TokenGate paper page (thelatestinai.com), Figure 1(c): the gated attention lets the top-K
+// selector learn end to end; aitualizate.com article, section on training the top-K selection.
+// With s = (w2 . GELU(W1 h + b1) + b2) / T and the upstream d score of each kept row:
+//   z = W1 h + b1,  ds' = dscore / T,  u = ds' w2 * GELU'(z),  q = ds' GELU(z)  (per row, dg values),
+//   dW1 = sum_rows u h^T,  db1 = sum_rows u,  dw2 = sum_rows q,  db2 = sum_rows ds'.
+//
+// Three kernels, deterministic (fixed reduction orders, no atomics), caller workspace:
+//   1. gate_z_tc: per (128 kept rows, ZN columns of dg), z = H W1^T (M = 128, N = ZN, K = d,
+//      both operands K-major as stored, fp32 in TMEM; ZN = 32, 64 or 128, the narrowest that
+//      keeps the grid within one wave, since the epilogue is the longer part of a CTA's work). The epilogue (one row per thread) forms
+//      u and q, stores u transposed in bf16 (the next product's A operand; rows past M are zero)
+//      and adds u and q over the warp's 32 rows (a fixed butterfly that leaves column c0 + l in
+//      lane l), one partial per warp and column.
+//   2. gate_dw1_tc: per (128 rows of dg, 128 columns of d, split of the kept rows),
+//      dW1 = u^T H (M = 128, N = 128, K = kept rows in chunks of 64; H is the N-contiguous B
+//      operand). With more than one split each writes a partial block; the fp32 tile leaves
+//      through shared memory in row-contiguous runs.
+//   3. gate_reduce_tc: the splits' blocks in split order; db1 and dw2 from the warp partials in
+//      row order; db2 = T^-1 sum dscore.
+// u is rounded to bf16 for the second product (its fp32 value feeds db1); the products accumulate
+// in fp32. Every wait is bounded; on a timeout a CTA records TG_DEV_TIMEOUT, drains its copies and
+// products, frees TMEM and returns, and the reduction writes no output (given a status word).
+#include <cuda_bf16.h>
+
+#include "tg_gate_bwd.cuh"
+#include "tg_sm100.cuh"
+
+namespace tg {
+namespace {
+
+using namespace sm100;
+
+constexpr int GT = 128;        // rows of a product tile (kept rows in pass 1, rows of dg in pass 2)
+constexpr int GN = 128;        // columns of d per pass-2 tile
+constexpr int KCH = 64;        // K elements per pipeline stage (one 128-byte swizzle row)
+constexpr int WST = 6;         // pass-2 stages (32 KB each)
+constexpr int GTHREADS = 192;  // warp 0: TMA, 1: MMA + TMEM, 2-5: epilogue (TMEM lane quarters 2, 3, 0, 1)
+constexpr int MAX_SPLITS = 4;
+
+__device__ __forceinline__ float gelu_exact(float z) { return 0.5f * z * (1.f + erff(z * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_grad(float z) {
+  return 0.5f * (1.f + erff(z * 0.70710678118654752f)) + z * 0.39894228040143268f * expf(-0.5f * z * z);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Bounded wait used only while draining after an abort (one second at most).
+__device__ __forceinline__ void settle(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < 1000000000ull) {
+  }
+}
+
+// Sums v[i] over the 32 lanes for every i: afterwards v[0] of lane l holds the sum of v[l]. At the
+// step with offset o a lane keeps the half of its live values whose index has bit o equal to its
+// own lane's bit o and adds the partner's values for that half.
+__device__ __forceinline__ void lane_transpose_sum(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const bool hi = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = hi ? v[i] : v[i + o];
+      const float keep = hi ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
+
+// The CTA's barriers and TMEM slot sit after the stages.
+struct Ctl {
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* accdone;
+  uint64_t* drain;
+  uint64_t* probe;  // test hook: a barrier nothing signals
+  uint32_t* tmem_slot;
+  volatile int* abort;
+};
+
+template <int NS>
+__device__ __forceinline__ Ctl ctl_at(uint8_t* p) {
+  Ctl c;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p);
+  c.full = bars;
+  c.empty = bars + NS;
+  c.accdone = bars + 2 * NS;
+  c.drain = bars + 2 * NS + 1;
+  c.probe = bars + 2 * NS + 2;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 3);
+  c.abort = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
+  return c;
+}
+
+// Thread 0: the barriers, then the test probe's wait (a no-op unless a test asked for it; it runs
+// before any copy or product is issued, so a CTA that then skips its work has nothing in flight).
+template <int NS>
+__device__ __forceinline__ void ctl_init(const Ctl& c, uint64_t probe_ns, int32_t* dev_status) {
+  for (int s = 0; s < NS; ++s) {
+    mbar_init(&c.full[s], 1);
+    mbar_init(&c.empty[s], 1);
+  }
+  mbar_init(c.accdone, 1);
+  mbar_init(c.drain, 1);
+  *c.abort = 0;
+  fence_barrier_init();
+  wait_probe(c.probe, probe_ns, c.abort, dev_status);
+}
+
+// After an abort, the producer waits (bounded) for the copies it issued that nobody consumed.
+template <int NS>
+__device__ __forceinline__ void drain_copies(const Ctl& c, int issued) {
+  for (int k = issued - NS < 0 ? 0 : issued - NS; k < issued; ++k) settle(&c.full[k % NS], (k / NS) & 1);
+}
+
+// ------------------------------------------------------------------ 1. z, u, q per 128 x ZN tile
+template <int ZN>
+struct ZCfg {
+  static constexpr int A_BYTES = GT * KCH * 2;  // 128 kept rows x 64 columns of H
+  static constexpr int B_BYTES = ZN * KCH * 2;  // ZN rows of W1 x 64 columns
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int NS = (200 * 1024) / STAGE < 8 ? (200 * 1024) / STAGE : 8;
+  static constexpr int SMEM = 1024 + NS * STAGE + 256;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(GT, ZN, false);
+  static_assert(ZN % 32 == 0 && ZN >= 32 && ZN <= 256, "TMEM columns and loads of 32");
+  static_assert(STAGE % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+// grid (Mp / 128, dg / ZN). part: [2][4 * (Mp / 128)][dg] fp32, the u sums then the q sums, one
+// row per (row tile, epilogue warp).
+template <int ZN>
+__global__ void __launch_bounds__(GTHREADS, 1)
+    gate_z_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW, int M, int d, int dg,
+              const float* __restrict__ b1, const __nv_bfloat16* __restrict__ w2, float inv_t,
+              const float* __restrict__ dscore, __nv_bfloat16* __restrict__ uT, int Mp, float* __restrict__ part,
+              int32_t* __restrict__ dev_status, uint64_t probe_ns) {
+  using C = ZCfg<ZN>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const Ctl ct = ctl_at<NS>(smem + NS * C::STAGE);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, cb = blockIdx.y, nk = d / KCH;
+  if (threadIdx.x == 0) {
+    ctl_init<NS>(ct, probe_ns, dev_status);
+    prefetch_tmap(&tmH);
+    prefetch_tmap(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(ct.tmem_slot, ZN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  griddep_launch_dependents();
+  griddep_wait();  // the d score and the workspace's earlier readers are done from here on
+  const uint32_t tmem = *ct.tmem_slot;
+  const bool skip = *ct.abort;  // only the test probe sets it this early
+  if (skip) {
+  } else if (warp == 0) {  // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      int issued = 0;
+      for (int kc = 0; kc < nk; ++kc) {
+        const int s = kc % NS;
+        if (kc >= NS && !mbar_wait(&ct.empty[s], ((kc / NS) - 1) & 1, ct.abort, dev_status)) break;
+        uint8_t* st = smem + s * C::STAGE;
+        mbar_arrive_expect_tx(&ct.full[s], C::STAGE);
+        tma_load_2d(st, &tmH, kc * KCH, tile * GT, &ct.full[s]);
+        tma_load_2d(st + C::A_BYTES, &tmW, kc * KCH, cb * ZN, &ct.full[s]);
+        ++issued;
+      }
+      if (*ct.abort) drain_copies<NS>(ct, issued);
+    }
+  } else if (warp == 1) {  // -------------------------------------------------------- MMA
+    if (lane == 0) {
+      bool ok = true;
+      for (int kc = 0; kc < nk; ++kc) {
+        const int s = kc % NS;
+        if (!mbar_wait(&ct.full[s], (kc / NS) & 1, ct.abort, dev_status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + s * C::STAGE), b = a + C::A_BYTES;
+#pragma unroll
+        for (int k = 0; k < KCH / 16; ++k)
+          mma_ss(tmem, sdesc_sw128(a + k * 32, 16, 1024), sdesc_sw128(b + k * 32, 16, 1024), C::IDESC,
+                 (kc > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&ct.empty[s]);
+      }
+      if (ok) mma_commit(ct.accdone);
+      mma_commit(ct.drain);
+      settle(ct.drain, 0);
+    }
+  } else {  // ------------------------------------------------------ epilogue: one row per thread
+    const int q4 = warp & 3, r = q4 * 32 + lane, t = tile * GT + r;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const bool valid = t < M;
+    const float dsp = valid ? __ldcg(dscore + t) * inv_t : 0.f;
+    float* pu = part + (int64_t)(tile * 4 + q4) * dg + cb * ZN;
+    float* pq = pu + (int64_t)4 * (Mp / GT) * dg;
+    if (__all_sync(0xffffffffu, mbar_wait(ct.accdone, 0, ct.abort, dev_status))) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < ZN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + c0, v);
+        tmem_wait_ld();
+        float us[32], qs[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = cb * ZN + c0 + e;
+          const float z = __uint_as_float(v[e]) + (b1 ? __ldg(b1 + c) : 0.f);
+          const float u = valid ? dsp * __bfloat162float(w2[c]) * gelu_grad(z) : 0.f;
+          us[e] = u;
+          qs[e] = valid ? dsp * gelu_exact(z) : 0.f;
+          uT[(int64_t)c * Mp + t] = __float2bfloat16_rn(u);  // consecutive lanes: consecutive rows
+        }
+        lane_transpose_sum(us, lane);
+        lane_transpose_sum(qs, lane);
+        pu[c0 + lane] = us[0];
+        pq[c0 + lane] = qs[0];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, ZN);
+}
+
+// ------------------------------------------------------------------ 2. dW1 = u^T H, split over rows
+struct WCfg {
+  static constexpr int A_BYTES = GT * KCH * 2;  // 128 rows of dg x 64 kept rows (u^T)
+  static constexpr int B_BOX = KCH * 64 * 2;    // 64 kept rows x 64 columns of d
+  static constexpr int B_BYTES = (GN / 64) * B_BOX;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int SMEM = 1024 + WST * STAGE + 256;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(GT, GN, true);
+  static_assert(WST * STAGE >= GT * GN * 4, "the stages hold the fp32 tile at the end");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+// grid (dg / 128, d / 256, splits); split z takes the 64-row chunks [z cps, min(nchunk, (z+1) cps)).
+// out: dW1 [dg][d] (one split) or the partial blocks [splits][dg][d].
+__global__ void __launch_bounds__(GTHREADS, 1)
+    gate_dw1_tc(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmHB, int d, int nchunk,
+                int cps, float* __restrict__ out, int64_t out_split_stride, int32_t* __restrict__ dev_status,
+                uint64_t probe_ns) {
+  using C = WCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const Ctl ct = ctl_at<WST>(smem + WST * C::STAGE);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gi = blockIdx.x, nj = blockIdx.y, sp = blockIdx.z;
+  const int k0 = sp * cps, nk = min(nchunk, k0 + cps) - k0;  // >= 1 by the plan
+  if (threadIdx.x == 0) {
+    ctl_init<WST>(ct, probe_ns, dev_status);
+    prefetch_tmap(&tmU);
+    prefetch_tmap(&tmHB);
+  }
+  if (warp == 1) {
+    tmem_alloc(ct.tmem_slot, GN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  griddep_launch_dependents();
+  griddep_wait();  // u^T of the previous kernel is complete from here on
+  const uint32_t tmem = *ct.tmem_slot;
+  const bool skip = *ct.abort;  // only the test probe sets it this early
+  bool done = false;
+  if (skip) {
+  } else if (warp == 0) {  // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      int issued = 0;
+      for (int k = 0; k < nk; ++k) {
+        const int s = k % WST, kc = k0 + k;
+        if (k >= WST && !mbar_wait(&ct.empty[s], ((k / WST) - 1) & 1, ct.abort, dev_status)) break;
+        uint8_t* st = smem + s * C::STAGE;
+        mbar_arrive_expect_tx(&ct.full[s], C::STAGE);
+        tma_load_2d(st, &tmU, kc * KCH, gi * GT, &ct.full[s]);
+#pragma unroll
+        for (int bx = 0; bx < GN / 64; ++bx)
+          tma_load_2d(st + C::A_BYTES + bx * C::B_BOX, &tmHB, nj * GN + bx * 64, kc * KCH, &ct.full[s]);
+        ++issued;
+      }
+      if (*ct.abort) drain_copies<WST>(ct, issued);
+    }
+  } else if (warp == 1) {  // -------------------------------------------------------- MMA
+    if (lane == 0) {
+      bool ok = true;
+      for (int k = 0; k < nk; ++k) {
+        const int s = k % WST;
+        if (!mbar_wait(&ct.full[s], (k / WST) & 1, ct.abort, dev_status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + s * C::STAGE), b = a + C::A_BYTES;
+        // A: 128 rows of u^T x 64 kept rows, K-major. B: 64 kept rows x 256 columns of d as four
+        // boxes of 64 columns (N-contiguous; the leading offset steps from box to box), 16 kept
+        // rows (2048 bytes) per instruction.
+#pragma unroll
+        for (int kk = 0; kk < KCH / 16; ++kk)
+          mma_ss(tmem, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 2048, C::B_BOX, 1024), C::IDESC,
+                 (k > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&ct.empty[s]);
+      }
+      if (ok) mma_commit(ct.accdone);
+      mma_commit(ct.drain);
+      settle(ct.drain, 0);
+    }
+  } else {  // ------------------------------------------ epilogue: the tile into shared memory
+    const int q4 = warp & 3, r = q4 * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    done = __all_sync(0xffffffffu, mbar_wait(ct.accdone, 0, ct.abort, dev_status));
+    if (done) {
+      tc_fence_after();
+      // fp32 [128][256]; the 16-byte slot x of row r sits at x ^ (r % 8) (conflict-free both ways)
+      float4* row = reinterpret_cast<float4*>(smem) + r * (GN / 4);
+#pragma unroll 1
+      for (int cc = 0; cc < GN; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + cc, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          row[((cc >> 2) + i) ^ (r & 7)] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                       __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+      }
+    }
+  }
+  // every thread takes part; a CTA with any epilogue warp that timed out writes nothing
+  const bool all_done = __syncthreads_or(warp >= 2 && !done) == 0;
+  if (all_done && warp >= 2) {
+    const float4* stg = reinterpret_cast<const float4*>(smem);
+    float* dst = out + (int64_t)sp * out_split_stride + (int64_t)gi * GT * d + (int64_t)nj * GN;
+#pragma unroll 4
+    for (int i = threadIdx.x - 64; i < GT * GN / 4; i += 128) {
+      const int row = i / (GN / 4), x = i % (GN / 4);  // a warp stores one row of 512 bytes
+      *reinterpret_cast<float4*>(dst + (int64_t)row * d + x * 4) = stg[row * (GN / 4) + (x ^ (row & 7))];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, GN);
+}
+
+// ------------------------------------------------------------------ 3. sums in a fixed order
+// Threads [0, n_w / 4) with splits > 1: one float4 of dW1 each, the splits' partial blocks added
+// in split order (all loads issued before the first add). The blocks after them: one warp per
+// column h of dg, db1[h] and dw2[h] from the P warp partials (lane l adds rows l, l + 32, ... in
+// order; a fixed shuffle tree adds the lanes); warp dg: db2. Nothing is written when the status
+// word holds TG_DEV_TIMEOUT.
+__global__ void __launch_bounds__(256) gate_reduce_tc(const float* __restrict__ wpart, int splits, int64_t n_w,
+                                                      float* __restrict__ dW1, int nbw, const float* __restrict__ part,
+                                                      int P, int dg, const float* __restrict__ dscore, int M,
+                                                      float inv_t, float* __restrict__ db1, float* __restrict__ dw2,
+                                                      float* __restrict__ db2, const int32_t* __restrict__ dev_status) {
+  griddep_wait();
+  if (dev_status && (__ldcg(dev_status) & TG_DEV_TIMEOUT)) return;  // a product gave up: write nothing
+  if ((int)blockIdx.x < nbw) {
+    const int64_t n4 = n_w / 4, i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const float4* src = reinterpret_cast<const float4*>(wpart) + i;
+    float4 v[MAX_SPLITS];
+#pragma unroll
+    for (int s = 0; s < MAX_SPLITS; ++s)
+      if (s < splits) v[s] = __ldcg(src + s * n4);
+    float4 acc = v[0];
+#pragma unroll
+    for (int s = 1; s < MAX_SPLITS; ++s)
+      if (s < splits) {
+        acc.x += v[s].x;
+        acc.y += v[s].y;
+        acc.z += v[s].z;
+        acc.w += v[s].w;
+      }
+    reinterpret_cast<float4*>(dW1)[i] = acc;
+    return;
+  }
+  const int h = ((int)blockIdx.x - nbw) * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (h > dg) return;
+  float su = 0.f, sq = 0.f;
+  if (h < dg) {
+    const float* pq = part + (int64_t)P * dg;
+    for (int p = lane; p < P; p += 32) {
+      su += __ldcg(part + (int64_t)p * dg + h);
+      sq += __ldcg(pq + (int64_t)p * dg + h);
+    }
+  } else {
+    for (int t = lane; t < M; t += 32) su += __ldcg(dscore + t);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    su += __shfl_xor_sync(0xffffffffu, su, o);
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  }
+  if (lane == 0) {
+    if (h < dg) {
+      if (db1) db1[h] = su;
+      if (dw2) dw2[h] = sq;
+    } else if (db2) {
+      *db2 = su * inv_t;
+    }
+  }
+}
+
+int64_t al256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+}  // namespace
+
+bool gate_bwd_tc_shape(int64_t M, int d, int dg) {
+  return M >= 1 && M <= INT32_MAX - GT && dg % GT == 0 && dg >= GT && d % GN == 0 && d >= GN;
+}
+
+void gate_bwd_tc_plan(GateBwdPlan& p, int64_t M, int d, int dg, int sms) {
+  p.tc = true;
+  p.tc_Mp = (int)((M + GT - 1) / GT * GT);
+  p.tc_nchunk = (int)((M + KCH - 1) / KCH);
+  const int row_tiles = p.tc_Mp / GT;
+  p.tc_zn = 128;
+  for (int zn = 32; zn < 128; zn *= 2)
+    if ((int64_t)row_tiles * (dg / zn) <= sms) {
+      p.tc_zn = zn;
+      break;
+    }
+  const int tiles = (dg / GT) * (d / GN);
+  int splits = (sms + tiles - 1) / tiles;
+  splits = splits < 1 ? 1 : (splits > MAX_SPLITS ? MAX_SPLITS : splits);
+  p.tc_cps = (p.tc_nchunk + splits - 1) / splits;
+  p.tc_splits = (p.tc_nchunk + p.tc_cps - 1) / p.tc_cps;  // every split has at least one chunk
+  p.tc_off_part = al256((int64_t)p.tc_Mp * dg * 2);
+  p.tc_off_w = p.tc_off_part + al256((int64_t)2 * 4 * row_tiles * dg * 4);
+  p.tc_bytes = p.tc_off_w + (p.tc_splits > 1 ? al256((int64_t)p.tc_splits * dg * d * 4) : 0);
+}
+
+namespace {
+
+template <int ZN>
+cudaError_t launch_z(cudaLaunchConfig_t c, const CUtensorMap& tH, const CUtensorMap& tW, int M, int d, int dg,
+                     const float* b1, const void* w2, float inv_t, const float* dscore, __nv_bfloat16* uT, int Mp,
+                     float* part, int32_t* dev_status, uint64_t probe) {
+  c.gridDim = dim3((unsigned)(Mp / GT), (unsigned)(dg / ZN));
+  c.dynamicSmemBytes = (size_t)ZCfg<ZN>::SMEM;
+  return cudaLaunchKernelEx(&c, gate_z_tc<ZN>, tH, tW, M, d, dg, b1, static_cast<const __nv_bfloat16*>(w2), inv_t,
+                            dscore, uT, Mp, part, dev_status, probe);
+}
+
+}  // namespace
+
+tg_status launch_gate_bwd_tc(const void* H, int64_t M, int d, const void* W1, const float* b1, const void* w2,
+                             float inv_t, int dg, const float* dscore, float* dW1, float* db1, float* dw2, float* db2,
+                             void* ws, const GateBwdPlan& p, int sms, int32_t* dev_status, cudaStream_t st) {
+  (void)sms;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* uT = reinterpret_cast<__nv_bfloat16*>(base);
+  float* part = reinterpret_cast<float*>(base + p.tc_off_part);
+  float* wpart = p.tc_splits > 1 ? reinterpret_cast<float*>(base + p.tc_off_w) : dW1;
+  CUtensorMap tH, tW, tU, tHB;
+  if (!make_tmap_bf16_2d(&tH, H, (uint64_t)M, (uint64_t)d, (uint64_t)d, GT, KCH) ||
+      !make_tmap_bf16_2d(&tW, W1, (uint64_t)dg, (uint64_t)d, (uint64_t)d, (uint32_t)p.tc_zn, KCH) ||
+      !make_tmap_bf16_2d(&tU, uT, (uint64_t)dg, (uint64_t)p.tc_Mp, (uint64_t)p.tc_Mp, GT, KCH) ||
+      !make_tmap_bf16_2d(&tHB, H, (uint64_t)M, (uint64_t)d, (uint64_t)d, KCH, 64))
+    return fail(TG_ERR_CUDA, "tg_gate_mlp_bwd: building the TMA tensor maps failed");
+  if (attrs_needed(ATTR_GATE_TC)) {
+    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    cudaError_t e = cudaFuncSetAttribute(gate_z_tc<32>, a, ZCfg<32>::SMEM);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(gate_z_tc<64>, a, ZCfg<64>::SMEM);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(gate_z_tc<128>, a, ZCfg<128>::SMEM);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(gate_dw1_tc, a, WCfg::SMEM);
+    if (e != cudaSuccess) return cuda_status(e, "tg_gate_mlp_bwd: cudaFuncSetAttribute");
+    mark_attrs_set(ATTR_GATE_TC);
+  }
+  const uint64_t probe = wait_probe_ns();
+  cudaLaunchAttribute pdl[1] = {pdl_attribute(PDL_BWD)};
+  cudaLaunchConfig_t c = {};
+  c.blockDim = dim3(GTHREADS);
+  c.stream = st;
+  c.attrs = pdl;
+  c.numAttrs = 1;
+  cudaError_t e;
+  if (p.tc_zn == 32)
+    e = launch_z<32>(c, tH, tW, (int)M, d, dg, b1, w2, inv_t, dscore, uT, p.tc_Mp, part, dev_status, probe);
+  else if (p.tc_zn == 64)
+    e = launch_z<64>(c, tH, tW, (int)M, d, dg, b1, w2, inv_t, dscore, uT, p.tc_Mp, part, dev_status, probe);
+  else
+    e = launch_z<128>(c, tH, tW, (int)M, d, dg, b1, w2, inv_t, dscore, uT, p.tc_Mp, part, dev_status, probe);
+  if (e != cudaSuccess) return cuda_status(e, "tg_gate_mlp_bwd: z launch");
+  c.gridDim = dim3((unsigned)(dg / GT), (unsigned)(d / GN), (unsigned)p.tc_splits);
+  c.dynamicSmemBytes = (size_t)WCfg::SMEM;
+  e = cudaLaunchKernelEx(&c, gate_dw1_tc, tU, tHB, d, p.tc_nchunk, p.tc_cps, wpart, (int64_t)dg * d, dev_status,
+                         probe);
+  if (e != cudaSuccess) return cuda_status(e, "tg_gate_mlp_bwd: dW1 launch");
+  const int64_t n_w = (int64_t)dg * d;
+  const int nbw = p.tc_splits > 1 ? (int)((n_w / 4 + 255) / 256) : 0;
+  c.gridDim = dim3((unsigned)(nbw + (dg + 1 + 7) / 8));
+  c.blockDim = dim3(256);
+  c.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&c, gate_reduce_tc, (const float*)wpart, p.tc_splits, n_w, dW1, nbw, (const float*)part,
+                         4 * (p.tc_Mp / GT), dg, dscore, (int)M, inv_t, db1, dw2, db2, (const int32_t*)dev_status);
+  return cuda_status(e, "tg_gate_mlp_bwd: reduce launch");
+}
+
+}  // namespace tg

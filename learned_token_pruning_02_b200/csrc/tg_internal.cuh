@@ -34,7 +34,7 @@ enum {
   ATTR_SCORE64 = 0, ATTR_SCORE128, ATTR_SCORE256,
   ATTR_SELECT, ATTR_GATHER,
   ATTR_ATTN64, ATTR_ATTN64_UN, ATTR_ATTN128, ATTR_ATTN128_UN,
-  ATTR_QKV, ATTR_SLOTS
+  ATTR_QKV, ATTR_GATE_TC, ATTR_SLOTS
 };
 bool attrs_needed(int slot);
 void mark_attrs_set(int slot);

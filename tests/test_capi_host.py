@@ -283,7 +283,7 @@ def test_gate_mlp_bwd_arguments_and_workspace(L):
     args = lambda **kw: [kw.get(n, v) for n, v in (
         ("dt", 1), ("H", fake), ("M", 2176), ("d", 2048), ("W1", fake), ("b1", None), ("w2", fake), ("T", 1.0),
         ("dg", 256), ("ds", fake), ("dW1", fake), ("db1", None), ("dw2", None), ("db2", None), ("ws", ws),
-        ("wsb", need), ("stream", None))]
+        ("wsb", need), ("status", None), ("stream", None))]
     assert L.tg_gate_mlp_bwd(*args(d=2000)) == 2
     assert L.tg_gate_mlp_bwd(*args(dg=100)) == 2
     assert L.tg_gate_mlp_bwd(*args(T=0.0)) == 1

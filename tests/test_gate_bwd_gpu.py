@@ -1,7 +1,8 @@
 """Gradients of the gate network's parameters (tg_gate_mlp_bwd) against the oracle's
 gate_mlp_grad: dW1, db1, dw2, db2 within the tolerance of the dtype (max-abs-relative 1e-4 for
 f32, 2e-2 for bf16), deterministic, and the end-to-end training path: the chain's kept rows,
-the attention backward's d score, then these gradients."""
+the attention backward's d score, then these gradients. bf16 shapes with dg % 128 == 0 and
+d % 128 == 0 run on the tensor cores, the others on the CUDA cores."""
 import math
 
 import numpy as np
@@ -25,9 +26,15 @@ def _check(got, ref, tol):
         assert err <= tol, (name, err)
 
 
+# bf16 with dg % 128 == 0 and d % 128 == 0 runs the tensor-core kernels (one row, a ragged tail of
+# 1 and of 65 rows past a 64-row chunk, three dg tiles, several splits, first-product tiles of 32,
+# 64 and 128 columns of dg: 2176, 4352 and 10000 rows); the rest the CUDA cores.
 @pytest.mark.parametrize("dtype,M,d,dg,T", [("f32", 96, 256, 64, 1.0), ("f32", 333, 512, 128, 0.6),
                                             ("bf16", 2176, 2048, 256, 1.0), ("bf16", 1, 128, 64, 2.0),
-                                            ("bf16", 4352, 2048, 256, 1.3)])
+                                            ("bf16", 4352, 2048, 256, 1.3), ("bf16", 1, 256, 128, 1.0),
+                                            ("bf16", 129, 256, 128, 0.7), ("bf16", 1000, 512, 384, 1.0),
+                                            ("bf16", 65, 1024, 256, 2.0), ("bf16", 200, 128, 128, 1.0),
+                                            ("bf16", 10000, 256, 128, 0.9)])
 def test_gate_mlp_bwd_matches_oracle(dtype, M, d, dg, T):
     g = np.random.default_rng(M + d)
 

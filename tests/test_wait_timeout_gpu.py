@@ -113,6 +113,39 @@ def test_backward_waits_run_out_and_the_context_stays_usable():
     assert st0.item() == 0
 
 
+def test_gate_bwd_waits_run_out_and_the_context_stays_usable():
+    """tg_gate_mlp_bwd (bf16, tensor-core shape): with the hook on, its products time out, record
+    TG_DEV_TIMEOUT and the call writes none of its outputs; with the hook off it matches the oracle."""
+    g = np.random.default_rng(6)
+    M, d, dg = 300, 512, 128
+    H = ti.f32_to_bf16_bits(g.standard_normal((M, d)).astype(np.float32))
+    W1 = ti.f32_to_bf16_bits((g.standard_normal((dg, d)) / math.sqrt(d)).astype(np.float32))
+    w2 = ti.f32_to_bf16_bits((g.standard_normal(dg) / math.sqrt(dg)).astype(np.float32))
+    b1 = (g.standard_normal(dg) * 0.1).astype(np.float32)
+    ds = (g.standard_normal(M) * 0.01).astype(np.float32)
+    args = (to_dev(H, "bf16"), to_dev(W1, "bf16"), to_dev(b1, "f32"), to_dev(w2, "bf16"), to_dev(ds, "f32"))
+    sent = lambda *shape: torch.full(shape, 5.0, device="cuda")
+    outs = dict(dW1=sent(dg, d), db1=sent(dg), dw2=sent(dg), db2=sent(1))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        tg.tg_set_test_wait_probe(PROBE_NS)
+        tg.tg_gate_mlp_bwd(*args, dev_status=st, **outs)
+        torch.cuda.synchronize()
+    finally:
+        tg.tg_set_test_wait_probe(0)
+    assert st.item() & tg.TG_DEV_TIMEOUT, st.item()
+    assert torch.equal(outs["dW1"], sent(dg, d)) and torch.equal(outs["db1"], sent(dg))
+    assert torch.equal(outs["dw2"], sent(dg)) and torch.equal(outs["db2"], sent(1))
+
+    st0 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = tg.tg_gate_mlp_bwd(*args, dev_status=st0)
+    torch.cuda.synchronize()
+    ref = orc.gate_mlp_grad(ti.widen(H, "bf16"), ti.widen(W1, "bf16"), b1, ti.widen(w2, "bf16"), ds)
+    for x, r in zip(got, ref):
+        assert max_abs_rel(from_dev(x), np.atleast_1d(r)) <= TOL["bf16"]
+    assert st0.item() == 0
+
+
 def test_probe_off_by_default_and_thread_local():
     """The hook is per host thread: another thread's setting does not reach this one."""
     import threading

@@ -57,6 +57,7 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     need = L.tg_gate_mlp_bwd_workspace_size(M, d, dg)
     assert need > 16 << 20
     fake = ctypes.c_void_p(0x1000)
-    st = L.tg_gate_mlp_bwd_noalloc(1, fake, M, d, fake, None, fake, 1.0, dg, fake, fake, None, None, None, None)
+    st = L.tg_gate_mlp_bwd_noalloc(1, fake, M, d, fake, None, fake, 1.0, dg, fake, fake, None, None, None, None,
+                                   None)
     assert st == 2  # TG_ERR_UNSUPPORTED, nothing launched
     assert b"scratch" in L.tg_last_error()
