@@ -356,8 +356,8 @@ def projected_chain_time(tg, torch, dev, cb, flush, reps):
 
 def gate_bwd_time(tg, torch, dev, cb, reps):
     """Gradients of the gate network from d score of the bench workload's kept rows (seeded
-    N(0, 0.01) d score): two tcgen05 products (recompute z with the GELU' epilogue, then u^T H over
-    row splits) and an ordered reduction."""
+    N(0, 0.01) d score): two tcgen05 products (z split over d, then u^T H split over the kept rows),
+    the GELU' pass between them and an ordered reduction."""
     gen = torch.Generator(device=dev)
     gen.manual_seed(20265)
     Hk = cb.out["H_kept"]
@@ -380,8 +380,8 @@ def gate_bwd_time(tg, torch, dev, cb, reps):
     t = e0.elapsed_time(e1) / reps / 1e3
     flops = 4.0 * M * d * dg
     return {"shape": f"M={M} kept rows, d={d}, dg={dg}", "us": t * 1e6, "tflops": flops / t / 1e12,
-            "note": "tcgen05 kernels (z = H W1^T per 128x128 tile with the GELU' epilogue, then dW1 = u^T H over "
-                    "row splits, then an ordered reduction), back to back, L2 warm"}
+            "note": "tcgen05 z = H W1^T (K split), GELU' pass, tcgen05 dW1 = u^T H (row splits), ordered "
+                    "reduction; back to back, L2 warm"}
 
 
 def split_select_times(tg, torch, dev, reps):

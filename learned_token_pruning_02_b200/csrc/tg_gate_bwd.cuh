@@ -8,9 +8,10 @@ namespace tg {
 // Workspace layouts for M kept rows; the workspace query has no dtype, so `bytes` covers both.
 // CUDA-core kernels: u [M, dg] fp32 at 0; the row tiles' column sums of u and of ds' GELU(z) at
 // off_part; with more than one row split, the splits' dW1 blocks at off_w.
-// Tensor-core kernels (bf16, tc set): u^T [dg, tc_Mp] bf16 at 0; the warp partials of u and of
-// ds' GELU(z) [2][4 tc_Mp / 128][dg] fp32 at tc_off_part; with more than one split of the kept
-// rows, the splits' dW1 blocks at tc_off_w.
+// Tensor-core kernels (bf16, tc set): u^T [dg, tc_Mp] bf16 at 0; the 256-row block sums of u, of
+// ds' GELU(z) and of ds' at tc_off_part; at tc_off_big the split partials of z [tc_ks][dg][tc_Mp]
+// fp32, and after they are consumed, with more than one split of the kept rows, the splits' dW1
+// blocks.
 struct GateBwdPlan {
   int n_tiles = 0;         // 64-row tiles
   int splits = 1;          // row splits of the dW1 accumulation
@@ -18,11 +19,12 @@ struct GateBwdPlan {
   int64_t off_part = 0, off_w = 0;
   bool tc = false;         // the shape suits the tensor-core kernels
   int tc_Mp = 0;           // kept rows rounded up to 128
-  int tc_zn = 128;         // columns of dg per tile of the first product (32, 64 or 128)
+  int tc_ks = 1;           // splits of the first product's K (columns of d)
+  int tc_ublocks = 0;      // 256-row blocks of the u pass
   int tc_nchunk = 0;       // 64-row chunks of the kept rows
   int tc_cps = 0;          // chunks per split
   int tc_splits = 1;
-  int64_t tc_off_part = 0, tc_off_w = 0, tc_bytes = 0;
+  int64_t tc_off_part = 0, tc_off_big = 0, tc_bytes = 0;
   int64_t bytes = 0;
 };
 

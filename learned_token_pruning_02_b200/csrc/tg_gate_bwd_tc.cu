@@ -6,19 +6,20 @@
 //   z = W1 h + b1,  ds' = dscore / T,  u = ds' w2 * GELU'(z),  q = ds' GELU(z)  (per row, dg values),
 //   dW1 = sum_rows u h^T,  db1 = sum_rows u,  dw2 = sum_rows q,  db2 = sum_rows ds'.
 //
-// Three kernels, deterministic (fixed reduction orders, no atomics), caller workspace:
-//   1. gate_z_tc: per (128 kept rows, ZN columns of dg), z = H W1^T (M = 128, N = ZN, K = d,
-//      both operands K-major as stored, fp32 in TMEM; ZN = 32, 64 or 128, the narrowest that
-//      keeps the grid within one wave, since the epilogue is the longer part of a CTA's work). The epilogue (one row per thread) forms
-//      u and q, stores u transposed in bf16 (the next product's A operand; rows past M are zero)
-//      and adds u and q over the warp's 32 rows (a fixed butterfly that leaves column c0 + l in
-//      lane l), one partial per warp and column.
-//   2. gate_dw1_tc: per (128 rows of dg, 128 columns of d, split of the kept rows),
+// Four kernels, deterministic (fixed reduction orders, no atomics), caller workspace:
+//   1. gate_zpart_tc: per (128 kept rows, 128 columns of dg, split of d), the split's part of
+//      z = H W1^T (M = 128, N = 128, K = d / ks, both operands K-major as stored, fp32 in TMEM),
+//      stored transposed in fp32. Splitting K keeps the grid near one CTA per SM with a quarter
+//      (ks = 4) of the bytes per CTA that a whole-K tile would load.
+//   2. gate_u_kernel (CUDA cores, all SMs): z = the partials in split order + b1, then u and q
+//      (zero past M), u^T in bf16 (the next product's A operand) and the 256-row block sums of
+//      u, q and ds' (fixed shuffle tree, then the warps in order).
+//   3. gate_dw1_tc: per (128 rows of dg, 128 columns of d, split of the kept rows),
 //      dW1 = u^T H (M = 128, N = 128, K = kept rows in chunks of 64; H is the N-contiguous B
 //      operand). With more than one split each writes a partial block; the fp32 tile leaves
 //      through shared memory in row-contiguous runs.
-//   3. gate_reduce_tc: the splits' blocks in split order; db1 and dw2 from the warp partials in
-//      row order; db2 = T^-1 sum dscore.
+//   4. gate_reduce_tc: the splits' blocks in split order; db1, dw2 and db2 from the block sums in
+//      block order.
 // u is rounded to bf16 for the second product (its fp32 value feeds db1); the products accumulate
 // in fp32. Every wait is bounded; on a timeout a CTA records TG_DEV_TIMEOUT, drains its copies and
 // products, frees TMEM and returns, and the reduction writes no output (given a status word).
@@ -33,6 +34,7 @@ namespace {
 using namespace sm100;
 
 constexpr int GT = 128;        // rows of a product tile (kept rows in pass 1, rows of dg in pass 2)
+constexpr int ZN = 128;        // columns of dg per pass-1 tile
 constexpr int GN = 128;        // columns of d per pass-2 tile
 constexpr int KCH = 64;        // K elements per pipeline stage (one 128-byte swizzle row)
 constexpr int WST = 6;         // pass-2 stages (32 KB each)
@@ -52,22 +54,6 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 __device__ __forceinline__ void settle(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < 1000000000ull) {
-  }
-}
-
-// Sums v[i] over the 32 lanes for every i: afterwards v[0] of lane l holds the sum of v[l]. At the
-// step with offset o a lane keeps the half of its live values whose index has bit o equal to its
-// own lane's bit o and adds the partner's values for that half.
-__device__ __forceinline__ void lane_transpose_sum(float (&v)[32], int lane) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const bool hi = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < o; ++i) {
-      const float send = hi ? v[i] : v[i + o];
-      const float keep = hi ? v[i + o] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
   }
 }
 
@@ -117,35 +103,31 @@ __device__ __forceinline__ void drain_copies(const Ctl& c, int issued) {
   for (int k = issued - NS < 0 ? 0 : issued - NS; k < issued; ++k) settle(&c.full[k % NS], (k / NS) & 1);
 }
 
-// ------------------------------------------------------------------ 1. z, u, q per 128 x ZN tile
-template <int ZN>
+// ------------------------------------------------------------------ 1. z partials per 128 x 128 tile
 struct ZCfg {
   static constexpr int A_BYTES = GT * KCH * 2;  // 128 kept rows x 64 columns of H
-  static constexpr int B_BYTES = ZN * KCH * 2;  // ZN rows of W1 x 64 columns
+  static constexpr int B_BYTES = ZN * KCH * 2;  // 128 rows of W1 x 64 columns
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int NS = (200 * 1024) / STAGE < 8 ? (200 * 1024) / STAGE : 8;
+  static constexpr int NS = 6;
   static constexpr int SMEM = 1024 + NS * STAGE + 256;
   static constexpr uint32_t IDESC = idesc_bf16_f32(GT, ZN, false);
-  static_assert(ZN % 32 == 0 && ZN >= 32 && ZN <= 256, "TMEM columns and loads of 32");
-  static_assert(STAGE % 1024 == 0, "swizzle atoms stay aligned");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
-// grid (Mp / 128, dg / ZN). part: [2][4 * (Mp / 128)][dg] fp32, the u sums then the q sums, one
-// row per (row tile, epilogue warp).
-template <int ZN>
+// grid (Mp / 128, dg / 128, ks): split k takes the columns [k d / ks, (k + 1) d / ks) of H and W1.
+// zp: [ks][dg][Mp] fp32, the split's part of z transposed (consecutive lanes store consecutive
+// kept rows). Rows past M read zeros and give zero.
 __global__ void __launch_bounds__(GTHREADS, 1)
-    gate_z_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW, int M, int d, int dg,
-              const float* __restrict__ b1, const __nv_bfloat16* __restrict__ w2, float inv_t,
-              const float* __restrict__ dscore, __nv_bfloat16* __restrict__ uT, int Mp, float* __restrict__ part,
-              int32_t* __restrict__ dev_status, uint64_t probe_ns) {
-  using C = ZCfg<ZN>;
+    gate_zpart_tc(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW, int d, int dg,
+                  int Mp, float* __restrict__ zp, int32_t* __restrict__ dev_status, uint64_t probe_ns) {
+  using C = ZCfg;
   constexpr int NS = C::NS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const Ctl ct = ctl_at<NS>(smem + NS * C::STAGE);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, cb = blockIdx.y, nk = d / KCH;
+  const int tile = blockIdx.x, cb = blockIdx.y, ks = blockIdx.z;
+  const int nk = d / (KCH * (int)gridDim.z), kc0 = ks * nk;
   if (threadIdx.x == 0) {
     ctl_init<NS>(ct, probe_ns, dev_status);
     prefetch_tmap(&tmH);
@@ -158,21 +140,20 @@ __global__ void __launch_bounds__(GTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_launch_dependents();
-  griddep_wait();  // the d score and the workspace's earlier readers are done from here on
+  griddep_wait();  // earlier readers of the workspace are done from here on
   const uint32_t tmem = *ct.tmem_slot;
   const bool skip = *ct.abort;  // only the test probe sets it this early
   if (skip) {
   } else if (warp == 0) {  // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       int issued = 0;
-      for (int kc = 0; kc < nk; ++kc) {
-        const int s = kc % NS;
-        if (kc >= NS && !mbar_wait(&ct.empty[s], ((kc / NS) - 1) & 1, ct.abort, dev_status)) break;
+      for (int k = 0; k < nk; ++k) {
+        const int s = k % NS;
+        if (k >= NS && !mbar_wait(&ct.empty[s], ((k / NS) - 1) & 1, ct.abort, dev_status)) break;
         uint8_t* st = smem + s * C::STAGE;
         mbar_arrive_expect_tx(&ct.full[s], C::STAGE);
-        tma_load_2d(st, &tmH, kc * KCH, tile * GT, &ct.full[s]);
-        tma_load_2d(st + C::A_BYTES, &tmW, kc * KCH, cb * ZN, &ct.full[s]);
+        tma_load_2d(st, &tmH, (kc0 + k) * KCH, tile * GT, &ct.full[s]);
+        tma_load_2d(st + C::A_BYTES, &tmW, (kc0 + k) * KCH, cb * ZN, &ct.full[s]);
         ++issued;
       }
       if (*ct.abort) drain_copies<NS>(ct, issued);
@@ -180,18 +161,18 @@ __global__ void __launch_bounds__(GTHREADS, 1)
   } else if (warp == 1) {  // -------------------------------------------------------- MMA
     if (lane == 0) {
       bool ok = true;
-      for (int kc = 0; kc < nk; ++kc) {
-        const int s = kc % NS;
-        if (!mbar_wait(&ct.full[s], (kc / NS) & 1, ct.abort, dev_status)) {
+      for (int k = 0; k < nk; ++k) {
+        const int s = k % NS;
+        if (!mbar_wait(&ct.full[s], (k / NS) & 1, ct.abort, dev_status)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t a = smem_u32(smem + s * C::STAGE), b = a + C::A_BYTES;
 #pragma unroll
-        for (int k = 0; k < KCH / 16; ++k)
-          mma_ss(tmem, sdesc_sw128(a + k * 32, 16, 1024), sdesc_sw128(b + k * 32, 16, 1024), C::IDESC,
-                 (kc > 0 || k > 0) ? 1u : 0u);
+        for (int kk = 0; kk < KCH / 16; ++kk)
+          mma_ss(tmem, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 32, 16, 1024), C::IDESC,
+                 (k > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&ct.empty[s]);
       }
       if (ok) mma_commit(ct.accdone);
@@ -199,12 +180,9 @@ __global__ void __launch_bounds__(GTHREADS, 1)
       settle(ct.drain, 0);
     }
   } else {  // ------------------------------------------------------ epilogue: one row per thread
-    const int q4 = warp & 3, r = q4 * 32 + lane, t = tile * GT + r;
+    const int q4 = warp & 3, r = q4 * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const bool valid = t < M;
-    const float dsp = valid ? __ldcg(dscore + t) * inv_t : 0.f;
-    float* pu = part + (int64_t)(tile * 4 + q4) * dg + cb * ZN;
-    float* pq = pu + (int64_t)4 * (Mp / GT) * dg;
+    float* dst = zp + ((int64_t)ks * dg + cb * ZN) * Mp + tile * GT + r;
     if (__all_sync(0xffffffffu, mbar_wait(ct.accdone, 0, ct.abort, dev_status))) {
       tc_fence_after();
 #pragma unroll 1
@@ -212,27 +190,90 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + c0, v);
         tmem_wait_ld();
-        float us[32], qs[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = cb * ZN + c0 + e;
-          const float z = __uint_as_float(v[e]) + (b1 ? __ldg(b1 + c) : 0.f);
-          const float u = valid ? dsp * __bfloat162float(w2[c]) * gelu_grad(z) : 0.f;
-          us[e] = u;
-          qs[e] = valid ? dsp * gelu_exact(z) : 0.f;
-          uT[(int64_t)c * Mp + t] = __float2bfloat16_rn(u);  // consecutive lanes: consecutive rows
-        }
-        lane_transpose_sum(us, lane);
-        lane_transpose_sum(qs, lane);
-        pu[c0 + lane] = us[0];
-        pq[c0 + lane] = qs[0];
+        for (int e = 0; e < 32; ++e) __stcg(dst + (int64_t)(c0 + e) * Mp, __uint_as_float(v[e]));
       }
     }
   }
+  griddep_launch_dependents();  // after the stores: the u pass's blocks do not wait beside the products
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, ZN);
+}
+
+// ------------------------------------------------------------------ 1b. u, q and their column sums
+// grid (ceil(Mp / 256), dg / UCOLS), 256 threads: thread t of block x is kept row 256 x + t and
+// takes UCOLS columns of dg. z = the splits' partials added in split order + b1; u and q as above
+// (zero past M); u^T in bf16 for every row below Mp. cs: [2 P][dg] + [P] fp32 (P = gridDim.x),
+// the block's sums of u (rows [0, P)) and of q (rows [P, 2P)) over its 256 rows, then P more
+// values: the block's sum of ds' (entry x, written by the blocks with y == 0). Block sums: a
+// fixed shuffle tree per warp, then the 8 warps in order.
+constexpr int UCOLS = 8;
+
+template <int KS>
+__global__ void __launch_bounds__(256) gate_u_kernel(const float* __restrict__ zp, int M, int Mp, int dg,
+                                                     const float* __restrict__ b1, const __nv_bfloat16* __restrict__ w2,
+                                                     float inv_t, const float* __restrict__ dscore,
+                                                     __nv_bfloat16* __restrict__ uT, float* __restrict__ cs) {
+  __shared__ float red[8][2 * UCOLS + 1];
+  griddep_wait();  // the z partials are complete from here on
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 256 + threadIdx.x, c0 = blockIdx.y * UCOLS, P = gridDim.x;
+  const bool valid = t < M, inside = t < Mp;
+  const float dsp = valid ? __ldcg(dscore + t) * inv_t : 0.f;
+  float zk[KS][UCOLS];  // every partial is requested before the first add
+#pragma unroll
+  for (int k = 0; k < KS; ++k)
+#pragma unroll
+    for (int j = 0; j < UCOLS; ++j) zk[k][j] = inside ? __ldcg(zp + ((int64_t)k * dg + c0 + j) * Mp + t) : 0.f;
+  float us[UCOLS], qs[UCOLS];
+#pragma unroll
+  for (int j = 0; j < UCOLS; ++j) {
+    const int c = c0 + j;
+    float z = zk[0][j];
+#pragma unroll
+    for (int k = 1; k < KS; ++k) z += zk[k][j];
+    z += b1 ? __ldg(b1 + c) : 0.f;
+    const float u = valid ? dsp * __bfloat162float(w2[c]) * gelu_grad(z) : 0.f;
+    us[j] = u;
+    qs[j] = valid ? dsp * gelu_exact(z) : 0.f;
+    if (inside) uT[(int64_t)c * Mp + t] = __float2bfloat16_rn(u);
+  }
+  float sd = dsp;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int j = 0; j < UCOLS; ++j) {
+      us[j] += __shfl_xor_sync(0xffffffffu, us[j], o);
+      qs[j] += __shfl_xor_sync(0xffffffffu, qs[j], o);
+    }
+    sd += __shfl_xor_sync(0xffffffffu, sd, o);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < UCOLS; ++j) {
+      red[warp][j] = us[j];
+      red[warp][UCOLS + j] = qs[j];
+    }
+    red[warp][2 * UCOLS] = sd;
+  }
+  __syncthreads();
+  if (threadIdx.x < 2 * UCOLS + 1) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) a += red[w][threadIdx.x];
+    const int j = threadIdx.x;
+    if (j < UCOLS)
+      cs[(int64_t)blockIdx.x * dg + c0 + j] = a;
+    else if (j < 2 * UCOLS)
+      cs[(int64_t)(P + blockIdx.x) * dg + c0 + j - UCOLS] = a;
+    else if (blockIdx.y == 0)
+      cs[(int64_t)2 * P * dg + blockIdx.x] = a;
+  }
+  // the next kernel's CTAs take their SMs only now: launched earlier they would sit beside this
+  // grid's blocks while it runs
+  griddep_launch_dependents();
 }
 
 // ------------------------------------------------------------------ 2. dW1 = u^T H, split over rows
@@ -272,7 +313,6 @@ __global__ void __launch_bounds__(GTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_launch_dependents();
   griddep_wait();  // u^T of the previous kernel is complete from here on
   const uint32_t tmem = *ct.tmem_slot;
   const bool skip = *ct.abort;  // only the test probe sets it this early
@@ -340,6 +380,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
   }
   // every thread takes part; a CTA with any epilogue warp that timed out writes nothing
   const bool all_done = __syncthreads_or(warp >= 2 && !done) == 0;
+  griddep_launch_dependents();  // the products are done: the reduction's blocks may start
   if (all_done && warp >= 2) {
     const float4* stg = reinterpret_cast<const float4*>(smem);
     float* dst = out + (int64_t)sp * out_split_stride + (int64_t)gi * GT * d + (int64_t)nj * GN;
@@ -358,13 +399,12 @@ __global__ void __launch_bounds__(GTHREADS, 1)
 // ------------------------------------------------------------------ 3. sums in a fixed order
 // Threads [0, n_w / 4) with splits > 1: one float4 of dW1 each, the splits' partial blocks added
 // in split order (all loads issued before the first add). The blocks after them: one warp per
-// column h of dg, db1[h] and dw2[h] from the P warp partials (lane l adds rows l, l + 32, ... in
-// order; a fixed shuffle tree adds the lanes); warp dg: db2. Nothing is written when the status
-// word holds TG_DEV_TIMEOUT.
+// column h of dg, db1[h] and dw2[h] from the P block sums of gate_u_kernel (lane l adds rows l,
+// l + 32, ... in order; a fixed shuffle tree adds the lanes); warp dg: db2 from the P sums of ds'.
+// Nothing is written when the status word holds TG_DEV_TIMEOUT.
 __global__ void __launch_bounds__(256) gate_reduce_tc(const float* __restrict__ wpart, int splits, int64_t n_w,
-                                                      float* __restrict__ dW1, int nbw, const float* __restrict__ part,
-                                                      int P, int dg, const float* __restrict__ dscore, int M,
-                                                      float inv_t, float* __restrict__ db1, float* __restrict__ dw2,
+                                                      float* __restrict__ dW1, int nbw, const float* __restrict__ cs,
+                                                      int P, int dg, float* __restrict__ db1, float* __restrict__ dw2,
                                                       float* __restrict__ db2, const int32_t* __restrict__ dev_status) {
   griddep_wait();
   if (dev_status && (__ldcg(dev_status) & TG_DEV_TIMEOUT)) return;  // a product gave up: write nothing
@@ -392,13 +432,12 @@ __global__ void __launch_bounds__(256) gate_reduce_tc(const float* __restrict__ 
   if (h > dg) return;
   float su = 0.f, sq = 0.f;
   if (h < dg) {
-    const float* pq = part + (int64_t)P * dg;
     for (int p = lane; p < P; p += 32) {
-      su += __ldcg(part + (int64_t)p * dg + h);
-      sq += __ldcg(pq + (int64_t)p * dg + h);
+      su += __ldcg(cs + (int64_t)p * dg + h);
+      sq += __ldcg(cs + (int64_t)(P + p) * dg + h);
     }
   } else {
-    for (int t = lane; t < M; t += 32) su += __ldcg(dscore + t);
+    for (int p = lane; p < P; p += 32) su += __ldcg(cs + (int64_t)2 * P * dg + p);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -410,7 +449,7 @@ __global__ void __launch_bounds__(256) gate_reduce_tc(const float* __restrict__ 
       if (db1) db1[h] = su;
       if (dw2) dw2[h] = sq;
     } else if (db2) {
-      *db2 = su * inv_t;
+      *db2 = su;
     }
   }
 }
@@ -420,43 +459,30 @@ int64_t al256(int64_t x) { return (x + 255) & ~int64_t(255); }
 }  // namespace
 
 bool gate_bwd_tc_shape(int64_t M, int d, int dg) {
-  return M >= 1 && M <= INT32_MAX - GT && dg % GT == 0 && dg >= GT && d % GN == 0 && d >= GN;
+  return M >= 1 && M <= INT32_MAX - 256 && dg % GT == 0 && dg >= GT && d % GN == 0 && d >= GN;
 }
 
 void gate_bwd_tc_plan(GateBwdPlan& p, int64_t M, int d, int dg, int sms) {
   p.tc = true;
   p.tc_Mp = (int)((M + GT - 1) / GT * GT);
   p.tc_nchunk = (int)((M + KCH - 1) / KCH);
-  const int row_tiles = p.tc_Mp / GT;
-  p.tc_zn = 128;
-  for (int zn = 32; zn < 128; zn *= 2)
-    if ((int64_t)row_tiles * (dg / zn) <= sms) {
-      p.tc_zn = zn;
-      break;
-    }
+  const int64_t row_tiles = p.tc_Mp / GT, z_tiles = row_tiles * (dg / ZN);
+  p.tc_ks = 1;  // split the first product's K while the grid stays within one wave
+  while (p.tc_ks < 8 && z_tiles * p.tc_ks * 2 <= sms && d % (KCH * p.tc_ks * 2) == 0) p.tc_ks *= 2;
+  p.tc_ublocks = (p.tc_Mp + 255) / 256;
   const int tiles = (dg / GT) * (d / GN);
   int splits = (sms + tiles - 1) / tiles;
   splits = splits < 1 ? 1 : (splits > MAX_SPLITS ? MAX_SPLITS : splits);
   p.tc_cps = (p.tc_nchunk + splits - 1) / splits;
   p.tc_splits = (p.tc_nchunk + p.tc_cps - 1) / p.tc_cps;  // every split has at least one chunk
+  // u^T, the block sums, then one region for the z partials and, once they are consumed, the
+  // dW1 split partials (the kernels that use them run one after the other on the stream)
   p.tc_off_part = al256((int64_t)p.tc_Mp * dg * 2);
-  p.tc_off_w = p.tc_off_part + al256((int64_t)2 * 4 * row_tiles * dg * 4);
-  p.tc_bytes = p.tc_off_w + (p.tc_splits > 1 ? al256((int64_t)p.tc_splits * dg * d * 4) : 0);
+  p.tc_off_big = p.tc_off_part + al256(((int64_t)2 * p.tc_ublocks * dg + p.tc_ublocks) * 4);
+  const int64_t zbytes = (int64_t)p.tc_ks * dg * p.tc_Mp * 4;
+  const int64_t wbytes = p.tc_splits > 1 ? (int64_t)p.tc_splits * dg * d * 4 : 0;
+  p.tc_bytes = p.tc_off_big + al256(zbytes > wbytes ? zbytes : wbytes);
 }
-
-namespace {
-
-template <int ZN>
-cudaError_t launch_z(cudaLaunchConfig_t c, const CUtensorMap& tH, const CUtensorMap& tW, int M, int d, int dg,
-                     const float* b1, const void* w2, float inv_t, const float* dscore, __nv_bfloat16* uT, int Mp,
-                     float* part, int32_t* dev_status, uint64_t probe) {
-  c.gridDim = dim3((unsigned)(Mp / GT), (unsigned)(dg / ZN));
-  c.dynamicSmemBytes = (size_t)ZCfg<ZN>::SMEM;
-  return cudaLaunchKernelEx(&c, gate_z_tc<ZN>, tH, tW, M, d, dg, b1, static_cast<const __nv_bfloat16*>(w2), inv_t,
-                            dscore, uT, Mp, part, dev_status, probe);
-}
-
-}  // namespace
 
 tg_status launch_gate_bwd_tc(const void* H, int64_t M, int d, const void* W1, const float* b1, const void* w2,
                              float inv_t, int dg, const float* dscore, float* dW1, float* db1, float* dw2, float* db2,
@@ -464,39 +490,43 @@ tg_status launch_gate_bwd_tc(const void* H, int64_t M, int d, const void* W1, co
   (void)sms;
   uint8_t* base = static_cast<uint8_t*>(ws);
   __nv_bfloat16* uT = reinterpret_cast<__nv_bfloat16*>(base);
-  float* part = reinterpret_cast<float*>(base + p.tc_off_part);
-  float* wpart = p.tc_splits > 1 ? reinterpret_cast<float*>(base + p.tc_off_w) : dW1;
+  float* cs = reinterpret_cast<float*>(base + p.tc_off_part);
+  float* zp = reinterpret_cast<float*>(base + p.tc_off_big);
+  float* wpart = p.tc_splits > 1 ? reinterpret_cast<float*>(base + p.tc_off_big) : dW1;
   CUtensorMap tH, tW, tU, tHB;
   if (!make_tmap_bf16_2d(&tH, H, (uint64_t)M, (uint64_t)d, (uint64_t)d, GT, KCH) ||
-      !make_tmap_bf16_2d(&tW, W1, (uint64_t)dg, (uint64_t)d, (uint64_t)d, (uint32_t)p.tc_zn, KCH) ||
+      !make_tmap_bf16_2d(&tW, W1, (uint64_t)dg, (uint64_t)d, (uint64_t)d, ZN, KCH) ||
       !make_tmap_bf16_2d(&tU, uT, (uint64_t)dg, (uint64_t)p.tc_Mp, (uint64_t)p.tc_Mp, GT, KCH) ||
       !make_tmap_bf16_2d(&tHB, H, (uint64_t)M, (uint64_t)d, (uint64_t)d, KCH, 64))
     return fail(TG_ERR_CUDA, "tg_gate_mlp_bwd: building the TMA tensor maps failed");
   if (attrs_needed(ATTR_GATE_TC)) {
     const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
-    cudaError_t e = cudaFuncSetAttribute(gate_z_tc<32>, a, ZCfg<32>::SMEM);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(gate_z_tc<64>, a, ZCfg<64>::SMEM);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(gate_z_tc<128>, a, ZCfg<128>::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(gate_zpart_tc, a, ZCfg::SMEM);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(gate_dw1_tc, a, WCfg::SMEM);
     if (e != cudaSuccess) return cuda_status(e, "tg_gate_mlp_bwd: cudaFuncSetAttribute");
     mark_attrs_set(ATTR_GATE_TC);
   }
   const uint64_t probe = wait_probe_ns();
-  cudaLaunchAttribute pdl[1] = {pdl_attribute(PDL_BWD)};
+  cudaLaunchAttribute pdl[1] = {pdl_attribute(PDL_GATE)};
   cudaLaunchConfig_t c = {};
   c.blockDim = dim3(GTHREADS);
   c.stream = st;
   c.attrs = pdl;
   c.numAttrs = 1;
-  cudaError_t e;
-  if (p.tc_zn == 32)
-    e = launch_z<32>(c, tH, tW, (int)M, d, dg, b1, w2, inv_t, dscore, uT, p.tc_Mp, part, dev_status, probe);
-  else if (p.tc_zn == 64)
-    e = launch_z<64>(c, tH, tW, (int)M, d, dg, b1, w2, inv_t, dscore, uT, p.tc_Mp, part, dev_status, probe);
-  else
-    e = launch_z<128>(c, tH, tW, (int)M, d, dg, b1, w2, inv_t, dscore, uT, p.tc_Mp, part, dev_status, probe);
+  c.gridDim = dim3((unsigned)(p.tc_Mp / GT), (unsigned)(dg / ZN), (unsigned)p.tc_ks);
+  c.dynamicSmemBytes = (size_t)ZCfg::SMEM;
+  cudaError_t e = cudaLaunchKernelEx(&c, gate_zpart_tc, tH, tW, d, dg, p.tc_Mp, zp, dev_status, probe);
   if (e != cudaSuccess) return cuda_status(e, "tg_gate_mlp_bwd: z launch");
+  c.gridDim = dim3((unsigned)p.tc_ublocks, (unsigned)(dg / UCOLS));
+  c.blockDim = dim3(256);
+  c.dynamicSmemBytes = 0;
+  auto ku = p.tc_ks == 8 ? gate_u_kernel<8> : p.tc_ks == 4 ? gate_u_kernel<4> : p.tc_ks == 2 ? gate_u_kernel<2>
+                                                                                               : gate_u_kernel<1>;
+  e = cudaLaunchKernelEx(&c, ku, (const float*)zp, (int)M, p.tc_Mp, dg, b1, static_cast<const __nv_bfloat16*>(w2),
+                         inv_t, dscore, uT, cs);
+  if (e != cudaSuccess) return cuda_status(e, "tg_gate_mlp_bwd: u launch");
   c.gridDim = dim3((unsigned)(dg / GT), (unsigned)(d / GN), (unsigned)p.tc_splits);
+  c.blockDim = dim3(GTHREADS);
   c.dynamicSmemBytes = (size_t)WCfg::SMEM;
   e = cudaLaunchKernelEx(&c, gate_dw1_tc, tU, tHB, d, p.tc_nchunk, p.tc_cps, wpart, (int64_t)dg * d, dev_status,
                          probe);
@@ -506,8 +536,8 @@ tg_status launch_gate_bwd_tc(const void* H, int64_t M, int d, const void* W1, co
   c.gridDim = dim3((unsigned)(nbw + (dg + 1 + 7) / 8));
   c.blockDim = dim3(256);
   c.dynamicSmemBytes = 0;
-  e = cudaLaunchKernelEx(&c, gate_reduce_tc, (const float*)wpart, p.tc_splits, n_w, dW1, nbw, (const float*)part,
-                         4 * (p.tc_Mp / GT), dg, dscore, (int)M, inv_t, db1, dw2, db2, (const int32_t*)dev_status);
+  e = cudaLaunchKernelEx(&c, gate_reduce_tc, (const float*)wpart, p.tc_splits, n_w, dW1, nbw, (const float*)cs,
+                         p.tc_ublocks, dg, db1, dw2, db2, (const int32_t*)dev_status);
   return cuda_status(e, "tg_gate_mlp_bwd: reduce launch");
 }
 

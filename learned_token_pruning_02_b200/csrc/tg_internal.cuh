@@ -43,7 +43,9 @@ void mark_attrs_set(int slot);
 // their prologue while the previous kernel drains; each waits on griddepcontrol.wait before
 // its first global memory access). TG_DISABLE_PDL=1 in the environment turns it off.
 // kernel ids for the launch-chaining mask
-enum { PDL_SCORE = 1, PDL_SELECT = 2, PDL_GATHER = 4, PDL_ATTN = 8, PDL_QKV = 16, PDL_BWD = 32 };
+// (default: every bit but PDL_GATE, whose four short kernels measured slower chained than in
+// plain stream order, 23.6 against 20.7 us per call replayed from a CUDA graph at 2176 x 2048)
+enum { PDL_SCORE = 1, PDL_SELECT = 2, PDL_GATHER = 4, PDL_ATTN = 8, PDL_QKV = 16, PDL_BWD = 32, PDL_GATE = 64 };
 bool pdl_enabled(int kernel_id);
 inline cudaLaunchAttribute pdl_attribute(int kernel_id) {
   cudaLaunchAttribute a;
