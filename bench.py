@@ -357,7 +357,9 @@ def projected_chain_time(tg, torch, dev, cb, flush, reps):
 def gate_bwd_time(tg, torch, dev, cb, reps):
     """Gradients of the gate network from d score of the bench workload's kept rows (seeded
     N(0, 0.01) d score): two tcgen05 products (z split over d, then u^T H split over the kept rows),
-    the GELU' pass between them and an ordered reduction."""
+    the GELU' pass between them and an ordered reduction. `us` is the device time per call, from
+    `reps` calls captured once into a CUDA graph and replayed; `eager_us` times the same calls
+    launched one by one (the host's launch work per call is longer than the GPU's)."""
     gen = torch.Generator(device=dev)
     gen.manual_seed(20265)
     Hk = cb.out["H_kept"]
@@ -377,11 +379,30 @@ def gate_bwd_time(tg, torch, dev, cb, reps):
         run()
     e1.record(stream)
     torch.cuda.synchronize()
+    t_eager = e0.elapsed_time(e1) / reps / 1e3
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        run()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(reps):
+            run()
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
     t = e0.elapsed_time(e1) / reps / 1e3
+    del graph
     flops = 4.0 * M * d * dg
     return {"shape": f"M={M} kept rows, d={d}, dg={dg}", "us": t * 1e6, "tflops": flops / t / 1e12,
+            "eager_us": t_eager * 1e6,
             "note": "tcgen05 z = H W1^T (K split), GELU' pass, tcgen05 dW1 = u^T H (row splits), ordered "
-                    "reduction; back to back, L2 warm"}
+                    "reduction; device time per call from a CUDA graph of back-to-back calls, L2 warm"}
 
 
 def split_select_times(tg, torch, dev, reps):
