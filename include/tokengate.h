@@ -84,7 +84,9 @@ const char* tg_last_error(void);
  * tg_topk_candidates, tg_topk_merge and tg_gated_attn_bwd. 1.2 gives tg_score a device
  * status word (its last argument before the stream) and a temperature (after b2, also in
  * tg_prefill_above_L), and adds tg_set_test_wait_probe, tg_gate_mlp_bwd and its
- * workspace query, and tg_prefill_projected. */
+ * workspace query, and tg_prefill_projected. 1.3 adds tg_gate_mlp_bwd_noalloc and gives
+ * tg_gate_mlp_bwd a device status word (its last argument before the stream; a changed
+ * signature, so 1.2 callers of it must be rebuilt). */
 int32_t tg_version(void);
 
 /* Test hook for the bounded waits, off by default (limit_ns = 0). With limit_ns > 0, every

@@ -145,7 +145,7 @@ const char* tg_status_string(int32_t st) {
 
 const char* tg_last_error(void) { return g_err; }
 
-int32_t tg_version(void) { return (1 << 16) | 2; }
+int32_t tg_version(void) { return (1 << 16) | 3; }
 
 tg_status tg_set_test_wait_probe(int64_t limit_ns) {
   g_err[0] = 0;

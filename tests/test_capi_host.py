@@ -45,7 +45,8 @@ def test_status_strings_and_version(L):
     assert L.tg_status_string(4) == b"TG_ERR_CUDA"
     assert L.tg_status_string(99) == b"TG_ERR_UNKNOWN"
     assert L.tg_version() >> 16 == 1
-    assert L.tg_version() & 0xffff >= 2  # 1.1: projection, split selection, backward; 1.2: score status
+    assert L.tg_version() & 0xffff >= 3  # 1.1: projection, split selection, backward; 1.2: score status;
+    # 1.3: allocation-free gate gradients, status word of tg_gate_mlp_bwd
     assert L.tg_set_test_wait_probe(-1) == 1
     assert L.tg_set_test_wait_probe(0) == 0
 
