@@ -440,15 +440,14 @@ tg_status tg_gate_mlp_bwd(tg_dtype dtype, const void* H_kept, int64_t M, int32_t
   if (!H_kept || !W1 || !w2 || !dscore) return fail(TG_ERR_INVALID_ARG, "H_kept, W1, w2 and dscore are required");
   if (!aligned16(H_kept) || !aligned16(W1) || !aligned16(dW1))
     return fail(TG_ERR_UNSUPPORTED, "H_kept, W1 and dW1 must be 16-byte aligned");
-  const int sms = device_sm_count();
-  const GateBwdPlan p = gate_bwd_plan(M, d, dg, sms);
+  const GateBwdPlan p = gate_bwd_plan(M, d, dg, device_sm_count());
   if (!ws || ws_bytes < (size_t)p.bytes || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(TG_ERR_WORKSPACE, "the workspace needs %lld bytes at a 256-byte aligned address",
                 (long long)p.bytes);
   st = check_device();
   if (st != TG_OK) return st;
   return launch_gate_bwd(dtype, H_kept, M, d, W1, b1, w2, (float)(1.0 / (double)temperature), dg, dscore, dW1, db1,
-                         dw2, db2, ws, p, sms, dev_status, (cudaStream_t)stream);
+                         dw2, db2, ws, p, dev_status, (cudaStream_t)stream);
 }
 
 tg_status tg_gate_mlp_bwd_noalloc(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W1,
@@ -459,8 +458,7 @@ tg_status tg_gate_mlp_bwd_noalloc(tg_dtype dtype, const void* H_kept, int64_t M,
   tg_status st = gate_bwd_check(dtype, M, d, dg, temperature);
   if (st != TG_OK) return st;
   if (M > 0) {
-    const int sms = device_sm_count();
-    const GateBwdPlan p = gate_bwd_plan(M, d, dg, sms);
+    const GateBwdPlan p = gate_bwd_plan(M, d, dg, device_sm_count());
     if (p.bytes > (int64_t)TG_GATE_NOALLOC_SCRATCH_BYTES)
       return fail(TG_ERR_UNSUPPORTED,
                   "tg_gate_mlp_bwd_noalloc: M=%lld, d=%d, dg=%d need %lld bytes of scratch, more than the fixed "
@@ -476,7 +474,7 @@ tg_status tg_gate_mlp_bwd_noalloc(tg_dtype dtype, const void* H_kept, int64_t M,
     st = gate_bwd_fixed_scratch(&scratch);
     if (st != TG_OK) return st;
     return launch_gate_bwd(dtype, H_kept, M, d, W1, b1, w2, (float)(1.0 / (double)temperature), dg, dscore, dW1,
-                           db1, dw2, db2, scratch, p, sms, dev_status, (cudaStream_t)stream);
+                           db1, dw2, db2, scratch, p, dev_status, (cudaStream_t)stream);
   }
   // no rows: the workspace entry point writes the zero gradients without touching any workspace
   return tg_gate_mlp_bwd(dtype, H_kept, M, d, W1, b1, w2, temperature, dg, dscore, dW1, db1, dw2, db2, nullptr, 0,

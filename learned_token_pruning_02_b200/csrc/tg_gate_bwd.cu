@@ -253,10 +253,10 @@ GateBwdPlan gate_bwd_plan(int64_t M, int d, int dg, int sms) {
 
 tg_status launch_gate_bwd(tg_dtype dt, const void* H, int64_t M, int d, const void* W1, const float* b1,
                           const void* w2, float inv_t, int dg, const float* dscore, float* dW1, float* db1,
-                          float* dw2, float* db2, void* ws, const GateBwdPlan& p, int sms, int32_t* dev_status,
+                          float* dw2, float* db2, void* ws, const GateBwdPlan& p, int32_t* dev_status,
                           cudaStream_t st) {
   if (dt == TG_BF16 && p.tc)
-    return launch_gate_bwd_tc(H, M, d, W1, b1, w2, inv_t, dg, dscore, dW1, db1, dw2, db2, ws, p, sms, dev_status, st);
+    return launch_gate_bwd_tc(H, M, d, W1, b1, w2, inv_t, dg, dscore, dW1, db1, dw2, db2, ws, p, dev_status, st);
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* U = reinterpret_cast<float*>(base);
   float* part_db1 = reinterpret_cast<float*>(base + p.off_part);

@@ -36,7 +36,7 @@ bool gate_bwd_tc_shape(int64_t M, int d, int dg);
 void gate_bwd_tc_plan(GateBwdPlan& p, int64_t M, int d, int dg, int sms);
 tg_status launch_gate_bwd_tc(const void* H, int64_t M, int d, const void* W1, const float* b1, const void* w2,
                              float inv_t, int dg, const float* dscore, float* dW1, float* db1, float* dw2, float* db2,
-                             void* ws, const GateBwdPlan& p, int sms, int32_t* dev_status, cudaStream_t st);
+                             void* ws, const GateBwdPlan& p, int32_t* dev_status, cudaStream_t st);
 
 // Device address, on the current device, of the library's fixed scratch array for
 // tg_gate_mlp_bwd_noalloc (TG_GATE_NOALLOC_SCRATCH_BYTES); looked up once per device.
@@ -44,7 +44,6 @@ tg_status gate_bwd_fixed_scratch(void** ptr);
 
 tg_status launch_gate_bwd(tg_dtype dt, const void* H, int64_t M, int d, const void* W1, const float* b1,
                           const void* w2, float inv_t, int dg, const float* dscore, float* dW1, float* db1,
-                          float* dw2, float* db2, void* ws, const GateBwdPlan& p, int sms, int32_t* dev_status,
-                          cudaStream_t st);
+                          float* dw2, float* db2, void* ws, const GateBwdPlan& p, int32_t* dev_status, cudaStream_t st);
 
 }  // namespace tg

@@ -486,8 +486,7 @@ void gate_bwd_tc_plan(GateBwdPlan& p, int64_t M, int d, int dg, int sms) {
 
 tg_status launch_gate_bwd_tc(const void* H, int64_t M, int d, const void* W1, const float* b1, const void* w2,
                              float inv_t, int dg, const float* dscore, float* dW1, float* db1, float* dw2, float* db2,
-                             void* ws, const GateBwdPlan& p, int sms, int32_t* dev_status, cudaStream_t st) {
-  (void)sms;
+                             void* ws, const GateBwdPlan& p, int32_t* dev_status, cudaStream_t st) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   __nv_bfloat16* uT = reinterpret_cast<__nv_bfloat16*>(base);
   float* cs = reinterpret_cast<float*>(base + p.tc_off_part);
