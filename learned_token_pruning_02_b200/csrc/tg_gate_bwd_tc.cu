@@ -21,8 +21,9 @@
 //   4. gate_reduce_tc: the splits' blocks in split order; db1, dw2 and db2 from the block sums in
 //      block order.
 // u is rounded to bf16 for the second product (its fp32 value feeds db1); the products accumulate
-// in fp32. Every wait is bounded; on a timeout a CTA records TG_DEV_TIMEOUT, drains its copies and
-// products, frees TMEM and returns, and the reduction writes no output (given a status word).
+// in fp32. GELU and GELU' share one exponential (erf from Abramowitz & Stegun 7.1.26). Every wait
+// is bounded; on a timeout a CTA records TG_DEV_TIMEOUT, drains its copies and products, frees
+// TMEM and returns, and the reduction writes no output (given a status word).
 #include <cuda_bf16.h>
 
 #include "tg_gate_bwd.cuh"
@@ -41,9 +42,45 @@ constexpr int WST = 6;         // pass-2 stages (32 KB each)
 constexpr int GTHREADS = 192;  // warp 0: TMA, 1: MMA + TMEM, 2-5: epilogue (TMEM lane quarters 2, 3, 0, 1)
 constexpr int MAX_SPLITS = 4;
 
-__device__ __forceinline__ float gelu_exact(float z) { return 0.5f * z * (1.f + erff(z * 0.70710678118654752f)); }
-__device__ __forceinline__ float gelu_grad(float z) {
-  return 0.5f * (1.f + erff(z * 0.70710678118654752f)) + z * 0.39894228040143268f * expf(-0.5f * z * z);
+// GELU(z) = z Phi(z) and GELU'(z) = Phi(z) + z phi(z) together, with erf from Abramowitz &
+// Stegun, Handbook of Mathematical Functions, formula 7.1.26: for x >= 0,
+// erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) e^(-x^2), t = 1 / (1 + p x), with
+// |error| <= 1.5e-7. At x = |z| / sqrt 2 the factor e^(-x^2) = e^(-z^2 / 2) is the one the normal
+// density phi needs too, so one exponential and one reciprocal serve both values (1/sqrt 2 is
+// folded into p).
+__device__ __forceinline__ void gelu_and_grad(float z, float* g, float* gp) {
+  constexpr float kP = (float)(0.3275911 * 0.70710678118654752440);
+  constexpr float kA1 = 0.254829592f, kA2 = -0.284496736f, kA3 = 1.421413741f, kA4 = -1.453152027f,
+                  kA5 = 1.061405429f;
+  const float az = fabsf(z);
+  const float e = ex2(-0.72134752044448170368f * z * z);  // e^(-z^2 / 2) = 2^(-z^2 log2(e) / 2)
+  float t;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(kP, az, 1.f)));
+  const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, kA5, kA4), kA3), kA2), kA1);
+  const float tail = 0.5f * poly * e;  // 1 - Phi(|z|)
+  const float Phi = z >= 0.f ? 1.f - tail : tail;
+  *g = z * Phi;
+  *gp = fmaf(z * 0.39894228040143268f, e, Phi);  // + z phi(z)
+}
+
+// Sums v[i] over the 32 lanes for every i (NV a power of two up to 32): afterwards v[0] of lane l
+// holds the warp's sum of v[l % NV]. At the step with offset o < NV a lane keeps the half of its
+// live values whose index has bit o equal to its own lane's bit o and adds the partner's values
+// for that half; the offsets from NV up then add the groups of NV lanes. A fixed order throughout.
+template <int NV>
+__device__ __forceinline__ void lane_transpose_sum(float (&v)[NV], int lane) {
+#pragma unroll
+  for (int o = NV / 2; o > 0; o >>= 1) {
+    const bool hi = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = hi ? v[i] : v[i + o];
+      const float keep = hi ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+#pragma unroll
+  for (int o = NV; o < 32; o <<= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -204,12 +241,14 @@ __global__ void __launch_bounds__(GTHREADS, 1)
 
 // ------------------------------------------------------------------ 1b. u, q and their column sums
 // grid (ceil(Mp / 256), dg / UCOLS), 256 threads: thread t of block x is kept row 256 x + t and
-// takes UCOLS columns of dg. z = the splits' partials added in split order + b1; u and q as above
-// (zero past M); u^T in bf16 for every row below Mp. cs: [2 P][dg] + [P] fp32 (P = gridDim.x),
-// the block's sums of u (rows [0, P)) and of q (rows [P, 2P)) over its 256 rows, then P more
-// values: the block's sum of ds' (entry x, written by the blocks with y == 0). Block sums: a
-// fixed shuffle tree per warp, then the 8 warps in order.
-constexpr int UCOLS = 8;
+// takes UCOLS = 4 columns of dg. z = the splits' partials added in split order + b1; u and q as
+// above (zero past M); u^T in bf16 for every row below Mp. cs: [2 P][dg] + [P] fp32 (P =
+// gridDim.x), the block's sums of u (rows [0, P)) and of q (rows [P, 2P)) over its 256 rows, then
+// P more values: the block's sum of ds' (entry x, written by the blocks with y == 0). Block sums:
+// the 8 values of a thread (u and q of its 4 columns) go through one lane butterfly (lane l ends
+// with the warp's sum of value l % 8), ds' through a shuffle tree, then the 8 warps add in order.
+// Few columns per thread keep many warps resident: the pass waits on its loads, not on issue.
+constexpr int UCOLS = 4;
 
 template <int KS>
 __global__ void __launch_bounds__(256) gate_u_kernel(const float* __restrict__ zp, int M, int Mp, int dg,
@@ -222,42 +261,31 @@ __global__ void __launch_bounds__(256) gate_u_kernel(const float* __restrict__ z
   const int t = blockIdx.x * 256 + threadIdx.x, c0 = blockIdx.y * UCOLS, P = gridDim.x;
   const bool valid = t < M, inside = t < Mp;
   const float dsp = valid ? __ldcg(dscore + t) * inv_t : 0.f;
-  float zk[KS][UCOLS];  // every partial is requested before the first add
+  float v[2 * UCOLS];  // u of the columns, then q
 #pragma unroll
-  for (int k = 0; k < KS; ++k)
+  for (int j = 0; j < UCOLS; ++j) {
+    float z = inside ? __ldcg(zp + ((int64_t)c0 + j) * Mp + t) : 0.f;
 #pragma unroll
-    for (int j = 0; j < UCOLS; ++j) zk[k][j] = inside ? __ldcg(zp + ((int64_t)k * dg + c0 + j) * Mp + t) : 0.f;
-  float us[UCOLS], qs[UCOLS];
+    for (int k = 1; k < KS; ++k) z += inside ? __ldcg(zp + ((int64_t)k * dg + c0 + j) * Mp + t) : 0.f;
+    v[j] = z;
+  }
 #pragma unroll
   for (int j = 0; j < UCOLS; ++j) {
     const int c = c0 + j;
-    float z = zk[0][j];
-#pragma unroll
-    for (int k = 1; k < KS; ++k) z += zk[k][j];
-    z += b1 ? __ldg(b1 + c) : 0.f;
-    const float u = valid ? dsp * __bfloat162float(w2[c]) * gelu_grad(z) : 0.f;
-    us[j] = u;
-    qs[j] = valid ? dsp * gelu_exact(z) : 0.f;
+    const float z = v[j] + (b1 ? __ldg(b1 + c) : 0.f);
+    float g, gp;
+    gelu_and_grad(z, &g, &gp);
+    const float u = valid ? dsp * __bfloat162float(w2[c]) * gp : 0.f;
+    v[j] = u;
+    v[UCOLS + j] = valid ? dsp * g : 0.f;
     if (inside) uT[(int64_t)c * Mp + t] = __float2bfloat16_rn(u);
   }
+  lane_transpose_sum(v, lane);
   float sd = dsp;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-    for (int j = 0; j < UCOLS; ++j) {
-      us[j] += __shfl_xor_sync(0xffffffffu, us[j], o);
-      qs[j] += __shfl_xor_sync(0xffffffffu, qs[j], o);
-    }
-    sd += __shfl_xor_sync(0xffffffffu, sd, o);
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int j = 0; j < UCOLS; ++j) {
-      red[warp][j] = us[j];
-      red[warp][UCOLS + j] = qs[j];
-    }
-    red[warp][2 * UCOLS] = sd;
-  }
+  for (int o = 16; o > 0; o >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);
+  if (lane < 2 * UCOLS) red[warp][lane] = v[0];
+  if (lane == 0) red[warp][2 * UCOLS] = sd;
   __syncthreads();
   if (threadIdx.x < 2 * UCOLS + 1) {
     float a = 0.f;

@@ -52,6 +52,12 @@ def test_gate_mlp_bwd_matches_oracle(dtype, M, d, dg, T):
     torch.cuda.synchronize()
     ref = orc.gate_mlp_grad(ti.widen(H, dtype), ti.widen(W1, dtype), b1, ti.widen(w2, dtype), ds, temperature=T)
     _check(got, ref, TOL[dtype])
+    # db1, dw2 and db2 are fp32 sums of fp32 values on both paths (only dW1 takes u in bf16), so
+    # they hold a bound far below the bf16 tolerance: this pins the GELU / GELU' evaluation (erf
+    # from Abramowitz & Stegun 7.1.26 on the tensor-core path, |error| <= 1.5e-7)
+    for name, x, r in zip(("db1", "dw2", "db2"), got[1:], ref[1:]):
+        err = max_abs_rel(from_dev(x), np.atleast_1d(r))
+        assert err <= 1e-3, (name, err)
     for a, b in zip(got, again):  # deterministic
         assert np.array_equal(bits(a), bits(b))
 
