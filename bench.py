@@ -203,7 +203,8 @@ def bandwidth_instances(tg, torch, dev, peak_gbs, reps):
     their bandwidth where the bench workload is latency-bound: select over 64 sequences of
     131072 seeded N(0,1) scores (question tail 256, K=4096 each; 33.5 MB read) and a gather of
     65536 of 131072 rows of d=2048 bf16 (537 MB moved). L2 is flushed before every launch; each
-    launch is timed alone with CUDA events on its stream."""
+    launch is timed alone with CUDA events on its stream. The select runs both as one cluster per
+    sequence (tg_topk_select) and as the four-kernel stream over all SMs (tg_topk_select_stream)."""
     gen = torch.Generator(device=dev)
     gen.manual_seed(20260)
     stream = torch.cuda.current_stream()
@@ -235,7 +236,12 @@ def bandwidth_instances(tg, torch, dev, peak_gbs, reps):
     byts = B * (N - q) * 4 + m_tot * 4
     out["select"] = {"shape": f"{B} sequences x {N} tokens, question tail {q}, K={K}", "bytes": byts,
                      "us": t * 1e6, "gbs": byts / t / 1e9, "frac": byts / t / 1e9 / peak_gbs}
-    del sc, kept
+    ws = torch.empty(tg.tg_topk_select_stream_workspace_size(seqlens, q_len, k), device=dev, dtype=torch.uint8)
+    t = timed(lambda: tg.tg_topk_select_stream(sc, seqlens, q_len, k, kept_idx=kept, cu_kept_dev=cu_dev, ws=ws))
+    out["select_stream"] = {"shape": out["select"]["shape"], "bytes": byts, "us": t * 1e6, "gbs": byts / t / 1e9,
+                            "frac": byts / t / 1e9 / peak_gbs,
+                            "note": "tg_topk_select_stream: histogram, candidates, threshold, compaction over all SMs"}
+    del sc, kept, ws
     N, d, q = 131072, 2048, 256
     K = 65536 - q
     H = torch.randn(N, d, device=dev, generator=gen, dtype=torch.float32).to(torch.bfloat16)

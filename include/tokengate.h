@@ -84,7 +84,8 @@ const char* tg_last_error(void);
  * tg_topk_candidates, tg_topk_merge and tg_gated_attn_bwd. 1.2 gives tg_score a device
  * status word (its last argument before the stream) and a temperature (after b2, also in
  * tg_prefill_above_L), and adds tg_set_test_wait_probe, tg_gate_mlp_bwd and its
- * workspace query, and tg_prefill_projected. 1.3 adds tg_gate_mlp_bwd_noalloc and gives
+ * workspace query, and tg_prefill_projected. 1.3 adds tg_gate_mlp_bwd_noalloc,
+ * tg_topk_select_stream and its workspace query, and gives
  * tg_gate_mlp_bwd a device status word (its last argument before the stream; a changed
  * signature, so 1.2 callers of it must be rebuilt). */
 int32_t tg_version(void);
@@ -144,6 +145,28 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
  * Supported: N_b - q_b <= TG_MAX_CTX. */
 tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
                          int32_t* cu_kept_dev, int32_t* dev_status, void* stream);
+
+/* Workspace bytes tg_topk_select_stream needs for these sequences (0 when seqs is invalid or
+ * empty). Host only. About 8 bytes per context token of the sequences that are pruned (the
+ * worst case of the candidate lists) plus 1 MiB; at 64 sequences of 131072 tokens, 68 MB. */
+size_t tg_topk_select_stream_workspace_size(const tg_seqs* seqs);
+
+/* tg_topk_select for many long sequences at once: the same outputs bit for bit (kept_idx,
+ * cu_kept_dev, TG_DEV_NAN_SCORE), computed as a stream over all SMs instead of one thread-block
+ * cluster per sequence. The context is cut into chunks of 8192 tokens; four kernels run in
+ * stream order: a 12-bit histogram of the order keys per sequence (integer atomics), the bin
+ * holding the K-th largest key and the candidates in it, the exact threshold with each chunk's
+ * output offset and quota of keys equal to it (lower positions first), and an ascending
+ * compaction. The scores are read from HBM once; the later passes find them in L2 while the
+ * batch's scores fit there. Deterministic: only integer counts decide anything.
+ *   score, seqs, kept_idx, cu_kept_dev, dev_status: as for tg_topk_select
+ *   ws       device workspace of at least tg_topk_select_stream_workspace_size(seqs) bytes,
+ *            256-byte aligned (TG_ERR_WORKSPACE otherwise); owned by the caller, contents need
+ *            no initialisation
+ * Supported: N_b - q_b <= TG_MAX_CTX; any number of sequences (launched 64 at a time). */
+tg_status tg_topk_select_stream(const float* score, const tg_seqs* seqs, int32_t* kept_idx,
+                                int32_t* cu_kept_dev, void* ws, size_t ws_bytes,
+                                int32_t* dev_status, void* stream);
 
 /* Projection of the kept rows for a layer above L (aitualizate.com TokenGate article,
  * phase 3: those layers process only the kept tokens, at their original positions). The

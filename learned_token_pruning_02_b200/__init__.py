@@ -37,6 +37,8 @@ EXPORTS = (
     "tg_gate_mlp_bwd",
     "tg_prefill_projected",
     "tg_gate_mlp_bwd_noalloc",
+    "tg_topk_select_stream_workspace_size",
+    "tg_topk_select_stream",
 )
 
 
@@ -101,6 +103,10 @@ def lib() -> ctypes.CDLL:
     L.tg_set_test_wait_probe.argtypes = [_I64]
     L.tg_topk_select.restype = _I32
     L.tg_topk_select.argtypes = [_VP, _SEQP, _VP, _VP, _VP, _VP]
+    L.tg_topk_select_stream_workspace_size.restype = ctypes.c_size_t
+    L.tg_topk_select_stream_workspace_size.argtypes = [_SEQP]
+    L.tg_topk_select_stream.restype = _I32
+    L.tg_topk_select_stream.argtypes = [_VP, _SEQP, _VP, _VP, _VP, ctypes.c_size_t, _VP, _VP]
     L.tg_qkv_rope.restype = _I32
     L.tg_qkv_rope.argtypes = [_I32, _VP, _I64, _I32, _VP, _VP, _I32, _I32, _I32, _F, _VP, _VP, _VP, _VP, _VP]
     L.tg_topk_candidates.restype = _I32
@@ -242,6 +248,34 @@ def tg_topk_select(score, seqlens, q_len, k, kept_idx=None, cu_kept_dev=None, de
         cu_kept_dev = torch.empty(s.B + 1, device=score.device, dtype=torch.int32)
     _check("tg_topk_select", lib().tg_topk_select(_ptr(score), s.ref(), _ptr(kept_idx), _ptr(cu_kept_dev),
                                                   _ptr(dev_status), _stream(stream)))
+    return kept_idx, cu_kept_dev
+
+
+def tg_topk_select_stream_workspace_size(seqlens, q_len, k) -> int:
+    """Workspace bytes of tg_topk_select_stream for these sequences (host only)."""
+    return int(lib().tg_topk_select_stream_workspace_size(Seqs(seqlens, q_len, k).ref()))
+
+
+def tg_topk_select_stream(score, seqlens, q_len, k, kept_idx=None, cu_kept_dev=None, ws=None, dev_status=None,
+                          stream=None):
+    """tg_topk_select for many long sequences at once (the same outputs bit for bit), from four
+    kernels over all SMs. ``ws`` is a uint8 device buffer of at least
+    tg_topk_select_stream_workspace_size bytes (allocated here when not given)."""
+    _want(torch.float32, score=score)
+    _want(torch.int32, kept_idx=kept_idx, cu_kept_dev=cu_kept_dev, dev_status=dev_status)
+    _cuda(score, kept_idx, cu_kept_dev, ws, dev_status)
+    s = Seqs(seqlens, q_len, k)
+    cu = tg_kept_counts(seqlens, q_len, k)
+    if kept_idx is None:
+        kept_idx = torch.empty(cu[-1], device=score.device, dtype=torch.int32)
+    if cu_kept_dev is None:
+        cu_kept_dev = torch.empty(s.B + 1, device=score.device, dtype=torch.int32)
+    need = lib().tg_topk_select_stream_workspace_size(s.ref())
+    if ws is None:
+        ws = torch.empty(max(need, 1), device=score.device, dtype=torch.uint8)
+    _check("tg_topk_select_stream", lib().tg_topk_select_stream(
+        _ptr(score), s.ref(), _ptr(kept_idx), _ptr(cu_kept_dev), _ptr(ws), ws.numel() * ws.element_size(),
+        _ptr(dev_status), _stream(stream)))
     return kept_idx, cu_kept_dev
 
 

@@ -193,6 +193,20 @@ tg_status tg_score(tg_dtype dtype, const void* H, int64_t ldh, int64_t n_tok, in
 }
 
 // The selector with optional per-row outputs pos, g and log g (the chained prefill).
+// Per-sequence descriptors of the select (seqs already checked).
+static std::vector<SelSeq> sel_seqs(const tg_seqs* seqs) {
+  std::vector<SelSeq> d(seqs->B);
+  int64_t start = 0, off = 0;
+  for (int b = 0; b < seqs->B; ++b) {
+    int32_t N = seqs->seqlens[b], q = seqs->q_len[b];
+    int32_t m = kept_rows(seqs, b);
+    d[b] = SelSeq{(int32_t)start, N - q, q, m - q, (int32_t)off, b, (int32_t)(start + N - q), (int32_t)start};
+    start += N;
+    off += m;
+  }
+  return d;
+}
+
 static tg_status select_impl(const float* score, const tg_seqs* seqs, int32_t* kept_idx, int32_t* cu_kept_dev,
                              int32_t* dev_status, void* stream, int32_t* pos, float* g, float* logg,
                              uint32_t flags) {
@@ -204,15 +218,7 @@ static tg_status select_impl(const float* score, const tg_seqs* seqs, int32_t* k
     return fail(TG_ERR_INVALID_ARG, "score and kept_idx are required");
   st = check_device();
   if (st != TG_OK) return st;
-  std::vector<SelSeq> d(seqs->B);
-  int64_t start = 0, off = 0;
-  for (int b = 0; b < seqs->B; ++b) {
-    int32_t N = seqs->seqlens[b], q = seqs->q_len[b];
-    int32_t m = kept_rows(seqs, b);
-    d[b] = SelSeq{(int32_t)start, N - q, q, m - q, (int32_t)off, b, (int32_t)(start + N - q), (int32_t)start};
-    start += N;
-    off += m;
-  }
+  const std::vector<SelSeq> d = sel_seqs(seqs);
   cudaStream_t s = (cudaStream_t)stream;
   for (int b0 = 0; b0 < seqs->B; b0 += kMaxSeqPerLaunch) {
     int nb = seqs->B - b0 < kMaxSeqPerLaunch ? seqs->B - b0 : kMaxSeqPerLaunch;
@@ -228,6 +234,32 @@ tg_status tg_topk_select(const float* score, const tg_seqs* seqs, int32_t* kept_
                          int32_t* cu_kept_dev, int32_t* dev_status, void* stream) {
   g_err[0] = 0;
   return select_impl(score, seqs, kept_idx, cu_kept_dev, dev_status, stream, nullptr, nullptr, nullptr, 0);
+}
+
+size_t tg_topk_select_stream_workspace_size(const tg_seqs* seqs) {
+  int64_t n_tot = 0, m_tot = 0;
+  if (check_seqs(seqs, &n_tot, &m_tot) != TG_OK || seqs->B == 0) return 0;
+  const std::vector<SelSeq> d = sel_seqs(seqs);
+  return (size_t)select_stream_workspace(d.data(), seqs->B);
+}
+
+tg_status tg_topk_select_stream(const float* score, const tg_seqs* seqs, int32_t* kept_idx, int32_t* cu_kept_dev,
+                                void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  g_err[0] = 0;
+  int64_t n_tot = 0, m_tot = 0;
+  tg_status st = check_seqs(seqs, &n_tot, &m_tot);
+  if (st != TG_OK) return st;
+  if (seqs->B == 0) return TG_OK;
+  if ((n_tot > 0 && !score) || (m_tot > 0 && !kept_idx))
+    return fail(TG_ERR_INVALID_ARG, "score and kept_idx are required");
+  const std::vector<SelSeq> d = sel_seqs(seqs);
+  const int64_t need = select_stream_workspace(d.data(), seqs->B);
+  if (!ws || ws_bytes < (size_t)need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(TG_ERR_WORKSPACE, "tg_topk_select_stream: the workspace needs %lld bytes at a 256-byte aligned address",
+                (long long)need);
+  st = check_device();
+  if (st != TG_OK) return st;
+  return launch_select_stream(score, d.data(), seqs->B, kept_idx, cu_kept_dev, dev_status, ws, (cudaStream_t)stream);
 }
 
 tg_status tg_qkv_rope(tg_dtype dtype, const void* H_kept, int64_t M, int32_t d, const void* W_qkv,

@@ -98,6 +98,13 @@ tg_status launch_select(const float* score, const SelSeq* seqs, int nseq, int n_
                         float* logg = nullptr, uint32_t flags = 0, const int32_t* idxmap = nullptr,
                         float* kept_score = nullptr);
 
+// The many-sequence form of the select (csrc/tg_select_stream.cu): the same outputs as
+// launch_select without its optional ones, from four kernels over all SMs and a workspace of
+// select_stream_workspace(seqs, nseq) bytes (256-byte aligned). Any number of sequences.
+int64_t select_stream_workspace(const SelSeq* seqs, int nseq);
+tg_status launch_select_stream(const float* score, const SelSeq* seqs, int nseq, int32_t* kept_idx,
+                               int32_t* cu_kept_dev, int32_t* dev_status, void* ws, cudaStream_t st);
+
 struct GatherSeq {
   int32_t start;    // packed row of the sequence's first token
   int32_t n;        // tokens N

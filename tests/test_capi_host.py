@@ -296,3 +296,25 @@ def test_gate_mlp_bwd_arguments_and_workspace(L):
     assert L.tg_gate_mlp_bwd(*args(ws=None)) == 3
     assert L.tg_gate_mlp_bwd(*args(ws=V(0x10080))) == 3  # workspace not 256-byte aligned
     assert b"workspace" in L.tg_last_error()
+
+
+def test_select_stream_workspace_and_arguments(L):
+    """tg_topk_select_stream sizes its workspace on the host and checks it before any CUDA call."""
+    V = ctypes.c_void_p
+    seqlens, q_len, k = (131072,) * 64, (256,) * 64, (4096,) * 64
+    s = tg.Seqs(seqlens, q_len, k)
+    need = L.tg_topk_select_stream_workspace_size(s.ref())
+    ctx = sum(n - q for n, q in zip(seqlens, q_len))
+    assert need >= ctx * 8  # the candidate lists' worst case
+    assert need < ctx * 8 + (2 << 20)
+    # sequences that keep nothing or everything need no candidate space
+    assert L.tg_topk_select_stream_workspace_size(tg.Seqs((1000, 1000), (0, 0), (0, 1000)).ref()) < (2 << 20)
+    assert L.tg_topk_select_stream_workspace_size(tg.Seqs((10,), (11,), (1,)).ref()) == 0  # q > N
+    fake, ws = V(0x1000), V(0x100000)
+    call = lambda ws=ws, wsb=need, seqs=s: L.tg_topk_select_stream(fake, seqs.ref(), fake, fake, ws, wsb, None, None)
+    assert call(wsb=need - 1) == 3  # TG_ERR_WORKSPACE
+    assert call(ws=None) == 3
+    assert call(ws=V(0x100080)) == 3  # not 256-byte aligned
+    assert b"workspace" in L.tg_last_error()
+    assert call(seqs=tg.Seqs((10,), (11,), (1,))) == 1  # TG_ERR_INVALID_ARG
+    assert L.tg_topk_select_stream(None, tg.Seqs((10,), (0,), (1,)).ref(), fake, fake, ws, need, None, None) == 1
