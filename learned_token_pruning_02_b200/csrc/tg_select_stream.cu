@@ -10,11 +10,10 @@
 // issue and barriers. Here the work is cut into chunks of 8192 keys of one sequence, and four
 // kernels run in stream order (the scores are read from HBM once; the later passes find them in
 // L2):
-//   1. select_hist_kernel (one CTA of 256 threads per chunk of 8192 keys): order keys, a 12-bit histogram in shared memory,
-//      added to the sequence's global histogram with integer atomics (exact, so the totals do not
-//      depend on their order).
-//      The sequence's last CTA to finish (a counter, no waiting) finds the bin b1 that holds the
-//      K-th largest key.
+//   1. select_hist_kernel (one CTA of 256 threads per chunk): order keys, a 12-bit histogram in
+//      shared memory, added to the sequence's global histogram with integer atomics (exact, so the
+//      totals do not depend on their order). The sequence's last CTA to finish (a counter behind
+//      a fence, no waiting) finds the bin b1 that holds the K-th largest key.
 //   2. select_cand_kernel (one CTA per chunk): counts its keys above bin b1 and appends its keys
 //      in the bin, with their positions, to the sequence's candidate list (one slot reservation
 //      per CTA).
@@ -84,15 +83,15 @@ __device__ __forceinline__ int seq_of_chunk(const StreamParams& p, int c) {
 
 // Loads the chunk's keys into registers, thread-major: thread t holds positions t * SROWS + i of
 // the chunk (i = 0..SROWS-1), so the chunk's order is the threads' order and then i. Whole
-// 128-byte runs load as eight 16-byte vectors when the sequence starts on a 16-byte boundary;
-// the ragged end and unaligned sequences load word by word. Keys past the context are 0 and not
+// 128-byte runs load as eight 16-byte vectors when their address is 16-byte aligned; the ragged
+// end and unaligned runs load word by word. Keys past the context are 0 and not
 // valid (nvalid_out: this thread's valid keys). Returns whether a NaN score was seen.
 __device__ __forceinline__ bool load_chunk(const float* __restrict__ score, const StreamSeq& sq, int chunk_in_seq,
                                            uint32_t (&k)[SROWS], int* nvalid_out) {
   const int base = chunk_in_seq * CH + (int)threadIdx.x * SROWS;
   const int nvalid = max(0, min(SROWS, sq.n_ctx - base));
   const float* src = score + sq.start + base;
-  if (nvalid == SROWS && ((sq.start & 3) == 0)) {
+  if (nvalid == SROWS && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
     const float4* s4 = reinterpret_cast<const float4*>(src);
 #pragma unroll
     for (int j = 0; j < SROWS / 4; ++j) {

@@ -96,3 +96,17 @@ def test_select_stream_byte_heavy_shape():
     seqlens, q_len, k = (131072,) * 64, (256,) * 64, (4096,) * 64
     s = ti.bf16_bits_to_f32(ti.f32_to_bf16_bits(g.standard_normal(sum(seqlens)).astype(np.float32)))
     assert _check(s, seqlens, q_len, k) == 0
+
+
+def test_select_stream_unaligned_score_pointer():
+    """Scores that start 4 bytes past a 16-byte boundary load word by word, with the same result."""
+    g = np.random.default_rng(9)
+    n = 40000
+    s = g.standard_normal(n + 1).astype(np.float32)
+    sd = torch.from_numpy(s).to(DEV)[1:]
+    assert sd.data_ptr() % 16 == 4
+    kept, cu = tg.tg_topk_select_stream(sd, (n,), (100,), (1234,))
+    torch.cuda.synchronize()
+    ref, ref_cu = orc.topk_select(s[1:], (n,), (100,), (1234,))
+    assert np.array_equal(kept.cpu().numpy(), ref.astype(np.int32))
+    assert cu.cpu().numpy().tolist() == ref_cu.tolist()
