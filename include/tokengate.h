@@ -153,7 +153,7 @@ size_t tg_topk_select_stream_workspace_size(const tg_seqs* seqs);
 
 /* tg_topk_select for many long sequences at once: the same outputs bit for bit (kept_idx,
  * cu_kept_dev, TG_DEV_NAN_SCORE), computed as a stream over all SMs instead of one thread-block
- * cluster per sequence. The context is cut into chunks of 8192 tokens; four kernels run in
+ * cluster per sequence. The context is cut into chunks of 4096 tokens; four kernels run in
  * stream order: a 12-bit histogram of the order keys per sequence (integer atomics), the bin
  * holding the K-th largest key and the candidates in it, the exact threshold with each chunk's
  * output offset and quota of keys equal to it (lower positions first), and an ascending

@@ -32,7 +32,7 @@
 namespace tg {
 namespace {
 
-constexpr int SNT = 256;               // threads per chunk CTA
+constexpr int SNT = 128;               // threads per chunk CTA
 constexpr int SROWS = 32;              // keys per thread
 constexpr int CH = SNT * SROWS;        // keys per chunk
 constexpr int NB12 = 4096;             // first-level bins (top 12 bits of the order key)
@@ -145,7 +145,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int* total)
 }
 
 // ------------------------------------------------------------------ 1. histograms
-__global__ void __launch_bounds__(SNT, 4) select_hist_kernel(const float* __restrict__ score,
+__global__ void __launch_bounds__(SNT, 8) select_hist_kernel(const float* __restrict__ score,
                                                              const __grid_constant__ StreamParams p,
                                                              uint32_t* __restrict__ ghist, uint32_t* __restrict__ sinfo,
                                                              int32_t* __restrict__ dev_status) {
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(SNT, 4) select_hist_kernel(const float* __rest
 }
 
 // ------------------------------------------------------------------ 2. threshold bin, candidates
-__global__ void __launch_bounds__(SNT, 4) select_cand_kernel(const float* __restrict__ score,
+__global__ void __launch_bounds__(SNT, 8) select_cand_kernel(const float* __restrict__ score,
                                                              const __grid_constant__ StreamParams p,
                                                              uint32_t* __restrict__ sinfo, uint32_t* __restrict__ cinfo,
                                                              uint2* __restrict__ cand) {
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(RNT) select_resolve_kernel(const __grid_consta
 }
 
 // ------------------------------------------------------------------ 4. ordered compaction
-__global__ void __launch_bounds__(SNT, 4) select_compact_kernel(const float* __restrict__ score,
+__global__ void __launch_bounds__(SNT, 8) select_compact_kernel(const float* __restrict__ score,
                                                              const __grid_constant__ StreamParams p,
                                                              const uint32_t* __restrict__ sinfo,
                                                              const uint32_t* __restrict__ cinfo, int32_t* __restrict__ kept,
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(SNT, 4) select_compact_kernel(const float* __r
     mg |= (ok && k[i] > T) ? (1u << i) : 0u;
     me |= (ok && k[i] == T) ? (1u << i) : 0u;
   }
-  // the keys > T and == T before this thread (a chunk holds 8192 keys: no carry between halves)
+  // the keys > T and == T before this thread (a chunk holds 4096 keys: no carry between halves)
   const int before = block_excl_scan<SNT>((__popc(mg) << 16) | __popc(me), warp_tot, nullptr);
   int GT = before >> 16, EQ = before & 0xffff;
   bool overflow = false;

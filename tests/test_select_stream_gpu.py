@@ -42,9 +42,9 @@ def _check(s, seqlens, q_len, k):
     ((0, 5, 0), (0, 2, 0), (3, 1, 3)),  # empty sequences
     ((1,), (0,), (1,)),
     ((16385,), (1,), (16383,)),       # K = n_ctx - 1, a last chunk of one key
-    ((8193,), (0,), (4096,)),         # a last chunk of one key, unaligned thread runs at the end
-    ((40000,), (0,), (40000,)),       # every key kept across five chunks
-    ((262144,), (0,), (1000,)),       # the largest context: 32 chunks
+    ((8193,), (0,), (4096,)),         # a last chunk of one key
+    ((40000,), (0,), (40000,)),       # every key kept across ten chunks
+    ((262144,), (0,), (1000,)),       # the largest context: 64 chunks
 ])
 def test_select_stream_edge_cases(case):
     seqlens, q_len, k = case
