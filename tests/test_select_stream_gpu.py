@@ -41,7 +41,7 @@ def _check(s, seqlens, q_len, k):
     ((64,), (64,), (8,)),             # question only
     ((0, 5, 0), (0, 2, 0), (3, 1, 3)),  # empty sequences
     ((1,), (0,), (1,)),
-    ((16385,), (1,), (16383,)),       # K = n_ctx - 1, a last chunk of one key
+    ((16385,), (1,), (16383,)),       # K = n_ctx - 1 over four whole chunks
     ((8193,), (0,), (4096,)),         # a last chunk of one key
     ((40000,), (0,), (40000,)),       # every key kept across ten chunks
     ((262144,), (0,), (1000,)),       # the largest context: 64 chunks
