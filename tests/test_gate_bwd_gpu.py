@@ -29,13 +29,15 @@ def _check(got, ref, tol):
 # bf16 with dg % 128 == 0 and d % 128 == 0 runs the tensor-core kernels: one row, ragged tails of
 # 1 and of 65 rows past a 64-row chunk, three and four dg tiles, d = 384 (three K chunks per split),
 # the first product's K split 8, 4, 2 and 1 ways (65, 1000 / 2176, 4352, 10000 rows) and several
-# row splits of dW1; the rest runs on the CUDA cores.
+# row splits of dW1, and 100000 rows (782 row tiles, the u pass over 391 row blocks); the rest
+# runs on the CUDA cores.
 @pytest.mark.parametrize("dtype,M,d,dg,T", [("f32", 96, 256, 64, 1.0), ("f32", 333, 512, 128, 0.6),
                                             ("bf16", 2176, 2048, 256, 1.0), ("bf16", 1, 128, 64, 2.0),
                                             ("bf16", 4352, 2048, 256, 1.3), ("bf16", 1, 256, 128, 1.0),
                                             ("bf16", 129, 256, 128, 0.7), ("bf16", 1000, 512, 384, 1.0),
                                             ("bf16", 65, 1024, 256, 2.0), ("bf16", 200, 128, 128, 1.0),
-                                            ("bf16", 10000, 256, 128, 0.9), ("bf16", 700, 384, 512, 1.0)])
+                                            ("bf16", 10000, 256, 128, 0.9), ("bf16", 700, 384, 512, 1.0),
+                                            ("bf16", 100000, 256, 128, 1.0)])
 def test_gate_mlp_bwd_matches_oracle(dtype, M, d, dg, T):
     g = np.random.default_rng(M + d)
 
