@@ -15,8 +15,11 @@
 //     the old one) and the key tiles K_j (128 keys) into a 3-deep ring that runs across items;
 //     warp 2 loads V_j into the stage of chain j % 2; warp 3 stages each tile's per-key bias
 //     gain*log2(e)*log g_j in shared memory (a key with g = 0 is closed whatever the gain).
-//   * warp 1 (one thread): tcgen05.mma. S_j = Q K_j^T (M=128, N=128, K=D) into the chain's TMEM
-//     S buffer; O_c += P_j V_j with P_j read from TMEM (A operand in tensor memory) and V_j from
+//   * warp 1: tcgen05.mma, issued by one elected lane while the whole warp runs the schedule
+//     (its loop counters and operand descriptors stay warp-uniform, so issuing a product takes
+//     few instructions on a scheduler it shares with two softmax warps). S_j = Q K_j^T
+//     (M=128, N=128, K=D) into the chain's TMEM S buffer; O_c += P_j V_j with P_j read from
+//     TMEM (A operand in tensor memory) and V_j from
 //     shared memory (N-contiguous operand), in two halves of 64 keys so the first half enters the
 //     tensor core while the softmax computes the second. S_{j+2} is issued right after PV_j: the
 //     MMAs of one thread execute in issue order, so it overwrites P_j only after PV_j read it.
@@ -44,7 +47,7 @@ using namespace sm100;
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int NTHREADS = 384;  // warp 0: Q/K loads, 1: MMA, 2: V loads + bias, 3: idle, 4-11: softmax
+constexpr int NTHREADS = 384;  // warp 0: Q/K loads, 1: MMA, 2: V loads, 3: key bias, 4-11: softmax
 constexpr int KS = 3;           // K ring depth
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -77,6 +80,15 @@ struct ACfg {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// One lane of the (converged) warp, chosen by the hardware; the others get false.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -324,7 +336,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (warp == 1) {  // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {
+      const bool leader = elect_one();
       const uint32_t qa = smem_u32(smem + C::Q_OFF);
       int jk = 0;           // key tiles consumed (ring position)
       int pc[2] = {0, 0};  // PV products issued per chain
@@ -339,16 +352,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // way; its first PV products wait until the merge of the item before has read O.
       auto issue_s = [&](int c) -> bool {
         const int ks = jk % KS;
-        if (!mbar_wait(&kfull[ks], (jk / KS) & 1, abort, dev_status)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&kfull[ks], (jk / KS) & 1, abort, dev_status))) return false;
         tc_fence_after();
         const uint32_t ka = smem_u32(smem + C::K_OFF + ks * C::TILE_BYTES);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          mma_ss(tmem + c * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+            mma_ss(tmem + c * BKV, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), C::IDESC_QK, kk > 0);
+          }
+          mma_commit(&sfull[c]);
+          mma_commit(&kempty[ks]);
         }
-        mma_commit(&sfull[c]);
-        mma_commit(&kempty[ks]);
+        __syncwarp();
         ++jk;
         return true;
       };
@@ -356,45 +372,54 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int k = 0, w = item_of(0, G); ok && w < n_items; w = item_of(++k, G)) {
         const Item it = decode_item(w, Hq, p);
         const int nt = it.t + 1;
-        ok = mbar_wait(qfull, k & 1, abort, dev_status);
+        ok = __all_sync(0xffffffffu, mbar_wait(qfull, k & 1, abort, dev_status));
         for (int j = 0; ok && j < 2 && j < nt; ++j) ok = issue_s(j);
-        if (ok && nt <= 2) mma_commit(qempty);  // every S product of the item is issued
+        if (ok && nt <= 2 && leader) mma_commit(qempty);  // every S product of the item is issued
         for (int j = 0; ok && j < nt; ++j) {
           const int c = j & 1;
-          if (!mbar_wait(&phalf[c], pc[c] & 1, abort, dev_status) ||
-              !mbar_wait(&vfull[c], pc[c] & 1, abort, dev_status) ||
-              (j == 0 && k > 0 && !mbar_wait(oempty, (k - 1) & 1, abort, dev_status))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&phalf[c], pc[c] & 1, abort, dev_status) &&
+                                           mbar_wait(&vfull[c], pc[c] & 1, abort, dev_status) &&
+                                           (j != 0 || k == 0 || mbar_wait(oempty, (k - 1) & 1, abort, dev_status)))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t va = smem_u32(smem + C::V_OFF + c * C::TILE_BYTES);
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < BKV / 32; ++kk)  // keys 0-63: their P is in TMEM
-            mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
-                   C::IDESC_PV, (j >= 2 || kk > 0) ? 1u : 0u);
-          if (!mbar_wait(&pready[c], pc[c] & 1, abort, dev_status)) {
+            for (int kk = 0; kk < BKV / 32; ++kk)  // keys 0-63: their P is in TMEM
+              mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
+                     C::IDESC_PV, (j >= 2 || kk > 0) ? 1u : 0u);
+          }
+          __syncwarp();
+          if (!__all_sync(0xffffffffu, mbar_wait(&pready[c], pc[c] & 1, abort, dev_status))) {
             ok = false;
             break;
           }
           tc_fence_after();
+          if (leader) {
 #pragma unroll
-          for (int kk = BKV / 32; kk < BKV / 16; ++kk)  // keys 64-127
-            mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
-                   C::IDESC_PV, 1u);
-          mma_commit(&pvdone[c]);
-          mma_commit(&vempty[c]);
+            for (int kk = BKV / 32; kk < BKV / 16; ++kk)  // keys 64-127
+              mma_ts(tmem + 256 + c * D, tmem + c * BKV + kk * 8, sdesc_sw128(va + kk * 2048, BKV * 128, 1024),
+                     C::IDESC_PV, 1u);
+            mma_commit(&pvdone[c]);
+            mma_commit(&vempty[c]);
+          }
+          __syncwarp();
           ++pc[c];
           if (j + 2 < nt) {
             ok = issue_s(c);
-            if (ok && j + 3 == nt) mma_commit(qempty);  // that was the item's last S product
+            if (ok && j + 3 == nt && leader) mma_commit(qempty);  // that was the item's last S product
           }
         }
       }
-      mma_commit(drain);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {
+      if (leader) {
+        mma_commit(drain);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {
+        }
       }
+      __syncwarp();
     }
   }
   } else if (!skip) {  // ----------------------------------------------------- softmax warpgroups
