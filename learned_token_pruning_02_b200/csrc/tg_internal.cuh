@@ -29,12 +29,12 @@ uint64_t wait_probe_ns();
 // Function attributes (shared-memory size, carveout) apply per device. True until
 // mark_attrs_set(slot) is called on the current device; slots name the launchers.
 // Template kernels take one slot per instantiation (score: dg 64/128/256; attention: D 64/128
-// times the normalised / unnormalised form).
+// times the normalised / unnormalised form; projection: 128- and 256-row tiles).
 enum {
   ATTR_SCORE64 = 0, ATTR_SCORE128, ATTR_SCORE256,
   ATTR_SELECT, ATTR_GATHER,
   ATTR_ATTN64, ATTR_ATTN64_UN, ATTR_ATTN128, ATTR_ATTN128_UN,
-  ATTR_QKV, ATTR_GATE_TC, ATTR_SLOTS
+  ATTR_QKV, ATTR_GATE_TC, ATTR_QKV2, ATTR_SLOTS
 };
 bool attrs_needed(int slot);
 void mark_attrs_set(int slot);

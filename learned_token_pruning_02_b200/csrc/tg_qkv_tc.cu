@@ -7,12 +7,17 @@
 // rotary details; the reading taken: Q/K/V = H_kept W^T with one stacked W [(Hq + 2 Hkv) D, d],
 // Q and K rotated with rotate-half pairing (i, i + D/2) by angle pos * theta^(-2i/D).
 //
-// Design (B200, bf16 in, fp32 accumulate), one CTA per SM walking 128-row x 256-column tiles
-// of X = H_kept W^T:
-//   * warp 0 streams 128 x 64 slices of H_kept through a 7-deep TMA ring, warp 10 streams the
-//     matching 256 x 64 slices of W through a 3-deep ring (both 128-byte swizzle);
-//   * one thread issues tcgen05.mma M=128 N=256 K=16 into a double-buffered TMEM accumulator,
-//     so the epilogue of tile t overlaps the products of tile t+1;
+// Design (B200, bf16 in, fp32 accumulate), one CTA per SM walking 128- or 256-row x
+// 256-column tiles of X = H_kept W^T:
+//   * warp 0 streams 128 x 64 slices of H_kept through a 7-deep TMA ring (256 x 64 slices
+//     through a 3-deep ring for 256-row tiles), warp 10 streams the matching 256 x 64 slices of
+//     W through a 3-deep ring (all 128-byte swizzle);
+//   * one elected lane of warp 1 issues tcgen05.mma M=128 N=256 K=16. With 128-row tiles the
+//     two TMEM accumulators are a double buffer, so the epilogue of tile t overlaps the products
+//     of tile t+1. Once 128-row tiles would take more than one round of the SMs, a tile is 256
+//     rows: both accumulators take one tile, its two 128-row products read every W slice from
+//     shared memory once (a third fewer operand bytes per product, and at 2176 kept rows 144
+//     tiles in one round instead of 272 in two), at the cost of an exposed epilogue;
 //   * warps 2-9 are the epilogue: per TMEM lane quarter two warps, each owning a 128-column half
 //     of the tile (one head for D = 128, two for D = 64). For a Q or K head a thread loads
 //     columns i and i + D/2 together, rotates the pair, and stores bf16 rows. The angle
@@ -28,20 +33,38 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;  // kept rows per tile
 constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 64;
 constexpr int NEPI = 8;                    // epilogue warps (warps 2..9)
 constexpr int WPROD = 2 + NEPI;            // warp that streams W
 constexpr int NTHREADS = 32 * (3 + NEPI);  // 352
-constexpr int A_BYTES = BM * BK * 2;       // 16 KB
 constexpr int B_BYTES = BN * BK * 2;       // 32 KB
-constexpr int AS = 7, WS = 3;              // ring depths
+constexpr int WS = 3;                      // W ring depth
 constexpr int TAIL = 1024;
-constexpr int SMEM = 1024 + AS * A_BYTES + WS * B_BYTES + TAIL;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false);
-static_assert(SMEM <= 227 * 1024, "shared memory budget");
+constexpr uint32_t IDESC = idesc_bf16_f32(128, BN, false);
+
+// A tile is NACC x 128 kept rows by 256 columns, with NACC accumulators of 128 x 256 fp32 in TMEM.
+//   NACC = 1: the two accumulators are a double buffer, so a tile's epilogue overlaps the next
+//             tile's products (a 7-deep ring of 16 KB H_kept slices);
+//   NACC = 2: both hold one tile, whose two 128-row products share every W slice, which cuts the
+//             operand bytes per product by a third (a 3-deep ring of 32 KB H_kept slices).
+template <int NACC>
+struct QCfg {
+  static constexpr int BM = 128 * NACC;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int AS = NACC == 1 ? 7 : 3;
+  static constexpr int NSET = 2 / NACC;  // accumulator sets in TMEM
+  static constexpr int SMEM = 1024 + AS * A_BYTES + WS * B_BYTES + TAIL;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+// One lane of the (converged) warp, chosen by the hardware; the others get false.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}" : "=r"(pred));
+  return pred != 0;
+}
 
 struct QKVParams {
   int M;        // kept rows
@@ -53,11 +76,14 @@ struct QKVParams {
   double inv[64];      // theta^(-2i/D), i < D/2
 };
 
+template <int NACC>
 __global__ void __launch_bounds__(NTHREADS, 1)
     qkv_rope_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ Qo, __nv_bfloat16* __restrict__ Ko,
                     __nv_bfloat16* __restrict__ Vo, int32_t* __restrict__ dev_status, uint64_t probe_ns,
                     const __grid_constant__ QKVParams p) {
+  using C = QCfg<NACC>;
+  constexpr int BM = C::BM, AS = C::AS, A_BYTES = C::A_BYTES, NSET = C::NSET;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smem_w = smem + AS * A_BYTES;
@@ -66,8 +92,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* aempty = afull + AS;                        // [AS]
   uint64_t* wfull = aempty + AS;                        // [WS]
   uint64_t* wempty = wfull + WS;                        // [WS]
-  uint64_t* accf = wempty + WS;                         // [2] accumulator complete
-  uint64_t* acce = accf + 2;                            // [2] accumulator consumed
+  uint64_t* accf = wempty + WS;                         // [NSET] accumulator set complete
+  uint64_t* acce = accf + 2;                            // [NSET] accumulator set consumed
   uint64_t* drain = acce + 2;
   uint64_t* probe = drain + 1;  // test hook: a barrier nothing signals
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(probe + 1);
@@ -83,7 +109,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&wfull[s], 1);
       mbar_init(&wempty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NSET; ++a) {
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], NEPI);
     }
@@ -146,29 +172,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {  // ------------------------------------------------------------ MMA issuer
+    {  // -------------------------- MMA issuer: the warp runs the schedule, one elected lane issues
+      const bool leader = elect_one();
       int as = 0, ws = 0;
       uint32_t aph = 0, wph = 0;
       int it = 0;
       for (int tile = blockIdx.x; tile < p.tiles && !*abort; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        if (!mbar_wait(&acce[acc], ((it >> 1) & 1) ^ 1u, abort, dev_status)) break;
+        const int set = it % NSET;
+        if (!__all_sync(0xffffffffu, mbar_wait(&acce[set], ((it / NSET) & 1) ^ 1u, abort, dev_status))) break;
         tc_fence_after();
-        const uint32_t d = tmem + acc * BN;
+        const uint32_t d = tmem + set * NACC * BN;
         bool ok = true;
         for (int i = 0; i < nk; ++i) {
-          if (!mbar_wait(&afull[as], aph, abort, dev_status) || !mbar_wait(&wfull[ws], wph, abort, dev_status)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&afull[as], aph, abort, dev_status) &&
+                                           mbar_wait(&wfull[ws], wph, abort, dev_status))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + as * A_BYTES);
           const uint32_t b0 = smem_u32(smem_w + ws * B_BYTES);
+          if (leader) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            mma_ss(d, sdesc_sw128(a0 + 32 * k, 16, 1024), sdesc_sw128(b0 + 32 * k, 16, 1024), IDESC, (i | k) != 0);
-          mma_commit(&aempty[as]);
-          mma_commit(&wempty[ws]);
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint64_t bd = sdesc_sw128(b0 + 32 * k, 16, 1024);
+#pragma unroll
+              for (int a = 0; a < NACC; ++a)  // rows 128a..128a+127 of the slice start 16 KB apart
+                mma_ss(d + a * BN, sdesc_sw128(a0 + a * (128 * 128) + 32 * k, 16, 1024), bd, IDESC, (i | k) != 0);
+            }
+            mma_commit(&aempty[as]);
+            mma_commit(&wempty[ws]);
+          }
+          __syncwarp();
           if (++as == AS) {
             as = 0;
             aph ^= 1u;
@@ -179,9 +214,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         if (!ok) break;
-        mma_commit(&accf[acc]);
+        if (leader) mma_commit(&accf[set]);
+        __syncwarp();
       }
-      mma_commit(drain);  // every product issued above completes before TMEM can be released
+      if (leader) mma_commit(drain);  // every product issued above completes before TMEM can be released
+      __syncwarp();
     }
   } else if (warp < WPROD) {  // ------------------------------------ epilogue: warps 2..9
     const int half = (warp - 2) >> 2;  // which 128-column half of the tile
@@ -191,11 +228,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     int it = 0;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
-      const int acc = it & 1;
+      const int set = it % NSET;
       // warp-uniform: the tcgen05.ld below is warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&accf[acc], (it >> 1) & 1, abort, dev_status))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&accf[set], (it / NSET) & 1, abort, dev_status))) break;
       tc_fence_after();
-      const int gm = (tile / p.tiles_n) * BM + r;
+#pragma unroll 1
+      for (int a = 0; a < NACC; ++a) {  // the tile's 128-row blocks
+      const int acc = set * NACC + a;    // accumulator in TMEM
+      const int gm = (tile / p.tiles_n) * BM + a * 128 + r;
       const bool valid = gm < p.M;
       const double pr = (valid && p.rotate) ? (double)pos[gm] : 0.0;  // pos may be NULL without rotation
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * BN + half * 128;
@@ -258,9 +298,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
       }
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[acc]);  // the accumulator may take the next tile
+      if (lane == 0) mbar_arrive(&acce[set]);  // the accumulators may take the next tile
     }
   }
 
@@ -276,6 +317,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+template <int NACC>
+tg_status launch_qkv_nacc(const void* Hk, int64_t M, int d, const void* W, const int32_t* pos, int N,
+                          QKVParams& p, void* Q, void* K, void* V, int32_t* dev_status, cudaStream_t st) {
+  using C = QCfg<NACC>;
+  p.tiles = (int)((M + C::BM - 1) / C::BM) * p.tiles_n;
+  CUtensorMap tmA, tmW;
+  if (!make_tmap_bf16_2d(&tmA, Hk, (uint64_t)M, (uint64_t)d, (uint64_t)d, C::BM, BK) ||
+      !make_tmap_bf16_2d(&tmW, W, (uint64_t)N, (uint64_t)d, (uint64_t)d, BN, BK))
+    return fail(TG_ERR_CUDA, "tg_qkv_rope: building the TMA tensor maps failed");
+  const int slot = NACC == 1 ? ATTR_QKV : ATTR_QKV2;
+  if (attrs_needed(slot)) {
+    cudaError_t e = cudaFuncSetAttribute(qkv_rope_kernel<NACC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return cuda_status(e, "tg_qkv_rope: cudaFuncSetAttribute");
+    mark_attrs_set(slot);
+  }
+  int ctas = device_sm_count();
+  if (ctas > p.tiles) ctas = p.tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = (size_t)C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute(PDL_QKV)};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, qkv_rope_kernel<NACC>, tmA, tmW, pos, static_cast<__nv_bfloat16*>(Q),
+                                        static_cast<__nv_bfloat16*>(K), static_cast<__nv_bfloat16*>(V), dev_status,
+                                        wait_probe_ns(), p),
+                     "tg_qkv_rope: launch");
+}
+
 }  // namespace
 
 tg_status launch_qkv_rope(const void* Hk, int64_t M, int d, const void* W, const int32_t* pos, int Hq, int Hkv,
@@ -285,36 +357,17 @@ tg_status launch_qkv_rope(const void* Hk, int64_t M, int d, const void* W, const
   p.M = (int)M;
   p.nk = d / BK;
   p.tiles_n = N / BN;
-  p.tiles = (int)((M + BM - 1) / BM) * p.tiles_n;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.D = D;
   p.rotate = theta > 0.f ? 1 : 0;
   for (int i = 0; i < D / 2; ++i) p.inv[i] = p.rotate ? pow((double)theta, -2.0 * i / D) : 0.0;
-  if (p.tiles == 0) return TG_OK;
-  CUtensorMap tmA, tmW;
-  if (!make_tmap_bf16_2d(&tmA, Hk, (uint64_t)M, (uint64_t)d, (uint64_t)d, BM, BK) ||
-      !make_tmap_bf16_2d(&tmW, W, (uint64_t)N, (uint64_t)d, (uint64_t)d, BN, BK))
-    return fail(TG_ERR_CUDA, "tg_qkv_rope: building the TMA tensor maps failed");
-  if (attrs_needed(ATTR_QKV)) {
-    cudaError_t e = cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (e != cudaSuccess) return cuda_status(e, "tg_qkv_rope: cudaFuncSetAttribute");
-    mark_attrs_set(ATTR_QKV);
-  }
-  int ctas = device_sm_count();
-  if (ctas > p.tiles) ctas = p.tiles;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)ctas);
-  cfg.blockDim = dim3(NTHREADS);
-  cfg.dynamicSmemBytes = (size_t)SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1] = {pdl_attribute(PDL_QKV)};
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, qkv_rope_kernel, tmA, tmW, pos, static_cast<__nv_bfloat16*>(Q),
-                                        static_cast<__nv_bfloat16*>(K), static_cast<__nv_bfloat16*>(V), dev_status,
-                                        wait_probe_ns(), p),
-                     "tg_qkv_rope: launch");
+  const int64_t tiles128 = (M + 127) / 128 * p.tiles_n;
+  if (tiles128 == 0) return TG_OK;
+  // 256-row tiles once 128-row tiles would take more than one round of the SMs: fewer operand
+  // bytes per product; below that, 128-row tiles keep more SMs busy.
+  if (tiles128 > device_sm_count()) return launch_qkv_nacc<2>(Hk, M, d, W, pos, N, p, Q, K, V, dev_status, st);
+  return launch_qkv_nacc<1>(Hk, M, d, W, pos, N, p, Q, K, V, dev_status, st);
 }
 
 }  // namespace tg

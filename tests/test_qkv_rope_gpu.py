@@ -1,7 +1,9 @@
 """Projection of the kept rows to Q/K/V with rotary embedding at original positions
 (tg_qkv_rope) against the oracle's qkv_rope, within the bf16 tolerance. Cases cover two heads
 per 128-column half (D = 64), the Qwen3-1.7B shapes, positions near 128K tokens (angles of
-about 1e5 radians before reduction) and no rotation."""
+about 1e5 radians before reduction), no rotation, and both tile heights: 128-row tiles while
+they fit one round of the SMs, 256-row tiles (two accumulators sharing every W slice) beyond,
+with a ragged last tile and several tiles per SM."""
 import numpy as np
 import pytest
 import torch
@@ -15,9 +17,11 @@ pytestmark = pytest.mark.gpu
 
 CASES = [  # (M, d, Hq, Hkv, D, theta, max position)
     (300, 256, 4, 2, 64, 1.0e4, 3000),
-    (1088, 2048, 16, 8, 128, 1.0e6, 8192),
+    (1088, 2048, 16, 8, 128, 1.0e6, 8192),       # 144 tiles of 128 rows: one round of the SMs
     (256, 256, 2, 1, 128, 1.0e4, 131072),
     (200, 512, 2, 1, 128, 0.0, 1000),
+    (2300, 2048, 16, 8, 128, 1.0e6, 32768),      # 256-row tiles, the last one 252 rows deep
+    (4352, 1024, 16, 8, 128, 1.0e6, 131072),     # 256-row tiles, about two per SM
 ]
 
 
