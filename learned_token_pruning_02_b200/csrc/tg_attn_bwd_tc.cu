@@ -323,37 +323,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     } else if (warp == 1) {  // ------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      {
+        const bool leader = elect_one();
         const uint32_t ka = smem_u32(smem + C::K_OFF), va = smem_u32(smem + C::V_OFF);
         auto qa = [&](int n) { return smem_u32(smem + C::Q_OFF + (n & 1) * 2 * C::TILE); };
         auto issue_ss = [&](uint32_t d, uint32_t a, uint32_t bq) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t o = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-            mma_ss(d, sdesc_sw128(a + o, 16, 1024), sdesc_sw128(bq + o, 16, 1024), C::IDESC_S, kk > 0);
+            if (leader) mma_ss(d, sdesc_sw128(a + o, 16, 1024), sdesc_sw128(bq + o, 16, 1024), C::IDESC_S, kk > 0);
           }
         };
         // Program per step n: dP^T_n into region A once the epilogue holds S^T_n, dV_n once P^T_n
         // is in TMEM, S^T_{n+1} into A once the epilogue holds dP^T_n, dK_n once dS^T_n is in TMEM.
-        bool ok = mbar_wait(kvfull, 0, abort, dev_status) && mbar_wait(&qfull[0], 0, abort, dev_status);
+        bool ok = __all_sync(0xffffffffu, mbar_wait(kvfull, 0, abort, dev_status)) && __all_sync(0xffffffffu, mbar_wait(&qfull[0], 0, abort, dev_status));
         if (ok) {
           tc_fence_after();
           issue_ss(tmem + 0, ka, qa(0));  // S^T_0 = K Q_0^T
-          mma_commit(sfull);
+          if (leader) mma_commit(sfull);
         }
         for (int n = 0; ok && n < N; ++n) {
           const uint32_t ph = n & 1;
           const uint32_t q_a = qa(n), do_a = q_a + C::TILE;
-          if (!mbar_wait(sfree, ph, abort, dev_status)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(sfree, ph, abort, dev_status))) {
             ok = false;
             break;
           }
           tc_fence_after();
           issue_ss(tmem + 0, va, do_a);  // dP^T_n = V dO_n^T
-          mma_commit(dpfull);
+          if (leader) mma_commit(dpfull);
           // dV += P^T dO in the two query halves, each as soon as its P^T is in TMEM
           for (int c = 0; c < 2; ++c) {
-            if (!mbar_wait(&pready[c], ph, abort, dev_status)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&pready[c], ph, abort, dev_status))) {
               ok = false;
               break;
             }
@@ -361,24 +362,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const int kk = 4 * c + k4;
-              mma_ts(tmem + C::T_DV, tmem + C::T_P + c * 32 + k4 * 8, sdesc_sw128(do_a + kk * 2048, BT * 128, 1024),
+              if (leader) mma_ts(tmem + C::T_DV, tmem + C::T_P + c * 32 + k4 * 8, sdesc_sw128(do_a + kk * 2048, BT * 128, 1024),
                      C::IDESC_G, (n > 0 || kk > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
-          mma_commit(pfree);
+          if (leader) mma_commit(pfree);
           if (n + 1 < N) {  // S^T_{n+1} = K Q_{n+1}^T into region A
-            if (!mbar_wait(afree, ph, abort, dev_status) ||
-                !mbar_wait(&qfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, dev_status)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(afree, ph, abort, dev_status)) ||
+                !__all_sync(0xffffffffu, mbar_wait(&qfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, dev_status))) {
               ok = false;
               break;
             }
             tc_fence_after();
             issue_ss(tmem + 0, ka, qa(n + 1));
-            mma_commit(sfull);
+            if (leader) mma_commit(sfull);
           }
           for (int c = 0; c < 2; ++c) {  // dK += dS^T Q
-            if (!mbar_wait(&dsready[c], ph, abort, dev_status)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&dsready[c], ph, abort, dev_status))) {
               ok = false;
               break;
             }
@@ -386,17 +387,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const int kk = 4 * c + k4;
-              mma_ts(tmem + C::T_DK, tmem + C::T_DS + c * 32 + k4 * 8, sdesc_sw128(q_a + kk * 2048, BT * 128, 1024),
+              if (leader) mma_ts(tmem + C::T_DK, tmem + C::T_DS + c * 32 + k4 * 8, sdesc_sw128(q_a + kk * 2048, BT * 128, 1024),
                      C::IDESC_G, (n > 0 || kk > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
-          mma_commit(dsfree);
-          mma_commit(&qempty[n & 1]);  // the stage's Q and dO are no longer read
+          if (leader) mma_commit(dsfree);
+          if (leader) mma_commit(&qempty[n & 1]);  // the stage's Q and dO are no longer read
         }
-        if (ok) mma_commit(accdone);
-        mma_commit(drain);
-        settle(drain, 0);
+        if (ok && leader) mma_commit(accdone);
+        if (leader) mma_commit(drain);
+        if (leader) settle(drain, 0);
+        __syncwarp();
       }
     } else if (warp == 3) {  // ----------------------------------- per-query vectors stager
       // -lse * log2(e) (-inf for rows past the sequence, whose lse reads as +inf) and -Dv of
@@ -791,37 +793,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     } else if (warp == 1) {  // ------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      {
+        const bool leader = elect_one();
         const uint32_t qa = smem_u32(smem + C::Q_OFF), doa = smem_u32(smem + C::DO_OFF);
         auto ka = [&](int j) { return smem_u32(smem + C::K_OFF + (j % C::KSL) * C::TILE); };
         auto issue_ss = [&](uint32_t d, uint32_t a, uint32_t bk) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t o = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-            mma_ss(d, sdesc_sw128(a + o, 16, 1024), sdesc_sw128(bk + o, 16, 1024), C::IDESC_S, kk > 0);
+            if (leader) mma_ss(d, sdesc_sw128(a + o, 16, 1024), sdesc_sw128(bk + o, 16, 1024), C::IDESC_S, kk > 0);
           }
         };
         auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T into buffer j % 2
-          if (!mbar_wait(&kfull[j % C::KSL], (j / C::KSL) & 1, abort, dev_status)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&kfull[j % C::KSL], (j / C::KSL) & 1, abort, dev_status))) return false;
           tc_fence_after();
           issue_ss(tmem + (j & 1) * 128, qa, ka(j));
-          mma_commit(&sfull[j & 1]);
+          if (leader) mma_commit(&sfull[j & 1]);
           return true;
         };
         auto issue_dp = [&](int j) -> bool {  // dP_j = dO V_j^T
-          if (!mbar_wait(&vfull[j & 1], (j >> 1) & 1, abort, dev_status)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&vfull[j & 1], (j >> 1) & 1, abort, dev_status))) return false;
           tc_fence_after();
           issue_ss(tmem + C::T_DP, doa, smem_u32(smem + C::V_OFF + (j & 1) * C::TILE));
-          mma_commit(dpfull);
-          mma_commit(&vempty[j & 1]);
+          if (leader) mma_commit(dpfull);
+          if (leader) mma_commit(&vempty[j & 1]);
           return true;
         };
-        bool ok = mbar_wait(qfull, 0, abort, dev_status);
+        bool ok = __all_sync(0xffffffffu, mbar_wait(qfull, 0, abort, dev_status));
         ok = ok && issue_s(0) && issue_dp(0) && (N < 2 || issue_s(1));
         for (int j = 0; ok && j < N; ++j) {
           const uint32_t k_a = ka(j);
           for (int c = 0; c < 2; ++c) {  // dQ += dS K_j, each key half as soon as its dS is in TMEM
-            if (!mbar_wait(&dsready[c], j & 1, abort, dev_status)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&dsready[c], j & 1, abort, dev_status))) {
               ok = false;
               break;
             }
@@ -829,20 +832,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const int kk = 4 * c + k4;
-              mma_ts(tmem + C::T_DQ, tmem + C::T_DP + c * 64 + k4 * 8, sdesc_sw128(k_a + kk * 2048, BT * 128, 1024),
+              if (leader) mma_ts(tmem + C::T_DQ, tmem + C::T_DP + c * 64 + k4 * 8, sdesc_sw128(k_a + kk * 2048, BT * 128, 1024),
                      C::IDESC_G, (j > 0 || kk > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
-          mma_commit(&kempty[j % C::KSL]);
+          if (leader) mma_commit(&kempty[j % C::KSL]);
           // dP_{j+1} overwrites dS_j only after dQ_j read it; S_{j+2} reuses S_j's buffer, which
           // the epilogue finished reading before it wrote dS_j
           if (j + 1 < N) ok = issue_dp(j + 1);
           if (ok && j + 2 < N) ok = issue_s(j + 2);
         }
-        if (ok) mma_commit(accdone);
-        mma_commit(drain);
-        settle(drain, 0);
+        if (ok && leader) mma_commit(accdone);
+        if (leader) mma_commit(drain);
+        if (leader) settle(drain, 0);
+        __syncwarp();
       }
     } else if (warp == 3) {  // ------------------------------------------- key bias stager
       const float gain2 = (gain ? __ldcg(gain + h) : 1.f) * kLog2e;

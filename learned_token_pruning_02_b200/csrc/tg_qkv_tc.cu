@@ -59,13 +59,6 @@ struct QCfg {
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
-// One lane of the (converged) warp, chosen by the hardware; the others get false.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t pred = 0;
-  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}" : "=r"(pred));
-  return pred != 0;
-}
-
 struct QKVParams {
   int M;        // kept rows
   int nk;       // d / 64
