@@ -197,30 +197,34 @@ __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {  // ------------------------------------------------------------ MMA issuer
+    {  // --------------------------- MMA issuer: the warp runs the schedule, one elected lane issues
+      const bool leader = elect_one();
       int hs = 0, ws = 0;
       uint32_t hph = 0, wph = 0;
       int it = 0;
       for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x, ++it) {
         const int acc = it & 1;
-        if (!mbar_wait(&acce[acc], ((it >> 1) & 1) ^ 1u, abort, dev_status)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&acce[acc], ((it >> 1) & 1) ^ 1u, abort, dev_status))) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * DG;
         bool ok = true;
         for (int i = 0; i < nk; ++i) {
-          if (!mbar_wait(&hfull[hs], hph, abort, dev_status) || !mbar_wait(&wfull[ws], wph, abort, dev_status)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&hfull[hs], hph, abort, dev_status) &&
+                                           mbar_wait(&wfull[ws], wph, abort, dev_status))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + hs * C::A_BYTES);
           const uint32_t b0 = smem_u32(smem_w + ws * C::B_BYTES);
+          if (leader) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            mma_ss(d, sdesc_sw128(a0 + 32 * k, 16, 1024), sdesc_sw128(b0 + 32 * k, 16, 1024), C::IDESC,
-                   (i | k) != 0);
-          mma_commit(&hempty[hs]);
-          mma_commit(&wempty[ws]);
+            for (int k = 0; k < BK / 16; ++k)
+              mma_ss(d, sdesc_sw128(a0 + 32 * k, 16, 1024), sdesc_sw128(b0 + 32 * k, 16, 1024), C::IDESC, (i | k) != 0);
+            mma_commit(&hempty[hs]);
+            mma_commit(&wempty[ws]);
+          }
+          __syncwarp();
           if (++hs == C::HS) {
             hs = 0;
             hph ^= 1u;
@@ -231,9 +235,9 @@ __global__ void __launch_bounds__(Cfg<DG>::NTHREADS, 1)
           }
         }
         if (!ok) break;
-        mma_commit(&accf[acc]);
+        if (leader) mma_commit(&accf[acc]);
       }
-      mma_commit(drain);  // every MMA issued above completes before TMEM can be released
+      if (leader) mma_commit(drain);  // every MMA issued above completes before TMEM can be released
     }
   } else if (warp < WPROD) {  // ------------------------------------ epilogue: warps 2..9
     const int grp = (warp - 2) >> 2;  // column group
