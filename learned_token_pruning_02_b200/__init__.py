@@ -149,6 +149,13 @@ def _dtype(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
 
 
+def _like(ref_name, ref, **named):
+    """Operands the C ABI reads in the element type of `ref` (bf16 or fp32) must share its dtype."""
+    for name, t in named.items():
+        if t is not None and t.dtype != ref.dtype:
+            raise TypeError(f"{name} must have {ref_name}'s dtype {ref.dtype}, got {t.dtype}")
+
+
 def _want(dtype, **named):
     """Side tensors (scores, gates, positions, indices, status words, gradients) must have the
     library's fixed dtype and be contiguous: the C ABI reads them as plain arrays."""
@@ -217,6 +224,7 @@ def tg_score(H, W1, b1, w2, b2: float, score=None, dev_status=None, stream=None,
     """Gate-MLP score of every token: (w2 . GELU(W1 h + b1) + b2) / temperature (float32 [n_tok])."""
     _want(torch.float32, b1=b1, score=score)
     _want(torch.int32, dev_status=dev_status)
+    _like("H", H, W1=W1, w2=w2)
     _cuda(H, W1, b1, w2, score, dev_status)
     n_tok, d = H.shape
     assert H.stride(1) == 1 and W1.is_contiguous() and w2.is_contiguous()
@@ -283,6 +291,7 @@ def tg_qkv_rope(H_kept, W_qkv, pos, Hq: int, Hkv: int, D: int, rope_theta: float
                 dev_status=None, stream=None):
     """Q, K, V of the kept rows (bf16), Q and K rotated at their original positions: (Q, K, V)."""
     _want(torch.int32, pos=pos, dev_status=dev_status)
+    _like("H_kept", H_kept, W_qkv=W_qkv, Q=Q, K=K, V=V)
     M, d = H_kept.shape
     _contig(H_kept=H_kept, W_qkv=W_qkv)
     _shape("W_qkv", W_qkv, ((Hq + 2 * Hkv) * D, d))
@@ -339,6 +348,7 @@ def tg_gather(H, score, kept_idx, seqlens, q_len, k, flags=0, H_kept=None, pos=N
     """Kept rows of H with their positions and gate values: (H_kept, pos, g, logg)."""
     _want(torch.float32, score=score, g=g, logg=logg)
     _want(torch.int32, kept_idx=kept_idx, pos=pos, dev_status=dev_status)
+    _like("H", H, H_kept=H_kept)
     _cuda(H, score, kept_idx, H_kept, pos, g, logg, dev_status)
     s = Seqs(seqlens, q_len, k)
     m = kept_idx.numel()
@@ -359,6 +369,7 @@ def tg_gated_attn_fwd(Q, K, V, logg, pos, cu_kept, softmax_scale: float, head_ga
     """Token-gated causal attention over the kept tokens: (O [M, Hq, D], lse [Hq, M] or None)."""
     _want(torch.float32, logg=logg, head_gain=head_gain, lse=lse)
     _want(torch.int32, pos=pos, dev_status=dev_status)
+    _like("Q", Q, K=K, V=V, O=O)
     _cuda(Q, K, V, logg, pos, head_gain, O, lse, dev_status)
     M, Hq, D = Q.shape
     Hkv = K.shape[1]
@@ -434,6 +445,7 @@ def tg_gate_mlp_bwd(H_kept, W1, b1, w2, dscore, temperature: float = 1.0, dW1=No
     ``dev_status`` an int32 device word that a timed-out wait ORs TG_DEV_TIMEOUT into."""
     _want(torch.float32, b1=b1, dscore=dscore, dW1=dW1, db1=db1, dw2=dw2, db2=db2)
     _want(torch.int32, dev_status=dev_status)
+    _like("H_kept", H_kept, W1=W1, w2=w2)
     M, d = H_kept.shape
     dg = W1.shape[0]
     _contig(H_kept=H_kept, W1=W1, w2=w2)
@@ -467,6 +479,7 @@ def tg_gate_mlp_bwd_noalloc(H_kept, W1, b1, w2, dscore, dW1, db1, dw2, db2, temp
     the place of the workspace, and every output buffer is the caller's (nothing is allocated
     here either). Calls on one device share the array: do not let them overlap on the GPU."""
     _want(torch.float32, b1=b1, dscore=dscore, dW1=dW1, db1=db1, dw2=dw2, db2=db2)
+    _like("H_kept", H_kept, W1=W1, w2=w2)
     M, d = H_kept.shape
     dg = W1.shape[0]
     _contig(H_kept=H_kept, W1=W1, w2=w2)
@@ -491,6 +504,7 @@ def tg_prefill_above_L(H, W1, b1, w2, b2, seqlens, q_len, k, layers, softmax_sca
     """
     _want(torch.float32, b1=b1, head_gain=head_gain)
     _want(torch.int32, dev_status=dev_status)
+    _like("H", H, W1=W1, w2=w2)
     _cuda(H, W1, b1, w2, head_gain, dev_status)
     s = Seqs(seqlens, q_len, k)
     cu = tg_kept_counts(seqlens, q_len, k)
@@ -537,6 +551,7 @@ def tg_prefill_projected(H, W1, b1, w2, b2, seqlens, q_len, k, W_qkv, rope_theta
     kept_idx, cu_kept_dev, H_kept, pos, g, logg and per-layer lists Q, K_cache, V_cache, O, lse."""
     _want(torch.float32, b1=b1, head_gain=head_gain)
     _want(torch.int32, dev_status=dev_status)
+    _like("H", H, W1=W1, w2=w2, **{f"W_qkv[{i}]": W for i, W in enumerate(W_qkv)})
     n_tok, d = H.shape
     for i, W in enumerate(W_qkv):
         _contig(**{f"W_qkv[{i}]": W})

@@ -196,25 +196,32 @@ __global__ void __launch_bounds__(GTHREADS, 1)
       if (*ct.abort) drain_copies<NS>(ct, issued);
     }
   } else if (warp == 1) {  // -------------------------------------------------------- MMA
-    if (lane == 0) {
+    {  // the warp runs the schedule, one elected lane issues
+      const bool leader = elect_one();
       bool ok = true;
       for (int k = 0; k < nk; ++k) {
         const int s = k % NS;
-        if (!mbar_wait(&ct.full[s], (k / NS) & 1, ct.abort, dev_status)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&ct.full[s], (k / NS) & 1, ct.abort, dev_status))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t a = smem_u32(smem + s * C::STAGE), b = a + C::A_BYTES;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < KCH / 16; ++kk)
-          mma_ss(tmem, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 32, 16, 1024), C::IDESC,
-                 (k > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&ct.empty[s]);
+          for (int kk = 0; kk < KCH / 16; ++kk)
+            mma_ss(tmem, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 32, 16, 1024), C::IDESC,
+                   (k > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&ct.empty[s]);
+        }
+        __syncwarp();
       }
-      if (ok) mma_commit(ct.accdone);
-      mma_commit(ct.drain);
-      settle(ct.drain, 0);
+      if (ok && leader) mma_commit(ct.accdone);
+      if (leader) {
+        mma_commit(ct.drain);
+        settle(ct.drain, 0);
+      }
+      __syncwarp();
     }
   } else {  // ------------------------------------------------------ epilogue: one row per thread
     const int q4 = warp & 3, r = q4 * 32 + lane;
@@ -363,11 +370,12 @@ __global__ void __launch_bounds__(GTHREADS, 1)
       if (*ct.abort) drain_copies<WST>(ct, issued);
     }
   } else if (warp == 1) {  // -------------------------------------------------------- MMA
-    if (lane == 0) {
+    {  // the warp runs the schedule, one elected lane issues
+      const bool leader = elect_one();
       bool ok = true;
       for (int k = 0; k < nk; ++k) {
         const int s = k % WST;
-        if (!mbar_wait(&ct.full[s], (k / WST) & 1, ct.abort, dev_status)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&ct.full[s], (k / WST) & 1, ct.abort, dev_status))) {
           ok = false;
           break;
         }
@@ -376,15 +384,21 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         // A: 128 rows of u^T x 64 kept rows, K-major. B: 64 kept rows x 256 columns of d as four
         // boxes of 64 columns (N-contiguous; the leading offset steps from box to box), 16 kept
         // rows (2048 bytes) per instruction.
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < KCH / 16; ++kk)
-          mma_ss(tmem, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 2048, C::B_BOX, 1024), C::IDESC,
-                 (k > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&ct.empty[s]);
+          for (int kk = 0; kk < KCH / 16; ++kk)
+            mma_ss(tmem, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(b + kk * 2048, C::B_BOX, 1024), C::IDESC,
+                   (k > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&ct.empty[s]);
+        }
+        __syncwarp();
       }
-      if (ok) mma_commit(ct.accdone);
-      mma_commit(ct.drain);
-      settle(ct.drain, 0);
+      if (ok && leader) mma_commit(ct.accdone);
+      if (leader) {
+        mma_commit(ct.drain);
+        settle(ct.drain, 0);
+      }
+      __syncwarp();
     }
   } else {  // ------------------------------------------ epilogue: the tile into shared memory
     const int q4 = warp & 3, r = q4 * 32 + lane;

@@ -202,6 +202,31 @@ def test_binding_refuses_wrong_side_dtypes():
                              dQ=torch.zeros(4, 2, 64, dtype=torch.bfloat16))
 
 
+def test_binding_refuses_mixed_element_types():
+    """Operands read in the element type of H (or Q) must share its dtype: an fp32 w2 beside bf16
+    H would otherwise be read as bf16 pairs of its bytes."""
+    import torch
+    bf, f32 = torch.bfloat16, torch.float32
+    H = torch.zeros(8, 128, dtype=bf)
+    W1, b1 = torch.zeros(64, 128, dtype=bf), torch.zeros(64)
+    with pytest.raises(TypeError, match="w2 must have H's dtype"):
+        tg.tg_score(H, W1, b1, torch.zeros(64, dtype=f32), 0.0)
+    with pytest.raises(TypeError, match="W1 must have H_kept's dtype"):
+        tg.tg_gate_mlp_bwd(H, W1.float(), b1, torch.zeros(64, dtype=bf), torch.zeros(8))
+    with pytest.raises(TypeError, match="w2 must have H_kept's dtype"):
+        tg.tg_gate_mlp_bwd_noalloc(H, W1, b1, torch.zeros(64), torch.zeros(8), torch.zeros(64, 128),
+                                   torch.zeros(64), torch.zeros(64), torch.zeros(1))
+    with pytest.raises(TypeError, match="W_qkv must have H_kept's dtype"):
+        tg.tg_qkv_rope(H, torch.zeros(4 * 64, 128), None, 2, 1, 64, 0.0)
+    with pytest.raises(TypeError, match="H_kept must have H's dtype"):
+        tg.tg_gather(H, torch.zeros(8), torch.zeros(4, dtype=torch.int32), (8,), (2,), (2,),
+                     H_kept=torch.zeros(4, 128))
+    Q = torch.zeros(4, 2, 64, dtype=bf)
+    with pytest.raises(TypeError, match="V must have Q's dtype"):
+        tg.tg_gated_attn_fwd(Q, torch.zeros(4, 1, 64, dtype=bf), torch.zeros(4, 1, 64), None,
+                             torch.arange(4, dtype=torch.int32), [0, 4], 0.1)
+
+
 def test_binding_checks_projection_shapes():
     """tg_qkv_rope builds its TMA maps from M, d and the head counts, so a short W_qkv or a
     strided H_kept would be read wrongly on the device: the binding refuses them first."""
