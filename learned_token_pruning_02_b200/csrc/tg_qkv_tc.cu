@@ -10,17 +10,19 @@
 // Design (B200, bf16 in, fp32 accumulate), one CTA per SM walking 128- or 256-row x
 // 256-column tiles of X = H_kept W^T:
 //   * warp 0 streams 128 x 64 slices of H_kept through a 7-deep TMA ring (256 x 64 slices
-//     through a 3-deep ring for 256-row tiles), warp 10 streams the matching 256 x 64 slices of
-//     W through a 3-deep ring (all 128-byte swizzle);
+//     through a 3-deep ring for 256-row tiles), the last warp streams the matching 256 x 64
+//     slices of W through a 3-deep ring (all 128-byte swizzle);
 //   * one elected lane of warp 1 issues tcgen05.mma M=128 N=256 K=16. With 128-row tiles the
 //     two TMEM accumulators are a double buffer, so the epilogue of tile t overlaps the products
 //     of tile t+1. Once 128-row tiles would take more than one round of the SMs, a tile is 256
 //     rows: both accumulators take one tile, its two 128-row products read every W slice from
 //     shared memory once (a third fewer operand bytes per product, and at 2176 kept rows 144
-//     tiles in one round instead of 272 in two), at the cost of an exposed epilogue;
-//   * warps 2-9 are the epilogue: per TMEM lane quarter two warps, each owning a 128-column half
-//     of the tile (one head for D = 128, two for D = 64). For a Q or K head a thread loads
-//     columns i and i + D/2 together, rotates the pair, and stores bf16 rows. The angle
+//     tiles in one round instead of 272 in two); the epilogue is no longer overlapped, so it
+//     gets twice the warps (16, one set of 8 per 128-row block);
+//   * warps 2-9 (2-17 for 256-row tiles) are the epilogue: per TMEM lane quarter and 128-row
+//     block two warps, each owning a 128-column half of the tile (one head for D = 128, two for
+//     D = 64). For a Q or K head a thread loads columns i and i + D/2 together, rotates the
+//     pair, and stores bf16 rows. The angle
 //     pos * theta^(-2i/D) reaches about 1e5 radians at 128K-token positions, so it is formed
 //     and reduced to [-pi, pi] in double before a fast single-precision sine and cosine.
 //   * Every wait is bounded (about 2 s); on a timeout the CTA sets TG_DEV_TIMEOUT, drains its
@@ -35,9 +37,6 @@ using namespace sm100;
 
 constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 64;
-constexpr int NEPI = 8;                    // epilogue warps (warps 2..9)
-constexpr int WPROD = 2 + NEPI;            // warp that streams W
-constexpr int NTHREADS = 32 * (3 + NEPI);  // 352
 constexpr int B_BYTES = BN * BK * 2;       // 32 KB
 constexpr int WS = 3;                      // W ring depth
 constexpr int TAIL = 1024;
@@ -55,6 +54,9 @@ struct QCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int AS = NACC == 1 ? 7 : 3;
   static constexpr int NSET = 2 / NACC;  // accumulator sets in TMEM
+  static constexpr int NEPI = 8 * NACC;  // epilogue warps (warps 2..): 8 per 128-row block
+  static constexpr int WPROD = 2 + NEPI;  // warp that streams W
+  static constexpr int NTHREADS = 32 * (3 + NEPI);
   static constexpr int SMEM = 1024 + AS * A_BYTES + WS * B_BYTES + TAIL;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
@@ -70,13 +72,13 @@ struct QKVParams {
 };
 
 template <int NACC>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(QCfg<NACC>::NTHREADS, 1)
     qkv_rope_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ Qo, __nv_bfloat16* __restrict__ Ko,
                     __nv_bfloat16* __restrict__ Vo, int32_t* __restrict__ dev_status, uint64_t probe_ns,
                     const __grid_constant__ QKVParams p) {
   using C = QCfg<NACC>;
-  constexpr int BM = C::BM, AS = C::AS, A_BYTES = C::A_BYTES, NSET = C::NSET;
+  constexpr int BM = C::BM, AS = C::AS, A_BYTES = C::A_BYTES, NSET = C::NSET, NEPI = C::NEPI, WPROD = C::WPROD;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smem_w = smem + AS * A_BYTES;
@@ -213,8 +215,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (leader) mma_commit(drain);  // every product issued above completes before TMEM can be released
       __syncwarp();
     }
-  } else if (warp < WPROD) {  // ------------------------------------ epilogue: warps 2..9
-    const int half = (warp - 2) >> 2;  // which 128-column half of the tile
+  } else if (warp < WPROD) {  // ------------------------------------ epilogue: warps 2..WPROD-1
+    const int half = ((warp - 2) >> 2) & 1;  // which 128-column half of the tile
+    const int ablk = (warp - 2) >> 3;        // which 128-row block of the tile
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
     const int D = p.D;
@@ -225,8 +228,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // warp-uniform: the tcgen05.ld below is warp-collective
       if (!__all_sync(0xffffffffu, mbar_wait(&accf[set], (it / NSET) & 1, abort, dev_status))) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int a = 0; a < NACC; ++a) {  // the tile's 128-row blocks
+      {
+      const int a = ablk;                // the tile's 128-row block of this warp
       const int acc = set * NACC + a;    // accumulator in TMEM
       const int gm = (tile / p.tiles_n) * BM + a * 128 + r;
       const bool valid = gm < p.M;
@@ -329,7 +332,7 @@ tg_status launch_qkv_nacc(const void* Hk, int64_t M, int d, const void* W, const
   if (ctas > p.tiles) ctas = p.tiles;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)ctas);
-  cfg.blockDim = dim3(NTHREADS);
+  cfg.blockDim = dim3(C::NTHREADS);
   cfg.dynamicSmemBytes = (size_t)C::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1] = {pdl_attribute(PDL_QKV)};
